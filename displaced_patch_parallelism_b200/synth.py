@@ -1,0 +1,255 @@
+"""Seeded synthetic inputs for the displaced-patch block step.
+
+This module is shared by the CPU oracle's tests, the CUDA parity tests and the
+benchmark.  It holds no arithmetic of the method itself: only random draws, the
+bf16 storage rounding of those draws, and the workload shapes.
+
+The shapes stand in for the SDXL workloads that "DistriFusion: Distributed
+Parallel Inference for High-Resolution Diffusion Models" (study.space summary,
+Experiments; atlas.scime.ai summary, Key results) evaluates on COCO Captions
+with the SDXL model: 1024x1024 images (latent 128x128) and 3840x3840 images
+(latent 480x480).  Neither the dataset nor the weights exist here, so every
+tensor is drawn from a seeded ``torch.Generator`` on the CPU.
+
+Drawing rules (one reading, stated once):
+  * step-0 activations ~ N(0, 1) with the workload seed;
+  * step k >= 1 adds N(0, drift^2) drawn with seed ``drift_seed_base + k``
+    to the previous step's fp32 activations (the 1x64x32x32 case uses seed 1
+    for its only displaced step);
+  * conv weights are Kaiming-normal, std sqrt(2 / (Cin * 9));
+  * attention projection weights ~ N(0, 0.02^2);
+  * all of a block's weights come from ONE generator seeded once, drawn in the
+    order listed by ``Workload.weight_specs``;
+  * bf16 workloads store every drawn tensor rounded to bf16 (round to nearest
+    even); fp32 workloads keep fp32.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Dict, List, Optional, Tuple
+
+import torch
+
+# Step modes (same numbering as the C ABI).
+SYNC, DISPLACED, NAIVE = 0, 1, 2
+MODE_NAMES = {SYNC: "sync", DISPLACED: "displaced", NAIVE: "naive"}
+
+
+def mode_for_step(step: int, warmup: int) -> int:
+    """Mode of denoising step ``step`` given ``warmup`` synchronous steps.
+
+    Warm-up steps run synchronously (atlas.scime.ai summary, ablation rows on
+    warm-up steps).  With zero warm-up there is no previous step to borrow
+    context from, so step 0 runs as independent patches (the naive baseline).
+    """
+    if step < warmup:
+        return SYNC
+    if step == 0:
+        return NAIVE
+    return DISPLACED
+
+
+def randn(shape, seed: int, std: float = 1.0) -> torch.Tensor:
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    t = torch.randn(*shape, generator=g, dtype=torch.float32)
+    return t * std if std != 1.0 else t
+
+
+def store(t: torch.Tensor, dtype: str) -> torch.Tensor:
+    """Round an fp32 tensor to the workload's storage type, returned as fp32."""
+    if dtype == "bf16":
+        return t.to(torch.bfloat16).to(torch.float32)
+    if dtype == "fp32":
+        return t.to(torch.float32)
+    raise ValueError(dtype)
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    """One synthetic workload: a block kind, its shapes and its seeds."""
+
+    name: str
+    kind: str                 # "gn_conv" | "resblock" | "attn" | "unet_mini"
+    C: int                    # channels of the block input
+    H: int
+    W: int
+    P: int                    # virtual row patches
+    dtype: str = "bf16"
+    G: int = 32
+    eps: float = 1e-5
+    heads: int = 0
+    head_dim: int = 64
+    Cout: int = 0             # output channels (0 = same as C)
+    silu: bool = True
+    steps: int = 50
+    warmup: int = 4
+    drift: float = 0.05
+    seed: int = 0
+    drift_seed_base: int = 1000
+    weight_seed: int = 2
+    first_drift_seed: Optional[int] = None  # overrides drift_seed_base + 1
+
+    @property
+    def cout(self) -> int:
+        return self.Cout or self.C
+
+    def drift_seed(self, step: int) -> int:
+        if step == 1 and self.first_drift_seed is not None:
+            return self.first_drift_seed
+        return self.drift_seed_base + step
+
+    def weight_specs(self) -> List[Tuple[str, Tuple[int, ...], float]]:
+        """(name, shape, std) of every weight, in draw order."""
+        C, Co = self.C, self.cout
+        if self.kind == "gn_conv":
+            return [("conv_w", (Co, C, 3, 3), math.sqrt(2.0 / (C * 9)))]
+        if self.kind == "resblock":
+            specs = [("conv1_w", (Co, C, 3, 3), math.sqrt(2.0 / (C * 9))),
+                     ("conv2_w", (Co, Co, 3, 3), math.sqrt(2.0 / (Co * 9)))]
+            if Co != C:
+                specs.append(("short_w", (Co, C, 1, 1), math.sqrt(2.0 / C)))
+            return specs
+        if self.kind == "attn":
+            return [("wq", (C, C), 0.02), ("wk", (C, C), 0.02),
+                    ("wv", (C, C), 0.02), ("wo", (C, C), 0.02)]
+        if self.kind == "unet_mini":
+            return unet_mini_weight_specs(self.C)
+        raise ValueError(self.kind)
+
+
+def unet_mini_weight_specs(cin: int) -> List[Tuple[str, Tuple[int, ...], float]]:
+    """Weights of the mini U-Net chain, in draw order (Kaiming for convs)."""
+    def conv(name, co, ci, k=3):
+        return (name, (co, ci, k, k), math.sqrt(2.0 / (ci * k * k)))
+
+    def lin(name, c):
+        return (name, (c, c), math.sqrt(2.0 / c))
+
+    s = [conv("conv_in_w", 320, cin)]
+    s += [conv("rb1.conv1_w", 320, 320), conv("rb1.conv2_w", 320, 320)]
+    s += [conv("down1_w", 320, 320)]
+    s += [conv("rb2.conv1_w", 640, 320), conv("rb2.conv2_w", 640, 640),
+          ("rb2.short_w", (640, 320, 1, 1), math.sqrt(2.0 / 320))]
+    s += [lin("at2.wq", 640), lin("at2.wk", 640), lin("at2.wv", 640), lin("at2.wo", 640)]
+    s += [conv("down2_w", 640, 640)]
+    s += [conv("rb3.conv1_w", 1280, 640), conv("rb3.conv2_w", 1280, 1280),
+          ("rb3.short_w", (1280, 640, 1, 1), math.sqrt(2.0 / 640))]
+    s += [lin("at3.wq", 1280), lin("at3.wk", 1280), lin("at3.wv", 1280), lin("at3.wo", 1280)]
+    return s
+
+
+# The five synthetic workloads (logical NCHW shapes, N = 1).
+WORKLOADS: Dict[str, Workload] = {
+    "tiny_fp32_gn_conv": Workload(
+        name="tiny_fp32_gn_conv", kind="gn_conv", C=64, H=32, W=32, P=2,
+        dtype="fp32", steps=2, warmup=1, drift=0.05, seed=0, first_drift_seed=1,
+        weight_seed=2),
+    "resblock_320x128x128": Workload(
+        name="resblock_320x128x128", kind="resblock", C=320, H=128, W=128, P=4,
+        steps=50, warmup=4, drift=0.05),
+    "attn_640x64x64": Workload(
+        name="attn_640x64x64", kind="attn", C=640, H=64, W=64, P=4, heads=10,
+        head_dim=64, silu=False, steps=50, warmup=4, drift=0.05),
+    "gn_conv_320x480x480": Workload(
+        name="gn_conv_320x480x480", kind="gn_conv", C=320, H=480, W=480, P=8,
+        steps=50, warmup=4, drift=0.05),
+    "unet_mini_4x128x128": Workload(
+        name="unet_mini_4x128x128", kind="unet_mini", C=4, H=128, W=128, P=4,
+        steps=10, warmup=2, drift=0.03, weight_seed=7),
+}
+
+
+def make_weights(wl: Workload, random_affine: bool = False,
+                 affine_seed: int = 99) -> Dict[str, torch.Tensor]:
+    """All weights of ``wl`` as fp32 tensors holding storage-rounded values.
+
+    GroupNorm scale/shift are 1/0 and biases 0 as the workloads state; with
+    ``random_affine`` they are drawn instead (unit tests use this so that an
+    indexing slip in gamma, beta or a bias cannot hide behind zeros).
+    """
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(wl.weight_seed))
+    out: Dict[str, torch.Tensor] = {}
+    for name, shape, std in wl.weight_specs():
+        out[name] = store(torch.randn(*shape, generator=g) * std, wl.dtype)
+    # affine parameters and biases
+    ga = torch.Generator(device="cpu")
+    ga.manual_seed(int(affine_seed))
+
+    def vec(n, kind):
+        if not random_affine:
+            return torch.ones(n) if kind == "gamma" else torch.zeros(n)
+        if kind == "gamma":
+            return 1.0 + 0.25 * torch.randn(n, generator=ga)
+        return 0.25 * torch.randn(n, generator=ga)
+
+    for name, c, kind in affine_specs(wl):
+        out[name] = vec(c, kind).to(torch.float32)
+    return out
+
+
+def affine_specs(wl: Workload) -> List[Tuple[str, int, str]]:
+    C, Co = wl.C, wl.cout
+    if wl.kind == "gn_conv":
+        return [("gn_gamma", C, "gamma"), ("gn_beta", C, "beta"), ("conv_b", Co, "bias")]
+    if wl.kind == "resblock":
+        s = [("gn1_gamma", C, "gamma"), ("gn1_beta", C, "beta"), ("conv1_b", Co, "bias"),
+             ("gn2_gamma", Co, "gamma"), ("gn2_beta", Co, "beta"), ("conv2_b", Co, "bias")]
+        if Co != C:
+            s.append(("short_b", Co, "bias"))
+        return s
+    if wl.kind == "attn":
+        return [("gn_gamma", C, "gamma"), ("gn_beta", C, "beta"), ("bq", C, "bias"),
+                ("bk", C, "bias"), ("bv", C, "bias"), ("bo", C, "bias")]
+    if wl.kind == "unet_mini":
+        s = [("conv_in_b", 320, "bias")]
+        for pre, ci, co in (("rb1", 320, 320), ("rb2", 320, 640), ("rb3", 640, 1280)):
+            s += [(pre + ".gn1_gamma", ci, "gamma"), (pre + ".gn1_beta", ci, "beta"),
+                  (pre + ".conv1_b", co, "bias"), (pre + ".gn2_gamma", co, "gamma"),
+                  (pre + ".gn2_beta", co, "beta"), (pre + ".conv2_b", co, "bias")]
+            if ci != co:
+                s.append((pre + ".short_b", co, "bias"))
+        s += [("down1_b", 320, "bias"), ("down2_b", 640, "bias")]
+        for pre, c in (("at2", 640), ("at3", 1280)):
+            s += [(pre + ".gn_gamma", c, "gamma"), (pre + ".gn_beta", c, "beta"),
+                  (pre + ".bq", c, "bias"), (pre + ".bk", c, "bias"),
+                  (pre + ".bv", c, "bias"), (pre + ".bo", c, "bias")]
+        return s
+    raise ValueError(wl.kind)
+
+
+class InputStream:
+    """The per-step block inputs x_0, x_1, ... of a workload (logical NCHW).
+
+    ``x(k)`` returns the storage-rounded input of step k as fp32 (1, C, H, W).
+    The fp32 chain is kept unrounded between steps; only what a step consumes
+    is rounded.
+    """
+
+    def __init__(self, wl: Workload, shape: Optional[Tuple[int, ...]] = None):
+        self.wl = wl
+        self.shape = shape or (1, wl.C, wl.H, wl.W)
+        self._chain = [randn(self.shape, wl.seed)]
+
+    def x(self, k: int) -> torch.Tensor:
+        while len(self._chain) <= k:
+            j = len(self._chain)
+            self._chain.append(self._chain[-1] + randn(self.shape, self.wl.drift_seed(j), self.wl.drift))
+        return store(self._chain[k], self.wl.dtype)
+
+
+def nchw_to_nhwc(t: torch.Tensor) -> torch.Tensor:
+    """(1, C, H, W) -> contiguous (H, W, C)."""
+    return t[0].permute(1, 2, 0).contiguous()
+
+
+def nhwc_to_nchw(t: torch.Tensor) -> torch.Tensor:
+    """(H, W, C) -> (1, C, H, W)."""
+    return t.permute(2, 0, 1).unsqueeze(0).contiguous()
+
+
+def conv_weight_to_device(w: torch.Tensor) -> torch.Tensor:
+    """(Cout, Cin, kh, kw) -> contiguous (Cout, kh, kw, Cin): one K-major row per output channel."""
+    return w.permute(0, 2, 3, 1).contiguous()

@@ -1,0 +1,417 @@
+"""CPU oracle for the displaced-patch-parallelism block step.  TEST INFRASTRUCTURE ONLY.
+
+Only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline leg
+may import this module.  The product path (the CUDA library and its Python
+binding) never does, and shares no code with it.
+
+What it computes is the method of "DistriFusion: Distributed Parallel Inference
+for High-Resolution Diffusion Models": the image latent is split into P row
+patches; each patch computes its own rows with fresh activations and takes the
+context it needs from other patches out of the previous denoising step's
+("stale", "displaced") activations (study.space summary, Method; atlas.scime.ai
+summary, Approach), with a corrected asynchronous GroupNorm (atlas.scime.ai
+summary, Approach and the GroupNorm ablation rows).  Attention keeps the full
+set of keys and values, fresh for the patch's own tokens and stale for the
+others (gist.science PipeFusion explainer, Problem Statement and Memory
+Efficiency, describing DistriFusion's full-spatial K/V buffers).
+
+Arithmetic is fp64 numpy throughout.  Where the GPU stores an intermediate in
+bf16 (GroupNorm output, conv output feeding the next GroupNorm, q/k/v, the
+attention output, block outputs) the oracle rounds to bf16 at the same point
+(``store``); pass ``storage="none"`` to keep everything unrounded.
+
+Readings of what the pages leave open (each also listed in the design notes):
+  R1  corrected statistics on raw moments (E[x], E[x^2]):
+        used = stale_global + w * (fresh_local - stale_local),  w = 1 by default
+  R2  a negative corrected variance falls back to the patch's fresh variance
+  R3  zero warm-up: step 0 runs as independent patches (zero context)
+  R4  equal row bands of H/P rows; equal-weight averages across bands
+  R5  the stale tensor of a conv is its input (after GroupNorm and SiLU)
+  R6  block structures: see ``gn_conv_step``, ``resblock_step``, ``attn_step``,
+      ``unet_mini_step``
+  R7  every 3x3 conv, stride 1 or 2, pads by one and takes halo rows from
+      other bands per mode; stride-2 output bands are Ho/P rows
+
+Parity pins (the tests under tests/test_oracle_*.py): P = 1 reduces to the
+library full-image block (torch group_norm / conv2d / softmax attention);
+brute-force loops on tiny inputs; naive mode equals independent crops; an
+unchanged input makes displaced equal sync; a uniform drift makes the
+corrected statistics exact; halo and attention locality; zero warm-up differs
+from sync.  ``unet_mini_step`` is pinned only through its parts and the P = 1
+reduction of the whole chain.
+"""
+from __future__ import annotations
+
+import math
+from typing import Dict, Optional, Tuple
+
+import numpy as np
+import torch
+
+SYNC, DISPLACED, NAIVE = 0, 1, 2
+
+
+# --------------------------------------------------------------------------
+# storage rounding
+# --------------------------------------------------------------------------
+def to_bf16(x: np.ndarray) -> np.ndarray:
+    """Round to bf16 (nearest even) and return as fp64.
+
+    fp64 -> fp32 -> bf16: the GPU rounds an fp32 value, so the oracle rounds
+    through fp32 as well.
+    """
+    f32 = np.ascontiguousarray(x, dtype=np.float32)
+    u = f32.view(np.uint32).astype(np.uint64)
+    lsb = (u >> 16) & 1
+    u = (u + 0x7FFF + lsb) >> 16 << 16
+    nan = np.isnan(f32)
+    out = (u & 0xFFFFFFFF).astype(np.uint32).view(np.float32).astype(np.float64)
+    out[nan] = np.nan
+    return out
+
+
+def store(x: np.ndarray, storage: str) -> np.ndarray:
+    if storage == "bf16":
+        return to_bf16(x)
+    if storage == "fp32":
+        return np.asarray(x, dtype=np.float32).astype(np.float64)
+    if storage == "none":
+        return np.asarray(x, dtype=np.float64)
+    raise ValueError(storage)
+
+
+# --------------------------------------------------------------------------
+# GroupNorm (atlas.scime.ai summary: Approach; GroupNorm ablation rows)
+# --------------------------------------------------------------------------
+def gn_fresh_local(x: np.ndarray, P: int, G: int) -> np.ndarray:
+    """Per (band p, group g) raw moments of the fresh input.
+
+    x: (C, H, W).  Band p is rows [p*H/P, (p+1)*H/P); group g is channels
+    [g*C/G, (g+1)*C/G).  Returns f[p, g] = (mean x, mean x^2).
+    """
+    C, H, W = x.shape
+    hb, cg = H // P, C // G
+    f = np.empty((P, G, 2))
+    for p in range(P):
+        for g in range(G):
+            v = x[g * cg:(g + 1) * cg, p * hb:(p + 1) * hb, :]
+            f[p, g, 0] = v.mean()
+            f[p, g, 1] = (v * v).mean()
+    return f
+
+
+def gn_used_stats(f: np.ndarray, mode: int, stale_global: Optional[np.ndarray],
+                  stale_local: Optional[np.ndarray], w: float = 1.0
+                  ) -> Tuple[np.ndarray, int]:
+    """Statistics each band normalises with.  Returns (used[p, g] = (mean, var), fallbacks).
+
+    sync:       the exact whole-image moments, i.e. the average of the bands'
+                moments (equal bands);
+    displaced:  stale whole-image moments corrected by the band's own drift,
+                stale_global + w * (fresh_local - stale_local)   (reading R1);
+    naive:      the band's own moments only.
+    var = E[x^2] - E[x]^2; a negative var falls back to the band's fresh var (R2).
+    """
+    P, G, _ = f.shape
+    if mode == SYNC:
+        m = np.broadcast_to(f.mean(axis=0), f.shape).copy()
+    elif mode == DISPLACED:
+        if stale_global is None or stale_local is None:
+            raise ValueError("displaced GroupNorm needs the previous step's statistics")
+        m = stale_global[None, :, :] + w * (f - stale_local)
+    elif mode == NAIVE:
+        m = f.copy()
+    else:
+        raise ValueError(mode)
+    mean = m[..., 0]
+    var = m[..., 1] - mean * mean
+    fresh_var = f[..., 1] - f[..., 0] * f[..., 0]
+    neg = var < 0
+    var = np.where(neg, fresh_var, var)
+    return np.stack([mean, var], axis=-1), int(neg.sum())
+
+
+def gn_apply(x: np.ndarray, used: np.ndarray, gamma: np.ndarray, beta: np.ndarray,
+             P: int, G: int, eps: float, silu: bool) -> np.ndarray:
+    """y = (x - mean) / sqrt(var + eps) * gamma_c + beta_c, per band and group; then SiLU."""
+    C, H, W = x.shape
+    hb, cg = H // P, C // G
+    y = np.empty_like(x, dtype=np.float64)
+    for p in range(P):
+        for g in range(G):
+            cs = slice(g * cg, (g + 1) * cg)
+            rs = slice(p * hb, (p + 1) * hb)
+            mean, var = used[p, g]
+            y[cs, rs, :] = ((x[cs, rs, :] - mean) / math.sqrt(var + eps)
+                            * gamma[cs, None, None] + beta[cs, None, None])
+    if silu:
+        y = y / (1.0 + np.exp(-y))
+    return y
+
+
+def groupnorm_async(x, gamma, beta, P, G, eps, w, silu, mode, stale_global, stale_local):
+    """One GroupNorm layer: returns (y, fresh_local, used, fallbacks)."""
+    f = gn_fresh_local(x, P, G)
+    used, nneg = gn_used_stats(f, mode, stale_global, stale_local, w)
+    return gn_apply(x, used, gamma, beta, P, G, eps, silu), f, used, nneg
+
+
+def refresh_stats(f: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """Next step's stale statistics: (stale_global = mean over bands, stale_local = f)."""
+    return f.mean(axis=0), f.copy()
+
+
+# --------------------------------------------------------------------------
+# 3x3 convolution with stale halo rows (study.space summary, Method)
+# --------------------------------------------------------------------------
+def conv3x3_halo(a_fresh: np.ndarray, a_stale: Optional[np.ndarray], weight: np.ndarray,
+                 bias: Optional[np.ndarray], residual: Optional[np.ndarray], P: int,
+                 mode: int, stride: int = 1) -> np.ndarray:
+    """3x3 conv, padding 1, whose input rows depend on the band being computed.
+
+    Output row r of band p reads input row rho = stride*r + kh - 1:
+      rho outside [0, H)         -> zeros (ordinary padding)
+      rho in band p              -> a_fresh
+      rho in another band        -> sync: a_fresh, displaced: a_stale, naive: zeros
+    Columns use ordinary zero padding.  Then + bias (+ residual).
+    a_*: (Cin, H, W); weight: (Cout, Cin, 3, 3); returns (Cout, Ho, Wo).
+    """
+    Cin, H, W = a_fresh.shape
+    Cout = weight.shape[0]
+    Ho = (H - 1) // stride + 1
+    Wo = (W - 1) // stride + 1
+    hb_in, hb_out = H // P, Ho // P
+    if mode == DISPLACED and a_stale is None:
+        raise ValueError("displaced conv needs the previous step's activations")
+    out = np.zeros((Cout, Ho, Wo))
+    for p in range(P):
+        r0, r1 = p * hb_out, (p + 1) * hb_out
+        lo = stride * r0 - 1
+        hi = stride * (r1 - 1) + 1
+        used = np.zeros((Cin, hi - lo + 1, W + 2))
+        for rho in range(lo, hi + 1):
+            if rho < 0 or rho >= H:
+                continue
+            if rho // hb_in == p or mode == SYNC:
+                src = a_fresh
+            elif mode == DISPLACED:
+                src = a_stale
+            else:
+                continue
+            used[:, rho - lo, 1:W + 1] = src[:, rho, :]
+        nr = r1 - r0
+        for kh in range(3):
+            for kw in range(3):
+                patch = used[:, kh:kh + stride * (nr - 1) + 1:stride,
+                             kw:kw + stride * (Wo - 1) + 1:stride]
+                out[:, r0:r1, :] += np.tensordot(weight[:, :, kh, kw], patch, axes=(1, 0))
+    if bias is not None:
+        out += bias[:, None, None]
+    if residual is not None:
+        out += residual
+    return out
+
+
+def conv1x1(x: np.ndarray, weight: np.ndarray, bias: Optional[np.ndarray]) -> np.ndarray:
+    """Pointwise conv (the ResBlock shortcut when channels change)."""
+    out = np.tensordot(weight[:, :, 0, 0], x, axes=(1, 0))
+    if bias is not None:
+        out += bias[:, None, None]
+    return out
+
+
+# --------------------------------------------------------------------------
+# self-attention over stitched fresh / stale K and V
+# (gist.science PipeFusion explainer, Problem Statement, on DistriFusion)
+# --------------------------------------------------------------------------
+def attention_stale_kv(q: np.ndarray, k_fresh: np.ndarray, v_fresh: np.ndarray,
+                       k_stale: Optional[np.ndarray], v_stale: Optional[np.ndarray],
+                       P: int, heads: int, scale: float, mode: int) -> np.ndarray:
+    """Per band p and head: softmax(q_p K^T * scale) V over the keys band p sees.
+
+    Keys and values of band p's own tokens are fresh.  The others are stale
+    (displaced), fresh (sync) or left out (naive).  q, k, v: (T, heads*d).
+    """
+    T, Cq = q.shape
+    d = Cq // heads
+    tb = T // P
+    if mode == DISPLACED and (k_stale is None or v_stale is None):
+        raise ValueError("displaced attention needs the previous step's keys and values")
+    o = np.zeros_like(q, dtype=np.float64)
+    for p in range(P):
+        own = slice(p * tb, (p + 1) * tb)
+        if mode == NAIVE:
+            K, V = k_fresh[own], v_fresh[own]
+        elif mode == SYNC:
+            K, V = k_fresh, v_fresh
+        elif mode == DISPLACED:
+            K, V = k_stale.copy(), v_stale.copy()
+            K[own], V[own] = k_fresh[own], v_fresh[own]
+        else:
+            raise ValueError(mode)
+        for h in range(heads):
+            hs = slice(h * d, (h + 1) * d)
+            s = (q[own, hs] @ K[:, hs].T) * scale
+            s = s - s.max(axis=1, keepdims=True)
+            e = np.exp(s)
+            o[own, hs] = (e / e.sum(axis=1, keepdims=True)) @ V[:, hs]
+    return o
+
+
+def linear(x: np.ndarray, w: np.ndarray, b: Optional[np.ndarray]) -> np.ndarray:
+    """x @ w.T + b with w stored (out, in)."""
+    y = x @ w.T
+    return y + b if b is not None else y
+
+
+# --------------------------------------------------------------------------
+# blocks (reading R6) with their cross-step state
+# --------------------------------------------------------------------------
+class GNState:
+    def __init__(self):
+        self.stale_global = None  # (G, 2)
+        self.stale_local = None   # (P, G, 2)
+
+    def refresh(self, f):
+        self.stale_global, self.stale_local = refresh_stats(f)
+
+
+def _gn(st: GNState, x, gamma, beta, P, G, eps, w, silu, mode, trace, key):
+    y, f, used, nneg = groupnorm_async(x, gamma, beta, P, G, eps, w, silu, mode,
+                                       st.stale_global, st.stale_local)
+    if trace is not None:
+        trace[key + ".fresh_local"] = f
+        trace[key + ".used"] = used
+        trace[key + ".fallbacks"] = nneg
+    return y, f
+
+
+def _a(x) -> np.ndarray:
+    if isinstance(x, torch.Tensor):
+        return x.detach().to(torch.float64).numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def gn_conv_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float,
+                 silu: bool, mode: int, storage: str, trace: Optional[Dict] = None):
+    """GroupNorm (+SiLU) -> 3x3 conv with stale halo.  x: (C, H, W)."""
+    x = _a(x)
+    gn = state.setdefault("gn", GNState())
+    a, f = _gn(gn, x, _a(wts["gn_gamma"]), _a(wts["gn_beta"]), P, G, eps, w, silu, mode,
+               trace, "gn")
+    a = store(a, storage)
+    out = conv3x3_halo(a, state.get("a_stale"), _a(wts["conv_w"]), _a(wts["conv_b"]), None,
+                       P, mode)
+    out = store(out, storage)
+    if trace is not None:
+        trace["a"] = a
+    gn.refresh(f)
+    state["a_stale"] = a
+    return out
+
+
+def resblock_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float,
+                  mode: int, storage: str, trace: Optional[Dict] = None, prefix: str = ""):
+    """GN -> SiLU -> conv1 -> GN -> SiLU -> conv2 -> + x (or + 1x1 shortcut(x))."""
+    x = _a(x)
+    W_ = lambda n: _a(wts[prefix + n])
+    gn1 = state.setdefault("gn1", GNState())
+    gn2 = state.setdefault("gn2", GNState())
+    a1, f1 = _gn(gn1, x, W_("gn1_gamma"), W_("gn1_beta"), P, G, eps, w, True, mode, trace,
+                 prefix + "gn1")
+    a1 = store(a1, storage)
+    h = store(conv3x3_halo(a1, state.get("a1_stale"), W_("conv1_w"), W_("conv1_b"), None, P,
+                           mode), storage)
+    a2, f2 = _gn(gn2, h, W_("gn2_gamma"), W_("gn2_beta"), P, G, eps, w, True, mode, trace,
+                 prefix + "gn2")
+    a2 = store(a2, storage)
+    if (prefix + "short_w") in wts:
+        res = store(conv1x1(x, W_("short_w"), W_("short_b")), storage)
+    else:
+        res = x
+    out = store(conv3x3_halo(a2, state.get("a2_stale"), W_("conv2_w"), W_("conv2_b"), res, P,
+                             mode), storage)
+    if trace is not None:
+        trace[prefix + "a1"], trace[prefix + "h"], trace[prefix + "a2"] = a1, h, a2
+    gn1.refresh(f1)
+    gn2.refresh(f2)
+    state["a1_stale"], state["a2_stale"] = a1, a2
+    return out
+
+
+def attn_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float, heads: int,
+              mode: int, storage: str, trace: Optional[Dict] = None, prefix: str = ""):
+    """GN (no SiLU) -> q, k, v projections -> stale-K/V attention -> out proj + bias -> + x.
+
+    x: (C, H, W); tokens are pixels in raster order, so band p's tokens are
+    rows [p*H/P, (p+1)*H/P) of the image.
+    """
+    x = _a(x)
+    C, H, Wd = x.shape
+    W_ = lambda n: _a(wts[prefix + n])
+    gn = state.setdefault("gn", GNState())
+    a, f = _gn(gn, x, W_("gn_gamma"), W_("gn_beta"), P, G, eps, w, False, mode, trace,
+               prefix + "gn")
+    a = store(a, storage)
+    tok = a.reshape(C, H * Wd).T                       # (T, C)
+    q = store(linear(tok, W_("wq"), W_("bq")), storage)
+    k = store(linear(tok, W_("wk"), W_("bk")), storage)
+    v = store(linear(tok, W_("wv"), W_("bv")), storage)
+    d = C // heads
+    o = store(attention_stale_kv(q, k, v, state.get("k_stale"), state.get("v_stale"), P,
+                                 heads, 1.0 / math.sqrt(d), mode), storage)
+    out_tok = linear(o, W_("wo"), W_("bo")) + x.reshape(C, H * Wd).T
+    out = store(out_tok.T.reshape(C, H, Wd), storage)
+    if trace is not None:
+        trace[prefix + "a"], trace[prefix + "q"] = a, q
+        trace[prefix + "k"], trace[prefix + "v"], trace[prefix + "o"] = k, v, o
+    gn.refresh(f)
+    state["k_stale"], state["v_stale"] = k, v
+    return out
+
+
+def unet_mini_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float,
+                   mode: int, storage: str, trace: Optional[Dict] = None):
+    """conv_in -> ResBlock(320) -> down -> ResBlock(320->640) -> Attn(640, 10 heads)
+    -> down -> ResBlock(640->1280) -> Attn(1280, 20 heads)   (reading R6/R7).
+
+    Every 3x3 conv, conv_in and the stride-2 downsamplers included, takes its
+    halo rows from the previous step's copy of its own input.
+    """
+    x = _a(x)
+    A = lambda n: _a(wts[n])
+    sub = lambda n: state.setdefault(n, {})
+
+    def conv_layer(name, inp, wname, bname, stride):
+        st = sub(name)
+        y = conv3x3_halo(inp, st.get("a_stale"), A(wname), A(bname), None, P, mode, stride)
+        st["a_stale"] = inp
+        return store(y, storage)
+
+    h = conv_layer("conv_in", x, "conv_in_w", "conv_in_b", 1)
+    h = resblock_step(sub("rb1"), h, wts, P, G, eps, w, mode, storage, trace, "rb1.")
+    h = conv_layer("down1", h, "down1_w", "down1_b", 2)
+    h = resblock_step(sub("rb2"), h, wts, P, G, eps, w, mode, storage, trace, "rb2.")
+    h = attn_step(sub("at2"), h, wts, P, G, eps, w, 10, mode, storage, trace, "at2.")
+    h = conv_layer("down2", h, "down2_w", "down2_b", 2)
+    h = resblock_step(sub("rb3"), h, wts, P, G, eps, w, mode, storage, trace, "rb3.")
+    h = attn_step(sub("at3"), h, wts, P, G, eps, w, 20, mode, storage, trace, "at3.")
+    return h
+
+
+def block_step(kind: str, state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float,
+               mode: int, storage: str, heads: int = 0, silu: bool = True,
+               trace: Optional[Dict] = None):
+    """Dispatch one block step by kind; x is (C, H, W) (a leading batch of 1 is dropped)."""
+    x = _a(x)
+    if x.ndim == 4:
+        x = x[0]
+    if kind == "gn_conv":
+        return gn_conv_step(state, x, wts, P, G, eps, w, silu, mode, storage, trace)
+    if kind == "resblock":
+        return resblock_step(state, x, wts, P, G, eps, w, mode, storage, trace)
+    if kind == "attn":
+        return attn_step(state, x, wts, P, G, eps, w, heads, mode, storage, trace)
+    if kind == "unet_mini":
+        return unet_mini_step(state, x, wts, P, G, eps, w, mode, storage, trace)
+    raise ValueError(kind)

@@ -1,0 +1,462 @@
+"""Pins of the CPU oracle against facts fixed by the pages and by mathematics.
+
+The pages print no worked example, so the oracle is pinned by:
+  * the P = 1 reduction to the ordinary full-image block (library routines:
+    torch group_norm, conv2d, scaled_dot_product_attention), which the pages
+    require as "no quality degradation" of the original model when nothing is
+    displaced (study.space summary, Abstract);
+  * brute-force loops on tiny inputs (conv, attention, GroupNorm moments);
+  * naive mode equal to independent crops (atlas.scime.ai summary, the naive
+    patch baseline rows);
+  * an unchanged input making displaced equal sync;
+  * a uniform drift making the corrected statistics exact (reading R1, w = 1);
+  * halo and attention locality;
+  * zero warm-up distinguishable from sync (atlas.scime.ai summary, warm-up
+    ablation rows).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+from oracle import dp_oracle as O
+
+SYNC, DISPLACED, NAIVE = O.SYNC, O.DISPLACED, O.NAIVE
+
+
+def rng(seed):
+    return np.random.default_rng(seed)
+
+
+def rand_gn_conv_weights(r, C, Co):
+    return {
+        "gn_gamma": 1 + 0.3 * r.standard_normal(C), "gn_beta": 0.3 * r.standard_normal(C),
+        "conv_w": r.standard_normal((Co, C, 3, 3)) * math.sqrt(2 / (9 * C)),
+        "conv_b": 0.3 * r.standard_normal(Co),
+    }
+
+
+def rand_res_weights(r, C, Co, prefix=""):
+    w = {
+        "gn1_gamma": 1 + 0.3 * r.standard_normal(C), "gn1_beta": 0.3 * r.standard_normal(C),
+        "conv1_w": r.standard_normal((Co, C, 3, 3)) * math.sqrt(2 / (9 * C)),
+        "conv1_b": 0.3 * r.standard_normal(Co),
+        "gn2_gamma": 1 + 0.3 * r.standard_normal(Co), "gn2_beta": 0.3 * r.standard_normal(Co),
+        "conv2_w": r.standard_normal((Co, Co, 3, 3)) * math.sqrt(2 / (9 * Co)),
+        "conv2_b": 0.3 * r.standard_normal(Co),
+    }
+    if C != Co:
+        w["short_w"] = r.standard_normal((Co, C, 1, 1)) * math.sqrt(2 / C)
+        w["short_b"] = 0.3 * r.standard_normal(Co)
+    return {prefix + k: v for k, v in w.items()}
+
+
+def rand_attn_weights(r, C, prefix=""):
+    w = {"gn_gamma": 1 + 0.3 * r.standard_normal(C), "gn_beta": 0.3 * r.standard_normal(C)}
+    for n in ("wq", "wk", "wv", "wo"):
+        w[n] = r.standard_normal((C, C)) * (1.0 / math.sqrt(C))
+    for n in ("bq", "bk", "bv", "bo"):
+        w[n] = 0.3 * r.standard_normal(C)
+    return {prefix + k: v for k, v in w.items()}
+
+
+T64 = lambda a: torch.from_numpy(np.asarray(a, dtype=np.float64))
+
+
+# ---------------------------------------------------------------- library blocks
+def lib_gn_conv(x, w, G, eps, silu=True):
+    t = F.group_norm(T64(x)[None], G, T64(w["gn_gamma"]), T64(w["gn_beta"]), eps)
+    if silu:
+        t = F.silu(t)
+    return F.conv2d(t, T64(w["conv_w"]), T64(w["conv_b"]), padding=1)[0].numpy()
+
+
+def lib_resblock(x, w, G, eps, prefix=""):
+    g = lambda n: T64(w[prefix + n])
+    t = F.silu(F.group_norm(T64(x)[None], G, g("gn1_gamma"), g("gn1_beta"), eps))
+    h = F.conv2d(t, g("conv1_w"), g("conv1_b"), padding=1)
+    t = F.silu(F.group_norm(h, G, g("gn2_gamma"), g("gn2_beta"), eps))
+    res = T64(x)[None]
+    if prefix + "short_w" in w:
+        res = F.conv2d(res, g("short_w"), g("short_b"))
+    return (F.conv2d(t, g("conv2_w"), g("conv2_b"), padding=1) + res)[0].numpy()
+
+
+def lib_attn(x, w, G, eps, heads, prefix=""):
+    g = lambda n: T64(w[prefix + n])
+    C, H, W = x.shape
+    t = F.group_norm(T64(x)[None], G, g("gn_gamma"), g("gn_beta"), eps)[0]
+    tok = t.reshape(C, H * W).T
+    q = tok @ g("wq").T + g("bq")
+    k = tok @ g("wk").T + g("bk")
+    v = tok @ g("wv").T + g("bv")
+    d = C // heads
+    sh = lambda z: z.reshape(H * W, heads, d).permute(1, 0, 2)
+    o = F.scaled_dot_product_attention(sh(q), sh(k), sh(v))
+    o = o.permute(1, 0, 2).reshape(H * W, C)
+    out = o @ g("wo").T + g("bo") + T64(x).reshape(C, H * W).T
+    return out.T.reshape(C, H, W).numpy()
+
+
+def run_two_steps(kind, x0, x1, w, P, G, mode1, heads=0, wgt=1.0, silu=True):
+    st = {}
+    O.block_step(kind, st, x0, w, P, G, 1e-5, wgt, SYNC, "none", heads=heads, silu=silu)
+    tr = {}
+    y = O.block_step(kind, st, x1, w, P, G, 1e-5, wgt, mode1, "none", heads=heads, silu=silu,
+                     trace=tr)
+    return y, tr, st
+
+
+# ---------------------------------------------------------------- P = 1 reduction
+@pytest.mark.parametrize("mode", [SYNC, DISPLACED, NAIVE])
+def test_p1_gn_conv_equals_library(mode):
+    r = rng(1)
+    C, H, W = 16, 6, 7
+    w = rand_gn_conv_weights(r, C, 12)
+    x0, x1 = r.standard_normal((C, H, W)), r.standard_normal((C, H, W))
+    y, _, _ = run_two_steps("gn_conv", x0, x1, w, 1, 4, mode)
+    np.testing.assert_allclose(y, lib_gn_conv(x1, w, 4, 1e-5), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("mode", [SYNC, DISPLACED])
+@pytest.mark.parametrize("co", [8, 16])
+def test_p1_resblock_equals_library(mode, co):
+    r = rng(2)
+    C, H, W = 8, 5, 6
+    w = rand_res_weights(r, C, co)
+    x0, x1 = r.standard_normal((C, H, W)), r.standard_normal((C, H, W))
+    y, _, _ = run_two_steps("resblock", x0, x1, w, 1, 4, mode)
+    np.testing.assert_allclose(y, lib_resblock(x1, w, 4, 1e-5), rtol=0, atol=1e-11)
+
+
+@pytest.mark.parametrize("mode", [SYNC, DISPLACED])
+def test_p1_attn_equals_library(mode):
+    r = rng(3)
+    C, H, W = 16, 4, 5
+    w = rand_attn_weights(r, C)
+    x0, x1 = r.standard_normal((C, H, W)), r.standard_normal((C, H, W))
+    y, _, _ = run_two_steps("attn", x0, x1, w, 1, 4, mode, heads=4)
+    np.testing.assert_allclose(y, lib_attn(x1, w, 4, 1e-5, 4), rtol=0, atol=1e-11)
+
+
+@pytest.mark.parametrize("H,W", [(8, 8), (6, 10), (7, 5)])
+def test_p1_stride2_conv_equals_library(H, W):
+    r = rng(4)
+    a = r.standard_normal((5, H, W))
+    wt = r.standard_normal((3, 5, 3, 3))
+    b = r.standard_normal(3)
+    y = O.conv3x3_halo(a, None, wt, b, None, 1, SYNC, stride=2)
+    ref = F.conv2d(T64(a)[None], T64(wt), T64(b), stride=2, padding=1)[0].numpy()
+    np.testing.assert_allclose(y, ref, rtol=0, atol=1e-12)
+
+
+def test_conv1x1_equals_library():
+    r = rng(5)
+    a = r.standard_normal((6, 4, 5))
+    wt = r.standard_normal((3, 6, 1, 1))
+    b = r.standard_normal(3)
+    ref = F.conv2d(T64(a)[None], T64(wt), T64(b))[0].numpy()
+    np.testing.assert_allclose(O.conv1x1(a, wt, b), ref, rtol=0, atol=1e-12)
+
+
+def test_p1_unet_mini_displaced_equals_sync():
+    """The whole chain with one band: displacement changes nothing."""
+    from displaced_patch_parallelism_b200 import synth
+    wl = synth.WORKLOADS["unet_mini_4x128x128"]
+    # shrink: the chain's structure with tiny spatial size
+    r = rng(6)
+    wts = {}
+    for name, shape, std in synth.unet_mini_weight_specs(4):
+        wts[name] = r.standard_normal(shape) * std
+    for name, c, kind in synth.affine_specs(wl):
+        wts[name] = (1 + 0.2 * r.standard_normal(c)) if kind == "gamma" else 0.2 * r.standard_normal(c)
+    x0, x1 = r.standard_normal((4, 8, 8)), r.standard_normal((4, 8, 8))
+    outs = {}
+    for m in (SYNC, DISPLACED):
+        st = {}
+        O.unet_mini_step(st, x0, wts, 1, 32, 1e-5, 1.0, SYNC, "none")
+        outs[m] = O.unet_mini_step(st, x1, wts, 1, 32, 1e-5, 1.0, m, "none")
+    np.testing.assert_allclose(outs[DISPLACED], outs[SYNC], rtol=0, atol=1e-10)
+    assert outs[SYNC].shape == (1280, 2, 2)
+
+
+# ---------------------------------------------------------------- brute force
+def brute_conv(a_fresh, a_stale, wt, b, P, mode, stride):
+    Cin, H, W = a_fresh.shape
+    Co = wt.shape[0]
+    Ho, Wo = (H - 1) // stride + 1, (W - 1) // stride + 1
+    out = np.zeros((Co, Ho, Wo))
+    for co in range(Co):
+        for r in range(Ho):
+            band = r // (Ho // P)
+            for c in range(Wo):
+                s = b[co]
+                for ci in range(Cin):
+                    for kh in range(3):
+                        for kw in range(3):
+                            rr, cc = stride * r + kh - 1, stride * c + kw - 1
+                            if not (0 <= rr < H and 0 <= cc < W):
+                                continue
+                            if rr // (H // P) == band:
+                                v = a_fresh[ci, rr, cc]
+                            elif mode == SYNC:
+                                v = a_fresh[ci, rr, cc]
+                            elif mode == DISPLACED:
+                                v = a_stale[ci, rr, cc]
+                            else:
+                                v = 0.0
+                            s += wt[co, ci, kh, kw] * v
+                out[co, r, c] = s
+    return out
+
+
+@pytest.mark.parametrize("mode", [SYNC, DISPLACED, NAIVE])
+@pytest.mark.parametrize("stride,H,P", [(1, 6, 3), (1, 8, 2), (2, 8, 2), (2, 12, 3)])
+def test_conv_matches_brute_force(mode, stride, H, P):
+    r = rng(10 + stride + H)
+    Cin, Co, W = 3, 2, 5
+    af, ast = r.standard_normal((Cin, H, W)), r.standard_normal((Cin, H, W))
+    wt, b = r.standard_normal((Co, Cin, 3, 3)), r.standard_normal(Co)
+    got = O.conv3x3_halo(af, ast, wt, b, None, P, mode, stride)
+    np.testing.assert_allclose(got, brute_conv(af, ast, wt, b, P, mode, stride), rtol=0,
+                               atol=1e-12)
+
+
+def brute_attention(q, kf, vf, ks, vs, P, heads, scale, mode):
+    T, C = q.shape
+    d = C // heads
+    o = np.zeros((T, C))
+    for i in range(T):
+        band = i // (T // P)
+        for h in range(heads):
+            logits, vals = [], []
+            for j in range(T):
+                own = j // (T // P) == band
+                if own or mode == SYNC:
+                    kk, vv = kf[j], vf[j]
+                elif mode == DISPLACED:
+                    kk, vv = ks[j], vs[j]
+                else:
+                    continue
+                logits.append(sum(q[i, h * d + e] * kk[h * d + e] for e in range(d)) * scale)
+                vals.append(vv[h * d:(h + 1) * d])
+            z = sum(math.exp(l) for l in logits)
+            for l, vv in zip(logits, vals):
+                o[i, h * d:(h + 1) * d] += math.exp(l) / z * vv
+    return o
+
+
+@pytest.mark.parametrize("mode", [SYNC, DISPLACED, NAIVE])
+def test_attention_matches_brute_force(mode):
+    r = rng(20)
+    T, heads, d, P = 6, 2, 3, 3
+    q, kf, vf, ks, vs = (r.standard_normal((T, heads * d)) for _ in range(5))
+    got = O.attention_stale_kv(q, kf, vf, ks, vs, P, heads, 0.7, mode)
+    np.testing.assert_allclose(got, brute_attention(q, kf, vf, ks, vs, P, heads, 0.7, mode),
+                               rtol=0, atol=1e-12)
+
+
+def test_gn_moments_match_brute_force():
+    r = rng(21)
+    C, H, W, P, G = 6, 4, 3, 2, 3
+    x = r.standard_normal((C, H, W))
+    f = O.gn_fresh_local(x, P, G)
+    for p in range(P):
+        for g in range(G):
+            vals = [x[c, rr, cc] for c in range(C) for rr in range(H) for cc in range(W)
+                    if c // (C // G) == g and rr // (H // P) == p]
+            assert len(vals) == (C // G) * (H // P) * W
+            assert abs(f[p, g, 0] - sum(vals) / len(vals)) < 1e-14
+            assert abs(f[p, g, 1] - sum(v * v for v in vals) / len(vals)) < 1e-14
+
+
+# ---------------------------------------------------------------- sync / naive
+@pytest.mark.parametrize("P", [2, 4])
+def test_sync_groupnorm_is_exact_full_image(P):
+    r = rng(30 + P)
+    C, H, W, G = 8, 8, 5, 4
+    x = r.standard_normal((C, H, W)) * 2 + 0.5
+    gm, bt = 1 + r.standard_normal(C) * 0.3, r.standard_normal(C) * 0.3
+    y, f, used, _ = O.groupnorm_async(x, gm, bt, P, G, 1e-5, 1.0, False, SYNC, None, None)
+    ref = F.group_norm(T64(x)[None], G, T64(gm), T64(bt), 1e-5)[0].numpy()
+    np.testing.assert_allclose(y, ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("kind", ["gn_conv", "attn"])
+def test_naive_equals_independent_crops(kind):
+    r = rng(40)
+    C, H, W, P, G, heads = 8, 8, 4, 4, 4, 2
+    w = rand_gn_conv_weights(r, C, 6) if kind == "gn_conv" else rand_attn_weights(r, C)
+    x = r.standard_normal((C, H, W))
+    y = O.block_step(kind, {}, x, w, P, G, 1e-5, 1.0, NAIVE, "none", heads=heads)
+    hb = H // P
+    for p in range(P):
+        crop = x[:, p * hb:(p + 1) * hb, :]
+        ref = lib_gn_conv(crop, w, G, 1e-5) if kind == "gn_conv" else lib_attn(crop, w, G, 1e-5, heads)
+        np.testing.assert_allclose(y[:, p * hb:(p + 1) * hb, :], ref, rtol=0, atol=1e-11)
+
+
+@pytest.mark.parametrize("kind", ["gn_conv", "resblock", "attn"])
+def test_zero_warmup_distinguishable_from_sync(kind):
+    """Zero warm-up (step 0 naive) must differ from an exact-sync step 0."""
+    r = rng(41)
+    C, H, W, P, G, heads = 8, 8, 6, 4, 4, 2
+    w = {"gn_conv": lambda: rand_gn_conv_weights(r, C, C), "resblock": lambda: rand_res_weights(r, C, C),
+         "attn": lambda: rand_attn_weights(r, C)}[kind]()
+    x = r.standard_normal((C, H, W))
+    ys = O.block_step(kind, {}, x, w, P, G, 1e-5, 1.0, SYNC, "none", heads=heads)
+    yn = O.block_step(kind, {}, x, w, P, G, 1e-5, 1.0, NAIVE, "none", heads=heads)
+    rel = np.linalg.norm(yn - ys) / np.linalg.norm(ys)
+    assert rel > 1e-3
+
+
+# ---------------------------------------------------------------- displaced invariants
+@pytest.mark.parametrize("kind", ["gn_conv", "resblock", "attn"])
+def test_unchanged_input_displaced_equals_sync(kind):
+    r = rng(50)
+    C, H, W, P, G, heads = 8, 8, 6, 4, 4, 2
+    w = {"gn_conv": lambda: rand_gn_conv_weights(r, C, C), "resblock": lambda: rand_res_weights(r, C, C),
+         "attn": lambda: rand_attn_weights(r, C)}[kind]()
+    x = r.standard_normal((C, H, W))
+    yd, trd, _ = run_two_steps(kind, x, x, w, P, G, DISPLACED, heads=heads)
+    ys, trs, _ = run_two_steps(kind, x, x, w, P, G, SYNC, heads=heads)
+    np.testing.assert_allclose(yd, ys, rtol=0, atol=1e-11)
+    for k in trd:
+        if k.endswith(".used"):
+            np.testing.assert_allclose(trd[k], trs[k], rtol=0, atol=1e-13)
+
+
+def _zero_band_mean(x, P, G):
+    C, H, W = x.shape
+    hb, cg = H // P, C // G
+    x = x.copy()
+    for p in range(P):
+        for g in range(G):
+            v = x[g * cg:(g + 1) * cg, p * hb:(p + 1) * hb, :]
+            v -= v.mean()
+    return x
+
+
+def test_uniform_drift_makes_corrected_stats_exact():
+    """Stale bands with equal per-group means, fresh = stale + delta_g: w = 1 is exact."""
+    r = rng(60)
+    C, H, W, P, G = 8, 8, 5, 4, 4
+    stale = _zero_band_mean(r.standard_normal((C, H, W)), P, G)
+    delta = np.repeat(r.standard_normal(G) * 0.3, C // G)[:, None, None]
+    fresh = stale + delta
+    f_stale = O.gn_fresh_local(stale, P, G)
+    sg, sl = O.refresh_stats(f_stale)
+    f = O.gn_fresh_local(fresh, P, G)
+    exact, _ = O.gn_used_stats(f, SYNC, None, None)
+    used, nneg = O.gn_used_stats(f, DISPLACED, sg, sl, 1.0)
+    assert nneg == 0
+    np.testing.assert_allclose(used, exact, rtol=0, atol=1e-13)
+    # w = 1/P (own band fresh, other bands stale) is not exact under a uniform drift
+    used_p, _ = O.gn_used_stats(f, DISPLACED, sg, sl, 1.0 / P)
+    assert np.abs(used_p - exact).max() > 1e-3
+
+
+def test_displaced_stats_formula_sign_and_weight():
+    """One band drifts alone: the correction moves only that band's statistics, by w * drift."""
+    r = rng(61)
+    C, H, W, P, G = 4, 8, 4, 4, 2
+    stale = r.standard_normal((C, H, W))
+    fresh = stale.copy()
+    fresh[:, 2:4, :] += 0.5          # band 1 drifts by +0.5
+    sg, sl = O.refresh_stats(O.gn_fresh_local(stale, P, G))
+    f = O.gn_fresh_local(fresh, P, G)
+    for w in (1.0, 0.25):
+        used, _ = O.gn_used_stats(f, DISPLACED, sg, sl, w)
+        for p in range(P):
+            expect_mean = sg[:, 0] + (w * 0.5 if p == 1 else 0.0)
+            np.testing.assert_allclose(used[p, :, 0], expect_mean, rtol=0, atol=1e-13)
+
+
+def test_negative_corrected_variance_falls_back_to_fresh():
+    r = rng(62)
+    C, H, W, P, G = 4, 4, 4, 2, 2
+    x = r.standard_normal((C, H, W))
+    f = O.gn_fresh_local(x, P, G)
+    sg = np.zeros((G, 2))
+    sl = f.copy()
+    sl[0, 0, 1] += 10.0               # band 0 group 0: corrected E[x^2] goes very negative
+    used, nneg = O.gn_used_stats(f, DISPLACED, sg, sl, 1.0)
+    assert nneg == 1
+    assert abs(used[0, 0, 1] - (f[0, 0, 1] - f[0, 0, 0] ** 2)) < 1e-14
+    assert used[1, 1, 1] >= 0
+
+
+def test_halo_locality():
+    """Only the stale rows adjacent to a band edge reach the displaced conv output."""
+    r = rng(70)
+    C, H, W, P, G = 8, 16, 5, 4, 4
+    w = rand_gn_conv_weights(r, C, 6)
+    x0, x1 = r.standard_normal((C, H, W)), r.standard_normal((C, H, W))
+    st = {}
+    O.block_step("gn_conv", st, x0, w, P, G, 1e-5, 1.0, SYNC, "none")
+    base_state = {"gn": st["gn"], "a_stale": st["a_stale"].copy()}
+    y0 = O.block_step("gn_conv", {"gn": _copy_gn(st["gn"]), "a_stale": st["a_stale"].copy()},
+                      x1, w, P, G, 1e-5, 1.0, DISPLACED, "none")
+    hb = H // P
+    # interior rows (offsets 1 and 2 in a 4-row band) are nobody's halo
+    a = base_state["a_stale"].copy()
+    for p in range(P):
+        a[:, p * hb + 1:p * hb + 3, :] += 5.0
+    y1 = O.block_step("gn_conv", {"gn": _copy_gn(st["gn"]), "a_stale": a}, x1, w, P, G, 1e-5,
+                      1.0, DISPLACED, "none")
+    np.testing.assert_array_equal(y1, y0)
+    # the first row of band 1 is band 0's bottom halo: only output row hb-1 changes
+    a = base_state["a_stale"].copy()
+    a[:, hb, :] += 5.0
+    y2 = O.block_step("gn_conv", {"gn": _copy_gn(st["gn"]), "a_stale": a}, x1, w, P, G, 1e-5,
+                      1.0, DISPLACED, "none")
+    changed = np.abs(y2 - y0).max(axis=(0, 2)) > 0
+    assert changed.tolist() == [r_ == hb - 1 for r_ in range(H)]
+
+
+def _copy_gn(g):
+    c = O.GNState()
+    c.stale_global, c.stale_local = g.stale_global.copy(), g.stale_local.copy()
+    return c
+
+
+def test_attention_locality():
+    """A band's own stale K/V rows are never read; other bands' stale rows are."""
+    r = rng(71)
+    T, heads, d, P = 16, 2, 4, 4
+    q, kf, vf, ks, vs = (r.standard_normal((T, heads * d)) for _ in range(5))
+    base = O.attention_stale_kv(q, kf, vf, ks, vs, P, heads, 0.5, DISPLACED)
+    tb = T // P
+    for p in range(P):
+        ks2, vs2 = ks.copy(), vs.copy()
+        ks2[p * tb:(p + 1) * tb] += 3.0
+        vs2[p * tb:(p + 1) * tb] -= 2.0
+        o = O.attention_stale_kv(q, kf, vf, ks2, vs2, P, heads, 0.5, DISPLACED)
+        own = slice(p * tb, (p + 1) * tb)
+        np.testing.assert_array_equal(o[own], base[own])
+        other = np.ones(T, bool)
+        other[own] = False
+        assert np.abs(o[other] - base[other]).min(axis=1).max() > 0
+
+
+def test_refresh_makes_fresh_the_next_stale():
+    r = rng(72)
+    C, H, W, P, G = 8, 8, 4, 4, 4
+    w = rand_gn_conv_weights(r, C, 4)
+    x = r.standard_normal((C, H, W))
+    st, tr = {}, {}
+    O.block_step("gn_conv", st, x, w, P, G, 1e-5, 1.0, SYNC, "none", trace=tr)
+    np.testing.assert_array_equal(st["a_stale"], tr["a"])
+    np.testing.assert_array_equal(st["gn"].stale_local, tr["gn.fresh_local"])
+    np.testing.assert_allclose(st["gn"].stale_global, tr["gn.fresh_local"].mean(axis=0),
+                               rtol=0, atol=0)
+
+
+def test_bf16_rounding_matches_library():
+    r = rng(80)
+    x = np.concatenate([r.standard_normal(100000) * 10, [0.0, -0.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8,
+                                                          -(1.0 + 2 ** -8), 65504.0, 1e-40]])
+    ref = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(O.to_bf16(x), ref)
