@@ -1,0 +1,438 @@
+#!/usr/bin/env python
+"""Benchmark of the displaced-patch block step; rank 0 prints one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one ``dp_block_step`` of the workload (default: the SDXL 1024 px
+top-resolution ResBlock, latent 1x320x128x128, P = 4 bands) in displaced mode,
+on synthetic inputs already resident in HBM.  Every step's kernels are timed
+with CUDA events recorded on the launching stream (``dp_block_step_timed``);
+L2 is flushed (a 256 MiB write) between steps, outside the timed events.
+With N > 1 (torchrun) every rank runs an independent replica on its own GPU:
+the path has no data exchange on one GPU per image, so there is no
+collective; the time is the max over ranks.
+
+``--impl reference`` times the CPU oracle instead (the only reference this
+method has), on the host cores, on a row crop of the same block sized so the
+whole run stays within a few minutes.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "displaced U-Net block step latency & TFLOP/s; GroupNorm GB/s; % of roofline"
+FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def kernel_source_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "displaced_patch_parallelism_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(key, src_hash):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the current source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(key)
+    if not e or e.get("source_hash") != src_hash:
+        return None
+    return e.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons while the timed region runs."""
+
+    REASONS = {0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def start(self):
+        if self.ok:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if self._thread:
+            self._stop.set()
+            self._thread.join()
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def block_kind(B, wl):
+    return {"gn_conv": B.GN_CONV, "resblock": B.RESBLOCK, "attn": B.ATTN}[wl.kind]
+
+
+def launch_roles(wl):
+    """Kernel role of each launch of one block step (dp_block_launch_count order)."""
+    if wl.kind == "gn_conv":
+        return ["gn_stats", "gn_apply", "conv"]
+    if wl.kind == "resblock":
+        r = ["gn_stats", "gn_apply", "conv", "gn_stats", "gn_apply"]
+        return r + (["linear", "conv"] if wl.cout != wl.C else ["conv"])
+    return ["gn_stats", "gn_apply", "linear", "attn", "linear"]
+
+
+def algorithmic_work(wl):
+    """Per-launch algorithmic work of every launch: (flops, bytes)."""
+    e = 2 if wl.dtype == "bf16" else 4
+    hw = wl.H * wl.W
+    out = []
+    if wl.kind in ("gn_conv", "resblock"):
+        chans = [wl.C, wl.cout]
+        convs = [(wl.C, wl.cout), (wl.cout, wl.cout)]
+        gi = ci = 0
+        for role in launch_roles(wl):
+            if role == "gn_stats":
+                out.append((0.0, hw * chans[gi] * e))
+            elif role == "gn_apply":
+                out.append((0.0, 2 * hw * chans[gi] * e))
+                gi += 1
+            elif role == "conv":
+                cin, co = convs[ci]
+                out.append((2.0 * hw * co * 9 * cin, hw * (cin * 2 + co) * e))
+                ci += 1
+            else:
+                out.append((2.0 * hw * wl.cout * wl.C, hw * (wl.C + wl.cout) * e))
+        return out
+    C, T = wl.C, hw
+    return [(0.0, T * C * e), (0.0, 2 * T * C * e), (2.0 * T * 3 * C * C, T * 4 * C * e),
+            (4.0 * T * T * C, T * 4 * C * e * 1.0), (2.0 * T * C * C, T * 3 * C * e)]
+
+
+def cpu_baseline_ours(wl, seconds):
+    """The oracle, as it stands, timed on this host: full displaced steps until `seconds` pass."""
+    from displaced_patch_parallelism_b200 import synth
+    from oracle import dp_oracle as O
+    wts = {n: v.double().numpy() for n, v in synth.make_weights(wl).items()}
+    xs = synth.InputStream(wl)
+    st = {}
+    O.block_step(wl.kind, st, xs.x(0)[0], wts, wl.P, wl.G, wl.eps, 1.0, synth.SYNC, wl.dtype,
+                 heads=wl.heads, silu=wl.silu)
+    x1 = xs.x(1)[0]
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        O.block_step(wl.kind, st, x1, wts, wl.P, wl.G, wl.eps, 1.0, synth.DISPLACED, wl.dtype,
+                     heads=wl.heads, silu=wl.silu)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return reps, el
+
+
+def wl_flops(wl):
+    hw = wl.H * wl.W
+    if wl.kind == "gn_conv":
+        return 2.0 * hw * wl.cout * 9 * wl.C
+    if wl.kind == "resblock":
+        f = 2.0 * hw * wl.cout * 9 * wl.C + 2.0 * hw * wl.cout * 9 * wl.cout
+        return f + (2.0 * hw * wl.cout * wl.C if wl.cout != wl.C else 0.0)
+    return 2.0 * hw * 3 * wl.C * wl.C + 4.0 * hw * hw * wl.C + 2.0 * hw * wl.C * wl.C
+
+
+def run_reference(args, wl):
+    """The CPU oracle on the host cores: each step a displaced step of a row crop of the block."""
+    import dataclasses
+
+    from displaced_patch_parallelism_b200 import synth
+    from oracle import dp_oracle as O
+    budget = 150.0
+    cores = len(os.sched_getaffinity(0))
+
+    def crop(rows_per_band):
+        return dataclasses.replace(wl, H=wl.P * rows_per_band)
+
+    def one_step_time(w):
+        wts = {n: v.double().numpy() for n, v in synth.make_weights(w).items()}
+        xs = synth.InputStream(w)
+        st = {}
+        O.block_step(w.kind, st, xs.x(0)[0], wts, w.P, w.G, w.eps, 1.0, synth.SYNC, w.dtype,
+                     heads=w.heads, silu=w.silu)
+        t0 = time.perf_counter()
+        O.block_step(w.kind, st, xs.x(1)[0], wts, w.P, w.G, w.eps, 1.0, synth.DISPLACED, w.dtype,
+                     heads=w.heads, silu=w.silu)
+        return time.perf_counter() - t0, wts, st, xs
+
+    hb = wl.H // wl.P
+    if wl.kind == "attn":
+        rows = hb  # attention blocks need whole 128-token tiles: keep the full image
+    else:
+        t_small, *_ = one_step_time(crop(2))
+        per_row = t_small / (2 * wl.P)
+        fit = int((budget / max(1, args.steps + args.warmup)) / max(per_row, 1e-6) / wl.P)
+        rows = max(2, min(hb, fit))
+    w = crop(rows)
+    _, wts, st, xs = one_step_time(w)
+    x = xs.x(2)[0]
+    for _ in range(args.warmup):
+        O.block_step(w.kind, st, x, wts, w.P, w.G, w.eps, 1.0, synth.DISPLACED, w.dtype,
+                     heads=w.heads, silu=w.silu)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        O.block_step(w.kind, st, x, wts, w.P, w.G, w.eps, 1.0, synth.DISPLACED, w.dtype,
+                     heads=w.heads, silu=w.silu)
+    el = time.perf_counter() - t0
+    flops = wl_flops(w)
+    value = flops * args.steps / el / 1e12
+    sample = (f"displaced step of the {wl.name} block on a {w.C}x{w.H}x{w.W} row crop "
+              f"({rows} rows per band, {flops / 1e9:.2f} GFLOP per step)")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, wl):
+    import torch
+
+    from displaced_patch_parallelism_b200 import binding as B
+    from displaced_patch_parallelism_b200 import synth
+    from displaced_patch_parallelism_b200.weights import block_weights
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dist = None
+    if ws > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    wts = synth.make_weights(wl)
+    dw = block_weights(wl.kind, wts, tdt, dev)
+    blk = B.Block(block_kind(B, wl), wl.H, wl.W, wl.C, wl.cout, wl.G, wl.P, wl.heads,
+                  B.BF16 if wl.dtype == "bf16" else B.FP32, wl.silu, wl.eps, 1.0, device=dev)
+    xs = synth.InputStream(wl)
+    pool = 4
+    host_x = [synth.nchw_to_nhwc(xs.x(k)).to(tdt).pin_memory() for k in range(pool)]
+    dev_x = [h.to(dev) for h in host_x]
+    out = torch.empty(wl.H, wl.W, wl.cout, dtype=tdt, device=dev)
+    host_out = torch.empty(out.shape, dtype=tdt).pin_memory()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    n_launch = blk.launches
+    roles = launch_roles(wl)
+    assert len(roles) == n_launch
+
+    warm = max(args.warmup, wl.warmup + 1)
+    for i in range(warm):
+        blk.step(dev_x[i % pool], out, dw, B.dp_mode_for_step(i, wl.warmup))
+    torch.cuda.synchronize()
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_launch + 1)]
+              for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    wall0 = time.perf_counter()
+    for k in range(args.steps):
+        flush.zero_()
+        blk.step_timed(dev_x[k % pool], out, dw, B.DISPLACED, events[k])
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    clocks = sampler.stop()
+    if dist:
+        dist.barrier()
+    per_launch = [[events[k][i].elapsed_time(events[k][i + 1]) for i in range(n_launch)]
+                  for k in range(args.steps)]
+    step_ms = [events[k][0].elapsed_time(events[k][n_launch]) for k in range(args.steps)]
+    total_ms = sum(step_ms)
+    if dist:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    # end-to-end: pinned host input -> device, block step, result -> pinned host, every step
+    e2e_ms = 0.0
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    xin = torch.empty_like(dev_x[0])
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for k in range(args.steps):
+        flush.zero_()
+        ev0[k].record()
+        xin.copy_(host_x[k % pool], non_blocking=True)
+        blk.step(xin, out, dw, B.DISPLACED)
+        host_out.copy_(out, non_blocking=True)
+        ev1[k].record()
+    torch.cuda.synchronize()
+    e2e_ms = sum(ev0[k].elapsed_time(ev1[k]) for k in range(args.steps))
+    if dist:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+        dist.barrier()
+    status = B.dp_device_status()
+
+    flops = blk.flops
+    value = ws * flops * args.steps / (total_ms * 1e-3) / 1e12
+    e2e_value = ws * flops * args.steps / (e2e_ms * 1e-3) / 1e12
+
+    # per-kernel roles: mean duration, share, roofline of the dominant one
+    work = algorithmic_work(wl)
+    peaks = load_peaks()
+    role_ms, role_n = {}, {}
+    for k in range(args.steps):
+        for i, r in enumerate(roles):
+            role_ms[r] = role_ms.get(r, 0.0) + per_launch[k][i]
+            role_n[r] = role_n.get(r, 0) + 1
+    kernels = {}
+    for r in role_ms:
+        idx = [i for i, rr in enumerate(roles) if rr == r]
+        fl = sum(work[i][0] for i in idx) / len(idx)
+        by = sum(work[i][1] for i in idx) / len(idx)
+        avg_us = role_ms[r] / role_n[r] * 1e3
+        kernels[r] = {"launches": role_n[r], "avg_us": round(avg_us, 2),
+                      "share": round(role_ms[r] / sum(role_ms.values()), 4),
+                      "tflops": round(fl / (avg_us * 1e-6) / 1e12, 1) if fl else None,
+                      "gbs": round(by / (avg_us * 1e-6) / 1e9, 1)}
+    dominant = max(role_ms, key=lambda r: role_ms[r])
+    dk = kernels[dominant]
+    src = {"conv": ["dp_gemm.cu"], "linear": ["dp_gemm.cu"], "attn": ["dp_attn.cu"],
+           "gn_stats": ["dp_gn.cu"], "gn_apply": ["dp_gn.cu"]}[dominant]
+    traffic = load_traffic(f"{dominant}:{wl.name}", kernel_source_hash(src))
+    if dk["tflops"]:
+        roof = {"bound": "tensor", "achieved": dk["tflops"], "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": round(dk["tflops"] / peaks["bf16_tflops"], 4),
+                "traffic": traffic, "kernel": dominant,
+                "peak_source": f"{peaks['source']} bf16 burst",
+                "frac_of_sustained": round(dk["tflops"] / peaks["bf16_tflops_sustained"], 4)
+                if peaks.get("bf16_tflops_sustained") else None}
+    else:
+        roof = {"bound": "hbm", "achieved": dk["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(dk["gbs"] / peaks["hbm_gbs"], 4), "traffic": traffic,
+                "kernel": dominant, "peak_source": f"{peaks['source']} copy"}
+    gn_ms = role_ms.get("gn_stats", 0.0) + role_ms.get("gn_apply", 0.0)
+    gn_bytes = sum(work[i][1] for i, r in enumerate(roles) if r.startswith("gn")) * args.steps
+    gn = {"achieved_gbs": round(gn_bytes / (gn_ms * 1e-3) / 1e9, 1) if gn_ms else None,
+          "peak": peaks["hbm_gbs"], "bytes_model": "stats: read x; apply: read x + write y"}
+    if gn["achieved_gbs"]:
+        gn["frac"] = round(gn["achieved_gbs"] / peaks["hbm_gbs"], 4)
+
+    line = {"metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+            "data": "synthetic",
+            "config": {"workload": wl.name, "shape_nchw": [1, wl.C, wl.H, wl.W], "P": wl.P,
+                       "mode": "displaced", "l2": "flushed between steps (256 MiB write, untimed)",
+                       "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
+            "roofline": roof, "kernels": kernels, "groupnorm": gn,
+            "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": dev_x[0].numel() * dev_x[0].element_size(),
+                    "d2h_bytes_per_step": out.numel() * out.element_size()},
+            "gpu_launches": n_launch * args.steps, "clocks": clocks,
+            "wall_s_timed_region": round(wall, 4), "device_status": status}
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        reps, el = cpu_baseline_ours(wl, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": round(wl_flops(wl) * reps / el / 1e12, 6), "unit": "TFLOP/s",
+                                "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+                                "sample": f"{reps} full displaced steps of {wl.name} in {el:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="resblock_320x128x128")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    from displaced_patch_parallelism_b200 import synth
+    wl = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        _, rank, _ = dist_env()
+        if rank == 0:
+            run_reference(args, wl)
+        return
+    run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    main()

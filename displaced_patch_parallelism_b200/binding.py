@@ -1,0 +1,256 @@
+"""ctypes binding of ``libdp.so``: argument marshalling only.
+
+Every function here has the name and argument order of its C counterpart in
+``include/dp.h``.  Tensors are passed as device pointers (``torch.Tensor`` on a
+CUDA device, an ``int`` address, or ``None`` for NULL); ``stream=None`` means
+torch's current CUDA stream.  A non-zero status raises ``DPError``.  There is
+no fallback: if the library is missing or a call fails, the caller sees it.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG_DIR, "libdp.so")
+
+DP_OK, DP_ERR_INVALID_ARG, DP_ERR_UNSUPPORTED, DP_ERR_STATE, DP_ERR_CUDA, DP_ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
+SYNC, DISPLACED, NAIVE = 0, 1, 2
+BF16, FP32 = 0, 1
+GN_CONV, RESBLOCK, ATTN = 0, 1, 2
+
+ERR_NAMES = {DP_ERR_INVALID_ARG: "DP_ERR_INVALID_ARG", DP_ERR_UNSUPPORTED: "DP_ERR_UNSUPPORTED",
+             DP_ERR_STATE: "DP_ERR_STATE", DP_ERR_CUDA: "DP_ERR_CUDA",
+             DP_ERR_TIMEOUT: "DP_ERR_TIMEOUT"}
+
+
+class DPError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"{ERR_NAMES.get(code, code)}: {msg}")
+        self.code = code
+
+
+class BlockDesc(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int),
+                ("C", ctypes.c_int), ("Cout", ctypes.c_int), ("G", ctypes.c_int),
+                ("P", ctypes.c_int), ("heads", ctypes.c_int), ("dtype", ctypes.c_int),
+                ("silu", ctypes.c_int), ("eps", ctypes.c_float), ("w", ctypes.c_float)]
+
+
+class BlockState(ctypes.Structure):
+    _fields_ = [("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+                ("cur", ctypes.c_int), ("steps_done", ctypes.c_int)]
+
+
+_V, _I, _F, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+_SIGS = {
+    "dp_last_error": ([], ctypes.c_char_p),
+    "dp_version": ([], ctypes.c_char_p),
+    "dp_mode_for_step": ([_I, _I], _I),
+    "dp_device_status": ([_V, ctypes.POINTER(_I)], _I),
+    "dp_groupnorm_workspace_size": ([_I, _I, _I, _I, _I], _SZ),
+    "dp_groupnorm_async": ([_V, _V, _V, _V, _I, _I, _I, _I, _I, _F, _F, _I, _I, _I, _V, _V, _V, _V,
+                            _V, _SZ, _V], _I),
+    "dp_conv3x3_halo": ([_V, _V, _V, _V, _V, _V, _I, _I, _I, _I, _I, _I, _I, _I, _V], _I),
+    "dp_conv3x3_halo_small": ([_V, _V, _V, _V, _V, _I, _I, _I, _I, _I, _I, _V], _I),
+    "dp_linear": ([_V, _V, _V, _V, _V, _V, _V, _I, _I, _I, _I, _V], _I),
+    "dp_attn_stale_kv": ([_V, _V, _V, _V, _V, _V, _I, _I, _I, _I, _F, _I, _V], _I),
+    "dp_refresh_stale": ([_V, _V, _SZ, _I, _I, _I, _V], _I),
+    "dp_refresh_stats": ([_V, _V, _V, _I, _I, _V], _I),
+    "dp_block_desc_init": ([ctypes.POINTER(BlockDesc), _I, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _F], _I),
+    "dp_block_workspace_size": ([ctypes.POINTER(BlockDesc)], _SZ),
+    "dp_block_state_init": ([ctypes.POINTER(BlockDesc), ctypes.POINTER(BlockState), _V, _SZ, _V], _I),
+    "dp_block_step": ([ctypes.POINTER(BlockDesc), ctypes.POINTER(BlockState), _V, _V,
+                       ctypes.POINTER(_V), _I, _I, _V], _I),
+    "dp_block_flops": ([ctypes.POINTER(BlockDesc)], ctypes.c_double),
+    "dp_block_launch_count": ([ctypes.POINTER(BlockDesc)], _I),
+    "dp_block_step_timed": ([ctypes.POINTER(BlockDesc), ctypes.POINTER(BlockState), _V, _V,
+                             ctypes.POINTER(_V), _I, _I, _V, ctypes.POINTER(_V), _I], _I),
+}
+
+_LIB = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library; raises if it has not been built."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is not built: run `python -m displaced_patch_parallelism_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGS.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _LIB = L
+    return _LIB
+
+
+def _p(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _s(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(rc: int) -> int:
+    if rc != DP_OK:
+        raise DPError(rc, lib().dp_last_error().decode())
+    return rc
+
+
+def dp_version() -> str:
+    return lib().dp_version().decode()
+
+
+def dp_mode_for_step(step: int, warmup: int) -> int:
+    rc = lib().dp_mode_for_step(step, warmup)
+    if rc < 0:
+        _check(rc)
+    return rc
+
+
+def dp_device_status(stream=None) -> int:
+    st = ctypes.c_int(0)
+    _check(lib().dp_device_status(_s(stream), ctypes.byref(st)))
+    return st.value
+
+
+def dp_groupnorm_workspace_size(H, W, C, G, P) -> int:
+    return lib().dp_groupnorm_workspace_size(H, W, C, G, P)
+
+
+def dp_groupnorm_async(x, y, gamma, beta, H, W, C, G, P, eps, w, silu, mode, dtype, stale_global,
+                       stale_local, fresh_local, used_stats, workspace, workspace_bytes=None,
+                       stream=None):
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return _check(lib().dp_groupnorm_async(
+        _p(x), _p(y), _p(gamma), _p(beta), H, W, C, G, P, eps, w, int(silu), mode, dtype,
+        _p(stale_global), _p(stale_local), _p(fresh_local), _p(used_stats), _p(workspace),
+        workspace_bytes, _s(stream)))
+
+
+def dp_conv3x3_halo(a_fresh, a_stale, weight, bias, residual, out, H, W, Cin, Cout, stride, P,
+                    mode, dtype, stream=None):
+    return _check(lib().dp_conv3x3_halo(_p(a_fresh), _p(a_stale), _p(weight), _p(bias),
+                                        _p(residual), _p(out), H, W, Cin, Cout, stride, P, mode,
+                                        dtype, _s(stream)))
+
+
+def dp_conv3x3_halo_small(a_fresh, a_stale, weight, bias, out, H, W, Cin, Cout, P, mode,
+                          stream=None):
+    return _check(lib().dp_conv3x3_halo_small(_p(a_fresh), _p(a_stale), _p(weight), _p(bias),
+                                              _p(out), H, W, Cin, Cout, P, mode, _s(stream)))
+
+
+def dp_linear(x, weight, bias, residual, out0, out1, out2, M, N, K, split, stream=None):
+    return _check(lib().dp_linear(_p(x), _p(weight), _p(bias), _p(residual), _p(out0), _p(out1),
+                                  _p(out2), M, N, K, split, _s(stream)))
+
+
+def dp_attn_stale_kv(q, k_fresh, v_fresh, k_stale, v_stale, o, T, heads, head_dim, P, scale,
+                     mode, stream=None):
+    return _check(lib().dp_attn_stale_kv(_p(q), _p(k_fresh), _p(v_fresh), _p(k_stale),
+                                         _p(v_stale), _p(o), T, heads, head_dim, P, scale, mode,
+                                         _s(stream)))
+
+
+def dp_refresh_stale(fresh, stale, row_bytes, rows, P, band=-1, stream=None):
+    return _check(lib().dp_refresh_stale(_p(fresh), _p(stale), row_bytes, rows, P, band,
+                                         _s(stream)))
+
+
+def dp_refresh_stats(fresh_local, stale_local, stale_global, P, G, stream=None):
+    return _check(lib().dp_refresh_stats(_p(fresh_local), _p(stale_local), _p(stale_global), P, G,
+                                         _s(stream)))
+
+
+def dp_block_desc_init(kind, H, W, C, Cout, G, P, heads, dtype, silu, eps, w) -> BlockDesc:
+    d = BlockDesc()
+    _check(lib().dp_block_desc_init(ctypes.byref(d), kind, H, W, C, Cout, G, P, heads, dtype,
+                                    int(silu), eps, w))
+    return d
+
+
+def dp_block_workspace_size(d: BlockDesc) -> int:
+    n = lib().dp_block_workspace_size(ctypes.byref(d))
+    if n == 0:
+        raise DPError(DP_ERR_INVALID_ARG, lib().dp_last_error().decode())
+    return n
+
+
+def dp_block_state_init(d: BlockDesc, workspace, workspace_bytes=None, stream=None) -> BlockState:
+    s = BlockState()
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().dp_block_state_init(ctypes.byref(d), ctypes.byref(s), _p(workspace),
+                                     workspace_bytes, _s(stream)))
+    return s
+
+
+def dp_block_step(d: BlockDesc, s: BlockState, x, out, weights: Sequence, mode: int, stream=None):
+    arr = (ctypes.c_void_p * len(weights))(*[_p(w) for w in weights])
+    return _check(lib().dp_block_step(ctypes.byref(d), ctypes.byref(s), _p(x), _p(out), arr,
+                                      len(weights), mode, _s(stream)))
+
+
+def dp_block_launch_count(d: BlockDesc) -> int:
+    n = lib().dp_block_launch_count(ctypes.byref(d))
+    if n < 0:
+        _check(n)
+    return n
+
+
+def dp_block_step_timed(d: BlockDesc, s: BlockState, x, out, weights: Sequence, mode: int, events,
+                        stream=None):
+    """``events``: torch.cuda.Event objects (timing enabled), at least launches + 1."""
+    arr = (ctypes.c_void_p * len(weights))(*[_p(w) for w in weights])
+    ev = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    return _check(lib().dp_block_step_timed(ctypes.byref(d), ctypes.byref(s), _p(x), _p(out), arr,
+                                            len(weights), mode, _s(stream), ev, len(events)))
+
+
+def dp_block_flops(d: BlockDesc) -> float:
+    return lib().dp_block_flops(ctypes.byref(d))
+
+
+class Block:
+    """A block descriptor, its device workspace (a torch uint8 tensor) and its state."""
+
+    def __init__(self, kind, H, W, C, Cout=0, G=32, P=4, heads=0, dtype=BF16, silu=True,
+                 eps=1e-5, w=1.0, device="cuda", stream=None):
+        import torch
+        self.desc = dp_block_desc_init(kind, H, W, C, Cout, G, P, heads, dtype, silu, eps, w)
+        self.ws_bytes = dp_block_workspace_size(self.desc)
+        self.workspace = torch.empty(self.ws_bytes, dtype=torch.uint8, device=device)
+        self.state = dp_block_state_init(self.desc, self.workspace, self.ws_bytes, stream)
+
+    def step(self, x, out, weights, mode, stream=None):
+        return dp_block_step(self.desc, self.state, x, out, weights, mode, stream)
+
+    def step_timed(self, x, out, weights, mode, events, stream=None):
+        return dp_block_step_timed(self.desc, self.state, x, out, weights, mode, events, stream)
+
+    @property
+    def launches(self) -> int:
+        return dp_block_launch_count(self.desc)
+
+    @property
+    def flops(self) -> float:
+        return dp_block_flops(self.desc)

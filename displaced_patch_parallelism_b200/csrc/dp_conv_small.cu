@@ -1,0 +1,110 @@
+// dp_conv_small.cu -- direct 3x3 conv for a handful of input channels.
+//
+// The latent entering a U-Net has 4 channels; a 3x3 conv from it has
+// K = 36, too short for a tensor-core tile, so it runs on the CUDA cores.
+// Same halo rule as the tensor-core conv ("DistriFusion", study.space
+// summary, Method): rows of other bands come from the fresh input (sync), the
+// previous step's input (displaced) or nowhere (naive).
+//
+// One thread computes 8 consecutive output channels of one pixel; the whole
+// filter bank sits in shared memory as fp32, laid out [tap][ci][co] so that
+// the 8 channels of a thread are contiguous.
+#include "dp_common.cuh"
+#include "dp_internal.h"
+
+namespace dp {
+
+__global__ void __launch_bounds__(256) conv3x3_small_kernel(
+    const __nv_bfloat16* __restrict__ af, const __nv_bfloat16* __restrict__ as,
+    const __nv_bfloat16* __restrict__ w, const float* __restrict__ bias,
+    __nv_bfloat16* __restrict__ out, int H, int W, int Cin, int Cout, int hb, int mode) {
+  extern __shared__ float sw[];   // [9][Cin][Cout]
+  const int nw = 9 * Cin * Cout;
+  for (int i = threadIdx.x; i < nw; i += blockDim.x) {
+    const int co = i % Cout, k = i / Cout;          // k = tap * Cin + ci
+    const int tap = k / Cin, ci = k % Cin;
+    sw[i] = __bfloat162float(w[(static_cast<size_t>(co) * 9 + tap) * Cin + ci]);
+  }
+  __syncthreads();
+  const int groups = Cout / 8;
+  const long idx = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<long>(H) * W * groups) return;
+  const int g = static_cast<int>(idx % groups);
+  const long pix = idx / groups;
+  const int r = static_cast<int>(pix / W), c = static_cast<int>(pix % W);
+  const int band = r / hb;
+  float acc[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] = bias ? bias[g * 8 + j] : 0.f;
+  for (int kh = 0; kh < 3; ++kh) {
+    const int rho = r + kh - 1;
+    if (rho < 0 || rho >= H) continue;
+    const __nv_bfloat16* src = af;
+    if (rho / hb != band) {
+      if (mode == DP_MODE_DISPLACED) src = as;
+      else if (mode == DP_MODE_NAIVE) continue;
+    }
+    for (int kw = 0; kw < 3; ++kw) {
+      const int col = c + kw - 1;
+      if (col < 0 || col >= W) continue;
+      const __nv_bfloat16* px = src + (static_cast<size_t>(rho) * W + col) * Cin;
+      const float* wt = sw + (kh * 3 + kw) * Cin * Cout + g * 8;
+      for (int ci = 0; ci < Cin; ++ci) {
+        const float v = __bfloat162float(px[ci]);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[j] = fmaf(v, wt[ci * Cout + j], acc[j]);
+      }
+    }
+  }
+  uint4 u;
+  u.x = pack_bf16x2(acc[0], acc[1]);
+  u.y = pack_bf16x2(acc[2], acc[3]);
+  u.z = pack_bf16x2(acc[4], acc[5]);
+  u.w = pack_bf16x2(acc[6], acc[7]);
+  *reinterpret_cast<uint4*>(out + pix * Cout + g * 8) = u;
+}
+
+int conv3x3_small_launch(const void* af, const void* as, const void* w, const float* bias,
+                         void* out, int H, int W, int Cin, int Cout, int P, int mode,
+                         cudaStream_t stream) {
+  const size_t smem = static_cast<size_t>(9) * Cin * Cout * sizeof(float);
+  static int attr_mask = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (smem > 48 * 1024 && !(attr_mask & (1 << (dev & 31)))) {
+    int rc = cuda_check(cudaFuncSetAttribute(conv3x3_small_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024),
+                        "small conv smem attribute");
+    if (rc) return rc;
+    attr_mask |= 1 << (dev & 31);
+  }
+  const long threads = static_cast<long>(H) * W * (Cout / 8);
+  const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+  mark_launch(stream);
+  conv3x3_small_kernel<<<blocks, 256, smem, stream>>>(
+      static_cast<const __nv_bfloat16*>(af), static_cast<const __nv_bfloat16*>(as ? as : af),
+      static_cast<const __nv_bfloat16*>(w), bias, static_cast<__nv_bfloat16*>(out), H, W, Cin,
+      Cout, H / P, mode);
+  return cuda_check(cudaGetLastError(), "small conv launch");
+}
+
+}  // namespace dp
+
+extern "C" int dp_conv3x3_halo_small(const void* a_fresh, const void* a_stale, const void* weight,
+                                     const float* bias, void* out, int H, int W, int Cin,
+                                     int Cout, int P, int mode, void* stream) {
+  if (!a_fresh || !weight || !out) return dp::set_error(DP_ERR_INVALID_ARG, "small conv: null pointer");
+  if (H <= 0 || W <= 0 || Cin <= 0 || Cout <= 0 || P <= 0)
+    return dp::set_error(DP_ERR_INVALID_ARG, "small conv: non-positive size");
+  if (mode < DP_MODE_SYNC || mode > DP_MODE_NAIVE)
+    return dp::set_error(DP_ERR_INVALID_ARG, "small conv: bad mode %d", mode);
+  if (mode == DP_MODE_DISPLACED && !a_stale)
+    return dp::set_error(DP_ERR_INVALID_ARG, "small conv: displaced mode needs the stale buffer");
+  if (Cin > 16 || Cout % 8 || 9L * Cin * Cout * 4 > 200 * 1024)
+    return dp::set_error(DP_ERR_UNSUPPORTED, "small conv: needs Cin <= 16, Cout %% 8 == 0, small filter bank");
+  if (H % P) return dp::set_error(DP_ERR_UNSUPPORTED, "small conv: H %% P != 0");
+  if (!dp::aligned16(out)) return dp::set_error(DP_ERR_UNSUPPORTED, "small conv: out not 16-byte aligned");
+  if (out == a_fresh || out == a_stale) return dp::set_error(DP_ERR_INVALID_ARG, "small conv: out aliases an input");
+  return dp::conv3x3_small_launch(a_fresh, a_stale, weight, bias, out, H, W, Cin, Cout, P, mode,
+                                  static_cast<cudaStream_t>(stream));
+}

@@ -1,0 +1,568 @@
+// dp_gemm.cu -- tcgen05 implicit GEMM: the stale-halo 3x3 conv and the token
+// projections.
+//
+// Conv semantics ("DistriFusion", study.space summary, Method): a band keeps
+// its interaction with the other bands by reading their rows from the
+// previous step's activations.  For output row r of band p, input row
+// rho = stride*r + kh - 1 comes from the fresh buffer if it lies in band p,
+// otherwise from the fresh buffer (sync), the stale buffer (displaced) or
+// nowhere (naive: zeros); outside the image it is zero padding.
+//
+// B200 design:
+//  * one persistent CTA per SM, 192 threads in three roles:
+//      warp 0     TMA producer (one lane): A and B tiles into a STAGES-deep
+//                 ring of 128-byte-swizzled shared-memory stages;
+//      warp 1     MMA issuer (one lane): tcgen05.mma 128 x BN x 16 into a
+//                 tensor-memory accumulator, double buffered so the
+//                 epilogue of tile i overlaps the main loop of tile i+1;
+//      warps 2-5  epilogue: tcgen05.ld, + bias (+ residual), cast, store.
+//  * implicit GEMM for the conv: M = output pixels (a tile is R rows x Wt
+//    columns, R*Wt = 128), N = Cout, K = 9 taps x Cin.  Each tap's A tile is
+//    R TMA boxes of one image row each, so every box has exactly one source:
+//    the fresh map, the stale map, or an out-of-range row that TMA fills with
+//    zeros.  Column halos use TMA's out-of-bounds zero fill too, so no
+//    padded copy of the activations is ever made.
+//  * stride 2 views the image as [H][W/2][2*Cin] (two neighbouring columns
+//    side by side in the channel axis): the three column taps become two
+//    channel halves of pairs c-1 and c, and the same TMA boxes serve.
+//  * tf32 (fp32 storage) uses the same tiles with 32 fp32 per 128-byte row.
+#include <algorithm>
+#include <cstring>
+#include <type_traits>
+
+#include "dp_common.cuh"
+#include "dp_internal.h"
+
+namespace dp {
+
+struct GemmParams {
+  CUtensorMap tmA0;   // plain A, or the conv's fresh activations
+  CUtensorMap tmA1;   // the conv's stale activations
+  CUtensorMap tmB;    // weights, [N][K] K-major
+  int a_mode;         // 0: plain [M][K] rows, 1: 3x3 conv
+  int M;
+  int H, W, Ho, Wo, Cin, stride, hb_in, hb_out, mode, R, Wt, tiles_w, kc;
+  int N, n_tiles, m_tiles, k_blocks;
+  const float* bias;
+  const void* residual;
+  void* out0;
+  void* out1;
+  void* out2;
+  int ld_out;   // elements per row of each output buffer
+  int split;    // output columns per buffer
+  int* status;
+};
+
+template <int BN, bool TF32>
+struct GemmCfg {
+  static constexpr int BM = 128;
+  static constexpr int ELEM = TF32 ? 4 : 2;
+  static constexpr int BK = 128 / ELEM;          // elements per 128-byte row
+  static constexpr int A_BYTES = BM * 128;
+  static constexpr int B_BYTES = BN * 128;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES_RAW = (200 * 1024) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  static constexpr int ACC = (2 * BN <= 512) ? 2 : 1;
+  static constexpr int COLS_NEED = ACC * BN;
+  static constexpr int TMEM_COLS =
+      COLS_NEED <= 32 ? 32 : COLS_NEED <= 64 ? 64 : COLS_NEED <= 128 ? 128 : COLS_NEED <= 256 ? 256 : 512;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 256;
+  static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
+  static_assert(B_BYTES % 1024 == 0, "stage alignment");
+};
+
+// Bounded wait that ignores the abort flag (teardown of an aborted block).
+__device__ __forceinline__ void mbar_wait_teardown(uint64_t* bar, uint32_t parity) {
+  const unsigned long long t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return;
+  }
+}
+
+template <int BN, bool TF32>
+__global__ void __launch_bounds__(192, 1) igemm_kernel(const __grid_constant__ GemmParams p) {
+  using C = GemmCfg<BN, TF32>;
+  using OutT = typename std::conditional<TF32, float, __nv_bfloat16>::type;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + C::STAGES * C::A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::STAGES * C::B_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* acc_full = empty + C::STAGES;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = warp_id(), lane = lane_id();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&p.tmA0);
+    if (p.a_mode == 1) prefetch_tmap(&p.tmA1);
+    prefetch_tmap(&p.tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int num_tiles = p.m_tiles * p.n_tiles;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0;          // bit s: stage s has a load in flight
+      uint32_t issued_par = 0;      // bit s: parity of that load's phase
+      for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x) {
+        const int mt = tile / p.n_tiles, nt = tile - mt * p.n_tiles;
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status)) goto producer_done;
+          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+          uint8_t* a_dst = sA + stage * C::A_BYTES;
+          if (p.a_mode == 0) {
+            tma_load_2d(a_dst, &p.tmA0, &full[stage], kb * C::BK, mt * 128);
+          } else {
+            const int tap = kb / p.kc, cb = kb - tap * p.kc;
+            const int kh = tap / 3, kw = tap - kh * 3;
+            const int tr = mt / p.tiles_w, tc = mt - tr * p.tiles_w;
+            const int r0 = tr * p.R, c0 = tc * p.Wt;
+            int kx, cx;
+            if (p.stride == 1) {
+              kx = cb * C::BK;
+              cx = c0 + kw - 1;
+            } else {
+              kx = (kw == 1 ? 0 : p.Cin) + cb * C::BK;
+              cx = c0 - (kw == 0 ? 1 : 0);
+            }
+            for (int i = 0; i < p.R; ++i) {
+              const int r = r0 + i;
+              const int rho = p.stride * r + kh - 1;
+              const CUtensorMap* m = &p.tmA0;
+              int ry = rho;
+              if (r >= p.Ho) {
+                ry = -1;                                   // ragged tile row: zeros
+              } else if (rho >= 0 && rho < p.H && rho / p.hb_in != r / p.hb_out) {
+                if (p.mode == DP_MODE_DISPLACED) m = &p.tmA1;       // stale halo row
+                else if (p.mode == DP_MODE_NAIVE) ry = -1;          // invisible band
+              }
+              tma_load_3d(a_dst + i * p.Wt * 128, m, &full[stage], kx, cx, ry);
+            }
+          }
+          tma_load_2d(sB + stage * C::B_BYTES, &p.tmB, &full[stage], kb * C::BK, nt * BN);
+          issued |= 1u << stage;
+          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    producer_done:
+      if (*abort_flag) {
+        // Let every load in flight land before the block's shared memory goes away.
+        for (int s = 0; s < C::STAGES; ++s)
+          if (issued & (1u << s)) mbar_wait_teardown(&full[s], (issued_par >> s) & 1u);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      constexpr uint32_t idesc = idesc_dense(128, BN, TF32 ? 2 : 1, 0, 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+        const int buf = C::ACC == 2 ? (it & 1) : 0;
+        const int use = C::ACC == 2 ? (it >> 1) : it;
+        if (!mbar_wait(&acc_empty[buf], (use & 1) ^ 1, abort_flag, p.status)) goto mma_done;
+        tc_fence_after();
+        const uint32_t d = tmem + buf * BN;
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.status)) goto mma_done;
+          tc_fence_after();
+          const uint64_t ad = sdesc_sw128(smem_u32(sA + stage * C::A_BYTES), 1024);
+          const uint64_t bd = sdesc_sw128(smem_u32(sB + stage * C::B_BYTES), 1024);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            if (TF32)
+              umma_tf32_ss(d, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0);
+            else
+              umma_f16_ss(d, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0);
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        umma_commit(&acc_full[buf]);
+      }
+    mma_done:
+      if (*abort_flag) {
+        umma_commit(drain);
+        mbar_wait_teardown(drain, 0);
+      }
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue
+    const int q = warp & 3;                 // TMEM lane quarter this warp can read
+    const int row = q * 32 + lane;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+      const int buf = C::ACC == 2 ? (it & 1) : 0;
+      const int use = C::ACC == 2 ? (it >> 1) : it;
+      if (!mbar_wait(&acc_full[buf], use & 1, abort_flag, p.status)) break;
+      tc_fence_after();
+      const int mt = tile / p.n_tiles, nt = tile - mt * p.n_tiles;
+      bool valid;
+      size_t pix;
+      if (p.a_mode == 0) {
+        const int m = mt * 128 + row;
+        valid = m < p.M;
+        pix = static_cast<size_t>(m);
+      } else {
+        const int tr = mt / p.tiles_w, tc = mt - tr * p.tiles_w;
+        const int r = tr * p.R + row / p.Wt, c = tc * p.Wt + row % p.Wt;
+        valid = r < p.Ho && c < p.Wo;
+        pix = static_cast<size_t>(r) * p.Wo + c;
+      }
+      const int n0 = nt * BN;
+      const int seg = n0 / p.split;
+      OutT* outp = static_cast<OutT*>(seg == 0 ? p.out0 : seg == 1 ? p.out1 : p.out2);
+      const int ncol0 = n0 - seg * p.split;
+      OutT* orow = outp + pix * p.ld_out + ncol0;
+      const OutT* rrow =
+          p.residual ? static_cast<const OutT*>(p.residual) + pix * p.N + n0 : nullptr;
+#pragma unroll 1
+      for (int ch = 0; ch < BN / 32; ++ch) {
+        uint32_t r[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * BN + ch * 32, r);
+        tmem_wait_ld();
+        if (ch == BN / 32 - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        }
+        if (!valid) continue;
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+        if (p.bias) {
+          const float4* b4 = reinterpret_cast<const float4*>(p.bias + n0 + ch * 32);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float4 b = __ldg(b4 + j);
+            v[4 * j] += b.x;
+            v[4 * j + 1] += b.y;
+            v[4 * j + 2] += b.z;
+            v[4 * j + 3] += b.w;
+          }
+        }
+        if (TF32) {
+          if (rrow) {
+            const float4* r4 = reinterpret_cast<const float4*>(rrow + ch * 32);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float4 x = r4[j];
+              v[4 * j] += x.x;
+              v[4 * j + 1] += x.y;
+              v[4 * j + 2] += x.z;
+              v[4 * j + 3] += x.w;
+            }
+          }
+          float4* o4 = reinterpret_cast<float4*>(orow + ch * 32);
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            o4[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        } else {
+          if (rrow) {
+            const uint4* r4 = reinterpret_cast<const uint4*>(rrow + ch * 32);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              uint4 u = r4[j];
+              const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(h[e]);
+                v[8 * j + 2 * e] += f.x;
+                v[8 * j + 2 * e + 1] += f.y;
+              }
+            }
+          }
+          uint4* o4 = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint4 u;
+            u.x = pack_bf16x2(v[8 * j], v[8 * j + 1]);
+            u.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
+            u.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
+            u.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
+            o4[j] = u;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int BN, bool TF32>
+static int launch_t(const GemmParams& p, cudaStream_t s) {
+  using C = GemmCfg<BN, TF32>;
+  static int attr_dev_mask = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!(attr_dev_mask & (1 << (dev & 31)))) {
+    int rc = cuda_check(cudaFuncSetAttribute(igemm_kernel<BN, TF32>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM),
+                        "gemm smem attribute");
+    if (rc) return rc;
+    attr_dev_mask |= 1 << (dev & 31);
+  }
+  const int tiles = p.m_tiles * p.n_tiles;
+  const int grid = std::min(tiles, num_sms());
+  mark_launch(s);
+  igemm_kernel<BN, TF32><<<grid, 192, C::SMEM, s>>>(p);
+  return cuda_check(cudaGetLastError(), "gemm launch");
+}
+
+static int launch_gemm(const GemmParams& p, int BN, bool tf32, cudaStream_t s) {
+  if (tf32) {
+    switch (BN) {
+      case 64: return launch_t<64, true>(p, s);
+      case 128: return launch_t<128, true>(p, s);
+      default: break;
+    }
+  } else {
+    switch (BN) {
+      case 32: return launch_t<32, false>(p, s);
+      case 64: return launch_t<64, false>(p, s);
+      case 96: return launch_t<96, false>(p, s);
+      case 128: return launch_t<128, false>(p, s);
+      case 160: return launch_t<160, false>(p, s);
+      case 192: return launch_t<192, false>(p, s);
+      case 256: return launch_t<256, false>(p, s);
+      default: break;
+    }
+  }
+  return set_error(DP_ERR_UNSUPPORTED, "gemm: no kernel for BN=%d", BN);
+}
+
+// Tile width in N: the candidate that divides `split` with the fewest
+// wave-quantised columns per SM (a small per-tile cost favours wider tiles).
+static int pick_bn(int m_tiles, int N, int split, bool tf32) {
+  static const int bf16_c[] = {256, 192, 160, 128, 96, 64, 32};
+  static const int tf32_c[] = {128, 64};
+  const int* c = tf32 ? tf32_c : bf16_c;
+  const int nc = tf32 ? 2 : 7;
+  int best = 0;
+  long best_cost = 0;
+  for (int i = 0; i < nc; ++i) {
+    const int bn = c[i];
+    if (split % bn) continue;
+    const long tiles = static_cast<long>(m_tiles) * (N / bn);
+    const long waves = (tiles + num_sms() - 1) / num_sms();
+    const long cost = waves * (bn + 32);
+    if (!best || cost < best_cost) {
+      best = bn;
+      best_cost = cost;
+    }
+  }
+  return best;
+}
+
+int conv3x3_launch(const void* a_fresh, const void* a_stale, const void* weight,
+                   const float* bias, const void* residual, void* out, int H, int W, int Cin,
+                   int Cout, int stride, int P, int mode, int dtype, cudaStream_t stream) {
+  const bool tf32 = dtype == DP_FP32;
+  const int e = tf32 ? 4 : 2;
+  const int BK = 128 / e;
+  const int Ho = (H - 1) / stride + 1, Wo = (W - 1) / stride + 1;
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  p.a_mode = 1;
+  p.H = H;
+  p.W = W;
+  p.Ho = Ho;
+  p.Wo = Wo;
+  p.Cin = Cin;
+  p.stride = stride;
+  p.hb_in = H / P;
+  p.hb_out = Ho / P;
+  p.mode = mode;
+  // tile shape: Wt columns x R rows, Wt a power of two in [8, 128] wasting the fewest columns
+  int Wt = 128, waste_best = 1 << 30;
+  for (int w = 128; w >= 8; w >>= 1) {
+    const int waste = ((Wo + w - 1) / w) * w - Wo;
+    if (waste < waste_best) {
+      waste_best = waste;
+      Wt = w;
+    }
+  }
+  p.Wt = Wt;
+  p.R = 128 / Wt;
+  p.tiles_w = (Wo + Wt - 1) / Wt;
+  p.m_tiles = p.tiles_w * ((Ho + p.R - 1) / p.R);
+  p.kc = Cin / BK;
+  p.k_blocks = 9 * p.kc;
+  p.N = Cout;
+  p.split = Cout;
+  p.ld_out = Cout;
+  p.bias = bias;
+  p.residual = residual;
+  p.out0 = out;
+  p.status = device_status_ptr();
+  const int BN = pick_bn(p.m_tiles, Cout, Cout, tf32);
+  if (!BN) return set_error(DP_ERR_UNSUPPORTED, "conv: no N tile divides Cout=%d", Cout);
+  p.n_tiles = Cout / BN;
+  const CUtensorMapDataType dt =
+      tf32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  uint64_t dims[3], str[2];
+  uint32_t box[3] = {static_cast<uint32_t>(BK), static_cast<uint32_t>(Wt), 1};
+  if (stride == 1) {
+    dims[0] = Cin; dims[1] = W; dims[2] = H;
+    str[0] = static_cast<uint64_t>(Cin) * e;
+    str[1] = static_cast<uint64_t>(W) * Cin * e;
+  } else {
+    dims[0] = 2 * static_cast<uint64_t>(Cin); dims[1] = W / 2; dims[2] = H;
+    str[0] = 2 * static_cast<uint64_t>(Cin) * e;
+    str[1] = static_cast<uint64_t>(W) * Cin * e;
+  }
+  int rc = encode_tmap(&p.tmA0, dt, 3, const_cast<void*>(a_fresh), dims, str, box,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc) return rc;
+  rc = encode_tmap(&p.tmA1, dt, 3, const_cast<void*>(a_stale ? a_stale : a_fresh), dims, str, box,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc) return rc;
+  uint64_t bdims[2] = {9 * static_cast<uint64_t>(Cin), static_cast<uint64_t>(Cout)};
+  uint64_t bstr[1] = {9 * static_cast<uint64_t>(Cin) * e};
+  uint32_t bbox[2] = {static_cast<uint32_t>(BK), static_cast<uint32_t>(BN)};
+  rc = encode_tmap(&p.tmB, dt, 2, const_cast<void*>(weight), bdims, bstr, bbox,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc) return rc;
+  return launch_gemm(p, BN, tf32, stream);
+}
+
+int linear_launch(const void* x, const void* weight, const float* bias, const void* residual,
+                  void* out0, void* out1, void* out2, int M, int N, int K, int split,
+                  cudaStream_t stream) {
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  p.a_mode = 0;
+  p.M = M;
+  p.m_tiles = (M + 127) / 128;
+  p.k_blocks = K / 64;
+  p.N = N;
+  p.split = split;
+  p.ld_out = split;
+  p.bias = bias;
+  p.residual = residual;
+  p.out0 = out0;
+  p.out1 = out1;
+  p.out2 = out2;
+  p.status = device_status_ptr();
+  const int BN = pick_bn(p.m_tiles, N, split, false);
+  if (!BN) return set_error(DP_ERR_UNSUPPORTED, "linear: no N tile divides split=%d", split);
+  p.n_tiles = N / BN;
+  uint64_t adims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
+  uint64_t astr[1] = {static_cast<uint64_t>(K) * 2};
+  uint32_t abox[2] = {64, 128};
+  int rc = encode_tmap(&p.tmA0, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), adims,
+                       astr, abox, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc) return rc;
+  uint64_t bdims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N)};
+  uint32_t bbox[2] = {64, static_cast<uint32_t>(BN)};
+  rc = encode_tmap(&p.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(weight), bdims,
+                   astr, bbox, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc) return rc;
+  return launch_gemm(p, BN, false, stream);
+}
+
+int conv3x3_validate(const void* a_fresh, const void* a_stale, const void* weight,
+                     const void* residual, const void* out, int H, int W, int Cin, int Cout,
+                     int stride, int P, int mode, int dtype) {
+  if (!a_fresh || !weight || !out) return set_error(DP_ERR_INVALID_ARG, "conv: null pointer");
+  if (H <= 0 || W <= 0 || Cin <= 0 || Cout <= 0 || P <= 0)
+    return set_error(DP_ERR_INVALID_ARG, "conv: non-positive size");
+  if (mode < DP_MODE_SYNC || mode > DP_MODE_NAIVE)
+    return set_error(DP_ERR_INVALID_ARG, "conv: bad mode %d", mode);
+  if (dtype != DP_BF16 && dtype != DP_FP32) return set_error(DP_ERR_INVALID_ARG, "conv: bad dtype");
+  if (stride != 1 && stride != 2) return set_error(DP_ERR_UNSUPPORTED, "conv: stride must be 1 or 2");
+  if (mode == DP_MODE_DISPLACED && !a_stale)
+    return set_error(DP_ERR_INVALID_ARG, "conv: displaced mode needs the stale buffer");
+  const int BK = dtype == DP_FP32 ? 32 : 64;
+  if (Cin % BK) return set_error(DP_ERR_UNSUPPORTED, "conv: Cin must be a multiple of %d", BK);
+  if (Cout % 32) return set_error(DP_ERR_UNSUPPORTED, "conv: Cout must be a multiple of 32");
+  if (dtype == DP_FP32 && Cout % 64) return set_error(DP_ERR_UNSUPPORTED, "conv: fp32 needs Cout %% 64 == 0");
+  const int Ho = (H - 1) / stride + 1;
+  if (H % P || Ho % P) return set_error(DP_ERR_UNSUPPORTED, "conv: rows not divisible by P");
+  if (stride == 2 && (W % 2)) return set_error(DP_ERR_UNSUPPORTED, "conv: stride 2 needs even W");
+  if (!aligned16(a_fresh) || (a_stale && !aligned16(a_stale)) || !aligned16(weight) ||
+      !aligned16(out) || (residual && !aligned16(residual)))
+    return set_error(DP_ERR_UNSUPPORTED, "conv: pointers must be 16-byte aligned");
+  if (a_stale && (a_stale == out)) return set_error(DP_ERR_INVALID_ARG, "conv: out aliases a_stale");
+  if (a_fresh == out) return set_error(DP_ERR_INVALID_ARG, "conv: out aliases a_fresh");
+  return DP_OK;
+}
+
+}  // namespace dp
+
+extern "C" {
+
+int dp_conv3x3_halo(const void* a_fresh, const void* a_stale, const void* weight,
+                    const float* bias, const void* residual, void* out, int H, int W, int Cin,
+                    int Cout, int stride, int P, int mode, int dtype, void* stream) {
+  int rc = dp::conv3x3_validate(a_fresh, a_stale, weight, residual, out, H, W, Cin, Cout, stride,
+                                P, mode, dtype);
+  if (rc) return rc;
+  if (bias && !dp::aligned16(bias)) return dp::set_error(DP_ERR_UNSUPPORTED, "conv: bias not 16-byte aligned");
+  return dp::conv3x3_launch(a_fresh, a_stale, weight, bias, residual, out, H, W, Cin, Cout, stride,
+                            P, mode, dtype, static_cast<cudaStream_t>(stream));
+}
+
+int dp_linear(const void* x, const void* weight, const float* bias, const void* residual,
+              void* out0, void* out1, void* out2, int M, int N, int K, int split, void* stream) {
+  if (!x || !weight || !out0) return dp::set_error(DP_ERR_INVALID_ARG, "linear: null pointer");
+  if (M <= 0 || N <= 0 || K <= 0 || split <= 0)
+    return dp::set_error(DP_ERR_INVALID_ARG, "linear: non-positive size");
+  if (K % 64) return dp::set_error(DP_ERR_UNSUPPORTED, "linear: K must be a multiple of 64");
+  if (split % 32 || N % split || N / split > 3)
+    return dp::set_error(DP_ERR_UNSUPPORTED, "linear: need split %% 32 == 0, N = k*split, k <= 3");
+  const int nseg = N / split;
+  if ((nseg > 1 && !out1) || (nseg > 2 && !out2))
+    return dp::set_error(DP_ERR_INVALID_ARG, "linear: missing output buffer");
+  if (residual && nseg != 1)
+    return dp::set_error(DP_ERR_UNSUPPORTED, "linear: residual needs a single output");
+  if (!dp::aligned16(x) || !dp::aligned16(weight) || !dp::aligned16(out0) ||
+      (out1 && !dp::aligned16(out1)) || (out2 && !dp::aligned16(out2)) ||
+      (residual && !dp::aligned16(residual)) || (bias && !dp::aligned16(bias)))
+    return dp::set_error(DP_ERR_UNSUPPORTED, "linear: pointers must be 16-byte aligned");
+  return dp::linear_launch(x, weight, bias, residual, out0, out1, out2, M, N, K, split,
+                           static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,31 @@
+// dp_internal.h -- launchers shared between the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace dp {
+
+size_t gn_workspace_bytes(int P, int G);
+int gn_launch(const void* x, void* y, const float* gamma, const float* beta, int H, int W, int C,
+              int G, int P, float eps, float w, int silu, int mode, int dtype,
+              const float* stale_global, const float* stale_local, float* fresh_local,
+              float* fresh_global, float* used, void* workspace, cudaStream_t stream);
+int conv3x3_validate(const void* a_fresh, const void* a_stale, const void* weight,
+                     const void* residual, const void* out, int H, int W, int Cin, int Cout,
+                     int stride, int P, int mode, int dtype);
+int conv3x3_launch(const void* a_fresh, const void* a_stale, const void* weight,
+                   const float* bias, const void* residual, void* out, int H, int W, int Cin,
+                   int Cout, int stride, int P, int mode, int dtype, cudaStream_t stream);
+int linear_launch(const void* x, const void* weight, const float* bias, const void* residual,
+                  void* out0, void* out1, void* out2, int M, int N, int K, int split,
+                  cudaStream_t stream);
+int attn_validate(const void* q, const void* kf, const void* vf, const void* ks, const void* vs,
+                  const void* o, int T, int heads, int head_dim, int P, int mode);
+int attn_launch(const void* q, const void* kf, const void* vf, const void* ks, const void* vs,
+                void* o, int T, int heads, int P, float scale, int mode, cudaStream_t stream);
+void recorder_begin(void* const* events, int n);
+int recorder_end();
+int copy_launch(const void* src, void* dst, size_t bytes, cudaStream_t stream);
+
+}  // namespace dp

@@ -1,0 +1,50 @@
+"""Marshalling of a block's weights into the device layouts ``dp_block_step`` expects.
+
+Layout changes only (no arithmetic of the method): conv filters go from
+(Cout, Cin, 3, 3) to [Cout][3][3][Cin]; the q, k and v projection matrices are
+stacked into one [3C][C] matrix so a single GEMM produces all three; GroupNorm
+scale/shift and biases are fp32.
+"""
+from __future__ import annotations
+
+from typing import Dict, List
+
+import torch
+
+
+def _t(a, dtype, device):
+    t = a if isinstance(a, torch.Tensor) else torch.as_tensor(a)
+    return t.to(torch.float32).to(dtype).contiguous().to(device)
+
+
+def _conv(w, dtype, device):
+    t = w if isinstance(w, torch.Tensor) else torch.as_tensor(w)
+    return t.to(torch.float32).permute(0, 2, 3, 1).contiguous().to(dtype).to(device)
+
+
+def block_weights(kind: str, wts: Dict, dtype: torch.dtype = torch.bfloat16, device="cuda",
+                  prefix: str = "") -> List[torch.Tensor]:
+    """Device tensors in the order ``dp_block_step`` documents for ``kind``."""
+    g = lambda n: wts[prefix + n]
+    f32 = torch.float32
+    if kind == "gn_conv":
+        return [_t(g("gn_gamma"), f32, device), _t(g("gn_beta"), f32, device),
+                _conv(g("conv_w"), dtype, device), _t(g("conv_b"), f32, device)]
+    if kind == "resblock":
+        out = [_t(g("gn1_gamma"), f32, device), _t(g("gn1_beta"), f32, device),
+               _conv(g("conv1_w"), dtype, device), _t(g("conv1_b"), f32, device),
+               _t(g("gn2_gamma"), f32, device), _t(g("gn2_beta"), f32, device),
+               _conv(g("conv2_w"), dtype, device), _t(g("conv2_b"), f32, device)]
+        if (prefix + "short_w") in wts:
+            sw = g("short_w")
+            sw = sw if isinstance(sw, torch.Tensor) else torch.as_tensor(sw)
+            out += [_t(sw.reshape(sw.shape[0], sw.shape[1]), dtype, device),
+                    _t(g("short_b"), f32, device)]
+        return out
+    if kind == "attn":
+        cat = lambda *xs: torch.cat([x if isinstance(x, torch.Tensor) else torch.as_tensor(x) for x in xs])
+        return [_t(g("gn_gamma"), f32, device), _t(g("gn_beta"), f32, device),
+                _t(cat(g("wq"), g("wk"), g("wv")), dtype, device),
+                _t(cat(g("bq"), g("bk"), g("bv")), f32, device),
+                _t(g("wo"), dtype, device), _t(g("bo"), f32, device)]
+    raise ValueError(kind)

@@ -1,0 +1,296 @@
+/*
+ * dp.h -- C ABI of the displaced-patch-parallelism block step for B200 (sm_100a).
+ *
+ * The method is DistriFusion's displaced patch parallelism ("DistriFusion:
+ * Distributed Parallel Inference for High-Resolution Diffusion Models",
+ * study.space summary, Method; atlas.scime.ai summary, Approach): an image
+ * latent is split into P row patches ("bands"); every band computes its own
+ * rows with fresh activations and takes the context it needs from the other
+ * bands out of the previous denoising step's activations.  Here all P bands
+ * live on one GPU and are computed in one launch per layer; the paper's
+ * per-layer AllGather becomes a device-local refresh of the stale buffers.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Every call returns an int status: DP_OK or one of the DP_ERR_* codes.
+ *    dp_last_error() returns a message for the calling thread's last error.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL is the legacy default stream) and never synchronises.  Kernel-side
+ *    failures (a bounded wait that ran out) are recorded in a device status
+ *    word that dp_device_status() reads.
+ *  - The caller owns every buffer.  No call allocates, frees or keeps a
+ *    pointer past its return, except that dp_block_state remembers its
+ *    workspace pointer.
+ *  - Device pointers must be 16-byte aligned.  Images are NHWC (row-major
+ *    [H][W][C], batch 1); token matrices are row-major [T][C] with tokens in
+ *    raster order of the image, so band p of an HxW image is the contiguous
+ *    token range [p*T/P, (p+1)*T/P).
+ *  - Bands are equal: H % P == 0 (DP_ERR_UNSUPPORTED otherwise).
+ *  - Modes: DP_MODE_SYNC (warm-up step: every band sees fresh context),
+ *    DP_MODE_DISPLACED (other bands' context is the stale previous step),
+ *    DP_MODE_NAIVE (other bands are invisible: zero halo, own keys only).
+ *  - dtype: DP_BF16 (bf16 storage, fp32 accumulation) or DP_FP32 (fp32
+ *    storage; the 3x3 conv then multiplies in tf32 with fp32 accumulation).
+ *    Statistics, GroupNorm scale/shift and biases are always fp32.
+ */
+#ifndef DP_H
+#define DP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DP_API __attribute__((visibility("default")))
+#else
+#define DP_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* status codes */
+#define DP_OK 0
+#define DP_ERR_INVALID_ARG (-1) /* null pointer, bad size, bad enum            */
+#define DP_ERR_UNSUPPORTED (-2) /* shape / alignment / dtype the kernels lack   */
+#define DP_ERR_STATE (-3)       /* displaced step before any step filled state  */
+#define DP_ERR_CUDA (-4)        /* a CUDA runtime or driver call failed         */
+#define DP_ERR_TIMEOUT (-5)     /* a device-side bounded wait ran out           */
+
+/* step modes */
+#define DP_MODE_SYNC 0
+#define DP_MODE_DISPLACED 1
+#define DP_MODE_NAIVE 2
+
+/* storage types */
+#define DP_BF16 0
+#define DP_FP32 1
+
+/* block kinds for dp_block_desc_init */
+#define DP_BLOCK_GN_CONV 0  /* GroupNorm (+SiLU) -> 3x3 conv                                */
+#define DP_BLOCK_RESBLOCK 1 /* GN -> SiLU -> conv1 -> GN -> SiLU -> conv2 -> + x / shortcut */
+#define DP_BLOCK_ATTN 2     /* GN -> q,k,v proj -> stale-K/V attention -> out proj -> + x   */
+
+/* Message for the calling thread's last failed call ("" if none). */
+DP_API const char* dp_last_error(void);
+
+/* Library version string. */
+DP_API const char* dp_version(void);
+
+/*
+ * Mode of denoising step `step` with `warmup` synchronous warm-up steps.
+ * Warm-up steps run synchronously (atlas.scime.ai summary, warm-up ablation
+ * rows: removing them hurts quality).  With zero warm-up, step 0 has no
+ * previous step to borrow context from and runs as independent patches
+ * (DP_MODE_NAIVE).  Later steps are DP_MODE_DISPLACED.
+ */
+DP_API int dp_mode_for_step(int step, int warmup);
+
+/*
+ * Reads and clears the device status word that kernels set when a bounded
+ * wait runs out.  Synchronises `stream` first.  *status receives DP_OK or
+ * DP_ERR_TIMEOUT.  Returns DP_ERR_CUDA if the read fails.
+ */
+DP_API int dp_device_status(void* stream, int* status);
+
+/* ------------------------------------------------------------------------
+ * Corrected asynchronous GroupNorm, fused with SiLU and the storage cast.
+ * (atlas.scime.ai summary, Approach: "a corrected asynchronous GroupNorm";
+ *  GroupNorm ablation rows: on-device-only, stale-only and synchronous
+ *  statistics are the alternatives it improves on.)
+ *
+ * For band p and group g (C/G consecutive channels) the fresh raw moments
+ * f[p][g] = (E[x], E[x^2]) over the band's rows are reduced from x.  The
+ * moments each band normalises with are
+ *   SYNC:       the whole-image moments, mean over bands of f;
+ *   DISPLACED:  stale_global[g] + w * (f[p][g] - stale_local[p][g]);
+ *   NAIVE:      f[p][g].
+ * var = E[x^2] - E[x]^2; a negative corrected var falls back to the band's
+ * fresh var.  Then y = (x - mean) * rsqrt(var + eps) * gamma_c + beta_c, and
+ * if silu != 0, y = y * sigmoid(y); y is stored in `dtype`.
+ *
+ *  x            [H][W][C] dtype, device, read
+ *  y            [H][W][C] dtype, device, written (may not alias x)
+ *  gamma, beta  [C] fp32, device
+ *  stale_global [G][2] fp32 (mean, E[x^2]), device; read in DISPLACED only
+ *  stale_local  [P][G][2] fp32, device; read in DISPLACED only
+ *  fresh_local  [P][G][2] fp32, device, written: f (the next step's stale_local)
+ *  used_stats   [P][G][2] fp32 (mean, var), device, written
+ *  workspace    device scratch of dp_groupnorm_workspace_size() bytes; it must
+ *               be zero-filled before its first use and is left zero-filled
+ *               by every call that completes.  Calls that overlap on the GPU
+ *               must not share a workspace.
+ * Needs C % G == 0, C % 8 == 0 (bf16) or C % 4 == 0 (fp32), C/8 <= 1024.
+ * ---------------------------------------------------------------------- */
+DP_API size_t dp_groupnorm_workspace_size(int H, int W, int C, int G, int P);
+DP_API int dp_groupnorm_async(const void* x, void* y, const float* gamma, const float* beta,
+                       int H, int W, int C, int G, int P, float eps, float w, int silu,
+                       int mode, int dtype, const float* stale_global,
+                       const float* stale_local, float* fresh_local, float* used_stats,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * 3x3 convolution, padding 1, stride 1 or 2, whose halo rows come from the
+ * stale buffer (study.space summary, Method: patches reuse the previous
+ * step's activations to keep their interaction).
+ *
+ * Output row r of band p (band = Ho/P output rows) reads input row
+ * rho = stride*r + kh - 1: rho outside [0,H) is zero padding; rho inside
+ * band p (band = H/P input rows) comes from a_fresh; rho in another band
+ * comes from a_fresh (SYNC), a_stale (DISPLACED) or is zero (NAIVE).
+ * Columns use ordinary zero padding.  out = conv + bias (+ residual).
+ *
+ *  a_fresh, a_stale  [H][W][Cin] dtype, device (a_stale read in DISPLACED only)
+ *  weight            [Cout][3][3][Cin] dtype, device
+ *  bias              [Cout] fp32, device, or NULL
+ *  residual          [Ho][Wo][Cout] dtype, device, or NULL
+ *  out               [Ho][Wo][Cout] dtype, device, written
+ * Ho = (H-1)/stride + 1.  Needs Cin % 64 == 0 (bf16) or % 32 == 0 (fp32),
+ * Cout % 32 == 0 (fp32: Cout % 64 == 0), H % P == 0, Ho % P == 0, W even when
+ * stride 2.  Any W works; ragged tiles are masked.
+ * Runs on the tensor cores (tcgen05, operands staged by TMA).
+ * ---------------------------------------------------------------------- */
+DP_API int dp_conv3x3_halo(const void* a_fresh, const void* a_stale, const void* weight,
+                    const float* bias, const void* residual, void* out, int H, int W,
+                    int Cin, int Cout, int stride, int P, int mode, int dtype, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Direct 3x3 conv for few input channels (the latent input conv), same
+ * halo rule and layouts as dp_conv3x3_halo, stride 1, bf16 only.
+ * Needs Cin <= 16, Cout % 8 == 0.  Runs on the CUDA cores.
+ * ---------------------------------------------------------------------- */
+DP_API int dp_conv3x3_halo_small(const void* a_fresh, const void* a_stale, const void* weight,
+                          const float* bias, void* out, int H, int W, int Cin, int Cout,
+                          int P, int mode, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Token projection y = x W^T + bias (+ residual), bf16, on the tensor cores:
+ * the q/k/v and output projections around the attention, and the 1x1
+ * shortcut conv of a ResBlock whose channels change.
+ *
+ *  x         [M][K] bf16, device
+ *  weight    [N][K] bf16, device (an nn.Linear-style (out, in) matrix)
+ *  bias      [N] fp32 or NULL;  residual [M][N] bf16 or NULL
+ *  out0..2   output column ranges [0,split), [split,2*split), [2*split,3*split)
+ *            go to out0, out1, out2 ([M][split] each); with split == N only
+ *            out0 is used.  The fused q/k/v projection writes k and v
+ *            straight into the fresh half of the caller's K/V buffers.
+ * Needs K % 64 == 0, split % 32 == 0, N % split == 0, N / split <= 3.
+ * ---------------------------------------------------------------------- */
+DP_API int dp_linear(const void* x, const void* weight, const float* bias, const void* residual,
+              void* out0, void* out1, void* out2, int M, int N, int K, int split,
+              void* stream);
+
+/* ------------------------------------------------------------------------
+ * Self-attention over stitched fresh / stale keys and values (gist.science
+ * PipeFusion explainer, Problem Statement: DistriFusion keeps full-spatial K
+ * and V of every layer on every device).  For a query in band p and each
+ * head: softmax(q K^T * scale) V over the keys band p sees: band p's own keys
+ * and values are fresh; the other bands' are fresh (SYNC), stale (DISPLACED)
+ * or left out (NAIVE).
+ *
+ *  q, k_fresh, v_fresh, k_stale, v_stale, o   [T][heads*head_dim] bf16, device
+ *  (k_stale, v_stale read in DISPLACED only; o may not alias an input)
+ * Needs head_dim == 64, T % P == 0 and (T/P) % 128 == 0.
+ * Runs on the tensor cores (tcgen05, S and O in tensor memory).
+ * ---------------------------------------------------------------------- */
+DP_API int dp_attn_stale_kv(const void* q, const void* k_fresh, const void* v_fresh,
+                     const void* k_stale, const void* v_stale, void* o, int T, int heads,
+                     int head_dim, int P, float scale, int mode, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Stale-buffer refresh: the device-local replacement of the paper's
+ * per-layer AllGather (atlas.scime.ai summary, Approach: AllGather overlaps
+ * computation; limitations: NCCL kernels take SMs).  Copies the rows of band
+ * `band` (all bands if band == -1) from `fresh` to `stale`; a band is
+ * rows/P rows of row_bytes bytes.  row_bytes % 16 == 0, rows % P == 0.
+ * fresh and stale may not overlap.
+ * ---------------------------------------------------------------------- */
+DP_API int dp_refresh_stale(const void* fresh, void* stale, size_t row_bytes, int rows, int P,
+                     int band, void* stream);
+
+/* Statistics refresh: stale_local = fresh_local; stale_global[g] = mean over
+ * bands of fresh_local[p][g].  All [.][2] fp32 device arrays. */
+DP_API int dp_refresh_stats(const float* fresh_local, float* stale_local, float* stale_global,
+                     int P, int G, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Block step: one U-Net block over all P bands, with its cross-step state
+ * (stale activations, stale K/V, stale GroupNorm statistics) held in a
+ * caller-allocated device workspace.  The refresh at the end of a step is a
+ * ping-pong flip of the fresh/stale halves: 0 bytes move.
+ *
+ * Setup:  dp_block_desc_init -> dp_block_workspace_size -> caller allocates
+ *         -> dp_block_state_init (zero-fills, steps_done = 0).
+ * ---------------------------------------------------------------------- */
+typedef struct dp_block_desc {
+  int kind;       /* DP_BLOCK_*                                   */
+  int H, W;       /* image rows and columns                       */
+  int C, Cout;    /* input / output channels (ATTN: Cout == C)    */
+  int G, P;       /* GroupNorm groups, bands                      */
+  int heads;      /* ATTN: heads (head_dim 64)                    */
+  int dtype;      /* DP_BF16 or DP_FP32 (FP32: GN_CONV only)      */
+  int silu;       /* GN_CONV: SiLU after GroupNorm                */
+  float eps;      /* GroupNorm epsilon                            */
+  float w;        /* weight of the corrected-statistics drift term */
+} dp_block_desc;
+
+typedef struct dp_block_state {
+  void* workspace;        /* device memory of dp_block_workspace_size() bytes */
+  size_t workspace_bytes;
+  int cur;                /* which half of each ping-pong pair is stale       */
+  int steps_done;         /* steps completed since dp_block_state_init        */
+} dp_block_state;
+
+DP_API int dp_block_desc_init(dp_block_desc* d, int kind, int H, int W, int C, int Cout, int G,
+                       int P, int heads, int dtype, int silu, float eps, float w);
+DP_API size_t dp_block_workspace_size(const dp_block_desc* d);
+DP_API int dp_block_state_init(const dp_block_desc* d, dp_block_state* s, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
+/*
+ * Runs one step of the block in `mode` and then refreshes the state.
+ *  x    block input, [H][W][C] dtype, device (ATTN: the same image as tokens)
+ *  out  block output, [H][W][Cout] dtype, device (may not alias x)
+ *  weights: device pointers, in this order per kind --
+ *   GN_CONV:  gn_gamma[C], gn_beta[C], conv_w[Cout][3][3][C], conv_b[Cout]
+ *   RESBLOCK: gn1_gamma[C], gn1_beta[C], conv1_w[Cout][3][3][C], conv1_b[Cout],
+ *             gn2_gamma[Cout], gn2_beta[Cout], conv2_w[Cout][3][3][Cout],
+ *             conv2_b[Cout], then if C != Cout: short_w[Cout][C], short_b[Cout]
+ *   ATTN:     gn_gamma[C], gn_beta[C], wqkv[3C][C] (the q, k and v (out, in)
+ *             matrices stacked), bqkv[3C], wo[C][C], bo[C]
+ *  Weight matrices are `dtype`; gamma, beta and biases fp32 (biases may be NULL).
+ * Returns DP_ERR_STATE for DISPLACED before any completed step.
+ */
+DP_API int dp_block_step(const dp_block_desc* d, dp_block_state* s, const void* x, void* out,
+                  const void* const* weights, int n_weights, int mode, void* stream);
+
+/*
+ * Number of kernel launches one dp_block_step makes for this descriptor, in
+ * this order --
+ *   GN_CONV:  GN statistics, GN apply, conv
+ *   RESBLOCK: GN1 statistics, GN1 apply, conv1, GN2 statistics, GN2 apply,
+ *             [1x1 shortcut if C != Cout], conv2
+ *   ATTN:     GN statistics, GN apply, q/k/v projection, attention, out projection
+ * Negative status on a bad descriptor.
+ */
+DP_API int dp_block_launch_count(const dp_block_desc* d);
+
+/*
+ * dp_block_step that also records events[i] (cudaEvent_t, passed as void*)
+ * on `stream` just before its i-th kernel launch and events[n] after the
+ * last, n = dp_block_launch_count(d); n_events must be >= n + 1.  The
+ * elapsed time between events[i] and events[i+1] is launch i's duration.
+ */
+DP_API int dp_block_step_timed(const dp_block_desc* d, dp_block_state* s, const void* x, void* out,
+                               const void* const* weights, int n_weights, int mode, void* stream,
+                               void* const* events, int n_events);
+
+/* Algorithmic FLOPs of one block step (multiply-adds count 2). */
+DP_API double dp_block_flops(const dp_block_desc* d);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DP_H */

@@ -212,6 +212,42 @@ def conv3x3_halo(a_fresh: np.ndarray, a_stale: Optional[np.ndarray], weight: np.
     return out
 
 
+def conv3x3_halo_rows(a_fresh: np.ndarray, a_stale: Optional[np.ndarray], weight: np.ndarray,
+                      bias: Optional[np.ndarray], P: int, mode: int, rows, stride: int = 1
+                      ) -> np.ndarray:
+    """Only the output rows ``rows`` of ``conv3x3_halo`` (no residual), one row at a time.
+
+    Same rule as ``conv3x3_halo``, applied to the three input rows one output
+    row reads; used to check single rows of full-size images.
+    Returns (Cout, len(rows), Wo).
+    """
+    Cin, H, W = a_fresh.shape
+    Ho = (H - 1) // stride + 1
+    Wo = (W - 1) // stride + 1
+    hb_in, hb_out = H // P, Ho // P
+    out = np.zeros((weight.shape[0], len(rows), Wo))
+    for i, r in enumerate(rows):
+        p = r // hb_out
+        for kh in range(3):
+            rho = stride * r + kh - 1
+            if rho < 0 or rho >= H:
+                continue
+            if rho // hb_in == p or mode == SYNC:
+                src = a_fresh
+            elif mode == DISPLACED:
+                src = a_stale
+            else:
+                continue
+            line = np.zeros((Cin, W + 2))
+            line[:, 1:W + 1] = src[:, rho, :]
+            for kw in range(3):
+                seg = line[:, kw:kw + stride * (Wo - 1) + 1:stride]
+                out[:, i, :] += weight[:, :, kh, kw] @ seg
+    if bias is not None:
+        out += bias[:, None, None]
+    return out
+
+
 def conv1x1(x: np.ndarray, weight: np.ndarray, bias: Optional[np.ndarray]) -> np.ndarray:
     """Pointwise conv (the ResBlock shortcut when channels change)."""
     out = np.tensordot(weight[:, :, 0, 0], x, axes=(1, 0))
@@ -293,7 +329,8 @@ def _a(x) -> np.ndarray:
 
 
 def gn_conv_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float,
-                 silu: bool, mode: int, storage: str, trace: Optional[Dict] = None):
+                 silu: bool, mode: int, storage: str, trace: Optional[Dict] = None,
+                 final_storage: Optional[str] = None):
     """GroupNorm (+SiLU) -> 3x3 conv with stale halo.  x: (C, H, W)."""
     x = _a(x)
     gn = state.setdefault("gn", GNState())
@@ -302,7 +339,7 @@ def gn_conv_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float
     a = store(a, storage)
     out = conv3x3_halo(a, state.get("a_stale"), _a(wts["conv_w"]), _a(wts["conv_b"]), None,
                        P, mode)
-    out = store(out, storage)
+    out = store(out, final_storage or storage)
     if trace is not None:
         trace["a"] = a
     gn.refresh(f)
@@ -311,7 +348,8 @@ def gn_conv_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float
 
 
 def resblock_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float,
-                  mode: int, storage: str, trace: Optional[Dict] = None, prefix: str = ""):
+                  mode: int, storage: str, trace: Optional[Dict] = None, prefix: str = "",
+                  final_storage: Optional[str] = None):
     """GN -> SiLU -> conv1 -> GN -> SiLU -> conv2 -> + x (or + 1x1 shortcut(x))."""
     x = _a(x)
     W_ = lambda n: _a(wts[prefix + n])
@@ -330,7 +368,7 @@ def resblock_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: floa
     else:
         res = x
     out = store(conv3x3_halo(a2, state.get("a2_stale"), W_("conv2_w"), W_("conv2_b"), res, P,
-                             mode), storage)
+                             mode), final_storage or storage)
     if trace is not None:
         trace[prefix + "a1"], trace[prefix + "h"], trace[prefix + "a2"] = a1, h, a2
     gn1.refresh(f1)
@@ -340,7 +378,8 @@ def resblock_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: floa
 
 
 def attn_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float, heads: int,
-              mode: int, storage: str, trace: Optional[Dict] = None, prefix: str = ""):
+              mode: int, storage: str, trace: Optional[Dict] = None, prefix: str = "",
+              final_storage: Optional[str] = None):
     """GN (no SiLU) -> q, k, v projections -> stale-K/V attention -> out proj + bias -> + x.
 
     x: (C, H, W); tokens are pixels in raster order, so band p's tokens are
@@ -361,7 +400,7 @@ def attn_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float, h
     o = store(attention_stale_kv(q, k, v, state.get("k_stale"), state.get("v_stale"), P,
                                  heads, 1.0 / math.sqrt(d), mode), storage)
     out_tok = linear(o, W_("wo"), W_("bo")) + x.reshape(C, H * Wd).T
-    out = store(out_tok.T.reshape(C, H, Wd), storage)
+    out = store(out_tok.T.reshape(C, H, Wd), final_storage or storage)
     if trace is not None:
         trace[prefix + "a"], trace[prefix + "q"] = a, q
         trace[prefix + "k"], trace[prefix + "v"], trace[prefix + "o"] = k, v, o
@@ -371,7 +410,8 @@ def attn_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float, h
 
 
 def unet_mini_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float,
-                   mode: int, storage: str, trace: Optional[Dict] = None):
+                   mode: int, storage: str, trace: Optional[Dict] = None,
+                   final_storage: Optional[str] = None):
     """conv_in -> ResBlock(320) -> down -> ResBlock(320->640) -> Attn(640, 10 heads)
     -> down -> ResBlock(640->1280) -> Attn(1280, 20 heads)   (reading R6/R7).
 
@@ -395,23 +435,31 @@ def unet_mini_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: flo
     h = attn_step(sub("at2"), h, wts, P, G, eps, w, 10, mode, storage, trace, "at2.")
     h = conv_layer("down2", h, "down2_w", "down2_b", 2)
     h = resblock_step(sub("rb3"), h, wts, P, G, eps, w, mode, storage, trace, "rb3.")
-    h = attn_step(sub("at3"), h, wts, P, G, eps, w, 20, mode, storage, trace, "at3.")
+    h = attn_step(sub("at3"), h, wts, P, G, eps, w, 20, mode, storage, trace, "at3.",
+                  final_storage)
     return h
 
 
 def block_step(kind: str, state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float,
                mode: int, storage: str, heads: int = 0, silu: bool = True,
-               trace: Optional[Dict] = None):
-    """Dispatch one block step by kind; x is (C, H, W) (a leading batch of 1 is dropped)."""
+               trace: Optional[Dict] = None, final_storage: Optional[str] = None):
+    """Dispatch one block step by kind; x is (C, H, W) (a leading batch of 1 is dropped).
+
+    ``final_storage`` (default: ``storage``) is the rounding of the block's
+    output alone; intermediates always use ``storage``.
+    """
     x = _a(x)
     if x.ndim == 4:
         x = x[0]
     if kind == "gn_conv":
-        return gn_conv_step(state, x, wts, P, G, eps, w, silu, mode, storage, trace)
+        return gn_conv_step(state, x, wts, P, G, eps, w, silu, mode, storage, trace,
+                            final_storage)
     if kind == "resblock":
-        return resblock_step(state, x, wts, P, G, eps, w, mode, storage, trace)
+        return resblock_step(state, x, wts, P, G, eps, w, mode, storage, trace,
+                             final_storage=final_storage)
     if kind == "attn":
-        return attn_step(state, x, wts, P, G, eps, w, heads, mode, storage, trace)
+        return attn_step(state, x, wts, P, G, eps, w, heads, mode, storage, trace,
+                         final_storage=final_storage)
     if kind == "unet_mini":
-        return unet_mini_step(state, x, wts, P, G, eps, w, mode, storage, trace)
+        return unet_mini_step(state, x, wts, P, G, eps, w, mode, storage, trace, final_storage)
     raise ValueError(kind)

@@ -1,0 +1,64 @@
+"""Shared helpers of the parity tests: layout marshalling and the comparison bar.
+
+Tolerances (stated once, used by every bf16 parity check): max-abs <= 2e-2 and
+relative L2 <= 5e-3 against the oracle's unrounded output; GroupNorm
+statistics (fp32) within 1e-4 absolute.
+"""
+import numpy as np
+import torch
+
+ATOL = 2e-2
+RL2 = 5e-3
+STATS_ATOL = 1e-4
+
+
+def tdtype(dtype: str):
+    return torch.bfloat16 if dtype == "bf16" else torch.float32
+
+
+def rounded(a: np.ndarray, dtype: str) -> np.ndarray:
+    """Values representable in the storage type (the inputs both sides consume)."""
+    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(tdtype(dtype))
+    return t.to(torch.float64).numpy()
+
+
+def dev_img(a_chw: np.ndarray, dtype: str) -> torch.Tensor:
+    """(C, H, W) host array -> contiguous NHWC device tensor of the storage type."""
+    t = torch.from_numpy(np.ascontiguousarray(a_chw, dtype=np.float32)).permute(1, 2, 0).contiguous()
+    return t.to(tdtype(dtype)).cuda()
+
+
+def host_img(t_hwc: torch.Tensor) -> np.ndarray:
+    return t_hwc.float().cpu().permute(2, 0, 1).contiguous().double().numpy()
+
+
+def dev_mat(a: np.ndarray, dtype: str = "bf16") -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(tdtype(dtype)).cuda()
+
+
+def dev_f32(a) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
+
+
+def host(t: torch.Tensor) -> np.ndarray:
+    return t.float().cpu().double().numpy()
+
+
+def conv_w_dev(w_oihw: np.ndarray, dtype: str) -> torch.Tensor:
+    """(Cout, Cin, 3, 3) -> device [Cout][3][3][Cin]."""
+    t = torch.from_numpy(np.ascontiguousarray(w_oihw, dtype=np.float32)).permute(0, 2, 3, 1).contiguous()
+    return t.to(tdtype(dtype)).cuda()
+
+
+def check(gpu: np.ndarray, ref: np.ndarray, atol=ATOL, rl2=RL2, what=""):
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert gpu.shape == ref.shape, (what, gpu.shape, ref.shape)
+    assert np.isfinite(gpu).all(), f"{what}: non-finite GPU output"
+    diff = np.abs(gpu - ref)
+    maxabs = float(diff.max()) if diff.size else 0.0
+    nref = float(np.linalg.norm(ref))
+    rel = float(np.linalg.norm(gpu - ref) / nref) if nref > 0 else float(np.linalg.norm(gpu - ref))
+    assert maxabs <= atol, f"{what}: max-abs {maxabs:.3e} > {atol:.1e} (rel-L2 {rel:.2e})"
+    assert rel <= rl2, f"{what}: rel-L2 {rel:.3e} > {rl2:.1e} (max-abs {maxabs:.2e})"
+    return maxabs, rel

@@ -1,0 +1,137 @@
+"""C-ABI checks that need no GPU: the library loads, exports every declared
+symbol, and rejects bad arguments on the host before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def B():
+    from displaced_patch_parallelism_b200 import binding
+    if not os.path.exists(binding.LIB_PATH):
+        from displaced_patch_parallelism_b200 import build
+        build.build()
+    binding.lib()
+    return binding
+
+
+def declared_symbols():
+    names = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", h)).read()
+            names += re.findall(r"^DP_API\s+[\w\s\*]+?\b(dp_\w+)\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_block_calls():
+    names = declared_symbols()
+    for n in ("dp_groupnorm_async", "dp_conv3x3_halo", "dp_attn_stale_kv", "dp_refresh_stale",
+              "dp_block_step"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(B):
+    lib = ctypes.CDLL(B.LIB_PATH)
+    missing = [n for n in declared_symbols() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_mode_for_step(B):
+    assert B.dp_mode_for_step(0, 0) == B.NAIVE
+    assert B.dp_mode_for_step(0, 4) == B.SYNC
+    assert B.dp_mode_for_step(3, 4) == B.SYNC
+    assert B.dp_mode_for_step(4, 4) == B.DISPLACED
+    assert B.dp_mode_for_step(1, 0) == B.DISPLACED
+    with pytest.raises(B.DPError):
+        B.dp_mode_for_step(-1, 0)
+
+
+def test_mode_for_step_matches_input_module(B):
+    from displaced_patch_parallelism_b200 import synth
+    for w in range(4):
+        for s in range(8):
+            assert B.dp_mode_for_step(s, w) == synth.mode_for_step(s, w)
+
+
+def test_block_desc_validation(B):
+    d = B.dp_block_desc_init(B.RESBLOCK, 128, 128, 320, 320, 32, 4, 0, B.BF16, 1, 1e-5, 1.0)
+    assert B.dp_block_workspace_size(d) > 4 * 128 * 128 * 320 * 2
+    assert B.dp_block_launch_count(d) == 6
+    assert abs(B.dp_block_flops(d) - 2 * 2 * 128 * 128 * 320 * 9 * 320) < 1
+    d2 = B.dp_block_desc_init(B.RESBLOCK, 64, 64, 320, 640, 32, 4, 0, B.BF16, 1, 1e-5, 1.0)
+    assert B.dp_block_launch_count(d2) == 7
+    da = B.dp_block_desc_init(B.ATTN, 64, 64, 640, 640, 32, 4, 10, B.BF16, 0, 1e-5, 1.0)
+    assert B.dp_block_launch_count(da) == 5
+    bad = [
+        (B.RESBLOCK, 130, 128, 320, 320, 32, 4, 0, B.BF16, B.DP_ERR_UNSUPPORTED),   # H % P
+        (B.RESBLOCK, 128, 128, 320, 320, 33, 4, 0, B.BF16, B.DP_ERR_UNSUPPORTED),   # C % G
+        (B.ATTN, 64, 64, 640, 640, 32, 4, 9, B.BF16, B.DP_ERR_UNSUPPORTED),         # heads*64 != C
+        (B.ATTN, 8, 8, 128, 128, 32, 4, 2, B.BF16, B.DP_ERR_UNSUPPORTED),           # 16 tokens/band
+        (B.RESBLOCK, 64, 64, 64, 64, 32, 4, 0, B.FP32, B.DP_ERR_UNSUPPORTED),       # fp32 resblock
+        (7, 64, 64, 64, 64, 32, 4, 0, B.BF16, B.DP_ERR_INVALID_ARG),                # kind
+        (B.GN_CONV, 0, 64, 64, 64, 32, 4, 0, B.BF16, B.DP_ERR_INVALID_ARG),         # H = 0
+    ]
+    for kind, H, W, C, Co, G, P, heads, dt, code in bad:
+        with pytest.raises(B.DPError) as e:
+            B.dp_block_desc_init(kind, H, W, C, Co, G, P, heads, dt, 1, 1e-5, 1.0)
+        assert e.value.code == code, (kind, H, W, C, G, P, heads)
+
+
+def test_kernel_calls_reject_bad_arguments_on_the_host(B):
+    # null pointers and unsupported shapes return before any CUDA call
+    with pytest.raises(B.DPError) as e:
+        B.dp_conv3x3_halo(None, None, None, None, None, None, 8, 8, 64, 64, 1, 2, B.SYNC, B.BF16, 0)
+    assert e.value.code == B.DP_ERR_INVALID_ARG
+    with pytest.raises(B.DPError) as e:   # Cin not a multiple of 64
+        B.dp_conv3x3_halo(16, 16, 16, None, None, 32, 8, 8, 48, 64, 1, 2, B.SYNC, B.BF16, 0)
+    assert e.value.code == B.DP_ERR_UNSUPPORTED
+    with pytest.raises(B.DPError) as e:   # stride 3
+        B.dp_conv3x3_halo(16, 16, 16, None, None, 32, 8, 8, 64, 64, 3, 2, B.SYNC, B.BF16, 0)
+    assert e.value.code == B.DP_ERR_UNSUPPORTED
+    with pytest.raises(B.DPError) as e:   # displaced without the stale buffer
+        B.dp_conv3x3_halo(16, None, 16, None, None, 32, 8, 8, 64, 64, 1, 2, B.DISPLACED, B.BF16, 0)
+    assert e.value.code == B.DP_ERR_INVALID_ARG
+    with pytest.raises(B.DPError) as e:   # misaligned pointer
+        B.dp_conv3x3_halo(18, 16, 16, None, None, 32, 8, 8, 64, 64, 1, 2, B.SYNC, B.BF16, 0)
+    assert e.value.code == B.DP_ERR_UNSUPPORTED
+    with pytest.raises(B.DPError) as e:   # head_dim 128
+        B.dp_attn_stale_kv(16, 16, 16, 16, 16, 32, 256, 2, 128, 2, 0.1, B.SYNC, 0)
+    assert e.value.code == B.DP_ERR_UNSUPPORTED
+    with pytest.raises(B.DPError) as e:   # band of 96 tokens
+        B.dp_attn_stale_kv(16, 16, 16, 16, 16, 32, 192, 2, 64, 2, 0.1, B.SYNC, 0)
+    assert e.value.code == B.DP_ERR_UNSUPPORTED
+    with pytest.raises(B.DPError) as e:   # o aliases q
+        B.dp_attn_stale_kv(16, 32, 48, 64, 80, 16, 256, 2, 64, 2, 0.1, B.SYNC, 0)
+    assert e.value.code == B.DP_ERR_INVALID_ARG
+    with pytest.raises(B.DPError) as e:   # linear K % 64
+        B.dp_linear(16, 16, None, None, 32, None, None, 10, 64, 48, 64, 0)
+    assert e.value.code == B.DP_ERR_UNSUPPORTED
+    with pytest.raises(B.DPError) as e:   # groupnorm: C % G
+        B.dp_groupnorm_async(16, 32, 16, 16, 8, 8, 30, 32, 2, 1e-5, 1.0, 1, B.SYNC, B.BF16, None, None,
+                             16, 16, 16, 1 << 20, 0)
+    assert e.value.code == B.DP_ERR_UNSUPPORTED
+    with pytest.raises(B.DPError) as e:   # groupnorm: workspace too small
+        B.dp_groupnorm_async(16, 32, 16, 16, 8, 8, 64, 32, 2, 1e-5, 1.0, 1, B.SYNC, B.BF16, None, None,
+                             16, 16, 16, 8, 0)
+    assert e.value.code == B.DP_ERR_INVALID_ARG
+    with pytest.raises(B.DPError) as e:   # groupnorm: displaced without stale statistics
+        B.dp_groupnorm_async(16, 32, 16, 16, 8, 8, 64, 32, 2, 1e-5, 1.0, 1, B.DISPLACED, B.BF16, None,
+                             None, 16, 16, 16, 1 << 20, 0)
+    assert e.value.code == B.DP_ERR_INVALID_ARG
+    with pytest.raises(B.DPError) as e:   # refresh: overlapping buffers
+        B.dp_refresh_stale(1024, 1024 + 256, 256, 8, 2, -1, 0)
+    assert e.value.code == B.DP_ERR_INVALID_ARG
+    with pytest.raises(B.DPError) as e:   # refresh: bad band
+        B.dp_refresh_stale(1024, 1 << 20, 256, 8, 2, 5, 0)
+    assert e.value.code == B.DP_ERR_INVALID_ARG
+    assert "refresh" in B.lib().dp_last_error().decode()
+
+
+def test_groupnorm_workspace_size(B):
+    assert B.dp_groupnorm_workspace_size(128, 128, 320, 32, 4) >= 256 + 4 * 32 * 2 * 8
+    assert B.dp_groupnorm_workspace_size(128, 128, 320, 32, 0) == 0

@@ -1,0 +1,213 @@
+"""Parity of every C-ABI kernel call against the CPU oracle, on seeded inputs.
+
+Sizes span several tiles and ragged tails; every mode (sync, displaced,
+naive) is covered.  Bar: see tests/helpers.py.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from displaced_patch_parallelism_b200 import binding as B
+from oracle import dp_oracle as O
+from tests.helpers import (ATOL, RL2, STATS_ATOL, check, conv_w_dev, dev_f32, dev_img, dev_mat,
+                           host, host_img, rounded)
+
+pytestmark = pytest.mark.gpu
+MODES = [B.SYNC, B.DISPLACED, B.NAIVE]
+
+
+def rng(seed):
+    return np.random.default_rng(seed)
+
+
+# ---------------------------------------------------------------- GroupNorm
+GN_CASES = [
+    # C, H, W, P, G, dtype, silu
+    (64, 32, 32, 2, 32, "fp32", True),
+    (320, 32, 20, 4, 32, "bf16", True),
+    (640, 16, 16, 4, 32, "bf16", False),
+    (96, 24, 9, 8, 32, "bf16", True),
+    (1280, 8, 8, 2, 32, "bf16", True),
+]
+
+
+@pytest.mark.parametrize("case", GN_CASES)
+@pytest.mark.parametrize("mode", MODES)
+def test_groupnorm_parity(case, mode):
+    C, H, W, P, G, dtype, silu = case
+    r = rng(C + H + mode)
+    xs = rounded(r.standard_normal((C, H, W)) * 1.3 + 0.2, dtype)
+    x = rounded(xs + 0.05 * r.standard_normal((C, H, W)) + 0.02, dtype)
+    gamma = 1 + 0.3 * r.standard_normal(C)
+    beta = 0.3 * r.standard_normal(C)
+    sg, sl = O.refresh_stats(O.gn_fresh_local(xs, P, G))
+    sg, sl = sg.astype(np.float32).astype(np.float64), sl.astype(np.float32).astype(np.float64)
+    y_ref, f_ref, used_ref, _ = O.groupnorm_async(x, gamma, beta, P, G, 1e-5, 1.0, silu, mode, sg, sl)
+
+    xd = dev_img(x, dtype)
+    yd = torch.empty_like(xd)
+    fresh = torch.zeros(P * G * 2, device="cuda")
+    used = torch.zeros(P * G * 2, device="cuda")
+    ws = torch.zeros(B.dp_groupnorm_workspace_size(H, W, C, G, P), dtype=torch.uint8, device="cuda")
+    for _ in range(2):  # twice: the workspace must be left ready for reuse
+        B.dp_groupnorm_async(xd, yd, dev_f32(gamma), dev_f32(beta), H, W, C, G, P, 1e-5, 1.0, silu,
+                             mode, B.BF16 if dtype == "bf16" else B.FP32, dev_f32(sg), dev_f32(sl),
+                             fresh, used, ws)
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(host(fresh).reshape(P, G, 2), f_ref, rtol=0, atol=STATS_ATOL)
+    np.testing.assert_allclose(host(used).reshape(P, G, 2), used_ref, rtol=0, atol=STATS_ATOL)
+    if dtype == "fp32":
+        check(host_img(yd), y_ref, atol=1e-4, rl2=1e-5, what="gn fp32")
+    else:
+        check(host_img(yd), y_ref, what="gn bf16")
+    assert B.dp_device_status() == 0
+
+
+def test_groupnorm_full_size_stats():
+    """Statistics at the 1x320x480x480, P = 8 size, displaced mode."""
+    C, H, W, P, G = 320, 480, 480, 8, 32
+    r = rng(5)
+    xs = rounded(r.standard_normal((C, H, W), dtype=np.float32), "bf16")
+    x = rounded(xs + 0.05 * r.standard_normal((C, H, W), dtype=np.float32), "bf16")
+    sg, sl = O.refresh_stats(O.gn_fresh_local(xs, P, G))
+    f_ref = O.gn_fresh_local(x, P, G)
+    used_ref, _ = O.gn_used_stats(f_ref, B.DISPLACED, sg, sl, 1.0)
+    xd = dev_img(x, "bf16")
+    yd = torch.empty_like(xd)
+    fresh = torch.zeros(P * G * 2, device="cuda")
+    used = torch.zeros(P * G * 2, device="cuda")
+    ws = torch.zeros(B.dp_groupnorm_workspace_size(H, W, C, G, P), dtype=torch.uint8, device="cuda")
+    B.dp_groupnorm_async(xd, yd, dev_f32(np.ones(C)), dev_f32(np.zeros(C)), H, W, C, G, P, 1e-5,
+                         1.0, 1, B.DISPLACED, B.BF16, dev_f32(sg), dev_f32(sl), fresh, used, ws)
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(host(fresh).reshape(P, G, 2), f_ref, rtol=0, atol=STATS_ATOL)
+    np.testing.assert_allclose(host(used).reshape(P, G, 2), used_ref, rtol=0, atol=STATS_ATOL)
+    # sampled rows of the output: band edges and interiors
+    rows = [0, 59, 60, 61, 239, 240, 479]
+    y = yd[rows].float().cpu().permute(2, 0, 1).double().numpy()
+    sub = np.stack([x[:, rr, :] for rr in rows], axis=1)
+    ref_rows = np.empty_like(sub)
+    for i, rr in enumerate(rows):
+        u = used_ref[rr // (H // P)]
+        one = O.gn_apply(sub[:, i:i + 1, :], u[None], np.ones(C), np.zeros(C), 1, G, 1e-5, True)
+        ref_rows[:, i:i + 1, :] = one
+    check(y, ref_rows, what="gn full-size rows")
+
+
+# ---------------------------------------------------------------- conv
+CONV_CASES = [
+    # Cin, Cout, H, W, P, stride, dtype, residual
+    (64, 64, 16, 16, 4, 1, "bf16", False),
+    (128, 96, 12, 20, 3, 1, "bf16", True),
+    (64, 160, 32, 40, 4, 1, "bf16", True),
+    (320, 320, 16, 24, 4, 1, "bf16", True),
+    (64, 64, 16, 16, 2, 2, "bf16", False),
+    (128, 64, 24, 36, 3, 2, "bf16", True),
+    (64, 64, 16, 16, 2, 1, "fp32", False),
+    (64, 128, 8, 10, 2, 1, "fp32", True),
+]
+
+
+@pytest.mark.parametrize("case", CONV_CASES)
+@pytest.mark.parametrize("mode", MODES)
+def test_conv3x3_halo_parity(case, mode):
+    Cin, Cout, H, W, P, stride, dtype, use_res = case
+    r = rng(Cin + Cout + H + W + stride + mode)
+    af = rounded(r.standard_normal((Cin, H, W)), dtype)
+    ast = rounded(r.standard_normal((Cin, H, W)), dtype)
+    wt = rounded(r.standard_normal((Cout, Cin, 3, 3)) * math.sqrt(2 / (9 * Cin)), dtype)
+    b = 0.3 * r.standard_normal(Cout)
+    Ho, Wo = (H - 1) // stride + 1, (W - 1) // stride + 1
+    res = rounded(r.standard_normal((Cout, Ho, Wo)), dtype) if use_res else None
+    ref = O.conv3x3_halo(af, ast, wt, b, res, P, mode, stride)
+    out = torch.empty(Ho, Wo, Cout, dtype=torch.bfloat16 if dtype == "bf16" else torch.float32,
+                      device="cuda")
+    B.dp_conv3x3_halo(dev_img(af, dtype), dev_img(ast, dtype), conv_w_dev(wt, dtype), dev_f32(b),
+                      dev_img(res, dtype) if use_res else None, out, H, W, Cin, Cout, stride, P,
+                      mode, B.BF16 if dtype == "bf16" else B.FP32)
+    torch.cuda.synchronize()
+    check(host_img(out), ref, what=f"conv {case} mode {mode}")
+    assert B.dp_device_status() == 0
+
+
+def test_conv_small_parity():
+    for mode in MODES:
+        r = rng(40 + mode)
+        Cin, Cout, H, W, P = 4, 64, 16, 12, 4
+        af = rounded(r.standard_normal((Cin, H, W)), "bf16")
+        ast = rounded(r.standard_normal((Cin, H, W)), "bf16")
+        wt = rounded(r.standard_normal((Cout, Cin, 3, 3)) * math.sqrt(2 / (9 * Cin)), "bf16")
+        b = 0.3 * r.standard_normal(Cout)
+        ref = O.conv3x3_halo(af, ast, wt, b, None, P, mode)
+        out = torch.empty(H, W, Cout, dtype=torch.bfloat16, device="cuda")
+        B.dp_conv3x3_halo_small(dev_img(af, "bf16"), dev_img(ast, "bf16"), conv_w_dev(wt, "bf16"),
+                                dev_f32(b), out, H, W, Cin, Cout, P, mode)
+        torch.cuda.synchronize()
+        check(host_img(out), ref, what=f"small conv mode {mode}")
+
+
+# ---------------------------------------------------------------- linear
+@pytest.mark.parametrize("M,N,K,split,use_res", [(300, 192, 128, 192, True), (256, 384, 128, 128, False),
+                                                 (4096, 1920, 640, 640, False),
+                                                 (1000, 640, 320, 640, True)])
+def test_linear_parity(M, N, K, split, use_res):
+    r = rng(M + N + K)
+    x = rounded(r.standard_normal((M, K)), "bf16")
+    w = rounded(r.standard_normal((N, K)) / math.sqrt(K), "bf16")
+    b = 0.3 * r.standard_normal(N)
+    res = rounded(r.standard_normal((M, N)), "bf16") if use_res else None
+    ref = x @ w.T + b + (res if use_res else 0)
+    outs = [torch.empty(M, split, dtype=torch.bfloat16, device="cuda") for _ in range(N // split)]
+    outs += [None] * (3 - len(outs))
+    B.dp_linear(dev_mat(x), dev_mat(w), dev_f32(b), dev_mat(res) if use_res else None, outs[0],
+                outs[1], outs[2], M, N, K, split)
+    torch.cuda.synchronize()
+    got = np.concatenate([host(o) for o in outs if o is not None], axis=1)
+    check(got, ref, what="linear")
+
+
+# ---------------------------------------------------------------- attention
+@pytest.mark.parametrize("T,heads,P,qscale", [(512, 2, 2, 1.0), (512, 2, 4, 3.0), (1024, 3, 2, 1.0),
+                                              (4096, 10, 4, 1.0)])
+@pytest.mark.parametrize("mode", MODES)
+def test_attention_parity(T, heads, P, qscale, mode):
+    r = rng(T + heads + P + mode)
+    C = heads * 64
+    q = rounded(qscale * r.standard_normal((T, C)), "bf16")
+    kf, vf, ks, vs = (rounded(r.standard_normal((T, C)), "bf16") for _ in range(4))
+    ref = O.attention_stale_kv(q, kf, vf, ks, vs, P, heads, 0.125, mode)
+    o = torch.empty(T, C, dtype=torch.bfloat16, device="cuda")
+    B.dp_attn_stale_kv(dev_mat(q), dev_mat(kf), dev_mat(vf), dev_mat(ks), dev_mat(vs), o, T, heads, 64,
+                       P, 0.125, mode)
+    torch.cuda.synchronize()
+    check(host(o), ref, what=f"attention T={T} P={P} mode={mode}")
+    assert B.dp_device_status() == 0
+
+
+# ---------------------------------------------------------------- refresh
+def test_refresh_is_an_exact_copy():
+    g = torch.Generator(device="cpu").manual_seed(3)
+    H, W, C, P = 64, 48, 320, 4
+    fresh = torch.randint(-2 ** 15, 2 ** 15, (H, W, C), generator=g, dtype=torch.int16).cuda()
+    stale = torch.zeros_like(fresh)
+    B.dp_refresh_stale(fresh, stale, W * C * 2, H, P, 2)
+    torch.cuda.synchronize()
+    hb = H // P
+    assert torch.equal(stale[2 * hb:3 * hb], fresh[2 * hb:3 * hb])
+    assert int(stale[:2 * hb].abs().sum()) == 0 and int(stale[3 * hb:].abs().sum()) == 0
+    B.dp_refresh_stale(fresh, stale, W * C * 2, H, P, -1)
+    torch.cuda.synchronize()
+    assert torch.equal(stale, fresh)
+
+
+def test_refresh_stats():
+    P, G = 4, 32
+    f = torch.randn(P * G * 2, device="cuda")
+    sl = torch.zeros_like(f)
+    sg = torch.zeros(G * 2, device="cuda")
+    B.dp_refresh_stats(f, sl, sg, P, G)
+    torch.cuda.synchronize()
+    assert torch.equal(sl, f)
+    torch.testing.assert_close(sg.view(G, 2), f.view(P, G, 2).double().mean(0).float(), rtol=0, atol=1e-6)

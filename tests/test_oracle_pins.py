@@ -460,3 +460,17 @@ def test_bf16_rounding_matches_library():
                                                           -(1.0 + 2 ** -8), 65504.0, 1e-40]])
     ref = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
     np.testing.assert_array_equal(O.to_bf16(x), ref)
+
+
+@pytest.mark.parametrize("mode", [SYNC, DISPLACED, NAIVE])
+@pytest.mark.parametrize("stride", [1, 2])
+def test_conv_rows_matches_whole_image(mode, stride):
+    """The per-row restatement used at full size agrees with the whole-image one."""
+    r = rng(90 + stride)
+    Cin, Co, H, W, P = 4, 3, 12, 10, 3
+    af, ast = r.standard_normal((Cin, H, W)), r.standard_normal((Cin, H, W))
+    wt, b = r.standard_normal((Co, Cin, 3, 3)), r.standard_normal(Co)
+    full = O.conv3x3_halo(af, ast, wt, b, None, P, mode, stride)
+    rows = list(range(full.shape[1]))
+    np.testing.assert_allclose(O.conv3x3_halo_rows(af, ast, wt, b, P, mode, rows, stride), full,
+                               rtol=0, atol=1e-12)
