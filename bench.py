@@ -295,6 +295,10 @@ def run_ours(args, wl):
 
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_launch + 1)]
               for _ in range(args.steps)]
+    for row in events:          # torch creates the CUDA event on its first record
+        for e in row:
+            e.record()
+    torch.cuda.synchronize()
     sampler = ClockSampler(local)
     if dist:
         dist.barrier()

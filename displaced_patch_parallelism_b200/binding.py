@@ -221,7 +221,10 @@ def dp_block_step_timed(d: BlockDesc, s: BlockState, x, out, weights: Sequence, 
                         stream=None):
     """``events``: torch.cuda.Event objects (timing enabled), at least launches + 1."""
     arr = (ctypes.c_void_p * len(weights))(*[_p(w) for w in weights])
-    ev = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    handles = [e.cuda_event for e in events]
+    if not all(handles):
+        raise ValueError("events must be created before use (record each once first)")
+    ev = (ctypes.c_void_p * len(events))(*handles)
     return _check(lib().dp_block_step_timed(ctypes.byref(d), ctypes.byref(s), _p(x), _p(out), arr,
                                             len(weights), mode, _s(stream), ev, len(events)))
 

@@ -3,6 +3,13 @@
 Tolerances (stated once, used by every bf16 parity check): max-abs <= 2e-2 and
 relative L2 <= 5e-3 against the oracle's unrounded output; GroupNorm
 statistics (fp32) within 1e-4 absolute.
+
+Storing a value y in bf16 alone moves it by up to half an ulp, <= 2^-8 |y|,
+which exceeds 2e-2 once |y| >= 8.  Unit cases whose outputs reach that range
+(random affine parameters, channel-changing shortcuts) therefore use the
+storage-aware bound |gpu - ref| <= 2e-2 + 2^-8 |ref| per element
+(``storage_rel=BF16_HALF_ULP``); the five workloads' own chains keep the
+plain 2e-2 bound.
 """
 import numpy as np
 import torch
@@ -10,6 +17,7 @@ import torch
 ATOL = 2e-2
 RL2 = 5e-3
 STATS_ATOL = 1e-4
+BF16_HALF_ULP = 2.0 ** -8
 
 
 def tdtype(dtype: str):
@@ -50,7 +58,7 @@ def conv_w_dev(w_oihw: np.ndarray, dtype: str) -> torch.Tensor:
     return t.to(tdtype(dtype)).cuda()
 
 
-def check(gpu: np.ndarray, ref: np.ndarray, atol=ATOL, rl2=RL2, what=""):
+def check(gpu: np.ndarray, ref: np.ndarray, atol=ATOL, rl2=RL2, what="", storage_rel=0.0):
     gpu = np.asarray(gpu, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     assert gpu.shape == ref.shape, (what, gpu.shape, ref.shape)
@@ -59,6 +67,11 @@ def check(gpu: np.ndarray, ref: np.ndarray, atol=ATOL, rl2=RL2, what=""):
     maxabs = float(diff.max()) if diff.size else 0.0
     nref = float(np.linalg.norm(ref))
     rel = float(np.linalg.norm(gpu - ref) / nref) if nref > 0 else float(np.linalg.norm(gpu - ref))
-    assert maxabs <= atol, f"{what}: max-abs {maxabs:.3e} > {atol:.1e} (rel-L2 {rel:.2e})"
+    excess = diff - (atol + storage_rel * np.abs(ref))
+    if diff.size and excess.max() > 0:
+        i = np.unravel_index(int(np.argmax(excess)), diff.shape)
+        raise AssertionError(f"{what}: |diff| {diff[i]:.3e} at {i} (ref {ref[i]:.4f}, gpu {gpu[i]:.4f}) "
+                             f"exceeds {atol:.1e} + {storage_rel:.2e}*|ref|; max-abs {maxabs:.3e}, "
+                             f"rel-L2 {rel:.2e}")
     assert rel <= rl2, f"{what}: rel-L2 {rel:.3e} > {rl2:.1e} (max-abs {maxabs:.2e})"
     return maxabs, rel

@@ -14,7 +14,7 @@ from displaced_patch_parallelism_b200 import binding as B
 from displaced_patch_parallelism_b200 import synth
 from displaced_patch_parallelism_b200.weights import block_weights
 from oracle import dp_oracle as O
-from tests.helpers import check, dev_img, host_img
+from tests.helpers import BF16_HALF_ULP, check, dev_img, host_img
 
 pytestmark = pytest.mark.gpu
 KIND = {"gn_conv": B.GN_CONV, "resblock": B.RESBLOCK, "attn": B.ATTN}
@@ -25,7 +25,7 @@ def make_block(wl):
                    B.BF16 if wl.dtype == "bf16" else B.FP32, wl.silu, wl.eps, 1.0)
 
 
-def run_chain(wl, modes, random_affine):
+def run_chain(wl, modes, random_affine, storage_rel=0.0):
     wts = synth.make_weights(wl, random_affine=random_affine)
     tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
     dev_w = block_weights(wl.kind, wts, tdt)
@@ -41,7 +41,7 @@ def run_chain(wl, modes, random_affine):
                            wl.G, wl.eps, 1.0, mode, wl.dtype, heads=wl.heads, silu=wl.silu,
                            final_storage="none")
         torch.cuda.synchronize()
-        check(host_img(out), ref, what=f"{wl.name} step {k} mode {mode}")
+        check(host_img(out), ref, what=f"{wl.name} step {k} mode {mode}", storage_rel=storage_rel)
     assert B.dp_device_status() == 0
 
 
@@ -64,7 +64,7 @@ def test_resblock_zero_warmup():
 def test_resblock_channel_change():
     wl = synth.Workload(name="resblock_320to640x64x64", kind="resblock", C=320, Cout=640, H=64, W=64,
                         P=4)
-    run_chain(wl, [B.SYNC, B.DISPLACED], True)
+    run_chain(wl, [B.SYNC, B.DISPLACED], True, storage_rel=BF16_HALF_ULP)
 
 
 def test_attn_640x64x64():
@@ -75,7 +75,7 @@ def test_attn_640x64x64():
 def test_attn_1280x32x32_zero_warmup():
     wl = synth.Workload(name="attn_1280x32x32", kind="attn", C=1280, H=32, W=32, P=4, heads=20,
                         silu=False)
-    run_chain(wl, [B.NAIVE, B.DISPLACED, B.SYNC], True)
+    run_chain(wl, [B.NAIVE, B.DISPLACED, B.SYNC], True, storage_rel=BF16_HALF_ULP)
 
 
 def test_gn_conv_320x480x480_sampled_rows():
