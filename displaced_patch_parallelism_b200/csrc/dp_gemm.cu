@@ -131,8 +131,36 @@ __global__ void __launch_bounds__(192, 1) igemm_kernel(const __grid_constant__ G
       uint32_t phase = 0;
       uint32_t issued = 0;          // bit s: stage s has a load in flight
       uint32_t issued_par = 0;      // bit s: parity of that load's phase
+      // Per-tile address work is hoisted out of the K loop: the producer is a
+      // single thread and runtime divisions per K block would starve the MMAs.
+      int ry_tab[3 * 16];             // input row of (kh, box i), -1 for zeros
+      uint64_t stale_mask = 0;        // bit kh*16+i: box comes from the stale map
       for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x) {
         const int mt = tile / p.n_tiles, nt = tile - mt * p.n_tiles;
+        int c0 = 0;
+        if (p.a_mode == 1) {
+          const int tr = mt / p.tiles_w, tc = mt - tr * p.tiles_w;
+          const int r0 = tr * p.R;
+          c0 = tc * p.Wt;
+          stale_mask = 0;
+          for (int i = 0; i < p.R; ++i) {
+            const int r = r0 + i;
+            const int band = r / p.hb_out;
+            const int lo = band * p.hb_in, hi = lo + p.hb_in;     // input rows of this band
+            for (int kh = 0; kh < 3; ++kh) {
+              const int rho = p.stride * r + kh - 1;
+              int ry = rho;
+              if (r >= p.Ho) {
+                ry = -1;                                          // ragged tile row: zeros
+              } else if (rho >= 0 && rho < p.H && (rho < lo || rho >= hi)) {
+                if (p.mode == DP_MODE_DISPLACED) stale_mask |= 1ull << (kh * 16 + i);
+                else if (p.mode == DP_MODE_NAIVE) ry = -1;        // invisible band
+              }
+              ry_tab[kh * 16 + i] = ry;
+            }
+          }
+        }
+        int kh = 0, kw = 0, cb = 0;
         for (int kb = 0; kb < p.k_blocks; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status)) goto producer_done;
           mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
@@ -140,10 +168,6 @@ __global__ void __launch_bounds__(192, 1) igemm_kernel(const __grid_constant__ G
           if (p.a_mode == 0) {
             tma_load_2d(a_dst, &p.tmA0, &full[stage], kb * C::BK, mt * 128);
           } else {
-            const int tap = kb / p.kc, cb = kb - tap * p.kc;
-            const int kh = tap / 3, kw = tap - kh * 3;
-            const int tr = mt / p.tiles_w, tc = mt - tr * p.tiles_w;
-            const int r0 = tr * p.R, c0 = tc * p.Wt;
             int kx, cx;
             if (p.stride == 1) {
               kx = cb * C::BK;
@@ -152,18 +176,17 @@ __global__ void __launch_bounds__(192, 1) igemm_kernel(const __grid_constant__ G
               kx = (kw == 1 ? 0 : p.Cin) + cb * C::BK;
               cx = c0 - (kw == 0 ? 1 : 0);
             }
-            for (int i = 0; i < p.R; ++i) {
-              const int r = r0 + i;
-              const int rho = p.stride * r + kh - 1;
-              const CUtensorMap* m = &p.tmA0;
-              int ry = rho;
-              if (r >= p.Ho) {
-                ry = -1;                                   // ragged tile row: zeros
-              } else if (rho >= 0 && rho < p.H && rho / p.hb_in != r / p.hb_out) {
-                if (p.mode == DP_MODE_DISPLACED) m = &p.tmA1;       // stale halo row
-                else if (p.mode == DP_MODE_NAIVE) ry = -1;          // invisible band
+            const int* ryk = ry_tab + kh * 16;
+            const uint32_t sk = static_cast<uint32_t>(stale_mask >> (kh * 16));
+            for (int i = 0; i < p.R; ++i)
+              tma_load_3d(a_dst + i * p.Wt * 128, ((sk >> i) & 1u) ? &p.tmA1 : &p.tmA0,
+                          &full[stage], kx, cx, ryk[i]);
+            if (++cb == p.kc) {
+              cb = 0;
+              if (++kw == 3) {
+                kw = 0;
+                ++kh;
               }
-              tma_load_3d(a_dst + i * p.Wt * 128, m, &full[stage], kx, cx, ry);
             }
           }
           tma_load_2d(sB + stage * C::B_BYTES, &p.tmB, &full[stage], kb * C::BK, nt * BN);
@@ -186,6 +209,8 @@ __global__ void __launch_bounds__(192, 1) igemm_kernel(const __grid_constant__ G
     if (lane == 0) {
       // ------------------------------------------------------------ MMA issuer
       constexpr uint32_t idesc = idesc_dense(128, BN, TF32 ? 2 : 1, 0, 0);
+      const uint64_t a_desc0 = sdesc_sw128(smem_u32(sA), 1024);
+      const uint64_t b_desc0 = sdesc_sw128(smem_u32(sB), 1024);
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
@@ -198,8 +223,8 @@ __global__ void __launch_bounds__(192, 1) igemm_kernel(const __grid_constant__ G
         for (int kb = 0; kb < p.k_blocks; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag, p.status)) goto mma_done;
           tc_fence_after();
-          const uint64_t ad = sdesc_sw128(smem_u32(sA + stage * C::A_BYTES), 1024);
-          const uint64_t bd = sdesc_sw128(smem_u32(sB + stage * C::B_BYTES), 1024);
+          const uint64_t ad = a_desc0 + static_cast<uint64_t>((stage * C::A_BYTES) >> 4);
+          const uint64_t bd = b_desc0 + static_cast<uint64_t>((stage * C::B_BYTES) >> 4);
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             if (TF32)

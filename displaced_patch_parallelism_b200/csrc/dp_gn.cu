@@ -14,9 +14,10 @@
 //     16-byte channel vector of a pixel fixed (block size = a multiple of the
 //     vectors per pixel), so it accumulates per-channel sums in registers and
 //     never has to split a vector across groups (C/G = 10 at C = 320).  The
-//     block folds channels into groups and writes fp64 partials; the last
-//     block to finish (atomic ticket) reduces the partials and computes the
-//     fresh moments and the moments each band uses.
+//     block folds lanes into channels and channels into groups, then adds
+//     its group sums into an fp64 accumulator with atomics; the last block to
+//     finish (atomic ticket) turns the sums into the fresh moments and the
+//     moments each band uses, and clears the accumulator for the next call.
 //  2. gn_apply: y = x * scale_c + shift_c (+ SiLU), cast and stored with
 //     16-byte vectors.  Blocks walk the image in the reverse order of the
 //     stats pass so that the most recently read part of x is still in L2.
@@ -27,7 +28,7 @@
 
 namespace dp {
 
-constexpr int kGnMaxSplits = 64;   // partial sums per band
+constexpr int kGnMaxSplits = 64;   // blocks per band
 
 template <typename T>
 struct Vec;
@@ -77,7 +78,7 @@ struct GnArgs {
 
 template <typename T>
 __global__ void __launch_bounds__(1024) gn_stats_kernel(const T* __restrict__ x, GnArgs a,
-                                                        double* __restrict__ partial,
+                                                        double* __restrict__ acc,
                                                         unsigned* __restrict__ counter,
                                                         const float* __restrict__ stale_global,
                                                         const float* __restrict__ stale_local,
@@ -129,17 +130,26 @@ __global__ void __launch_bounds__(1024) gn_stats_kernel(const T* __restrict__ x,
     ssq[pl * a.C + v * V + j] = sq[j];
   }
   __syncthreads();
+  // lanes -> channels (row 0 of the scratch), then channels -> groups
+  for (int c = threadIdx.x; c < a.C; c += blockDim.x) {
+    float cs = 0.f, cq = 0.f;
+    for (int l = 0; l < a.lanes; ++l) {
+      cs += ssum[l * a.C + c];
+      cq += ssq[l * a.C + c];
+    }
+    ssum[c] = cs;
+    ssq[c] = cq;
+  }
+  __syncthreads();
   const int cg = a.C / a.G;
   for (int g = threadIdx.x; g < a.G; g += blockDim.x) {
     double ds = 0.0, dq = 0.0;
-    for (int l = 0; l < a.lanes; ++l)
-      for (int c = g * cg; c < (g + 1) * cg; ++c) {
-        ds += ssum[l * a.C + c];
-        dq += ssq[l * a.C + c];
-      }
-    double* dst = partial + ((static_cast<size_t>(p) * a.S + s) * a.G + g) * 2;
-    dst[0] = ds;
-    dst[1] = dq;
+    for (int c = g * cg; c < (g + 1) * cg; ++c) {
+      ds += ssum[c];
+      dq += ssq[c];
+    }
+    atomicAdd(acc + (p * a.G + g) * 2, ds);
+    atomicAdd(acc + (p * a.G + g) * 2 + 1, dq);
   }
   __threadfence();
   __syncthreads();
@@ -151,18 +161,11 @@ __global__ void __launch_bounds__(1024) gn_stats_kernel(const T* __restrict__ x,
   // Last block: fresh moments, then the moments every band normalises with.
   double* f = reinterpret_cast<double*>(gn_smem);   // [P][G][2]
   const double n = static_cast<double>(a.HWp) * cg;
-  for (int i = threadIdx.x; i < a.P * a.G; i += blockDim.x) {
-    const int pp = i / a.G, g = i % a.G;
-    double ds = 0.0, dq = 0.0;
-    for (int k = 0; k < a.S; ++k) {
-      const double* src = partial + ((static_cast<size_t>(pp) * a.S + k) * a.G + g) * 2;
-      ds += __ldcg(src);
-      dq += __ldcg(src + 1);
-    }
-    f[2 * i] = ds / n;
-    f[2 * i + 1] = dq / n;
-    fresh_local[2 * i] = static_cast<float>(ds / n);
-    fresh_local[2 * i + 1] = static_cast<float>(dq / n);
+  for (int i = threadIdx.x; i < a.P * a.G * 2; i += blockDim.x) {
+    const double m = __ldcg(acc + i) / n;
+    acc[i] = 0.0;                                    // ready for the next call
+    f[i] = m;
+    fresh_local[i] = static_cast<float>(m);
   }
   __syncthreads();
   for (int i = threadIdx.x; i < a.P * a.G; i += blockDim.x) {
@@ -299,7 +302,7 @@ static int gn_validate(const void* x, const void* y, int H, int W, int C, int G,
 }
 
 size_t gn_workspace_bytes(int P, int G) {
-  return 256 + static_cast<size_t>(P) * kGnMaxSplits * G * 2 * sizeof(double);
+  return 256 + static_cast<size_t>(P) * G * 2 * sizeof(double);
 }
 
 // Internal entry shared by the ABI call and the block step.
@@ -314,7 +317,7 @@ int gn_launch(const void* x, void* y, const float* gamma, const float* beta, int
   a.silu = silu;
   a.mode = mode;
   unsigned* counter = static_cast<unsigned*>(workspace);
-  double* partial = reinterpret_cast<double*>(static_cast<char*>(workspace) + 256);
+  double* acc = reinterpret_cast<double*>(static_cast<char*>(workspace) + 256);
   const int threads = a.vpp * a.lanes;
   const int blocks = a.P * a.S;
   size_t smem_stats = static_cast<size_t>(a.lanes) * C * 2 * sizeof(float);
@@ -341,7 +344,7 @@ int gn_launch(const void* x, void* y, const float* gamma, const float* beta, int
   if (dtype == DP_BF16) {
     mark_launch(stream);
     gn_stats_kernel<__nv_bfloat16><<<blocks, threads, smem_stats, stream>>>(
-        static_cast<const __nv_bfloat16*>(x), a, partial, counter, stale_global, stale_local,
+        static_cast<const __nv_bfloat16*>(x), a, acc, counter, stale_global, stale_local,
         fresh_local, fresh_global, used);
     mark_launch(stream);
     gn_apply_kernel<__nv_bfloat16><<<blocks, threads, smem_apply, stream>>>(
@@ -350,7 +353,7 @@ int gn_launch(const void* x, void* y, const float* gamma, const float* beta, int
   } else {
     mark_launch(stream);
     gn_stats_kernel<float><<<blocks, threads, smem_stats, stream>>>(
-        static_cast<const float*>(x), a, partial, counter, stale_global, stale_local, fresh_local,
+        static_cast<const float*>(x), a, acc, counter, stale_global, stale_local, fresh_local,
         fresh_global, used);
     mark_launch(stream);
     gn_apply_kernel<float><<<blocks, threads, smem_apply, stream>>>(
