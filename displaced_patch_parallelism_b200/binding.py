@@ -52,6 +52,8 @@ _SIGS = {
     "dp_groupnorm_workspace_size": ([_I, _I, _I, _I, _I], _SZ),
     "dp_groupnorm_async": ([_V, _V, _V, _V, _I, _I, _I, _I, _I, _F, _F, _I, _I, _I, _V, _V, _V, _V,
                             _V, _SZ, _V], _I),
+    "dp_groupnorm_async_noalloc": ([_V, _V, _V, _V, _I, _I, _I, _I, _I, _F, _F, _I, _I, _I, _V, _V,
+                                    _V, _V, _V], _I),
     "dp_conv3x3_halo": ([_V, _V, _V, _V, _V, _V, _I, _I, _I, _I, _I, _I, _I, _I, _V], _I),
     "dp_conv3x3_halo_small": ([_V, _V, _V, _V, _V, _I, _I, _I, _I, _I, _I, _V], _I),
     "dp_linear": ([_V, _V, _V, _V, _V, _V, _V, _I, _I, _I, _I, _V], _I),
@@ -144,6 +146,13 @@ def dp_groupnorm_async(x, y, gamma, beta, H, W, C, G, P, eps, w, silu, mode, dty
         _p(x), _p(y), _p(gamma), _p(beta), H, W, C, G, P, eps, w, int(silu), mode, dtype,
         _p(stale_global), _p(stale_local), _p(fresh_local), _p(used_stats), _p(workspace),
         workspace_bytes, _s(stream)))
+
+
+def dp_groupnorm_async_noalloc(x, y, gamma, beta, H, W, C, G, P, eps, w, silu, mode, dtype,
+                               stale_global, stale_local, fresh_local, used_stats, stream=None):
+    return _check(lib().dp_groupnorm_async_noalloc(
+        _p(x), _p(y), _p(gamma), _p(beta), H, W, C, G, P, eps, w, int(silu), mode, dtype,
+        _p(stale_global), _p(stale_local), _p(fresh_local), _p(used_stats), _s(stream)))
 
 
 def dp_conv3x3_halo(a_fresh, a_stale, weight, bias, residual, out, H, W, Cin, Cout, stride, P,

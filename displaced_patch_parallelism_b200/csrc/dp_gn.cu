@@ -23,6 +23,8 @@
 //     stats pass so that the most recently read part of x is still in L2.
 #include <math.h>
 
+#include <mutex>
+
 #include "dp_common.cuh"
 #include "dp_internal.h"
 
@@ -362,6 +364,34 @@ int gn_launch(const void* x, void* y, const float* gamma, const float* beta, int
   return cuda_check(cudaGetLastError(), "groupnorm launch");
 }
 
+// ---------------------------------------------------------------------------
+// Scratch for callers that cannot allocate device memory.  It is a fixed
+// file-scope array that every GPU loading this library holds until the
+// process exits.  Host code must not hand the array's name to a kernel: on
+// the host that name is only a stand-in, so its device address is looked up
+// once per device with cudaGetSymbolAddress and that address is passed on.
+constexpr size_t kGnStaticScratchBytes = 32 * 1024;
+static __device__ __align__(256) unsigned char g_gn_static_scratch[kGnStaticScratchBytes];
+
+static int gn_static_scratch(void** out) {
+  static void* ptrs[64] = {nullptr};
+  static std::mutex mu;
+  int dev = 0;
+  int rc = cuda_check(cudaGetDevice(&dev), "noalloc groupnorm: current device");
+  if (rc) return rc;
+  if (dev < 0 || dev >= 64) return set_error(DP_ERR_UNSUPPORTED, "noalloc groupnorm: device %d", dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    rc = cuda_check(cudaGetSymbolAddress(&p, g_gn_static_scratch),
+                    "noalloc groupnorm: scratch address");
+    if (rc) return rc;
+    ptrs[dev] = p;
+  }
+  *out = ptrs[dev];
+  return DP_OK;
+}
+
 }  // namespace dp
 
 extern "C" {
@@ -392,6 +422,36 @@ int dp_groupnorm_async(const void* x, void* y, const float* gamma, const float* 
   return dp::gn_launch(x, y, gamma, beta, H, W, C, G, P, eps, w, silu, mode, dtype, stale_global,
                        stale_local, fresh_local, nullptr, used_stats, workspace,
                        static_cast<cudaStream_t>(stream));
+}
+
+int dp_groupnorm_async_noalloc(const void* x, void* y, const float* gamma, const float* beta,
+                               int H, int W, int C, int G, int P, float eps, float w, int silu,
+                               int mode, int dtype, const float* stale_global,
+                               const float* stale_local, float* fresh_local, float* used_stats,
+                               void* stream) {
+  int rc = dp::gn_validate(x, y, H, W, C, G, P, dtype, mode);
+  if (rc) return rc;
+  if (!gamma || !beta || !fresh_local || !used_stats)
+    return dp::set_error(DP_ERR_INVALID_ARG, "noalloc groupnorm: null gamma/beta/fresh_local/used");
+  if (mode == DP_MODE_DISPLACED && (!stale_global || !stale_local))
+    return dp::set_error(DP_ERR_INVALID_ARG, "noalloc groupnorm: displaced mode needs stale statistics");
+  if (!(eps > 0.f)) return dp::set_error(DP_ERR_INVALID_ARG, "noalloc groupnorm: eps must be > 0");
+  const size_t need = dp::gn_workspace_bytes(P, G);
+  if (need > dp::kGnStaticScratchBytes)
+    return dp::set_error(DP_ERR_UNSUPPORTED,
+                         "noalloc groupnorm: P=%d, G=%d needs %zu bytes of scratch; the static "
+                         "scratch holds %zu",
+                         P, G, need, dp::kGnStaticScratchBytes);
+  void* scratch = nullptr;
+  rc = dp::gn_static_scratch(&scratch);
+  if (rc) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // The completion ticket and the fp64 accumulator must start at zero; a call
+  // that did not complete could have left them elsewhere.
+  rc = dp::cuda_check(cudaMemsetAsync(scratch, 0, need, s), "noalloc groupnorm: clear scratch");
+  if (rc) return rc;
+  return dp::gn_launch(x, y, gamma, beta, H, W, C, G, P, eps, w, silu, mode, dtype, stale_global,
+                       stale_local, fresh_local, nullptr, used_stats, scratch, s);
 }
 
 }  // extern "C"

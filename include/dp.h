@@ -130,6 +130,36 @@ DP_API int dp_groupnorm_async(const void* x, void* y, const float* gamma, const 
                        void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * dp_groupnorm_async for callers that cannot allocate device memory.  The
+ * paper has no counterpart of this call; it exists for integration only.
+ *
+ * Some callers have no way to obtain a workspace: code that runs where
+ * cudaMalloc is off limits (it can synchronise the device, which a latency-
+ * critical or real-time loop cannot afford), hosts with a fixed device-memory
+ * budget granted up front, and plain C callers without a caching allocator.
+ * This entry point takes the same arguments as dp_groupnorm_async minus the
+ * workspace and uses a fixed scratch array inside the library instead.
+ *
+ *  - Limit: the scratch holds 32 KiB, enough for P * G up to 2032 (bands x
+ *    groups); larger requests return DP_ERR_UNSUPPORTED with a message.
+ *  - Every GPU that loads the library holds those 32 KiB until the process
+ *    exits.
+ *  - The first call on a device looks the array's device address up
+ *    (cudaGetSymbolAddress); make that first call before any stream capture.
+ *  - Each call clears the part of the scratch it uses (a cudaMemsetAsync of
+ *    256 + 16 * P * G bytes on `stream`) before its kernels; nothing is
+ *    allocated.
+ *  - All calls share the one array and it keeps the last call's contents:
+ *    calls whose kernels overlap on the GPU (different streams, no ordering)
+ *    race on it and give wrong results.  Order them on one stream.
+ * ---------------------------------------------------------------------- */
+DP_API int dp_groupnorm_async_noalloc(const void* x, void* y, const float* gamma,
+                                      const float* beta, int H, int W, int C, int G, int P,
+                                      float eps, float w, int silu, int mode, int dtype,
+                                      const float* stale_global, const float* stale_local,
+                                      float* fresh_local, float* used_stats, void* stream);
+
+/* ------------------------------------------------------------------------
  * 3x3 convolution, padding 1, stride 1 or 2, whose halo rows come from the
  * stale buffer (study.space summary, Method: patches reuse the previous
  * step's activations to keep their interaction).
