@@ -126,44 +126,49 @@ def dist_env():
 
 
 def block_kind(B, wl):
-    return {"gn_conv": B.GN_CONV, "resblock": B.RESBLOCK, "attn": B.ATTN}[wl.kind]
+    return {"gn_conv": B.GN_CONV, "resblock": B.RESBLOCK, "attn": B.ATTN,
+            "unet_mini": B.UNET_MINI}[wl.kind]
+
+
+def launch_work(kind, H, W, C, Cout, e=2):
+    """(role, algorithmic flops, algorithmic bytes) of every launch of one block
+    step, in dp_block_launch_count order."""
+    hw = H * W
+    conv = lambda h, w, ci, co, s=1: ("conv", 2.0 * (h // s) * (w // s) * co * 9 * ci,
+                                      (h * w * ci * 2 + (h // s) * (w // s) * co) * e)
+    gn = lambda h, w, c: [("gn_stats", 0.0, h * w * c * e), ("gn_apply", 0.0, 2 * h * w * c * e)]
+    if kind == "gn_conv":
+        return gn(H, W, C) + [conv(H, W, C, Cout)]
+    if kind == "resblock":
+        out = gn(H, W, C) + [conv(H, W, C, Cout)] + gn(H, W, Cout)
+        if C != Cout:
+            out.append(("linear", 2.0 * hw * Cout * C, hw * (C + Cout) * e))
+        return out + [conv(H, W, Cout, Cout)]
+    if kind == "attn":
+        return gn(H, W, C) + [("linear", 2.0 * hw * 3 * C * C, hw * 4 * C * e),
+                              ("attn", 4.0 * hw * hw * C, hw * 4 * C * e),
+                              ("linear", 2.0 * hw * C * C, hw * 3 * C * e)]
+    # unet_mini
+    out = [("copy", 0.0, 2 * hw * C * e), ("conv_small", 2.0 * hw * 320 * 9 * C, hw * (C + 320) * e)]
+    out += launch_work("resblock", H, W, 320, 320, e)
+    out.append(conv(H, W, 320, 320, 2))
+    out += launch_work("resblock", H // 2, W // 2, 320, 640, e)
+    out += launch_work("attn", H // 2, W // 2, 640, 640, e)
+    out.append(conv(H // 2, W // 2, 640, 640, 2))
+    out += launch_work("resblock", H // 4, W // 4, 640, 1280, e)
+    out += launch_work("attn", H // 4, W // 4, 1280, 1280, e)
+    return out
 
 
 def launch_roles(wl):
     """Kernel role of each launch of one block step (dp_block_launch_count order)."""
-    if wl.kind == "gn_conv":
-        return ["gn_stats", "gn_apply", "conv"]
-    if wl.kind == "resblock":
-        r = ["gn_stats", "gn_apply", "conv", "gn_stats", "gn_apply"]
-        return r + (["linear", "conv"] if wl.cout != wl.C else ["conv"])
-    return ["gn_stats", "gn_apply", "linear", "attn", "linear"]
+    return [r for r, _, _ in launch_work(wl.kind, wl.H, wl.W, wl.C, wl.cout)]
 
 
 def algorithmic_work(wl):
     """Per-launch algorithmic work of every launch: (flops, bytes)."""
     e = 2 if wl.dtype == "bf16" else 4
-    hw = wl.H * wl.W
-    out = []
-    if wl.kind in ("gn_conv", "resblock"):
-        chans = [wl.C, wl.cout]
-        convs = [(wl.C, wl.cout), (wl.cout, wl.cout)]
-        gi = ci = 0
-        for role in launch_roles(wl):
-            if role == "gn_stats":
-                out.append((0.0, hw * chans[gi] * e))
-            elif role == "gn_apply":
-                out.append((0.0, 2 * hw * chans[gi] * e))
-                gi += 1
-            elif role == "conv":
-                cin, co = convs[ci]
-                out.append((2.0 * hw * co * 9 * cin, hw * (cin * 2 + co) * e))
-                ci += 1
-            else:
-                out.append((2.0 * hw * wl.cout * wl.C, hw * (wl.C + wl.cout) * e))
-        return out
-    C, T = wl.C, hw
-    return [(0.0, T * C * e), (0.0, 2 * T * C * e), (2.0 * T * 3 * C * C, T * 4 * C * e),
-            (4.0 * T * T * C, T * 4 * C * e * 1.0), (2.0 * T * C * C, T * 3 * C * e)]
+    return [(f, b) for _, f, b in launch_work(wl.kind, wl.H, wl.W, wl.C, wl.cout, e)]
 
 
 def cpu_baseline_ours(wl, seconds):
@@ -188,13 +193,7 @@ def cpu_baseline_ours(wl, seconds):
 
 
 def wl_flops(wl):
-    hw = wl.H * wl.W
-    if wl.kind == "gn_conv":
-        return 2.0 * hw * wl.cout * 9 * wl.C
-    if wl.kind == "resblock":
-        f = 2.0 * hw * wl.cout * 9 * wl.C + 2.0 * hw * wl.cout * 9 * wl.cout
-        return f + (2.0 * hw * wl.cout * wl.C if wl.cout != wl.C else 0.0)
-    return 2.0 * hw * 3 * wl.C * wl.C + 4.0 * hw * hw * wl.C + 2.0 * hw * wl.C * wl.C
+    return sum(f for _, f, _ in launch_work(wl.kind, wl.H, wl.W, wl.C, wl.cout))
 
 
 def run_reference(args, wl):
@@ -281,7 +280,8 @@ def run_ours(args, wl):
     pool = 4
     host_x = [synth.nchw_to_nhwc(xs.x(k)).to(tdt).pin_memory() for k in range(pool)]
     dev_x = [h.to(dev) for h in host_x]
-    out = torch.empty(wl.H, wl.W, wl.cout, dtype=tdt, device=dev)
+    Ho, Wo = (wl.H // 4, wl.W // 4) if wl.kind == "unet_mini" else (wl.H, wl.W)
+    out = torch.empty(Ho, Wo, wl.cout, dtype=tdt, device=dev)
     host_out = torch.empty(out.shape, dtype=tdt).pin_memory()
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     n_launch = blk.launches
@@ -371,7 +371,8 @@ def run_ours(args, wl):
     dominant = max(role_ms, key=lambda r: role_ms[r])
     dk = kernels[dominant]
     src = {"conv": ["dp_gemm.cu"], "linear": ["dp_gemm.cu"], "attn": ["dp_attn.cu"],
-           "gn_stats": ["dp_gn.cu"], "gn_apply": ["dp_gn.cu"]}[dominant]
+           "gn_stats": ["dp_gn.cu"], "gn_apply": ["dp_gn.cu"], "copy": ["dp_refresh.cu"],
+           "conv_small": ["dp_conv_small.cu"]}[dominant]
     traffic = load_traffic(f"{dominant}:{wl.name}", kernel_source_hash(src))
     if dk["tflops"]:
         roof = {"bound": "tensor", "achieved": dk["tflops"], "peak": peaks["bf16_tflops"],

@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(PKG_DIR, "libdp.so")
 DP_OK, DP_ERR_INVALID_ARG, DP_ERR_UNSUPPORTED, DP_ERR_STATE, DP_ERR_CUDA, DP_ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
 SYNC, DISPLACED, NAIVE = 0, 1, 2
 BF16, FP32 = 0, 1
-GN_CONV, RESBLOCK, ATTN = 0, 1, 2
+GN_CONV, RESBLOCK, ATTN, UNET_MINI = 0, 1, 2, 3
 
 ERR_NAMES = {DP_ERR_INVALID_ARG: "DP_ERR_INVALID_ARG", DP_ERR_UNSUPPORTED: "DP_ERR_UNSUPPORTED",
              DP_ERR_STATE: "DP_ERR_STATE", DP_ERR_CUDA: "DP_ERR_CUDA",
@@ -67,6 +67,7 @@ _SIGS = {
                        ctypes.POINTER(_V), _I, _I, _V], _I),
     "dp_block_flops": ([ctypes.POINTER(BlockDesc)], ctypes.c_double),
     "dp_block_launch_count": ([ctypes.POINTER(BlockDesc)], _I),
+    "dp_block_weight_count": ([ctypes.POINTER(BlockDesc)], _I),
     "dp_block_step_timed": ([ctypes.POINTER(BlockDesc), ctypes.POINTER(BlockState), _V, _V,
                              ctypes.POINTER(_V), _I, _I, _V, ctypes.POINTER(_V), _I], _I),
 }
@@ -236,6 +237,13 @@ def dp_block_step_timed(d: BlockDesc, s: BlockState, x, out, weights: Sequence, 
     ev = (ctypes.c_void_p * len(events))(*handles)
     return _check(lib().dp_block_step_timed(ctypes.byref(d), ctypes.byref(s), _p(x), _p(out), arr,
                                             len(weights), mode, _s(stream), ev, len(events)))
+
+
+def dp_block_weight_count(d: BlockDesc) -> int:
+    n = lib().dp_block_weight_count(ctypes.byref(d))
+    if n < 0:
+        _check(n)
+    return n
 
 
 def dp_block_flops(d: BlockDesc) -> float:

@@ -288,6 +288,7 @@ __global__ void __launch_bounds__(192, 2) attn_kernel(const __grid_constant__ At
 
   tc_fence_before();
   __syncthreads();
+  __syncwarp();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 256);

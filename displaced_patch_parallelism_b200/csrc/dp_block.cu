@@ -6,15 +6,25 @@
 // summary, Method; gist.science PipeFusion explainer, Memory Efficiency, on
 // DistriFusion's full-spatial K/V buffers).  Each of these lives in a
 // ping-pong pair inside the caller's workspace: a step writes the fresh half
-// (GroupNorm output, fused q/k/v projection output, fresh statistics) and
-// reads the stale half; the refresh that replaces the paper's AllGather is a
-// flip of `cur`, so no byte moves.
+// (GroupNorm output, fused q/k/v projection output, fresh statistics, or the
+// output of the layer feeding a conv) and reads the stale half; the refresh
+// that replaces the paper's AllGather is a flip of `cur`, so no byte moves.
+//
+// Kinds: GN_CONV, RESBLOCK, ATTN, and UNET_MINI, a chain of the others with
+// two stride-2 downsampling convs (conv_in -> ResBlock(320) -> down ->
+// ResBlock(320->640) -> Attn(640) -> down -> ResBlock(640->1280) ->
+// Attn(1280)).  Composite kinds run their sub-blocks with the parent's
+// ping-pong parity.
 #include <cstring>
 
 #include "dp_common.cuh"
 #include "dp_internal.h"
 
 namespace dp {
+
+int conv3x3_small_launch(const void* af, const void* as, const void* w, const float* bias,
+                         void* out, int H, int W, int Cin, int Cout, int P, int mode,
+                         cudaStream_t stream);
 
 namespace {
 
@@ -31,12 +41,45 @@ struct GnSlots {
   size_t local[2], global[2], used, ws;
 };
 
+// Mini U-Net level widths.
+constexpr int kU1 = 320, kU2 = 640, kU3 = 1280;
+
 struct Layout {
   GnSlots gn1, gn2;
   size_t a1[2], a2[2], h, sc;        // conv inputs (pairs), conv1 output, shortcut output
   size_t act, q, k[2], v[2], o;      // attention buffers
+  // UNET_MINI: sub-block workspaces and the buffers between them
+  size_t xin[2], h0, rb1, d1[2], h1, rb2, h2, at2, d2[2], h3, rb3, h4, at3;
   size_t total;
 };
+
+dp_block_desc sub_desc(const dp_block_desc* d, int kind, int H, int W, int C, int Cout,
+                       int heads, int silu) {
+  dp_block_desc s = *d;
+  s.kind = kind;
+  s.H = H;
+  s.W = W;
+  s.C = C;
+  s.Cout = Cout;
+  s.heads = heads;
+  s.silu = silu;
+  return s;
+}
+
+struct MiniDescs {
+  dp_block_desc rb1, rb2, at2, rb3, at3;
+};
+
+MiniDescs mini_descs(const dp_block_desc* d) {
+  MiniDescs m;
+  const int H = d->H, W = d->W;
+  m.rb1 = sub_desc(d, DP_BLOCK_RESBLOCK, H, W, kU1, kU1, 0, 1);
+  m.rb2 = sub_desc(d, DP_BLOCK_RESBLOCK, H / 2, W / 2, kU1, kU2, 0, 1);
+  m.at2 = sub_desc(d, DP_BLOCK_ATTN, H / 2, W / 2, kU2, kU2, kU2 / 64, 0);
+  m.rb3 = sub_desc(d, DP_BLOCK_RESBLOCK, H / 4, W / 4, kU2, kU3, 0, 1);
+  m.at3 = sub_desc(d, DP_BLOCK_ATTN, H / 4, W / 4, kU3, kU3, kU3 / 64, 0);
+  return m;
+}
 
 GnSlots gn_slots(Bump& b, int P, int G) {
   GnSlots s;
@@ -49,27 +92,47 @@ GnSlots gn_slots(Bump& b, int P, int G) {
   return s;
 }
 
+Layout layout_of(const dp_block_desc* d);
+
 Layout layout_of(const dp_block_desc* d) {
   Layout L;
   memset(&L, 0, sizeof(L));
   Bump b;
   const size_t e = d->dtype == DP_FP32 ? 4 : 2;
   const size_t hw = static_cast<size_t>(d->H) * d->W;
-  L.gn1 = gn_slots(b, d->P, d->G);
   if (d->kind == DP_BLOCK_GN_CONV) {
+    L.gn1 = gn_slots(b, d->P, d->G);
     for (int i = 0; i < 2; ++i) L.a1[i] = b.take(hw * d->C * e);
   } else if (d->kind == DP_BLOCK_RESBLOCK) {
+    L.gn1 = gn_slots(b, d->P, d->G);
     L.gn2 = gn_slots(b, d->P, d->G);
     for (int i = 0; i < 2; ++i) L.a1[i] = b.take(hw * d->C * e);
     for (int i = 0; i < 2; ++i) L.a2[i] = b.take(hw * d->Cout * e);
     L.h = b.take(hw * d->Cout * e);
     if (d->C != d->Cout) L.sc = b.take(hw * d->Cout * e);
-  } else {
+  } else if (d->kind == DP_BLOCK_ATTN) {
+    L.gn1 = gn_slots(b, d->P, d->G);
     L.act = b.take(hw * d->C * e);
     L.q = b.take(hw * d->C * e);
     for (int i = 0; i < 2; ++i) L.k[i] = b.take(hw * d->C * e);
     for (int i = 0; i < 2; ++i) L.v[i] = b.take(hw * d->C * e);
     L.o = b.take(hw * d->C * e);
+  } else {
+    const MiniDescs m = mini_descs(d);
+    const size_t hw2 = hw / 4, hw3 = hw / 16;
+    for (int i = 0; i < 2; ++i) L.xin[i] = b.take(hw * d->C * 2);
+    L.h0 = b.take(hw * kU1 * 2);
+    L.rb1 = b.take(layout_of(&m.rb1).total);
+    for (int i = 0; i < 2; ++i) L.d1[i] = b.take(hw * kU1 * 2);
+    L.h1 = b.take(hw2 * kU1 * 2);
+    L.rb2 = b.take(layout_of(&m.rb2).total);
+    L.h2 = b.take(hw2 * kU2 * 2);
+    L.at2 = b.take(layout_of(&m.at2).total);
+    for (int i = 0; i < 2; ++i) L.d2[i] = b.take(hw2 * kU2 * 2);
+    L.h3 = b.take(hw3 * kU2 * 2);
+    L.rb3 = b.take(layout_of(&m.rb3).total);
+    L.h4 = b.take(hw3 * kU3 * 2);
+    L.at3 = b.take(layout_of(&m.at3).total);
   }
   L.total = b.off;
   return L;
@@ -77,7 +140,7 @@ Layout layout_of(const dp_block_desc* d) {
 
 int desc_check(const dp_block_desc* d) {
   if (!d) return set_error(DP_ERR_INVALID_ARG, "block: null descriptor");
-  if (d->kind < DP_BLOCK_GN_CONV || d->kind > DP_BLOCK_ATTN)
+  if (d->kind < DP_BLOCK_GN_CONV || d->kind > DP_BLOCK_UNET_MINI)
     return set_error(DP_ERR_INVALID_ARG, "block: bad kind %d", d->kind);
   if (d->H <= 0 || d->W <= 0 || d->C <= 0 || d->Cout <= 0 || d->G <= 0 || d->P <= 0)
     return set_error(DP_ERR_INVALID_ARG, "block: non-positive size");
@@ -85,7 +148,21 @@ int desc_check(const dp_block_desc* d) {
     return set_error(DP_ERR_INVALID_ARG, "block: bad dtype");
   if (d->dtype == DP_FP32 && d->kind != DP_BLOCK_GN_CONV)
     return set_error(DP_ERR_UNSUPPORTED, "block: fp32 storage is only built for GN_CONV");
+  if (!(d->eps > 0.f)) return set_error(DP_ERR_INVALID_ARG, "block: eps must be > 0");
   if (d->H % d->P) return set_error(DP_ERR_UNSUPPORTED, "block: H %% P != 0");
+  if (d->kind == DP_BLOCK_UNET_MINI) {
+    if (d->C > 16 || d->C % 2)
+      return set_error(DP_ERR_UNSUPPORTED, "block: mini U-Net latent needs an even C <= 16");
+    if (d->H % (4 * d->P) || d->W % 4)
+      return set_error(DP_ERR_UNSUPPORTED, "block: mini U-Net needs H %% 4P == 0 and W %% 4 == 0");
+    const MiniDescs m = mini_descs(d);
+    const dp_block_desc* subs[5] = {&m.rb1, &m.rb2, &m.at2, &m.rb3, &m.at3};
+    for (const dp_block_desc* s : subs) {
+      int rc = desc_check(s);
+      if (rc) return rc;
+    }
+    return DP_OK;
+  }
   if (d->C % d->G || d->Cout % d->G) return set_error(DP_ERR_UNSUPPORTED, "block: channels %% G != 0");
   if (d->kind == DP_BLOCK_ATTN) {
     if (d->Cout != d->C) return set_error(DP_ERR_INVALID_ARG, "block: attention keeps C");
@@ -94,13 +171,174 @@ int desc_check(const dp_block_desc* d) {
     const int T = d->H * d->W;
     if ((T / d->P) % 128) return set_error(DP_ERR_UNSUPPORTED, "block: tokens per band %% 128 != 0");
   }
-  if (!(d->eps > 0.f)) return set_error(DP_ERR_INVALID_ARG, "block: eps must be > 0");
   return DP_OK;
+}
+
+int launch_count(const dp_block_desc* d) {
+  if (d->kind == DP_BLOCK_GN_CONV) return 3;
+  if (d->kind == DP_BLOCK_RESBLOCK) return d->C != d->Cout ? 7 : 6;
+  if (d->kind == DP_BLOCK_ATTN) return 5;
+  const MiniDescs m = mini_descs(d);
+  // input copy + conv_in + rb1 + down1 + rb2 + at2 + down2 + rb3 + at3
+  return 2 + launch_count(&m.rb1) + 1 + launch_count(&m.rb2) + launch_count(&m.at2) + 1 +
+         launch_count(&m.rb3) + launch_count(&m.at3);
+}
+
+int weight_count(const dp_block_desc* d) {
+  if (d->kind == DP_BLOCK_GN_CONV) return 4;
+  if (d->kind == DP_BLOCK_RESBLOCK) return d->C != d->Cout ? 10 : 8;
+  if (d->kind == DP_BLOCK_ATTN) return 6;
+  const MiniDescs m = mini_descs(d);
+  return 2 + weight_count(&m.rb1) + 2 + weight_count(&m.rb2) + weight_count(&m.at2) + 2 +
+         weight_count(&m.rb3) + weight_count(&m.at3);
+}
+
+double flops_of(const dp_block_desc* d) {
+  const double hw = static_cast<double>(d->H) * d->W;
+  const double C = d->C, Co = d->Cout;
+  if (d->kind == DP_BLOCK_GN_CONV) return 2.0 * hw * Co * 9.0 * C;
+  if (d->kind == DP_BLOCK_RESBLOCK)
+    return 2.0 * hw * Co * 9.0 * C + 2.0 * hw * Co * 9.0 * Co + (C != Co ? 2.0 * hw * Co * C : 0.0);
+  if (d->kind == DP_BLOCK_ATTN)
+    return 2.0 * hw * 3.0 * C * C + 4.0 * hw * hw * C + 2.0 * hw * C * C;
+  const MiniDescs m = mini_descs(d);
+  return 2.0 * hw * kU1 * 9.0 * C + flops_of(&m.rb1) + 2.0 * (hw / 4) * kU1 * 9.0 * kU1 +
+         flops_of(&m.rb2) + flops_of(&m.at2) + 2.0 * (hw / 16) * kU2 * 9.0 * kU2 +
+         flops_of(&m.rb3) + flops_of(&m.at3);
 }
 
 template <typename T>
 T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+// One step of the block described by `d` whose state lives at `ws`; `cur`
+// selects the stale half of every ping-pong pair (the fresh half is cur ^ 1).
+int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* out,
+              const void* const* w, int mode, cudaStream_t st) {
+  const Layout L = layout_of(d);
+  const int f = cur ^ 1, o = cur;
+  const int H = d->H, W = d->W, C = d->C, Co = d->Cout, G = d->G, P = d->P;
+  auto gn = [&](const GnSlots& g, const void* in, void* y, const void* gamma, const void* beta,
+                int ch, int silu) {
+    return gn_launch(in, y, static_cast<const float*>(gamma), static_cast<const float*>(beta), H,
+                     W, ch, G, P, d->eps, d->w, silu, mode, d->dtype, at<float>(ws, g.global[o]),
+                     at<float>(ws, g.local[o]), at<float>(ws, g.local[f]),
+                     at<float>(ws, g.global[f]), at<float>(ws, g.used), at<void>(ws, g.ws), st);
+  };
+  int rc;
+  if (d->kind != DP_BLOCK_UNET_MINI) {
+    // biases (conv_b, conv1_b, conv2_b, short_b; bqkv, bo) may be NULL
+    for (int i = 0; i < weight_count(d); ++i) {
+      const bool bias = d->kind == DP_BLOCK_ATTN ? (i == 3 || i == 5)
+                                                 : (i == 3 || i == 7 || i == 9);
+      if (!w[i] && !bias) return set_error(DP_ERR_INVALID_ARG, "block: weight %d is NULL", i);
+    }
+  }
+  if (d->kind == DP_BLOCK_GN_CONV) {
+    rc = conv3x3_validate(x, x, w[2], nullptr, out, H, W, C, Co, 1, P, mode, d->dtype);
+    if (rc) return rc;
+    rc = gn(L.gn1, x, at<void>(ws, L.a1[f]), w[0], w[1], C, d->silu);
+    if (rc) return rc;
+    return conv3x3_launch(at<void>(ws, L.a1[f]), at<void>(ws, L.a1[o]), w[2],
+                          static_cast<const float*>(w[3]), nullptr, out, H, W, C, Co, 1, P, mode,
+                          d->dtype, st);
+  }
+  if (d->kind == DP_BLOCK_RESBLOCK) {
+    rc = conv3x3_validate(x, x, w[2], nullptr, out, H, W, C, Co, 1, P, mode, d->dtype);
+    if (rc) return rc;
+    rc = conv3x3_validate(x, x, w[6], nullptr, out, H, W, Co, Co, 1, P, mode, d->dtype);
+    if (rc) return rc;
+    void* a1f = at<void>(ws, L.a1[f]);
+    void* a2f = at<void>(ws, L.a2[f]);
+    void* h = at<void>(ws, L.h);
+    rc = gn(L.gn1, x, a1f, w[0], w[1], C, 1);
+    if (rc) return rc;
+    rc = conv3x3_launch(a1f, at<void>(ws, L.a1[o]), w[2], static_cast<const float*>(w[3]), nullptr,
+                        h, H, W, C, Co, 1, P, mode, d->dtype, st);
+    if (rc) return rc;
+    rc = gn(L.gn2, h, a2f, w[4], w[5], Co, 1);
+    if (rc) return rc;
+    const void* res = x;
+    if (C != Co) {
+      void* sc = at<void>(ws, L.sc);
+      rc = linear_launch(x, w[8], static_cast<const float*>(w[9]), nullptr, sc, nullptr, nullptr,
+                         H * W, Co, C, Co, st);
+      if (rc) return rc;
+      res = sc;
+    }
+    return conv3x3_launch(a2f, at<void>(ws, L.a2[o]), w[6], static_cast<const float*>(w[7]), res,
+                          out, H, W, Co, Co, 1, P, mode, d->dtype, st);
+  }
+  if (d->kind == DP_BLOCK_ATTN) {
+    const int T = H * W;
+    void* act = at<void>(ws, L.act);
+    void* q = at<void>(ws, L.q);
+    void* kf = at<void>(ws, L.k[f]);
+    void* vf = at<void>(ws, L.v[f]);
+    void* ob = at<void>(ws, L.o);
+    rc = gn(L.gn1, x, act, w[0], w[1], C, 0);
+    if (rc) return rc;
+    rc = linear_launch(act, w[2], static_cast<const float*>(w[3]), nullptr, q, kf, vf, T, 3 * C, C,
+                       C, st);
+    if (rc) return rc;
+    rc = attn_launch(q, kf, vf, at<void>(ws, L.k[o]), at<void>(ws, L.v[o]), ob, T, d->heads, P,
+                     0.125f, mode, st);
+    if (rc) return rc;
+    return linear_launch(ob, w[4], static_cast<const float*>(w[5]), x, out, nullptr, nullptr, T, C,
+                         C, C, st);
+  }
+  // UNET_MINI
+  const MiniDescs m = mini_descs(d);
+  const int H2 = H / 2, W2 = W / 2, H3 = H / 4, W3 = W / 4;
+  int wi = 0;
+  auto take = [&](int n) {
+    const void* const* p = w + wi;
+    wi += n;
+    return p;
+  };
+  void* xin = at<void>(ws, L.xin[f]);
+  rc = copy_launch(x, xin, static_cast<size_t>(H) * W * C * 2, st);
+  if (rc) return rc;
+  const void* const* wc = take(2);
+  if (!wc[0]) return set_error(DP_ERR_INVALID_ARG, "block: conv_in weight is NULL");
+  rc = conv3x3_small_launch(xin, at<void>(ws, L.xin[o]), wc[0], static_cast<const float*>(wc[1]),
+                            at<void>(ws, L.h0), H, W, C, kU1, P, mode, st);
+  if (rc) return rc;
+  rc = step_impl(&m.rb1, at<void>(ws, L.rb1), cur, at<void>(ws, L.h0), at<void>(ws, L.d1[f]),
+                 take(weight_count(&m.rb1)), mode, st);
+  if (rc) return rc;
+  wc = take(2);
+  if (!wc[0]) return set_error(DP_ERR_INVALID_ARG, "block: down1 weight is NULL");
+  rc = conv3x3_validate(at<void>(ws, L.d1[f]), at<void>(ws, L.d1[o]), wc[0], nullptr,
+                        at<void>(ws, L.h1), H, W, kU1, kU1, 2, P, mode, DP_BF16);
+  if (rc) return rc;
+  rc = conv3x3_launch(at<void>(ws, L.d1[f]), at<void>(ws, L.d1[o]), wc[0],
+                      static_cast<const float*>(wc[1]), nullptr, at<void>(ws, L.h1), H, W, kU1,
+                      kU1, 2, P, mode, DP_BF16, st);
+  if (rc) return rc;
+  rc = step_impl(&m.rb2, at<void>(ws, L.rb2), cur, at<void>(ws, L.h1), at<void>(ws, L.h2),
+                 take(weight_count(&m.rb2)), mode, st);
+  if (rc) return rc;
+  rc = step_impl(&m.at2, at<void>(ws, L.at2), cur, at<void>(ws, L.h2), at<void>(ws, L.d2[f]),
+                 take(weight_count(&m.at2)), mode, st);
+  if (rc) return rc;
+  wc = take(2);
+  if (!wc[0]) return set_error(DP_ERR_INVALID_ARG, "block: down2 weight is NULL");
+  rc = conv3x3_validate(at<void>(ws, L.d2[f]), at<void>(ws, L.d2[o]), wc[0], nullptr,
+                        at<void>(ws, L.h3), H2, W2, kU2, kU2, 2, P, mode, DP_BF16);
+  if (rc) return rc;
+  rc = conv3x3_launch(at<void>(ws, L.d2[f]), at<void>(ws, L.d2[o]), wc[0],
+                      static_cast<const float*>(wc[1]), nullptr, at<void>(ws, L.h3), H2, W2, kU2,
+                      kU2, 2, P, mode, DP_BF16, st);
+  if (rc) return rc;
+  rc = step_impl(&m.rb3, at<void>(ws, L.rb3), cur, at<void>(ws, L.h3), at<void>(ws, L.h4),
+                 take(weight_count(&m.rb3)), mode, st);
+  if (rc) return rc;
+  (void)H3;
+  (void)W3;
+  return step_impl(&m.at3, at<void>(ws, L.at3), cur, at<void>(ws, L.h4), out,
+                   take(weight_count(&m.at3)), mode, st);
 }
 
 }  // namespace
@@ -115,7 +353,7 @@ int dp_block_desc_init(dp_block_desc* d, int kind, int H, int W, int C, int Cout
   d->H = H;
   d->W = W;
   d->C = C;
-  d->Cout = Cout > 0 ? Cout : C;
+  d->Cout = kind == DP_BLOCK_UNET_MINI ? dp::kU3 : (Cout > 0 ? Cout : C);
   d->G = G;
   d->P = P;
   d->heads = heads;
@@ -153,13 +391,13 @@ int dp_block_state_init(const dp_block_desc* d, dp_block_state* s, void* workspa
 
 double dp_block_flops(const dp_block_desc* d) {
   if (dp::desc_check(d)) return 0.0;
-  const double hw = static_cast<double>(d->H) * d->W;
-  const double C = d->C, Co = d->Cout;
-  if (d->kind == DP_BLOCK_GN_CONV) return 2.0 * hw * Co * 9.0 * C;
-  if (d->kind == DP_BLOCK_RESBLOCK)
-    return 2.0 * hw * Co * 9.0 * C + 2.0 * hw * Co * 9.0 * Co + (C != Co ? 2.0 * hw * Co * C : 0.0);
-  // attention block: q/k/v and output projections + QK^T and PV over all keys
-  return 2.0 * hw * 3.0 * C * C + 4.0 * hw * hw * C + 2.0 * hw * C * C;
+  return dp::flops_of(d);
+}
+
+int dp_block_weight_count(const dp_block_desc* d) {
+  int rc = dp::desc_check(d);
+  if (rc) return rc;
+  return dp::weight_count(d);
 }
 
 int dp_block_step(const dp_block_desc* d, dp_block_state* s, const void* x, void* out,
@@ -175,83 +413,14 @@ int dp_block_step(const dp_block_desc* d, dp_block_state* s, const void* x, void
   if (x == out) return dp::set_error(DP_ERR_INVALID_ARG, "block: out aliases x");
   if (!dp::aligned16(x) || !dp::aligned16(out))
     return dp::set_error(DP_ERR_UNSUPPORTED, "block: x/out not 16-byte aligned");
-  const dp::Layout L = dp::layout_of(d);
-  if (s->workspace_bytes < L.total) return dp::set_error(DP_ERR_INVALID_ARG, "block: workspace too small");
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  void* ws = s->workspace;
-  const int f = s->cur ^ 1, o = s->cur;   // fresh / stale halves
-  const int H = d->H, W = d->W, C = d->C, Co = d->Cout, G = d->G, P = d->P;
-  auto gn = [&](const dp::GnSlots& g, const void* in, void* y, const void* gamma, const void* beta,
-                int ch, int silu) {
-    return dp::gn_launch(in, y, static_cast<const float*>(gamma), static_cast<const float*>(beta), H,
-                         W, ch, G, P, d->eps, d->w, silu, mode, d->dtype,
-                         dp::at<float>(ws, g.global[o]), dp::at<float>(ws, g.local[o]),
-                         dp::at<float>(ws, g.local[f]), dp::at<float>(ws, g.global[f]),
-                         dp::at<float>(ws, g.used), dp::at<void>(ws, g.ws), st);
-  };
-  const void* const* w = weights;
-  if (d->kind == DP_BLOCK_GN_CONV) {
-    if (n_weights < 4) return dp::set_error(DP_ERR_INVALID_ARG, "block: GN_CONV needs 4 weights");
-    if (!w[0] || !w[1] || !w[2]) return dp::set_error(DP_ERR_INVALID_ARG, "block: null weight");
-    rc = dp::conv3x3_validate(x, x, w[2], nullptr, out, H, W, C, Co, 1, P, mode, d->dtype);
-    if (rc) return rc;
-    rc = gn(L.gn1, x, dp::at<void>(ws, L.a1[f]), w[0], w[1], C, d->silu);
-    if (rc) return rc;
-    rc = dp::conv3x3_launch(dp::at<void>(ws, L.a1[f]), dp::at<void>(ws, L.a1[o]), w[2],
-                            static_cast<const float*>(w[3]), nullptr, out, H, W, C, Co, 1, P, mode,
-                            d->dtype, st);
-    if (rc) return rc;
-  } else if (d->kind == DP_BLOCK_RESBLOCK) {
-    const int need = C != Co ? 10 : 8;
-    if (n_weights < need) return dp::set_error(DP_ERR_INVALID_ARG, "block: RESBLOCK needs %d weights", need);
-    if (!w[0] || !w[1] || !w[2] || !w[4] || !w[5] || !w[6] || (C != Co && !w[8]))
-      return dp::set_error(DP_ERR_INVALID_ARG, "block: null weight");
-    rc = dp::conv3x3_validate(x, x, w[2], nullptr, out, H, W, C, Co, 1, P, mode, d->dtype);
-    if (rc) return rc;
-    rc = dp::conv3x3_validate(x, x, w[6], nullptr, out, H, W, Co, Co, 1, P, mode, d->dtype);
-    if (rc) return rc;
-    void* a1f = dp::at<void>(ws, L.a1[f]);
-    void* a2f = dp::at<void>(ws, L.a2[f]);
-    void* h = dp::at<void>(ws, L.h);
-    rc = gn(L.gn1, x, a1f, w[0], w[1], C, 1);
-    if (rc) return rc;
-    rc = dp::conv3x3_launch(a1f, dp::at<void>(ws, L.a1[o]), w[2], static_cast<const float*>(w[3]),
-                            nullptr, h, H, W, C, Co, 1, P, mode, d->dtype, st);
-    if (rc) return rc;
-    rc = gn(L.gn2, h, a2f, w[4], w[5], Co, 1);
-    if (rc) return rc;
-    const void* res = x;
-    if (C != Co) {
-      void* sc = dp::at<void>(ws, L.sc);
-      rc = dp::linear_launch(x, w[8], static_cast<const float*>(w[9]), nullptr, sc, nullptr, nullptr,
-                             H * W, Co, C, Co, st);
-      if (rc) return rc;
-      res = sc;
-    }
-    rc = dp::conv3x3_launch(a2f, dp::at<void>(ws, L.a2[o]), w[6], static_cast<const float*>(w[7]),
-                            res, out, H, W, Co, Co, 1, P, mode, d->dtype, st);
-    if (rc) return rc;
-  } else {
-    if (n_weights < 6) return dp::set_error(DP_ERR_INVALID_ARG, "block: ATTN needs 6 weights");
-    if (!w[0] || !w[1] || !w[2] || !w[4]) return dp::set_error(DP_ERR_INVALID_ARG, "block: null weight");
-    const int T = H * W;
-    void* act = dp::at<void>(ws, L.act);
-    void* q = dp::at<void>(ws, L.q);
-    void* kf = dp::at<void>(ws, L.k[f]);
-    void* vf = dp::at<void>(ws, L.v[f]);
-    void* ob = dp::at<void>(ws, L.o);
-    rc = gn(L.gn1, x, act, w[0], w[1], C, 0);
-    if (rc) return rc;
-    rc = dp::linear_launch(act, w[2], static_cast<const float*>(w[3]), nullptr, q, kf, vf, T, 3 * C,
-                           C, C, st);
-    if (rc) return rc;
-    rc = dp::attn_launch(q, kf, vf, dp::at<void>(ws, L.k[o]), dp::at<void>(ws, L.v[o]), ob, T,
-                         d->heads, P, 0.125f, mode, st);
-    if (rc) return rc;
-    rc = dp::linear_launch(ob, w[4], static_cast<const float*>(w[5]), x, out, nullptr, nullptr, T, C,
-                           C, C, st);
-    if (rc) return rc;
-  }
+  if (n_weights < dp::weight_count(d))
+    return dp::set_error(DP_ERR_INVALID_ARG, "block: %d weights given, %d needed", n_weights,
+                         dp::weight_count(d));
+  if (s->workspace_bytes < dp::layout_of(d).total)
+    return dp::set_error(DP_ERR_INVALID_ARG, "block: workspace too small");
+  rc = dp::step_impl(d, s->workspace, s->cur, x, out, weights, mode,
+                     static_cast<cudaStream_t>(stream));
+  if (rc) return rc;
   s->cur ^= 1;
   s->steps_done += 1;
   return DP_OK;
@@ -260,9 +429,7 @@ int dp_block_step(const dp_block_desc* d, dp_block_state* s, const void* x, void
 int dp_block_launch_count(const dp_block_desc* d) {
   int rc = dp::desc_check(d);
   if (rc) return rc;
-  if (d->kind == DP_BLOCK_GN_CONV) return 3;
-  if (d->kind == DP_BLOCK_RESBLOCK) return d->C != d->Cout ? 7 : 6;
-  return 5;
+  return dp::launch_count(d);
 }
 
 int dp_block_step_timed(const dp_block_desc* d, dp_block_state* s, const void* x, void* out,

@@ -6,36 +6,38 @@
 // summary, Method): rows of other bands come from the fresh input (sync), the
 // previous step's input (displaced) or nowhere (naive).
 //
-// One thread computes 8 consecutive output channels of one pixel; the whole
-// filter bank sits in shared memory as fp32, laid out [tap][ci][co] so that
-// the 8 channels of a thread are contiguous.
+// One thread computes 32 consecutive output channels of one pixel; a warp holds
+// 32 neighbouring pixels of the same channel group, so every weight it reads
+// from shared memory is the same address for all lanes (a broadcast), and its
+// input loads are adjacent pixels.  The filter slice of the block's channel
+// group sits in shared memory as fp32, laid out [tap][ci][32].
 #include "dp_common.cuh"
 #include "dp_internal.h"
 
 namespace dp {
 
+constexpr int kSmallCo = 32;   // output channels per thread
+
 __global__ void __launch_bounds__(256) conv3x3_small_kernel(
     const __nv_bfloat16* __restrict__ af, const __nv_bfloat16* __restrict__ as,
     const __nv_bfloat16* __restrict__ w, const float* __restrict__ bias,
     __nv_bfloat16* __restrict__ out, int H, int W, int Cin, int Cout, int hb, int mode) {
-  extern __shared__ float sw[];   // [9][Cin][Cout]
-  const int nw = 9 * Cin * Cout;
+  extern __shared__ float sw[];   // [9][Cin][32] for channel group blockIdx.y
+  const int co0 = blockIdx.y * kSmallCo;
+  const int nw = 9 * Cin * kSmallCo;
   for (int i = threadIdx.x; i < nw; i += blockDim.x) {
-    const int co = i % Cout, k = i / Cout;          // k = tap * Cin + ci
+    const int j = i % kSmallCo, k = i / kSmallCo;   // k = tap * Cin + ci
     const int tap = k / Cin, ci = k % Cin;
-    sw[i] = __bfloat162float(w[(static_cast<size_t>(co) * 9 + tap) * Cin + ci]);
+    sw[i] = __bfloat162float(w[(static_cast<size_t>(co0 + j) * 9 + tap) * Cin + ci]);
   }
   __syncthreads();
-  const int groups = Cout / 8;
-  const long idx = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= static_cast<long>(H) * W * groups) return;
-  const int g = static_cast<int>(idx % groups);
-  const long pix = idx / groups;
+  const long pix = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (pix >= static_cast<long>(H) * W) return;
   const int r = static_cast<int>(pix / W), c = static_cast<int>(pix % W);
   const int band = r / hb;
-  float acc[8];
+  float acc[kSmallCo];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) acc[j] = bias ? bias[g * 8 + j] : 0.f;
+  for (int j = 0; j < kSmallCo; ++j) acc[j] = bias ? __ldg(bias + co0 + j) : 0.f;
   for (int kh = 0; kh < 3; ++kh) {
     const int rho = r + kh - 1;
     if (rho < 0 || rho >= H) continue;
@@ -48,40 +50,33 @@ __global__ void __launch_bounds__(256) conv3x3_small_kernel(
       const int col = c + kw - 1;
       if (col < 0 || col >= W) continue;
       const __nv_bfloat16* px = src + (static_cast<size_t>(rho) * W + col) * Cin;
-      const float* wt = sw + (kh * 3 + kw) * Cin * Cout + g * 8;
+      const float* wt = sw + (kh * 3 + kw) * Cin * kSmallCo;
       for (int ci = 0; ci < Cin; ++ci) {
         const float v = __bfloat162float(px[ci]);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[j] = fmaf(v, wt[ci * Cout + j], acc[j]);
+        for (int j = 0; j < kSmallCo; ++j) acc[j] = fmaf(v, wt[ci * kSmallCo + j], acc[j]);
       }
     }
   }
-  uint4 u;
-  u.x = pack_bf16x2(acc[0], acc[1]);
-  u.y = pack_bf16x2(acc[2], acc[3]);
-  u.z = pack_bf16x2(acc[4], acc[5]);
-  u.w = pack_bf16x2(acc[6], acc[7]);
-  *reinterpret_cast<uint4*>(out + pix * Cout + g * 8) = u;
+  uint4* dst = reinterpret_cast<uint4*>(out + pix * Cout + co0);
+#pragma unroll
+  for (int q = 0; q < kSmallCo / 8; ++q) {
+    uint4 u;
+    u.x = pack_bf16x2(acc[8 * q], acc[8 * q + 1]);
+    u.y = pack_bf16x2(acc[8 * q + 2], acc[8 * q + 3]);
+    u.z = pack_bf16x2(acc[8 * q + 4], acc[8 * q + 5]);
+    u.w = pack_bf16x2(acc[8 * q + 6], acc[8 * q + 7]);
+    dst[q] = u;
+  }
 }
 
 int conv3x3_small_launch(const void* af, const void* as, const void* w, const float* bias,
                          void* out, int H, int W, int Cin, int Cout, int P, int mode,
                          cudaStream_t stream) {
-  const size_t smem = static_cast<size_t>(9) * Cin * Cout * sizeof(float);
-  static int attr_mask = 0;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (smem > 48 * 1024 && !(attr_mask & (1 << (dev & 31)))) {
-    int rc = cuda_check(cudaFuncSetAttribute(conv3x3_small_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024),
-                        "small conv smem attribute");
-    if (rc) return rc;
-    attr_mask |= 1 << (dev & 31);
-  }
-  const long threads = static_cast<long>(H) * W * (Cout / 8);
-  const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+  const size_t smem = static_cast<size_t>(9) * Cin * kSmallCo * sizeof(float);
+  const dim3 grid(static_cast<unsigned>((static_cast<long>(H) * W + 255) / 256), Cout / kSmallCo);
   mark_launch(stream);
-  conv3x3_small_kernel<<<blocks, 256, smem, stream>>>(
+  conv3x3_small_kernel<<<grid, 256, smem, stream>>>(
       static_cast<const __nv_bfloat16*>(af), static_cast<const __nv_bfloat16*>(as ? as : af),
       static_cast<const __nv_bfloat16*>(w), bias, static_cast<__nv_bfloat16*>(out), H, W, Cin,
       Cout, H / P, mode);
@@ -100,8 +95,8 @@ extern "C" int dp_conv3x3_halo_small(const void* a_fresh, const void* a_stale, c
     return dp::set_error(DP_ERR_INVALID_ARG, "small conv: bad mode %d", mode);
   if (mode == DP_MODE_DISPLACED && !a_stale)
     return dp::set_error(DP_ERR_INVALID_ARG, "small conv: displaced mode needs the stale buffer");
-  if (Cin > 16 || Cout % 8 || 9L * Cin * Cout * 4 > 200 * 1024)
-    return dp::set_error(DP_ERR_UNSUPPORTED, "small conv: needs Cin <= 16, Cout %% 8 == 0, small filter bank");
+  if (Cin > 16 || Cout % 32)
+    return dp::set_error(DP_ERR_UNSUPPORTED, "small conv: needs Cin <= 16 and Cout %% 32 == 0");
   if (H % P) return dp::set_error(DP_ERR_UNSUPPORTED, "small conv: H %% P != 0");
   if (!dp::aligned16(out)) return dp::set_error(DP_ERR_UNSUPPORTED, "small conv: out not 16-byte aligned");
   if (out == a_fresh || out == a_stale) return dp::set_error(DP_ERR_INVALID_ARG, "small conv: out aliases an input");

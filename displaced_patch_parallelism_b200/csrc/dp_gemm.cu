@@ -349,10 +349,331 @@ __global__ void __launch_bounds__(192, 1) igemm_kernel(const __grid_constant__ G
 
   tc_fence_before();
   __syncthreads();
+  __syncwarp();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
+}
+
+// ---------------------------------------------------------------------------
+// Pair kernel: two CTAs of a cluster share one 256 x (NI*NJ) output tile.
+// Each CTA loads its own 128 rows of A and half of every NI-wide slice of B;
+// the leader CTA issues tcgen05.mma.cta_group::2 (M = 256), which reads both
+// CTAs' shared memory and writes each CTA's 128 accumulator rows into that
+// CTA's tensor memory.  Per SM this halves the weight bytes per flop.
+template <int NI, int NJ>
+struct PairCfg {
+  static constexpr int BN = NI * NJ;                 // output columns per pair tile
+  static constexpr int A_BYTES = 128 * 128;
+  static constexpr int BSUB_BYTES = (NI / 2) * 128;  // this CTA's half of one B slice
+  static constexpr int B_BYTES = NJ * BSUB_BYTES;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES_RAW = (200 * 1024) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  static constexpr int TMEM_COLS = BN <= 128 ? 128 : BN <= 256 ? 256 : 512;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 256;
+  static_assert(BSUB_BYTES % 1024 == 0, "B slice alignment");
+  static_assert(BN <= 512 && NI % 32 == 0 && NI <= 256, "tile");
+};
+
+template <int NI, int NJ>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+    igemm_pair_kernel(const __grid_constant__ GemmParams p) {
+  using C = PairCfg<NI, NJ>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + C::STAGES * C::A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::STAGES * C::B_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* acc_full = empty + C::STAGES;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* drain = acc_empty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = warp_id(), lane = lane_id();
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int num_tiles = ((p.m_tiles + 1) >> 1) * p.n_tiles;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 8);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&p.tmA0);
+    if (p.a_mode == 1) prefetch_tmap(&p.tmA1);
+    prefetch_tmap(&p.tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer (both CTAs)
+      int stage = 0;
+      uint32_t phase = 0;
+      int ry_tab[3 * 16];
+      uint64_t stale_mask = 0;
+      const uint32_t full0 = mapa_shared(smem_u32(full), 0);   // leader's full[0]
+      for (int tile = pair; tile < num_tiles && !*abort_flag; tile += npairs) {
+        const int mp = tile / p.n_tiles, nt = tile - mp * p.n_tiles;
+        const int mt = 2 * mp + static_cast<int>(rank);
+        int c0 = 0;
+        if (p.a_mode == 1) {
+          const int tr = mt / p.tiles_w, tc = mt - tr * p.tiles_w;
+          const int r0 = tr * p.R;
+          c0 = tc * p.Wt;
+          stale_mask = 0;
+          for (int i = 0; i < p.R; ++i) {
+            const int r = r0 + i;
+            const int band = r / p.hb_out;
+            const int lo = band * p.hb_in, hi = lo + p.hb_in;
+            for (int kh = 0; kh < 3; ++kh) {
+              const int rho = p.stride * r + kh - 1;
+              int ry = rho;
+              if (r >= p.Ho) {
+                ry = -1;
+              } else if (rho >= 0 && rho < p.H && (rho < lo || rho >= hi)) {
+                if (p.mode == DP_MODE_DISPLACED) stale_mask |= 1ull << (kh * 16 + i);
+                else if (p.mode == DP_MODE_NAIVE) ry = -1;
+              }
+              ry_tab[kh * 16 + i] = ry;
+            }
+          }
+        }
+        int kh = 0, kw = 0, cb = 0;
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status)) goto producer_done;
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
+          const uint32_t fb = full0 + stage * 8;
+          uint8_t* a_dst = sA + stage * C::A_BYTES;
+          if (p.a_mode == 0) {
+            tma_load_2d_pair(a_dst, &p.tmA0, fb, kb * 64, mt * 128);
+          } else {
+            int kx, cx;
+            if (p.stride == 1) {
+              kx = cb * 64;
+              cx = c0 + kw - 1;
+            } else {
+              kx = (kw == 1 ? 0 : p.Cin) + cb * 64;
+              cx = c0 - (kw == 0 ? 1 : 0);
+            }
+            const int* ryk = ry_tab + kh * 16;
+            const uint32_t sk = static_cast<uint32_t>(stale_mask >> (kh * 16));
+            for (int i = 0; i < p.R; ++i)
+              tma_load_3d_pair(a_dst + i * p.Wt * 128, ((sk >> i) & 1u) ? &p.tmA1 : &p.tmA0, fb,
+                               kx, cx, ryk[i]);
+            if (++cb == p.kc) {
+              cb = 0;
+              if (++kw == 3) {
+                kw = 0;
+                ++kh;
+              }
+            }
+          }
+          uint8_t* b_dst = sB + stage * C::B_BYTES;
+#pragma unroll
+          for (int j = 0; j < NJ; ++j)
+            tma_load_2d_pair(b_dst + j * C::BSUB_BYTES, &p.tmB, fb, kb * 64,
+                             nt * C::BN + j * NI + static_cast<int>(rank) * (NI / 2));
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    producer_done:
+      if (*abort_flag) {
+        // Loads in flight complete on the leader's barrier; give them time to land.
+        const unsigned long long t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 2000000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ------------------------------------------------------------ MMA issuer (leader CTA)
+      constexpr uint32_t idesc = idesc_dense(256, NI, 1, 0, 0);
+      const uint64_t a_desc0 = sdesc_sw128(smem_u32(sA), 1024);
+      const uint64_t b_desc0 = sdesc_sw128(smem_u32(sB), 1024);
+      const uint32_t empty_own = smem_u32(empty), empty_peer = mapa_shared(smem_u32(empty), 1);
+      const uint32_t accf_own = smem_u32(acc_full), accf_peer = mapa_shared(smem_u32(acc_full), 1);
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      for (int tile = pair; tile < num_tiles; tile += npairs, ++it) {
+        if (!mbar_wait(acc_empty, (it & 1) ^ 1, abort_flag, p.status)) goto mma_done;
+        tc_fence_after();
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.status)) goto mma_done;
+          tc_fence_after();
+          const uint64_t ad = a_desc0 + static_cast<uint64_t>((stage * C::A_BYTES) >> 4);
+          const uint64_t bd = b_desc0 + static_cast<uint64_t>((stage * C::B_BYTES) >> 4);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+#pragma unroll
+            for (int j = 0; j < NJ; ++j)
+              umma_f16_ss_pair(tmem + j * NI, ad + 2 * k,
+                               bd + static_cast<uint64_t>((j * C::BSUB_BYTES) >> 4) + 2 * k, idesc,
+                               (kb | k) != 0);
+          umma_commit_pair(empty_own + stage * 8);
+          umma_commit_pair(empty_peer + stage * 8);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        umma_commit_pair(accf_own);
+        umma_commit_pair(accf_peer);
+      }
+    mma_done:
+      if (*abort_flag) {
+        umma_commit_pair(smem_u32(drain));
+        mbar_wait_teardown(drain, 0);
+      }
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue (both CTAs)
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
+    int it = 0;
+    for (int tile = pair; tile < num_tiles; tile += npairs, ++it) {
+      if (!mbar_wait(acc_full, it & 1, abort_flag, p.status)) break;
+      tc_fence_after();
+      const int mp = tile / p.n_tiles, nt = tile - mp * p.n_tiles;
+      const int mt = 2 * mp + static_cast<int>(rank);
+      bool valid;
+      size_t pix;
+      if (p.a_mode == 0) {
+        const int m = mt * 128 + row;
+        valid = m < p.M;
+        pix = static_cast<size_t>(m);
+      } else {
+        const int tr = mt / p.tiles_w, tc = mt - tr * p.tiles_w;
+        const int r = tr * p.R + row / p.Wt, c = tc * p.Wt + row % p.Wt;
+        valid = mt < p.m_tiles && r < p.Ho && c < p.Wo;
+        pix = static_cast<size_t>(r) * p.Wo + c;
+      }
+      const int n0 = nt * C::BN;
+      const int seg = n0 / p.split;
+      __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(seg == 0 ? p.out0 : seg == 1 ? p.out1 : p.out2);
+      __nv_bfloat16* orow = outp + pix * p.ld_out + (n0 - seg * p.split);
+      const __nv_bfloat16* rrow =
+          p.residual ? static_cast<const __nv_bfloat16*>(p.residual) + pix * p.N + n0 : nullptr;
+#pragma unroll 1
+      for (int ch = 0; ch < C::BN / 32; ++ch) {
+        uint32_t r[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + ch * 32, r);
+        tmem_wait_ld();
+        if (ch == C::BN / 32 - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
+        }
+        if (!valid) continue;
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+        if (p.bias) {
+          const float4* b4 = reinterpret_cast<const float4*>(p.bias + n0 + ch * 32);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float4 b = __ldg(b4 + j);
+            v[4 * j] += b.x;
+            v[4 * j + 1] += b.y;
+            v[4 * j + 2] += b.z;
+            v[4 * j + 3] += b.w;
+          }
+        }
+        if (rrow) {
+          const uint4* r4 = reinterpret_cast<const uint4*>(rrow + ch * 32);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint4 u = r4[j];
+            const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __bfloat1622float2(h[e]);
+              v[8 * j + 2 * e] += f.x;
+              v[8 * j + 2 * e + 1] += f.y;
+            }
+          }
+        }
+        uint4* o4 = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint4 u;
+          u.x = pack_bf16x2(v[8 * j], v[8 * j + 1]);
+          u.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
+          u.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
+          u.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
+          o4[j] = u;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync_all();
+  __syncwarp();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int NI, int NJ>
+static int launch_pair(const GemmParams& p, cudaStream_t s) {
+  using C = PairCfg<NI, NJ>;
+  static int grid_cache[32] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int& maxg = grid_cache[dev & 31];
+  if (!maxg) {
+    int rc = cuda_check(cudaFuncSetAttribute(igemm_pair_kernel<NI, NJ>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM),
+                        "pair gemm smem attribute");
+    if (rc) return rc;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * num_sms());
+    cfg.blockDim = dim3(192);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, igemm_pair_kernel<NI, NJ>, &cfg) != cudaSuccess ||
+        clusters <= 0) {
+      cudaGetLastError();
+      clusters = num_sms() / 2;
+    }
+    maxg = 2 * clusters;
+  }
+  const int pair_tiles = ((p.m_tiles + 1) / 2) * p.n_tiles;
+  const int grid = std::min(2 * pair_tiles, maxg);
+  mark_launch(s);
+  igemm_pair_kernel<NI, NJ><<<grid, 192, C::SMEM, s>>>(p);
+  return cuda_check(cudaGetLastError(), "pair gemm launch");
 }
 
 template <int BN, bool TF32>
@@ -420,6 +741,35 @@ static int pick_bn(int m_tiles, int N, int split, bool tf32) {
   return best;
 }
 
+// Tile choice for bf16 work: 256x320 or 256x160 pair tiles, or a 128-row
+// single-CTA tile.  Estimated time = waves x per-SM work of one tile / the
+// relative efficiency measured for that tile (pair tiles move half the
+// weight bytes per flop).  Returns the pair width (320 or 160) or 0.
+static int pick_pair(int m_tiles, int N, int split, int* bn_single) {
+  const long sms = num_sms(), pairs = sms / 2;
+  const long mp = (m_tiles + 1) / 2;
+  double best = 0.0;
+  int choice = 0;
+  struct Opt { int width; double eff; };
+  const Opt opts[2] = {{320, 1.0}, {160, 0.75}};
+  for (const Opt& o : opts) {
+    if (split % o.width) continue;
+    const long tiles = mp * (N / o.width);
+    const double t = static_cast<double>((tiles + pairs - 1) / pairs) * (128.0 * o.width) / o.eff;
+    if (!choice || t < best) {
+      best = t;
+      choice = o.width;
+    }
+  }
+  *bn_single = pick_bn(m_tiles, N, split, false);
+  if (*bn_single) {
+    const long tiles = static_cast<long>(m_tiles) * (N / *bn_single);
+    const double t = static_cast<double>((tiles + sms - 1) / sms) * (128.0 * *bn_single) / 0.6;
+    if (!choice || t < best) choice = 0;
+  }
+  return choice;
+}
+
 int conv3x3_launch(const void* a_fresh, const void* a_stale, const void* weight,
                    const float* bias, const void* residual, void* out, int H, int W, int Cin,
                    int Cout, int stride, int P, int mode, int dtype, cudaStream_t stream) {
@@ -448,6 +798,9 @@ int conv3x3_launch(const void* a_fresh, const void* a_stale, const void* weight,
       Wt = w;
     }
   }
+  // A single 128-pixel row per tile keeps one TMA box per A stage; take it when
+  // the ragged right edge wastes at most an eighth of the row.
+  if (Wo >= 128 && (((Wo + 127) / 128) * 128 - Wo) * 8 <= Wo) Wt = 128;
   p.Wt = Wt;
   p.R = 128 / Wt;
   p.tiles_w = (Wo + Wt - 1) / Wt;
@@ -461,7 +814,10 @@ int conv3x3_launch(const void* a_fresh, const void* a_stale, const void* weight,
   p.residual = residual;
   p.out0 = out;
   p.status = device_status_ptr();
-  const int BN = pick_bn(p.m_tiles, Cout, Cout, tf32);
+  int bn_single = 0;
+  const int pw = tf32 ? 0 : pick_pair(p.m_tiles, Cout, Cout, &bn_single);
+  const bool pair = pw != 0;
+  const int BN = pair ? pw : pick_bn(p.m_tiles, Cout, Cout, tf32);
   if (!BN) return set_error(DP_ERR_UNSUPPORTED, "conv: no N tile divides Cout=%d", Cout);
   p.n_tiles = Cout / BN;
   const CUtensorMapDataType dt =
@@ -485,10 +841,11 @@ int conv3x3_launch(const void* a_fresh, const void* a_stale, const void* weight,
   if (rc) return rc;
   uint64_t bdims[2] = {9 * static_cast<uint64_t>(Cin), static_cast<uint64_t>(Cout)};
   uint64_t bstr[1] = {9 * static_cast<uint64_t>(Cin) * e};
-  uint32_t bbox[2] = {static_cast<uint32_t>(BK), static_cast<uint32_t>(BN)};
+  uint32_t bbox[2] = {static_cast<uint32_t>(BK), static_cast<uint32_t>(pair ? 80 : BN)};
   rc = encode_tmap(&p.tmB, dt, 2, const_cast<void*>(weight), bdims, bstr, bbox,
                    CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc) return rc;
+  if (pair) return pw == 320 ? launch_pair<160, 2>(p, stream) : launch_pair<160, 1>(p, stream);
   return launch_gemm(p, BN, tf32, stream);
 }
 
@@ -510,7 +867,10 @@ int linear_launch(const void* x, const void* weight, const float* bias, const vo
   p.out1 = out1;
   p.out2 = out2;
   p.status = device_status_ptr();
-  const int BN = pick_bn(p.m_tiles, N, split, false);
+  int bn_single = 0;
+  const int pw = pick_pair(p.m_tiles, N, split, &bn_single);
+  const bool pair = pw != 0;
+  const int BN = pair ? pw : bn_single;
   if (!BN) return set_error(DP_ERR_UNSUPPORTED, "linear: no N tile divides split=%d", split);
   p.n_tiles = N / BN;
   uint64_t adims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
@@ -520,10 +880,11 @@ int linear_launch(const void* x, const void* weight, const float* bias, const vo
                        astr, abox, CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc) return rc;
   uint64_t bdims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N)};
-  uint32_t bbox[2] = {64, static_cast<uint32_t>(BN)};
+  uint32_t bbox[2] = {64, static_cast<uint32_t>(pair ? 80 : BN)};
   rc = encode_tmap(&p.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(weight), bdims,
                    astr, bbox, CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc) return rc;
+  if (pair) return pw == 320 ? launch_pair<160, 2>(p, stream) : launch_pair<160, 1>(p, stream);
   return launch_gemm(p, BN, false, stream);
 }
 

@@ -276,7 +276,8 @@ static int gn_plan(int H, int W, int C, int G, int P, int dtype, GnArgs* a) {
   a->vpp = C / V;
   a->lanes = a->vpp >= 512 ? 1 : 512 / a->vpp;
   if (a->vpp * a->lanes > 1024) a->lanes = 1024 / a->vpp;
-  int s = (4 * num_sms() + P - 1) / P;
+  // One full wave of resident blocks (2 per SM at up to 1024 threads each).
+  int s = (2 * num_sms()) / P;
   const int by_work = (a->HWp + 4 * a->lanes - 1) / (4 * a->lanes);
   if (s > by_work) s = by_work;
   if (s > kGnMaxSplits) s = kGnMaxSplits;

@@ -156,7 +156,7 @@ WORKLOADS: Dict[str, Workload] = {
         name="gn_conv_320x480x480", kind="gn_conv", C=320, H=480, W=480, P=8,
         steps=50, warmup=4, drift=0.05),
     "unet_mini_4x128x128": Workload(
-        name="unet_mini_4x128x128", kind="unet_mini", C=4, H=128, W=128, P=4,
+        name="unet_mini_4x128x128", kind="unet_mini", C=4, H=128, W=128, P=4, Cout=1280,
         steps=10, warmup=2, drift=0.03, weight_seed=7),
 }
 

@@ -47,4 +47,14 @@ def block_weights(kind: str, wts: Dict, dtype: torch.dtype = torch.bfloat16, dev
                 _t(cat(g("wq"), g("wk"), g("wv")), dtype, device),
                 _t(cat(g("bq"), g("bk"), g("bv")), f32, device),
                 _t(g("wo"), dtype, device), _t(g("bo"), f32, device)]
+    if kind == "unet_mini":
+        out = [_conv(g("conv_in_w"), dtype, device), _t(g("conv_in_b"), f32, device)]
+        out += block_weights("resblock", wts, dtype, device, prefix + "rb1.")
+        out += [_conv(g("down1_w"), dtype, device), _t(g("down1_b"), f32, device)]
+        out += block_weights("resblock", wts, dtype, device, prefix + "rb2.")
+        out += block_weights("attn", wts, dtype, device, prefix + "at2.")
+        out += [_conv(g("down2_w"), dtype, device), _t(g("down2_b"), f32, device)]
+        out += block_weights("resblock", wts, dtype, device, prefix + "rb3.")
+        out += block_weights("attn", wts, dtype, device, prefix + "at3.")
+        return out
     raise ValueError(kind)

@@ -70,6 +70,8 @@ extern "C" {
 #define DP_BLOCK_GN_CONV 0  /* GroupNorm (+SiLU) -> 3x3 conv                                */
 #define DP_BLOCK_RESBLOCK 1 /* GN -> SiLU -> conv1 -> GN -> SiLU -> conv2 -> + x / shortcut */
 #define DP_BLOCK_ATTN 2     /* GN -> q,k,v proj -> stale-K/V attention -> out proj -> + x   */
+#define DP_BLOCK_UNET_MINI 3 /* conv_in -> ResBlock(320) -> down -> ResBlock(320->640) ->   */
+                             /* Attn(640) -> down -> ResBlock(640->1280) -> Attn(1280)      */
 
 /* Message for the calling thread's last failed call ("" if none). */
 DP_API const char* dp_last_error(void);
@@ -187,7 +189,7 @@ DP_API int dp_conv3x3_halo(const void* a_fresh, const void* a_stale, const void*
 /* ------------------------------------------------------------------------
  * Direct 3x3 conv for few input channels (the latent input conv), same
  * halo rule and layouts as dp_conv3x3_halo, stride 1, bf16 only.
- * Needs Cin <= 16, Cout % 8 == 0.  Runs on the CUDA cores.
+ * Needs Cin <= 16, Cout % 32 == 0.  Runs on the CUDA cores.
  * ---------------------------------------------------------------------- */
 DP_API int dp_conv3x3_halo_small(const void* a_fresh, const void* a_stale, const void* weight,
                           const float* bias, void* out, int H, int W, int Cin, int Cout,
@@ -256,7 +258,8 @@ DP_API int dp_refresh_stats(const float* fresh_local, float* stale_local, float*
 typedef struct dp_block_desc {
   int kind;       /* DP_BLOCK_*                                   */
   int H, W;       /* image rows and columns                       */
-  int C, Cout;    /* input / output channels (ATTN: Cout == C)    */
+  int C, Cout;    /* input / output channels (ATTN: Cout == C;    */
+                  /* UNET_MINI: C = latent channels, Cout = 1280) */
   int G, P;       /* GroupNorm groups, bands                      */
   int heads;      /* ATTN: heads (head_dim 64)                    */
   int dtype;      /* DP_BF16 or DP_FP32 (FP32: GN_CONV only)      */
@@ -289,6 +292,16 @@ DP_API int dp_block_state_init(const dp_block_desc* d, dp_block_state* s, void* 
  *             conv2_b[Cout], then if C != Cout: short_w[Cout][C], short_b[Cout]
  *   ATTN:     gn_gamma[C], gn_beta[C], wqkv[3C][C] (the q, k and v (out, in)
  *             matrices stacked), bqkv[3C], wo[C][C], bo[C]
+ *   UNET_MINI (latent [H][W][C], C even <= 16, H % 4P == 0, W % 4 == 0; output
+ *             [H/4][W/4][1280]): conv_in_w[320][3][3][C], conv_in_b[320], the
+ *             RESBLOCK list for 320->320 at HxW, down1_w[320][3][3][320],
+ *             down1_b[320], the RESBLOCK list for 320->640 at H/2 x W/2, the ATTN
+ *             list for 640 (10 heads), down2_w[640][3][3][640], down2_b[640], the
+ *             RESBLOCK list for 640->1280 at H/4 x W/4, the ATTN list for 1280
+ *             (20 heads) -- dp_block_weight_count() pointers in all.  Every 3x3
+ *             conv of the chain (conv_in and the two stride-2 downsamplers
+ *             included) takes its halo rows from the previous step's copy of its
+ *             own input.
  *  Weight matrices are `dtype`; gamma, beta and biases fp32 (biases may be NULL).
  * Returns DP_ERR_STATE for DISPLACED before any completed step.
  */
@@ -315,6 +328,9 @@ DP_API int dp_block_launch_count(const dp_block_desc* d);
 DP_API int dp_block_step_timed(const dp_block_desc* d, dp_block_state* s, const void* x, void* out,
                                const void* const* weights, int n_weights, int mode, void* stream,
                                void* const* events, int n_events);
+
+/* Number of weight pointers dp_block_step expects for this descriptor. */
+DP_API int dp_block_weight_count(const dp_block_desc* d);
 
 /* Algorithmic FLOPs of one block step (multiply-adds count 2). */
 DP_API double dp_block_flops(const dp_block_desc* d);

@@ -6,10 +6,16 @@ statistics (fp32) within 1e-4 absolute.
 
 Storing a value y in bf16 alone moves it by up to half an ulp, <= 2^-8 |y|,
 which exceeds 2e-2 once |y| >= 8.  Unit cases whose outputs reach that range
-(random affine parameters, channel-changing shortcuts) therefore use the
-storage-aware bound |gpu - ref| <= 2e-2 + 2^-8 |ref| per element
-(``storage_rel=BF16_HALF_ULP``); the five workloads' own chains keep the
-plain 2e-2 bound.
+(random affine parameters, channel-changing shortcuts, the mini U-Net chain
+whose outputs reach |y| ~ 40) therefore use the storage-aware bound
+|gpu - ref| <= 2e-2 + 2^-8 |ref| per element (``storage_rel=BF16_HALF_ULP``);
+the other four workloads' own chains keep the plain 2e-2 bound.
+
+Blocks with a channel-changing shortcut add a bf16-stored shortcut tensor
+whose elements can be larger than the output element they feed; a one-ulp
+storage flip there is bounded by 2^-7 * max|ref| rather than by the output
+element (``scale_rel``).  The 8-stage mini U-Net chain is held end to end to
+a bound derived from its depth (see tests/test_gpu_blocks.py).
 """
 import numpy as np
 import torch
@@ -58,7 +64,10 @@ def conv_w_dev(w_oihw: np.ndarray, dtype: str) -> torch.Tensor:
     return t.to(tdtype(dtype)).cuda()
 
 
-def check(gpu: np.ndarray, ref: np.ndarray, atol=ATOL, rl2=RL2, what="", storage_rel=0.0):
+def check(gpu: np.ndarray, ref: np.ndarray, atol=ATOL, rl2=RL2, what="", storage_rel=0.0,
+          scale_rel=0.0):
+    """max |gpu - ref| <= atol + storage_rel*|ref| + scale_rel*max|ref| per element, and
+    ||gpu - ref|| / ||ref|| <= rl2."""
     gpu = np.asarray(gpu, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     assert gpu.shape == ref.shape, (what, gpu.shape, ref.shape)
@@ -67,11 +76,13 @@ def check(gpu: np.ndarray, ref: np.ndarray, atol=ATOL, rl2=RL2, what="", storage
     maxabs = float(diff.max()) if diff.size else 0.0
     nref = float(np.linalg.norm(ref))
     rel = float(np.linalg.norm(gpu - ref) / nref) if nref > 0 else float(np.linalg.norm(gpu - ref))
-    excess = diff - (atol + storage_rel * np.abs(ref))
+    top = float(np.abs(ref).max()) if ref.size else 0.0
+    excess = diff - (atol + storage_rel * np.abs(ref) + scale_rel * top)
     if diff.size and excess.max() > 0:
         i = np.unravel_index(int(np.argmax(excess)), diff.shape)
         raise AssertionError(f"{what}: |diff| {diff[i]:.3e} at {i} (ref {ref[i]:.4f}, gpu {gpu[i]:.4f}) "
-                             f"exceeds {atol:.1e} + {storage_rel:.2e}*|ref|; max-abs {maxabs:.3e}, "
+                             f"exceeds {atol:.1e} + {storage_rel:.2e}*|ref| + {scale_rel:.2e}*{top:.2f}; "
+                             f"max-abs {maxabs:.3e}, "
                              f"rel-L2 {rel:.2e}")
     assert rel <= rl2, f"{what}: rel-L2 {rel:.3e} > {rl2:.1e} (max-abs {maxabs:.2e})"
     return maxabs, rel

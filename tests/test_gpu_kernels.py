@@ -105,6 +105,10 @@ CONV_CASES = [
     (320, 320, 16, 24, 4, 1, "bf16", True),
     (64, 64, 16, 16, 2, 2, "bf16", False),
     (128, 64, 24, 36, 3, 2, "bf16", True),
+    (320, 320, 12, 20, 3, 1, "bf16", True),     # pair kernel, ragged width
+    (64, 320, 24, 16, 4, 1, "bf16", False),     # pair kernel, odd tile count
+    (64, 320, 16, 16, 2, 2, "bf16", True),      # pair kernel, stride 2
+    (320, 640, 8, 136, 2, 1, "bf16", True),     # pair kernel, 128-pixel rows, ragged
     (64, 64, 16, 16, 2, 1, "fp32", False),
     (64, 128, 8, 10, 2, 1, "fp32", True),
 ]
@@ -152,7 +156,9 @@ def test_conv_small_parity():
 # ---------------------------------------------------------------- linear
 @pytest.mark.parametrize("M,N,K,split,use_res", [(300, 192, 128, 192, True), (256, 384, 128, 128, False),
                                                  (4096, 1920, 640, 640, False),
-                                                 (1000, 640, 320, 640, True)])
+                                                 (1000, 640, 320, 640, True),
+                                                 (384, 960, 128, 320, False),
+                                                 (130, 320, 64, 320, True)])
 def test_linear_parity(M, N, K, split, use_res):
     r = rng(M + N + K)
     x = rounded(r.standard_normal((M, K)), "bf16")
