@@ -130,45 +130,17 @@ def block_kind(B, wl):
             "unet_mini": B.UNET_MINI}[wl.kind]
 
 
-def launch_work(kind, H, W, C, Cout, e=2):
-    """(role, algorithmic flops, algorithmic bytes) of every launch of one block
-    step, in dp_block_launch_count order."""
-    hw = H * W
-    conv = lambda h, w, ci, co, s=1: ("conv", 2.0 * (h // s) * (w // s) * co * 9 * ci,
-                                      (h * w * ci * 2 + (h // s) * (w // s) * co) * e)
-    gn = lambda h, w, c: [("gn_stats", 0.0, h * w * c * e), ("gn_apply", 0.0, 2 * h * w * c * e)]
-    if kind == "gn_conv":
-        return gn(H, W, C) + [conv(H, W, C, Cout)]
-    if kind == "resblock":
-        out = gn(H, W, C) + [conv(H, W, C, Cout)] + gn(H, W, Cout)
-        if C != Cout:
-            out.append(("linear", 2.0 * hw * Cout * C, hw * (C + Cout) * e))
-        return out + [conv(H, W, Cout, Cout)]
-    if kind == "attn":
-        return gn(H, W, C) + [("linear", 2.0 * hw * 3 * C * C, hw * 4 * C * e),
-                              ("attn", 4.0 * hw * hw * C, hw * 4 * C * e),
-                              ("linear", 2.0 * hw * C * C, hw * 3 * C * e)]
-    # unet_mini
-    out = [("copy", 0.0, 2 * hw * C * e), ("conv_small", 2.0 * hw * 320 * 9 * C, hw * (C + 320) * e)]
-    out += launch_work("resblock", H, W, 320, 320, e)
-    out.append(conv(H, W, 320, 320, 2))
-    out += launch_work("resblock", H // 2, W // 2, 320, 640, e)
-    out += launch_work("attn", H // 2, W // 2, 640, 640, e)
-    out.append(conv(H // 2, W // 2, 640, 640, 2))
-    out += launch_work("resblock", H // 4, W // 4, 640, 1280, e)
-    out += launch_work("attn", H // 4, W // 4, 1280, 1280, e)
-    return out
+def block_desc(B, wl, H=None):
+    return B.dp_block_desc_init(block_kind(B, wl), H or wl.H, wl.W, wl.C, wl.cout, wl.G, wl.P,
+                                wl.heads, B.BF16 if wl.dtype == "bf16" else B.FP32, wl.silu,
+                                wl.eps, 1.0)
 
 
-def launch_roles(wl):
-    """Kernel role of each launch of one block step (dp_block_launch_count order)."""
-    return [r for r, _, _ in launch_work(wl.kind, wl.H, wl.W, wl.C, wl.cout)]
-
-
-def algorithmic_work(wl):
-    """Per-launch algorithmic work of every launch: (flops, bytes)."""
-    e = 2 if wl.dtype == "bf16" else 4
-    return [(f, b) for _, f, b in launch_work(wl.kind, wl.H, wl.W, wl.C, wl.cout, e)]
+def launch_plan(B, wl, mode):
+    """(kernel, algorithmic flops, algorithmic bytes) of every launch of one block step,
+    as the library reports them from the step's own code path."""
+    d = block_desc(B, wl)
+    return [B.dp_block_launch_info(d, mode, i) for i in range(B.dp_block_launch_count(d))]
 
 
 def cpu_baseline_ours(wl, seconds):
@@ -192,8 +164,9 @@ def cpu_baseline_ours(wl, seconds):
     return reps, el
 
 
-def wl_flops(wl):
-    return sum(f for _, f, _ in launch_work(wl.kind, wl.H, wl.W, wl.C, wl.cout))
+def wl_flops(wl, H=None):
+    from displaced_patch_parallelism_b200 import binding as B
+    return B.dp_block_flops(block_desc(B, wl, H))
 
 
 def run_reference(args, wl):
@@ -238,7 +211,7 @@ def run_reference(args, wl):
         O.block_step(w.kind, st, x, wts, w.P, w.G, w.eps, 1.0, synth.DISPLACED, w.dtype,
                      heads=w.heads, silu=w.silu)
     el = time.perf_counter() - t0
-    flops = wl_flops(w)
+    flops = wl_flops(wl, w.H)
     value = flops * args.steps / el / 1e12
     sample = (f"displaced step of the {wl.name} block on a {w.C}x{w.H}x{w.W} row crop "
               f"({rows} rows per band, {flops / 1e9:.2f} GFLOP per step)")
@@ -285,8 +258,9 @@ def run_ours(args, wl):
     host_out = torch.empty(out.shape, dtype=tdt).pin_memory()
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     n_launch = blk.launches
-    roles = launch_roles(wl)
-    assert len(roles) == n_launch
+    plan = launch_plan(B, wl, B.DISPLACED)
+    assert len(plan) == n_launch
+    roles = [r for r, _, _ in plan]
 
     warm = max(args.warmup, wl.warmup + 1)
     for i in range(warm):
@@ -351,7 +325,7 @@ def run_ours(args, wl):
     e2e_value = ws * flops * args.steps / (e2e_ms * 1e-3) / 1e12
 
     # per-kernel roles: mean duration, share, roofline of the dominant one
-    work = algorithmic_work(wl)
+    work = [(f, b) for _, f, b in plan]
     peaks = load_peaks()
     role_ms, role_n = {}, {}
     for k in range(args.steps):
@@ -371,8 +345,8 @@ def run_ours(args, wl):
     dominant = max(role_ms, key=lambda r: role_ms[r])
     dk = kernels[dominant]
     src = {"conv": ["dp_gemm.cu"], "linear": ["dp_gemm.cu"], "attn": ["dp_attn.cu"],
-           "gn_stats": ["dp_gn.cu"], "gn_apply": ["dp_gn.cu"], "copy": ["dp_refresh.cu"],
-           "conv_small": ["dp_conv_small.cu"]}[dominant]
+           "gn_stats": ["dp_gn.cu"], "gn_apply": ["dp_gn.cu"], "gn_fused": ["dp_gn.cu"],
+           "copy": ["dp_refresh.cu"], "conv_small": ["dp_conv_small.cu"]}[dominant]
     traffic = load_traffic(f"{dominant}:{wl.name}", kernel_source_hash(src))
     if dk["tflops"]:
         roof = {"bound": "tensor", "achieved": dk["tflops"], "peak": peaks["bf16_tflops"],
@@ -385,10 +359,11 @@ def run_ours(args, wl):
         roof = {"bound": "hbm", "achieved": dk["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(dk["gbs"] / peaks["hbm_gbs"], 4), "traffic": traffic,
                 "kernel": dominant, "peak_source": f"{peaks['source']} copy"}
-    gn_ms = role_ms.get("gn_stats", 0.0) + role_ms.get("gn_apply", 0.0)
+    gn_ms = sum(v for r, v in role_ms.items() if r.startswith("gn"))
     gn_bytes = sum(work[i][1] for i, r in enumerate(roles) if r.startswith("gn")) * args.steps
     gn = {"achieved_gbs": round(gn_bytes / (gn_ms * 1e-3) / 1e9, 1) if gn_ms else None,
-          "peak": peaks["hbm_gbs"], "bytes_model": "stats: read x; apply: read x + write y"}
+          "peak": peaks["hbm_gbs"],
+          "bytes_model": "single pass: read x + write y; two passes: stats read x, apply read x + write y"}
     if gn["achieved_gbs"]:
         gn["frac"] = round(gn["achieved_gbs"] / peaks["hbm_gbs"], 4)
 

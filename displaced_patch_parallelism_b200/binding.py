@@ -68,6 +68,8 @@ _SIGS = {
     "dp_block_flops": ([ctypes.POINTER(BlockDesc)], ctypes.c_double),
     "dp_block_launch_count": ([ctypes.POINTER(BlockDesc)], _I),
     "dp_block_weight_count": ([ctypes.POINTER(BlockDesc)], _I),
+    "dp_block_launch_info": ([ctypes.POINTER(BlockDesc), _I, _I, ctypes.POINTER(_I),
+                              ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)], _I),
     "dp_block_step_timed": ([ctypes.POINTER(BlockDesc), ctypes.POINTER(BlockState), _V, _V,
                              ctypes.POINTER(_V), _I, _I, _V, ctypes.POINTER(_V), _I], _I),
 }
@@ -237,6 +239,18 @@ def dp_block_step_timed(d: BlockDesc, s: BlockState, x, out, weights: Sequence, 
     ev = (ctypes.c_void_p * len(events))(*handles)
     return _check(lib().dp_block_step_timed(ctypes.byref(d), ctypes.byref(s), _p(x), _p(out), arr,
                                             len(weights), mode, _s(stream), ev, len(events)))
+
+
+KERNEL_NAMES = {0: "gn_stats", 1: "gn_apply", 2: "gn_fused", 3: "conv", 4: "linear", 5: "attn",
+                6: "copy", 7: "conv_small"}
+
+
+def dp_block_launch_info(d: BlockDesc, mode: int, i: int):
+    """(kernel name, algorithmic flops, algorithmic bytes) of launch i."""
+    k, f, b = ctypes.c_int(0), ctypes.c_double(0), ctypes.c_double(0)
+    _check(lib().dp_block_launch_info(ctypes.byref(d), mode, i, ctypes.byref(k), ctypes.byref(f),
+                                      ctypes.byref(b)))
+    return KERNEL_NAMES[k.value], f.value, b.value
 
 
 def dp_block_weight_count(d: BlockDesc) -> int:

@@ -8,7 +8,7 @@
 // DistriFusion).  Sync steps use fresh keys everywhere; naive steps see only
 // the band's own keys.
 //
-// B200 design (one CTA = 128 queries of one head, 192 threads, 2 CTAs/SM):
+// B200 design (one CTA = 128 queries of one head, 320 threads, 2 CTAs/SM):
 //   warp 0     TMA producer: Q once, then K/V tiles of 128 keys through a
 //              2-deep ring; each tile is taken whole from the fresh or the
 //              stale buffer (bands are multiples of 128 tokens);
@@ -16,10 +16,11 @@
 //              O += P V (128x64x128) with P read straight from tensor memory;
 //              S of tile j+1 is issued before O += P_j V_j so the tensor core
 //              works while the softmax warps exponentiate;
-//   warps 2-5  softmax: one query row per thread; S row -> registers, online
-//              max with lazy rescaling (O is only rescaled when the running
-//              maximum grows by more than 2^8), exp2, packed bf16 P back to
-//              tensor memory; final O / l, bf16 store.
+//   warps 2-9  softmax: two warps per 32 query rows, one half-row (64
+//              scores) per thread; S -> registers, online max with lazy
+//              rescaling (O is only rescaled when the running maximum grows by
+//              more than 2^8), exp2 (part on the FMA pipe), packed bf16 P back
+//              to tensor memory; final O / l, bf16 store.
 // Tensor memory per CTA (256 columns): S [0,128), P [128,192) as bf16 pairs,
 // O [192,256).
 #include <cstring>
@@ -40,12 +41,66 @@ struct AttnParams {
 
 constexpr int kAttnStages = 2;
 constexpr int kTile = 16384;                     // 128 rows x 128 bytes
-constexpr int kAttnSmem = kTile * (1 + 2 * kAttnStages) + 1024 + 256;
+constexpr int kAttnThreads = 320;               // producer, MMA, 8 softmax warps
+constexpr int kAttnTail = 4096;                  // barriers + max/sum exchange buffers
+constexpr int kAttnSmem = kTile * (1 + 2 * kAttnStages) + 1024 + kAttnTail;
 
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// ---- packed fp32x2 arithmetic (two lanes of work per FMA-pipe instruction)
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x for two values on the FMA pipe, so that part of the softmax's
+// exponentials leave the special-function unit (the bottleneck of this kernel
+// at head_dim 64).  Method: round-to-nearest range reduction x = n + f,
+// f in [-1/2, 1/2], by adding 1.5 * 2^23 (the sum's low mantissa bits hold n);
+// 2^f by a cubic fitted here for minimax relative error on [-1/2, 1/2]
+// (Remez exchange; max relative error 7.5e-5, far below the 2^-9 of the bf16
+// that P is rounded to); 2^n by adding n to the exponent field.  Inputs are
+// clamped at -125 so the result stays a normal number.
+__device__ __forceinline__ void exp2_poly_x2(uint64_t x2, float& e0, float& e1) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  float x0, x1;
+  f2_unpack(x2, x0, x1);
+  x2 = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t t2 = f2_add(x2, f2_pack(kMagic, kMagic));
+  const uint64_t n2 = f2_add(t2, f2_pack(-kMagic, -kMagic));
+  const uint64_t f2 = f2_fma(n2, f2_pack(-1.f, -1.f), x2);
+  uint64_t p2 = f2_fma(f2_pack(0.05517166905792616f, 0.05517166905792616f), f2,
+                       f2_pack(0.2426111221932161f, 0.2426111221932161f));
+  p2 = f2_fma(p2, f2, f2_pack(0.6932609854606553f, 0.6932609854606553f));
+  p2 = f2_fma(p2, f2, f2_pack(0.9999280735394012f, 0.9999280735394012f));
+  float t0, t1, p0, p1;
+  f2_unpack(t2, t0, t1);
+  f2_unpack(p2, p0, p1);
+  e0 = __int_as_float(__float_as_int(p0) + ((__float_as_int(t0) - 0x4B400000) << 23));
+  e1 = __int_as_float(__float_as_int(p1) + ((__float_as_int(t1) - 0x4B400000) << 23));
 }
 
 __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
@@ -65,7 +120,7 @@ __device__ __forceinline__ void attn_wait_teardown(uint64_t* bar, uint32_t parit
   }
 }
 
-__global__ void __launch_bounds__(192, 2) attn_kernel(const __grid_constant__ AttnParams p) {
+__global__ void __launch_bounds__(kAttnThreads, 2) attn_kernel(const __grid_constant__ AttnParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -81,8 +136,10 @@ __global__ void __launch_bounds__(192, 2) attn_kernel(const __grid_constant__ At
   uint64_t* p_full = s_free + 1;
   uint64_t* o_done = p_full + 1;
   uint64_t* drain = o_done + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* xbar = drain + 1;                                   // [4], one per row quarter
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xbar + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* red = reinterpret_cast<float*>(bars + 64);             // [2 parities][2 halves][128]
 
   const int warp = warp_id(), lane = lane_id();
   const int qtile = blockIdx.x, h = blockIdx.y;
@@ -99,8 +156,9 @@ __global__ void __launch_bounds__(192, 2) attn_kernel(const __grid_constant__ At
       mbar_init(&kv_empty[s], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(s_free, 4);
-    mbar_init(p_full, 4);
+    mbar_init(s_free, 8);
+    mbar_init(p_full, 8);
+    for (int i = 0; i < 4; ++i) mbar_init(&xbar[i], 2);
     mbar_init(o_done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -192,30 +250,52 @@ __global__ void __launch_bounds__(192, 2) attn_kernel(const __grid_constant__ At
     }
   } else {
     // -------------------------------------------------------------- softmax
+    // Warps w and w+4 share TMEM lanes 32*(w%4).. (the same 32 query rows)
+    // and split each row's 128 scores into halves, so 8 warps exponentiate.
+    // Per tile they exchange their half-row maxima through shared memory
+    // (double-buffered by tile parity, bounded mbarrier waits); each half
+    // keeps its own partial row sum and owns 32 of the 64 output columns.
     const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int row = q * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     const float c = p.scale_log2;
     float m_used = 0.f, l = 0.f;
     bool aborted = false;
+    auto exchange = [&](int use, float mine, float* other) -> bool {
+      float* buf = red + (use & 1) * 256;
+      buf[half * 128 + row] = mine;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&xbar[q]);
+      if (!mbar_wait(&xbar[q], use & 1, abort_flag, p.status)) return false;
+      *other = buf[(half ^ 1) * 128 + row];
+      return true;
+    };
     for (int j = 0; j < n_kv; ++j) {
       if (!mbar_wait(s_full, j & 1, abort_flag, p.status)) {
         aborted = true;
         break;
       }
       tc_fence_after();
-      uint32_t s[4][32];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) tmem_ld32(tS + lane_off + 32 * k, s[k]);
+      uint32_t s[2][32];
+      tmem_ld32(tS + lane_off + half * 64, s[0]);
+      tmem_ld32(tS + lane_off + half * 64 + 32, s[1]);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(s_free);
       float mx = __uint_as_float(s[0][0]);
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
+      for (int k = 0; k < 2; ++k)
 #pragma unroll
-        for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(s[k][i]));
-      const float m_tile = mx * c;
+        for (int i = 0; i < 32; i += 2)
+          mx = max3(mx, __uint_as_float(s[k][i]), __uint_as_float(s[k][i + 1]));
+      float mo;
+      if (!exchange(j, mx, &mo)) {
+        aborted = true;
+        break;
+      }
+      const float m_tile = fmaxf(mx, mo) * c;
       float alpha = 1.f;
       if (j == 0) {
         m_used = m_tile;
@@ -223,19 +303,32 @@ __global__ void __launch_bounds__(192, 2) attn_kernel(const __grid_constant__ At
         alpha = ex2_approx(m_used - m_tile);
         m_used = m_tile;
       }
-      // P_j = exp2(s * c - m_used), packed bf16 pairs
-      uint32_t pk[2][32];
-      float rs = 0.f;
+      // P_j = exp2(s * c - m_used), packed bf16 pairs.  3 of every 8 pairs take
+      // the FMA-pipe exponential, the rest the special-function unit.
+      uint32_t pk[32];
+      const uint64_t c2 = f2_pack(c, c), negm2 = f2_pack(-m_used, -m_used);
+      uint64_t sum2 = f2_pack(0.f, 0.f);
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
+      for (int k = 0; k < 2; ++k)
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float e0 = ex2_approx(fmaf(__uint_as_float(s[k][2 * i]), c, -m_used));
-          const float e1 = ex2_approx(fmaf(__uint_as_float(s[k][2 * i + 1]), c, -m_used));
-          rs += e0 + e1;
-          pk[k >> 1][(k & 1) * 16 + i] = pack_bf16x2(e0, e1);
+          const uint64_t x2 =
+              f2_fma(f2_pack(__uint_as_float(s[k][2 * i]), __uint_as_float(s[k][2 * i + 1])), c2, negm2);
+          float e0, e1;
+          if ((i & 7) < 3) {
+            exp2_poly_x2(x2, e0, e1);
+          } else {
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            e0 = ex2_approx(x0);
+            e1 = ex2_approx(x1);
+          }
+          sum2 = f2_add(sum2, f2_pack(e0, e1));
+          pk[k * 16 + i] = pack_bf16x2(e0, e1);
         }
-      l = l * alpha + rs;
+      float rs0, rs1;
+      f2_unpack(sum2, rs0, rs1);
+      l = l * alpha + (rs0 + rs1);
       if (j > 0) {
         // P_{j-1} V_{j-1} must be done before O is rescaled or P overwritten
         if (!mbar_wait(o_done, (j - 1) & 1, abort_flag, p.status)) {
@@ -244,45 +337,39 @@ __global__ void __launch_bounds__(192, 2) attn_kernel(const __grid_constant__ At
         }
         tc_fence_after();
         if (__any_sync(0xffffffffu, alpha != 1.f)) {
-          uint32_t o[2][32];
-          tmem_ld32(tO + lane_off, o[0]);
-          tmem_ld32(tO + lane_off + 32, o[1]);
+          uint32_t o[32];
+          tmem_ld32(tO + lane_off + half * 32, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int k = 0; k < 2; ++k)
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[k][i] = __float_as_uint(__uint_as_float(o[k][i]) * alpha);
-          tmem_st32(tO + lane_off, o[0]);
-          tmem_st32(tO + lane_off + 32, o[1]);
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tO + lane_off + half * 32, o);
         }
       }
-      tmem_st32(tP + lane_off, pk[0]);
-      tmem_st32(tP + lane_off + 32, pk[1]);
+      tmem_st32(tP + lane_off + half * 32, pk);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
     }
-    if (!aborted && n_kv > 0 && mbar_wait(o_done, (n_kv - 1) & 1, abort_flag, p.status)) {
+    float lo = 0.f;
+    if (!aborted && n_kv > 0 && exchange(n_kv, l, &lo) &&
+        mbar_wait(o_done, (n_kv - 1) & 1, abort_flag, p.status)) {
       tc_fence_after();
-      uint32_t o[2][32];
-      tmem_ld32(tO + lane_off, o[0]);
-      tmem_ld32(tO + lane_off + 32, o[1]);
+      uint32_t o[32];
+      tmem_ld32(tO + lane_off + half * 32, o);
       tmem_wait_ld();
-      const float inv = 1.f / l;
-      const int row = q0 + q * 32 + lane;
-      uint4* dst = reinterpret_cast<uint4*>(p.o + static_cast<size_t>(row) * p.ld + h * 64);
+      const float inv = 1.f / (l + lo);
+      uint4* dst = reinterpret_cast<uint4*>(p.o + static_cast<size_t>(q0 + row) * p.ld + h * 64 +
+                                            half * 32);
 #pragma unroll
-      for (int k = 0; k < 2; ++k)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          uint4 u;
-          u.x = pack_bf16x2(__uint_as_float(o[k][8 * i]) * inv, __uint_as_float(o[k][8 * i + 1]) * inv);
-          u.y = pack_bf16x2(__uint_as_float(o[k][8 * i + 2]) * inv, __uint_as_float(o[k][8 * i + 3]) * inv);
-          u.z = pack_bf16x2(__uint_as_float(o[k][8 * i + 4]) * inv, __uint_as_float(o[k][8 * i + 5]) * inv);
-          u.w = pack_bf16x2(__uint_as_float(o[k][8 * i + 6]) * inv, __uint_as_float(o[k][8 * i + 7]) * inv);
-          dst[k * 4 + i] = u;
-        }
+      for (int i = 0; i < 4; ++i) {
+        uint4 u;
+        u.x = pack_bf16x2(__uint_as_float(o[8 * i]) * inv, __uint_as_float(o[8 * i + 1]) * inv);
+        u.y = pack_bf16x2(__uint_as_float(o[8 * i + 2]) * inv, __uint_as_float(o[8 * i + 3]) * inv);
+        u.z = pack_bf16x2(__uint_as_float(o[8 * i + 4]) * inv, __uint_as_float(o[8 * i + 5]) * inv);
+        u.w = pack_bf16x2(__uint_as_float(o[8 * i + 6]) * inv, __uint_as_float(o[8 * i + 7]) * inv);
+        dst[i] = u;
+      }
     }
   }
 
@@ -331,7 +418,7 @@ int attn_launch(const void* q, const void* kf, const void* vf, const void* ks, c
   }
   dim3 grid(T / 128, heads);
   mark_launch(stream);
-  attn_kernel<<<grid, 192, kAttnSmem, stream>>>(a);
+  attn_kernel<<<grid, kAttnThreads, kAttnSmem, stream>>>(a);
   return cuda_check(cudaGetLastError(), "attention launch");
 }
 

@@ -174,16 +174,6 @@ int desc_check(const dp_block_desc* d) {
   return DP_OK;
 }
 
-int launch_count(const dp_block_desc* d) {
-  if (d->kind == DP_BLOCK_GN_CONV) return 3;
-  if (d->kind == DP_BLOCK_RESBLOCK) return d->C != d->Cout ? 7 : 6;
-  if (d->kind == DP_BLOCK_ATTN) return 5;
-  const MiniDescs m = mini_descs(d);
-  // input copy + conv_in + rb1 + down1 + rb2 + at2 + down2 + rb3 + at3
-  return 2 + launch_count(&m.rb1) + 1 + launch_count(&m.rb2) + launch_count(&m.at2) + 1 +
-         launch_count(&m.rb3) + launch_count(&m.at3);
-}
-
 int weight_count(const dp_block_desc* d) {
   if (d->kind == DP_BLOCK_GN_CONV) return 4;
   if (d->kind == DP_BLOCK_RESBLOCK) return d->C != d->Cout ? 10 : 8;
@@ -212,22 +202,73 @@ T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
 }
 
+// When a step runs in planning mode it records every launch it would make
+// (kernel kind, algorithmic flops, algorithmic bytes) instead of launching;
+// the launch count and per-launch work reported by the ABI come from here,
+// so they follow the step's own code path.
+struct LaunchRec {
+  int kind;
+  double flops, bytes;
+};
+struct Plan {
+  LaunchRec rec[128];
+  int n = 0;
+  void push(int kind, double flops, double bytes) {
+    if (n < 128) rec[n] = {kind, flops, bytes};
+    ++n;
+  }
+};
+
 // One step of the block described by `d` whose state lives at `ws`; `cur`
 // selects the stale half of every ping-pong pair (the fresh half is cur ^ 1).
 int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* out,
-              const void* const* w, int mode, cudaStream_t st) {
+              const void* const* w, int mode, cudaStream_t st, Plan* plan) {
   const Layout L = layout_of(d);
+  const double e = d->dtype == DP_FP32 ? 4.0 : 2.0;
   const int f = cur ^ 1, o = cur;
   const int H = d->H, W = d->W, C = d->C, Co = d->Cout, G = d->G, P = d->P;
   auto gn = [&](const GnSlots& g, const void* in, void* y, const void* gamma, const void* beta,
                 int ch, int silu) {
+    if (plan) {
+      const double bytes = static_cast<double>(H) * W * ch * e;
+      int nb, chunk, th;
+      size_t sm;
+      if (gn_fused_plan(H, W, ch, G, P, d->dtype, &nb, &chunk, &th, &sm)) {
+        plan->push(DP_KERNEL_GN_FUSED, 0.0, 2.0 * bytes);
+      } else {
+        plan->push(DP_KERNEL_GN_STATS, 0.0, bytes);
+        plan->push(DP_KERNEL_GN_APPLY, 0.0, 2.0 * bytes);
+      }
+      return DP_OK;
+    }
     return gn_launch(in, y, static_cast<const float*>(gamma), static_cast<const float*>(beta), H,
                      W, ch, G, P, d->eps, d->w, silu, mode, d->dtype, at<float>(ws, g.global[o]),
                      at<float>(ws, g.local[o]), at<float>(ws, g.local[f]),
                      at<float>(ws, g.global[f]), at<float>(ws, g.used), at<void>(ws, g.ws), st);
   };
+  // conv / linear / attention launches, or their records in planning mode
+  auto conv = [&](const void* af, const void* as, const void* wt, const void* b, const void* res,
+                  void* y, int h, int wd, int ci, int co, int stride) {
+    if (plan) {
+      const double ho = (h - 1) / stride + 1, wo = (wd - 1) / stride + 1;
+      plan->push(DP_KERNEL_CONV, 2.0 * ho * wo * co * 9.0 * ci,
+                 (static_cast<double>(h) * wd * ci + ho * wo * co * (res ? 2 : 1)) * e);
+      return DP_OK;
+    }
+    return conv3x3_launch(af, as, wt, static_cast<const float*>(b), res, y, h, wd, ci, co, stride, P,
+                          mode, d->dtype, st);
+  };
+  auto lin = [&](const void* in, const void* wt, const void* b, const void* res, void* o0, void* o1,
+                 void* o2, int M, int N, int K, int split) {
+    if (plan) {
+      plan->push(DP_KERNEL_LINEAR, 2.0 * M * N * static_cast<double>(K),
+                 (static_cast<double>(M) * K + static_cast<double>(M) * N * (res ? 2 : 1)) * e);
+      return DP_OK;
+    }
+    return linear_launch(in, wt, static_cast<const float*>(b), res, o0, o1, o2, M, N, K, split, st);
+  };
   int rc;
-  if (d->kind != DP_BLOCK_UNET_MINI) {
+  if (d->kind != DP_BLOCK_UNET_MINI && !plan) {
     // biases (conv_b, conv1_b, conv2_b, short_b; bqkv, bo) may be NULL
     for (int i = 0; i < weight_count(d); ++i) {
       const bool bias = d->kind == DP_BLOCK_ATTN ? (i == 3 || i == 5)
@@ -236,39 +277,39 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
     }
   }
   if (d->kind == DP_BLOCK_GN_CONV) {
-    rc = conv3x3_validate(x, x, w[2], nullptr, out, H, W, C, Co, 1, P, mode, d->dtype);
-    if (rc) return rc;
+    if (!plan) {
+      rc = conv3x3_validate(x, x, w[2], nullptr, out, H, W, C, Co, 1, P, mode, d->dtype);
+      if (rc) return rc;
+    }
     rc = gn(L.gn1, x, at<void>(ws, L.a1[f]), w[0], w[1], C, d->silu);
     if (rc) return rc;
-    return conv3x3_launch(at<void>(ws, L.a1[f]), at<void>(ws, L.a1[o]), w[2],
-                          static_cast<const float*>(w[3]), nullptr, out, H, W, C, Co, 1, P, mode,
-                          d->dtype, st);
+    return conv(at<void>(ws, L.a1[f]), at<void>(ws, L.a1[o]), w[2], w[3], nullptr, out, H, W, C, Co,
+                1);
   }
   if (d->kind == DP_BLOCK_RESBLOCK) {
-    rc = conv3x3_validate(x, x, w[2], nullptr, out, H, W, C, Co, 1, P, mode, d->dtype);
-    if (rc) return rc;
-    rc = conv3x3_validate(x, x, w[6], nullptr, out, H, W, Co, Co, 1, P, mode, d->dtype);
-    if (rc) return rc;
+    if (!plan) {
+      rc = conv3x3_validate(x, x, w[2], nullptr, out, H, W, C, Co, 1, P, mode, d->dtype);
+      if (rc) return rc;
+      rc = conv3x3_validate(x, x, w[6], nullptr, out, H, W, Co, Co, 1, P, mode, d->dtype);
+      if (rc) return rc;
+    }
     void* a1f = at<void>(ws, L.a1[f]);
     void* a2f = at<void>(ws, L.a2[f]);
     void* h = at<void>(ws, L.h);
     rc = gn(L.gn1, x, a1f, w[0], w[1], C, 1);
     if (rc) return rc;
-    rc = conv3x3_launch(a1f, at<void>(ws, L.a1[o]), w[2], static_cast<const float*>(w[3]), nullptr,
-                        h, H, W, C, Co, 1, P, mode, d->dtype, st);
+    rc = conv(a1f, at<void>(ws, L.a1[o]), w[2], w[3], nullptr, h, H, W, C, Co, 1);
     if (rc) return rc;
     rc = gn(L.gn2, h, a2f, w[4], w[5], Co, 1);
     if (rc) return rc;
     const void* res = x;
     if (C != Co) {
       void* sc = at<void>(ws, L.sc);
-      rc = linear_launch(x, w[8], static_cast<const float*>(w[9]), nullptr, sc, nullptr, nullptr,
-                         H * W, Co, C, Co, st);
+      rc = lin(x, w[8], w[9], nullptr, sc, nullptr, nullptr, H * W, Co, C, Co);
       if (rc) return rc;
       res = sc;
     }
-    return conv3x3_launch(a2f, at<void>(ws, L.a2[o]), w[6], static_cast<const float*>(w[7]), res,
-                          out, H, W, Co, Co, 1, P, mode, d->dtype, st);
+    return conv(a2f, at<void>(ws, L.a2[o]), w[6], w[7], res, out, H, W, Co, Co, 1);
   }
   if (d->kind == DP_BLOCK_ATTN) {
     const int T = H * W;
@@ -279,14 +320,17 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
     void* ob = at<void>(ws, L.o);
     rc = gn(L.gn1, x, act, w[0], w[1], C, 0);
     if (rc) return rc;
-    rc = linear_launch(act, w[2], static_cast<const float*>(w[3]), nullptr, q, kf, vf, T, 3 * C, C,
-                       C, st);
+    rc = lin(act, w[2], w[3], nullptr, q, kf, vf, T, 3 * C, C, C);
     if (rc) return rc;
-    rc = attn_launch(q, kf, vf, at<void>(ws, L.k[o]), at<void>(ws, L.v[o]), ob, T, d->heads, P,
-                     0.125f, mode, st);
-    if (rc) return rc;
-    return linear_launch(ob, w[4], static_cast<const float*>(w[5]), x, out, nullptr, nullptr, T, C,
-                         C, C, st);
+    if (plan) {
+      const double keys = mode == DP_MODE_NAIVE ? static_cast<double>(T) / P : T;
+      plan->push(DP_KERNEL_ATTN, 4.0 * T * keys * C, 4.0 * T * C * e);
+    } else {
+      rc = attn_launch(q, kf, vf, at<void>(ws, L.k[o]), at<void>(ws, L.v[o]), ob, T, d->heads, P,
+                       0.125f, mode, st);
+      if (rc) return rc;
+    }
+    return lin(ob, w[4], w[5], x, out, nullptr, nullptr, T, C, C, C);
   }
   // UNET_MINI
   const MiniDescs m = mini_descs(d);
@@ -298,47 +342,64 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
     return p;
   };
   void* xin = at<void>(ws, L.xin[f]);
-  rc = copy_launch(x, xin, static_cast<size_t>(H) * W * C * 2, st);
-  if (rc) return rc;
+  const size_t xbytes = static_cast<size_t>(H) * W * C * 2;
+  if (plan) {
+    plan->push(DP_KERNEL_COPY, 0.0, 2.0 * xbytes);
+    plan->push(DP_KERNEL_CONV_SMALL, 2.0 * H * W * kU1 * 9.0 * C,
+               static_cast<double>(H) * W * (C + kU1) * 2.0);
+  } else {
+    rc = copy_launch(x, xin, xbytes, st);
+    if (rc) return rc;
+  }
   const void* const* wc = take(2);
-  if (!wc[0]) return set_error(DP_ERR_INVALID_ARG, "block: conv_in weight is NULL");
-  rc = conv3x3_small_launch(xin, at<void>(ws, L.xin[o]), wc[0], static_cast<const float*>(wc[1]),
-                            at<void>(ws, L.h0), H, W, C, kU1, P, mode, st);
-  if (rc) return rc;
+  if (!plan) {
+    if (!wc[0]) return set_error(DP_ERR_INVALID_ARG, "block: conv_in weight is NULL");
+    rc = conv3x3_small_launch(xin, at<void>(ws, L.xin[o]), wc[0], static_cast<const float*>(wc[1]),
+                              at<void>(ws, L.h0), H, W, C, kU1, P, mode, st);
+    if (rc) return rc;
+  }
   rc = step_impl(&m.rb1, at<void>(ws, L.rb1), cur, at<void>(ws, L.h0), at<void>(ws, L.d1[f]),
-                 take(weight_count(&m.rb1)), mode, st);
+                 take(weight_count(&m.rb1)), mode, st, plan);
   if (rc) return rc;
   wc = take(2);
-  if (!wc[0]) return set_error(DP_ERR_INVALID_ARG, "block: down1 weight is NULL");
-  rc = conv3x3_validate(at<void>(ws, L.d1[f]), at<void>(ws, L.d1[o]), wc[0], nullptr,
-                        at<void>(ws, L.h1), H, W, kU1, kU1, 2, P, mode, DP_BF16);
-  if (rc) return rc;
-  rc = conv3x3_launch(at<void>(ws, L.d1[f]), at<void>(ws, L.d1[o]), wc[0],
-                      static_cast<const float*>(wc[1]), nullptr, at<void>(ws, L.h1), H, W, kU1,
-                      kU1, 2, P, mode, DP_BF16, st);
+  if (!plan) {
+    if (!wc[0]) return set_error(DP_ERR_INVALID_ARG, "block: down1 weight is NULL");
+    rc = conv3x3_validate(at<void>(ws, L.d1[f]), at<void>(ws, L.d1[o]), wc[0], nullptr,
+                          at<void>(ws, L.h1), H, W, kU1, kU1, 2, P, mode, DP_BF16);
+    if (rc) return rc;
+  }
+  rc = conv(at<void>(ws, L.d1[f]), at<void>(ws, L.d1[o]), wc[0], wc[1], nullptr, at<void>(ws, L.h1),
+            H, W, kU1, kU1, 2);
   if (rc) return rc;
   rc = step_impl(&m.rb2, at<void>(ws, L.rb2), cur, at<void>(ws, L.h1), at<void>(ws, L.h2),
-                 take(weight_count(&m.rb2)), mode, st);
+                 take(weight_count(&m.rb2)), mode, st, plan);
   if (rc) return rc;
   rc = step_impl(&m.at2, at<void>(ws, L.at2), cur, at<void>(ws, L.h2), at<void>(ws, L.d2[f]),
-                 take(weight_count(&m.at2)), mode, st);
+                 take(weight_count(&m.at2)), mode, st, plan);
   if (rc) return rc;
   wc = take(2);
-  if (!wc[0]) return set_error(DP_ERR_INVALID_ARG, "block: down2 weight is NULL");
-  rc = conv3x3_validate(at<void>(ws, L.d2[f]), at<void>(ws, L.d2[o]), wc[0], nullptr,
-                        at<void>(ws, L.h3), H2, W2, kU2, kU2, 2, P, mode, DP_BF16);
-  if (rc) return rc;
-  rc = conv3x3_launch(at<void>(ws, L.d2[f]), at<void>(ws, L.d2[o]), wc[0],
-                      static_cast<const float*>(wc[1]), nullptr, at<void>(ws, L.h3), H2, W2, kU2,
-                      kU2, 2, P, mode, DP_BF16, st);
+  if (!plan) {
+    if (!wc[0]) return set_error(DP_ERR_INVALID_ARG, "block: down2 weight is NULL");
+    rc = conv3x3_validate(at<void>(ws, L.d2[f]), at<void>(ws, L.d2[o]), wc[0], nullptr,
+                          at<void>(ws, L.h3), H2, W2, kU2, kU2, 2, P, mode, DP_BF16);
+    if (rc) return rc;
+  }
+  rc = conv(at<void>(ws, L.d2[f]), at<void>(ws, L.d2[o]), wc[0], wc[1], nullptr, at<void>(ws, L.h3),
+            H2, W2, kU2, kU2, 2);
   if (rc) return rc;
   rc = step_impl(&m.rb3, at<void>(ws, L.rb3), cur, at<void>(ws, L.h3), at<void>(ws, L.h4),
-                 take(weight_count(&m.rb3)), mode, st);
+                 take(weight_count(&m.rb3)), mode, st, plan);
   if (rc) return rc;
   (void)H3;
   (void)W3;
   return step_impl(&m.at3, at<void>(ws, L.at3), cur, at<void>(ws, L.h4), out,
-                   take(weight_count(&m.at3)), mode, st);
+                   take(weight_count(&m.at3)), mode, st, plan);
+}
+
+// Records the launches of one step of `d` in `mode`.
+int plan_of(const dp_block_desc* d, int mode, Plan* plan) {
+  static const void* const null_w[128] = {nullptr};
+  return step_impl(d, nullptr, 0, nullptr, nullptr, null_w, mode, nullptr, plan);
 }
 
 }  // namespace
@@ -419,7 +480,7 @@ int dp_block_step(const dp_block_desc* d, dp_block_state* s, const void* x, void
   if (s->workspace_bytes < dp::layout_of(d).total)
     return dp::set_error(DP_ERR_INVALID_ARG, "block: workspace too small");
   rc = dp::step_impl(d, s->workspace, s->cur, x, out, weights, mode,
-                     static_cast<cudaStream_t>(stream));
+                     static_cast<cudaStream_t>(stream), nullptr);
   if (rc) return rc;
   s->cur ^= 1;
   s->steps_done += 1;
@@ -429,7 +490,27 @@ int dp_block_step(const dp_block_desc* d, dp_block_state* s, const void* x, void
 int dp_block_launch_count(const dp_block_desc* d) {
   int rc = dp::desc_check(d);
   if (rc) return rc;
-  return dp::launch_count(d);
+  dp::Plan plan;
+  rc = dp::plan_of(d, DP_MODE_DISPLACED, &plan);
+  if (rc) return rc;
+  return plan.n;
+}
+
+int dp_block_launch_info(const dp_block_desc* d, int mode, int i, int* kind, double* flops,
+                         double* bytes) {
+  int rc = dp::desc_check(d);
+  if (rc) return rc;
+  if (mode < DP_MODE_SYNC || mode > DP_MODE_NAIVE)
+    return dp::set_error(DP_ERR_INVALID_ARG, "block: bad mode %d", mode);
+  dp::Plan plan;
+  rc = dp::plan_of(d, mode, &plan);
+  if (rc) return rc;
+  if (i < 0 || i >= plan.n || i >= 128)
+    return dp::set_error(DP_ERR_INVALID_ARG, "block: launch %d of %d", i, plan.n);
+  if (kind) *kind = plan.rec[i].kind;
+  if (flops) *flops = plan.rec[i].flops;
+  if (bytes) *bytes = plan.rec[i].bytes;
+  return DP_OK;
 }
 
 int dp_block_step_timed(const dp_block_desc* d, dp_block_state* s, const void* x, void* out,

@@ -868,7 +868,10 @@ int linear_launch(const void* x, const void* weight, const float* bias, const vo
   p.out2 = out2;
   p.status = device_status_ptr();
   int bn_single = 0;
-  const int pw = pick_pair(p.m_tiles, N, split, &bn_single);
+  // Short K (few K blocks per tile) does not amortise a pair tile's pipeline
+  // fill and un-overlapped epilogue; such projections stay on single-CTA tiles.
+  const int pw = p.k_blocks >= 16 ? pick_pair(p.m_tiles, N, split, &bn_single) : 0;
+  if (!pw) bn_single = pick_bn(p.m_tiles, N, split, false);
   const bool pair = pw != 0;
   const int BN = pair ? pw : bn_single;
   if (!BN) return set_error(DP_ERR_UNSUPPORTED, "linear: no N tile divides split=%d", split);

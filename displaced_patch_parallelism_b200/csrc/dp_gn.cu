@@ -31,6 +31,10 @@
 namespace dp {
 
 constexpr int kGnMaxSplits = 64;   // blocks per band
+// Each (band, group) accumulator (sum, sum of squares) gets its own 128-byte
+// line so that the atomics of many blocks spread over L2 slices instead of
+// queueing on the few lines a packed array would occupy.
+constexpr int kAccStride = 16;     // doubles between consecutive (band, group) pairs
 
 template <typename T>
 struct Vec;
@@ -150,8 +154,8 @@ __global__ void __launch_bounds__(1024) gn_stats_kernel(const T* __restrict__ x,
       ds += ssum[c];
       dq += ssq[c];
     }
-    atomicAdd(acc + (p * a.G + g) * 2, ds);
-    atomicAdd(acc + (p * a.G + g) * 2 + 1, dq);
+    atomicAdd(acc + (p * a.G + g) * kAccStride, ds);
+    atomicAdd(acc + (p * a.G + g) * kAccStride + 1, dq);
   }
   __threadfence();
   __syncthreads();
@@ -164,8 +168,9 @@ __global__ void __launch_bounds__(1024) gn_stats_kernel(const T* __restrict__ x,
   double* f = reinterpret_cast<double*>(gn_smem);   // [P][G][2]
   const double n = static_cast<double>(a.HWp) * cg;
   for (int i = threadIdx.x; i < a.P * a.G * 2; i += blockDim.x) {
-    const double m = __ldcg(acc + i) / n;
-    acc[i] = 0.0;                                    // ready for the next call
+    double* cell = acc + (i >> 1) * kAccStride + (i & 1);
+    const double m = __ldcg(cell) / n;
+    *cell = 0.0;                                     // ready for the next call
     f[i] = m;
     fresh_local[i] = static_cast<float>(m);
   }
@@ -267,6 +272,252 @@ __global__ void __launch_bounds__(1024) gn_apply_kernel(const T* __restrict__ x,
   }
 }
 
+// ---------------------------------------------------------------------------
+// Single-pass variant for tensors that fit in the GPU's shared memory: one
+// block per SM (cooperative launch, so all blocks are resident), each block
+// pulls its contiguous chunk of x into shared memory with bulk copies,
+// accumulates its (band, group) sums into the fp64 accumulator, meets the
+// other blocks at a grid barrier, turns the sums into the moments its bands
+// use, normalises its chunk in place and writes it back with bulk stores.
+// x is read from HBM once and y written once, in one launch.
+struct GnFusedArgs {
+  int HW, HWp, C, G, P, vpp, lanes, chunk;
+  float eps, w;
+  int silu, mode;
+};
+
+// Moments band pp normalises with for group g, from the fresh moments f
+// (f[(p*G+g)*2] = E[x], +1 = E[x^2]) of all bands; see the file comment.
+__device__ __forceinline__ void gn_used_moments(const double* f, int pp, int g, int P, int G,
+                                                int mode, float w, const float* stale_global,
+                                                const float* stale_local, double* m_out,
+                                                double* var_out, double* gm1_out,
+                                                double* gm2_out) {
+  const int i = pp * G + g;
+  double gm1 = 0.0, gm2 = 0.0;
+  for (int q = 0; q < P; ++q) {
+    gm1 += f[2 * (q * G + g)];
+    gm2 += f[2 * (q * G + g) + 1];
+  }
+  gm1 /= P;
+  gm2 /= P;
+  double m1, m2;
+  if (mode == DP_MODE_SYNC) {
+    m1 = gm1;
+    m2 = gm2;
+  } else if (mode == DP_MODE_DISPLACED) {
+    m1 = static_cast<double>(stale_global[2 * g]) + w * (f[2 * i] - static_cast<double>(stale_local[2 * i]));
+    m2 = static_cast<double>(stale_global[2 * g + 1]) +
+         w * (f[2 * i + 1] - static_cast<double>(stale_local[2 * i + 1]));
+  } else {
+    m1 = f[2 * i];
+    m2 = f[2 * i + 1];
+  }
+  double var = m2 - m1 * m1;
+  if (var < 0.0) var = f[2 * i + 1] - f[2 * i] * f[2 * i];
+  *m_out = m1;
+  *var_out = var;
+  *gm1_out = gm1;
+  *gm2_out = gm2;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(1024, 1) gn_fused_kernel(
+    const T* __restrict__ x, T* __restrict__ y, const float* __restrict__ gamma,
+    const float* __restrict__ beta, GnFusedArgs a, double* __restrict__ acc,
+    unsigned* __restrict__ bar, const float* __restrict__ stale_global,
+    const float* __restrict__ stale_local, float* __restrict__ fresh_local,
+    float* __restrict__ fresh_global, float* __restrict__ used, int* __restrict__ status) {
+  constexpr int V = Vec<T>::N;
+  extern __shared__ __align__(128) unsigned char gn_smem[];
+  T* data = reinterpret_cast<T*>(gn_smem);                               // [chunk][C]
+  const size_t data_bytes = ((static_cast<size_t>(a.chunk) * a.C * sizeof(T)) + 127) & ~size_t(127);
+  float* ssum = reinterpret_cast<float*>(gn_smem + data_bytes);          // [lanes][C]
+  float* ssq = ssum + a.lanes * a.C;                                     // [lanes][C]
+  double* f = reinterpret_cast<double*>(ssq + a.lanes * a.C);            // [P][G][2]
+  float* sscale = reinterpret_cast<float*>(f + a.P * a.G * 2);           // [C]
+  float* sshift = sscale + a.C;                                          // [C]
+  __shared__ __align__(8) uint64_t load_bar;
+  __shared__ int s_ok;
+
+  const int beg = blockIdx.x * a.chunk;
+  const int end = min(a.HW, beg + a.chunk);
+  const int npix = max(0, end - beg);
+  const int v = threadIdx.x % a.vpp, pl = threadIdx.x / a.vpp;
+  const bool worker = threadIdx.x < a.vpp * a.lanes;
+  const int cg = a.C / a.G;
+
+  // ---- phase 1: bulk-load the chunk
+  if (threadIdx.x == 0) {
+    mbar_init(&load_bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && npix > 0) {
+    const uint32_t total = static_cast<uint32_t>(npix) * a.C * sizeof(T);
+    mbar_arrive_expect_tx(&load_bar, total);
+    const char* src = reinterpret_cast<const char*>(x + static_cast<size_t>(beg) * a.C);
+    char* dst = reinterpret_cast<char*>(data);
+    for (uint32_t off = 0; off < total; off += 16384u) {
+      const uint32_t n = min(16384u, total - off);
+      bulk_load(dst + off, src + off, n, &load_bar);
+    }
+  }
+  if (npix > 0) {
+    // a load that never lands is recorded in *status; the block still meets
+    // the others at the grid barrier so that nobody waits on it
+    int no_abort = 0;
+    mbar_wait(&load_bar, 0, &no_abort, status);
+  }
+  __syncthreads();
+
+  // ---- per-(band, group) sums of the chunk, one band segment at a time
+  for (int b = npix > 0 ? beg / a.HWp : a.P; b < a.P && b * a.HWp < end; ++b) {
+    const int lo = max(beg, b * a.HWp) - beg, hi = min(end, (b + 1) * a.HWp) - beg;
+    float sum[V], sq[V];
+#pragma unroll
+    for (int j = 0; j < V; ++j) sum[j] = sq[j] = 0.f;
+    if (worker) {
+      for (int pix = lo + pl; pix < hi; pix += a.lanes) {
+        float t[V];
+        Vec<T>::load(data + static_cast<size_t>(pix) * a.C + v * V, t);
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+          sum[j] += t[j];
+          sq[j] = fmaf(t[j], t[j], sq[j]);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < V; ++j) {
+        ssum[pl * a.C + v * V + j] = sum[j];
+        ssq[pl * a.C + v * V + j] = sq[j];
+      }
+    }
+    __syncthreads();
+    for (int c = threadIdx.x; c < a.C; c += blockDim.x) {
+      float cs = 0.f, cq = 0.f;
+      for (int l = 0; l < a.lanes; ++l) {
+        cs += ssum[l * a.C + c];
+        cq += ssq[l * a.C + c];
+      }
+      ssum[c] = cs;
+      ssq[c] = cq;
+    }
+    __syncthreads();
+    for (int g = threadIdx.x; g < a.G; g += blockDim.x) {
+      double ds = 0.0, dq = 0.0;
+      for (int c = g * cg; c < (g + 1) * cg; ++c) {
+        ds += ssum[c];
+        dq += ssq[c];
+      }
+      atomicAdd(acc + (b * a.G + g) * kAccStride, ds);
+      atomicAdd(acc + (b * a.G + g) * kAccStride + 1, dq);
+    }
+    __syncthreads();
+  }
+
+  // ---- grid barrier (count, generation), bounded
+  if (threadIdx.x == 0) {
+    s_ok = 1;
+    volatile unsigned* gen = bar + 1;
+    const unsigned my_gen = *gen;
+    __threadfence();
+    if (atomicAdd(bar, 1u) == gridDim.x - 1) {
+      bar[0] = 0u;
+      __threadfence();
+      atomicAdd(bar + 1, 1u);
+    } else {
+      const unsigned long long t0 = globaltimer_ns();
+      while (*gen == my_gen) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+          atomicExch(status, DP_ERR_TIMEOUT);
+          s_ok = 0;
+          break;
+        }
+        __nanosleep(64);
+      }
+    }
+    __threadfence();
+  }
+  __syncthreads();
+  if (!s_ok) return;
+
+  // ---- moments (every block), outputs (block 0), accumulator reset (last reader)
+  const double n = static_cast<double>(a.HWp) * cg;
+  for (int i = threadIdx.x; i < a.P * a.G * 2; i += blockDim.x)
+    f[i] = __ldcg(acc + (i >> 1) * kAccStride + (i & 1)) / n;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(bar + 2, 1u) == gridDim.x - 1) {
+      for (int i = 0; i < a.P * a.G; ++i) {
+        acc[i * kAccStride] = 0.0;
+        acc[i * kAccStride + 1] = 0.0;
+      }
+      bar[2] = 0u;
+      __threadfence();
+    }
+  }
+  if (blockIdx.x == 0) {
+    for (int i = threadIdx.x; i < a.P * a.G; i += blockDim.x) {
+      double m1, var, gm1, gm2;
+      gn_used_moments(f, i / a.G, i % a.G, a.P, a.G, a.mode, a.w, stale_global, stale_local, &m1,
+                      &var, &gm1, &gm2);
+      used[2 * i] = static_cast<float>(m1);
+      used[2 * i + 1] = static_cast<float>(var);
+      fresh_local[2 * i] = static_cast<float>(f[2 * i]);
+      fresh_local[2 * i + 1] = static_cast<float>(f[2 * i + 1]);
+      if (fresh_global && i < a.G) {
+        fresh_global[2 * i] = static_cast<float>(gm1);
+        fresh_global[2 * i + 1] = static_cast<float>(gm2);
+      }
+    }
+  }
+
+  // ---- apply in shared memory, band segment by band segment, then store
+  for (int b = npix > 0 ? beg / a.HWp : a.P; b < a.P && b * a.HWp < end; ++b) {
+    const int lo = max(beg, b * a.HWp) - beg, hi = min(end, (b + 1) * a.HWp) - beg;
+    for (int c = threadIdx.x; c < a.C; c += blockDim.x) {
+      double m1, var, gm1, gm2;
+      gn_used_moments(f, b, c / cg, a.P, a.G, a.mode, a.w, stale_global, stale_local, &m1, &var,
+                      &gm1, &gm2);
+      const float sc = rsqrtf(static_cast<float>(var) + a.eps) * gamma[c];
+      sscale[c] = sc;
+      sshift[c] = beta[c] - static_cast<float>(m1) * sc;
+    }
+    __syncthreads();
+    if (worker) {
+      float sc[V], sh[V];
+#pragma unroll
+      for (int j = 0; j < V; ++j) {
+        sc[j] = sscale[v * V + j];
+        sh[j] = sshift[v * V + j];
+      }
+      for (int pix = lo + pl; pix < hi; pix += a.lanes) {
+        T* p = data + static_cast<size_t>(pix) * a.C + v * V;
+        float t[V];
+        Vec<T>::load(p, t);
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+          float z = fmaf(t[j], sc[j], sh[j]);
+          if (a.silu) z = __fdividef(z, 1.0f + __expf(-z));
+          t[j] = z;
+        }
+        Vec<T>::store(p, t);
+      }
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0 && npix > 0) {
+    fence_proxy_async_smem();
+    const uint32_t total = static_cast<uint32_t>(npix) * a.C * sizeof(T);
+    char* dst = reinterpret_cast<char*>(y + static_cast<size_t>(beg) * a.C);
+    const char* src = reinterpret_cast<const char*>(data);
+    for (uint32_t off = 0; off < total; off += 16384u) bulk_store(dst + off, src + off, min(16384u, total - off));
+    bulk_commit_and_wait_all();
+  }
+}
+
 static int gn_plan(int H, int W, int C, int G, int P, int dtype, GnArgs* a) {
   const int V = dtype == DP_BF16 ? 8 : 4;
   a->HWp = (H / P) * W;
@@ -305,7 +556,77 @@ static int gn_validate(const void* x, const void* y, int H, int W, int C, int G,
 }
 
 size_t gn_workspace_bytes(int P, int G) {
-  return 256 + static_cast<size_t>(P) * G * 2 * sizeof(double);
+  return 256 + static_cast<size_t>(P) * G * kAccStride * sizeof(double);
+}
+
+// Plan of the single-pass variant: blocks, chunk and shared memory; false if
+// the tensor does not fit.  Shared with the launch counter of the block step.
+bool gn_fused_plan(int H, int W, int C, int G, int P, int dtype, int* blocks, int* chunk,
+                   int* threads, size_t* smem) {
+  const int e = dtype == DP_BF16 ? 2 : 4;
+  const int V = 16 / e;
+  const int vpp = C / V;
+  if (vpp > 1024) return false;
+  int lanes = vpp >= 512 ? 1 : 512 / vpp;
+  if (vpp * lanes > 1024) lanes = 1024 / vpp;
+  const long HW = static_cast<long>(H) * W;
+  const int nb = num_sms();
+  const long ch = (HW + nb - 1) / nb;
+  const size_t data = ((static_cast<size_t>(ch) * C * e) + 127) & ~size_t(127);
+  const size_t need = data + static_cast<size_t>(lanes) * C * 8 + static_cast<size_t>(P) * G * 16 +
+                      static_cast<size_t>(C) * 8;
+  if (need > 200 * 1024) return false;
+  if ((static_cast<size_t>(ch) * C * e) % 16) return false;
+  *blocks = static_cast<int>((HW + ch - 1) / ch);
+  *chunk = static_cast<int>(ch);
+  *threads = ((vpp * lanes + 31) / 32) * 32;
+  *smem = need;
+  return true;
+}
+
+// Launches the single-pass variant if the tensor fits; returns false (and
+// leaves *rc untouched) when the two-kernel path must be used.
+static bool gn_fused_launch(const void* x, void* y, const float* gamma, const float* beta, int H,
+                            int W, int C, int G, int P, float eps, float w, int silu, int mode,
+                            int dtype, const float* stale_global, const float* stale_local,
+                            float* fresh_local, float* fresh_global, float* used, double* acc,
+                            unsigned* bar, cudaStream_t stream, int* rc) {
+  int blocks, chunk, threads;
+  size_t smem;
+  if (!gn_fused_plan(H, W, C, G, P, dtype, &blocks, &chunk, &threads, &smem)) return false;
+  static int attr_mask[2] = {0, 0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const void* fn = dtype == DP_BF16 ? reinterpret_cast<const void*>(gn_fused_kernel<__nv_bfloat16>)
+                                    : reinterpret_cast<const void*>(gn_fused_kernel<float>);
+  if (!(attr_mask[dtype] & (1 << (dev & 31)))) {
+    *rc = cuda_check(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024),
+                     "fused groupnorm smem attribute");
+    if (*rc) return true;
+    attr_mask[dtype] |= 1 << (dev & 31);
+  }
+  GnFusedArgs a;
+  a.HW = H * W;
+  a.HWp = (H / P) * W;
+  a.C = C;
+  a.G = G;
+  a.P = P;
+  a.vpp = C / (dtype == DP_BF16 ? 8 : 4);
+  a.lanes = a.vpp >= 512 ? 1 : 512 / a.vpp;
+  if (a.vpp * a.lanes > 1024) a.lanes = 1024 / a.vpp;
+  a.chunk = chunk;
+  a.eps = eps;
+  a.w = w;
+  a.silu = silu;
+  a.mode = mode;
+  int* status = device_status_ptr();
+  void* args[] = {const_cast<void**>(&x), &y, const_cast<float**>(&gamma), const_cast<float**>(&beta),
+                  &a, &acc, &bar, const_cast<float**>(&stale_global), const_cast<float**>(&stale_local),
+                  &fresh_local, &fresh_global, &used, &status};
+  mark_launch(stream);
+  *rc = cuda_check(cudaLaunchCooperativeKernel(fn, dim3(blocks), dim3(threads), args, smem, stream),
+                   "fused groupnorm launch");
+  return true;
 }
 
 // Internal entry shared by the ABI call and the block step.
@@ -321,6 +642,13 @@ int gn_launch(const void* x, void* y, const float* gamma, const float* beta, int
   a.mode = mode;
   unsigned* counter = static_cast<unsigned*>(workspace);
   double* acc = reinterpret_cast<double*>(static_cast<char*>(workspace) + 256);
+  {
+    int rc = 0;
+    if (gn_fused_launch(x, y, gamma, beta, H, W, C, G, P, eps, w, silu, mode, dtype, stale_global,
+                        stale_local, fresh_local, fresh_global, used, acc, counter + 4, stream,
+                        &rc))
+      return rc;
+  }
   const int threads = a.vpp * a.lanes;
   const int blocks = a.P * a.S;
   size_t smem_stats = static_cast<size_t>(a.lanes) * C * 2 * sizeof(float);
@@ -371,7 +699,7 @@ int gn_launch(const void* x, void* y, const float* gamma, const float* beta, int
 // process exits.  Host code must not hand the array's name to a kernel: on
 // the host that name is only a stand-in, so its device address is looked up
 // once per device with cudaGetSymbolAddress and that address is passed on.
-constexpr size_t kGnStaticScratchBytes = 32 * 1024;
+constexpr size_t kGnStaticScratchBytes = 64 * 1024;
 static __device__ __align__(256) unsigned char g_gn_static_scratch[kGnStaticScratchBytes];
 
 static int gn_static_scratch(void** out) {

@@ -7,6 +7,8 @@
 namespace dp {
 
 size_t gn_workspace_bytes(int P, int G);
+bool gn_fused_plan(int H, int W, int C, int G, int P, int dtype, int* blocks, int* chunk,
+                   int* threads, size_t* smem);
 int gn_launch(const void* x, void* y, const float* gamma, const float* beta, int H, int W, int C,
               int G, int P, float eps, float w, int silu, int mode, int dtype,
               const float* stale_global, const float* stale_local, float* fresh_local,

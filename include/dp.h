@@ -142,14 +142,14 @@ DP_API int dp_groupnorm_async(const void* x, void* y, const float* gamma, const 
  * This entry point takes the same arguments as dp_groupnorm_async minus the
  * workspace and uses a fixed scratch array inside the library instead.
  *
- *  - Limit: the scratch holds 32 KiB, enough for P * G up to 2032 (bands x
+ *  - Limit: the scratch holds 64 KiB, enough for P * G up to 510 (bands x
  *    groups); larger requests return DP_ERR_UNSUPPORTED with a message.
- *  - Every GPU that loads the library holds those 32 KiB until the process
+ *  - Every GPU that loads the library holds those 64 KiB until the process
  *    exits.
  *  - The first call on a device looks the array's device address up
  *    (cudaGetSymbolAddress); make that first call before any stream capture.
  *  - Each call clears the part of the scratch it uses (a cudaMemsetAsync of
- *    256 + 16 * P * G bytes on `stream`) before its kernels; nothing is
+ *    256 + 128 * P * G bytes on `stream`) before its kernels; nothing is
  *    allocated.
  *  - All calls share the one array and it keeps the last call's contents:
  *    calls whose kernels overlap on the GPU (different streams, no ordering)
@@ -308,16 +308,35 @@ DP_API int dp_block_state_init(const dp_block_desc* d, dp_block_state* s, void* 
 DP_API int dp_block_step(const dp_block_desc* d, dp_block_state* s, const void* x, void* out,
                   const void* const* weights, int n_weights, int mode, void* stream);
 
+/* Kernel kinds reported by dp_block_launch_info. */
+#define DP_KERNEL_GN_STATS 0   /* GroupNorm statistics pass                     */
+#define DP_KERNEL_GN_APPLY 1   /* GroupNorm apply pass                          */
+#define DP_KERNEL_GN_FUSED 2   /* single-pass GroupNorm (tensor fits on chip)   */
+#define DP_KERNEL_CONV 3       /* 3x3 halo conv (tensor cores)                  */
+#define DP_KERNEL_LINEAR 4     /* projection / 1x1 conv (tensor cores)          */
+#define DP_KERNEL_ATTN 5       /* stale-K/V attention (tensor cores)            */
+#define DP_KERNEL_COPY 6       /* device copy                                   */
+#define DP_KERNEL_CONV_SMALL 7 /* direct 3x3 conv for few input channels        */
+
 /*
- * Number of kernel launches one dp_block_step makes for this descriptor, in
- * this order --
- *   GN_CONV:  GN statistics, GN apply, conv
- *   RESBLOCK: GN1 statistics, GN1 apply, conv1, GN2 statistics, GN2 apply,
- *             [1x1 shortcut if C != Cout], conv2
- *   ATTN:     GN statistics, GN apply, q/k/v projection, attention, out projection
+ * Number of kernel launches one displaced dp_block_step makes for this
+ * descriptor.  A GroupNorm is one launch when its tensor fits in the GPU's
+ * shared memory and two (statistics, apply) otherwise.  Launch order --
+ *   GN_CONV:  GN, conv
+ *   RESBLOCK: GN1, conv1, GN2, [1x1 shortcut if C != Cout], conv2
+ *   ATTN:     GN, q/k/v projection, attention, out projection
+ *   UNET_MINI: input copy, conv_in, then its blocks and downsamplers in order
  * Negative status on a bad descriptor.
  */
 DP_API int dp_block_launch_count(const dp_block_desc* d);
+
+/*
+ * Kind (DP_KERNEL_*), algorithmic flops and algorithmic bytes of launch i of
+ * one dp_block_step in `mode`, from the same code path that makes the
+ * launches.  Bytes count each tensor a kernel must read or write once.
+ */
+DP_API int dp_block_launch_info(const dp_block_desc* d, int mode, int i, int* kind,
+                                double* flops, double* bytes);
 
 /*
  * dp_block_step that also records events[i] (cudaEvent_t, passed as void*)

@@ -61,12 +61,28 @@ def test_mode_for_step_matches_input_module(B):
 def test_block_desc_validation(B):
     d = B.dp_block_desc_init(B.RESBLOCK, 128, 128, 320, 320, 32, 4, 0, B.BF16, 1, 1e-5, 1.0)
     assert B.dp_block_workspace_size(d) > 4 * 128 * 128 * 320 * 2
-    assert B.dp_block_launch_count(d) == 6
+    # a GroupNorm whose tensor fits in shared memory is one launch
+    assert [B.dp_block_launch_info(d, B.DISPLACED, i)[0] for i in range(B.dp_block_launch_count(d))] \
+        == ["gn_fused", "conv", "gn_fused", "conv"]
     assert abs(B.dp_block_flops(d) - 2 * 2 * 128 * 128 * 320 * 9 * 320) < 1
+    assert abs(sum(B.dp_block_launch_info(d, B.DISPLACED, i)[1] for i in range(4))
+               - B.dp_block_flops(d)) < 1
     d2 = B.dp_block_desc_init(B.RESBLOCK, 64, 64, 320, 640, 32, 4, 0, B.BF16, 1, 1e-5, 1.0)
-    assert B.dp_block_launch_count(d2) == 7
+    assert [B.dp_block_launch_info(d2, B.SYNC, i)[0] for i in range(B.dp_block_launch_count(d2))] \
+        == ["gn_fused", "conv", "gn_fused", "linear", "conv"]
     da = B.dp_block_desc_init(B.ATTN, 64, 64, 640, 640, 32, 4, 10, B.BF16, 0, 1e-5, 1.0)
-    assert B.dp_block_launch_count(da) == 5
+    assert [B.dp_block_launch_info(da, B.DISPLACED, i)[0] for i in range(B.dp_block_launch_count(da))] \
+        == ["gn_fused", "linear", "attn", "linear"]
+    # naive attention sees only its own band's keys
+    assert B.dp_block_launch_info(da, B.NAIVE, 2)[1] * 4 == B.dp_block_launch_info(da, B.DISPLACED, 2)[1]
+    # the 480x480 tensor does not fit on chip: two GroupNorm passes
+    d4 = B.dp_block_desc_init(B.GN_CONV, 480, 480, 320, 320, 32, 8, 0, B.BF16, 1, 1e-5, 1.0)
+    assert [B.dp_block_launch_info(d4, B.DISPLACED, i)[0] for i in range(B.dp_block_launch_count(d4))] \
+        == ["gn_stats", "gn_apply", "conv"]
+    du = B.dp_block_desc_init(B.UNET_MINI, 128, 128, 4, 0, 32, 4, 0, B.BF16, 1, 1e-5, 1.0)
+    assert B.dp_block_weight_count(du) == 46
+    assert abs(B.dp_block_flops(du) - sum(B.dp_block_launch_info(du, B.DISPLACED, i)[1]
+                                          for i in range(B.dp_block_launch_count(du)))) < 1
     bad = [
         (B.RESBLOCK, 130, 128, 320, 320, 32, 4, 0, B.BF16, B.DP_ERR_UNSUPPORTED),   # H % P
         (B.RESBLOCK, 128, 128, 320, 320, 33, 4, 0, B.BF16, B.DP_ERR_UNSUPPORTED),   # C % G

@@ -30,6 +30,8 @@ GN_CASES = [
     (640, 16, 16, 4, 32, "bf16", False),
     (96, 24, 9, 8, 32, "bf16", True),
     (1280, 8, 8, 2, 32, "bf16", True),
+    (320, 256, 240, 4, 32, "bf16", True),    # too big for shared memory: two-pass kernels
+    (64, 512, 384, 8, 32, "fp32", False),    # two-pass, fp32
 ]
 
 

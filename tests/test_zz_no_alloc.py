@@ -55,7 +55,7 @@ def test_groupnorm_noalloc_matches_workspace_call_twice_in_a_row():
 
 def test_groupnorm_noalloc_rejects_oversized_requests():
     with pytest.raises(B.DPError) as e:
-        # P * G = 8 * 512 = 4096 is a valid GroupNorm but needs 64 KiB of scratch
+        # P * G = 8 * 512 = 4096 is a valid GroupNorm but needs 512 KiB of scratch
         B.dp_groupnorm_async_noalloc(16, 32, 16, 16, 8, 8, 1024, 512, 8, 1e-5, 1.0, 1, B.SYNC,
                                      B.BF16, None, None, 16, 16)
     assert e.value.code == B.DP_ERR_UNSUPPORTED
