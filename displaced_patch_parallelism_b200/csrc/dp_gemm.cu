@@ -39,6 +39,10 @@ struct GemmParams {
   CUtensorMap tmA0;   // plain A, or the conv's fresh activations
   CUtensorMap tmA1;   // the conv's stale activations
   CUtensorMap tmB;    // weights, [N][K] K-major
+  // Pair kernels only: output segments and residual as 32-column boxes of one
+  // epilogue warp's 32 rows (64-byte swizzle), for TMA stores and loads.
+  CUtensorMap tmO[3];
+  CUtensorMap tmR;
   int a_mode;         // 0: plain [M][K] rows, 1: 3x3 conv
   int M;
   int H, W, Ho, Wo, Cin, stride, hb_in, hb_out, mode, R, Wt, tiles_w, kc;
@@ -369,13 +373,171 @@ struct PairCfg {
   static constexpr int BSUB_BYTES = (NI / 2) * 128;  // this CTA's half of one B slice
   static constexpr int B_BYTES = NJ * BSUB_BYTES;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES_RAW = (200 * 1024) / STAGE_BYTES;
+  static constexpr int STAGES_RAW = (190 * 1024) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
   static constexpr int TMEM_COLS = BN <= 128 ? 128 : BN <= 256 ? 256 : 512;
-  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 256;
+  static constexpr int EPI_SLOT = 32 * 64;          // 32 rows x 32 bf16 columns
+  static constexpr int EPI_BYTES = 4 * 4 * EPI_SLOT;  // 4 warps x (2 output + 2 residual slots)
+  static constexpr int BIAS_BYTES = 4 * BN * 4;     // one fp32 copy per epilogue warp
+  static constexpr int SMEM = STAGES * STAGE_BYTES + EPI_BYTES + BIAS_BYTES + 1024 + 256;
   static_assert(BSUB_BYTES % 1024 == 0, "B slice alignment");
+  static_assert(SMEM <= 227 * 1024, "shared memory");
   static_assert(BN <= 512 && NI % 32 == 0 && NI <= 256, "tile");
 };
+
+constexpr int kEpiSlot = 32 * 64;   // one epilogue warp's 32 rows x 32 bf16 columns
+
+// Shared-memory state of one epilogue warp of a pair kernel.  Residual chunks
+// arrive by TMA two chunks ahead of use; finished chunks leave by TMA stores
+// from two alternating slots.  The counters give each slot's barrier phase.
+struct PairEpi {
+  uint8_t* out;      // 2 output slots
+  uint8_t* res;      // 2 residual slots
+  float* bias;       // the tile's BN bias values
+  uint64_t* rbar;    // one barrier per residual slot
+  uint32_t ri;       // residual chunks consumed so far
+  uint32_t rpend;    // residual loads issued and not yet consumed
+  uint32_t oi;       // output stores issued so far
+};
+
+// Byte offset of 16-byte chunk j of row i in a slot written with the 64-byte
+// swizzle (chunk index XOR address bits 7-8): conflict-free row-per-lane access.
+__device__ __forceinline__ uint32_t sw64_off(int i, int j) {
+  return static_cast<uint32_t>(i * 64 + ((j ^ ((i >> 1) & 3)) << 4));
+}
+
+// Box of one epilogue warp: first column of its output segment (x), first
+// pixel (y) and image row (z, convs), the output segment, and whether any of
+// its rows is inside the output.
+struct EpiBox {
+  int x, y, z, seg;
+  bool ok;
+};
+__device__ __forceinline__ EpiBox pair_epi_box(const GemmParams& p, int mt, int q, int n0) {
+  EpiBox b;
+  if (p.a_mode == 0) {
+    b.seg = n0 / p.split;
+    b.x = n0 - b.seg * p.split;
+    b.y = mt * 128 + q * 32;
+    b.z = 0;
+    b.ok = mt < p.m_tiles && b.y < p.M;
+  } else {
+    const int tr = mt / p.tiles_w, tc = mt - tr * p.tiles_w;
+    b.seg = 0;
+    b.x = n0;
+    b.z = tr * p.R + (q * 32) / p.Wt;
+    b.y = tc * p.Wt + (q * 32) % p.Wt;
+    b.ok = mt < p.m_tiles && b.z < p.Ho && b.y < p.Wo;
+  }
+  return b;
+}
+
+__device__ __forceinline__ void pair_epi_res_load(const GemmParams& p, const EpiBox& b, int col,
+                                                  uint8_t* dst, uint64_t* bar) {
+  mbar_arrive_expect_tx(bar, kEpiSlot);
+  if (p.a_mode == 0) tma_load_2d(dst, &p.tmR, bar, col, b.y);
+  else tma_load_3d(dst, &p.tmR, bar, col, b.y, b.z);
+}
+
+// Epilogue of one pair tile for one epilogue warp: this CTA's 128 accumulator
+// rows (TMEM lane quarter q) are drained in 32-column chunks; the accumulator
+// goes back to the leader after the last chunk; bias (staged in shared
+// memory) and residual (prefetched by TMA) are added and the bf16 chunk is
+// stored by TMA, ragged edges clipped by the tensor map.  Returns false when
+// a wait gave up (the caller tears down).
+template <int BN>
+__device__ __forceinline__ bool pair_epilogue_tile(const GemmParams& p, uint32_t tmem, int q, int lane,
+                                                   uint32_t rank, int tile, int it, uint64_t* acc_full,
+                                                   uint32_t acc_empty_leader, volatile int* abort_flag,
+                                                   PairEpi& e) {
+  constexpr int NCH = BN / 32;
+  static_assert(NCH >= 2, "chunks");
+  const int mp = tile / p.n_tiles, nt = tile - mp * p.n_tiles;
+  const int mt = 2 * mp + static_cast<int>(rank);
+  const int n0 = nt * BN;
+  const EpiBox b = pair_epi_box(p, mt, q, n0);
+  const bool res = p.residual != nullptr && b.ok;
+  // Staged while the MMA of this tile still runs: the bias row and the first
+  // two residual chunks.  The previous tile's reads of both are finished.
+  for (int i = lane; i < BN; i += 32) e.bias[i] = p.bias ? __ldg(p.bias + n0 + i) : 0.f;
+  if (res) {
+    if (lane == 0) {
+      fence_proxy_async_smem();
+      for (int c = 0; c < 2; ++c) {
+        const uint32_t s = (e.ri + c) & 1u;
+        pair_epi_res_load(p, b, n0 + c * 32, e.res + s * kEpiSlot, &e.rbar[s]);
+      }
+    }
+    e.rpend = 2;
+  }
+  __syncwarp();
+  if (!mbar_wait(acc_full, it & 1, abort_flag, p.status)) return false;
+  tc_fence_after();
+  const CUtensorMap* om = &p.tmO[b.seg];
+#pragma unroll 1
+  for (int ch = 0; ch < NCH; ++ch) {
+    uint32_t r[32];
+    tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + ch * 32, r);
+    tmem_wait_ld();
+    if (ch == NCH - 1) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
+    }
+    if (!b.ok) continue;
+    float v[32];
+    const float* bb = e.bias + ch * 32;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) + bb[j];
+    if (res) {
+      const uint32_t s = e.ri & 1u;
+      if (!mbar_wait(&e.rbar[s], (e.ri >> 1) & 1u, abort_flag, p.status)) return false;
+      const uint8_t* rs = e.res + s * kEpiSlot;
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        uint4 u = *reinterpret_cast<const uint4*>(rs + sw64_off(lane, jj));
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const float2 f = __bfloat1622float2(h[t]);
+          v[8 * jj + 2 * t] += f.x;
+          v[8 * jj + 2 * t + 1] += f.y;
+        }
+      }
+      ++e.ri;
+      --e.rpend;
+      __syncwarp();
+      if (ch + 2 < NCH) {
+        if (lane == 0) {
+          fence_proxy_async_smem();
+          pair_epi_res_load(p, b, n0 + (ch + 2) * 32, e.res + s * kEpiSlot, &e.rbar[s]);
+        }
+        ++e.rpend;
+      }
+    }
+    uint8_t* ob = e.out + (e.oi & 1u) * kEpiSlot;
+    if (lane == 0) bulk_wait_read_1();   // the store that last used this slot has read it
+    __syncwarp();
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      uint4 u;
+      u.x = pack_bf16x2(v[8 * jj], v[8 * jj + 1]);
+      u.y = pack_bf16x2(v[8 * jj + 2], v[8 * jj + 3]);
+      u.z = pack_bf16x2(v[8 * jj + 4], v[8 * jj + 5]);
+      u.w = pack_bf16x2(v[8 * jj + 6], v[8 * jj + 7]);
+      *reinterpret_cast<uint4*>(ob + sw64_off(lane, jj)) = u;
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      if (p.a_mode == 0) tma_store_2d(om, ob, b.x + ch * 32, b.y);
+      else tma_store_3d(om, ob, b.x + ch * 32, b.y, b.z);
+      bulk_commit();
+    }
+    ++e.oi;
+  }
+  return true;
+}
 
 template <int NI, int NJ>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
@@ -386,12 +548,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::STAGES * C::A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::STAGES * C::B_BYTES);
+  uint8_t* sEpi = sB + C::STAGES * C::B_BYTES;
+  float* sBias = reinterpret_cast<float*>(sEpi + C::EPI_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sEpi + C::EPI_BYTES + C::BIAS_BYTES);
   uint64_t* empty = full + C::STAGES;
   uint64_t* acc_full = empty + C::STAGES;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* drain = acc_empty + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* rbar = drain + 1;   // [epilogue warp][residual slot]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rbar + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = warp_id(), lane = lane_id();
@@ -407,11 +572,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 8);
     mbar_init(drain, 1);
+    for (int s = 0; s < 8; ++s) mbar_init(&rbar[s], 1);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&p.tmA0);
     if (p.a_mode == 1) prefetch_tmap(&p.tmA1);
     prefetch_tmap(&p.tmB);
+    prefetch_tmap(&p.tmO[0]);
+    if (p.residual) prefetch_tmap(&p.tmR);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
@@ -550,82 +718,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   } else {
     // -------------------------------------------------------------- epilogue (both CTAs)
     const int q = warp & 3;
-    const int row = q * 32 + lane;
     const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
+    PairEpi e;
+    e.out = sEpi + q * 4 * kEpiSlot;
+    e.res = e.out + 2 * kEpiSlot;
+    e.bias = sBias + q * C::BN;
+    e.rbar = rbar + 2 * q;
+    e.ri = e.rpend = e.oi = 0;
     int it = 0;
-    for (int tile = pair; tile < num_tiles; tile += npairs, ++it) {
-      if (!mbar_wait(acc_full, it & 1, abort_flag, p.status)) break;
-      tc_fence_after();
-      const int mp = tile / p.n_tiles, nt = tile - mp * p.n_tiles;
-      const int mt = 2 * mp + static_cast<int>(rank);
-      bool valid;
-      size_t pix;
-      if (p.a_mode == 0) {
-        const int m = mt * 128 + row;
-        valid = m < p.M;
-        pix = static_cast<size_t>(m);
-      } else {
-        const int tr = mt / p.tiles_w, tc = mt - tr * p.tiles_w;
-        const int r = tr * p.R + row / p.Wt, c = tc * p.Wt + row % p.Wt;
-        valid = mt < p.m_tiles && r < p.Ho && c < p.Wo;
-        pix = static_cast<size_t>(r) * p.Wo + c;
-      }
-      const int n0 = nt * C::BN;
-      const int seg = n0 / p.split;
-      __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(seg == 0 ? p.out0 : seg == 1 ? p.out1 : p.out2);
-      __nv_bfloat16* orow = outp + pix * p.ld_out + (n0 - seg * p.split);
-      const __nv_bfloat16* rrow =
-          p.residual ? static_cast<const __nv_bfloat16*>(p.residual) + pix * p.N + n0 : nullptr;
-#pragma unroll 1
-      for (int ch = 0; ch < C::BN / 32; ++ch) {
-        uint32_t r[32];
-        tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + ch * 32, r);
-        tmem_wait_ld();
-        if (ch == C::BN / 32 - 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
-        }
-        if (!valid) continue;
-        float v[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-        if (p.bias) {
-          const float4* b4 = reinterpret_cast<const float4*>(p.bias + n0 + ch * 32);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float4 b = __ldg(b4 + j);
-            v[4 * j] += b.x;
-            v[4 * j + 1] += b.y;
-            v[4 * j + 2] += b.z;
-            v[4 * j + 3] += b.w;
-          }
-        }
-        if (rrow) {
-          const uint4* r4 = reinterpret_cast<const uint4*>(rrow + ch * 32);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint4 u = r4[j];
-            const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 f = __bfloat1622float2(h[e]);
-              v[8 * j + 2 * e] += f.x;
-              v[8 * j + 2 * e + 1] += f.y;
-            }
-          }
-        }
-        uint4* o4 = reinterpret_cast<uint4*>(orow + ch * 32);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint4 u;
-          u.x = pack_bf16x2(v[8 * j], v[8 * j + 1]);
-          u.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
-          u.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
-          u.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
-          o4[j] = u;
-        }
-      }
+    for (int tile = pair; tile < num_tiles; tile += npairs, ++it)
+      if (!pair_epilogue_tile<C::BN>(p, tmem, q, lane, rank, tile, it, acc_full, acc_empty_leader,
+                                     abort_flag, e))
+        break;
+    if (lane == 0) {
+      // residual loads still in flight after an abort, then every store
+      for (uint32_t k = 0; k < e.rpend; ++k)
+        mbar_wait_teardown(&e.rbar[(e.ri + k) & 1u], ((e.ri + k) >> 1) & 1u);
+      bulk_wait_all();
     }
   }
 
@@ -636,6 +745,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     tc_fence_after();
     tmem_dealloc_pair(tmem, C::TMEM_COLS);
   }
+}
+
+// Tensor maps of a pair kernel's epilogue: each epilogue warp stores (and
+// loads residual) boxes of 32 channels x its 32 output rows with the 64-byte
+// swizzle.  Conv outputs are [Ho][Wo][Cout] (a warp's rows span min(Wt, 32)
+// pixels x 32 / min(Wt, 32) image rows); plain outputs are [M][ld_out] per
+// column segment and the residual is [M][N].
+static int encode_conv_epilogue(GemmParams& p, void* out, const void* residual, int Cout) {
+  const uint32_t bw = static_cast<uint32_t>(std::min(p.Wt, 32));
+  uint64_t dims[3] = {static_cast<uint64_t>(Cout), static_cast<uint64_t>(p.Wo),
+                      static_cast<uint64_t>(p.Ho)};
+  uint64_t str[2] = {static_cast<uint64_t>(Cout) * 2, static_cast<uint64_t>(p.Wo) * Cout * 2};
+  uint32_t box[3] = {32, bw, 32 / bw};
+  int rc = encode_tmap(&p.tmO[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, out, dims, str, box,
+                       CU_TENSOR_MAP_SWIZZLE_64B);
+  if (rc || !residual) return rc;
+  return encode_tmap(&p.tmR, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(residual), dims,
+                     str, box, CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
+static int encode_linear_epilogue(GemmParams& p, void* const outs[3], const void* residual) {
+  uint32_t box[2] = {32, 32};
+  for (int sgi = 0; sgi < p.N / p.split; ++sgi) {
+    uint64_t dims[2] = {static_cast<uint64_t>(p.split), static_cast<uint64_t>(p.M)};
+    uint64_t str[1] = {static_cast<uint64_t>(p.ld_out) * 2};
+    int rc = encode_tmap(&p.tmO[sgi], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, outs[sgi], dims, str, box,
+                         CU_TENSOR_MAP_SWIZZLE_64B);
+    if (rc) return rc;
+  }
+  if (!residual) return DP_OK;
+  uint64_t dims[2] = {static_cast<uint64_t>(p.N), static_cast<uint64_t>(p.M)};
+  uint64_t str[1] = {static_cast<uint64_t>(p.N) * 2};
+  return encode_tmap(&p.tmR, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(residual), dims,
+                     str, box, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 template <int NI, int NJ>
@@ -845,7 +988,11 @@ int conv3x3_launch(const void* a_fresh, const void* a_stale, const void* weight,
   rc = encode_tmap(&p.tmB, dt, 2, const_cast<void*>(weight), bdims, bstr, bbox,
                    CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc) return rc;
-  if (pair) return pw == 320 ? launch_pair<160, 2>(p, stream) : launch_pair<160, 1>(p, stream);
+  if (pair) {
+    rc = encode_conv_epilogue(p, out, residual, Cout);
+    if (rc) return rc;
+    return pw == 320 ? launch_pair<160, 2>(p, stream) : launch_pair<160, 1>(p, stream);
+  }
   return launch_gemm(p, BN, tf32, stream);
 }
 
@@ -887,7 +1034,12 @@ int linear_launch(const void* x, const void* weight, const float* bias, const vo
   rc = encode_tmap(&p.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(weight), bdims,
                    astr, bbox, CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc) return rc;
-  if (pair) return pw == 320 ? launch_pair<160, 2>(p, stream) : launch_pair<160, 1>(p, stream);
+  if (pair) {
+    void* const outs[3] = {out0, out1, out2};
+    rc = encode_linear_epilogue(p, outs, residual);
+    if (rc) return rc;
+    return pw == 320 ? launch_pair<160, 2>(p, stream) : launch_pair<160, 1>(p, stream);
+  }
   return launch_gemm(p, BN, false, stream);
 }
 

@@ -111,6 +111,8 @@ CONV_CASES = [
     (64, 320, 24, 16, 4, 1, "bf16", False),     # pair kernel, odd tile count
     (64, 320, 16, 16, 2, 2, "bf16", True),      # pair kernel, stride 2
     (320, 640, 8, 136, 2, 1, "bf16", True),     # pair kernel, 128-pixel rows, ragged
+    (320, 320, 64, 256, 4, 1, "bf16", True),    # halo-row pair kernel, 256x320 tiles
+    (320, 160, 6, 240, 3, 1, "bf16", False),    # halo-row pair kernel, 256x160, ragged row
     (64, 64, 16, 16, 2, 1, "fp32", False),
     (64, 128, 8, 10, 2, 1, "fp32", True),
 ]
