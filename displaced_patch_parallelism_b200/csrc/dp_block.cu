@@ -244,7 +244,8 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
     return gn_launch(in, y, static_cast<const float*>(gamma), static_cast<const float*>(beta), H,
                      W, ch, G, P, d->eps, d->w, silu, mode, d->dtype, at<float>(ws, g.global[o]),
                      at<float>(ws, g.local[o]), at<float>(ws, g.local[f]),
-                     at<float>(ws, g.global[f]), at<float>(ws, g.used), at<void>(ws, g.ws), st);
+                     at<float>(ws, g.global[f]), at<float>(ws, g.used), at<void>(ws, g.ws),
+                     gn_workspace_bytes(P, G), st);
   };
   // conv / linear / attention launches, or their records in planning mode
   auto conv = [&](const void* af, const void* as, const void* wt, const void* b, const void* res,

@@ -72,6 +72,31 @@ struct Vec<float> {
   }
 };
 
+// SiLU z / (1 + exp(-z)) with one special-function instruction: exp(-z) is
+// 2^(-z log2 e) from the hardware base-2 exponential (ex2.approx, about 22
+// correct bits), and the reciprocal of d = 1 + exp(-z) is Newton-Raphson
+// from a bit-pattern seed.  The seed K - bits(d) mirrors d's exponent and
+// mantissa about 1.0; K = 0x7EF31000 came from a scan of K over one binade
+// (relative error at most 5.1%), and two steps r += r (1 - d r) bring it to
+// 6.6e-6, far below a bf16 rounding.  The exponent argument is clamped at
+// 126 so that d and 1/d stay normal.
+__device__ __forceinline__ float silu_fast(float z) {
+  const float arg = fminf(-1.4426950408889634f * z, 126.f);
+  float e;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(arg));
+  const float d = 1.f + e;
+  float r = __int_as_float(0x7EF31000 - __float_as_int(d));
+  r = fmaf(r, fmaf(-d, r, 1.f), r);
+  r = fmaf(r, fmaf(-d, r, 1.f), r);
+  return z * r;
+}
+
+template <typename T, int N>
+__device__ __forceinline__ void silu_vec(float (&t)[N]) {
+#pragma unroll
+  for (int j = 0; j < N; ++j) t[j] = silu_fast(t[j]);
+}
+
 struct GnArgs {
   int HWp;      // pixels per band
   int C, G, P;
@@ -130,10 +155,13 @@ __global__ void __launch_bounds__(1024) gn_stats_kernel(const T* __restrict__ x,
       sq[j] = fmaf(t[j], t[j], sq[j]);
     }
   }
+  // 16-byte stores: scalar ones at this stride would conflict 8-way
 #pragma unroll
-  for (int j = 0; j < V; ++j) {
-    ssum[pl * a.C + v * V + j] = sum[j];
-    ssq[pl * a.C + v * V + j] = sq[j];
+  for (int j = 0; j < V; j += 4) {
+    *reinterpret_cast<float4*>(ssum + pl * a.C + v * V + j) =
+        make_float4(sum[j], sum[j + 1], sum[j + 2], sum[j + 3]);
+    *reinterpret_cast<float4*>(ssq + pl * a.C + v * V + j) =
+        make_float4(sq[j], sq[j + 1], sq[j + 2], sq[j + 3]);
   }
   __syncthreads();
   // lanes -> channels (row 0 of the scratch), then channels -> groups
@@ -246,11 +274,8 @@ __global__ void __launch_bounds__(1024) gn_apply_kernel(const T* __restrict__ x,
   T* yb = y + off;
   auto body = [&](float (&t)[V]) {
 #pragma unroll
-    for (int j = 0; j < V; ++j) {
-      float z = fmaf(t[j], sc[j], sh[j]);
-      if (a.silu) z = __fdividef(z, 1.0f + __expf(-z));
-      t[j] = z;
-    }
+    for (int j = 0; j < V; ++j) t[j] = fmaf(t[j], sc[j], sh[j]);
+    if (a.silu) silu_vec<T>(t);
   };
   int pix = beg + pl;
   for (; pix + 3 * a.lanes < end; pix += 4 * a.lanes) {
@@ -275,11 +300,13 @@ __global__ void __launch_bounds__(1024) gn_apply_kernel(const T* __restrict__ x,
 // ---------------------------------------------------------------------------
 // Single-pass variant for tensors that fit in the GPU's shared memory: one
 // block per SM (cooperative launch, so all blocks are resident), each block
-// pulls its contiguous chunk of x into shared memory with bulk copies,
-// accumulates its (band, group) sums into the fp64 accumulator, meets the
-// other blocks at a grid barrier, turns the sums into the moments its bands
-// use, normalises its chunk in place and writes it back with bulk stores.
-// x is read from HBM once and y written once, in one launch.
+// pulls its contiguous chunk of x into shared memory with bulk copies and
+// writes the sums of each (band segment, group) it holds to its own slot of
+// a partials array (no atomics: the order of every sum is fixed, so results
+// are reproducible).  After a grid barrier every block reduces the partials
+// of all bands in fp64, normalises its chunk from shared memory and stores
+// it straight to y.  x is read from HBM once and y written once, in one
+// launch.
 struct GnFusedArgs {
   int HW, HWp, C, G, P, vpp, lanes, chunk;
   float eps, w;
@@ -321,10 +348,25 @@ __device__ __forceinline__ void gn_used_moments(const double* f, int pp, int g, 
   *gm2_out = gm2;
 }
 
+// Grid-barrier primitives: release arrival, acquire polling.
+__device__ __forceinline__ unsigned atom_add_release_gpu(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.add.release.gpu.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(unsigned* p, unsigned v) {
+  asm volatile("st.release.gpu.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 template <typename T>
 __global__ void __launch_bounds__(1024, 1) gn_fused_kernel(
     const T* __restrict__ x, T* __restrict__ y, const float* __restrict__ gamma,
-    const float* __restrict__ beta, GnFusedArgs a, double* __restrict__ acc,
+    const float* __restrict__ beta, GnFusedArgs a, float2* __restrict__ part,
     unsigned* __restrict__ bar, const float* __restrict__ stale_global,
     const float* __restrict__ stale_local, float* __restrict__ fresh_local,
     float* __restrict__ fresh_global, float* __restrict__ used, int* __restrict__ status) {
@@ -337,6 +379,9 @@ __global__ void __launch_bounds__(1024, 1) gn_fused_kernel(
   double* f = reinterpret_cast<double*>(ssq + a.lanes * a.C);            // [P][G][2]
   float* sscale = reinterpret_cast<float*>(f + a.P * a.G * 2);           // [C]
   float* sshift = sscale + a.C;                                          // [C]
+  float* sgamma = sshift + a.C;                                          // [C]
+  float* sbeta = sgamma + a.C;                                           // [C]
+  float2* stage = reinterpret_cast<float2*>(sbeta + a.C);                // [G][slots]
   __shared__ __align__(8) uint64_t load_bar;
   __shared__ int s_ok;
 
@@ -346,22 +391,27 @@ __global__ void __launch_bounds__(1024, 1) gn_fused_kernel(
   const int v = threadIdx.x % a.vpp, pl = threadIdx.x / a.vpp;
   const bool worker = threadIdx.x < a.vpp * a.lanes;
   const int cg = a.C / a.G;
+  const size_t row_bytes = static_cast<size_t>(a.C) * sizeof(T);
 
-  // ---- phase 1: bulk-load the chunk
+  // ---- phase 1: bulk-load the chunk; gamma and beta meanwhile
   if (threadIdx.x == 0) {
     mbar_init(&load_bar, 1);
     fence_mbar_init();
   }
   __syncthreads();
   if (threadIdx.x == 0 && npix > 0) {
-    const uint32_t total = static_cast<uint32_t>(npix) * a.C * sizeof(T);
+    const uint32_t total = static_cast<uint32_t>(npix * row_bytes);
     mbar_arrive_expect_tx(&load_bar, total);
-    const char* src = reinterpret_cast<const char*>(x + static_cast<size_t>(beg) * a.C);
+    const char* src = reinterpret_cast<const char*>(x) + static_cast<size_t>(beg) * row_bytes;
     char* dst = reinterpret_cast<char*>(data);
     for (uint32_t off = 0; off < total; off += 16384u) {
       const uint32_t n = min(16384u, total - off);
       bulk_load(dst + off, src + off, n, &load_bar);
     }
+  }
+  for (int c = threadIdx.x; c < a.C; c += blockDim.x) {
+    sgamma[c] = __ldg(gamma + c);
+    sbeta[c] = __ldg(beta + c);
   }
   if (npix > 0) {
     // a load that never lands is recorded in *status; the block still meets
@@ -371,7 +421,8 @@ __global__ void __launch_bounds__(1024, 1) gn_fused_kernel(
   }
   __syncthreads();
 
-  // ---- per-(band, group) sums of the chunk, one band segment at a time
+  // ---- per-(band segment, group) sums of the chunk into this block's slots:
+  // the segment of band b in block i is slot i + b (unique, in order)
   for (int b = npix > 0 ? beg / a.HWp : a.P; b < a.P && b * a.HWp < end; ++b) {
     const int lo = max(beg, b * a.HWp) - beg, hi = min(end, (b + 1) * a.HWp) - beg;
     float sum[V], sq[V];
@@ -387,10 +438,13 @@ __global__ void __launch_bounds__(1024, 1) gn_fused_kernel(
           sq[j] = fmaf(t[j], t[j], sq[j]);
         }
       }
+      // 16-byte stores: scalar ones at this stride would conflict 8-way
 #pragma unroll
-      for (int j = 0; j < V; ++j) {
-        ssum[pl * a.C + v * V + j] = sum[j];
-        ssq[pl * a.C + v * V + j] = sq[j];
+      for (int j = 0; j < V; j += 4) {
+        *reinterpret_cast<float4*>(ssum + pl * a.C + v * V + j) =
+            make_float4(sum[j], sum[j + 1], sum[j + 2], sum[j + 3]);
+        *reinterpret_cast<float4*>(ssq + pl * a.C + v * V + j) =
+            make_float4(sq[j], sq[j + 1], sq[j + 2], sq[j + 3]);
       }
     }
     __syncthreads();
@@ -405,59 +459,69 @@ __global__ void __launch_bounds__(1024, 1) gn_fused_kernel(
     }
     __syncthreads();
     for (int g = threadIdx.x; g < a.G; g += blockDim.x) {
-      double ds = 0.0, dq = 0.0;
+      float ds = 0.f, dq = 0.f;
       for (int c = g * cg; c < (g + 1) * cg; ++c) {
         ds += ssum[c];
         dq += ssq[c];
       }
-      atomicAdd(acc + (b * a.G + g) * kAccStride, ds);
-      atomicAdd(acc + (b * a.G + g) * kAccStride + 1, dq);
+      __stcg(part + static_cast<size_t>(blockIdx.x + b) * a.G + g, make_float2(ds, dq));
     }
     __syncthreads();
   }
 
-  // ---- grid barrier (count, generation), bounded
+  // ---- grid barrier (count, generation), bounded.  The arrival releases
+  // this block's partials; the last block opens the barrier by bumping the
+  // generation and only then clears the count (the next launch on this
+  // workspace starts after this one has finished).
   if (threadIdx.x == 0) {
     s_ok = 1;
-    volatile unsigned* gen = bar + 1;
-    const unsigned my_gen = *gen;
-    __threadfence();
-    if (atomicAdd(bar, 1u) == gridDim.x - 1) {
+    const unsigned my_gen = ld_acquire_gpu(bar + 1);
+    if (atom_add_release_gpu(bar, 1u) == gridDim.x - 1) {
+      st_release_gpu(bar + 1, my_gen + 1u);
       bar[0] = 0u;
-      __threadfence();
-      atomicAdd(bar + 1, 1u);
     } else {
       const unsigned long long t0 = globaltimer_ns();
-      while (*gen == my_gen) {
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      uint32_t n = 0;
+      while (ld_acquire_gpu(bar + 1) == my_gen) {
+        if ((++n & 63u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
           atomicExch(status, DP_ERR_TIMEOUT);
           s_ok = 0;
           break;
         }
-        __nanosleep(64);
       }
     }
-    __threadfence();
   }
   __syncthreads();
   if (!s_ok) return;
 
-  // ---- moments (every block), outputs (block 0), accumulator reset (last reader)
-  const double n = static_cast<double>(a.HWp) * cg;
-  for (int i = threadIdx.x; i < a.P * a.G * 2; i += blockDim.x)
-    f[i] = __ldcg(acc + (i >> 1) * kAccStride + (i & 1)) / n;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    if (atomicAdd(bar + 2, 1u) == gridDim.x - 1) {
-      for (int i = 0; i < a.P * a.G; ++i) {
-        acc[i * kAccStride] = 0.0;
-        acc[i * kAccStride + 1] = 0.0;
+  // ---- fresh moments of every band: the partials are staged in shared
+  // memory with independent coalesced loads (transposed to [group][slot]),
+  // then one thread per (band, group) sums its segments in fp64 in order
+  {
+    const int nslots = gridDim.x + a.P - 1;
+    const int total = nslots * a.G;
+#pragma unroll 4
+    for (int k = threadIdx.x; k < total; k += blockDim.x) {
+      const int slot = k / a.G, g = k - slot * a.G;
+      stage[g * nslots + slot] = __ldcg(part + k);
+    }
+    __syncthreads();
+    const double n = static_cast<double>(a.HWp) * cg;
+    for (int pg = threadIdx.x; pg < a.P * a.G; pg += blockDim.x) {
+      const int b = pg / a.G, g = pg - b * a.G;
+      const int i_lo = (b * a.HWp) / a.chunk, i_hi = ((b + 1) * a.HWp - 1) / a.chunk;
+      const float2* row = stage + g * nslots + b;
+      double s1 = 0.0, s2 = 0.0;
+      for (int i = i_lo; i <= i_hi; ++i) {
+        const float2 pv = row[i];
+        s1 += pv.x;
+        s2 += pv.y;
       }
-      bar[2] = 0u;
-      __threadfence();
+      f[2 * pg] = s1 / n;
+      f[2 * pg + 1] = s2 / n;
     }
   }
+  __syncthreads();
   if (blockIdx.x == 0) {
     for (int i = threadIdx.x; i < a.P * a.G; i += blockDim.x) {
       double m1, var, gm1, gm2;
@@ -474,16 +538,17 @@ __global__ void __launch_bounds__(1024, 1) gn_fused_kernel(
     }
   }
 
-  // ---- apply in shared memory, band segment by band segment, then store
+  // ---- apply: normalise from shared memory, store straight to y with
+  // coalesced 16-byte stores (consecutive threads, consecutive vectors)
   for (int b = npix > 0 ? beg / a.HWp : a.P; b < a.P && b * a.HWp < end; ++b) {
     const int lo = max(beg, b * a.HWp) - beg, hi = min(end, (b + 1) * a.HWp) - beg;
     for (int c = threadIdx.x; c < a.C; c += blockDim.x) {
       double m1, var, gm1, gm2;
       gn_used_moments(f, b, c / cg, a.P, a.G, a.mode, a.w, stale_global, stale_local, &m1, &var,
                       &gm1, &gm2);
-      const float sc = rsqrtf(static_cast<float>(var) + a.eps) * gamma[c];
+      const float sc = rsqrtf(static_cast<float>(var) + a.eps) * sgamma[c];
       sscale[c] = sc;
-      sshift[c] = beta[c] - static_cast<float>(m1) * sc;
+      sshift[c] = sbeta[c] - static_cast<float>(m1) * sc;
     }
     __syncthreads();
     if (worker) {
@@ -493,28 +558,17 @@ __global__ void __launch_bounds__(1024, 1) gn_fused_kernel(
         sc[j] = sscale[v * V + j];
         sh[j] = sshift[v * V + j];
       }
+      T* yb = y + static_cast<size_t>(beg) * a.C + v * V;
       for (int pix = lo + pl; pix < hi; pix += a.lanes) {
-        T* p = data + static_cast<size_t>(pix) * a.C + v * V;
         float t[V];
-        Vec<T>::load(p, t);
+        Vec<T>::load(data + static_cast<size_t>(pix) * a.C + v * V, t);
 #pragma unroll
-        for (int j = 0; j < V; ++j) {
-          float z = fmaf(t[j], sc[j], sh[j]);
-          if (a.silu) z = __fdividef(z, 1.0f + __expf(-z));
-          t[j] = z;
-        }
-        Vec<T>::store(p, t);
+        for (int j = 0; j < V; ++j) t[j] = fmaf(t[j], sc[j], sh[j]);
+        if (a.silu) silu_vec<T>(t);
+        Vec<T>::store(yb + static_cast<size_t>(pix) * a.C, t);
       }
     }
-    __syncthreads();
-  }
-  if (threadIdx.x == 0 && npix > 0) {
-    fence_proxy_async_smem();
-    const uint32_t total = static_cast<uint32_t>(npix) * a.C * sizeof(T);
-    char* dst = reinterpret_cast<char*>(y + static_cast<size_t>(beg) * a.C);
-    const char* src = reinterpret_cast<const char*>(data);
-    for (uint32_t off = 0; off < total; off += 16384u) bulk_store(dst + off, src + off, min(16384u, total - off));
-    bulk_commit_and_wait_all();
+    __syncthreads();   // sscale/sshift are rewritten for the next segment
   }
 }
 
@@ -555,9 +609,22 @@ static int gn_validate(const void* x, const void* y, int H, int W, int C, int G,
   return DP_OK;
 }
 
-size_t gn_workspace_bytes(int P, int G) {
+// Workspace: [0, 256) completion ticket and grid-barrier words, then the
+// fp64 accumulator of the two-kernel path (its size is gn_acc_bytes; both
+// are left zero by every call that completes), then the fp32 partial sums
+// of the single-pass path (one (sum, sum of squares) pair per group for each
+// of at most kGnFusedMaxBlocks + P band segments; no initialisation needed).
+constexpr int kGnFusedMaxBlocks = 160;
+
+size_t gn_acc_bytes(int P, int G) {
   return 256 + static_cast<size_t>(P) * G * kAccStride * sizeof(double);
 }
+
+static size_t gn_partial_bytes(int P, int G) {
+  return static_cast<size_t>(kGnFusedMaxBlocks + P) * G * sizeof(float2);
+}
+
+size_t gn_workspace_bytes(int P, int G) { return gn_acc_bytes(P, G) + gn_partial_bytes(P, G); }
 
 // Plan of the single-pass variant: blocks, chunk and shared memory; false if
 // the tensor does not fit.  Shared with the launch counter of the block step.
@@ -567,16 +634,14 @@ bool gn_fused_plan(int H, int W, int C, int G, int P, int dtype, int* blocks, in
   const int V = 16 / e;
   const int vpp = C / V;
   if (vpp > 1024) return false;
-  int lanes = vpp >= 512 ? 1 : 512 / vpp;
-  if (vpp * lanes > 1024) lanes = 1024 / vpp;
+  const int lanes = 1024 / vpp;
   const long HW = static_cast<long>(H) * W;
-  const int nb = num_sms();
+  const int nb = std::min(num_sms(), kGnFusedMaxBlocks);
   const long ch = (HW + nb - 1) / nb;
   const size_t data = ((static_cast<size_t>(ch) * C * e) + 127) & ~size_t(127);
   const size_t need = data + static_cast<size_t>(lanes) * C * 8 + static_cast<size_t>(P) * G * 16 +
-                      static_cast<size_t>(C) * 8;
+                      static_cast<size_t>(C) * 16 + static_cast<size_t>(nb + P) * G * 8;
   if (need > 200 * 1024) return false;
-  if ((static_cast<size_t>(ch) * C * e) % 16) return false;
   *blocks = static_cast<int>((HW + ch - 1) / ch);
   *chunk = static_cast<int>(ch);
   *threads = ((vpp * lanes + 31) / 32) * 32;
@@ -589,7 +654,7 @@ bool gn_fused_plan(int H, int W, int C, int G, int P, int dtype, int* blocks, in
 static bool gn_fused_launch(const void* x, void* y, const float* gamma, const float* beta, int H,
                             int W, int C, int G, int P, float eps, float w, int silu, int mode,
                             int dtype, const float* stale_global, const float* stale_local,
-                            float* fresh_local, float* fresh_global, float* used, double* acc,
+                            float* fresh_local, float* fresh_global, float* used, float2* part,
                             unsigned* bar, cudaStream_t stream, int* rc) {
   int blocks, chunk, threads;
   size_t smem;
@@ -612,8 +677,7 @@ static bool gn_fused_launch(const void* x, void* y, const float* gamma, const fl
   a.G = G;
   a.P = P;
   a.vpp = C / (dtype == DP_BF16 ? 8 : 4);
-  a.lanes = a.vpp >= 512 ? 1 : 512 / a.vpp;
-  if (a.vpp * a.lanes > 1024) a.lanes = 1024 / a.vpp;
+  a.lanes = 1024 / a.vpp;
   a.chunk = chunk;
   a.eps = eps;
   a.w = w;
@@ -621,7 +685,7 @@ static bool gn_fused_launch(const void* x, void* y, const float* gamma, const fl
   a.mode = mode;
   int* status = device_status_ptr();
   void* args[] = {const_cast<void**>(&x), &y, const_cast<float**>(&gamma), const_cast<float**>(&beta),
-                  &a, &acc, &bar, const_cast<float**>(&stale_global), const_cast<float**>(&stale_local),
+                  &a, &part, &bar, const_cast<float**>(&stale_global), const_cast<float**>(&stale_local),
                   &fresh_local, &fresh_global, &used, &status};
   mark_launch(stream);
   *rc = cuda_check(cudaLaunchCooperativeKernel(fn, dim3(blocks), dim3(threads), args, smem, stream),
@@ -633,7 +697,8 @@ static bool gn_fused_launch(const void* x, void* y, const float* gamma, const fl
 int gn_launch(const void* x, void* y, const float* gamma, const float* beta, int H, int W, int C,
               int G, int P, float eps, float w, int silu, int mode, int dtype,
               const float* stale_global, const float* stale_local, float* fresh_local,
-              float* fresh_global, float* used, void* workspace, cudaStream_t stream) {
+              float* fresh_global, float* used, void* workspace, size_t workspace_bytes,
+              cudaStream_t stream) {
   GnArgs a;
   gn_plan(H, W, C, G, P, dtype, &a);
   a.eps = eps;
@@ -644,8 +709,10 @@ int gn_launch(const void* x, void* y, const float* gamma, const float* beta, int
   double* acc = reinterpret_cast<double*>(static_cast<char*>(workspace) + 256);
   {
     int rc = 0;
-    if (gn_fused_launch(x, y, gamma, beta, H, W, C, G, P, eps, w, silu, mode, dtype, stale_global,
-                        stale_local, fresh_local, fresh_global, used, acc, counter + 4, stream,
+    float2* part = reinterpret_cast<float2*>(static_cast<char*>(workspace) + gn_acc_bytes(P, G));
+    if (workspace_bytes >= gn_workspace_bytes(P, G) &&
+        gn_fused_launch(x, y, gamma, beta, H, W, C, G, P, eps, w, silu, mode, dtype, stale_global,
+                        stale_local, fresh_local, fresh_global, used, part, counter + 4, stream,
                         &rc))
       return rc;
   }
@@ -744,12 +811,12 @@ int dp_groupnorm_async(const void* x, void* y, const float* gamma, const float* 
     return dp::set_error(DP_ERR_INVALID_ARG, "groupnorm: null gamma/beta/fresh_local/used/workspace");
   if (mode == DP_MODE_DISPLACED && (!stale_global || !stale_local))
     return dp::set_error(DP_ERR_INVALID_ARG, "groupnorm: displaced mode needs stale statistics");
-  if (workspace_bytes < dp::gn_workspace_bytes(P, G))
+  if (workspace_bytes < dp::gn_acc_bytes(P, G))
     return dp::set_error(DP_ERR_INVALID_ARG, "groupnorm: workspace too small (%zu < %zu)",
-                         workspace_bytes, dp::gn_workspace_bytes(P, G));
+                         workspace_bytes, dp::gn_acc_bytes(P, G));
   if (!(eps > 0.f)) return dp::set_error(DP_ERR_INVALID_ARG, "groupnorm: eps must be > 0");
   return dp::gn_launch(x, y, gamma, beta, H, W, C, G, P, eps, w, silu, mode, dtype, stale_global,
-                       stale_local, fresh_local, nullptr, used_stats, workspace,
+                       stale_local, fresh_local, nullptr, used_stats, workspace, workspace_bytes,
                        static_cast<cudaStream_t>(stream));
 }
 
@@ -765,7 +832,7 @@ int dp_groupnorm_async_noalloc(const void* x, void* y, const float* gamma, const
   if (mode == DP_MODE_DISPLACED && (!stale_global || !stale_local))
     return dp::set_error(DP_ERR_INVALID_ARG, "noalloc groupnorm: displaced mode needs stale statistics");
   if (!(eps > 0.f)) return dp::set_error(DP_ERR_INVALID_ARG, "noalloc groupnorm: eps must be > 0");
-  const size_t need = dp::gn_workspace_bytes(P, G);
+  const size_t need = dp::gn_acc_bytes(P, G);
   if (need > dp::kGnStaticScratchBytes)
     return dp::set_error(DP_ERR_UNSUPPORTED,
                          "noalloc groupnorm: P=%d, G=%d needs %zu bytes of scratch; the static "
@@ -780,7 +847,8 @@ int dp_groupnorm_async_noalloc(const void* x, void* y, const float* gamma, const
   rc = dp::cuda_check(cudaMemsetAsync(scratch, 0, need, s), "noalloc groupnorm: clear scratch");
   if (rc) return rc;
   return dp::gn_launch(x, y, gamma, beta, H, W, C, G, P, eps, w, silu, mode, dtype, stale_global,
-                       stale_local, fresh_local, nullptr, used_stats, scratch, s);
+                       stale_local, fresh_local, nullptr, used_stats, scratch,
+                       dp::kGnStaticScratchBytes, s);
 }
 
 }  // extern "C"

@@ -6,13 +6,15 @@
 
 namespace dp {
 
+size_t gn_acc_bytes(int P, int G);
 size_t gn_workspace_bytes(int P, int G);
 bool gn_fused_plan(int H, int W, int C, int G, int P, int dtype, int* blocks, int* chunk,
                    int* threads, size_t* smem);
 int gn_launch(const void* x, void* y, const float* gamma, const float* beta, int H, int W, int C,
               int G, int P, float eps, float w, int silu, int mode, int dtype,
               const float* stale_global, const float* stale_local, float* fresh_local,
-              float* fresh_global, float* used, void* workspace, cudaStream_t stream);
+              float* fresh_global, float* used, void* workspace, size_t workspace_bytes,
+              cudaStream_t stream);
 int conv3x3_validate(const void* a_fresh, const void* a_stale, const void* weight,
                      const void* residual, const void* out, int H, int W, int Cin, int Cout,
                      int stride, int P, int mode, int dtype);

@@ -118,10 +118,19 @@ DP_API int dp_device_status(void* stream, int* status);
  *  stale_local  [P][G][2] fp32, device; read in DISPLACED only
  *  fresh_local  [P][G][2] fp32, device, written: f (the next step's stale_local)
  *  used_stats   [P][G][2] fp32 (mean, var), device, written
- *  workspace    device scratch of dp_groupnorm_workspace_size() bytes; it must
- *               be zero-filled before its first use and is left zero-filled
- *               by every call that completes.  Calls that overlap on the GPU
- *               must not share a workspace.
+ *  workspace    device scratch of dp_groupnorm_workspace_size() bytes.  Its
+ *               first 256 + 128 * P * G bytes must be zero-filled before its
+ *               first use and are left zero-filled by every call that
+ *               completes; the rest holds per-block partial sums and needs no
+ *               initialisation.  A workspace of at least 256 + 128 * P * G
+ *               bytes but smaller than the full size is accepted and runs the
+ *               two-kernel path.  Calls that overlap on the GPU must not share
+ *               a workspace.
+ *  workspace_bytes  its size; smaller than 256 + 128 * P * G is an error.
+ * Errors: DP_ERR_INVALID_ARG (null pointer, bad mode/dtype, eps <= 0, small
+ * workspace), DP_ERR_UNSUPPORTED (shape limits below, unaligned x/y).
+ * SiLU uses the hardware base-2 exponential and a Newton reciprocal (relative
+ * error below 1e-5 before the cast).
  * Needs C % G == 0, C % 8 == 0 (bf16) or C % 4 == 0 (fp32), C/8 <= 1024.
  * ---------------------------------------------------------------------- */
 DP_API size_t dp_groupnorm_workspace_size(int H, int W, int C, int G, int P);
