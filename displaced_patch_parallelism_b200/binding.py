@@ -57,7 +57,8 @@ _SIGS = {
     "dp_conv3x3_halo": ([_V, _V, _V, _V, _V, _V, _I, _I, _I, _I, _I, _I, _I, _I, _V], _I),
     "dp_conv3x3_halo_small": ([_V, _V, _V, _V, _V, _I, _I, _I, _I, _I, _I, _V], _I),
     "dp_linear": ([_V, _V, _V, _V, _V, _V, _V, _I, _I, _I, _I, _V], _I),
-    "dp_attn_stale_kv": ([_V, _V, _V, _V, _V, _V, _I, _I, _I, _I, _F, _I, _V], _I),
+    "dp_attn_workspace_size": ([], _SZ),
+    "dp_attn_stale_kv": ([_V, _V, _V, _V, _V, _V, _I, _I, _I, _I, _F, _I, _V, _SZ, _V], _I),
     "dp_refresh_stale": ([_V, _V, _SZ, _I, _I, _I, _V], _I),
     "dp_refresh_stats": ([_V, _V, _V, _I, _I, _V], _I),
     "dp_block_desc_init": ([ctypes.POINTER(BlockDesc), _I, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _F], _I),
@@ -176,11 +177,15 @@ def dp_linear(x, weight, bias, residual, out0, out1, out2, M, N, K, split, strea
                                   _p(out2), M, N, K, split, _s(stream)))
 
 
+def dp_attn_workspace_size():
+    return lib().dp_attn_workspace_size()
+
+
 def dp_attn_stale_kv(q, k_fresh, v_fresh, k_stale, v_stale, o, T, heads, head_dim, P, scale,
-                     mode, stream=None):
+                     mode, workspace=None, workspace_bytes=0, stream=None):
     return _check(lib().dp_attn_stale_kv(_p(q), _p(k_fresh), _p(v_fresh), _p(k_stale),
                                          _p(v_stale), _p(o), T, heads, head_dim, P, scale, mode,
-                                         _s(stream)))
+                                         _p(workspace), workspace_bytes, _s(stream)))
 
 
 def dp_refresh_stale(fresh, stale, row_bytes, rows, P, band=-1, stream=None):

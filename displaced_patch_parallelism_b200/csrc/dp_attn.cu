@@ -33,9 +33,18 @@ namespace dp {
 struct AttnParams {
   CUtensorMap tmQ, tmKf, tmVf, tmKs, tmVs;
   int T, heads, P, tb, mode;
+  // Work split: a unit is 128 queries of one head (units ordered head-major);
+  // it takes n_kv key tiles.  CTA b owns the iterations [b L, (b+1) L) of the
+  // W = units x n_kv (unit, key tile) iterations.
+  int n_qt, n_kv, W, L;
   float scale_log2;
   __nv_bfloat16* o;
   int ld;
+  // Partials of units cut between CTAs: slot 2b + 1 holds CTA b's last
+  // segment when it is a unit's start, slot 2b its first segment otherwise;
+  // each slot is 8 warp slices of 32 rows x (32 O columns, m, l, 2 pad).
+  float* part;
+  unsigned* count;          // [grid][8]: parts of the unit starting in CTA b done so far
   int* status;
 };
 
@@ -43,7 +52,22 @@ constexpr int kAttnStages = 2;
 constexpr int kTile = 16384;                     // 128 rows x 128 bytes
 constexpr int kAttnThreads = 320;               // producer, MMA, 8 softmax warps
 constexpr int kAttnTail = 4096;                  // barriers + max/sum exchange buffers
-constexpr int kAttnSmem = kTile * (1 + 2 * kAttnStages) + 1024 + kAttnTail;
+constexpr int kAttnSmem = kTile * (2 + 2 * kAttnStages) + 1024 + kAttnTail;
+constexpr int kSliceFloats = 32 * 36;           // one warp's 32 rows x (32 O, m, l, pad)
+constexpr int kSlotFloats = 8 * kSliceFloats;
+
+// The next run of consecutive key tiles of one unit in this CTA's range.
+struct AttnSeg {
+  int u, k0, k1;
+};
+__device__ __forceinline__ bool attn_next_seg(const AttnParams& p, int& it, int end, AttnSeg& s) {
+  if (it >= end) return false;
+  s.u = it / p.n_kv;
+  s.k0 = it - s.u * p.n_kv;
+  s.k1 = min(p.n_kv, s.k0 + (end - it));
+  it += s.k1 - s.k0;
+  return true;
+}
 
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
@@ -124,33 +148,35 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_kernel(const __grid_cons
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = smem + kTile;
+  uint8_t* sQ = smem;                                           // [2] query tiles
+  uint8_t* sK = smem + 2 * kTile;
   uint8_t* sV = sK + kAttnStages * kTile;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sV + kAttnStages * kTile);
-  uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;
+  uint64_t* q_full = bars;                                      // [2]
+  uint64_t* q_empty = q_full + 2;                               // [2]
+  uint64_t* kv_full = q_empty + 2;
   uint64_t* kv_empty = kv_full + kAttnStages;
   uint64_t* s_full = kv_empty + kAttnStages;
   uint64_t* s_free = s_full + 1;
   uint64_t* p_full = s_free + 1;
   uint64_t* o_done = p_full + 1;
-  uint64_t* drain = o_done + 1;
+  uint64_t* o_free = o_done + 1;
+  uint64_t* drain = o_free + 1;
   uint64_t* xbar = drain + 1;                                   // [4], one per row quarter
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xbar + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* red = reinterpret_cast<float*>(bars + 64);             // [2 parities][2 halves][128]
 
   const int warp = warp_id(), lane = lane_id();
-  const int qtile = blockIdx.x, h = blockIdx.y;
-  const int q0 = qtile * 128;
-  const int band = q0 / p.tb;
   const int band_tiles = p.tb / 128;
-  const int n_kv = p.mode == DP_MODE_NAIVE ? band_tiles : p.T / 128;
-  const int first_kv = p.mode == DP_MODE_NAIVE ? band * band_tiles : 0;
+  const int start = blockIdx.x * p.L;
+  const int end = min(p.W, start + p.L);
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&q_full[b], 1);
+      mbar_init(&q_empty[b], 1);
+    }
     for (int s = 0; s < kAttnStages; ++s) {
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
@@ -158,8 +184,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_kernel(const __grid_cons
     mbar_init(s_full, 1);
     mbar_init(s_free, 8);
     mbar_init(p_full, 8);
-    for (int i = 0; i < 4; ++i) mbar_init(&xbar[i], 2);
     mbar_init(o_done, 1);
+    mbar_init(o_free, 8);
+    for (int i = 0; i < 4; ++i) mbar_init(&xbar[i], 2);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -177,32 +204,47 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_kernel(const __grid_cons
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ producer
-      uint32_t issued = 0, issued_par = 0;
-      bool q_issued = false;
-      int stage = 0;
-      uint32_t phase = 0;
-      mbar_arrive_expect_tx(q_full, kTile);
-      tma_load_2d(sQ, &p.tmQ, q_full, h * 64, q0);
-      q_issued = true;
-      for (int j = 0; j < n_kv; ++j) {
-        const int t = first_kv + j;
-        const bool own = (t * 128) / p.tb == band;
-        const bool stale = !own && p.mode == DP_MODE_DISPLACED;
-        if (!mbar_wait(&kv_empty[stage], phase ^ 1u, abort_flag, p.status)) break;
-        mbar_arrive_expect_tx(&kv_full[stage], 2 * kTile);
-        tma_load_2d(sK + stage * kTile, stale ? &p.tmKs : &p.tmKf, &kv_full[stage], h * 64, t * 128);
-        tma_load_2d(sV + stage * kTile, stale ? &p.tmVs : &p.tmVf, &kv_full[stage], h * 64, t * 128);
-        issued |= 1u << stage;
-        issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
-        if (++stage == kAttnStages) {
-          stage = 0;
-          phase ^= 1u;
+      uint32_t issued = 0, issued_par = 0;        // bits 0-1: K/V stages, 2-3: Q buffers
+      int stage = 0, qb = 0;
+      uint32_t phase = 0, qpar[2] = {0u, 0u};
+      int it = start;
+      AttnSeg sg;
+      while (attn_next_seg(p, it, end, sg)) {
+        const int h = sg.u / p.n_qt, q0 = (sg.u - h * p.n_qt) * 128;
+        const int band = q0 / p.tb;
+        const int first_kv = p.mode == DP_MODE_NAIVE ? band * band_tiles : 0;
+        if (!mbar_wait(&q_empty[qb], qpar[qb] ^ 1u, abort_flag, p.status)) break;
+        mbar_arrive_expect_tx(&q_full[qb], kTile);
+        tma_load_2d(sQ + qb * kTile, &p.tmQ, &q_full[qb], h * 64, q0);
+        issued |= 4u << qb;
+        issued_par = (issued_par & ~(4u << qb)) | (qpar[qb] << (2 + qb));
+        qpar[qb] ^= 1u;
+        qb ^= 1;
+        bool ok = true;
+        for (int j = sg.k0; j < sg.k1; ++j) {
+          const int t = first_kv + j;
+          const bool own = (t * 128) / p.tb == band;
+          const bool stale = !own && p.mode == DP_MODE_DISPLACED;
+          if (!mbar_wait(&kv_empty[stage], phase ^ 1u, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&kv_full[stage], 2 * kTile);
+          tma_load_2d(sK + stage * kTile, stale ? &p.tmKs : &p.tmKf, &kv_full[stage], h * 64, t * 128);
+          tma_load_2d(sV + stage * kTile, stale ? &p.tmVs : &p.tmVf, &kv_full[stage], h * 64, t * 128);
+          issued |= 1u << stage;
+          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == kAttnStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
         }
+        if (!ok) break;
       }
       if (*abort_flag) {
-        if (q_issued) attn_wait_teardown(q_full, 0);
-        for (int s = 0; s < kAttnStages; ++s)
-          if (issued & (1u << s)) attn_wait_teardown(&kv_full[s], (issued_par >> s) & 1u);
+        for (int s = 0; s < 4; ++s)
+          if (issued & (1u << s))
+            attn_wait_teardown(s < 2 ? &kv_full[s] : &q_full[s - 2], (issued_par >> s) & 1u);
       }
     }
   } else if (warp == 1) {
@@ -210,38 +252,60 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_kernel(const __grid_cons
       // ------------------------------------------------------------ MMA issuer
       constexpr uint32_t idesc_qk = idesc_dense(128, 128, 1, 0, 0);
       constexpr uint32_t idesc_pv = idesc_dense(128, 64, 1, 0, 1);
-      const uint64_t qd = sdesc_sw128(smem_u32(sQ), 1024);
-      int stage = 0, prev_stage = 0;
-      uint32_t phase = 0;
-      bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
-      for (int j = 0; ok && j <= n_kv; ++j) {
-        if (j < n_kv) {
-          if (!mbar_wait(&kv_full[stage], phase, abort_flag, p.status)) break;
-          if (j > 0 && !mbar_wait(s_free, (j - 1) & 1, abort_flag, p.status)) break;
-          tc_fence_after();
-          const uint64_t kd = sdesc_sw128(smem_u32(sK + stage * kTile), 1024);
+      int stage = 0, prev_stage = 0, qb = 0;
+      uint32_t phase = 0, qpar[2] = {0u, 0u};
+      int t = 0, si = 0;       // key tiles and segments done by this CTA
+      int it = start;
+      AttnSeg sg;
+      bool ok = true;
+      while (ok && attn_next_seg(p, it, end, sg)) {
+        const int n = sg.k1 - sg.k0;
+        if (!mbar_wait(&q_full[qb], qpar[qb], abort_flag, p.status)) break;
+        qpar[qb] ^= 1u;
+        tc_fence_after();
+        const uint64_t qd = sdesc_sw128(smem_u32(sQ + qb * kTile), 1024);
+        for (int jj = 0; jj <= n; ++jj) {
+          const int tt = t + jj;
+          if (jj < n) {
+            if (!mbar_wait(&kv_full[stage], phase, abort_flag, p.status) ||
+                (tt > 0 && !mbar_wait(s_free, (tt - 1) & 1, abort_flag, p.status))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t kd = sdesc_sw128(smem_u32(sK + stage * kTile), 1024);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) umma_f16_ss(tS, qd + 2 * k, kd + 2 * k, idesc_qk, k != 0);
-          umma_commit(s_full);
-        }
-        if (j > 0) {
-          // O += P_{j-1} V_{j-1}
-          if (!mbar_wait(p_full, (j - 1) & 1, abort_flag, p.status)) break;
-          tc_fence_after();
-          const uint64_t vd = sdesc_sw128(smem_u32(sV + prev_stage * kTile), 1024);
+            for (int k = 0; k < 4; ++k) umma_f16_ss(tS, qd + 2 * k, kd + 2 * k, idesc_qk, k != 0);
+            umma_commit(s_full);
+            if (jj == n - 1) umma_commit(&q_empty[qb]);   // this segment's last read of Q
+          }
+          if (jj > 0) {
+            // O += P V of the previous key tile; the segment's first one
+            // overwrites O, so the softmax warps must have read the last O
+            if (!mbar_wait(p_full, (tt - 1) & 1, abort_flag, p.status) ||
+                (jj == 1 && si > 0 && !mbar_wait(o_free, (si - 1) & 1, abort_flag, p.status))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t vd = sdesc_sw128(smem_u32(sV + prev_stage * kTile), 1024);
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            umma_f16_ts(tO, tP + 8 * k, vd + 128 * k, idesc_pv, (j > 1 || k != 0));
-          umma_commit(&kv_empty[prev_stage]);
-          umma_commit(o_done);
-        }
-        if (j < n_kv) {
-          prev_stage = stage;
-          if (++stage == kAttnStages) {
-            stage = 0;
-            phase ^= 1u;
+            for (int k = 0; k < 8; ++k)
+              umma_f16_ts(tO, tP + 8 * k, vd + 128 * k, idesc_pv, (jj > 1 || k != 0));
+            umma_commit(&kv_empty[prev_stage]);
+            umma_commit(o_done);
+          }
+          if (jj < n) {
+            prev_stage = stage;
+            if (++stage == kAttnStages) {
+              stage = 0;
+              phase ^= 1u;
+            }
           }
         }
+        t += n;
+        ++si;
+        qb ^= 1;
       }
       if (*abort_flag) {
         umma_commit(drain);
@@ -253,123 +317,200 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_kernel(const __grid_cons
     // Warps w and w+4 share TMEM lanes 32*(w%4).. (the same 32 query rows)
     // and split each row's 128 scores into halves, so 8 warps exponentiate.
     // Per tile they exchange their half-row maxima through shared memory
-    // (double-buffered by tile parity, bounded mbarrier waits); each half
+    // (double-buffered by use parity, bounded mbarrier waits); each half
     // keeps its own partial row sum and owns 32 of the 64 output columns.
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
     const int row = q * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     const float c = p.scale_log2;
-    float m_used = 0.f, l = 0.f;
     bool aborted = false;
-    auto exchange = [&](int use, float mine, float* other) -> bool {
-      float* buf = red + (use & 1) * 256;
+    uint32_t xuse = 0;
+    auto exchange = [&](float mine, float* other) -> bool {
+      float* buf = red + (xuse & 1) * 256;
       buf[half * 128 + row] = mine;
       __syncwarp();
       if (lane == 0) mbar_arrive(&xbar[q]);
-      if (!mbar_wait(&xbar[q], use & 1, abort_flag, p.status)) return false;
+      const bool ok = mbar_wait(&xbar[q], xuse & 1, abort_flag, p.status);
+      ++xuse;
+      if (!ok) return false;
       *other = buf[(half ^ 1) * 128 + row];
       return true;
     };
-    for (int j = 0; j < n_kv; ++j) {
-      if (!mbar_wait(s_full, j & 1, abort_flag, p.status)) {
-        aborted = true;
-        break;
-      }
-      tc_fence_after();
-      uint32_t s[2][32];
-      tmem_ld32(tS + lane_off + half * 64, s[0]);
-      tmem_ld32(tS + lane_off + half * 64 + 32, s[1]);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_free);
-      float mx = __uint_as_float(s[0][0]);
-#pragma unroll
-      for (int k = 0; k < 2; ++k)
-#pragma unroll
-        for (int i = 0; i < 32; i += 2)
-          mx = max3(mx, __uint_as_float(s[k][i]), __uint_as_float(s[k][i + 1]));
-      float mo;
-      if (!exchange(j, mx, &mo)) {
-        aborted = true;
-        break;
-      }
-      const float m_tile = fmaxf(mx, mo) * c;
-      float alpha = 1.f;
-      if (j == 0) {
-        m_used = m_tile;
-      } else if (m_tile > m_used + 8.f) {
-        alpha = ex2_approx(m_used - m_tile);
-        m_used = m_tile;
-      }
-      // P_j = exp2(s * c - m_used), packed bf16 pairs.  3 of every 8 pairs take
-      // the FMA-pipe exponential, the rest the special-function unit.
-      uint32_t pk[32];
-      const uint64_t c2 = f2_pack(c, c), negm2 = f2_pack(-m_used, -m_used);
-      uint64_t sum2 = f2_pack(0.f, 0.f);
-#pragma unroll
-      for (int k = 0; k < 2; ++k)
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const uint64_t x2 =
-              f2_fma(f2_pack(__uint_as_float(s[k][2 * i]), __uint_as_float(s[k][2 * i + 1])), c2, negm2);
-          float e0, e1;
-          if ((i & 7) < 3) {
-            exp2_poly_x2(x2, e0, e1);
-          } else {
-            float x0, x1;
-            f2_unpack(x2, x0, x1);
-            e0 = ex2_approx(x0);
-            e1 = ex2_approx(x1);
-          }
-          sum2 = f2_add(sum2, f2_pack(e0, e1));
-          pk[k * 16 + i] = pack_bf16x2(e0, e1);
-        }
-      float rs0, rs1;
-      f2_unpack(sum2, rs0, rs1);
-      l = l * alpha + (rs0 + rs1);
-      if (j > 0) {
-        // P_{j-1} V_{j-1} must be done before O is rescaled or P overwritten
-        if (!mbar_wait(o_done, (j - 1) & 1, abort_flag, p.status)) {
+    int t = 0;
+    int it = start;
+    AttnSeg sg;
+    while (!aborted && attn_next_seg(p, it, end, sg)) {
+      const int n = sg.k1 - sg.k0;
+      float m_used = 0.f, l = 0.f;
+      for (int jj = 0; jj < n; ++jj) {
+        const int tt = t + jj;
+        if (!mbar_wait(s_full, tt & 1, abort_flag, p.status)) {
           aborted = true;
           break;
         }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
-          uint32_t o[32];
-          tmem_ld32(tO + lane_off + half * 32, o);
-          tmem_wait_ld();
+        uint32_t s[2][32];
+        tmem_ld32(tS + lane_off + half * 64, s[0]);
+        tmem_ld32(tS + lane_off + half * 64 + 32, s[1]);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free);
+        float mx = __uint_as_float(s[0][0]);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tO + lane_off + half * 32, o);
+        for (int k = 0; k < 2; ++k)
+#pragma unroll
+          for (int i = 0; i < 32; i += 2)
+            mx = max3(mx, __uint_as_float(s[k][i]), __uint_as_float(s[k][i + 1]));
+        float mo;
+        if (!exchange(mx, &mo)) {
+          aborted = true;
+          break;
         }
+        const float m_tile = fmaxf(mx, mo) * c;
+        float alpha = 1.f;
+        if (jj == 0) {
+          m_used = m_tile;
+        } else if (m_tile > m_used + 8.f) {
+          alpha = ex2_approx(m_used - m_tile);
+          m_used = m_tile;
+        }
+        // P = exp2(s * c - m_used), packed bf16 pairs.  3 of every 8 pairs take
+        // the FMA-pipe exponential, the rest the special-function unit.
+        uint32_t pk[32];
+        const uint64_t c2 = f2_pack(c, c), negm2 = f2_pack(-m_used, -m_used);
+        uint64_t sum2 = f2_pack(0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const uint64_t x2 =
+                f2_fma(f2_pack(__uint_as_float(s[k][2 * i]), __uint_as_float(s[k][2 * i + 1])), c2, negm2);
+            float e0, e1;
+            if ((i & 7) < 3) {
+              exp2_poly_x2(x2, e0, e1);
+            } else {
+              float x0, x1;
+              f2_unpack(x2, x0, x1);
+              e0 = ex2_approx(x0);
+              e1 = ex2_approx(x1);
+            }
+            sum2 = f2_add(sum2, f2_pack(e0, e1));
+            pk[k * 16 + i] = pack_bf16x2(e0, e1);
+          }
+        float rs0, rs1;
+        f2_unpack(sum2, rs0, rs1);
+        l = l * alpha + (rs0 + rs1);
+        if (tt > 0) {
+          // the previous P V must be done before P is overwritten (and, inside
+          // a segment, before O is rescaled)
+          if (!mbar_wait(o_done, (tt - 1) & 1, abort_flag, p.status)) {
+            aborted = true;
+            break;
+          }
+          tc_fence_after();
+          if (jj > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+            uint32_t o[32];
+            tmem_ld32(tO + lane_off + half * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(tO + lane_off + half * 32, o);
+          }
+        }
+        tmem_st32(tP + lane_off + half * 32, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full);
       }
-      tmem_st32(tP + lane_off + half * 32, pk);
-      tmem_wait_st();
+      if (aborted) break;
+      // ---- end of the segment: O leaves tensor memory
+      float lo = 0.f;
+      if (!exchange(l, &lo) || !mbar_wait(o_done, (t + n - 1) & 1, abort_flag, p.status)) {
+        aborted = true;
+        break;
+      }
+      tc_fence_after();
+      float acc[32];
+      {
+        uint32_t o[32];
+        tmem_ld32(tO + lane_off + half * 32, o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) acc[i] = __uint_as_float(o[i]);
+      }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
-    }
-    float lo = 0.f;
-    if (!aborted && n_kv > 0 && exchange(n_kv, l, &lo) &&
-        mbar_wait(o_done, (n_kv - 1) & 1, abort_flag, p.status)) {
-      tc_fence_after();
-      uint32_t o[32];
-      tmem_ld32(tO + lane_off + half * 32, o);
-      tmem_wait_ld();
-      const float inv = 1.f / (l + lo);
+      if (lane == 0) mbar_arrive(o_free);
+      const float lsum = l + lo;
+      const int h = sg.u / p.n_qt, q0 = (sg.u - h * p.n_qt) * 128;
+      float inv;
+      if (sg.k0 == 0 && sg.k1 == p.n_kv) {
+        inv = 1.f / lsum;
+      } else {
+        // A unit cut between CTAs b_lo..b_hi.  Each part stores this warp's
+        // slice (unnormalised O, row max m in the log2 domain, row sum l);
+        // the part that finishes last merges the others into its registers
+        // and writes O.  Nothing waits on another CTA.
+        const int b_lo = (sg.u * p.n_kv) / p.L, b_hi = ((sg.u + 1) * p.n_kv - 1) / p.L;
+        const int me = blockIdx.x;
+        const int wslice = warp - 2;
+        auto slice = [&](int b) {
+          return p.part + (static_cast<size_t>(2 * b + (b == b_lo ? 1 : 0)) * kSlotFloats +
+                           static_cast<size_t>(wslice) * kSliceFloats + lane * 36);
+        };
+        float* mine = slice(me);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          reinterpret_cast<float4*>(mine)[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+        *reinterpret_cast<float2*>(mine + 32) = make_float2(m_used, lsum);
+        __syncwarp();
+        unsigned last = 0;
+        if (lane == 0) {
+          __threadfence();
+          last = atomicAdd(p.count + b_lo * 8 + wslice, 1u) == static_cast<unsigned>(b_hi - b_lo);
+        }
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (!last) {
+          t += n;
+          continue;
+        }
+        __threadfence();
+        float m = m_used, ls = lsum;
+        for (int b = b_lo; b <= b_hi; ++b) {
+          if (b == me) continue;
+          const float* pc = slice(b);
+          const float2 ml = __ldcg(reinterpret_cast<const float2*>(pc + 32));
+          const float mn = fmaxf(m, ml.x);
+          const float a0 = ex2_approx(m - mn), a1 = ex2_approx(ml.x - mn);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(pc) + i);
+            acc[4 * i] = fmaf(acc[4 * i], a0, v.x * a1);
+            acc[4 * i + 1] = fmaf(acc[4 * i + 1], a0, v.y * a1);
+            acc[4 * i + 2] = fmaf(acc[4 * i + 2], a0, v.z * a1);
+            acc[4 * i + 3] = fmaf(acc[4 * i + 3], a0, v.w * a1);
+          }
+          ls = fmaf(ls, a0, ml.y * a1);
+          m = mn;
+        }
+        if (lane == 0) p.count[b_lo * 8 + wslice] = 0u;   // ready for the next call
+        inv = 1.f / ls;
+      }
       uint4* dst = reinterpret_cast<uint4*>(p.o + static_cast<size_t>(q0 + row) * p.ld + h * 64 +
                                             half * 32);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         uint4 u;
-        u.x = pack_bf16x2(__uint_as_float(o[8 * i]) * inv, __uint_as_float(o[8 * i + 1]) * inv);
-        u.y = pack_bf16x2(__uint_as_float(o[8 * i + 2]) * inv, __uint_as_float(o[8 * i + 3]) * inv);
-        u.z = pack_bf16x2(__uint_as_float(o[8 * i + 4]) * inv, __uint_as_float(o[8 * i + 5]) * inv);
-        u.w = pack_bf16x2(__uint_as_float(o[8 * i + 6]) * inv, __uint_as_float(o[8 * i + 7]) * inv);
+        u.x = pack_bf16x2(acc[8 * i] * inv, acc[8 * i + 1] * inv);
+        u.y = pack_bf16x2(acc[8 * i + 2] * inv, acc[8 * i + 3] * inv);
+        u.z = pack_bf16x2(acc[8 * i + 4] * inv, acc[8 * i + 5] * inv);
+        u.w = pack_bf16x2(acc[8 * i + 6] * inv, acc[8 * i + 7] * inv);
         dst[i] = u;
       }
+      t += n;
     }
   }
 
@@ -382,8 +523,18 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_kernel(const __grid_cons
   }
 }
 
+// Workspace of the balanced launch: per-CTA part counters (zero before first
+// use; every call leaves them zero), then two partial slots per CTA.
+static size_t attn_count_bytes(size_t slots) { return (slots * 8 * sizeof(unsigned) + 255) & ~size_t(255); }
+
+size_t attn_workspace_bytes() {
+  const size_t slots = 2 * static_cast<size_t>(num_sms());
+  return attn_count_bytes(slots) + 2 * slots * kSlotFloats * sizeof(float);
+}
+
 int attn_launch(const void* q, const void* kf, const void* vf, const void* ks, const void* vs,
-                void* o, int T, int heads, int P, float scale, int mode, cudaStream_t stream) {
+                void* o, int T, int heads, int P, float scale, int mode, void* workspace,
+                size_t workspace_bytes, cudaStream_t stream) {
   AttnParams a;
   memset(&a, 0, sizeof(a));
   const int ld = heads * 64;
@@ -416,7 +567,34 @@ int attn_launch(const void* q, const void* kf, const void* vf, const void* ks, c
     if (rc) return rc;
     attr_mask |= 1 << (dev & 31);
   }
-  dim3 grid(T / 128, heads);
+  a.n_qt = T / 128;
+  a.n_kv = mode == DP_MODE_NAIVE ? a.tb / 128 : T / 128;
+  const int units = a.n_qt * heads;
+  a.W = units * a.n_kv;
+  // Two CTAs fit on an SM (shared and tensor memory; the hardware places two
+  // although the occupancy calculator's register model allows one).  Balanced
+  // split: every CTA takes an equal run of (unit, key tile) iterations; the
+  // parts of a unit cut between CTAs are merged by whichever finishes last,
+  // so no CTA waits on another and any residency is correct.  Without a
+  // workspace each CTA takes one whole unit.
+  const int slots = 2 * num_sms();
+  // Cost in key-tile iterations of a paired CTA: a CTA's fixed cost (launch,
+  // set-up, first loads, epilogue) is about 5 of them and each cut segment
+  // about 2 more (measured on B200).  Whole units take ceil(units / slots)
+  // rounds; the split takes one round of L iterations.
+  const int L_split = (a.W + slots - 1) / slots;
+  const double t_whole = static_cast<double>((units + slots - 1) / slots) * (a.n_kv + 5);
+  const double t_split = L_split + 5 + 4;
+  const bool split = workspace && workspace_bytes >= attn_workspace_bytes() && units % slots != 0 &&
+                     t_split < 0.85 * t_whole;
+  if (split) {
+    a.L = L_split;
+    a.count = static_cast<unsigned*>(workspace);
+    a.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + attn_count_bytes(slots));
+  } else {
+    a.L = a.n_kv;
+  }
+  const int grid = (a.W + a.L - 1) / a.L;
   mark_launch(stream);
   attn_kernel<<<grid, kAttnThreads, kAttnSmem, stream>>>(a);
   return cuda_check(cudaGetLastError(), "attention launch");
@@ -444,12 +622,16 @@ int attn_validate(const void* q, const void* kf, const void* vf, const void* ks,
 
 }  // namespace dp
 
+extern "C" size_t dp_attn_workspace_size(void) { return dp::attn_workspace_bytes(); }
+
 extern "C" int dp_attn_stale_kv(const void* q, const void* k_fresh, const void* v_fresh,
                                 const void* k_stale, const void* v_stale, void* o, int T,
                                 int heads, int head_dim, int P, float scale, int mode,
-                                void* stream) {
+                                void* workspace, size_t workspace_bytes, void* stream) {
   int rc = dp::attn_validate(q, k_fresh, v_fresh, k_stale, v_stale, o, T, heads, head_dim, P, mode);
   if (rc) return rc;
+  if (workspace && !dp::aligned16(workspace))
+    return dp::set_error(DP_ERR_UNSUPPORTED, "attention: workspace not 16-byte aligned");
   return dp::attn_launch(q, k_fresh, v_fresh, k_stale, v_stale, o, T, heads, P, scale, mode,
-                         static_cast<cudaStream_t>(stream));
+                         workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }

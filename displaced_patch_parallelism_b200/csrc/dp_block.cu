@@ -48,6 +48,7 @@ struct Layout {
   GnSlots gn1, gn2;
   size_t a1[2], a2[2], h, sc;        // conv inputs (pairs), conv1 output, shortcut output
   size_t act, q, k[2], v[2], o;      // attention buffers
+  size_t attn_ws;                     // balanced attention split: flags + partials
   // UNET_MINI: sub-block workspaces and the buffers between them
   size_t xin[2], h0, rb1, d1[2], h1, rb2, h2, at2, d2[2], h3, rb3, h4, at3;
   size_t total;
@@ -117,6 +118,7 @@ Layout layout_of(const dp_block_desc* d) {
     for (int i = 0; i < 2; ++i) L.k[i] = b.take(hw * d->C * e);
     for (int i = 0; i < 2; ++i) L.v[i] = b.take(hw * d->C * e);
     L.o = b.take(hw * d->C * e);
+    L.attn_ws = b.take(attn_workspace_bytes());
   } else {
     const MiniDescs m = mini_descs(d);
     const size_t hw2 = hw / 4, hw3 = hw / 16;
@@ -328,7 +330,7 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
       plan->push(DP_KERNEL_ATTN, 4.0 * T * keys * C, 4.0 * T * C * e);
     } else {
       rc = attn_launch(q, kf, vf, at<void>(ws, L.k[o]), at<void>(ws, L.v[o]), ob, T, d->heads, P,
-                       0.125f, mode, st);
+                       0.125f, mode, at<void>(ws, L.attn_ws), attn_workspace_bytes(), st);
       if (rc) return rc;
     }
     return lin(ob, w[4], w[5], x, out, nullptr, nullptr, T, C, C, C);

@@ -26,8 +26,10 @@ int linear_launch(const void* x, const void* weight, const float* bias, const vo
                   cudaStream_t stream);
 int attn_validate(const void* q, const void* kf, const void* vf, const void* ks, const void* vs,
                   const void* o, int T, int heads, int head_dim, int P, int mode);
+size_t attn_workspace_bytes();
 int attn_launch(const void* q, const void* kf, const void* vf, const void* ks, const void* vs,
-                void* o, int T, int heads, int P, float scale, int mode, cudaStream_t stream);
+                void* o, int T, int heads, int P, float scale, int mode, void* workspace,
+                size_t workspace_bytes, cudaStream_t stream);
 void recorder_begin(void* const* events, int n);
 int recorder_end();
 int copy_launch(const void* src, void* dst, size_t bytes, cudaStream_t stream);

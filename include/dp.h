@@ -232,12 +232,23 @@ DP_API int dp_linear(const void* x, const void* weight, const float* bias, const
  *
  *  q, k_fresh, v_fresh, k_stale, v_stale, o   [T][heads*head_dim] bf16, device
  *  (k_stale, v_stale read in DISPLACED only; o may not alias an input)
+ *  workspace   NULL, or device scratch of dp_attn_workspace_size() bytes,
+ *              16-byte aligned, zero-filled before its first use (calls keep
+ *              it valid).  With it the (query tile, key tile) work is split
+ *              evenly over all resident CTAs, and a query tile cut between
+ *              two CTAs is finished by merging their partial softmax sums
+ *              through the workspace; without it each CTA takes whole query
+ *              tiles.  Calls that overlap on the GPU must not share it.
  * Needs head_dim == 64, T % P == 0 and (T/P) % 128 == 0.
  * Runs on the tensor cores (tcgen05, S and O in tensor memory).
+ * Errors: DP_ERR_INVALID_ARG (null q/k/v/o, bad mode, o aliasing an input,
+ * missing stale K/V in DISPLACED), DP_ERR_UNSUPPORTED (shape, alignment).
  * ---------------------------------------------------------------------- */
+DP_API size_t dp_attn_workspace_size(void);
 DP_API int dp_attn_stale_kv(const void* q, const void* k_fresh, const void* v_fresh,
                      const void* k_stale, const void* v_stale, void* o, int T, int heads,
-                     int head_dim, int P, float scale, int mode, void* stream);
+                     int head_dim, int P, float scale, int mode, void* workspace,
+                     size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
  * Stale-buffer refresh: the device-local replacement of the paper's

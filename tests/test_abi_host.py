@@ -116,13 +116,13 @@ def test_kernel_calls_reject_bad_arguments_on_the_host(B):
         B.dp_conv3x3_halo(18, 16, 16, None, None, 32, 8, 8, 64, 64, 1, 2, B.SYNC, B.BF16, 0)
     assert e.value.code == B.DP_ERR_UNSUPPORTED
     with pytest.raises(B.DPError) as e:   # head_dim 128
-        B.dp_attn_stale_kv(16, 16, 16, 16, 16, 32, 256, 2, 128, 2, 0.1, B.SYNC, 0)
+        B.dp_attn_stale_kv(16, 16, 16, 16, 16, 32, 256, 2, 128, 2, 0.1, B.SYNC, stream=0)
     assert e.value.code == B.DP_ERR_UNSUPPORTED
     with pytest.raises(B.DPError) as e:   # band of 96 tokens
-        B.dp_attn_stale_kv(16, 16, 16, 16, 16, 32, 192, 2, 64, 2, 0.1, B.SYNC, 0)
+        B.dp_attn_stale_kv(16, 16, 16, 16, 16, 32, 192, 2, 64, 2, 0.1, B.SYNC, stream=0)
     assert e.value.code == B.DP_ERR_UNSUPPORTED
     with pytest.raises(B.DPError) as e:   # o aliases q
-        B.dp_attn_stale_kv(16, 32, 48, 64, 80, 16, 256, 2, 64, 2, 0.1, B.SYNC, 0)
+        B.dp_attn_stale_kv(16, 32, 48, 64, 80, 16, 256, 2, 64, 2, 0.1, B.SYNC, stream=0)
     assert e.value.code == B.DP_ERR_INVALID_ARG
     with pytest.raises(B.DPError) as e:   # linear K % 64
         B.dp_linear(16, 16, None, None, 32, None, None, 10, 64, 48, 64, 0)

@@ -183,17 +183,25 @@ def test_linear_parity(M, N, K, split, use_res):
 @pytest.mark.parametrize("T,heads,P,qscale", [(512, 2, 2, 1.0), (512, 2, 4, 3.0), (1024, 3, 2, 1.0),
                                               (4096, 10, 4, 1.0)])
 @pytest.mark.parametrize("mode", MODES)
-def test_attention_parity(T, heads, P, qscale, mode):
+@pytest.mark.parametrize("split", [True, False], ids=["split", "whole_tiles"])
+def test_attention_parity(T, heads, P, qscale, mode, split):
+    """With a workspace the key tiles of a query tile may be cut between CTAs
+    (at T=512 and T=1024 every query tile is: a CTA gets one key tile) and the
+    partial softmax sums are merged; without one every CTA takes whole tiles."""
     r = rng(T + heads + P + mode)
     C = heads * 64
     q = rounded(qscale * r.standard_normal((T, C)), "bf16")
     kf, vf, ks, vs = (rounded(r.standard_normal((T, C)), "bf16") for _ in range(4))
     ref = O.attention_stale_kv(q, kf, vf, ks, vs, P, heads, 0.125, mode)
     o = torch.empty(T, C, dtype=torch.bfloat16, device="cuda")
-    B.dp_attn_stale_kv(dev_mat(q), dev_mat(kf), dev_mat(vf), dev_mat(ks), dev_mat(vs), o, T, heads, 64,
-                       P, 0.125, mode)
-    torch.cuda.synchronize()
-    check(host(o), ref, what=f"attention T={T} P={P} mode={mode}")
+    nws = B.dp_attn_workspace_size()
+    ws = torch.zeros(nws, dtype=torch.uint8, device="cuda") if split else None
+    for _ in range(2):   # the second call reuses the workspace's flags
+        o.zero_()
+        B.dp_attn_stale_kv(dev_mat(q), dev_mat(kf), dev_mat(vf), dev_mat(ks), dev_mat(vs), o, T, heads,
+                           64, P, 0.125, mode, ws, nws if split else 0)
+        torch.cuda.synchronize()
+        check(host(o), ref, what=f"attention T={T} P={P} mode={mode} split={split}")
     assert B.dp_device_status() == 0
 
 
