@@ -54,9 +54,10 @@ _SIGS = {
                             _V, _SZ, _V], _I),
     "dp_groupnorm_async_noalloc": ([_V, _V, _V, _V, _I, _I, _I, _I, _I, _F, _F, _I, _I, _I, _V, _V,
                                     _V, _V, _V], _I),
-    "dp_conv3x3_halo": ([_V, _V, _V, _V, _V, _V, _I, _I, _I, _I, _I, _I, _I, _I, _V], _I),
+    "dp_gemm_workspace_size": ([], _SZ),
+    "dp_conv3x3_halo": ([_V, _V, _V, _V, _V, _V, _I, _I, _I, _I, _I, _I, _I, _I, _V, _SZ, _V], _I),
     "dp_conv3x3_halo_small": ([_V, _V, _V, _V, _V, _I, _I, _I, _I, _I, _I, _V], _I),
-    "dp_linear": ([_V, _V, _V, _V, _V, _V, _V, _I, _I, _I, _I, _V], _I),
+    "dp_linear": ([_V, _V, _V, _V, _V, _V, _V, _I, _I, _I, _I, _V, _SZ, _V], _I),
     "dp_attn_workspace_size": ([], _SZ),
     "dp_attn_stale_kv": ([_V, _V, _V, _V, _V, _V, _I, _I, _I, _I, _F, _I, _V, _SZ, _V], _I),
     "dp_refresh_stale": ([_V, _V, _SZ, _I, _I, _I, _V], _I),
@@ -159,11 +160,15 @@ def dp_groupnorm_async_noalloc(x, y, gamma, beta, H, W, C, G, P, eps, w, silu, m
         _p(stale_global), _p(stale_local), _p(fresh_local), _p(used_stats), _s(stream)))
 
 
+def dp_gemm_workspace_size():
+    return lib().dp_gemm_workspace_size()
+
+
 def dp_conv3x3_halo(a_fresh, a_stale, weight, bias, residual, out, H, W, Cin, Cout, stride, P,
-                    mode, dtype, stream=None):
+                    mode, dtype, workspace=None, workspace_bytes=0, stream=None):
     return _check(lib().dp_conv3x3_halo(_p(a_fresh), _p(a_stale), _p(weight), _p(bias),
                                         _p(residual), _p(out), H, W, Cin, Cout, stride, P, mode,
-                                        dtype, _s(stream)))
+                                        dtype, _p(workspace), workspace_bytes, _s(stream)))
 
 
 def dp_conv3x3_halo_small(a_fresh, a_stale, weight, bias, out, H, W, Cin, Cout, P, mode,
@@ -172,9 +177,11 @@ def dp_conv3x3_halo_small(a_fresh, a_stale, weight, bias, out, H, W, Cin, Cout, 
                                               _p(out), H, W, Cin, Cout, P, mode, _s(stream)))
 
 
-def dp_linear(x, weight, bias, residual, out0, out1, out2, M, N, K, split, stream=None):
+def dp_linear(x, weight, bias, residual, out0, out1, out2, M, N, K, split, workspace=None,
+              workspace_bytes=0, stream=None):
     return _check(lib().dp_linear(_p(x), _p(weight), _p(bias), _p(residual), _p(out0), _p(out1),
-                                  _p(out2), M, N, K, split, _s(stream)))
+                                  _p(out2), M, N, K, split, _p(workspace), workspace_bytes,
+                                  _s(stream)))
 
 
 def dp_attn_workspace_size():
@@ -247,7 +254,7 @@ def dp_block_step_timed(d: BlockDesc, s: BlockState, x, out, weights: Sequence, 
 
 
 KERNEL_NAMES = {0: "gn_stats", 1: "gn_apply", 2: "gn_fused", 3: "conv", 4: "linear", 5: "attn",
-                6: "copy", 7: "conv_small"}
+                6: "copy", 7: "conv_small", 8: "splitk_finish"}
 
 
 def dp_block_launch_info(d: BlockDesc, mode: int, i: int):

@@ -48,7 +48,8 @@ struct Layout {
   GnSlots gn1, gn2;
   size_t a1[2], a2[2], h, sc;        // conv inputs (pairs), conv1 output, shortcut output
   size_t act, q, k[2], v[2], o;      // attention buffers
-  size_t attn_ws;                     // balanced attention split: flags + partials
+  size_t attn_ws;                     // balanced attention split: counters + partials
+  size_t gemm_ws;                     // split-K partials of the convs and projections
   // UNET_MINI: sub-block workspaces and the buffers between them
   size_t xin[2], h0, rb1, d1[2], h1, rb2, h2, at2, d2[2], h3, rb3, h4, at3;
   size_t total;
@@ -136,6 +137,7 @@ Layout layout_of(const dp_block_desc* d) {
     L.h4 = b.take(hw3 * kU3 * 2);
     L.at3 = b.take(layout_of(&m.at3).total);
   }
+  L.gemm_ws = b.take(gemm_workspace_bytes());
   L.total = b.off;
   return L;
 }
@@ -254,21 +256,35 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
                   void* y, int h, int wd, int ci, int co, int stride) {
     if (plan) {
       const double ho = (h - 1) / stride + 1, wo = (wd - 1) / stride + 1;
-      plan->push(DP_KERNEL_CONV, 2.0 * ho * wo * co * 9.0 * ci,
-                 (static_cast<double>(h) * wd * ci + ho * wo * co * (res ? 2 : 1)) * e);
+      const int S = conv3x3_splits(h, wd, ci, co, stride, d->dtype, true);
+      if (S == 1) {
+        plan->push(DP_KERNEL_CONV, 2.0 * ho * wo * co * 9.0 * ci,
+                   (static_cast<double>(h) * wd * ci + ho * wo * co * (res ? 2 : 1)) * e);
+      } else {
+        plan->push(DP_KERNEL_CONV, 2.0 * ho * wo * co * 9.0 * ci,
+                   static_cast<double>(h) * wd * ci * e + ho * wo * co * 4.0 * S);
+        plan->push(DP_KERNEL_SPLITK_FINISH, 0.0, ho * wo * co * (4.0 * S + e * (res ? 2 : 1)));
+      }
       return DP_OK;
     }
     return conv3x3_launch(af, as, wt, static_cast<const float*>(b), res, y, h, wd, ci, co, stride, P,
-                          mode, d->dtype, st);
+                          mode, d->dtype, at<void>(ws, L.gemm_ws), gemm_workspace_bytes(), st);
   };
   auto lin = [&](const void* in, const void* wt, const void* b, const void* res, void* o0, void* o1,
                  void* o2, int M, int N, int K, int split) {
     if (plan) {
-      plan->push(DP_KERNEL_LINEAR, 2.0 * M * N * static_cast<double>(K),
-                 (static_cast<double>(M) * K + static_cast<double>(M) * N * (res ? 2 : 1)) * e);
+      const int S = linear_splits(M, N, K, split, true);
+      const double mn = static_cast<double>(M) * N;
+      if (S == 1) {
+        plan->push(DP_KERNEL_LINEAR, 2.0 * mn * K, (static_cast<double>(M) * K + mn * (res ? 2 : 1)) * e);
+      } else {
+        plan->push(DP_KERNEL_LINEAR, 2.0 * mn * K, static_cast<double>(M) * K * e + mn * 4.0 * S);
+        plan->push(DP_KERNEL_SPLITK_FINISH, 0.0, mn * (4.0 * S + e * (res ? 2 : 1)));
+      }
       return DP_OK;
     }
-    return linear_launch(in, wt, static_cast<const float*>(b), res, o0, o1, o2, M, N, K, split, st);
+    return linear_launch(in, wt, static_cast<const float*>(b), res, o0, o1, o2, M, N, K, split,
+                         at<void>(ws, L.gemm_ws), gemm_workspace_bytes(), st);
   };
   int rc;
   if (d->kind != DP_BLOCK_UNET_MINI && !plan) {

@@ -55,7 +55,19 @@ struct GemmParams {
   int ld_out;   // elements per row of each output buffer
   int split;    // output columns per buffer
   int* status;
+  // Split K (pair kernels): each output tile is cut into `splits` runs of
+  // k-blocks; run r stores its fp32 partial, laid out like the output
+  // ([M][N]), at part + r * M * N, and a finish kernel adds the runs, bias
+  // and residual and stores the outputs.
+  int splits;
+  float* part;
 };
+
+// k-blocks [*kb0, *kb1) of run `r` of `splits` over `kb` k-blocks.
+__device__ __forceinline__ void split_range(int kb, int splits, int r, int* kb0, int* kb1) {
+  *kb0 = (r * kb) / splits;
+  *kb1 = ((r + 1) * kb) / splits;
+}
 
 template <int BN, bool TF32>
 struct GemmCfg {
@@ -447,11 +459,54 @@ __device__ __forceinline__ void pair_epi_res_load(const GemmParams& p, const Epi
 // a wait gave up (the caller tears down).
 template <int BN>
 __device__ __forceinline__ bool pair_epilogue_tile(const GemmParams& p, uint32_t tmem, int q, int lane,
-                                                   uint32_t rank, int tile, int it, uint64_t* acc_full,
+                                                   uint32_t rank, int item, int it, uint64_t* acc_full,
                                                    uint32_t acc_empty_leader, volatile int* abort_flag,
                                                    PairEpi& e) {
   constexpr int NCH = BN / 32;
   static_assert(NCH >= 2, "chunks");
+  const int tile = item / p.splits;
+  // Split K: this run's accumulator goes to its fp32 partial, rows at their
+  // output pixels; bias, residual and the cast are the finish kernel's.
+  if (p.splits > 1) {
+    const int run = item - tile * p.splits;
+    const int mp = tile / p.n_tiles, nt = tile - mp * p.n_tiles;
+    const int mt = 2 * mp + static_cast<int>(rank);
+    const int row = q * 32 + lane;
+    bool valid;
+    size_t pix;
+    if (p.a_mode == 0) {
+      const int m = mt * 128 + row;
+      valid = m < p.M;
+      pix = static_cast<size_t>(m);
+    } else {
+      const int tr = mt / p.tiles_w, tc = mt - tr * p.tiles_w;
+      const int r = tr * p.R + row / p.Wt, c = tc * p.Wt + row % p.Wt;
+      valid = mt < p.m_tiles && r < p.Ho && c < p.Wo;
+      pix = static_cast<size_t>(r) * p.Wo + c;
+    }
+    const size_t M = p.a_mode == 0 ? static_cast<size_t>(p.M) : static_cast<size_t>(p.Ho) * p.Wo;
+    float* dst = p.part + static_cast<size_t>(run) * M * p.N + pix * p.N + nt * BN;
+    if (!mbar_wait(acc_full, it & 1, abort_flag, p.status)) return false;
+    tc_fence_after();
+#pragma unroll 1
+    for (int ch = 0; ch < NCH; ++ch) {
+      uint32_t r[32];
+      tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + ch * 32, r);
+      tmem_wait_ld();
+      if (ch == NCH - 1) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
+      }
+      if (!valid) continue;
+      float4* d4 = reinterpret_cast<float4*>(dst + ch * 32);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        d4[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                            __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+    }
+    return true;
+  }
   const int mp = tile / p.n_tiles, nt = tile - mp * p.n_tiles;
   const int mt = 2 * mp + static_cast<int>(rank);
   const int n0 = nt * BN;
@@ -476,19 +531,23 @@ __device__ __forceinline__ bool pair_epilogue_tile(const GemmParams& p, uint32_t
   const CUtensorMap* om = &p.tmO[b.seg];
 #pragma unroll 1
   for (int ch = 0; ch < NCH; ++ch) {
-    uint32_t r[32];
-    tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + ch * 32, r);
-    tmem_wait_ld();
-    if (ch == NCH - 1) {
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
-    }
-    if (!b.ok) continue;
     float v[32];
+    {
+      uint32_t r[32];
+      tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + ch * 32, r);
+      tmem_wait_ld();
+      if (ch == NCH - 1) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
+      }
+      if (!b.ok) continue;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+    }
     const float* bb = e.bias + ch * 32;
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) + bb[j];
+    for (int j = 0; j < 32; ++j) v[j] += bb[j];
     if (res) {
       const uint32_t s = e.ri & 1u;
       if (!mbar_wait(&e.rbar[s], (e.ri >> 1) & 1u, abort_flag, p.status)) return false;
@@ -564,6 +623,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   const bool leader = rank == 0;
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int num_tiles = ((p.m_tiles + 1) >> 1) * p.n_tiles;
+  const int num_items = num_tiles * p.splits;
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
@@ -598,7 +658,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       int ry_tab[3 * 16];
       uint64_t stale_mask = 0;
       const uint32_t full0 = mapa_shared(smem_u32(full), 0);   // leader's full[0]
-      for (int tile = pair; tile < num_tiles && !*abort_flag; tile += npairs) {
+      for (int item = pair; item < num_items && !*abort_flag; item += npairs) {
+        const int tile = item / p.splits;
+        int kbeg, kend;
+        split_range(p.k_blocks, p.splits, item - tile * p.splits, &kbeg, &kend);
         const int mp = tile / p.n_tiles, nt = tile - mp * p.n_tiles;
         const int mt = 2 * mp + static_cast<int>(rank);
         int c0 = 0;
@@ -624,8 +687,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
             }
           }
         }
-        int kh = 0, kw = 0, cb = 0;
-        for (int kb = 0; kb < p.k_blocks; ++kb) {
+        int cb = kbeg % (p.kc > 0 ? p.kc : 1), kh = 0, kw = 0;
+        if (p.a_mode == 1) {
+          const int tap = kbeg / p.kc;
+          kh = tap / 3;
+          kw = tap - kh * 3;
+        }
+        for (int kb = kbeg; kb < kend; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status)) goto producer_done;
           if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
           const uint32_t fb = full0 + stage * 8;
@@ -684,10 +752,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
-      for (int tile = pair; tile < num_tiles; tile += npairs, ++it) {
+      for (int item = pair; item < num_items; item += npairs, ++it) {
+        const int tile = item / p.splits;
+        int kbeg, kend;
+        split_range(p.k_blocks, p.splits, item - tile * p.splits, &kbeg, &kend);
         if (!mbar_wait(acc_empty, (it & 1) ^ 1, abort_flag, p.status)) goto mma_done;
         tc_fence_after();
-        for (int kb = 0; kb < p.k_blocks; ++kb) {
+        for (int kb = kbeg; kb < kend; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag, p.status)) goto mma_done;
           tc_fence_after();
           const uint64_t ad = a_desc0 + static_cast<uint64_t>((stage * C::A_BYTES) >> 4);
@@ -698,7 +769,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
             for (int j = 0; j < NJ; ++j)
               umma_f16_ss_pair(tmem + j * NI, ad + 2 * k,
                                bd + static_cast<uint64_t>((j * C::BSUB_BYTES) >> 4) + 2 * k, idesc,
-                               (kb | k) != 0);
+                               (kb != kbeg || k != 0));
           umma_commit_pair(empty_own + stage * 8);
           umma_commit_pair(empty_peer + stage * 8);
           if (++stage == C::STAGES) {
@@ -726,8 +797,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     e.rbar = rbar + 2 * q;
     e.ri = e.rpend = e.oi = 0;
     int it = 0;
-    for (int tile = pair; tile < num_tiles; tile += npairs, ++it)
-      if (!pair_epilogue_tile<C::BN>(p, tmem, q, lane, rank, tile, it, acc_full, acc_empty_leader,
+    for (int item = pair; item < num_items; item += npairs, ++it)
+      if (!pair_epilogue_tile<C::BN>(p, tmem, q, lane, rank, item, it, acc_full, acc_empty_leader,
                                      abort_flag, e))
         break;
     if (lane == 0) {
@@ -812,7 +883,7 @@ static int launch_pair(const GemmParams& p, cudaStream_t s) {
     }
     maxg = 2 * clusters;
   }
-  const int pair_tiles = ((p.m_tiles + 1) / 2) * p.n_tiles;
+  const int pair_tiles = ((p.m_tiles + 1) / 2) * p.n_tiles * p.splits;
   const int grid = std::min(2 * pair_tiles, maxg);
   mark_launch(s);
   igemm_pair_kernel<NI, NJ><<<grid, 192, C::SMEM, s>>>(p);
@@ -888,40 +959,173 @@ static int pick_bn(int m_tiles, int N, int split, bool tf32) {
 // single-CTA tile.  Estimated time = waves x per-SM work of one tile / the
 // relative efficiency measured for that tile (pair tiles move half the
 // weight bytes per flop).  Returns the pair width (320 or 160) or 0.
-static int pick_pair(int m_tiles, int N, int split, int* bn_single) {
+// Operand fill limits these kernels: per SM, TMA brings about 55 bytes per
+// cycle into shared memory (measured), so a k-block of a tile with `cols`
+// MMA columns per SM and `b_rows` weight rows staged per SM takes
+// max(2 cols, (16 KiB of A + 128 b_rows) / 55) cycles.
+static double kblock_cycles(int cols, int b_rows) {
+  const double mma = 2.0 * cols, fill = (16384.0 + 128.0 * b_rows) / 55.0;
+  return mma > fill ? mma : fill;
+}
+
+// Pair tile width (0 = single-CTA tiles) and the number of K runs, from a
+// cycle model: waves x (k-blocks x kblock_cycles + 5000 per wave for pipeline
+// fill and epilogue); split K (only with a workspace) cuts K into runs of at
+// least 8 k-blocks, keeps all (tile, run) items in one wave and pays about
+// 16000 cycles for the finish kernel (measured 8-10 us).
+static int pick_pair(int m_tiles, int N, int split, int kb, bool can_split, int* bn_single,
+                     int* splits) {
   const long sms = num_sms(), pairs = sms / 2;
   const long mp = (m_tiles + 1) / 2;
   double best = 0.0;
   int choice = 0;
-  struct Opt { int width; double eff; };
-  const Opt opts[2] = {{320, 1.0}, {160, 0.75}};
-  for (const Opt& o : opts) {
-    if (split % o.width) continue;
-    const long tiles = mp * (N / o.width);
-    const double t = static_cast<double>((tiles + pairs - 1) / pairs) * (128.0 * o.width) / o.eff;
-    if (!choice || t < best) {
-      best = t;
-      choice = o.width;
+  *splits = 1;
+  for (int width : {320, 160}) {
+    if (split % width) continue;
+    const long tiles = mp * (N / width);
+    const double per = kblock_cycles(width, width / 2);
+    for (int S = 1; S <= 16; ++S) {
+      if (S > 1 && (!can_split || kb / S < 8 || tiles * S > pairs)) break;
+      const double t = static_cast<double>((tiles * S + pairs - 1) / pairs) *
+                           (((kb + S - 1) / S) * per + 5000.0) + (S > 1 ? 16000.0 : 0.0);
+      if (!choice || t < best) {
+        best = t;
+        choice = width;
+        *splits = S;
+      }
     }
   }
   *bn_single = pick_bn(m_tiles, N, split, false);
   if (*bn_single) {
     const long tiles = static_cast<long>(m_tiles) * (N / *bn_single);
-    const double t = static_cast<double>((tiles + sms - 1) / sms) * (128.0 * *bn_single) / 0.6;
-    if (!choice || t < best) choice = 0;
+    const double t = static_cast<double>((tiles + sms - 1) / sms) *
+                     (kb * kblock_cycles(*bn_single, *bn_single) + 5000.0);
+    if (!choice || t < best) {
+      choice = 0;
+      *splits = 1;
+    }
   }
   return choice;
 }
 
+// Split-K workspace: the fp32 partials of all runs, each laid out like the
+// output.  Runs x rows x columns never exceed one wave of 256 x 320 pair tiles.
+size_t gemm_workspace_bytes() {
+  const size_t pairs = static_cast<size_t>(num_sms()) / 2;
+  return pairs * 2 * 128 * 320 * sizeof(float);
+}
+
+static void set_split(GemmParams& p, int splits, void* workspace) {
+  p.splits = splits;
+  if (splits > 1) p.part = static_cast<float*>(workspace);
+}
+
+// out[m][n] = sum over runs of part[run][m][n] + bias[n] (+ residual[m][n]),
+// cast to bf16 into output segment n / split.  8 columns per thread, runs
+// added in order (the result does not depend on which run finished first).
+__global__ void __launch_bounds__(256) splitk_finish_kernel(
+    const float* __restrict__ part, int runs, int M, int N, int split, int ld_out,
+    const float* __restrict__ bias, const __nv_bfloat16* __restrict__ residual,
+    __nv_bfloat16* out0, __nv_bfloat16* out1, __nv_bfloat16* out2) {
+  const long idx = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int nv = N / 8;
+  if (idx >= static_cast<long>(M) * nv) return;
+  const int m = static_cast<int>(idx / nv), n = static_cast<int>(idx - static_cast<long>(m) * nv) * 8;
+  const size_t mn = static_cast<size_t>(M) * N;
+  const float4* src = reinterpret_cast<const float4*>(part + static_cast<size_t>(m) * N + n);
+  float v[8];
+  {
+    const float4 a = __ldcg(src), b = __ldcg(src + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+  for (int r = 1; r < runs; ++r) {
+    const float4* s4 = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(src) + r * mn);
+    const float4 a = __ldcg(s4), b = __ldcg(s4 + 1);
+    v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
+    v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
+  }
+  if (bias) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(bias + n));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(bias + n) + 1);
+    v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w;
+    v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
+  }
+  if (residual) {
+    uint4 u = *reinterpret_cast<const uint4*>(residual + static_cast<size_t>(m) * N + n);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(h[e]);
+      v[2 * e] += f.x;
+      v[2 * e + 1] += f.y;
+    }
+  }
+  const int seg = n / split;
+  __nv_bfloat16* o = seg == 0 ? out0 : seg == 1 ? out1 : out2;
+  uint4 u;
+  u.x = pack_bf16x2(v[0], v[1]);
+  u.y = pack_bf16x2(v[2], v[3]);
+  u.z = pack_bf16x2(v[4], v[5]);
+  u.w = pack_bf16x2(v[6], v[7]);
+  *reinterpret_cast<uint4*>(o + static_cast<size_t>(m) * ld_out + (n - seg * split)) = u;
+}
+
+static int launch_finish(const GemmParams& p, int M, cudaStream_t s) {
+  const long n = static_cast<long>(M) * (p.N / 8);
+  mark_launch(s);
+  splitk_finish_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(
+      p.part, p.splits, M, p.N, p.split, p.ld_out, p.bias,
+      static_cast<const __nv_bfloat16*>(p.residual), static_cast<__nv_bfloat16*>(p.out0),
+      static_cast<__nv_bfloat16*>(p.out1), static_cast<__nv_bfloat16*>(p.out2));
+  return cuda_check(cudaGetLastError(), "split-K finish launch");
+}
+
+// Conv tile shape: Wt columns x 128/Wt rows, Wt a power of two in [8, 128]
+// wasting the fewest columns; a single 128-pixel row per tile (one TMA box
+// per A stage) when the ragged right edge wastes at most an eighth of it.
+static int conv_tile_width(int Wo) {
+  int Wt = 128, waste_best = 1 << 30;
+  for (int w = 128; w >= 8; w >>= 1) {
+    const int waste = ((Wo + w - 1) / w) * w - Wo;
+    if (waste < waste_best) {
+      waste_best = waste;
+      Wt = w;
+    }
+  }
+  if (Wo >= 128 && (((Wo + 127) / 128) * 128 - Wo) * 8 <= Wo) Wt = 128;
+  return Wt;
+}
+
+int conv3x3_splits(int H, int W, int Cin, int Cout, int stride, int dtype, bool can_split) {
+  if (dtype == DP_FP32) return 1;
+  const int Ho = (H - 1) / stride + 1, Wo = (W - 1) / stride + 1;
+  const int Wt = conv_tile_width(Wo), R = 128 / Wt;
+  const int m_tiles = ((Wo + Wt - 1) / Wt) * ((Ho + R - 1) / R);
+  int bn_single = 0, splits = 1;
+  const int pw = pick_pair(m_tiles, Cout, Cout, 9 * (Cin / 64), can_split, &bn_single, &splits);
+  return pw ? splits : 1;
+}
+
+int linear_splits(int M, int N, int K, int split, bool can_split) {
+  const int kb = K / 64;
+  if (kb < 16) return 1;
+  int bn_single = 0, splits = 1;
+  const int pw = pick_pair((M + 127) / 128, N, split, kb, can_split, &bn_single, &splits);
+  return pw ? splits : 1;
+}
+
 int conv3x3_launch(const void* a_fresh, const void* a_stale, const void* weight,
                    const float* bias, const void* residual, void* out, int H, int W, int Cin,
-                   int Cout, int stride, int P, int mode, int dtype, cudaStream_t stream) {
+                   int Cout, int stride, int P, int mode, int dtype, void* workspace,
+                   size_t workspace_bytes, cudaStream_t stream) {
   const bool tf32 = dtype == DP_FP32;
   const int e = tf32 ? 4 : 2;
   const int BK = 128 / e;
   const int Ho = (H - 1) / stride + 1, Wo = (W - 1) / stride + 1;
   GemmParams p;
   memset(&p, 0, sizeof(p));
+  p.splits = 1;
   p.a_mode = 1;
   p.H = H;
   p.W = W;
@@ -932,18 +1136,7 @@ int conv3x3_launch(const void* a_fresh, const void* a_stale, const void* weight,
   p.hb_in = H / P;
   p.hb_out = Ho / P;
   p.mode = mode;
-  // tile shape: Wt columns x R rows, Wt a power of two in [8, 128] wasting the fewest columns
-  int Wt = 128, waste_best = 1 << 30;
-  for (int w = 128; w >= 8; w >>= 1) {
-    const int waste = ((Wo + w - 1) / w) * w - Wo;
-    if (waste < waste_best) {
-      waste_best = waste;
-      Wt = w;
-    }
-  }
-  // A single 128-pixel row per tile keeps one TMA box per A stage; take it when
-  // the ragged right edge wastes at most an eighth of the row.
-  if (Wo >= 128 && (((Wo + 127) / 128) * 128 - Wo) * 8 <= Wo) Wt = 128;
+  const int Wt = conv_tile_width(Wo);
   p.Wt = Wt;
   p.R = 128 / Wt;
   p.tiles_w = (Wo + Wt - 1) / Wt;
@@ -957,8 +1150,9 @@ int conv3x3_launch(const void* a_fresh, const void* a_stale, const void* weight,
   p.residual = residual;
   p.out0 = out;
   p.status = device_status_ptr();
-  int bn_single = 0;
-  const int pw = tf32 ? 0 : pick_pair(p.m_tiles, Cout, Cout, &bn_single);
+  int bn_single = 0, splits = 1;
+  const bool can_split = workspace && workspace_bytes >= gemm_workspace_bytes();
+  const int pw = tf32 ? 0 : pick_pair(p.m_tiles, Cout, Cout, p.k_blocks, can_split, &bn_single, &splits);
   const bool pair = pw != 0;
   const int BN = pair ? pw : pick_bn(p.m_tiles, Cout, Cout, tf32);
   if (!BN) return set_error(DP_ERR_UNSUPPORTED, "conv: no N tile divides Cout=%d", Cout);
@@ -991,16 +1185,20 @@ int conv3x3_launch(const void* a_fresh, const void* a_stale, const void* weight,
   if (pair) {
     rc = encode_conv_epilogue(p, out, residual, Cout);
     if (rc) return rc;
-    return pw == 320 ? launch_pair<160, 2>(p, stream) : launch_pair<160, 1>(p, stream);
+    set_split(p, splits, workspace);
+    rc = pw == 320 ? launch_pair<160, 2>(p, stream) : launch_pair<160, 1>(p, stream);
+    if (rc || splits == 1) return rc;
+    return launch_finish(p, Ho * Wo, stream);
   }
   return launch_gemm(p, BN, tf32, stream);
 }
 
 int linear_launch(const void* x, const void* weight, const float* bias, const void* residual,
                   void* out0, void* out1, void* out2, int M, int N, int K, int split,
-                  cudaStream_t stream) {
+                  void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   GemmParams p;
   memset(&p, 0, sizeof(p));
+  p.splits = 1;
   p.a_mode = 0;
   p.M = M;
   p.m_tiles = (M + 127) / 128;
@@ -1014,10 +1212,13 @@ int linear_launch(const void* x, const void* weight, const float* bias, const vo
   p.out1 = out1;
   p.out2 = out2;
   p.status = device_status_ptr();
-  int bn_single = 0;
+  int bn_single = 0, splits = 1;
+  const bool can_split = workspace && workspace_bytes >= gemm_workspace_bytes();
   // Short K (few K blocks per tile) does not amortise a pair tile's pipeline
   // fill and un-overlapped epilogue; such projections stay on single-CTA tiles.
-  const int pw = p.k_blocks >= 16 ? pick_pair(p.m_tiles, N, split, &bn_single) : 0;
+  const int pw = p.k_blocks >= 16
+                     ? pick_pair(p.m_tiles, N, split, p.k_blocks, can_split, &bn_single, &splits)
+                     : 0;
   if (!pw) bn_single = pick_bn(p.m_tiles, N, split, false);
   const bool pair = pw != 0;
   const int BN = pair ? pw : bn_single;
@@ -1038,7 +1239,10 @@ int linear_launch(const void* x, const void* weight, const float* bias, const vo
     void* const outs[3] = {out0, out1, out2};
     rc = encode_linear_epilogue(p, outs, residual);
     if (rc) return rc;
-    return pw == 320 ? launch_pair<160, 2>(p, stream) : launch_pair<160, 1>(p, stream);
+    set_split(p, splits, workspace);
+    rc = pw == 320 ? launch_pair<160, 2>(p, stream) : launch_pair<160, 1>(p, stream);
+    if (rc || splits == 1) return rc;
+    return launch_finish(p, M, stream);
   }
   return launch_gemm(p, BN, false, stream);
 }
@@ -1074,19 +1278,26 @@ int conv3x3_validate(const void* a_fresh, const void* a_stale, const void* weigh
 
 extern "C" {
 
+size_t dp_gemm_workspace_size(void) { return dp::gemm_workspace_bytes(); }
+
 int dp_conv3x3_halo(const void* a_fresh, const void* a_stale, const void* weight,
                     const float* bias, const void* residual, void* out, int H, int W, int Cin,
-                    int Cout, int stride, int P, int mode, int dtype, void* stream) {
+                    int Cout, int stride, int P, int mode, int dtype, void* workspace,
+                    size_t workspace_bytes, void* stream) {
   int rc = dp::conv3x3_validate(a_fresh, a_stale, weight, residual, out, H, W, Cin, Cout, stride,
                                 P, mode, dtype);
   if (rc) return rc;
   if (bias && !dp::aligned16(bias)) return dp::set_error(DP_ERR_UNSUPPORTED, "conv: bias not 16-byte aligned");
+  if (workspace && !dp::aligned16(workspace))
+    return dp::set_error(DP_ERR_UNSUPPORTED, "conv: workspace not 16-byte aligned");
   return dp::conv3x3_launch(a_fresh, a_stale, weight, bias, residual, out, H, W, Cin, Cout, stride,
-                            P, mode, dtype, static_cast<cudaStream_t>(stream));
+                            P, mode, dtype, workspace, workspace_bytes,
+                            static_cast<cudaStream_t>(stream));
 }
 
 int dp_linear(const void* x, const void* weight, const float* bias, const void* residual,
-              void* out0, void* out1, void* out2, int M, int N, int K, int split, void* stream) {
+              void* out0, void* out1, void* out2, int M, int N, int K, int split, void* workspace,
+              size_t workspace_bytes, void* stream) {
   if (!x || !weight || !out0) return dp::set_error(DP_ERR_INVALID_ARG, "linear: null pointer");
   if (M <= 0 || N <= 0 || K <= 0 || split <= 0)
     return dp::set_error(DP_ERR_INVALID_ARG, "linear: non-positive size");
@@ -1102,8 +1313,10 @@ int dp_linear(const void* x, const void* weight, const float* bias, const void* 
       (out1 && !dp::aligned16(out1)) || (out2 && !dp::aligned16(out2)) ||
       (residual && !dp::aligned16(residual)) || (bias && !dp::aligned16(bias)))
     return dp::set_error(DP_ERR_UNSUPPORTED, "linear: pointers must be 16-byte aligned");
-  return dp::linear_launch(x, weight, bias, residual, out0, out1, out2, M, N, K, split,
-                           static_cast<cudaStream_t>(stream));
+  if (workspace && !dp::aligned16(workspace))
+    return dp::set_error(DP_ERR_UNSUPPORTED, "linear: workspace not 16-byte aligned");
+  return dp::linear_launch(x, weight, bias, residual, out0, out1, out2, M, N, K, split, workspace,
+                           workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -18,12 +18,18 @@ int gn_launch(const void* x, void* y, const float* gamma, const float* beta, int
 int conv3x3_validate(const void* a_fresh, const void* a_stale, const void* weight,
                      const void* residual, const void* out, int H, int W, int Cin, int Cout,
                      int stride, int P, int mode, int dtype);
+size_t gemm_workspace_bytes();
+// K runs of a conv / projection (1: no split; more: the GEMM is followed by
+// the split-K finish kernel).
+int conv3x3_splits(int H, int W, int Cin, int Cout, int stride, int dtype, bool can_split);
+int linear_splits(int M, int N, int K, int split, bool can_split);
 int conv3x3_launch(const void* a_fresh, const void* a_stale, const void* weight,
                    const float* bias, const void* residual, void* out, int H, int W, int Cin,
-                   int Cout, int stride, int P, int mode, int dtype, cudaStream_t stream);
+                   int Cout, int stride, int P, int mode, int dtype, void* workspace,
+                   size_t workspace_bytes, cudaStream_t stream);
 int linear_launch(const void* x, const void* weight, const float* bias, const void* residual,
                   void* out0, void* out1, void* out2, int M, int N, int K, int split,
-                  cudaStream_t stream);
+                  void* workspace, size_t workspace_bytes, cudaStream_t stream);
 int attn_validate(const void* q, const void* kf, const void* vf, const void* ks, const void* vs,
                   const void* o, int T, int heads, int head_dim, int P, int mode);
 size_t attn_workspace_bytes();

@@ -186,14 +186,25 @@ DP_API int dp_groupnorm_async_noalloc(const void* x, void* y, const float* gamma
  *  bias              [Cout] fp32, device, or NULL
  *  residual          [Ho][Wo][Cout] dtype, device, or NULL
  *  out               [Ho][Wo][Cout] dtype, device, written
+ *  workspace         NULL, or device scratch of dp_gemm_workspace_size() bytes,
+ *                    16-byte aligned, zero-filled before its first use (every
+ *                    call leaves its counters zero).  With it, a conv with too
+ *                    few output tiles to fill the GPU cuts K into runs on
+ *                    separate SM pairs; each run stores an fp32 partial and
+ *                    the last run of a tile sums them in run order.  Calls
+ *                    that overlap on the GPU must not share it.
  * Ho = (H-1)/stride + 1.  Needs Cin % 64 == 0 (bf16) or % 32 == 0 (fp32),
  * Cout % 32 == 0 (fp32: Cout % 64 == 0), H % P == 0, Ho % P == 0, W even when
  * stride 2.  Any W works; ragged tiles are masked.
  * Runs on the tensor cores (tcgen05, operands staged by TMA).
+ * Errors: DP_ERR_INVALID_ARG (null pointers, bad mode/dtype, aliasing,
+ * missing stale buffer in DISPLACED), DP_ERR_UNSUPPORTED (shape, alignment).
  * ---------------------------------------------------------------------- */
+DP_API size_t dp_gemm_workspace_size(void);
 DP_API int dp_conv3x3_halo(const void* a_fresh, const void* a_stale, const void* weight,
                     const float* bias, const void* residual, void* out, int H, int W,
-                    int Cin, int Cout, int stride, int P, int mode, int dtype, void* stream);
+                    int Cin, int Cout, int stride, int P, int mode, int dtype,
+                    void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
  * Direct 3x3 conv for few input channels (the latent input conv), same
@@ -216,11 +227,13 @@ DP_API int dp_conv3x3_halo_small(const void* a_fresh, const void* a_stale, const
  *            go to out0, out1, out2 ([M][split] each); with split == N only
  *            out0 is used.  The fused q/k/v projection writes k and v
  *            straight into the fresh half of the caller's K/V buffers.
+ *  workspace  NULL, or the split-K scratch of dp_gemm_workspace_size() bytes
+ *             (same rules as for dp_conv3x3_halo).
  * Needs K % 64 == 0, split % 32 == 0, N % split == 0, N / split <= 3.
  * ---------------------------------------------------------------------- */
 DP_API int dp_linear(const void* x, const void* weight, const float* bias, const void* residual,
               void* out0, void* out1, void* out2, int M, int N, int K, int split,
-              void* stream);
+              void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
  * Self-attention over stitched fresh / stale keys and values (gist.science
@@ -337,6 +350,7 @@ DP_API int dp_block_step(const dp_block_desc* d, dp_block_state* s, const void* 
 #define DP_KERNEL_ATTN 5       /* stale-K/V attention (tensor cores)            */
 #define DP_KERNEL_COPY 6       /* device copy                                   */
 #define DP_KERNEL_CONV_SMALL 7 /* direct 3x3 conv for few input channels        */
+#define DP_KERNEL_SPLITK_FINISH 8 /* sum of split-K partials + bias + residual   */
 
 /*
  * Number of kernel launches one displaced dp_block_step makes for this

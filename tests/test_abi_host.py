@@ -79,6 +79,11 @@ def test_block_desc_validation(B):
     d4 = B.dp_block_desc_init(B.GN_CONV, 480, 480, 320, 320, 32, 8, 0, B.BF16, 1, 1e-5, 1.0)
     assert [B.dp_block_launch_info(d4, B.DISPLACED, i)[0] for i in range(B.dp_block_launch_count(d4))] \
         == ["gn_stats", "gn_apply", "conv"]
+    # the 1280-channel convs at 32x32 have 16 output tiles for 74 SM pairs: K is
+    # split into runs and a finish kernel adds them
+    d5 = B.dp_block_desc_init(B.RESBLOCK, 32, 32, 640, 1280, 32, 4, 0, B.BF16, 1, 1e-5, 1.0)
+    assert [B.dp_block_launch_info(d5, B.DISPLACED, i)[0] for i in range(B.dp_block_launch_count(d5))] \
+        == ["gn_fused", "conv", "splitk_finish", "gn_fused", "linear", "conv", "splitk_finish"]
     du = B.dp_block_desc_init(B.UNET_MINI, 128, 128, 4, 0, 32, 4, 0, B.BF16, 1, 1e-5, 1.0)
     assert B.dp_block_weight_count(du) == 46
     assert abs(B.dp_block_flops(du) - sum(B.dp_block_launch_info(du, B.DISPLACED, i)[1]
@@ -101,19 +106,19 @@ def test_block_desc_validation(B):
 def test_kernel_calls_reject_bad_arguments_on_the_host(B):
     # null pointers and unsupported shapes return before any CUDA call
     with pytest.raises(B.DPError) as e:
-        B.dp_conv3x3_halo(None, None, None, None, None, None, 8, 8, 64, 64, 1, 2, B.SYNC, B.BF16, 0)
+        B.dp_conv3x3_halo(None, None, None, None, None, None, 8, 8, 64, 64, 1, 2, B.SYNC, B.BF16, stream=0)
     assert e.value.code == B.DP_ERR_INVALID_ARG
     with pytest.raises(B.DPError) as e:   # Cin not a multiple of 64
-        B.dp_conv3x3_halo(16, 16, 16, None, None, 32, 8, 8, 48, 64, 1, 2, B.SYNC, B.BF16, 0)
+        B.dp_conv3x3_halo(16, 16, 16, None, None, 32, 8, 8, 48, 64, 1, 2, B.SYNC, B.BF16, stream=0)
     assert e.value.code == B.DP_ERR_UNSUPPORTED
     with pytest.raises(B.DPError) as e:   # stride 3
-        B.dp_conv3x3_halo(16, 16, 16, None, None, 32, 8, 8, 64, 64, 3, 2, B.SYNC, B.BF16, 0)
+        B.dp_conv3x3_halo(16, 16, 16, None, None, 32, 8, 8, 64, 64, 3, 2, B.SYNC, B.BF16, stream=0)
     assert e.value.code == B.DP_ERR_UNSUPPORTED
     with pytest.raises(B.DPError) as e:   # displaced without the stale buffer
-        B.dp_conv3x3_halo(16, None, 16, None, None, 32, 8, 8, 64, 64, 1, 2, B.DISPLACED, B.BF16, 0)
+        B.dp_conv3x3_halo(16, None, 16, None, None, 32, 8, 8, 64, 64, 1, 2, B.DISPLACED, B.BF16, stream=0)
     assert e.value.code == B.DP_ERR_INVALID_ARG
     with pytest.raises(B.DPError) as e:   # misaligned pointer
-        B.dp_conv3x3_halo(18, 16, 16, None, None, 32, 8, 8, 64, 64, 1, 2, B.SYNC, B.BF16, 0)
+        B.dp_conv3x3_halo(18, 16, 16, None, None, 32, 8, 8, 64, 64, 1, 2, B.SYNC, B.BF16, stream=0)
     assert e.value.code == B.DP_ERR_UNSUPPORTED
     with pytest.raises(B.DPError) as e:   # head_dim 128
         B.dp_attn_stale_kv(16, 16, 16, 16, 16, 32, 256, 2, 128, 2, 0.1, B.SYNC, stream=0)
@@ -125,7 +130,7 @@ def test_kernel_calls_reject_bad_arguments_on_the_host(B):
         B.dp_attn_stale_kv(16, 32, 48, 64, 80, 16, 256, 2, 64, 2, 0.1, B.SYNC, stream=0)
     assert e.value.code == B.DP_ERR_INVALID_ARG
     with pytest.raises(B.DPError) as e:   # linear K % 64
-        B.dp_linear(16, 16, None, None, 32, None, None, 10, 64, 48, 64, 0)
+        B.dp_linear(16, 16, None, None, 32, None, None, 10, 64, 48, 64, stream=0)
     assert e.value.code == B.DP_ERR_UNSUPPORTED
     with pytest.raises(B.DPError) as e:   # groupnorm: C % G
         B.dp_groupnorm_async(16, 32, 16, 16, 8, 8, 30, 32, 2, 1e-5, 1.0, 1, B.SYNC, B.BF16, None, None,

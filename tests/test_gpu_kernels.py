@@ -141,6 +141,61 @@ def test_conv3x3_halo_parity(case, mode):
     assert B.dp_device_status() == 0
 
 
+SPLIT_K_CONV_CASES = [
+    # Cin, Cout, H, W, P, stride, residual: few output tiles, long K
+    (640, 640, 16, 16, 2, 1, True),      # 2 pair tiles of 256x320, K runs across the GPU
+    (640, 1280, 32, 32, 4, 1, False),    # the 1280-channel stage shape
+    (640, 640, 64, 64, 4, 2, True),      # stride 2, 32x32 output
+    (640, 640, 24, 40, 4, 1, True),      # 8-pixel-wide tiles of 16 rows, ragged band
+]
+
+
+@pytest.mark.parametrize("case", SPLIT_K_CONV_CASES)
+@pytest.mark.parametrize("mode", [B.DISPLACED, B.SYNC])
+def test_conv3x3_split_k_parity(case, mode):
+    """With a workspace, convs with too few output tiles cut K into runs whose
+    fp32 partials the last run sums; checked against the oracle twice in a row
+    (the second call reuses the workspace's run counters)."""
+    Cin, Cout, H, W, P, stride, use_res = case
+    r = rng(7 * Cin + Cout + H + W + stride + mode)
+    af = rounded(r.standard_normal((Cin, H, W)), "bf16")
+    ast = rounded(r.standard_normal((Cin, H, W)), "bf16")
+    wt = rounded(r.standard_normal((Cout, Cin, 3, 3)) * math.sqrt(2 / (9 * Cin)), "bf16")
+    b = 0.3 * r.standard_normal(Cout)
+    Ho, Wo = (H - 1) // stride + 1, (W - 1) // stride + 1
+    res = rounded(r.standard_normal((Cout, Ho, Wo)), "bf16") if use_res else None
+    ref = O.conv3x3_halo(af, ast, wt, b, res, P, mode, stride)
+    nws = B.dp_gemm_workspace_size()
+    ws = torch.zeros(nws, dtype=torch.uint8, device="cuda")
+    out = torch.empty(Ho, Wo, Cout, dtype=torch.bfloat16, device="cuda")
+    for call in range(2):
+        out.zero_()
+        B.dp_conv3x3_halo(dev_img(af, "bf16"), dev_img(ast, "bf16"), conv_w_dev(wt, "bf16"), dev_f32(b),
+                          dev_img(res, "bf16") if use_res else None, out, H, W, Cin, Cout, stride, P,
+                          mode, B.BF16, ws, nws)
+        torch.cuda.synchronize()
+        check(host_img(out), ref, what=f"split-K conv {case} mode {mode} call {call}",
+              storage_rel=BF16_HALF_ULP)
+    assert B.dp_device_status() == 0
+
+
+def test_linear_split_k_parity():
+    r = rng(99)
+    M, N, K = 1024, 640, 5120
+    x = rounded(r.standard_normal((M, K)), "bf16")
+    w = rounded(r.standard_normal((N, K)) / math.sqrt(K), "bf16")
+    b = 0.3 * r.standard_normal(N)
+    res = rounded(r.standard_normal((M, N)), "bf16")
+    ref = x @ w.T + b + res
+    nws = B.dp_gemm_workspace_size()
+    ws = torch.zeros(nws, dtype=torch.uint8, device="cuda")
+    out = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    B.dp_linear(dev_mat(x), dev_mat(w), dev_f32(b), dev_mat(res), out, None, None, M, N, K, N, ws, nws)
+    torch.cuda.synchronize()
+    check(host(out), ref, what="split-K linear", storage_rel=BF16_HALF_ULP)
+    assert B.dp_device_status() == 0
+
+
 def test_conv_small_parity():
     for mode in MODES:
         r = rng(40 + mode)
