@@ -199,6 +199,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_kernel(const __grid_cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // set-up done: from here on this grid reads its predecessor's outputs
+  griddep_wait();
+  griddep_trigger();
   const uint32_t tS = tmem, tP = tmem + 128, tO = tmem + 192;
 
   if (warp == 0) {
@@ -597,8 +600,8 @@ int attn_launch(const void* q, const void* kf, const void* vf, const void* ks, c
   }
   const int grid = (a.W + a.L - 1) / a.L;
   mark_launch(stream);
-  attn_kernel<<<grid, kAttnThreads, kAttnSmem, stream>>>(a);
-  return cuda_check(cudaGetLastError(), "attention launch");
+  return launch_kernel(attn_kernel, dim3(grid), dim3(kAttnThreads), kAttnSmem, stream, false,
+                       "attention launch", a);
 }
 
 int attn_validate(const void* q, const void* kf, const void* vf, const void* ks, const void* vs,

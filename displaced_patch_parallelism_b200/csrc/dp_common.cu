@@ -6,6 +6,8 @@
 
 #include <mutex>
 
+#include <cstdlib>
+
 #include "dp_common.cuh"
 
 namespace dp {
@@ -23,6 +25,14 @@ struct LaunchRecorder {
   int idx = 0;
 };
 static thread_local LaunchRecorder t_rec;
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* v = getenv("DP_PDL");
+    return !(v && v[0] == '0');
+  }();
+  return on;
+}
 
 void mark_launch(cudaStream_t s) {
   if (t_rec.events && t_rec.idx < t_rec.n)

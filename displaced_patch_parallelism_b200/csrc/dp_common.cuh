@@ -30,12 +30,56 @@ int encode_tmap(CUtensorMap* map, CUtensorMapDataType dt, int rank, void* base,
 void mark_launch(cudaStream_t s);
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Programmatic dependent launch: every kernel of the library is launched so
+// that it may start while the previous kernel on the stream finishes; each
+// kernel sets itself up (barriers, tensor memory, tensor-map prefetch, its
+// read-only parameters) and then waits for its predecessor (griddep_wait)
+// before it touches any memory another kernel writes.  DP_PDL=0 in the
+// environment turns it off.
+bool pdl_enabled();
+
+// Launches `kernel` with the dependent-launch attribute (when enabled) and,
+// if asked, as a cooperative grid.
+template <typename... KArgs, typename... Args>
+int launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                  bool cooperative, const char* what, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  if (pdl_enabled()) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cooperative) {
+    attr[n].id = cudaLaunchAttributeCooperative;
+    attr[n].val.cooperative = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cuda_check(cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...), what);
+}
+
 // Wall-clock limit of one bounded wait inside a kernel.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
 
 // ---------------------------------------------------------------- device side
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Waits until the previous kernel on the stream has completed and its
+// writes are visible (no-op when it was not launched as a dependent).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the next kernel on the stream be scheduled once every block of this
+// grid has signalled or exited.
+__device__ __forceinline__ void griddep_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 __device__ __forceinline__ unsigned long long globaltimer_ns() {

@@ -6,7 +6,8 @@
 // summary, Method): rows of other bands come from the fresh input (sync), the
 // previous step's input (displaced) or nowhere (naive).
 //
-// One thread computes 32 consecutive output channels of one pixel; a warp holds
+// Up to 8 input channels: the register kernel below.  Otherwise one thread
+// computes 32 consecutive output channels of one pixel; a warp holds
 // 32 neighbouring pixels of the same channel group, so every weight it reads
 // from shared memory is the same address for all lanes (a broadcast), and its
 // input loads are adjacent pixels.  The filter slice of the block's channel
@@ -23,6 +24,8 @@ __global__ void __launch_bounds__(256) conv3x3_small_kernel(
     const __nv_bfloat16* __restrict__ w, const float* __restrict__ bias,
     __nv_bfloat16* __restrict__ out, int H, int W, int Cin, int Cout, int hb, int mode) {
   extern __shared__ float sw[];   // [9][Cin][32] for channel group blockIdx.y
+  griddep_wait();
+  griddep_trigger();
   const int co0 = blockIdx.y * kSmallCo;
   const int nw = 9 * Cin * kSmallCo;
   for (int i = threadIdx.x; i < nw; i += blockDim.x) {
@@ -70,17 +73,90 @@ __global__ void __launch_bounds__(256) conv3x3_small_kernel(
   }
 }
 
+// Register variant for up to 8 input channels (the latent input conv has
+// 4): a block takes 64 pixels of one output row; the 3 input rows it needs
+// (66 pixels, channels padded to CIN with zeros) are staged in shared memory
+// as fp32 with the halo rule applied, and each warp takes (32 output
+// channels, 32 pixels) items: a lane owns one output channel, keeps its
+// 9 x CIN filter taps in registers and reads each input value as a shared-
+// memory broadcast; a warp's 32 lanes store 32 consecutive channels of one
+// pixel.
+constexpr int kRegTile = 64;
+
+template <int CIN>
+__global__ void __launch_bounds__(256) conv3x3_small_reg_kernel(
+    const __nv_bfloat16* __restrict__ af, const __nv_bfloat16* __restrict__ as,
+    const __nv_bfloat16* __restrict__ w, const float* __restrict__ bias,
+    __nv_bfloat16* __restrict__ out, int H, int W, int Cin, int Cout, int hb, int mode) {
+  __shared__ __align__(16) float sx[3][kRegTile + 2][CIN];
+  const int r = blockIdx.y, c0 = blockIdx.x * kRegTile;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  griddep_wait();
+  griddep_trigger();
+  const int band = r / hb;
+  for (int i = threadIdx.x; i < 3 * (kRegTile + 2) * CIN; i += blockDim.x) {
+    const int ci = i % CIN, px = (i / CIN) % (kRegTile + 2), kh = i / (CIN * (kRegTile + 2));
+    const int rho = r + kh - 1, col = c0 + px - 1;
+    float v = 0.f;
+    if (ci < Cin && rho >= 0 && rho < H && col >= 0 && col < W) {
+      const __nv_bfloat16* src = af;
+      bool use = true;
+      if (rho / hb != band) {
+        if (mode == DP_MODE_DISPLACED) src = as;
+        else if (mode == DP_MODE_NAIVE) use = false;
+      }
+      if (use) v = __bfloat162float(src[(static_cast<size_t>(rho) * W + col) * Cin + ci]);
+    }
+    sx[kh][px][ci] = v;
+  }
+  __syncthreads();
+  const int groups = Cout / 32, chunks = kRegTile / 32;
+  for (int item = warp; item < groups * chunks; item += blockDim.x >> 5) {
+    const int g = item / chunks, ch = item - g * chunks;
+    const int co = g * 32 + lane;
+    float wr[9 * CIN];
+#pragma unroll
+    for (int k = 0; k < 9; ++k)
+#pragma unroll
+      for (int ci = 0; ci < CIN; ++ci)
+        wr[k * CIN + ci] = ci < Cin ? __bfloat162float(w[(static_cast<size_t>(co) * 9 + k) * Cin + ci]) : 0.f;
+    const float b0 = bias ? __ldg(bias + co) : 0.f;
+    for (int j = 0; j < 32; ++j) {
+      const int px = ch * 32 + j, c = c0 + px;
+      if (c >= W) break;
+      float acc = b0;
+#pragma unroll
+      for (int kh = 0; kh < 3; ++kh)
+#pragma unroll
+        for (int kw = 0; kw < 3; ++kw)
+#pragma unroll
+          for (int ci = 0; ci < CIN; ++ci) acc = fmaf(sx[kh][px + kw][ci], wr[(kh * 3 + kw) * CIN + ci], acc);
+      out[(static_cast<size_t>(r) * W + c) * Cout + co] = __float2bfloat16_rn(acc);
+    }
+  }
+}
+
 int conv3x3_small_launch(const void* af, const void* as, const void* w, const float* bias,
                          void* out, int H, int W, int Cin, int Cout, int P, int mode,
                          cudaStream_t stream) {
+  const auto* a0 = static_cast<const __nv_bfloat16*>(af);
+  const auto* a1 = static_cast<const __nv_bfloat16*>(as ? as : af);
+  const auto* wt = static_cast<const __nv_bfloat16*>(w);
+  auto* o = static_cast<__nv_bfloat16*>(out);
+  if (Cin <= 8) {
+    const dim3 grid(static_cast<unsigned>((W + kRegTile - 1) / kRegTile), static_cast<unsigned>(H));
+    mark_launch(stream);
+    if (Cin <= 4)
+      return launch_kernel(conv3x3_small_reg_kernel<4>, grid, dim3(256), 0, stream, false,
+                           "small conv launch", a0, a1, wt, bias, o, H, W, Cin, Cout, H / P, mode);
+    return launch_kernel(conv3x3_small_reg_kernel<8>, grid, dim3(256), 0, stream, false,
+                         "small conv launch", a0, a1, wt, bias, o, H, W, Cin, Cout, H / P, mode);
+  }
   const size_t smem = static_cast<size_t>(9) * Cin * kSmallCo * sizeof(float);
   const dim3 grid(static_cast<unsigned>((static_cast<long>(H) * W + 255) / 256), Cout / kSmallCo);
   mark_launch(stream);
-  conv3x3_small_kernel<<<grid, 256, smem, stream>>>(
-      static_cast<const __nv_bfloat16*>(af), static_cast<const __nv_bfloat16*>(as ? as : af),
-      static_cast<const __nv_bfloat16*>(w), bias, static_cast<__nv_bfloat16*>(out), H, W, Cin,
-      Cout, H / P, mode);
-  return cuda_check(cudaGetLastError(), "small conv launch");
+  return launch_kernel(conv3x3_small_kernel, grid, dim3(256), smem, stream, false, "small conv launch",
+                       a0, a1, wt, bias, o, H, W, Cin, Cout, H / P, mode);
 }
 
 }  // namespace dp

@@ -138,6 +138,9 @@ __global__ void __launch_bounds__(192, 1) igemm_kernel(const __grid_constant__ G
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // set-up done: from here on this grid reads its predecessor's outputs
+  griddep_wait();
+  griddep_trigger();
   const int num_tiles = p.m_tiles * p.n_tiles;
 
   if (warp == 0) {
@@ -649,6 +652,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // set-up done: from here on this grid reads its predecessor's outputs
+  griddep_wait();
+  griddep_trigger();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -886,8 +892,8 @@ static int launch_pair(const GemmParams& p, cudaStream_t s) {
   const int pair_tiles = ((p.m_tiles + 1) / 2) * p.n_tiles * p.splits;
   const int grid = std::min(2 * pair_tiles, maxg);
   mark_launch(s);
-  igemm_pair_kernel<NI, NJ><<<grid, 192, C::SMEM, s>>>(p);
-  return cuda_check(cudaGetLastError(), "pair gemm launch");
+  return launch_kernel(igemm_pair_kernel<NI, NJ>, dim3(grid), dim3(192), C::SMEM, s, false,
+                       "pair gemm launch", p);
 }
 
 template <int BN, bool TF32>
@@ -906,8 +912,8 @@ static int launch_t(const GemmParams& p, cudaStream_t s) {
   const int tiles = p.m_tiles * p.n_tiles;
   const int grid = std::min(tiles, num_sms());
   mark_launch(s);
-  igemm_kernel<BN, TF32><<<grid, 192, C::SMEM, s>>>(p);
-  return cuda_check(cudaGetLastError(), "gemm launch");
+  return launch_kernel(igemm_kernel<BN, TF32>, dim3(grid), dim3(192), C::SMEM, s, false,
+                       "gemm launch", p);
 }
 
 static int launch_gemm(const GemmParams& p, int BN, bool tf32, cudaStream_t s) {
@@ -1027,6 +1033,8 @@ __global__ void __launch_bounds__(256) splitk_finish_kernel(
     const float* __restrict__ part, int runs, int M, int N, int split, int ld_out,
     const float* __restrict__ bias, const __nv_bfloat16* __restrict__ residual,
     __nv_bfloat16* out0, __nv_bfloat16* out1, __nv_bfloat16* out2) {
+  griddep_wait();
+  griddep_trigger();
   const long idx = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int nv = N / 8;
   if (idx >= static_cast<long>(M) * nv) return;
@@ -1074,11 +1082,11 @@ __global__ void __launch_bounds__(256) splitk_finish_kernel(
 static int launch_finish(const GemmParams& p, int M, cudaStream_t s) {
   const long n = static_cast<long>(M) * (p.N / 8);
   mark_launch(s);
-  splitk_finish_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(
-      p.part, p.splits, M, p.N, p.split, p.ld_out, p.bias,
-      static_cast<const __nv_bfloat16*>(p.residual), static_cast<__nv_bfloat16*>(p.out0),
-      static_cast<__nv_bfloat16*>(p.out1), static_cast<__nv_bfloat16*>(p.out2));
-  return cuda_check(cudaGetLastError(), "split-K finish launch");
+  return launch_kernel(splitk_finish_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0,
+                       s, false, "split-K finish launch", static_cast<const float*>(p.part), p.splits,
+                       M, p.N, p.split, p.ld_out, p.bias, static_cast<const __nv_bfloat16*>(p.residual),
+                       static_cast<__nv_bfloat16*>(p.out0), static_cast<__nv_bfloat16*>(p.out1),
+                       static_cast<__nv_bfloat16*>(p.out2));
 }
 
 // Conv tile shape: Wt columns x 128/Wt rows, Wt a power of two in [8, 128]

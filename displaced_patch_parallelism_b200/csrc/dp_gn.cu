@@ -122,6 +122,8 @@ __global__ void __launch_bounds__(1024) gn_stats_kernel(const T* __restrict__ x,
   float* ssq = ssum + a.lanes * a.C;                          // [lanes][C]
   __shared__ int s_last;
 
+  griddep_wait();
+  griddep_trigger();
   const int p = blockIdx.x / a.S, s = blockIdx.x % a.S;
   const int v = threadIdx.x % a.vpp, pl = threadIdx.x / a.vpp;
   const int chunk = (a.HWp + a.S - 1) / a.S;
@@ -247,6 +249,8 @@ __global__ void __launch_bounds__(1024) gn_apply_kernel(const T* __restrict__ x,
   extern __shared__ __align__(16) unsigned char gn_smem[];
   float* sscale = reinterpret_cast<float*>(gn_smem);
   float* sshift = sscale + a.C;
+  griddep_wait();
+  griddep_trigger();
   const int b = gridDim.x - 1 - blockIdx.x;   // reverse walk: L2-hot tail first
   const int p = b / a.S, s = b % a.S;
   const int cg = a.C / a.G;
@@ -399,6 +403,8 @@ __global__ void __launch_bounds__(1024, 1) gn_fused_kernel(
     fence_mbar_init();
   }
   __syncthreads();
+  griddep_wait();
+  griddep_trigger();
   if (threadIdx.x == 0 && npix > 0) {
     const uint32_t total = static_cast<uint32_t>(npix * row_bytes);
     mbar_arrive_expect_tx(&load_bar, total);
@@ -688,6 +694,31 @@ static bool gn_fused_launch(const void* x, void* y, const float* gamma, const fl
                   &a, &part, &bar, const_cast<float**>(&stale_global), const_cast<float**>(&stale_local),
                   &fresh_local, &fresh_global, &used, &status};
   mark_launch(stream);
+  // cooperative (the grid barrier needs every block resident) and, when the
+  // driver takes both attributes, a dependent launch
+  static int pdl_ok = -1;
+  if (pdl_enabled() && pdl_ok != 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(blocks);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeCooperative;
+    attr[1].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    const cudaError_t e = cudaLaunchKernelExC(&cfg, fn, args);
+    if (e == cudaSuccess) {
+      pdl_ok = 1;
+      *rc = DP_OK;
+      return true;
+    }
+    cudaGetLastError();
+    pdl_ok = 0;
+  }
   *rc = cuda_check(cudaLaunchCooperativeKernel(fn, dim3(blocks), dim3(threads), args, smem, stream),
                    "fused groupnorm launch");
   return true;
@@ -739,25 +770,31 @@ int gn_launch(const void* x, void* y, const float* gamma, const float* beta, int
       attr_done[dtype] = true;
     }
   }
+  const float* cgl = stale_global;
+  const float* cll = stale_local;
+  const float* cused = used;
   if (dtype == DP_BF16) {
     mark_launch(stream);
-    gn_stats_kernel<__nv_bfloat16><<<blocks, threads, smem_stats, stream>>>(
-        static_cast<const __nv_bfloat16*>(x), a, acc, counter, stale_global, stale_local,
-        fresh_local, fresh_global, used);
+    int rc = launch_kernel(gn_stats_kernel<__nv_bfloat16>, dim3(blocks), dim3(threads), smem_stats,
+                           stream, false, "groupnorm stats launch",
+                           static_cast<const __nv_bfloat16*>(x), a, acc, counter, cgl, cll,
+                           fresh_local, fresh_global, used);
+    if (rc) return rc;
     mark_launch(stream);
-    gn_apply_kernel<__nv_bfloat16><<<blocks, threads, smem_apply, stream>>>(
-        static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(y), gamma, beta, used,
-        a);
-  } else {
-    mark_launch(stream);
-    gn_stats_kernel<float><<<blocks, threads, smem_stats, stream>>>(
-        static_cast<const float*>(x), a, acc, counter, stale_global, stale_local, fresh_local,
-        fresh_global, used);
-    mark_launch(stream);
-    gn_apply_kernel<float><<<blocks, threads, smem_apply, stream>>>(
-        static_cast<const float*>(x), static_cast<float*>(y), gamma, beta, used, a);
+    return launch_kernel(gn_apply_kernel<__nv_bfloat16>, dim3(blocks), dim3(threads), smem_apply,
+                         stream, false, "groupnorm apply launch",
+                         static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(y), gamma,
+                         beta, cused, a);
   }
-  return cuda_check(cudaGetLastError(), "groupnorm launch");
+  mark_launch(stream);
+  int rc = launch_kernel(gn_stats_kernel<float>, dim3(blocks), dim3(threads), smem_stats, stream,
+                         false, "groupnorm stats launch", static_cast<const float*>(x), a, acc,
+                         counter, cgl, cll, fresh_local, fresh_global, used);
+  if (rc) return rc;
+  mark_launch(stream);
+  return launch_kernel(gn_apply_kernel<float>, dim3(blocks), dim3(threads), smem_apply, stream, false,
+                       "groupnorm apply launch", static_cast<const float*>(x), static_cast<float*>(y),
+                       gamma, beta, cused, a);
 }
 
 // ---------------------------------------------------------------------------

@@ -15,6 +15,8 @@ namespace dp {
 
 __global__ void __launch_bounds__(256) copy16_kernel(const uint4* __restrict__ src,
                                                      uint4* __restrict__ dst, size_t n16) {
+  griddep_wait();
+  griddep_trigger();
   const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
   size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   for (; i + 3 * stride < n16; i += 4 * stride) {
@@ -31,6 +33,8 @@ __global__ void __launch_bounds__(256) copy16_kernel(const uint4* __restrict__ s
 __global__ void refresh_stats_kernel(const float* __restrict__ fresh_local,
                                      float* __restrict__ stale_local,
                                      float* __restrict__ stale_global, int P, int G) {
+  griddep_wait();
+  griddep_trigger();
   for (int i = threadIdx.x; i < P * G * 2; i += blockDim.x) stale_local[i] = fresh_local[i];
   for (int i = threadIdx.x; i < G * 2; i += blockDim.x) {
     const int g = i / 2, k = i % 2;
@@ -47,9 +51,8 @@ int copy_launch(const void* src, void* dst, size_t bytes, cudaStream_t stream) {
   const size_t cap = static_cast<size_t>(num_sms()) * 8;
   if (blocks > cap) blocks = cap;
   mark_launch(stream);
-  copy16_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-      static_cast<const uint4*>(src), static_cast<uint4*>(dst), n16);
-  return cuda_check(cudaGetLastError(), "refresh launch");
+  return launch_kernel(copy16_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, stream, false,
+                       "refresh launch", static_cast<const uint4*>(src), static_cast<uint4*>(dst), n16);
 }
 
 }  // namespace dp
@@ -80,9 +83,9 @@ int dp_refresh_stats(const float* fresh_local, float* stale_local, float* stale_
     return dp::set_error(DP_ERR_INVALID_ARG, "refresh_stats: null pointer");
   if (P <= 0 || G <= 0) return dp::set_error(DP_ERR_INVALID_ARG, "refresh_stats: bad P/G");
   dp::mark_launch(static_cast<cudaStream_t>(stream));
-  dp::refresh_stats_kernel<<<1, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      fresh_local, stale_local, stale_global, P, G);
-  return dp::cuda_check(cudaGetLastError(), "refresh_stats launch");
+  return dp::launch_kernel(dp::refresh_stats_kernel, dim3(1), dim3(256), 0,
+                           static_cast<cudaStream_t>(stream), false, "refresh_stats launch",
+                           fresh_local, stale_local, stale_global, P, G);
 }
 
 }  // extern "C"
