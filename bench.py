@@ -5,9 +5,11 @@
 
 A step is one ``dp_block_step`` of the workload (default: the SDXL 1024 px
 top-resolution ResBlock, latent 1x320x128x128, P = 4 bands) in displaced mode,
-on synthetic inputs already resident in HBM.  Every step's kernels are timed
-with CUDA events recorded on the launching stream (``dp_block_step_timed``);
-L2 is flushed (a 256 MiB write) between steps, outside the timed events.
+on synthetic inputs already resident in HBM.  Each step is timed with CUDA
+events recorded on the launching stream just before and after it; L2 is
+flushed (a 256 MiB write) between steps, outside the timed events.  A second
+pass with an event before every kernel (``dp_block_step_timed``) gives the
+per-kernel breakdown and the roofline of the dominant kernel.
 With N > 1 (torchrun) every rank runs an independent replica on its own GPU:
 the path has no data exchange on one GPU per image, so there is no
 collective; the time is the max over ranks.
@@ -267,11 +269,13 @@ def run_ours(args, wl):
         blk.step(dev_x[i % pool], out, dw, B.dp_mode_for_step(i, wl.warmup))
     torch.cuda.synchronize()
 
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_launch + 1)]
-              for _ in range(args.steps)]
-    for row in events:          # torch creates the CUDA event on its first record
-        for e in row:
-            e.record()
+    # Timed region: one event before and one after each step, so that the
+    # kernels of a step follow one another as they do in use (dependent
+    # launches overlap a kernel's set-up with its predecessor).
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for e in ev0 + ev1:          # torch creates the CUDA event on its first record
+        e.record()
     torch.cuda.synchronize()
     sampler = ClockSampler(local)
     if dist:
@@ -281,16 +285,33 @@ def run_ours(args, wl):
     wall0 = time.perf_counter()
     for k in range(args.steps):
         flush.zero_()
-        blk.step_timed(dev_x[k % pool], out, dw, B.DISPLACED, events[k])
+        ev0[k].record()
+        blk.step(dev_x[k % pool], out, dw, B.DISPLACED)
+        ev1[k].record()
     torch.cuda.synchronize()
     wall = time.perf_counter() - wall0
     clocks = sampler.stop()
     if dist:
         dist.barrier()
-    per_launch = [[events[k][i].elapsed_time(events[k][i + 1]) for i in range(n_launch)]
-                  for k in range(args.steps)]
-    step_ms = [events[k][0].elapsed_time(events[k][n_launch]) for k in range(args.steps)]
+    step_ms = [ev0[k].elapsed_time(ev1[k]) for k in range(args.steps)]
     total_ms = sum(step_ms)
+
+    # Per-kernel breakdown: a separate pass with an event before every launch
+    # (dp_block_step_timed); those events keep kernels from overlapping, so the
+    # per-kernel times add up to a little more than the step above.
+    n_bd = min(args.steps, 50)
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_launch + 1)]
+              for _ in range(n_bd)]
+    for row in events:
+        for e in row:
+            e.record()
+    torch.cuda.synchronize()
+    for k in range(n_bd):
+        flush.zero_()
+        blk.step_timed(dev_x[k % pool], out, dw, B.DISPLACED, events[k])
+    torch.cuda.synchronize()
+    per_launch = [[events[k][i].elapsed_time(events[k][i + 1]) for i in range(n_launch)]
+                  for k in range(n_bd)]
     if dist:
         t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -328,7 +349,7 @@ def run_ours(args, wl):
     work = [(f, b) for _, f, b in plan]
     peaks = load_peaks()
     role_ms, role_n = {}, {}
-    for k in range(args.steps):
+    for k in range(n_bd):
         for i, r in enumerate(roles):
             role_ms[r] = role_ms.get(r, 0.0) + per_launch[k][i]
             role_n[r] = role_n.get(r, 0) + 1
@@ -360,7 +381,7 @@ def run_ours(args, wl):
                 "frac": round(dk["gbs"] / peaks["hbm_gbs"], 4), "traffic": traffic,
                 "kernel": dominant, "peak_source": f"{peaks['source']} copy"}
     gn_ms = sum(v for r, v in role_ms.items() if r.startswith("gn"))
-    gn_bytes = sum(work[i][1] for i, r in enumerate(roles) if r.startswith("gn")) * args.steps
+    gn_bytes = sum(work[i][1] for i, r in enumerate(roles) if r.startswith("gn")) * n_bd
     gn = {"achieved_gbs": round(gn_bytes / (gn_ms * 1e-3) / 1e9, 1) if gn_ms else None,
           "peak": peaks["hbm_gbs"],
           "bytes_model": "single pass: read x + write y; two passes: stats read x, apply read x + write y"}

@@ -121,17 +121,25 @@ __global__ void __launch_bounds__(256) conv3x3_small_reg_kernel(
       for (int ci = 0; ci < CIN; ++ci)
         wr[k * CIN + ci] = ci < Cin ? __bfloat162float(w[(static_cast<size_t>(co) * 9 + k) * Cin + ci]) : 0.f;
     const float b0 = bias ? __ldg(bias + co) : 0.f;
-    for (int j = 0; j < 32; ++j) {
-      const int px = ch * 32 + j, c = c0 + px;
-      if (c >= W) break;
-      float acc = b0;
+    // four pixels at a time: independent accumulators hide the FMA latency
+    for (int j = 0; j < 32; j += 4) {
+      const int px = ch * 32 + j;
+      if (c0 + px >= W) break;
+      float acc[4] = {b0, b0, b0, b0};
 #pragma unroll
       for (int kh = 0; kh < 3; ++kh)
 #pragma unroll
         for (int kw = 0; kw < 3; ++kw)
 #pragma unroll
-          for (int ci = 0; ci < CIN; ++ci) acc = fmaf(sx[kh][px + kw][ci], wr[(kh * 3 + kw) * CIN + ci], acc);
-      out[(static_cast<size_t>(r) * W + c) * Cout + co] = __float2bfloat16_rn(acc);
+          for (int ci = 0; ci < CIN; ++ci) {
+            const float wv = wr[(kh * 3 + kw) * CIN + ci];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) acc[u] = fmaf(sx[kh][px + u + kw][ci], wv, acc[u]);
+          }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (c0 + px + u < W)
+          out[(static_cast<size_t>(r) * W + c0 + px + u) * Cout + co] = __float2bfloat16_rn(acc[u]);
     }
   }
 }
