@@ -9,18 +9,21 @@
 //     used[p][g] = stale_global[g] + w * (fresh_local[p][g] - stale_local[p][g])
 // on the raw moments (E[x], E[x^2]).
 //
-// Two bandwidth-bound kernels:
+// Two bandwidth-bound kernels (for tensors too large for the single-pass
+// variant further down), one block per SM, each streaming its share of a
+// band through a ring of shared-memory buffers filled by bulk copies:
 //  1. gn_stats: per-(band, group) sums of x and x^2.  Every thread keeps one
-//     16-byte channel vector of a pixel fixed (block size = a multiple of the
-//     vectors per pixel), so it accumulates per-channel sums in registers and
-//     never has to split a vector across groups (C/G = 10 at C = 320).  The
-//     block folds lanes into channels and channels into groups, then adds
-//     its group sums into an fp64 accumulator with atomics; the last block to
-//     finish (atomic ticket) turns the sums into the fresh moments and the
-//     moments each band uses, and clears the accumulator for the next call.
+//     16-byte channel vector fixed (block size = a multiple of the vectors per
+//     pixel), so it accumulates per-channel sums in registers and never has
+//     to split a vector across groups (C/G = 10 at C = 320).  The block folds
+//     lanes into channels and channels into groups, then adds its group sums
+//     into an fp64 accumulator with atomics; the last block to finish (atomic
+//     ticket) turns the sums into the fresh moments and the moments each band
+//     uses, and clears the accumulator for the next call.
 //  2. gn_apply: y = x * scale_c + shift_c (+ SiLU), cast and stored with
-//     16-byte vectors.  Blocks walk the image in the reverse order of the
-//     stats pass so that the most recently read part of x is still in L2.
+//     coalesced 16-byte vectors.  Blocks walk the image in the reverse order
+//     of the stats pass so that the most recently read part of x is still in
+//     L2.
 #include <math.h>
 
 #include <mutex>
@@ -103,8 +106,39 @@ struct GnArgs {
   int S;        // blocks per band
   int vpp;      // 16-byte vectors per pixel
   int lanes;    // pixel lanes per block (blockDim = vpp * lanes)
+  int piece;    // pixels per bulk copy (at most 32 KiB)
   float eps, w;
   int silu, mode;
+};
+
+// The two-pass kernels stream their share of x through a ring of kGnStages
+// shared-memory buffers filled by bulk copies (one block per SM, about
+// 128 KiB in flight per SM), so the number of bytes in flight no longer
+// depends on how many loads each thread keeps outstanding.
+constexpr int kGnStages = 4;
+constexpr int kGnPieceBytes = 32768;
+
+// Ring of one block's pixel range [beg, end) of band p.
+template <typename T>
+struct GnRing {
+  T* buf;              // [kGnStages][piece][C]
+  uint64_t* full;      // [kGnStages]
+  const T* src;        // first pixel of the range
+  int n, piece, C;     // pixels in the range, pixels per piece
+  __device__ int pieces() const { return (n + piece - 1) / piece; }
+  __device__ int count(int k) const { return min(piece, n - k * piece); }
+  __device__ T* stage(int k) const { return buf + static_cast<size_t>(k % kGnStages) * piece * C; }
+  // thread 0: copy piece k into its stage
+  __device__ void issue(int k) const {
+    const uint32_t bytes = static_cast<uint32_t>(count(k)) * C * sizeof(T);
+    uint64_t* bar = &full[k % kGnStages];
+    mbar_arrive_expect_tx(bar, bytes);
+    bulk_load(stage(k), src + static_cast<size_t>(k) * piece * C, bytes, bar);
+  }
+  __device__ bool wait(int k, int* status) const {
+    int no_abort = 0;
+    return mbar_wait(&full[k % kGnStages], (k / kGnStages) & 1, &no_abort, status);
+  }
 };
 
 template <typename T>
@@ -115,55 +149,64 @@ __global__ void __launch_bounds__(1024) gn_stats_kernel(const T* __restrict__ x,
                                                         const float* __restrict__ stale_local,
                                                         float* __restrict__ fresh_local,
                                                         float* __restrict__ fresh_global,
-                                                        float* __restrict__ used) {
+                                                        float* __restrict__ used,
+                                                        int* __restrict__ status) {
   constexpr int V = Vec<T>::N;
-  extern __shared__ __align__(16) unsigned char gn_smem[];
-  float* ssum = reinterpret_cast<float*>(gn_smem);           // [lanes][C]
+  extern __shared__ __align__(128) unsigned char gn_smem[];
+  T* ring = reinterpret_cast<T*>(gn_smem);                     // [kGnStages][piece][C]
+  float* ssum = reinterpret_cast<float*>(gn_smem + static_cast<size_t>(kGnStages) * a.piece * a.C * sizeof(T));
   float* ssq = ssum + a.lanes * a.C;                          // [lanes][C]
   __shared__ int s_last;
+  __shared__ __align__(8) uint64_t full[kGnStages];
 
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kGnStages; ++i) mbar_init(&full[i], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
   griddep_wait();
   griddep_trigger();
   const int p = blockIdx.x / a.S, s = blockIdx.x % a.S;
   const int v = threadIdx.x % a.vpp, pl = threadIdx.x / a.vpp;
+  const bool worker = threadIdx.x < a.vpp * a.lanes;
   const int chunk = (a.HWp + a.S - 1) / a.S;
-  const int beg = s * chunk;
+  const int beg = min(a.HWp, s * chunk);
   const int end = min(a.HWp, beg + chunk);
-  const T* xb = x + (static_cast<size_t>(p) * a.HWp) * a.C + v * V;
+  GnRing<T> rg{ring, full, x + (static_cast<size_t>(p) * a.HWp + beg) * a.C, end - beg, a.piece, a.C};
+  const int np = rg.pieces();
+  if (threadIdx.x == 0)
+    for (int k = 0; k < min(np, kGnStages); ++k) rg.issue(k);
 
   float sum[V], sq[V];
 #pragma unroll
   for (int j = 0; j < V; ++j) sum[j] = sq[j] = 0.f;
-  int pix = beg + pl;
-  for (; pix + 3 * a.lanes < end; pix += 4 * a.lanes) {
-    float t[4][V];
+  for (int k = 0; k < np; ++k) {
+    rg.wait(k, status);
+    const T* st = rg.stage(k) + v * V;
+    const int cnt = rg.count(k);
+    if (worker) {
+      for (int q = pl; q < cnt; q += a.lanes) {
+        float t[V];
+        Vec<T>::load(st + static_cast<size_t>(q) * a.C, t);
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
-      Vec<T>::load(xb + static_cast<size_t>(pix + u * a.lanes) * a.C, t[u]);
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-#pragma unroll
-      for (int j = 0; j < V; ++j) {
-        sum[j] += t[u][j];
-        sq[j] = fmaf(t[u][j], t[u][j], sq[j]);
+        for (int j = 0; j < V; ++j) {
+          sum[j] += t[j];
+          sq[j] = fmaf(t[j], t[j], sq[j]);
+        }
       }
-  }
-  for (; pix < end; pix += a.lanes) {
-    float t[V];
-    Vec<T>::load(xb + static_cast<size_t>(pix) * a.C, t);
-#pragma unroll
-    for (int j = 0; j < V; ++j) {
-      sum[j] += t[j];
-      sq[j] = fmaf(t[j], t[j], sq[j]);
     }
+    __syncthreads();   // the stage is free again
+    if (threadIdx.x == 0 && k + kGnStages < np) rg.issue(k + kGnStages);
   }
   // 16-byte stores: scalar ones at this stride would conflict 8-way
+  if (worker) {
 #pragma unroll
-  for (int j = 0; j < V; j += 4) {
-    *reinterpret_cast<float4*>(ssum + pl * a.C + v * V + j) =
-        make_float4(sum[j], sum[j + 1], sum[j + 2], sum[j + 3]);
-    *reinterpret_cast<float4*>(ssq + pl * a.C + v * V + j) =
-        make_float4(sq[j], sq[j + 1], sq[j + 2], sq[j + 3]);
+    for (int j = 0; j < V; j += 4) {
+      *reinterpret_cast<float4*>(ssum + pl * a.C + v * V + j) =
+          make_float4(sum[j], sum[j + 1], sum[j + 2], sum[j + 3]);
+      *reinterpret_cast<float4*>(ssq + pl * a.C + v * V + j) =
+          make_float4(sq[j], sq[j + 1], sq[j + 2], sq[j + 3]);
+    }
   }
   __syncthreads();
   // lanes -> channels (row 0 of the scratch), then channels -> groups
@@ -244,15 +287,30 @@ __global__ void __launch_bounds__(1024) gn_apply_kernel(const T* __restrict__ x,
                                                         const float* __restrict__ gamma,
                                                         const float* __restrict__ beta,
                                                         const float* __restrict__ used,
-                                                        GnArgs a) {
+                                                        GnArgs a, int* __restrict__ status) {
   constexpr int V = Vec<T>::N;
-  extern __shared__ __align__(16) unsigned char gn_smem[];
-  float* sscale = reinterpret_cast<float*>(gn_smem);
+  extern __shared__ __align__(128) unsigned char gn_smem[];
+  T* ring = reinterpret_cast<T*>(gn_smem);                     // [kGnStages][piece][C]
+  float* sscale = reinterpret_cast<float*>(gn_smem + static_cast<size_t>(kGnStages) * a.piece * a.C * sizeof(T));
   float* sshift = sscale + a.C;
+  __shared__ __align__(8) uint64_t full[kGnStages];
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kGnStages; ++i) mbar_init(&full[i], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
   griddep_wait();
   griddep_trigger();
   const int b = gridDim.x - 1 - blockIdx.x;   // reverse walk: L2-hot tail first
   const int p = b / a.S, s = b % a.S;
+  const int chunk = (a.HWp + a.S - 1) / a.S;
+  const int beg = min(a.HWp, s * chunk);
+  const int end = min(a.HWp, beg + chunk);
+  const size_t off = (static_cast<size_t>(p) * a.HWp + beg) * a.C;
+  GnRing<T> rg{ring, full, x + off, end - beg, a.piece, a.C};
+  const int np = rg.pieces();
+  if (threadIdx.x == 0)
+    for (int k = 0; k < min(np, kGnStages); ++k) rg.issue(k);
   const int cg = a.C / a.G;
   for (int c = threadIdx.x; c < a.C; c += blockDim.x) {
     const int g = c / cg;
@@ -264,40 +322,31 @@ __global__ void __launch_bounds__(1024) gn_apply_kernel(const T* __restrict__ x,
   }
   __syncthreads();
   const int v = threadIdx.x % a.vpp, pl = threadIdx.x / a.vpp;
+  const bool worker = threadIdx.x < a.vpp * a.lanes;
   float sc[V], sh[V];
 #pragma unroll
   for (int j = 0; j < V; ++j) {
-    sc[j] = sscale[v * V + j];
-    sh[j] = sshift[v * V + j];
+    sc[j] = worker ? sscale[v * V + j] : 0.f;
+    sh[j] = worker ? sshift[v * V + j] : 0.f;
   }
-  const int chunk = (a.HWp + a.S - 1) / a.S;
-  const int beg = s * chunk;
-  const int end = min(a.HWp, beg + chunk);
-  const size_t off = (static_cast<size_t>(p) * a.HWp) * a.C + v * V;
-  const T* xb = x + off;
-  T* yb = y + off;
-  auto body = [&](float (&t)[V]) {
+  T* yb = y + off + v * V;
+  for (int k = 0; k < np; ++k) {
+    rg.wait(k, status);
+    const T* st = rg.stage(k) + v * V;
+    const int cnt = rg.count(k);
+    if (worker) {
+      T* yk = yb + static_cast<size_t>(k) * a.piece * a.C;
+      for (int q = pl; q < cnt; q += a.lanes) {
+        float t[V];
+        Vec<T>::load(st + static_cast<size_t>(q) * a.C, t);
 #pragma unroll
-    for (int j = 0; j < V; ++j) t[j] = fmaf(t[j], sc[j], sh[j]);
-    if (a.silu) silu_vec<T>(t);
-  };
-  int pix = beg + pl;
-  for (; pix + 3 * a.lanes < end; pix += 4 * a.lanes) {
-    float t[4][V];
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-      Vec<T>::load(xb + static_cast<size_t>(pix + u * a.lanes) * a.C, t[u]);
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      body(t[u]);
-      Vec<T>::store(yb + static_cast<size_t>(pix + u * a.lanes) * a.C, t[u]);
+        for (int j = 0; j < V; ++j) t[j] = fmaf(t[j], sc[j], sh[j]);
+        if (a.silu) silu_vec<T>(t);
+        Vec<T>::store(yk + static_cast<size_t>(q) * a.C, t);
+      }
     }
-  }
-  for (; pix < end; pix += a.lanes) {
-    float t[V];
-    Vec<T>::load(xb + static_cast<size_t>(pix) * a.C, t);
-    body(t);
-    Vec<T>::store(yb + static_cast<size_t>(pix) * a.C, t);
+    __syncthreads();   // the stage is free again
+    if (threadIdx.x == 0 && k + kGnStages < np) rg.issue(k + kGnStages);
   }
 }
 
@@ -580,19 +629,21 @@ __global__ void __launch_bounds__(1024, 1) gn_fused_kernel(
 
 static int gn_plan(int H, int W, int C, int G, int P, int dtype, GnArgs* a) {
   const int V = dtype == DP_BF16 ? 8 : 4;
+  const int row_bytes = C * (dtype == DP_BF16 ? 2 : 4);
   a->HWp = (H / P) * W;
   a->C = C;
   a->G = G;
   a->P = P;
   a->vpp = C / V;
-  a->lanes = a->vpp >= 512 ? 1 : 512 / a->vpp;
-  if (a->vpp * a->lanes > 1024) a->lanes = 1024 / a->vpp;
-  // One full wave of resident blocks (2 per SM at up to 1024 threads each).
-  int s = (2 * num_sms()) / P;
-  const int by_work = (a->HWp + 4 * a->lanes - 1) / (4 * a->lanes);
-  if (s > by_work) s = by_work;
+  a->lanes = a->vpp >= 1024 ? 1 : 1024 / a->vpp;
+  // one block per SM, the SMs shared out among the bands
+  int s = num_sms() / P;
   if (s > kGnMaxSplits) s = kGnMaxSplits;
   a->S = s < 1 ? 1 : s;
+  const int chunk = (a->HWp + a->S - 1) / a->S;
+  int piece = kGnPieceBytes / row_bytes;
+  if (piece > chunk) piece = chunk;
+  a->piece = piece < 1 ? 1 : piece;
   return DP_OK;
 }
 
@@ -749,27 +800,45 @@ int gn_launch(const void* x, void* y, const float* gamma, const float* beta, int
   }
   const int threads = a.vpp * a.lanes;
   const int blocks = a.P * a.S;
-  size_t smem_stats = static_cast<size_t>(a.lanes) * C * 2 * sizeof(float);
-  const size_t smem_fin = static_cast<size_t>(P) * G * 2 * sizeof(double);
-  if (smem_fin > smem_stats) smem_stats = smem_fin;
-  const size_t smem_apply = static_cast<size_t>(C) * 2 * sizeof(float);
-  if (smem_stats > 48 * 1024 || smem_apply > 48 * 1024) {
-    static bool attr_done[2] = {false, false};
-    if (!attr_done[dtype]) {
-      if (dtype == DP_BF16) {
-        cudaFuncSetAttribute(gn_stats_kernel<__nv_bfloat16>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
-        cudaFuncSetAttribute(gn_apply_kernel<__nv_bfloat16>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
-      } else {
-        cudaFuncSetAttribute(gn_stats_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             160 * 1024);
-        cudaFuncSetAttribute(gn_apply_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             160 * 1024);
-      }
-      attr_done[dtype] = true;
+  const size_t ring = static_cast<size_t>(kGnStages) * a.piece * C * (dtype == DP_BF16 ? 2 : 4);
+  size_t red = static_cast<size_t>(a.lanes) * C * 2 * sizeof(float);
+  const size_t fin = static_cast<size_t>(P) * G * 2 * sizeof(double);
+  if (fin > ring + red) red = fin - ring;
+  const size_t smem_stats = ring + red;
+  const size_t smem_apply = ring + static_cast<size_t>(C) * 2 * sizeof(float);
+  if (smem_stats > 220 * 1024 || smem_apply > 220 * 1024)
+    return set_error(DP_ERR_UNSUPPORTED, "groupnorm: C = %d needs too much shared memory", C);
+  // dynamic shared memory above 48 KiB must be opted into; keep the largest
+  // size set so far per (dtype, device)
+  static size_t attr_set[2][32] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  size_t& done = attr_set[dtype][dev & 31];
+  const size_t need = smem_stats > smem_apply ? smem_stats : smem_apply;
+  if (need > done) {
+    const int lim = static_cast<int>(need);
+    int rc = 0;
+    if (dtype == DP_BF16) {
+      rc = cuda_check(cudaFuncSetAttribute(gn_stats_kernel<__nv_bfloat16>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, lim),
+                      "groupnorm stats smem attribute");
+      if (!rc)
+        rc = cuda_check(cudaFuncSetAttribute(gn_apply_kernel<__nv_bfloat16>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, lim),
+                        "groupnorm apply smem attribute");
+    } else {
+      rc = cuda_check(cudaFuncSetAttribute(gn_stats_kernel<float>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, lim),
+                      "groupnorm stats smem attribute");
+      if (!rc)
+        rc = cuda_check(cudaFuncSetAttribute(gn_apply_kernel<float>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, lim),
+                        "groupnorm apply smem attribute");
     }
+    if (rc) return rc;
+    done = need;
   }
+  int* status = device_status_ptr();
   const float* cgl = stale_global;
   const float* cll = stale_local;
   const float* cused = used;
@@ -778,23 +847,23 @@ int gn_launch(const void* x, void* y, const float* gamma, const float* beta, int
     int rc = launch_kernel(gn_stats_kernel<__nv_bfloat16>, dim3(blocks), dim3(threads), smem_stats,
                            stream, false, "groupnorm stats launch",
                            static_cast<const __nv_bfloat16*>(x), a, acc, counter, cgl, cll,
-                           fresh_local, fresh_global, used);
+                           fresh_local, fresh_global, used, status);
     if (rc) return rc;
     mark_launch(stream);
     return launch_kernel(gn_apply_kernel<__nv_bfloat16>, dim3(blocks), dim3(threads), smem_apply,
                          stream, false, "groupnorm apply launch",
                          static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(y), gamma,
-                         beta, cused, a);
+                         beta, cused, a, status);
   }
   mark_launch(stream);
   int rc = launch_kernel(gn_stats_kernel<float>, dim3(blocks), dim3(threads), smem_stats, stream,
                          false, "groupnorm stats launch", static_cast<const float*>(x), a, acc,
-                         counter, cgl, cll, fresh_local, fresh_global, used);
+                         counter, cgl, cll, fresh_local, fresh_global, used, status);
   if (rc) return rc;
   mark_launch(stream);
   return launch_kernel(gn_apply_kernel<float>, dim3(blocks), dim3(threads), smem_apply, stream, false,
                        "groupnorm apply launch", static_cast<const float*>(x), static_cast<float*>(y),
-                       gamma, beta, cused, a);
+                       gamma, beta, cused, a, status);
 }
 
 // ---------------------------------------------------------------------------

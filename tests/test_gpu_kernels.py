@@ -67,6 +67,40 @@ def test_groupnorm_parity(case, mode):
     assert B.dp_device_status() == 0
 
 
+@pytest.mark.parametrize("case", GN_CASES[:5])
+def test_groupnorm_two_pass_with_minimal_workspace(case):
+    """A workspace of only 256 + 128 P G bytes runs the two-kernel path even for
+    tensors the single-pass kernel could hold (tiny bands, fewer pixels per
+    block than SMs per band)."""
+    C, H, W, P, G, dtype, silu = case
+    mode = B.DISPLACED
+    r = rng(3 * C + H)
+    xs = rounded(r.standard_normal((C, H, W)) * 1.3 + 0.2, dtype)
+    x = rounded(xs + 0.05 * r.standard_normal((C, H, W)) + 0.02, dtype)
+    gamma = 1 + 0.3 * r.standard_normal(C)
+    beta = 0.3 * r.standard_normal(C)
+    sg, sl = O.refresh_stats(O.gn_fresh_local(xs, P, G))
+    sg, sl = sg.astype(np.float32).astype(np.float64), sl.astype(np.float32).astype(np.float64)
+    y_ref, f_ref, used_ref, _ = O.groupnorm_async(x, gamma, beta, P, G, 1e-5, 1.0, silu, mode, sg, sl)
+    xd = dev_img(x, dtype)
+    yd = torch.empty_like(xd)
+    fresh = torch.zeros(P * G * 2, device="cuda")
+    used = torch.zeros(P * G * 2, device="cuda")
+    ws = torch.zeros(256 + 128 * P * G, dtype=torch.uint8, device="cuda")
+    for _ in range(2):
+        B.dp_groupnorm_async(xd, yd, dev_f32(gamma), dev_f32(beta), H, W, C, G, P, 1e-5, 1.0, silu,
+                             mode, B.BF16 if dtype == "bf16" else B.FP32, dev_f32(sg), dev_f32(sl),
+                             fresh, used, ws)
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(host(fresh).reshape(P, G, 2), f_ref, rtol=0, atol=STATS_ATOL)
+    np.testing.assert_allclose(host(used).reshape(P, G, 2), used_ref, rtol=0, atol=STATS_ATOL)
+    if dtype == "fp32":
+        check(host_img(yd), y_ref, atol=1e-4, rl2=1e-5, what="gn fp32 two-pass")
+    else:
+        check(host_img(yd), y_ref, what="gn bf16 two-pass", storage_rel=BF16_HALF_ULP)
+    assert B.dp_device_status() == 0
+
+
 def test_groupnorm_full_size_stats():
     """Statistics at the 1x320x480x480, P = 8 size, displaced mode."""
     C, H, W, P, G = 320, 480, 480, 8, 32
