@@ -127,6 +127,21 @@ def dist_env():
     return ws, rank, local
 
 
+def max_over_ranks(x, dist, device):
+    """The largest of every rank's x (the job's time is the slowest replica's)."""
+    if dist is None:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(world_size, flops_per_step, steps, total_ms):
+    """Whole-job throughput: every replica runs `steps` steps of `flops_per_step`."""
+    return world_size * flops_per_step * steps / (total_ms * 1e-3) / 1e12
+
+
 def block_kind(B, wl):
     return {"gn_conv": B.GN_CONV, "resblock": B.RESBLOCK, "attn": B.ATTN,
             "unet_mini": B.UNET_MINI}[wl.kind]
@@ -312,10 +327,7 @@ def run_ours(args, wl):
     torch.cuda.synchronize()
     per_launch = [[events[k][i].elapsed_time(events[k][i + 1]) for i in range(n_launch)]
                   for k in range(n_bd)]
-    if dist:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dist, dev)
 
     # end-to-end: pinned host input -> device, block step, result -> pinned host, every step
     e2e_ms = 0.0
@@ -334,16 +346,14 @@ def run_ours(args, wl):
         ev1[k].record()
     torch.cuda.synchronize()
     e2e_ms = sum(ev0[k].elapsed_time(ev1[k]) for k in range(args.steps))
+    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
     if dist:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
         dist.barrier()
     status = B.dp_device_status()
 
     flops = blk.flops
-    value = ws * flops * args.steps / (total_ms * 1e-3) / 1e12
-    e2e_value = ws * flops * args.steps / (e2e_ms * 1e-3) / 1e12
+    value = job_tflops(ws, flops, args.steps, total_ms)
+    e2e_value = job_tflops(ws, flops, args.steps, e2e_ms)
 
     # per-kernel roles: mean duration, share, roofline of the dominant one
     work = [(f, b) for _, f, b in plan]
