@@ -377,6 +377,7 @@ def run_ours(args, wl):
     dk = kernels[dominant]
     src = {"conv": ["dp_gemm.cu"], "linear": ["dp_gemm.cu"], "attn": ["dp_attn.cu"],
            "gn_stats": ["dp_gn.cu"], "gn_apply": ["dp_gn.cu"], "gn_fused": ["dp_gn.cu"],
+           "gn_cluster": ["dp_gn.cu"],
            "copy": ["dp_refresh.cu"], "conv_small": ["dp_conv_small.cu"], "splitk_finish": ["dp_gemm.cu"]}[dominant]
     traffic = load_traffic(f"{dominant}:{wl.name}", kernel_source_hash(src))
     if dk["tflops"]:

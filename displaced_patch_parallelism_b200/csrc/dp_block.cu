@@ -237,7 +237,9 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
       const double bytes = static_cast<double>(H) * W * ch * e;
       int nb, chunk, th;
       size_t sm;
-      if (gn_fused_plan(H, W, ch, G, P, d->dtype, &nb, &chunk, &th, &sm)) {
+      if (gn_cluster_plan(H, W, ch, G, P, d->dtype, mode, &nb, &chunk, &th, &sm)) {
+        plan->push(DP_KERNEL_GN_CLUSTER, 0.0, 2.0 * bytes);
+      } else if (gn_fused_plan(H, W, ch, G, P, d->dtype, &nb, &chunk, &th, &sm)) {
         plan->push(DP_KERNEL_GN_FUSED, 0.0, 2.0 * bytes);
       } else {
         plan->push(DP_KERNEL_GN_STATS, 0.0, bytes);

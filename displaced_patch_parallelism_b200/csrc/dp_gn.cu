@@ -627,6 +627,195 @@ __global__ void __launch_bounds__(1024, 1) gn_fused_kernel(
   }
 }
 
+// ---------------------------------------------------------------------------
+// Cluster variant for DISPLACED and NAIVE steps, whose bands need only their
+// own fresh moments: one thread-block cluster per band (up to 16 CTAs, one
+// per SM) holds the band in shared memory.  Each CTA bulk-copies its chunk,
+// leaves its (group) sums in shared memory, and after a cluster barrier every
+// CTA adds all the cluster's sums through distributed shared memory (in rank
+// order, so every CTA gets the same bits).  It normalises its chunk from
+// shared memory and stores it.  No grid-wide barrier; the whole-image
+// moments (fresh_global) are formed by whichever band finishes last.
+struct GnClusterArgs {
+  int HWp, C, G, P, vpp, lanes, chunk, cpb;
+  float eps, w;
+  int silu, mode;
+};
+
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t cluster_addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
+  return v;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(512, 1) gn_cluster_kernel(
+    const T* __restrict__ x, T* __restrict__ y, const float* __restrict__ gamma,
+    const float* __restrict__ beta, GnClusterArgs a, unsigned* __restrict__ ticket,
+    const float* __restrict__ stale_global, const float* __restrict__ stale_local,
+    float* __restrict__ fresh_local, float* __restrict__ fresh_global, float* __restrict__ used,
+    int* __restrict__ status) {
+  constexpr int V = Vec<T>::N;
+  extern __shared__ __align__(128) unsigned char gn_smem[];
+  T* data = reinterpret_cast<T*>(gn_smem);                               // [chunk][C]
+  const size_t data_bytes = ((static_cast<size_t>(a.chunk) * a.C * sizeof(T)) + 127) & ~size_t(127);
+  float* ssum = reinterpret_cast<float*>(gn_smem + data_bytes);          // [lanes][C]
+  float* ssq = ssum + a.lanes * a.C;                                     // [lanes][C]
+  float* gpart = ssq + a.lanes * a.C;                                    // [G][2], read by the cluster
+  double* f = reinterpret_cast<double*>(gpart + 2 * a.G + (a.G & 1) * 2);  // [G][2]
+  float* sscale = reinterpret_cast<float*>(f + 2 * a.G);                 // [C]
+  float* sshift = sscale + a.C;                                          // [C]
+  __shared__ __align__(8) uint64_t load_bar;
+  __shared__ int s_last;
+
+  const int p = blockIdx.x / a.cpb;
+  const int rank = static_cast<int>(cluster_ctarank());
+  const int beg = min(a.HWp, rank * a.chunk);
+  const int end = min(a.HWp, beg + a.chunk);
+  const int npix = end - beg;
+  const int v = threadIdx.x % a.vpp, pl = threadIdx.x / a.vpp;
+  const bool worker = threadIdx.x < a.vpp * a.lanes;
+  const int cg = a.C / a.G;
+  const size_t row_bytes = static_cast<size_t>(a.C) * sizeof(T);
+
+  if (threadIdx.x == 0) {
+    mbar_init(&load_bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  griddep_wait();
+  griddep_trigger();
+  if (threadIdx.x == 0 && npix > 0) {
+    const uint32_t total = static_cast<uint32_t>(npix * row_bytes);
+    mbar_arrive_expect_tx(&load_bar, total);
+    const char* src = reinterpret_cast<const char*>(x) + (static_cast<size_t>(p) * a.HWp + beg) * row_bytes;
+    char* dst = reinterpret_cast<char*>(data);
+    for (uint32_t off = 0; off < total; off += 16384u)
+      bulk_load(dst + off, src + off, min(16384u, total - off), &load_bar);
+  }
+  if (npix > 0) {
+    int no_abort = 0;
+    mbar_wait(&load_bar, 0, &no_abort, status);
+  }
+  __syncthreads();
+
+  // ---- this CTA's (group) sums
+  {
+    float sum[V], sq[V];
+#pragma unroll
+    for (int j = 0; j < V; ++j) sum[j] = sq[j] = 0.f;
+    if (worker) {
+      for (int pix = pl; pix < npix; pix += a.lanes) {
+        float t[V];
+        Vec<T>::load(data + static_cast<size_t>(pix) * a.C + v * V, t);
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+          sum[j] += t[j];
+          sq[j] = fmaf(t[j], t[j], sq[j]);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < V; j += 4) {
+        *reinterpret_cast<float4*>(ssum + pl * a.C + v * V + j) =
+            make_float4(sum[j], sum[j + 1], sum[j + 2], sum[j + 3]);
+        *reinterpret_cast<float4*>(ssq + pl * a.C + v * V + j) =
+            make_float4(sq[j], sq[j + 1], sq[j + 2], sq[j + 3]);
+      }
+    }
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < a.C; c += blockDim.x) {
+    float cs = 0.f, cq = 0.f;
+    for (int l = 0; l < a.lanes; ++l) {
+      cs += ssum[l * a.C + c];
+      cq += ssq[l * a.C + c];
+    }
+    ssum[c] = cs;
+    ssq[c] = cq;
+  }
+  __syncthreads();
+  for (int g = threadIdx.x; g < a.G; g += blockDim.x) {
+    float ds = 0.f, dq = 0.f;
+    for (int c = g * cg; c < (g + 1) * cg; ++c) {
+      ds += ssum[c];
+      dq += ssq[c];
+    }
+    gpart[2 * g] = ds;
+    gpart[2 * g + 1] = dq;
+  }
+  cluster_sync_all();   // every CTA of the band has its sums in shared memory
+
+  // ---- the band's fresh moments, added over the cluster in rank order
+  const double n = static_cast<double>(a.HWp) * cg;
+  for (int i = threadIdx.x; i < 2 * a.G; i += blockDim.x) {
+    const uint32_t local = smem_u32(gpart + i);
+    double s = 0.0;
+    for (int k = 0; k < a.cpb; ++k) s += ld_dsmem_f32(mapa_shared(local, static_cast<uint32_t>(k)));
+    f[i] = s / n;
+  }
+  __syncthreads();
+  const float* sl = stale_local + static_cast<size_t>(p) * a.G * 2;
+  for (int c = threadIdx.x; c < a.C; c += blockDim.x) {
+    const int g = c / cg;
+    double m1 = f[2 * g], m2 = f[2 * g + 1];
+    if (a.mode == DP_MODE_DISPLACED) {
+      m1 = static_cast<double>(stale_global[2 * g]) + a.w * (m1 - static_cast<double>(sl[2 * g]));
+      m2 = static_cast<double>(stale_global[2 * g + 1]) + a.w * (m2 - static_cast<double>(sl[2 * g + 1]));
+    }
+    double var = m2 - m1 * m1;
+    if (var < 0.0) var = f[2 * g + 1] - f[2 * g] * f[2 * g];
+    const float sc = rsqrtf(static_cast<float>(var) + a.eps) * gamma[c];
+    sscale[c] = sc;
+    sshift[c] = beta[c] - static_cast<float>(m1) * sc;
+    if (rank == 0 && c % cg == 0) {
+      used[(p * a.G + g) * 2] = static_cast<float>(m1);
+      used[(p * a.G + g) * 2 + 1] = static_cast<float>(var);
+      fresh_local[(p * a.G + g) * 2] = static_cast<float>(f[2 * g]);
+      fresh_local[(p * a.G + g) * 2 + 1] = static_cast<float>(f[2 * g + 1]);
+    }
+  }
+  __syncthreads();
+
+  // ---- apply from shared memory, coalesced 16-byte stores
+  if (worker) {
+    float sc[V], sh[V];
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+      sc[j] = sscale[v * V + j];
+      sh[j] = sshift[v * V + j];
+    }
+    T* yb = y + (static_cast<size_t>(p) * a.HWp + beg) * a.C + v * V;
+    for (int pix = pl; pix < npix; pix += a.lanes) {
+      float t[V];
+      Vec<T>::load(data + static_cast<size_t>(pix) * a.C + v * V, t);
+#pragma unroll
+      for (int j = 0; j < V; ++j) t[j] = fmaf(t[j], sc[j], sh[j]);
+      if (a.silu) silu_vec<T>(t);
+      Vec<T>::store(yb + static_cast<size_t>(pix) * a.C, t);
+    }
+  }
+  // the cluster's other CTAs must be done reading gpart before this CTA leaves
+  cluster_sync_all();
+
+  // ---- the band that finishes last forms the whole-image moments
+  if (rank == 0 && fresh_global) {
+    if (threadIdx.x == 0) {
+      __threadfence();
+      s_last = atomicAdd(ticket, 1u) == static_cast<unsigned>(a.P - 1);
+    }
+    __syncthreads();
+    if (s_last) {
+      __threadfence();
+      for (int i = threadIdx.x; i < 2 * a.G; i += blockDim.x) {
+        double s = 0.0;
+        for (int q = 0; q < a.P; ++q) s += __ldcg(fresh_local + q * a.G * 2 + i);
+        fresh_global[i] = static_cast<float>(s / a.P);
+      }
+      if (threadIdx.x == 0) *ticket = 0u;
+    }
+  }
+}
+
 static int gn_plan(int H, int W, int C, int G, int P, int dtype, GnArgs* a) {
   const int V = dtype == DP_BF16 ? 8 : 4;
   const int row_bytes = C * (dtype == DP_BF16 ? 2 : 4);
@@ -703,6 +892,108 @@ bool gn_fused_plan(int H, int W, int C, int G, int P, int dtype, int* blocks, in
   *chunk = static_cast<int>(ch);
   *threads = ((vpp * lanes + 31) / 32) * 32;
   *smem = need;
+  return true;
+}
+
+// Plan of the cluster variant: CTAs per band (the cluster size), pixels per
+// CTA and shared memory; false for SYNC steps (they need every band's
+// moments) and when a band does not fit in 16 CTAs' shared memory.
+bool gn_cluster_plan(int H, int W, int C, int G, int P, int dtype, int mode, int* cpb, int* chunk,
+                     int* threads, size_t* smem) {
+  if (mode == DP_MODE_SYNC) return false;
+  const int e = dtype == DP_BF16 ? 2 : 4;
+  const int vpp = C / (16 / e);
+  if (vpp > 512) return false;
+  const int lanes = 512 / vpp;
+  const long HWp = static_cast<long>(H / P) * W;
+  const int n = static_cast<int>(HWp < 16 ? HWp : 16);
+  if (n < 1) return false;
+  const long ch = (HWp + n - 1) / n;
+  const size_t data = ((static_cast<size_t>(ch) * C * e) + 127) & ~size_t(127);
+  const size_t need = data + static_cast<size_t>(lanes) * C * 8 + static_cast<size_t>(G) * 8 + 16 +
+                      static_cast<size_t>(G) * 16 + static_cast<size_t>(C) * 8;
+  if (need > 220 * 1024) return false;
+  *cpb = n;
+  *chunk = static_cast<int>(ch);
+  *threads = ((vpp * lanes + 31) / 32) * 32;
+  *smem = need;
+  return true;
+}
+
+// Launches the cluster variant when it applies; false leaves the choice to
+// the other variants (*rc untouched).
+static bool gn_cluster_launch(const void* x, void* y, const float* gamma, const float* beta, int H,
+                              int W, int C, int G, int P, float eps, float w, int silu, int mode,
+                              int dtype, const float* stale_global, const float* stale_local,
+                              float* fresh_local, float* fresh_global, float* used, unsigned* ticket,
+                              cudaStream_t stream, int* rc) {
+  int cpb, chunk, threads;
+  size_t smem;
+  if (!gn_cluster_plan(H, W, C, G, P, dtype, mode, &cpb, &chunk, &threads, &smem)) return false;
+  const void* fn = dtype == DP_BF16 ? reinterpret_cast<const void*>(gn_cluster_kernel<__nv_bfloat16>)
+                                    : reinterpret_cast<const void*>(gn_cluster_kernel<float>);
+  static size_t attr_set[2][32] = {};
+  static int usable[2][32] = {};   // 0 unknown, 1 yes, -1 no
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (usable[dtype][dev & 31] < 0) return false;
+  if (smem > attr_set[dtype][dev & 31]) {
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+      cudaGetLastError();
+      usable[dtype][dev & 31] = -1;
+      return false;
+    }
+    attr_set[dtype][dev & 31] = smem;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(P * cpb);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cpb;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  int na = 1;
+  if (pdl_enabled()) {
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    na = 2;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  if (usable[dtype][dev & 31] == 0) {
+    int clusters = 0;
+    const cudaError_t e = cudaOccupancyMaxActiveClusters(&clusters, fn, &cfg);
+    if (e != cudaSuccess || clusters < 1) {
+      cudaGetLastError();
+      usable[dtype][dev & 31] = -1;
+      return false;
+    }
+    usable[dtype][dev & 31] = 1;
+  }
+  GnClusterArgs a;
+  a.HWp = (H / P) * W;
+  a.C = C;
+  a.G = G;
+  a.P = P;
+  a.vpp = C / (dtype == DP_BF16 ? 8 : 4);
+  a.lanes = 512 / a.vpp;
+  a.chunk = chunk;
+  a.cpb = cpb;
+  a.eps = eps;
+  a.w = w;
+  a.silu = silu;
+  a.mode = mode;
+  int* status = device_status_ptr();
+  void* args[] = {const_cast<void**>(&x), &y, const_cast<float**>(&gamma), const_cast<float**>(&beta),
+                  &a, &ticket, const_cast<float**>(&stale_global), const_cast<float**>(&stale_local),
+                  &fresh_local, &fresh_global, &used, &status};
+  mark_launch(stream);
+  *rc = cuda_check(cudaLaunchKernelExC(&cfg, fn, args), "cluster groupnorm launch");
   return true;
 }
 
@@ -791,6 +1082,9 @@ int gn_launch(const void* x, void* y, const float* gamma, const float* beta, int
   double* acc = reinterpret_cast<double*>(static_cast<char*>(workspace) + 256);
   {
     int rc = 0;
+    if (gn_cluster_launch(x, y, gamma, beta, H, W, C, G, P, eps, w, silu, mode, dtype, stale_global,
+                          stale_local, fresh_local, fresh_global, used, counter, stream, &rc))
+      return rc;
     float2* part = reinterpret_cast<float2*>(static_cast<char*>(workspace) + gn_acc_bytes(P, G));
     if (workspace_bytes >= gn_workspace_bytes(P, G) &&
         gn_fused_launch(x, y, gamma, beta, H, W, C, G, P, eps, w, silu, mode, dtype, stale_global,

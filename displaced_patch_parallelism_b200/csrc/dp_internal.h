@@ -8,6 +8,8 @@ namespace dp {
 
 size_t gn_acc_bytes(int P, int G);
 size_t gn_workspace_bytes(int P, int G);
+bool gn_cluster_plan(int H, int W, int C, int G, int P, int dtype, int mode, int* cpb, int* chunk,
+                     int* threads, size_t* smem);
 bool gn_fused_plan(int H, int W, int C, int G, int P, int dtype, int* blocks, int* chunk,
                    int* threads, size_t* smem);
 int gn_launch(const void* x, void* y, const float* gamma, const float* beta, int H, int W, int C,

@@ -351,6 +351,7 @@ DP_API int dp_block_step(const dp_block_desc* d, dp_block_state* s, const void* 
 #define DP_KERNEL_COPY 6       /* device copy                                   */
 #define DP_KERNEL_CONV_SMALL 7 /* direct 3x3 conv for few input channels        */
 #define DP_KERNEL_SPLITK_FINISH 8 /* sum of split-K partials + bias + residual   */
+#define DP_KERNEL_GN_CLUSTER 9  /* GroupNorm, one thread-block cluster per band */
 
 /*
  * Number of kernel launches one displaced dp_block_step makes for this

@@ -61,8 +61,11 @@ def test_mode_for_step_matches_input_module(B):
 def test_block_desc_validation(B):
     d = B.dp_block_desc_init(B.RESBLOCK, 128, 128, 320, 320, 32, 4, 0, B.BF16, 1, 1e-5, 1.0)
     assert B.dp_block_workspace_size(d) > 4 * 128 * 128 * 320 * 2
-    # a GroupNorm whose tensor fits in shared memory is one launch
+    # a GroupNorm whose tensor fits in shared memory is one launch: one cluster
+    # per band in displaced steps, a grid-wide single pass in sync steps
     assert [B.dp_block_launch_info(d, B.DISPLACED, i)[0] for i in range(B.dp_block_launch_count(d))] \
+        == ["gn_cluster", "conv", "gn_cluster", "conv"]
+    assert [B.dp_block_launch_info(d, B.SYNC, i)[0] for i in range(B.dp_block_launch_count(d))] \
         == ["gn_fused", "conv", "gn_fused", "conv"]
     assert abs(B.dp_block_flops(d) - 2 * 2 * 128 * 128 * 320 * 9 * 320) < 1
     assert abs(sum(B.dp_block_launch_info(d, B.DISPLACED, i)[1] for i in range(4))
@@ -72,7 +75,7 @@ def test_block_desc_validation(B):
         == ["gn_fused", "conv", "gn_fused", "linear", "conv"]
     da = B.dp_block_desc_init(B.ATTN, 64, 64, 640, 640, 32, 4, 10, B.BF16, 0, 1e-5, 1.0)
     assert [B.dp_block_launch_info(da, B.DISPLACED, i)[0] for i in range(B.dp_block_launch_count(da))] \
-        == ["gn_fused", "linear", "attn", "linear"]
+        == ["gn_cluster", "linear", "attn", "linear"]
     # naive attention sees only its own band's keys
     assert B.dp_block_launch_info(da, B.NAIVE, 2)[1] * 4 == B.dp_block_launch_info(da, B.DISPLACED, 2)[1]
     # the 480x480 tensor does not fit on chip: two GroupNorm passes
@@ -83,7 +86,7 @@ def test_block_desc_validation(B):
     # split into runs and a finish kernel adds them
     d5 = B.dp_block_desc_init(B.RESBLOCK, 32, 32, 640, 1280, 32, 4, 0, B.BF16, 1, 1e-5, 1.0)
     assert [B.dp_block_launch_info(d5, B.DISPLACED, i)[0] for i in range(B.dp_block_launch_count(d5))] \
-        == ["gn_fused", "conv", "splitk_finish", "gn_fused", "linear", "conv", "splitk_finish"]
+        == ["gn_cluster", "conv", "splitk_finish", "gn_cluster", "linear", "conv", "splitk_finish"]
     du = B.dp_block_desc_init(B.UNET_MINI, 128, 128, 4, 0, 32, 4, 0, B.BF16, 1, 1e-5, 1.0)
     assert B.dp_block_weight_count(du) == 46
     assert abs(B.dp_block_flops(du) - sum(B.dp_block_launch_info(du, B.DISPLACED, i)[1]
