@@ -94,11 +94,128 @@ __device__ __forceinline__ float silu_fast(float z) {
   return z * r;
 }
 
-template <typename T, int N>
-__device__ __forceinline__ void silu_vec(float (&t)[N]) {
-#pragma unroll
-  for (int j = 0; j < N; ++j) t[j] = silu_fast(t[j]);
+
+// SiLU of an fp32 pair with packed fp32x2 arithmetic: the same steps as
+// silu_fast (ex2 of -z log2 e clamped at 126, bit-pattern seed, two
+// Newton-Raphson steps for 1 / (1 + e)), two elements per FMA-pipe
+// instruction.
+__device__ __forceinline__ uint64_t silu_fast_x2(uint64_t z2) {
+  const uint64_t a2 = f2_mul(z2, f2_pack(-1.4426950408889634f, -1.4426950408889634f));
+  float a0, a1;
+  f2_unpack(a2, a0, a1);
+  a0 = fminf(a0, 126.f);
+  a1 = fminf(a1, 126.f);
+  float e0, e1;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e0) : "f"(a0));
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e1) : "f"(a1));
+  const uint64_t one2 = f2_pack(1.f, 1.f);
+  const uint64_t d2 = f2_add(f2_pack(e0, e1), one2);
+  float d0, d1;
+  f2_unpack(d2, d0, d1);
+  uint64_t r2 = f2_pack(__int_as_float(0x7EF31000 - __float_as_int(d0)),
+                        __int_as_float(0x7EF31000 - __float_as_int(d1)));
+  const uint64_t nd2 = d2 ^ 0x8000000080000000ull;   // -d in both halves
+  r2 = f2_fma(r2, f2_fma(nd2, r2, one2), r2);
+  r2 = f2_fma(r2, f2_fma(nd2, r2, one2), r2);
+  return f2_mul(z2, r2);
 }
+
+// Per-thread sums of x and x^2 over pixels for one 16-byte channel vector;
+// bf16 pairs go through packed fp32x2 adds and fmas.
+template <typename T>
+struct VecAcc;
+template <>
+struct VecAcc<__nv_bfloat16> {
+  uint64_t s[4] = {0, 0, 0, 0}, q[4] = {0, 0, 0, 0};
+  __device__ __forceinline__ void add(const __nv_bfloat16* p) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint64_t x2 = bf16x2_to_f2(w[k]);
+      s[k] = f2_add(s[k], x2);
+      q[k] = f2_fma(x2, x2, q[k]);
+    }
+  }
+  __device__ __forceinline__ void get(float (&sum)[8], float (&sq)[8]) const {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      f2_unpack(s[k], sum[2 * k], sum[2 * k + 1]);
+      f2_unpack(q[k], sq[2 * k], sq[2 * k + 1]);
+    }
+  }
+};
+template <>
+struct VecAcc<float> {
+  float s[4] = {0.f, 0.f, 0.f, 0.f}, q[4] = {0.f, 0.f, 0.f, 0.f};
+  __device__ __forceinline__ void add(const float* p) {
+    const float4 u = *reinterpret_cast<const float4*>(p);
+    const float t[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      s[k] += t[k];
+      q[k] = fmaf(t[k], t[k], q[k]);
+    }
+  }
+  __device__ __forceinline__ void get(float (&sum)[4], float (&sq)[4]) const {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      sum[k] = s[k];
+      sq[k] = q[k];
+    }
+  }
+};
+
+// y = x * scale + shift (+ SiLU) for one 16-byte channel vector; bf16 pairs
+// through packed fp32x2 arithmetic.
+template <typename T>
+struct VecApply;
+template <>
+struct VecApply<__nv_bfloat16> {
+  uint64_t sc[4], sh[4];
+  __device__ __forceinline__ VecApply(const float* scale, const float* shift) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      sc[k] = f2_pack(scale[2 * k], scale[2 * k + 1]);
+      sh[k] = f2_pack(shift[2 * k], shift[2 * k + 1]);
+    }
+  }
+  __device__ __forceinline__ void run(const __nv_bfloat16* src, __nv_bfloat16* dst, int silu) const {
+    const uint4 u = *reinterpret_cast<const uint4*>(src);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      uint64_t z2 = f2_fma(bf16x2_to_f2(w[k]), sc[k], sh[k]);
+      if (silu) z2 = silu_fast_x2(z2);
+      float z0, z1;
+      f2_unpack(z2, z0, z1);
+      o[k] = pack_bf16x2(z0, z1);
+    }
+    *reinterpret_cast<uint4*>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+};
+template <>
+struct VecApply<float> {
+  float sc[4], sh[4];
+  __device__ __forceinline__ VecApply(const float* scale, const float* shift) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      sc[k] = scale[k];
+      sh[k] = shift[k];
+    }
+  }
+  __device__ __forceinline__ void run(const float* src, float* dst, int silu) const {
+    const float4 u = *reinterpret_cast<const float4*>(src);
+    float t[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      t[k] = fmaf(t[k], sc[k], sh[k]);
+      if (silu) t[k] = silu_fast(t[k]);
+    }
+    *reinterpret_cast<float4*>(dst) = make_float4(t[0], t[1], t[2], t[3]);
+  }
+};
 
 struct GnArgs {
   int HWp;      // pixels per band
@@ -180,24 +297,20 @@ __global__ void __launch_bounds__(1024) gn_stats_kernel(const T* __restrict__ x,
   float sum[V], sq[V];
 #pragma unroll
   for (int j = 0; j < V; ++j) sum[j] = sq[j] = 0.f;
+  VecAcc<T> vacc;
   for (int k = 0; k < np; ++k) {
     rg.wait(k, status);
     const T* st = rg.stage(k) + v * V;
     const int cnt = rg.count(k);
     if (worker) {
       for (int q = pl; q < cnt; q += a.lanes) {
-        float t[V];
-        Vec<T>::load(st + static_cast<size_t>(q) * a.C, t);
-#pragma unroll
-        for (int j = 0; j < V; ++j) {
-          sum[j] += t[j];
-          sq[j] = fmaf(t[j], t[j], sq[j]);
-        }
+        vacc.add(st + static_cast<size_t>(q) * a.C);
       }
     }
     __syncthreads();   // the stage is free again
     if (threadIdx.x == 0 && k + kGnStages < np) rg.issue(k + kGnStages);
   }
+  vacc.get(sum, sq);
   // 16-byte stores: scalar ones at this stride would conflict 8-way
   if (worker) {
 #pragma unroll
@@ -329,6 +442,7 @@ __global__ void __launch_bounds__(1024) gn_apply_kernel(const T* __restrict__ x,
     sc[j] = worker ? sscale[v * V + j] : 0.f;
     sh[j] = worker ? sshift[v * V + j] : 0.f;
   }
+  const VecApply<T> ap(sc, sh);
   T* yb = y + off + v * V;
   for (int k = 0; k < np; ++k) {
     rg.wait(k, status);
@@ -337,12 +451,7 @@ __global__ void __launch_bounds__(1024) gn_apply_kernel(const T* __restrict__ x,
     if (worker) {
       T* yk = yb + static_cast<size_t>(k) * a.piece * a.C;
       for (int q = pl; q < cnt; q += a.lanes) {
-        float t[V];
-        Vec<T>::load(st + static_cast<size_t>(q) * a.C, t);
-#pragma unroll
-        for (int j = 0; j < V; ++j) t[j] = fmaf(t[j], sc[j], sh[j]);
-        if (a.silu) silu_vec<T>(t);
-        Vec<T>::store(yk + static_cast<size_t>(q) * a.C, t);
+        ap.run(st + static_cast<size_t>(q) * a.C, yk + static_cast<size_t>(q) * a.C, a.silu);
       }
     }
     __syncthreads();   // the stage is free again
@@ -483,16 +592,12 @@ __global__ void __launch_bounds__(1024, 1) gn_fused_kernel(
     float sum[V], sq[V];
 #pragma unroll
     for (int j = 0; j < V; ++j) sum[j] = sq[j] = 0.f;
+    VecAcc<T> vacc;
     if (worker) {
       for (int pix = lo + pl; pix < hi; pix += a.lanes) {
-        float t[V];
-        Vec<T>::load(data + static_cast<size_t>(pix) * a.C + v * V, t);
-#pragma unroll
-        for (int j = 0; j < V; ++j) {
-          sum[j] += t[j];
-          sq[j] = fmaf(t[j], t[j], sq[j]);
-        }
+        vacc.add(data + static_cast<size_t>(pix) * a.C + v * V);
       }
+      vacc.get(sum, sq);
       // 16-byte stores: scalar ones at this stride would conflict 8-way
 #pragma unroll
       for (int j = 0; j < V; j += 4) {
@@ -613,14 +718,10 @@ __global__ void __launch_bounds__(1024, 1) gn_fused_kernel(
         sc[j] = sscale[v * V + j];
         sh[j] = sshift[v * V + j];
       }
+      const VecApply<T> ap(sc, sh);
       T* yb = y + static_cast<size_t>(beg) * a.C + v * V;
       for (int pix = lo + pl; pix < hi; pix += a.lanes) {
-        float t[V];
-        Vec<T>::load(data + static_cast<size_t>(pix) * a.C + v * V, t);
-#pragma unroll
-        for (int j = 0; j < V; ++j) t[j] = fmaf(t[j], sc[j], sh[j]);
-        if (a.silu) silu_vec<T>(t);
-        Vec<T>::store(yb + static_cast<size_t>(pix) * a.C, t);
+        ap.run(data + static_cast<size_t>(pix) * a.C + v * V, yb + static_cast<size_t>(pix) * a.C, a.silu);
       }
     }
     __syncthreads();   // sscale/sshift are rewritten for the next segment
@@ -638,6 +739,7 @@ __global__ void __launch_bounds__(1024, 1) gn_fused_kernel(
 // moments (fresh_global) are formed by whichever band finishes last.
 struct GnClusterArgs {
   int HWp, C, G, P, vpp, lanes, chunk, cpb;
+  int slanes;   // pixel lanes of the statistics pass (lanes: of the apply pass)
   float eps, w;
   int silu, mode;
 };
@@ -649,7 +751,7 @@ __device__ __forceinline__ float ld_dsmem_f32(uint32_t cluster_addr) {
 }
 
 template <typename T>
-__global__ void __launch_bounds__(512, 1) gn_cluster_kernel(
+__global__ void __launch_bounds__(1024, 1) gn_cluster_kernel(
     const T* __restrict__ x, T* __restrict__ y, const float* __restrict__ gamma,
     const float* __restrict__ beta, GnClusterArgs a, unsigned* __restrict__ ticket,
     const float* __restrict__ stale_global, const float* __restrict__ stale_local,
@@ -659,9 +761,9 @@ __global__ void __launch_bounds__(512, 1) gn_cluster_kernel(
   extern __shared__ __align__(128) unsigned char gn_smem[];
   T* data = reinterpret_cast<T*>(gn_smem);                               // [chunk][C]
   const size_t data_bytes = ((static_cast<size_t>(a.chunk) * a.C * sizeof(T)) + 127) & ~size_t(127);
-  float* ssum = reinterpret_cast<float*>(gn_smem + data_bytes);          // [lanes][C]
-  float* ssq = ssum + a.lanes * a.C;                                     // [lanes][C]
-  float* gpart = ssq + a.lanes * a.C;                                    // [G][2], read by the cluster
+  float* ssum = reinterpret_cast<float*>(gn_smem + data_bytes);          // [slanes][C]
+  float* ssq = ssum + a.slanes * a.C;                                    // [slanes][C]
+  float* gpart = ssq + a.slanes * a.C;                                   // [G][2], read by the cluster
   double* f = reinterpret_cast<double*>(gpart + 2 * a.G + (a.G & 1) * 2);  // [G][2]
   float* sscale = reinterpret_cast<float*>(f + 2 * a.G);                 // [C]
   float* sshift = sscale + a.C;                                          // [C]
@@ -674,7 +776,8 @@ __global__ void __launch_bounds__(512, 1) gn_cluster_kernel(
   const int end = min(a.HWp, beg + a.chunk);
   const int npix = end - beg;
   const int v = threadIdx.x % a.vpp, pl = threadIdx.x / a.vpp;
-  const bool worker = threadIdx.x < a.vpp * a.lanes;
+  const bool worker = threadIdx.x < a.vpp * a.lanes;          // apply pass
+  const bool sworker = threadIdx.x < a.vpp * a.slanes;        // statistics pass
   const int cg = a.C / a.G;
   const size_t row_bytes = static_cast<size_t>(a.C) * sizeof(T);
 
@@ -704,16 +807,12 @@ __global__ void __launch_bounds__(512, 1) gn_cluster_kernel(
     float sum[V], sq[V];
 #pragma unroll
     for (int j = 0; j < V; ++j) sum[j] = sq[j] = 0.f;
-    if (worker) {
-      for (int pix = pl; pix < npix; pix += a.lanes) {
-        float t[V];
-        Vec<T>::load(data + static_cast<size_t>(pix) * a.C + v * V, t);
-#pragma unroll
-        for (int j = 0; j < V; ++j) {
-          sum[j] += t[j];
-          sq[j] = fmaf(t[j], t[j], sq[j]);
-        }
+    VecAcc<T> vacc;
+    if (sworker) {
+      for (int pix = pl; pix < npix; pix += a.slanes) {
+        vacc.add(data + static_cast<size_t>(pix) * a.C + v * V);
       }
+      vacc.get(sum, sq);
 #pragma unroll
       for (int j = 0; j < V; j += 4) {
         *reinterpret_cast<float4*>(ssum + pl * a.C + v * V + j) =
@@ -726,7 +825,7 @@ __global__ void __launch_bounds__(512, 1) gn_cluster_kernel(
   __syncthreads();
   for (int c = threadIdx.x; c < a.C; c += blockDim.x) {
     float cs = 0.f, cq = 0.f;
-    for (int l = 0; l < a.lanes; ++l) {
+    for (int l = 0; l < a.slanes; ++l) {
       cs += ssum[l * a.C + c];
       cq += ssq[l * a.C + c];
     }
@@ -784,14 +883,10 @@ __global__ void __launch_bounds__(512, 1) gn_cluster_kernel(
       sc[j] = sscale[v * V + j];
       sh[j] = sshift[v * V + j];
     }
+    const VecApply<T> ap(sc, sh);
     T* yb = y + (static_cast<size_t>(p) * a.HWp + beg) * a.C + v * V;
     for (int pix = pl; pix < npix; pix += a.lanes) {
-      float t[V];
-      Vec<T>::load(data + static_cast<size_t>(pix) * a.C + v * V, t);
-#pragma unroll
-      for (int j = 0; j < V; ++j) t[j] = fmaf(t[j], sc[j], sh[j]);
-      if (a.silu) silu_vec<T>(t);
-      Vec<T>::store(yb + static_cast<size_t>(pix) * a.C, t);
+      ap.run(data + static_cast<size_t>(pix) * a.C + v * V, yb + static_cast<size_t>(pix) * a.C, a.silu);
     }
   }
   // the cluster's other CTAs must be done reading gpart before this CTA leaves
@@ -904,13 +999,14 @@ bool gn_cluster_plan(int H, int W, int C, int G, int P, int dtype, int mode, int
   const int e = dtype == DP_BF16 ? 2 : 4;
   const int vpp = C / (16 / e);
   if (vpp > 512) return false;
-  const int lanes = 512 / vpp;
+  const int lanes = 1024 / vpp;          // apply pass: up to 1024 threads
+  const int slanes = 512 / vpp;          // statistics pass: its lane sums stay small
   const long HWp = static_cast<long>(H / P) * W;
   const int n = static_cast<int>(HWp < 16 ? HWp : 16);
   if (n < 1) return false;
   const long ch = (HWp + n - 1) / n;
   const size_t data = ((static_cast<size_t>(ch) * C * e) + 127) & ~size_t(127);
-  const size_t need = data + static_cast<size_t>(lanes) * C * 8 + static_cast<size_t>(G) * 8 + 16 +
+  const size_t need = data + static_cast<size_t>(slanes) * C * 8 + static_cast<size_t>(G) * 8 + 16 +
                       static_cast<size_t>(G) * 16 + static_cast<size_t>(C) * 8;
   if (need > 220 * 1024) return false;
   *cpb = n;
@@ -981,7 +1077,8 @@ static bool gn_cluster_launch(const void* x, void* y, const float* gamma, const 
   a.G = G;
   a.P = P;
   a.vpp = C / (dtype == DP_BF16 ? 8 : 4);
-  a.lanes = 512 / a.vpp;
+  a.lanes = 1024 / a.vpp;
+  a.slanes = 512 / a.vpp;
   a.chunk = chunk;
   a.cpb = cpb;
   a.eps = eps;
