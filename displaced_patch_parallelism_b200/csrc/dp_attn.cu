@@ -9,9 +9,11 @@
 // the band's own keys.
 //
 // B200 design (one CTA = 128 queries of one head, 320 threads, 2 CTAs/SM):
-//   warp 0     TMA producer: Q once, then K/V tiles of 128 keys through a
-//              2-deep ring; each tile is taken whole from the fresh or the
-//              stale buffer (bands are multiples of 128 tokens);
+//   warp 0     TMA producer: Q once per unit, then K and V tiles of 128 keys
+//              through two 2-deep rings (a K slot is free once S = Q K^T has
+//              read it, long before P V frees the V slot, so the next K loads
+//              early); each tile is taken whole from the fresh or the stale
+//              buffer (bands are multiples of 128 tokens);
 //   warp 1     MMA issuer: S = Q K^T (128x128x64) into tensor memory, then
 //              O += P V (128x64x128) with P read straight from tensor memory;
 //              S of tile j+1 is issued before O += P_j V_j so the tensor core
@@ -135,9 +137,11 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_kernel(const __grid_cons
   uint64_t* bars = reinterpret_cast<uint64_t*>(sV + kAttnStages * kTile);
   uint64_t* q_full = bars;                                      // [2]
   uint64_t* q_empty = q_full + 2;                               // [2]
-  uint64_t* kv_full = q_empty + 2;
-  uint64_t* kv_empty = kv_full + kAttnStages;
-  uint64_t* s_full = kv_empty + kAttnStages;
+  uint64_t* k_full = q_empty + 2;
+  uint64_t* k_empty = k_full + kAttnStages;
+  uint64_t* v_full = k_empty + kAttnStages;
+  uint64_t* v_empty = v_full + kAttnStages;
+  uint64_t* s_full = v_empty + kAttnStages;
   uint64_t* s_free = s_full + 1;
   uint64_t* p_full = s_free + 1;
   uint64_t* o_done = p_full + 1;
@@ -159,8 +163,10 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_kernel(const __grid_cons
       mbar_init(&q_empty[b], 1);
     }
     for (int s = 0; s < kAttnStages; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     mbar_init(s_full, 1);
     mbar_init(s_free, 8);
@@ -188,7 +194,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_kernel(const __grid_cons
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ producer
-      uint32_t issued = 0, issued_par = 0;        // bits 0-1: K/V stages, 2-3: Q buffers
+      // loads in flight, for the teardown after an abort: bits 0-1 K slots,
+      // 2-3 V slots, 4-5 Q buffers (with the parity each will complete)
+      uint32_t issued = 0, issued_par = 0;
       int stage = 0, qb = 0;
       uint32_t phase = 0, qpar[2] = {0u, 0u};
       int it = start;
@@ -200,8 +208,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_kernel(const __grid_cons
         if (!mbar_wait(&q_empty[qb], qpar[qb] ^ 1u, abort_flag, p.status)) break;
         mbar_arrive_expect_tx(&q_full[qb], kTile);
         tma_load_2d(sQ + qb * kTile, &p.tmQ, &q_full[qb], h * 64, q0);
-        issued |= 4u << qb;
-        issued_par = (issued_par & ~(4u << qb)) | (qpar[qb] << (2 + qb));
+        issued |= 16u << qb;
+        issued_par = (issued_par & ~(16u << qb)) | (qpar[qb] << (4 + qb));
         qpar[qb] ^= 1u;
         qb ^= 1;
         bool ok = true;
@@ -209,15 +217,22 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_kernel(const __grid_cons
           const int t = first_kv + j;
           const bool own = (t * 128) / p.tb == band;
           const bool stale = !own && p.mode == DP_MODE_DISPLACED;
-          if (!mbar_wait(&kv_empty[stage], phase ^ 1u, abort_flag, p.status)) {
+          if (!mbar_wait(&k_empty[stage], phase ^ 1u, abort_flag, p.status)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&kv_full[stage], 2 * kTile);
-          tma_load_2d(sK + stage * kTile, stale ? &p.tmKs : &p.tmKf, &kv_full[stage], h * 64, t * 128);
-          tma_load_2d(sV + stage * kTile, stale ? &p.tmVs : &p.tmVf, &kv_full[stage], h * 64, t * 128);
+          mbar_arrive_expect_tx(&k_full[stage], kTile);
+          tma_load_2d(sK + stage * kTile, stale ? &p.tmKs : &p.tmKf, &k_full[stage], h * 64, t * 128);
           issued |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+          if (!mbar_wait(&v_empty[stage], phase ^ 1u, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&v_full[stage], kTile);
+          tma_load_2d(sV + stage * kTile, stale ? &p.tmVs : &p.tmVf, &v_full[stage], h * 64, t * 128);
+          issued |= 4u << stage;
+          issued_par = (issued_par & ~(4u << stage)) | (phase << (2 + stage));
           if (++stage == kAttnStages) {
             stage = 0;
             phase ^= 1u;
@@ -226,9 +241,10 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_kernel(const __grid_cons
         if (!ok) break;
       }
       if (*abort_flag) {
-        for (int s = 0; s < 4; ++s)
+        for (int s = 0; s < 6; ++s)
           if (issued & (1u << s))
-            attn_wait_teardown(s < 2 ? &kv_full[s] : &q_full[s - 2], (issued_par >> s) & 1u);
+            attn_wait_teardown(s < 2 ? &k_full[s] : s < 4 ? &v_full[s - 2] : &q_full[s - 4],
+                               (issued_par >> s) & 1u);
       }
     }
   } else if (warp == 1) {
@@ -237,7 +253,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_kernel(const __grid_cons
       constexpr uint32_t idesc_qk = idesc_dense(128, 128, 1, 0, 0);
       constexpr uint32_t idesc_pv = idesc_dense(128, 64, 1, 0, 1);
       int stage = 0, prev_stage = 0, qb = 0;
-      uint32_t phase = 0, qpar[2] = {0u, 0u};
+      uint32_t phase = 0, prev_phase = 0, qpar[2] = {0u, 0u};
       int t = 0, si = 0;       // key tiles and segments done by this CTA
       int it = start;
       AttnSeg sg;
@@ -251,7 +267,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_kernel(const __grid_cons
         for (int jj = 0; jj <= n; ++jj) {
           const int tt = t + jj;
           if (jj < n) {
-            if (!mbar_wait(&kv_full[stage], phase, abort_flag, p.status) ||
+            if (!mbar_wait(&k_full[stage], phase, abort_flag, p.status) ||
                 (tt > 0 && !mbar_wait(s_free, (tt - 1) & 1, abort_flag, p.status))) {
               ok = false;
               break;
@@ -261,12 +277,14 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_kernel(const __grid_cons
 #pragma unroll
             for (int k = 0; k < 4; ++k) umma_f16_ss(tS, qd + 2 * k, kd + 2 * k, idesc_qk, k != 0);
             umma_commit(s_full);
+            umma_commit(&k_empty[stage]);
             if (jj == n - 1) umma_commit(&q_empty[qb]);   // this segment's last read of Q
           }
           if (jj > 0) {
             // O += P V of the previous key tile; the segment's first one
             // overwrites O, so the softmax warps must have read the last O
             if (!mbar_wait(p_full, (tt - 1) & 1, abort_flag, p.status) ||
+                !mbar_wait(&v_full[prev_stage], prev_phase, abort_flag, p.status) ||
                 (jj == 1 && si > 0 && !mbar_wait(o_free, (si - 1) & 1, abort_flag, p.status))) {
               ok = false;
               break;
@@ -276,11 +294,12 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_kernel(const __grid_cons
 #pragma unroll
             for (int k = 0; k < 8; ++k)
               umma_f16_ts(tO, tP + 8 * k, vd + 128 * k, idesc_pv, (jj > 1 || k != 0));
-            umma_commit(&kv_empty[prev_stage]);
+            umma_commit(&v_empty[prev_stage]);
             umma_commit(o_done);
           }
           if (jj < n) {
             prev_stage = stage;
+            prev_phase = phase;
             if (++stage == kAttnStages) {
               stage = 0;
               phase ^= 1u;
