@@ -75,49 +75,28 @@ struct Vec<float> {
   }
 };
 
-// SiLU z / (1 + exp(-z)) with one special-function instruction: exp(-z) is
-// 2^(-z log2 e) from the hardware base-2 exponential (ex2.approx, about 22
-// correct bits), and the reciprocal of d = 1 + exp(-z) is Newton-Raphson
-// from a bit-pattern seed.  The seed K - bits(d) mirrors d's exponent and
-// mantissa about 1.0; K = 0x7EF31000 came from a scan of K over one binade
-// (relative error at most 5.1%), and two steps r += r (1 - d r) bring it to
-// 6.6e-6, far below a bf16 rounding.  The exponent argument is clamped at
-// 126 so that d and 1/d stay normal.
-__device__ __forceinline__ float silu_fast(float z) {
-  const float arg = fminf(-1.4426950408889634f * z, 126.f);
-  float e;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(arg));
-  const float d = 1.f + e;
-  float r = __int_as_float(0x7EF31000 - __float_as_int(d));
-  r = fmaf(r, fmaf(-d, r, 1.f), r);
-  r = fmaf(r, fmaf(-d, r, 1.f), r);
-  return z * r;
+// SiLU(z) = z sigmoid(z) = h + h tanh(h) with h = z / 2 (sigmoid(z) =
+// (1 + tanh(z / 2)) / 2): one special-function instruction per element (the
+// hardware tanh.approx), and saturation at large |z| gives z or 0 with no
+// overflow.  Measured against an fp64 SiLU on B200: relative error at most
+// 8.5e-5 on outputs above 1e-3, far below a bf16 rounding.
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
+__device__ __forceinline__ float silu_fast(float z) {
+  const float h = 0.5f * z;
+  return fmaf(h, tanh_approx(h), h);
+}
 
-// SiLU of an fp32 pair with packed fp32x2 arithmetic: the same steps as
-// silu_fast (ex2 of -z log2 e clamped at 126, bit-pattern seed, two
-// Newton-Raphson steps for 1 / (1 + e)), two elements per FMA-pipe
-// instruction.
+// The same for an fp32 pair in packed fp32x2 arithmetic.
 __device__ __forceinline__ uint64_t silu_fast_x2(uint64_t z2) {
-  const uint64_t a2 = f2_mul(z2, f2_pack(-1.4426950408889634f, -1.4426950408889634f));
-  float a0, a1;
-  f2_unpack(a2, a0, a1);
-  a0 = fminf(a0, 126.f);
-  a1 = fminf(a1, 126.f);
-  float e0, e1;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e0) : "f"(a0));
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e1) : "f"(a1));
-  const uint64_t one2 = f2_pack(1.f, 1.f);
-  const uint64_t d2 = f2_add(f2_pack(e0, e1), one2);
-  float d0, d1;
-  f2_unpack(d2, d0, d1);
-  uint64_t r2 = f2_pack(__int_as_float(0x7EF31000 - __float_as_int(d0)),
-                        __int_as_float(0x7EF31000 - __float_as_int(d1)));
-  const uint64_t nd2 = d2 ^ 0x8000000080000000ull;   // -d in both halves
-  r2 = f2_fma(r2, f2_fma(nd2, r2, one2), r2);
-  r2 = f2_fma(r2, f2_fma(nd2, r2, one2), r2);
-  return f2_mul(z2, r2);
+  const uint64_t h2 = f2_mul(z2, f2_pack(0.5f, 0.5f));
+  float h0, h1;
+  f2_unpack(h2, h0, h1);
+  return f2_fma(h2, f2_pack(tanh_approx(h0), tanh_approx(h1)), h2);
 }
 
 // Per-thread sums of x and x^2 over pixels for one 16-byte channel vector;
