@@ -9,7 +9,8 @@
 // nowhere (naive: zeros); outside the image it is zero padding.
 //
 // B200 design:
-//  * one persistent CTA per SM, 192 threads in three roles:
+//  * one persistent CTA per SM, 192 threads in three roles (the 2-SM pair
+//    kernel below: 320, with two epilogue warps per TMEM lane quarter):
 //      warp 0     TMA producer (one lane): A and B tiles into a STAGES-deep
 //                 ring of 128-byte-swizzled shared-memory stages;
 //      warp 1     MMA issuer (one lane): tcgen05.mma 128 x BN x 16 into a
@@ -39,10 +40,9 @@ struct GemmParams {
   CUtensorMap tmA0;   // plain A, or the conv's fresh activations
   CUtensorMap tmA1;   // the conv's stale activations
   CUtensorMap tmB;    // weights, [N][K] K-major
-  // Pair kernels only: output segments and residual as 32-column boxes of one
-  // epilogue warp's 32 rows (64-byte swizzle), for TMA stores and loads.
+  // Pair kernels only: output segments as 32-column boxes of one epilogue
+  // warp's 32 rows (64-byte swizzle), for TMA stores.
   CUtensorMap tmO[3];
-  CUtensorMap tmR;
   int a_mode;         // 0: plain [M][K] rows, 1: 3x3 conv
   int M;
   int H, W, Ho, Wo, Cin, stride, hb_in, hb_out, mode, R, Wt, tiles_w, kc;
@@ -392,8 +392,8 @@ struct PairCfg {
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
   static constexpr int TMEM_COLS = BN <= 128 ? 128 : BN <= 256 ? 256 : 512;
   static constexpr int EPI_SLOT = 32 * 64;          // 32 rows x 32 bf16 columns
-  static constexpr int EPI_BYTES = 4 * 4 * EPI_SLOT;  // 4 warps x (2 output + 2 residual slots)
-  static constexpr int BIAS_BYTES = 4 * BN * 4;     // one fp32 copy per epilogue warp
+  static constexpr int EPI_BYTES = 8 * 2 * EPI_SLOT;  // 8 warps x 2 output slots
+  static constexpr int BIAS_BYTES = 8 * BN * 4;     // one fp32 copy per epilogue warp
   static constexpr int SMEM = STAGES * STAGE_BYTES + EPI_BYTES + BIAS_BYTES + 1024 + 256;
   static_assert(BSUB_BYTES % 1024 == 0, "B slice alignment");
   static_assert(SMEM <= 227 * 1024, "shared memory");
@@ -402,16 +402,11 @@ struct PairCfg {
 
 constexpr int kEpiSlot = 32 * 64;   // one epilogue warp's 32 rows x 32 bf16 columns
 
-// Shared-memory state of one epilogue warp of a pair kernel.  Residual chunks
-// arrive by TMA two chunks ahead of use; finished chunks leave by TMA stores
-// from two alternating slots.  The counters give each slot's barrier phase.
+// Shared-memory state of one epilogue warp of a pair kernel: finished chunks
+// leave by TMA stores from two alternating slots.
 struct PairEpi {
   uint8_t* out;      // 2 output slots
-  uint8_t* res;      // 2 residual slots
   float* bias;       // the tile's BN bias values
-  uint64_t* rbar;    // one barrier per residual slot
-  uint32_t ri;       // residual chunks consumed so far
-  uint32_t rpend;    // residual loads issued and not yet consumed
   uint32_t oi;       // output stores issued so far
 };
 
@@ -447,26 +442,35 @@ __device__ __forceinline__ EpiBox pair_epi_box(const GemmParams& p, int mt, int 
   return b;
 }
 
-__device__ __forceinline__ void pair_epi_res_load(const GemmParams& p, const EpiBox& b, int col,
-                                                  uint8_t* dst, uint64_t* bar) {
-  mbar_arrive_expect_tx(bar, kEpiSlot);
-  if (p.a_mode == 0) tma_load_2d(dst, &p.tmR, bar, col, b.y);
-  else tma_load_3d(dst, &p.tmR, bar, col, b.y, b.z);
+// Output pixel of accumulator row `row` of M tile mt, and whether it exists.
+__device__ __forceinline__ bool pair_row_pixel(const GemmParams& p, int mt, int row, size_t* pix) {
+  if (p.a_mode == 0) {
+    const int m = mt * 128 + row;
+    *pix = static_cast<size_t>(m);
+    return mt < p.m_tiles && m < p.M;
+  }
+  const int tr = mt / p.tiles_w, tc = mt - tr * p.tiles_w;
+  const int r = tr * p.R + row / p.Wt, c = tc * p.Wt + row % p.Wt;
+  *pix = static_cast<size_t>(r) * p.Wo + c;
+  return mt < p.m_tiles && r < p.Ho && c < p.Wo;
 }
 
 // Epilogue of one pair tile for one epilogue warp: this CTA's 128 accumulator
-// rows (TMEM lane quarter q) are drained in 32-column chunks; the accumulator
-// goes back to the leader after the last chunk; bias (staged in shared
-// memory) and residual (prefetched by TMA) are added and the bf16 chunk is
-// stored by TMA, ragged edges clipped by the tensor map.  Returns false when
-// a wait gave up (the caller tears down).
+// rows (TMEM lane quarter q) are drained in 32-column chunks, two warps per
+// lane quarter taking alternate chunks (half = 0: chunks 0, 2, ...; 1: 1, 3,
+// ...); each warp hands the accumulator back to the leader after its last
+// chunk.  Bias (staged in shared memory) and residual (each lane's row loaded
+// one chunk ahead into registers) are added and the bf16 chunk is stored by
+// TMA, ragged edges clipped by the tensor map.  Returns false when a wait gave
+// up (the caller tears down).
 template <int BN>
-__device__ __forceinline__ bool pair_epilogue_tile(const GemmParams& p, uint32_t tmem, int q, int lane,
-                                                   uint32_t rank, int item, int it, uint64_t* acc_full,
-                                                   uint32_t acc_empty_leader, volatile int* abort_flag,
-                                                   PairEpi& e) {
+__device__ __forceinline__ bool pair_epilogue_tile(const GemmParams& p, uint32_t tmem, int q, int half,
+                                                   int lane, uint32_t rank, int item, int it,
+                                                   uint64_t* acc_full, uint32_t acc_empty_leader,
+                                                   volatile int* abort_flag, PairEpi& e) {
   constexpr int NCH = BN / 32;
   static_assert(NCH >= 2, "chunks");
+  const int last_ch = ((NCH - 1 - half) / 2) * 2 + half;   // this warp's last chunk
   const int tile = item / p.splits;
   // Split K: this run's accumulator goes to its fp32 partial, rows at their
   // output pixels; bias, residual and the cast are the finish kernel's.
@@ -474,29 +478,18 @@ __device__ __forceinline__ bool pair_epilogue_tile(const GemmParams& p, uint32_t
     const int run = item - tile * p.splits;
     const int mp = tile / p.n_tiles, nt = tile - mp * p.n_tiles;
     const int mt = 2 * mp + static_cast<int>(rank);
-    const int row = q * 32 + lane;
-    bool valid;
     size_t pix;
-    if (p.a_mode == 0) {
-      const int m = mt * 128 + row;
-      valid = m < p.M;
-      pix = static_cast<size_t>(m);
-    } else {
-      const int tr = mt / p.tiles_w, tc = mt - tr * p.tiles_w;
-      const int r = tr * p.R + row / p.Wt, c = tc * p.Wt + row % p.Wt;
-      valid = mt < p.m_tiles && r < p.Ho && c < p.Wo;
-      pix = static_cast<size_t>(r) * p.Wo + c;
-    }
+    const bool valid = pair_row_pixel(p, mt, q * 32 + lane, &pix);
     const size_t M = p.a_mode == 0 ? static_cast<size_t>(p.M) : static_cast<size_t>(p.Ho) * p.Wo;
     float* dst = p.part + static_cast<size_t>(run) * M * p.N + pix * p.N + nt * BN;
     if (!mbar_wait(acc_full, it & 1, abort_flag, p.status)) return false;
     tc_fence_after();
 #pragma unroll 1
-    for (int ch = 0; ch < NCH; ++ch) {
+    for (int ch = half; ch < NCH; ch += 2) {
       uint32_t r[32];
       tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + ch * 32, r);
       tmem_wait_ld();
-      if (ch == NCH - 1) {
+      if (ch == last_ch) {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
@@ -514,32 +507,32 @@ __device__ __forceinline__ bool pair_epilogue_tile(const GemmParams& p, uint32_t
   const int mt = 2 * mp + static_cast<int>(rank);
   const int n0 = nt * BN;
   const EpiBox b = pair_epi_box(p, mt, q, n0);
-  const bool res = p.residual != nullptr && b.ok;
-  // Staged while the MMA of this tile still runs: the bias row and the first
-  // two residual chunks.  The previous tile's reads of both are finished.
+  const uint4* rrow = nullptr;
+  if (p.residual && b.ok) {
+    size_t pix;
+    if (pair_row_pixel(p, mt, q * 32 + lane, &pix))
+      rrow = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.residual) + pix * p.N + n0);
+  }
+  // Staged while the MMA of this tile still runs: the bias row and this
+  // lane's first residual chunk.  The previous tile's reads are finished.
   for (int i = lane; i < BN; i += 32) e.bias[i] = p.bias ? __ldg(p.bias + n0 + i) : 0.f;
-  if (res) {
-    if (lane == 0) {
-      fence_proxy_async_smem();
-      for (int c = 0; c < 2; ++c) {
-        const uint32_t s = (e.ri + c) & 1u;
-        pair_epi_res_load(p, b, n0 + c * 32, e.res + s * kEpiSlot, &e.rbar[s]);
-      }
-    }
-    e.rpend = 2;
+  uint4 rv[4];
+  if (rrow) {
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) rv[jj] = __ldg(rrow + half * 4 + jj);
   }
   __syncwarp();
   if (!mbar_wait(acc_full, it & 1, abort_flag, p.status)) return false;
   tc_fence_after();
   const CUtensorMap* om = &p.tmO[b.seg];
 #pragma unroll 1
-  for (int ch = 0; ch < NCH; ++ch) {
+  for (int ch = half; ch < NCH; ch += 2) {
     float v[32];
     {
       uint32_t r[32];
       tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + ch * 32, r);
       tmem_wait_ld();
-      if (ch == NCH - 1) {
+      if (ch == last_ch) {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
@@ -551,14 +544,10 @@ __device__ __forceinline__ bool pair_epilogue_tile(const GemmParams& p, uint32_t
     const float* bb = e.bias + ch * 32;
 #pragma unroll
     for (int j = 0; j < 32; ++j) v[j] += bb[j];
-    if (res) {
-      const uint32_t s = e.ri & 1u;
-      if (!mbar_wait(&e.rbar[s], (e.ri >> 1) & 1u, abort_flag, p.status)) return false;
-      const uint8_t* rs = e.res + s * kEpiSlot;
+    if (rrow) {
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj) {
-        uint4 u = *reinterpret_cast<const uint4*>(rs + sw64_off(lane, jj));
-        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&rv[jj]);
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
           const float2 f = __bfloat1622float2(h[t]);
@@ -566,15 +555,9 @@ __device__ __forceinline__ bool pair_epilogue_tile(const GemmParams& p, uint32_t
           v[8 * jj + 2 * t + 1] += f.y;
         }
       }
-      ++e.ri;
-      --e.rpend;
-      __syncwarp();
       if (ch + 2 < NCH) {
-        if (lane == 0) {
-          fence_proxy_async_smem();
-          pair_epi_res_load(p, b, n0 + (ch + 2) * 32, e.res + s * kEpiSlot, &e.rbar[s]);
-        }
-        ++e.rpend;
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) rv[jj] = __ldg(rrow + (ch + 2) * 4 + jj);
       }
     }
     uint8_t* ob = e.out + (e.oi & 1u) * kEpiSlot;
@@ -602,7 +585,7 @@ __device__ __forceinline__ bool pair_epilogue_tile(const GemmParams& p, uint32_t
 }
 
 template <int NI, int NJ>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
     igemm_pair_kernel(const __grid_constant__ GemmParams p) {
   using C = PairCfg<NI, NJ>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -617,8 +600,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   uint64_t* acc_full = empty + C::STAGES;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* drain = acc_empty + 1;
-  uint64_t* rbar = drain + 1;   // [epilogue warp][residual slot]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rbar + 8);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = warp_id(), lane = lane_id();
@@ -633,16 +615,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       mbar_init(&empty[s], 1);
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 8);
+    mbar_init(acc_empty, 16);   // 8 epilogue warps in each CTA
     mbar_init(drain, 1);
-    for (int s = 0; s < 8; ++s) mbar_init(&rbar[s], 1);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&p.tmA0);
     if (p.a_mode == 1) prefetch_tmap(&p.tmA1);
     prefetch_tmap(&p.tmB);
     prefetch_tmap(&p.tmO[0]);
-    if (p.residual) prefetch_tmap(&p.tmR);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
@@ -764,20 +744,59 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         split_range(p.k_blocks, p.splits, item - tile * p.splits, &kbeg, &kend);
         if (!mbar_wait(acc_empty, (it & 1) ^ 1, abort_flag, p.status)) goto mma_done;
         tc_fence_after();
-        for (int kb = kbeg; kb < kend; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, p.status)) goto mma_done;
+        // Two k-blocks per wait: tcgen05.mma issue blocks until the pipe
+        // takes the instruction, so the wait, fence and commits between
+        // k-blocks leave the pipe idle unless enough MMAs are queued behind
+        // them (measured: 8 MMAs of 256x160x16 per wait run at 88 % of the
+        // pipe, 16 per wait at 100 %).
+        for (int kb = kbeg; kb < kend;) {
+          const int nb = kend - kb >= 2 ? 2 : 1;
+          int stage2 = stage + 1;
+          uint32_t phase2 = phase;
+          if (stage2 == C::STAGES) {
+            stage2 = 0;
+            phase2 ^= 1u;
+          }
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.status) ||
+              (nb == 2 && !mbar_wait(&full[stage2], phase2, abort_flag, p.status)))
+            goto mma_done;
           tc_fence_after();
           const uint64_t ad = a_desc0 + static_cast<uint64_t>((stage * C::A_BYTES) >> 4);
           const uint64_t bd = b_desc0 + static_cast<uint64_t>((stage * C::B_BYTES) >> 4);
+          if (nb == 2) {
+            const uint64_t ad2 = a_desc0 + static_cast<uint64_t>((stage2 * C::A_BYTES) >> 4);
+            const uint64_t bd2 = b_desc0 + static_cast<uint64_t>((stage2 * C::B_BYTES) >> 4);
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
+            for (int k = 0; k < 4; ++k)
 #pragma unroll
-            for (int j = 0; j < NJ; ++j)
-              umma_f16_ss_pair(tmem + j * NI, ad + 2 * k,
-                               bd + static_cast<uint64_t>((j * C::BSUB_BYTES) >> 4) + 2 * k, idesc,
-                               (kb != kbeg || k != 0));
-          umma_commit_pair(empty_own + stage * 8);
-          umma_commit_pair(empty_peer + stage * 8);
+              for (int j = 0; j < NJ; ++j)
+                umma_f16_ss_pair(tmem + j * NI, ad + 2 * k,
+                                 bd + static_cast<uint64_t>((j * C::BSUB_BYTES) >> 4) + 2 * k, idesc,
+                                 (kb != kbeg || k != 0));
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+#pragma unroll
+              for (int j = 0; j < NJ; ++j)
+                umma_f16_ss_pair(tmem + j * NI, ad2 + 2 * k,
+                                 bd2 + static_cast<uint64_t>((j * C::BSUB_BYTES) >> 4) + 2 * k, idesc, 1u);
+            umma_commit_pair(empty_own + stage * 8);
+            umma_commit_pair(empty_peer + stage * 8);
+            umma_commit_pair(empty_own + stage2 * 8);
+            umma_commit_pair(empty_peer + stage2 * 8);
+          } else {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+#pragma unroll
+              for (int j = 0; j < NJ; ++j)
+                umma_f16_ss_pair(tmem + j * NI, ad + 2 * k,
+                                 bd + static_cast<uint64_t>((j * C::BSUB_BYTES) >> 4) + 2 * k, idesc,
+                                 (kb != kbeg || k != 0));
+            umma_commit_pair(empty_own + stage * 8);
+            umma_commit_pair(empty_peer + stage * 8);
+          }
+          kb += nb;
+          stage = nb == 2 ? stage2 : stage;
+          phase = nb == 2 ? phase2 : phase;
           if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -796,23 +815,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     // -------------------------------------------------------------- epilogue (both CTAs)
     const int q = warp & 3;
     const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
+    const int ew = warp - 2, half = ew >> 2;
     PairEpi e;
-    e.out = sEpi + q * 4 * kEpiSlot;
-    e.res = e.out + 2 * kEpiSlot;
-    e.bias = sBias + q * C::BN;
-    e.rbar = rbar + 2 * q;
-    e.ri = e.rpend = e.oi = 0;
+    e.out = sEpi + ew * 2 * kEpiSlot;
+    e.bias = sBias + ew * C::BN;
+    e.oi = 0;
     int it = 0;
     for (int item = pair; item < num_items; item += npairs, ++it)
-      if (!pair_epilogue_tile<C::BN>(p, tmem, q, lane, rank, item, it, acc_full, acc_empty_leader,
-                                     abort_flag, e))
+      if (!pair_epilogue_tile<C::BN>(p, tmem, q, half, lane, rank, item, it, acc_full,
+                                     acc_empty_leader, abort_flag, e))
         break;
-    if (lane == 0) {
-      // residual loads still in flight after an abort, then every store
-      for (uint32_t k = 0; k < e.rpend; ++k)
-        mbar_wait_teardown(&e.rbar[(e.ri + k) & 1u], ((e.ri + k) >> 1) & 1u);
-      bulk_wait_all();
-    }
+    if (lane == 0) bulk_wait_all();   // every store has finished reading its slot
   }
 
   tc_fence_before();
@@ -824,25 +837,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   }
 }
 
-// Tensor maps of a pair kernel's epilogue: each epilogue warp stores (and
-// loads residual) boxes of 32 channels x its 32 output rows with the 64-byte
-// swizzle.  Conv outputs are [Ho][Wo][Cout] (a warp's rows span min(Wt, 32)
-// pixels x 32 / min(Wt, 32) image rows); plain outputs are [M][ld_out] per
-// column segment and the residual is [M][N].
-static int encode_conv_epilogue(GemmParams& p, void* out, const void* residual, int Cout) {
+// Tensor maps of a pair kernel's epilogue: each epilogue warp stores boxes of
+// 32 channels x its 32 output rows with the 64-byte swizzle.  Conv outputs
+// are [Ho][Wo][Cout] (a warp's rows span min(Wt, 32) pixels x 32 / min(Wt, 32)
+// image rows); plain outputs are [M][ld_out] per column segment.
+static int encode_conv_epilogue(GemmParams& p, void* out, int Cout) {
   const uint32_t bw = static_cast<uint32_t>(std::min(p.Wt, 32));
   uint64_t dims[3] = {static_cast<uint64_t>(Cout), static_cast<uint64_t>(p.Wo),
                       static_cast<uint64_t>(p.Ho)};
   uint64_t str[2] = {static_cast<uint64_t>(Cout) * 2, static_cast<uint64_t>(p.Wo) * Cout * 2};
   uint32_t box[3] = {32, bw, 32 / bw};
-  int rc = encode_tmap(&p.tmO[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, out, dims, str, box,
-                       CU_TENSOR_MAP_SWIZZLE_64B);
-  if (rc || !residual) return rc;
-  return encode_tmap(&p.tmR, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(residual), dims,
-                     str, box, CU_TENSOR_MAP_SWIZZLE_64B);
+  return encode_tmap(&p.tmO[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, out, dims, str, box,
+                     CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
-static int encode_linear_epilogue(GemmParams& p, void* const outs[3], const void* residual) {
+static int encode_linear_epilogue(GemmParams& p, void* const outs[3]) {
   uint32_t box[2] = {32, 32};
   for (int sgi = 0; sgi < p.N / p.split; ++sgi) {
     uint64_t dims[2] = {static_cast<uint64_t>(p.split), static_cast<uint64_t>(p.M)};
@@ -851,11 +860,7 @@ static int encode_linear_epilogue(GemmParams& p, void* const outs[3], const void
                          CU_TENSOR_MAP_SWIZZLE_64B);
     if (rc) return rc;
   }
-  if (!residual) return DP_OK;
-  uint64_t dims[2] = {static_cast<uint64_t>(p.N), static_cast<uint64_t>(p.M)};
-  uint64_t str[1] = {static_cast<uint64_t>(p.N) * 2};
-  return encode_tmap(&p.tmR, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(residual), dims,
-                     str, box, CU_TENSOR_MAP_SWIZZLE_64B);
+  return DP_OK;
 }
 
 template <int NI, int NJ>
@@ -877,7 +882,7 @@ static int launch_pair(const GemmParams& p, cudaStream_t s) {
     attr.val.clusterDim.y = 1;
     attr.val.clusterDim.z = 1;
     cfg.gridDim = dim3(2 * num_sms());
-    cfg.blockDim = dim3(192);
+    cfg.blockDim = dim3(320);
     cfg.dynamicSmemBytes = C::SMEM;
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
@@ -892,7 +897,7 @@ static int launch_pair(const GemmParams& p, cudaStream_t s) {
   const int pair_tiles = ((p.m_tiles + 1) / 2) * p.n_tiles * p.splits;
   const int grid = std::min(2 * pair_tiles, maxg);
   mark_launch(s);
-  return launch_kernel(igemm_pair_kernel<NI, NJ>, dim3(grid), dim3(192), C::SMEM, s, false,
+  return launch_kernel(igemm_pair_kernel<NI, NJ>, dim3(grid), dim3(320), C::SMEM, s, false,
                        "pair gemm launch", p);
 }
 
@@ -1191,7 +1196,7 @@ int conv3x3_launch(const void* a_fresh, const void* a_stale, const void* weight,
                    CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc) return rc;
   if (pair) {
-    rc = encode_conv_epilogue(p, out, residual, Cout);
+    rc = encode_conv_epilogue(p, out, Cout);
     if (rc) return rc;
     set_split(p, splits, workspace);
     rc = pw == 320 ? launch_pair<160, 2>(p, stream) : launch_pair<160, 1>(p, stream);
@@ -1245,7 +1250,7 @@ int linear_launch(const void* x, const void* weight, const float* bias, const vo
   if (rc) return rc;
   if (pair) {
     void* const outs[3] = {out0, out1, out2};
-    rc = encode_linear_epilogue(p, outs, residual);
+    rc = encode_linear_epilogue(p, outs);
     if (rc) return rc;
     set_split(p, splits, workspace);
     rc = pw == 320 ? launch_pair<160, 2>(p, stream) : launch_pair<160, 1>(p, stream);
