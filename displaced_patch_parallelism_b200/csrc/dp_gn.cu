@@ -744,8 +744,9 @@ __global__ void __launch_bounds__(1024, 1) gn_cluster_kernel(
   float* ssq = ssum + a.slanes * a.C;                                    // [slanes][C]
   float* gpart = ssq + a.slanes * a.C;                                   // [G][2], read by the cluster
   double* f = reinterpret_cast<double*>(gpart + 2 * a.G + (a.G & 1) * 2);  // [G][2]
-  float* sscale = reinterpret_cast<float*>(f + 2 * a.G);                 // [C]
-  float* sshift = sscale + a.C;                                          // [C]
+  float* sscale = reinterpret_cast<float*>(f + 2 * a.G);                 // [C]: gamma, then the scale
+  float* sshift = sscale + a.C;                                          // [C]: beta, then the shift
+  float* sstale = sshift + a.C;                                          // [G][2] global, [G][2] band
   __shared__ __align__(8) uint64_t load_bar;
   __shared__ int s_last;
 
@@ -775,23 +776,44 @@ __global__ void __launch_bounds__(1024, 1) gn_cluster_kernel(
     for (uint32_t off = 0; off < total; off += 16384u)
       bulk_load(dst + off, src + off, min(16384u, total - off), &load_bar);
   }
+  // while the band arrives: the affine parameters and the stale moments
+  for (int c = threadIdx.x; c < a.C; c += blockDim.x) {
+    sscale[c] = gamma[c];
+    sshift[c] = beta[c];
+  }
+  if (a.mode == DP_MODE_DISPLACED) {
+    for (int i = threadIdx.x; i < 2 * a.G; i += blockDim.x) {
+      sstale[i] = stale_global[i];
+      sstale[2 * a.G + i] = stale_local[static_cast<size_t>(p) * a.G * 2 + i];
+    }
+  }
   if (npix > 0) {
     int no_abort = 0;
     mbar_wait(&load_bar, 0, &no_abort, status);
   }
   __syncthreads();
 
-  // ---- this CTA's (group) sums
+  // ---- this CTA's (group) sums: per-thread channel-vector sums over the
+  // thread's pixels (two interleaved accumulators), then lanes -> channels
+  // -> groups
   {
     float sum[V], sq[V];
-#pragma unroll
-    for (int j = 0; j < V; ++j) sum[j] = sq[j] = 0.f;
-    VecAcc<T> vacc;
     if (sworker) {
-      for (int pix = pl; pix < npix; pix += a.slanes) {
-        vacc.add(data + static_cast<size_t>(pix) * a.C + v * V);
+      VecAcc<T> acc0, acc1;
+      int pix = pl;
+      for (; pix + a.slanes < npix; pix += 2 * a.slanes) {
+        acc0.add(data + static_cast<size_t>(pix) * a.C + v * V);
+        acc1.add(data + static_cast<size_t>(pix + a.slanes) * a.C + v * V);
       }
-      vacc.get(sum, sq);
+      if (pix < npix) acc0.add(data + static_cast<size_t>(pix) * a.C + v * V);
+      float s1[V], q1[V];
+      acc0.get(sum, sq);
+      acc1.get(s1, q1);
+#pragma unroll
+      for (int j = 0; j < V; ++j) {
+        sum[j] += s1[j];
+        sq[j] += q1[j];
+      }
 #pragma unroll
       for (int j = 0; j < V; j += 4) {
         *reinterpret_cast<float4*>(ssum + pl * a.C + v * V + j) =
@@ -831,20 +853,22 @@ __global__ void __launch_bounds__(1024, 1) gn_cluster_kernel(
     for (int k = 0; k < a.cpb; ++k) s += ld_dsmem_f32(mapa_shared(local, static_cast<uint32_t>(k)));
     f[i] = s / n;
   }
+  // no more reads of other CTAs' shared memory: arrive now, wait at exit
+  cluster_arrive();
   __syncthreads();
-  const float* sl = stale_local + static_cast<size_t>(p) * a.G * 2;
   for (int c = threadIdx.x; c < a.C; c += blockDim.x) {
     const int g = c / cg;
     double m1 = f[2 * g], m2 = f[2 * g + 1];
     if (a.mode == DP_MODE_DISPLACED) {
-      m1 = static_cast<double>(stale_global[2 * g]) + a.w * (m1 - static_cast<double>(sl[2 * g]));
-      m2 = static_cast<double>(stale_global[2 * g + 1]) + a.w * (m2 - static_cast<double>(sl[2 * g + 1]));
+      m1 = static_cast<double>(sstale[2 * g]) + a.w * (m1 - static_cast<double>(sstale[2 * a.G + 2 * g]));
+      m2 = static_cast<double>(sstale[2 * g + 1]) +
+           a.w * (m2 - static_cast<double>(sstale[2 * a.G + 2 * g + 1]));
     }
     double var = m2 - m1 * m1;
     if (var < 0.0) var = f[2 * g + 1] - f[2 * g] * f[2 * g];
-    const float sc = rsqrtf(static_cast<float>(var) + a.eps) * gamma[c];
+    const float sc = rsqrtf(static_cast<float>(var) + a.eps) * sscale[c];
+    sshift[c] = sshift[c] - static_cast<float>(m1) * sc;
     sscale[c] = sc;
-    sshift[c] = beta[c] - static_cast<float>(m1) * sc;
     if (rank == 0 && c % cg == 0) {
       used[(p * a.G + g) * 2] = static_cast<float>(m1);
       used[(p * a.G + g) * 2 + 1] = static_cast<float>(var);
@@ -854,7 +878,8 @@ __global__ void __launch_bounds__(1024, 1) gn_cluster_kernel(
   }
   __syncthreads();
 
-  // ---- apply from shared memory, coalesced 16-byte stores
+  // ---- apply from shared memory, coalesced 16-byte stores, two pixels per
+  // iteration
   if (worker) {
     float sc[V], sh[V];
 #pragma unroll
@@ -864,12 +889,17 @@ __global__ void __launch_bounds__(1024, 1) gn_cluster_kernel(
     }
     const VecApply<T> ap(sc, sh);
     T* yb = y + (static_cast<size_t>(p) * a.HWp + beg) * a.C + v * V;
-    for (int pix = pl; pix < npix; pix += a.lanes) {
+    int pix = pl;
+    for (; pix + a.lanes < npix; pix += 2 * a.lanes) {
       ap.run(data + static_cast<size_t>(pix) * a.C + v * V, yb + static_cast<size_t>(pix) * a.C, a.silu);
+      ap.run(data + static_cast<size_t>(pix + a.lanes) * a.C + v * V,
+             yb + static_cast<size_t>(pix + a.lanes) * a.C, a.silu);
     }
+    if (pix < npix)
+      ap.run(data + static_cast<size_t>(pix) * a.C + v * V, yb + static_cast<size_t>(pix) * a.C, a.silu);
   }
-  // the cluster's other CTAs must be done reading gpart before this CTA leaves
-  cluster_sync_all();
+  // the cluster's other CTAs are done reading gpart before this CTA leaves
+  cluster_wait();
 
   // ---- the band that finishes last forms the whole-image moments
   if (rank == 0 && fresh_global) {
@@ -986,7 +1016,8 @@ bool gn_cluster_plan(int H, int W, int C, int G, int P, int dtype, int mode, int
   const long ch = (HWp + n - 1) / n;
   const size_t data = ((static_cast<size_t>(ch) * C * e) + 127) & ~size_t(127);
   const size_t need = data + static_cast<size_t>(slanes) * C * 8 + static_cast<size_t>(G) * 8 + 16 +
-                      static_cast<size_t>(G) * 16 + static_cast<size_t>(C) * 8;
+                      static_cast<size_t>(G) * 16 + static_cast<size_t>(C) * 8 +
+                      static_cast<size_t>(G) * 16;
   if (need > 220 * 1024) return false;
   *cpb = n;
   *chunk = static_cast<int>(ch);
