@@ -251,7 +251,11 @@ def test_conv_small_parity():
                                                  (4096, 1920, 640, 640, False),
                                                  (1000, 640, 320, 640, True),
                                                  (384, 960, 128, 320, False),
-                                                 (130, 320, 64, 320, True)])
+                                                 (130, 320, 64, 320, True),
+                                                 # pair tiles with a residual; several tiles per
+                                                 # SM pair reuse both accumulators; ragged M
+                                                 (4096, 640, 640, 640, True),
+                                                 (3000, 1280, 512, 1280, True)])
 def test_linear_parity(M, N, K, split, use_res):
     r = rng(M + N + K)
     x = rounded(r.standard_normal((M, K)), "bf16")
