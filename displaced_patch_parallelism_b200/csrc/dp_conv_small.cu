@@ -76,24 +76,29 @@ __global__ void __launch_bounds__(256) conv3x3_small_kernel(
 // Register variant for up to 8 input channels (the latent input conv has
 // 4): a block takes 64 pixels of one output row; the 3 input rows it needs
 // (66 pixels, channels padded to CIN with zeros) are staged in shared memory
-// as fp32 with the halo rule applied, and each warp takes (32 output
-// channels, 32 pixels) items: a lane owns one output channel, keeps its
-// 9 x CIN filter taps in registers and reads each input value as a shared-
-// memory broadcast; a warp's 32 lanes store 32 consecutive channels of one
+// as fp32 with the halo rule applied.  A warp owns a group of 32 output
+// channels for the whole tile (a lane owns one channel and keeps its 9 x CIN
+// filter taps in registers, loaded once).  It walks the tile 4 pixels at a
+// time: per input row it reads the 6 pixels those 4 outputs touch as 16-byte
+// shared-memory broadcasts (CIN / 4 vectors each) and does 3 x 4 x CIN FMAs
+// per vector read.  A warp's 32 lanes store 32 consecutive channels of one
 // pixel.
 constexpr int kRegTile = 64;
 
 template <int CIN>
-__global__ void __launch_bounds__(256) conv3x3_small_reg_kernel(
+__global__ void __launch_bounds__(320) conv3x3_small_reg_kernel(
     const __nv_bfloat16* __restrict__ af, const __nv_bfloat16* __restrict__ as,
     const __nv_bfloat16* __restrict__ w, const float* __restrict__ bias,
     __nv_bfloat16* __restrict__ out, int H, int W, int Cin, int Cout, int hb, int mode) {
-  __shared__ __align__(16) float sx[3][kRegTile + 2][CIN];
+  static_assert(CIN % 4 == 0, "float4 staging");
+  constexpr int NV = CIN / 4;
+  __shared__ __align__(16) float4 sx[3][kRegTile + 2][NV];
   const int r = blockIdx.y, c0 = blockIdx.x * kRegTile;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
   griddep_wait();
   griddep_trigger();
   const int band = r / hb;
+  float* sxf = reinterpret_cast<float*>(sx);
   for (int i = threadIdx.x; i < 3 * (kRegTile + 2) * CIN; i += blockDim.x) {
     const int ci = i % CIN, px = (i / CIN) % (kRegTile + 2), kh = i / (CIN * (kRegTile + 2));
     const int rho = r + kh - 1, col = c0 + px - 1;
@@ -107,39 +112,64 @@ __global__ void __launch_bounds__(256) conv3x3_small_reg_kernel(
       }
       if (use) v = __bfloat162float(src[(static_cast<size_t>(rho) * W + col) * Cin + ci]);
     }
-    sx[kh][px][ci] = v;
+    sxf[i] = v;
   }
   __syncthreads();
-  const int groups = Cout / 32, chunks = kRegTile / 32;
-  for (int item = warp; item < groups * chunks; item += blockDim.x >> 5) {
-    const int g = item / chunks, ch = item - g * chunks;
+  const int groups = Cout / 32;
+  const int npx = min(kRegTile, W - c0);
+  for (int g = warp; g < groups; g += nwarps) {
     const int co = g * 32 + lane;
     float wr[9 * CIN];
+    if (Cin == CIN && (reinterpret_cast<uintptr_t>(w) & 7u) == 0) {
+      // the lane's 9 x CIN taps are contiguous: 8-byte loads (a quarter of
+      // the sectors that 2-byte loads at this lane stride touch)
+      const uint2* wv = reinterpret_cast<const uint2*>(w + static_cast<size_t>(co) * 9 * CIN);
 #pragma unroll
-    for (int k = 0; k < 9; ++k)
+      for (int i = 0; i < 9 * CIN / 4; ++i) {
+        const uint2 u = __ldg(wv + i);
+        const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+        const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+        wr[4 * i] = lo.x;
+        wr[4 * i + 1] = lo.y;
+        wr[4 * i + 2] = hi.x;
+        wr[4 * i + 3] = hi.y;
+      }
+    } else {
 #pragma unroll
-      for (int ci = 0; ci < CIN; ++ci)
-        wr[k * CIN + ci] = ci < Cin ? __bfloat162float(w[(static_cast<size_t>(co) * 9 + k) * Cin + ci]) : 0.f;
+      for (int k = 0; k < 9; ++k)
+#pragma unroll
+        for (int ci = 0; ci < CIN; ++ci)
+          wr[k * CIN + ci] = ci < Cin ? __bfloat162float(w[(static_cast<size_t>(co) * 9 + k) * Cin + ci]) : 0.f;
+    }
     const float b0 = bias ? __ldg(bias + co) : 0.f;
-    // four pixels at a time: independent accumulators hide the FMA latency
-    for (int j = 0; j < 32; j += 4) {
-      const int px = ch * 32 + j;
-      if (c0 + px >= W) break;
+    __nv_bfloat16* orow = out + (static_cast<size_t>(r) * W + c0) * Cout + co;
+    for (int px = 0; px < npx; px += 4) {
       float acc[4] = {b0, b0, b0, b0};
 #pragma unroll
-      for (int kh = 0; kh < 3; ++kh)
+      for (int kh = 0; kh < 3; ++kh) {
+        float4 xv[6][NV];
+#pragma unroll
+        for (int t = 0; t < 6; ++t)
+#pragma unroll
+          for (int q = 0; q < NV; ++q) xv[t][q] = sx[kh][px + t][q];
 #pragma unroll
         for (int kw = 0; kw < 3; ++kw)
 #pragma unroll
-          for (int ci = 0; ci < CIN; ++ci) {
-            const float wv = wr[(kh * 3 + kw) * CIN + ci];
+          for (int q = 0; q < NV; ++q) {
+            const float* wk = wr + (kh * 3 + kw) * CIN + 4 * q;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) acc[u] = fmaf(sx[kh][px + u + kw][ci], wv, acc[u]);
+            for (int u = 0; u < 4; ++u) {
+              const float4 x = xv[u + kw][q];
+              acc[u] = fmaf(x.x, wk[0], acc[u]);
+              acc[u] = fmaf(x.y, wk[1], acc[u]);
+              acc[u] = fmaf(x.z, wk[2], acc[u]);
+              acc[u] = fmaf(x.w, wk[3], acc[u]);
+            }
           }
+      }
 #pragma unroll
       for (int u = 0; u < 4; ++u)
-        if (c0 + px + u < W)
-          out[(static_cast<size_t>(r) * W + c0 + px + u) * Cout + co] = __float2bfloat16_rn(acc[u]);
+        if (px + u < npx) orow[static_cast<size_t>(px + u) * Cout] = __float2bfloat16_rn(acc[u]);
     }
   }
 }
@@ -155,9 +185,9 @@ int conv3x3_small_launch(const void* af, const void* as, const void* w, const fl
     const dim3 grid(static_cast<unsigned>((W + kRegTile - 1) / kRegTile), static_cast<unsigned>(H));
     mark_launch(stream);
     if (Cin <= 4)
-      return launch_kernel(conv3x3_small_reg_kernel<4>, grid, dim3(256), 0, stream, false,
+      return launch_kernel(conv3x3_small_reg_kernel<4>, grid, dim3(320), 0, stream, false,
                            "small conv launch", a0, a1, wt, bias, o, H, W, Cin, Cout, H / P, mode);
-    return launch_kernel(conv3x3_small_reg_kernel<8>, grid, dim3(256), 0, stream, false,
+    return launch_kernel(conv3x3_small_reg_kernel<8>, grid, dim3(320), 0, stream, false,
                          "small conv launch", a0, a1, wt, bias, o, H, W, Cin, Cout, H / P, mode);
   }
   const size_t smem = static_cast<size_t>(9) * Cin * kSmallCo * sizeof(float);
