@@ -8,6 +8,9 @@
 // DistriFusion).  Sync steps use fresh keys everywhere; naive steps see only
 // the band's own keys.
 //
+// Two kernels.  Bands of a multiple of 256 tokens take attn_pair_kernel (two
+// query tiles per CTA, ping-ponged on the tensor core; described above it).
+// Other bands take attn_kernel:
 // B200 design (one CTA = 128 queries of one head, 320 threads, 2 CTAs/SM):
 //   warp 0     TMA producer: Q once per unit, then K and V tiles of 128 keys
 //              through two 2-deep rings (a K slot is free once S = Q K^T has
@@ -89,8 +92,9 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 // f in [-1/2, 1/2], by adding 1.5 * 2^23 (the sum's low mantissa bits hold n);
 // 2^f by a cubic fitted here for minimax relative error on [-1/2, 1/2]
 // (Remez exchange; max relative error 7.5e-5, far below the 2^-9 of the bf16
-// that P is rounded to); 2^n by adding n to the exponent field.  Inputs are
-// clamped at -125 so the result stays a normal number.
+// that P is rounded to); 2^n by adding n to the exponent field (the low bits
+// of t = x + 1.5 * 2^23 hold n, and the magic's own bits vanish in the shift
+// by 23).  Inputs are clamped at -125 so the result stays a normal number.
 __device__ __forceinline__ void exp2_poly_x2(uint64_t x2, float& e0, float& e1) {
   constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
   float x0, x1;
@@ -106,8 +110,8 @@ __device__ __forceinline__ void exp2_poly_x2(uint64_t x2, float& e0, float& e1) 
   float t0, t1, p0, p1;
   f2_unpack(t2, t0, t1);
   f2_unpack(p2, p0, p1);
-  e0 = __int_as_float(__float_as_int(p0) + ((__float_as_int(t0) - 0x4B400000) << 23));
-  e1 = __int_as_float(__float_as_int(p1) + ((__float_as_int(t1) - 0x4B400000) << 23));
+  e0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  e1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
 __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
@@ -527,13 +531,472 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_kernel(const __grid_cons
   }
 }
 
+// ---------------------------------------------------------------------------
+// Two query tiles per CTA (bands whose size is a multiple of 256 tokens).
+//
+// A unit is 256 queries of one head: query tiles A and B (rows q0.. and
+// q0+128..) of the same band, so every key tile comes from the same buffer
+// for both and is loaded once for both.  One CTA per SM, 352 threads:
+//   warp 0       TMA producer: both query tiles once per unit (double-
+//                buffered), K and V tiles of 128 keys through 3-deep rings;
+//   warps 1, 10  MMA issuers of tiles A and B.  `tcgen05.mma` returns only
+//                when the pipe accepts it, and one thread issues a 128x64x16
+//                P V instruction in about 56 cycles against 32 of math, so
+//                each tile has its own issuer.  Per key tile j an issuer
+//                computes S(j) = Q K_j^T as soon as the softmax warps have read
+//                S(j-1) out of tensor memory, then O += P(j-1) V_(j-1);
+//   warps 2-5    softmax of tile A, warps 6-9 of tile B: one thread per query
+//                row (no exchange between warps), online maximum with lazy
+//                rescaling (O is rescaled only when the running maximum grows
+//                by more than 2^8), exp2 (1 in 4 on the FMA pipe), bf16 P to
+//                tensor memory; at the end of a unit O / l, stored as bf16.
+// Tensor memory (512 columns): S_A [0,128), S_B [128,256), O_A [256,320),
+// O_B [320,384), P_A [384,448), P_B [448,512) (P as bf16 pairs).
+constexpr int kPairStages = 3;
+constexpr int kPairThreads = 352;
+constexpr int kPairOutBytes = 8 * 4096;                   // per softmax warp: 32 rows x 128 B
+constexpr int kPairSmem = 1024 + 4 * kTile + 2 * kPairStages * kTile + kPairOutBytes + kAttnTail;
+// A partial of one softmax warp: 17 float4 columns x 32 lanes (O's 16 float4
+// per row, then m, l), lane-contiguous so that every access is coalesced.
+constexpr int kPairSliceFloats = 17 * 32 * 4;
+constexpr int kPairSlotFloats = 8 * kPairSliceFloats;    // the 8 softmax warps
+static_assert(kPairSmem > 114 * 1024, "one CTA per SM: it allocates all of tensor memory");
+
+__global__ void __launch_bounds__(kPairThreads, 1) attn_pair_kernel(const __grid_constant__ AttnParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem;                                           // [2 buffers][tiles A, B]
+  uint8_t* sK = smem + 4 * kTile;
+  uint8_t* sV = sK + kPairStages * kTile;
+  uint8_t* sOut = sV + kPairStages * kTile;                     // [8 softmax warps][32 rows][128 B]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + kPairOutBytes);
+  uint64_t* q_full = bars;                                      // [2]
+  uint64_t* q_empty = q_full + 2;                               // [2]
+  uint64_t* k_full = q_empty + 2;                               // [stages]
+  uint64_t* k_empty = k_full + kPairStages;
+  uint64_t* v_full = k_empty + kPairStages;
+  uint64_t* v_empty = v_full + kPairStages;
+  uint64_t* s_full = v_empty + kPairStages;                     // [2], per query tile
+  uint64_t* s_free = s_full + 2;                                // [2]
+  uint64_t* p_full = s_free + 2;                                // [2]
+  uint64_t* o_done = p_full + 2;                                // [2]
+  uint64_t* o_free = o_done + 2;                                // [2]
+  uint64_t* drain = o_free + 2;                                 // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = warp_id(), lane = lane_id();
+  const int band_tiles = p.tb / 128;
+  const int start = blockIdx.x * p.L;
+  const int end = min(p.W, start + p.L);
+
+  if (threadIdx.x == 0) {
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&q_full[b], 1);
+      mbar_init(&q_empty[b], 2);
+      mbar_init(&s_full[b], 1);
+      mbar_init(&s_free[b], 4);
+      mbar_init(&p_full[b], 4);
+      mbar_init(&o_done[b], 1);
+      mbar_init(&o_free[b], 4);
+      mbar_init(&drain[b], 1);
+    }
+    for (int s = 0; s < kPairStages; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 2);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 2);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  griddep_wait();
+  griddep_trigger();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      // loads in flight, for the teardown after an abort: bits 0-2 K slots,
+      // 3-5 V slots, 6-7 Q buffers (with the parity each will complete)
+      uint32_t issued = 0, issued_par = 0;
+      int stage = 0, qb = 0;
+      uint32_t phase = 0, qpar[2] = {0u, 0u};
+      int it = start;
+      AttnSeg sg;
+      bool ok = true;
+      while (ok && attn_next_seg(p, it, end, sg)) {
+        const int h = sg.u / p.n_qt, q0 = (sg.u - h * p.n_qt) * 256;
+        const int band = q0 / p.tb;
+        const int first_kv = p.mode == DP_MODE_NAIVE ? band * band_tiles : 0;
+        if (!mbar_wait(&q_empty[qb], qpar[qb] ^ 1u, abort_flag, p.status)) break;
+        mbar_arrive_expect_tx(&q_full[qb], 2 * kTile);
+        tma_load_2d(sQ + (2 * qb) * kTile, &p.tmQ, &q_full[qb], h * 64, q0);
+        tma_load_2d(sQ + (2 * qb + 1) * kTile, &p.tmQ, &q_full[qb], h * 64, q0 + 128);
+        issued |= 64u << qb;
+        issued_par = (issued_par & ~(64u << qb)) | (qpar[qb] << (6 + qb));
+        qpar[qb] ^= 1u;
+        qb ^= 1;
+        for (int j = sg.k0; j < sg.k1; ++j) {
+          const int t = first_kv + j;
+          const bool own = (t * 128) / p.tb == band;
+          const bool stale = !own && p.mode == DP_MODE_DISPLACED;
+          if (!mbar_wait(&k_empty[stage], phase ^ 1u, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&k_full[stage], kTile);
+          tma_load_2d(sK + stage * kTile, stale ? &p.tmKs : &p.tmKf, &k_full[stage], h * 64, t * 128);
+          issued |= 1u << stage;
+          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+          if (!mbar_wait(&v_empty[stage], phase ^ 1u, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&v_full[stage], kTile);
+          tma_load_2d(sV + stage * kTile, stale ? &p.tmVs : &p.tmVf, &v_full[stage], h * 64, t * 128);
+          issued |= 8u << stage;
+          issued_par = (issued_par & ~(8u << stage)) | (phase << (3 + stage));
+          if (++stage == kPairStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (*abort_flag) {
+        for (int s = 0; s < 8; ++s)
+          if (issued & (1u << s))
+            attn_wait_teardown(s < 3 ? &k_full[s] : s < 6 ? &v_full[s - 3] : &q_full[s - 6],
+                               (issued_par >> s) & 1u);
+      }
+    }
+  } else if (warp == 1 || warp == 10) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      const int tile = warp == 1 ? 0 : 1;
+      constexpr uint32_t idesc_qk = idesc_dense(128, 128, 1, 0, 0);
+      constexpr uint32_t idesc_pv = idesc_dense(128, 64, 1, 0, 1);
+      const uint32_t tS = tmem + 128 * tile, tO = tmem + 256 + 64 * tile, tP = tmem + 384 + 64 * tile;
+      int stage = 0, prev_stage = 0, qb = 0;
+      uint32_t phase = 0, prev_phase = 0, qpar[2] = {0u, 0u};
+      int t = 0, si = 0;       // key tiles and segments done by this CTA
+      int it = start;
+      AttnSeg sg;
+      bool ok = true;
+      while (ok && attn_next_seg(p, it, end, sg)) {
+        const int n = sg.k1 - sg.k0;
+        if (!mbar_wait(&q_full[qb], qpar[qb], abort_flag, p.status)) break;
+        qpar[qb] ^= 1u;
+        tc_fence_after();
+        const uint64_t qd = sdesc_sw128(smem_u32(sQ + (2 * qb + tile) * kTile), 1024);
+        for (int jj = 0; jj <= n; ++jj) {
+          const int tt = t + jj;
+          if (jj < n) {
+            // S(j) once the softmax warps have read S(j-1)
+            if (!mbar_wait(&k_full[stage], phase, abort_flag, p.status) ||
+                (tt > 0 && !mbar_wait(&s_free[tile], (tt - 1) & 1, abort_flag, p.status))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t kd = sdesc_sw128(smem_u32(sK + stage * kTile), 1024);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) umma_f16_ss(tS, qd + 2 * k, kd + 2 * k, idesc_qk, k != 0);
+            umma_commit(&s_full[tile]);
+            umma_commit(&k_empty[stage]);
+            if (jj == n - 1) umma_commit(&q_empty[qb]);   // this segment's last read of Q
+          }
+          if (jj > 0) {
+            // O += P V of the previous key tile; the segment's first one
+            // overwrites O, so the softmax warps must have read the last O
+            if (!mbar_wait(&p_full[tile], (tt - 1) & 1, abort_flag, p.status) ||
+                !mbar_wait(&v_full[prev_stage], prev_phase, abort_flag, p.status) ||
+                (jj == 1 && si > 0 && !mbar_wait(&o_free[tile], (si - 1) & 1, abort_flag, p.status))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t vd = sdesc_sw128(smem_u32(sV + prev_stage * kTile), 1024);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) umma_f16_ts(tO, tP + 8 * k, vd + 128 * k, idesc_pv, (jj > 1 || k != 0));
+            umma_commit(&v_empty[prev_stage]);
+            umma_commit(&o_done[tile]);
+          }
+          if (jj < n) {
+            prev_stage = stage;
+            prev_phase = phase;
+            if (++stage == kPairStages) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+        t += n;
+        ++si;
+        qb ^= 1;
+      }
+      if (*abort_flag) {
+        umma_commit(&drain[tile]);
+        attn_wait_teardown(&drain[tile], 0);
+      }
+    }
+  } else {
+    // -------------------------------------------------------------- softmax
+    const int tile = (warp - 2) >> 2;          // query tile A (0) or B (1)
+    const int q = warp & 3;                    // tensor memory lane quarter
+    const int row = q * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    const uint32_t tS = tmem + 128 * tile + lane_off;
+    const uint32_t tO = tmem + 256 + 64 * tile + lane_off;
+    const uint32_t tP = tmem + 384 + 64 * tile + lane_off;
+    const float c = p.scale_log2;
+    bool aborted = false;
+    int t = 0, si = 0;
+    int it = start;
+    AttnSeg sg;
+    while (!aborted && attn_next_seg(p, it, end, sg)) {
+      const int n = sg.k1 - sg.k0;
+      float m_used = 0.f, l = 0.f;
+      for (int jj = 0; jj < n; ++jj) {
+        const int tt = t + jj;
+        if (!mbar_wait(&s_full[tile], tt & 1, abort_flag, p.status)) {
+          aborted = true;
+          break;
+        }
+        tc_fence_after();
+        // Row maximum from two loads of 64 columns; columns 64-127 stay in
+        // registers, columns 0-63 are read again after them (fewer live
+        // registers than holding the whole row), and only then is S released.
+        uint32_t sa[32], sb[32];
+        tmem_ld32(tS, sa);
+        tmem_ld32(tS + 32, sb);
+        tmem_wait_ld();
+        float m0 = fmaxf(__uint_as_float(sa[0]), __uint_as_float(sa[1]));
+        float m1 = fmaxf(__uint_as_float(sa[16]), __uint_as_float(sa[17]));
+        float m2 = fmaxf(__uint_as_float(sb[0]), __uint_as_float(sb[1]));
+        float m3 = fmaxf(__uint_as_float(sb[16]), __uint_as_float(sb[17]));
+#pragma unroll
+        for (int i = 2; i < 16; i += 2) {
+          m0 = max3(m0, __uint_as_float(sa[i]), __uint_as_float(sa[i + 1]));
+          m1 = max3(m1, __uint_as_float(sa[16 + i]), __uint_as_float(sa[17 + i]));
+          m2 = max3(m2, __uint_as_float(sb[i]), __uint_as_float(sb[i + 1]));
+          m3 = max3(m3, __uint_as_float(sb[16 + i]), __uint_as_float(sb[17 + i]));
+        }
+        tmem_ld32(tS + 64, sa);
+        tmem_ld32(tS + 96, sb);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; i += 2) {
+          m0 = max3(m0, __uint_as_float(sa[i]), __uint_as_float(sa[i + 1]));
+          m1 = max3(m1, __uint_as_float(sa[16 + i]), __uint_as_float(sa[17 + i]));
+          m2 = max3(m2, __uint_as_float(sb[i]), __uint_as_float(sb[i + 1]));
+          m3 = max3(m3, __uint_as_float(sb[16 + i]), __uint_as_float(sb[17 + i]));
+        }
+        const float m_tile = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) * c;
+        float alpha = 1.f;
+        if (jj == 0) {
+          m_used = m_tile;
+        } else if (m_tile > m_used + 8.f) {
+          alpha = ex2_approx(m_used - m_tile);
+          m_used = m_tile;
+        }
+        // P = exp2(s * c - m_used) as bf16 pairs; 1 pair in 4 takes the
+        // FMA-pipe exponential
+        const uint64_t c2 = f2_pack(c, c), negm2 = f2_pack(-m_used, -m_used);
+        uint64_t sum2 = f2_pack(0.f, 0.f);
+        auto chunk = [&](const uint32_t (&sk)[32], uint32_t (&pk)[16]) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const uint64_t x2 =
+                f2_fma(f2_pack(__uint_as_float(sk[2 * i]), __uint_as_float(sk[2 * i + 1])), c2, negm2);
+            float e0, e1;
+            if ((i & 7) < 2) {
+              exp2_poly_x2(x2, e0, e1);
+            } else {
+              float x0, x1;
+              f2_unpack(x2, x0, x1);
+              e0 = ex2_approx(x0);
+              e1 = ex2_approx(x1);
+            }
+            sum2 = f2_add(sum2, f2_pack(e0, e1));
+            pk[i] = pack_bf16x2(e0, e1);
+          }
+        };
+        uint32_t pk[16];
+        chunk(sa, pk);
+        if (tt > 0) {
+          // the previous P V must be done before P is overwritten (and, inside
+          // a segment, before O is rescaled)
+          if (!mbar_wait(&o_done[tile], (tt - 1) & 1, abort_flag, p.status)) {
+            aborted = true;
+            break;
+          }
+          tc_fence_after();
+          if (jj > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+              uint32_t o[32];
+              tmem_ld32(tO + 32 * hf, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+              tmem_st32(tO + 32 * hf, o);
+            }
+          }
+        }
+        tmem_st16(tP + 32, pk);
+        chunk(sb, pk);
+        tmem_st16(tP + 48, pk);
+        tmem_ld32(tS, sa);
+        tmem_ld32(tS + 32, sb);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_free[tile]);   // S(j+1) may now be computed
+        chunk(sa, pk);
+        tmem_st16(tP, pk);
+        chunk(sb, pk);
+        tmem_st16(tP + 16, pk);
+        float rs0, rs1;
+        f2_unpack(sum2, rs0, rs1);
+        l = l * alpha + (rs0 + rs1);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[tile]);
+      }
+      if (aborted) break;
+      // ---- end of the segment: O leaves tensor memory
+      if (!mbar_wait(&o_done[tile], (t + n - 1) & 1, abort_flag, p.status)) {
+        aborted = true;
+        break;
+      }
+      tc_fence_after();
+      float acc[64];
+      {
+        uint32_t o[2][32];
+        tmem_ld32(tO, o[0]);
+        tmem_ld32(tO + 32, o[1]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          acc[i] = __uint_as_float(o[0][i]);
+          acc[32 + i] = __uint_as_float(o[1][i]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_free[tile]);
+      const int h = sg.u / p.n_qt, q0 = (sg.u - h * p.n_qt) * 256;
+      float inv;
+      if (sg.k0 == 0 && sg.k1 == p.n_kv) {
+        inv = 1.f / l;
+      } else {
+        // A unit cut between CTAs b_lo..b_hi: each part stores its rows
+        // (unnormalised O, row max m in the log2 domain, row sum l); the part
+        // that finishes last merges the others and writes O.  Nothing waits on
+        // another CTA.
+        const int b_lo = (sg.u * p.n_kv) / p.L, b_hi = ((sg.u + 1) * p.n_kv - 1) / p.L;
+        const int me = blockIdx.x;
+        const int wslice = warp - 2;
+        auto slice = [&](int b) {
+          return reinterpret_cast<float4*>(p.part + static_cast<size_t>(2 * b + (b == b_lo ? 1 : 0)) * kPairSlotFloats +
+                                           static_cast<size_t>(wslice) * kPairSliceFloats) + lane;
+        };
+        float4* mine = slice(me);
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          mine[32 * i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+        mine[32 * 16] = make_float4(m_used, l, 0.f, 0.f);
+        __syncwarp();
+        unsigned last = 0;
+        if (lane == 0) {
+          __threadfence();
+          last = atomicAdd(p.count + b_lo * 8 + wslice, 1u) == static_cast<unsigned>(b_hi - b_lo);
+        }
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (!last) {
+          t += n;
+          ++si;
+          continue;
+        }
+        __threadfence();
+        float m = m_used, ls = l;
+        for (int b = b_lo; b <= b_hi; ++b) {
+          if (b == me) continue;
+          const float4* pc = slice(b);
+          const float4 ml = __ldcg(pc + 32 * 16);
+          float4 v[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = __ldcg(pc + 32 * i);
+          const float mn = fmaxf(m, ml.x);
+          const float a0 = ex2_approx(m - mn), a1 = ex2_approx(ml.x - mn);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            acc[4 * i] = fmaf(acc[4 * i], a0, v[i].x * a1);
+            acc[4 * i + 1] = fmaf(acc[4 * i + 1], a0, v[i].y * a1);
+            acc[4 * i + 2] = fmaf(acc[4 * i + 2], a0, v[i].z * a1);
+            acc[4 * i + 3] = fmaf(acc[4 * i + 3], a0, v[i].w * a1);
+          }
+          ls = fmaf(ls, a0, ml.y * a1);
+          m = mn;
+        }
+        if (lane == 0) p.count[b_lo * 8 + wslice] = 0u;   // ready for the next call
+        inv = 1.f / ls;
+      }
+      // O / l as bf16: each lane writes its row into the warp's staging rows
+      // (16-byte chunks rotated by the row, so 8 lanes cover all banks), then
+      // 8 lanes per row store 128 contiguous bytes
+      uint8_t* stage_rows = sOut + (warp - 2) * 4096;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        uint4 u;
+        u.x = pack_bf16x2(acc[8 * i] * inv, acc[8 * i + 1] * inv);
+        u.y = pack_bf16x2(acc[8 * i + 2] * inv, acc[8 * i + 3] * inv);
+        u.z = pack_bf16x2(acc[8 * i + 4] * inv, acc[8 * i + 5] * inv);
+        u.w = pack_bf16x2(acc[8 * i + 6] * inv, acc[8 * i + 7] * inv);
+        *reinterpret_cast<uint4*>(stage_rows + lane * 128 + ((i ^ (lane & 7)) << 4)) = u;
+      }
+      __syncwarp();
+      const int row0 = q0 + 128 * tile + q * 32;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int rr = 4 * k + (lane >> 3), ch = lane & 7;
+        const uint4 u = *reinterpret_cast<const uint4*>(stage_rows + rr * 128 + ((ch ^ (rr & 7)) << 4));
+        *reinterpret_cast<uint4*>(p.o + static_cast<size_t>(row0 + rr) * p.ld + h * 64 + ch * 8) = u;
+      }
+      __syncwarp();
+      t += n;
+      ++si;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  __syncwarp();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 // Workspace of the balanced launch: per-CTA part counters (zero before first
 // use; every call leaves them zero), then two partial slots per CTA.
 static size_t attn_count_bytes(size_t slots) { return (slots * 8 * sizeof(unsigned) + 255) & ~size_t(255); }
 
 size_t attn_workspace_bytes() {
-  const size_t slots = 2 * static_cast<size_t>(num_sms());
-  return attn_count_bytes(slots) + 2 * slots * kSlotFloats * sizeof(float);
+  // counters for up to two CTAs per SM; two partial slots per CTA of either kernel
+  const size_t sms = static_cast<size_t>(num_sms());
+  const size_t one = 2 * (2 * sms) * kSlotFloats, pair = 2 * sms * kPairSlotFloats;
+  return attn_count_bytes(2 * sms) + (one > pair ? one : pair) * sizeof(float);
 }
 
 int attn_launch(const void* q, const void* kf, const void* vf, const void* ks, const void* vs,
@@ -561,6 +1024,9 @@ int attn_launch(const void* q, const void* kf, const void* vf, const void* ks, c
   a.o = static_cast<__nv_bfloat16*>(o);
   a.ld = ld;
   a.status = device_status_ptr();
+  // Bands of a multiple of 256 tokens take the two-tile kernel (one CTA per
+  // SM); others the one-tile kernel (two CTAs per SM).
+  const bool pair = a.tb % 256 == 0;
   static int attr_mask = 0;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -568,24 +1034,27 @@ int attn_launch(const void* q, const void* kf, const void* vf, const void* ks, c
     int rc = cuda_check(cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              kAttnSmem),
                         "attention smem attribute");
+    if (!rc)
+      rc = cuda_check(cudaFuncSetAttribute(attn_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           kPairSmem),
+                      "attention smem attribute");
     if (rc) return rc;
     attr_mask |= 1 << (dev & 31);
   }
-  a.n_qt = T / 128;
+  a.n_qt = T / (pair ? 256 : 128);
   a.n_kv = mode == DP_MODE_NAIVE ? a.tb / 128 : T / 128;
   const int units = a.n_qt * heads;
   a.W = units * a.n_kv;
-  // Two CTAs fit on an SM (shared and tensor memory; the hardware places two
-  // although the occupancy calculator's register model allows one).  Balanced
-  // split: every CTA takes an equal run of (unit, key tile) iterations; the
-  // parts of a unit cut between CTAs are merged by whichever finishes last,
-  // so no CTA waits on another and any residency is correct.  Without a
-  // workspace each CTA takes one whole unit.
-  const int slots = 2 * num_sms();
-  // Cost in key-tile iterations of a paired CTA: a CTA's fixed cost (launch,
-  // set-up, first loads, epilogue) is about 5 of them and each cut segment
-  // about 2 more (measured on B200).  Whole units take ceil(units / slots)
-  // rounds; the split takes one round of L iterations.
+  // Balanced split: every CTA takes an equal run of (unit, key tile)
+  // iterations; the parts of a unit cut between CTAs are merged by whichever
+  // finishes last, so no CTA waits on another and any residency is correct.
+  // Without a workspace each CTA takes one whole unit.  The one-tile kernel
+  // fits two CTAs on an SM (shared and tensor memory), the two-tile kernel one.
+  const int slots = (pair ? 1 : 2) * num_sms();
+  // Cost in key-tile iterations of a CTA: its fixed cost (launch, set-up,
+  // first loads, epilogue) is about 5 of them and each cut segment about 2
+  // more (measured on B200 with the one-tile kernel).  Whole units take
+  // ceil(units / slots) rounds; the split takes one round of L iterations.
   const int L_split = (a.W + slots - 1) / slots;
   const double t_whole = static_cast<double>((units + slots - 1) / slots) * (a.n_kv + 5);
   const double t_split = L_split + 5 + 4;
@@ -594,12 +1063,15 @@ int attn_launch(const void* q, const void* kf, const void* vf, const void* ks, c
   if (split) {
     a.L = L_split;
     a.count = static_cast<unsigned*>(workspace);
-    a.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + attn_count_bytes(slots));
+    a.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + attn_count_bytes(2 * num_sms()));
   } else {
     a.L = a.n_kv;
   }
   const int grid = (a.W + a.L - 1) / a.L;
   mark_launch(stream);
+  if (pair)
+    return launch_kernel(attn_pair_kernel, dim3(grid), dim3(kPairThreads), kPairSmem, stream, false,
+                         "attention launch", a);
   return launch_kernel(attn_kernel, dim3(grid), dim3(kAttnThreads), kAttnSmem, stream, false,
                        "attention launch", a);
 }

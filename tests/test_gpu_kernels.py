@@ -274,13 +274,15 @@ def test_linear_parity(M, N, K, split, use_res):
 
 # ---------------------------------------------------------------- attention
 @pytest.mark.parametrize("T,heads,P,qscale", [(512, 2, 2, 1.0), (512, 2, 4, 3.0), (1024, 3, 2, 1.0),
-                                              (2048, 4, 16, 1.0), (4096, 10, 4, 1.0)])
+                                              (1536, 5, 2, 2.0), (2048, 4, 16, 1.0), (4096, 10, 4, 1.0)])
 @pytest.mark.parametrize("mode", MODES)
 @pytest.mark.parametrize("split", [True, False], ids=["split", "whole_tiles"])
 def test_attention_parity(T, heads, P, qscale, mode, split):
     """With a workspace the key tiles of a query tile may be cut between CTAs
-    (the cost model cuts them at T=1024, 2048 and 4096) and the partial
-    softmax sums are merged; without one every CTA takes whole tiles."""
+    (the cost model cuts them at T=1024, 1536, 2048 and 4096) and the partial
+    softmax sums are merged; without one every CTA takes whole tiles.  Bands
+    of 256, 512, 768 and 1024 tokens run the two-query-tile kernel, bands of
+    128 tokens the one-tile kernel."""
     r = rng(T + heads + P + mode)
     C = heads * 64
     q = rounded(qscale * r.standard_normal((T, C)), "bf16")
