@@ -536,30 +536,31 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_kernel(const __grid_cons
 //
 // A unit is 256 queries of one head: query tiles A and B (rows q0.. and
 // q0+128..) of the same band, so every key tile comes from the same buffer
-// for both and is loaded once for both.  One CTA per SM, 352 threads:
+// for both and is loaded once for both.  One CTA per SM, 608 threads:
 //   warp 0       TMA producer: both query tiles once per unit (double-
 //                buffered), K and V tiles of 128 keys through 3-deep rings;
-//   warps 1, 10  MMA issuers of tiles A and B.  `tcgen05.mma` returns only
+//   warps 1, 2   MMA issuers of tiles A and B.  `tcgen05.mma` returns only
 //                when the pipe accepts it, and one thread issues a 128x64x16
 //                P V instruction in about 56 cycles against 32 of math, so
 //                each tile has its own issuer.  Per key tile j an issuer
 //                computes S(j) = Q K_j^T as soon as the softmax warps have read
 //                S(j-1) out of tensor memory, then O += P(j-1) V_(j-1);
-//   warps 2-5    softmax of tile A, warps 6-9 of tile B: one thread per query
-//                row (no exchange between warps), online maximum with lazy
+//   warps 3-10   softmax of tile A, warps 11-18 of tile B: 16 query rows per
+//                warp, four threads per row; online maximum with lazy
 //                rescaling (O is rescaled only when the running maximum grows
 //                by more than 2^8), exp2 (1 in 4 on the FMA pipe), bf16 P to
 //                tensor memory; at the end of a unit O / l, stored as bf16.
 // Tensor memory (512 columns): S_A [0,128), S_B [128,256), O_A [256,320),
 // O_B [320,384), P_A [384,448), P_B [448,512) (P as bf16 pairs).
 constexpr int kPairStages = 3;
-constexpr int kPairThreads = 352;
-constexpr int kPairOutBytes = 8 * 4096;                   // per softmax warp: 32 rows x 128 B
+constexpr int kPairThreads = 608;
+constexpr int kPairOutBytes = 16 * 2048;                  // per softmax warp: 16 rows x 128 B
 constexpr int kPairSmem = 1024 + 4 * kTile + 2 * kPairStages * kTile + kPairOutBytes + kAttnTail;
-// A partial of one softmax warp: 17 float4 columns x 32 lanes (O's 16 float4
-// per row, then m, l), lane-contiguous so that every access is coalesced.
-constexpr int kPairSliceFloats = 17 * 32 * 4;
-constexpr int kPairSlotFloats = 8 * kPairSliceFloats;    // the 8 softmax warps
+// A partial of one softmax warp: 9 float4 columns x 32 lanes (a thread's 32
+// O values, then m and l of its two rows), lane-contiguous so that every
+// access is coalesced.
+constexpr int kPairSliceFloats = 9 * 32 * 4;
+constexpr int kPairSlotFloats = 16 * kPairSliceFloats;   // the 16 softmax warps
 static_assert(kPairSmem > 114 * 1024, "one CTA per SM: it allocates all of tensor memory");
 
 __global__ void __launch_bounds__(kPairThreads, 1) attn_pair_kernel(const __grid_constant__ AttnParams p) {
@@ -569,7 +570,7 @@ __global__ void __launch_bounds__(kPairThreads, 1) attn_pair_kernel(const __grid
   uint8_t* sQ = smem;                                           // [2 buffers][tiles A, B]
   uint8_t* sK = smem + 4 * kTile;
   uint8_t* sV = sK + kPairStages * kTile;
-  uint8_t* sOut = sV + kPairStages * kTile;                     // [8 softmax warps][32 rows][128 B]
+  uint8_t* sOut = sV + kPairStages * kTile;                     // [16 softmax warps][16 rows][128 B]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + kPairOutBytes);
   uint64_t* q_full = bars;                                      // [2]
   uint64_t* q_empty = q_full + 2;                               // [2]
@@ -596,10 +597,10 @@ __global__ void __launch_bounds__(kPairThreads, 1) attn_pair_kernel(const __grid
       mbar_init(&q_full[b], 1);
       mbar_init(&q_empty[b], 2);
       mbar_init(&s_full[b], 1);
-      mbar_init(&s_free[b], 4);
-      mbar_init(&p_full[b], 4);
+      mbar_init(&s_free[b], 8);
+      mbar_init(&p_full[b], 8);
       mbar_init(&o_done[b], 1);
-      mbar_init(&o_free[b], 4);
+      mbar_init(&o_free[b], 8);
       mbar_init(&drain[b], 1);
     }
     for (int s = 0; s < kPairStages; ++s) {
@@ -678,10 +679,10 @@ __global__ void __launch_bounds__(kPairThreads, 1) attn_pair_kernel(const __grid
                                (issued_par >> s) & 1u);
       }
     }
-  } else if (warp == 1 || warp == 10) {
+  } else if (warp == 1 || warp == 2) {
     if (lane == 0) {
       // ------------------------------------------------------------ MMA issuer
-      const int tile = warp == 1 ? 0 : 1;
+      const int tile = warp - 1;
       constexpr uint32_t idesc_qk = idesc_dense(128, 128, 1, 0, 0);
       constexpr uint32_t idesc_pv = idesc_dense(128, 64, 1, 0, 1);
       const uint32_t tS = tmem + 128 * tile, tO = tmem + 256 + 64 * tile, tP = tmem + 384 + 64 * tile;
@@ -750,13 +751,22 @@ __global__ void __launch_bounds__(kPairThreads, 1) attn_pair_kernel(const __grid
     }
   } else {
     // -------------------------------------------------------------- softmax
-    const int tile = (warp - 2) >> 2;          // query tile A (0) or B (1)
-    const int q = warp & 3;                    // tensor memory lane quarter
-    const int row = q * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    // Warp w (3..18): query tile (w-3)/8, TMEM lane quarter w%4 (the only
+    // lanes a warp may access), 16-row half ((w-3)/4)%2 of that quarter.
+    // With the 16x256b load shape, thread t holds rows t/4 and t/4+8 of the
+    // warp's 16 and, of each group of 8 columns, columns 2(t%4) and +1: a
+    // row's maximum and sum take two shuffles, and the thread's bf16 pairs
+    // are exactly the P words it stores with the 16x128b shape.
+    const int tile = (warp - 3) >> 3;
+    const int q = warp & 3;
+    const int half = ((warp - 3) >> 2) & 1;
+    const int wslice = warp - 3;
+    const int rbase = q * 32 + half * 16;                 // first row of the warp in the tile
+    const uint32_t lane_off = static_cast<uint32_t>(rbase) << 16;
     const uint32_t tS = tmem + 128 * tile + lane_off;
     const uint32_t tO = tmem + 256 + 64 * tile + lane_off;
     const uint32_t tP = tmem + 384 + 64 * tile + lane_off;
+    const int r = lane >> 2, cq = lane & 3;
     const float c = p.scale_log2;
     bool aborted = false;
     int t = 0, si = 0;
@@ -764,7 +774,7 @@ __global__ void __launch_bounds__(kPairThreads, 1) attn_pair_kernel(const __grid
     AttnSeg sg;
     while (!aborted && attn_next_seg(p, it, end, sg)) {
       const int n = sg.k1 - sg.k0;
-      float m_used = 0.f, l = 0.f;
+      float mA = 0.f, mB = 0.f, lA = 0.f, lB = 0.f;   // rows r and r+8: running max (log2), partial sum
       for (int jj = 0; jj < n; ++jj) {
         const int tt = t + jj;
         if (!mbar_wait(&s_full[tile], tt & 1, abort_flag, p.status)) {
@@ -772,66 +782,75 @@ __global__ void __launch_bounds__(kPairThreads, 1) attn_pair_kernel(const __grid
           break;
         }
         tc_fence_after();
-        // Row maximum from two loads of 64 columns; columns 64-127 stay in
-        // registers, columns 0-63 are read again after them (fewer live
-        // registers than holding the whole row), and only then is S released.
+        // Row maxima from both halves of S; columns 64-127 stay in registers,
+        // columns 0-63 are read again after them (fewer live registers), and
+        // only then is S released.
         uint32_t sa[32], sb[32];
-        tmem_ld32(tS, sa);
-        tmem_ld32(tS + 32, sb);
+        tmem_ld16x256_x8(tS, sa);
+        tmem_ld16x256_x8(tS + 64, sb);
         tmem_wait_ld();
-        float m0 = fmaxf(__uint_as_float(sa[0]), __uint_as_float(sa[1]));
-        float m1 = fmaxf(__uint_as_float(sa[16]), __uint_as_float(sa[17]));
-        float m2 = fmaxf(__uint_as_float(sb[0]), __uint_as_float(sb[1]));
-        float m3 = fmaxf(__uint_as_float(sb[16]), __uint_as_float(sb[17]));
+        float xa0 = fmaxf(__uint_as_float(sa[0]), __uint_as_float(sa[1]));
+        float xa1 = fmaxf(__uint_as_float(sb[0]), __uint_as_float(sb[1]));
+        float xb0 = fmaxf(__uint_as_float(sa[2]), __uint_as_float(sa[3]));
+        float xb1 = fmaxf(__uint_as_float(sb[2]), __uint_as_float(sb[3]));
 #pragma unroll
-        for (int i = 2; i < 16; i += 2) {
-          m0 = max3(m0, __uint_as_float(sa[i]), __uint_as_float(sa[i + 1]));
-          m1 = max3(m1, __uint_as_float(sa[16 + i]), __uint_as_float(sa[17 + i]));
-          m2 = max3(m2, __uint_as_float(sb[i]), __uint_as_float(sb[i + 1]));
-          m3 = max3(m3, __uint_as_float(sb[16 + i]), __uint_as_float(sb[17 + i]));
+        for (int k = 1; k < 8; ++k) {
+          xa0 = max3(xa0, __uint_as_float(sa[4 * k]), __uint_as_float(sa[4 * k + 1]));
+          xa1 = max3(xa1, __uint_as_float(sb[4 * k]), __uint_as_float(sb[4 * k + 1]));
+          xb0 = max3(xb0, __uint_as_float(sa[4 * k + 2]), __uint_as_float(sa[4 * k + 3]));
+          xb1 = max3(xb1, __uint_as_float(sb[4 * k + 2]), __uint_as_float(sb[4 * k + 3]));
         }
-        tmem_ld32(tS + 64, sa);
-        tmem_ld32(tS + 96, sb);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; i += 2) {
-          m0 = max3(m0, __uint_as_float(sa[i]), __uint_as_float(sa[i + 1]));
-          m1 = max3(m1, __uint_as_float(sa[16 + i]), __uint_as_float(sa[17 + i]));
-          m2 = max3(m2, __uint_as_float(sb[i]), __uint_as_float(sb[i + 1]));
-          m3 = max3(m3, __uint_as_float(sb[16 + i]), __uint_as_float(sb[17 + i]));
-        }
-        const float m_tile = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) * c;
-        float alpha = 1.f;
+        float xa = fmaxf(xa0, xa1), xb = fmaxf(xb0, xb1);
+        xa = fmaxf(xa, __shfl_xor_sync(0xffffffffu, xa, 1));
+        xb = fmaxf(xb, __shfl_xor_sync(0xffffffffu, xb, 1));
+        xa = fmaxf(xa, __shfl_xor_sync(0xffffffffu, xa, 2));
+        xb = fmaxf(xb, __shfl_xor_sync(0xffffffffu, xb, 2));
+        const float mtA = xa * c, mtB = xb * c;
+        float alA = 1.f, alB = 1.f;
         if (jj == 0) {
-          m_used = m_tile;
-        } else if (m_tile > m_used + 8.f) {
-          alpha = ex2_approx(m_used - m_tile);
-          m_used = m_tile;
+          mA = mtA;
+          mB = mtB;
+        } else {
+          if (mtA > mA + 8.f) {
+            alA = ex2_approx(mA - mtA);
+            mA = mtA;
+          }
+          if (mtB > mB + 8.f) {
+            alB = ex2_approx(mB - mtB);
+            mB = mtB;
+          }
         }
-        // P = exp2(s * c - m_used) as bf16 pairs; 1 pair in 4 takes the
-        // FMA-pipe exponential
-        const uint64_t c2 = f2_pack(c, c), negm2 = f2_pack(-m_used, -m_used);
-        uint64_t sum2 = f2_pack(0.f, 0.f);
-        auto chunk = [&](const uint32_t (&sk)[32], uint32_t (&pk)[16]) {
+        // P = exp2(s * c - m) as bf16 pairs; 1 pair in 4 takes the FMA-pipe
+        // exponential
+        const uint64_t c2 = f2_pack(c, c), nA2 = f2_pack(-mA, -mA), nB2 = f2_pack(-mB, -mB);
+        uint64_t sumA2 = f2_pack(0.f, 0.f), sumB2 = f2_pack(0.f, 0.f);
+        auto exps = [&](const uint32_t (&sk)[32], uint32_t (&pk)[16]) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const uint64_t x2 =
-                f2_fma(f2_pack(__uint_as_float(sk[2 * i]), __uint_as_float(sk[2 * i + 1])), c2, negm2);
-            float e0, e1;
-            if ((i & 7) < 2) {
-              exp2_poly_x2(x2, e0, e1);
-            } else {
-              float x0, x1;
-              f2_unpack(x2, x0, x1);
-              e0 = ex2_approx(x0);
-              e1 = ex2_approx(x1);
+          for (int k = 0; k < 8; ++k) {
+#pragma unroll
+            for (int rw = 0; rw < 2; ++rw) {
+              const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sk[4 * k + 2 * rw]),
+                                                 __uint_as_float(sk[4 * k + 2 * rw + 1])),
+                                         c2, rw ? nB2 : nA2);
+              float e0, e1;
+              if ((k & 3) == 0) {
+                exp2_poly_x2(x2, e0, e1);
+              } else {
+                float x0, x1;
+                f2_unpack(x2, x0, x1);
+                e0 = ex2_approx(x0);
+                e1 = ex2_approx(x1);
+              }
+              if (rw)
+                sumB2 = f2_add(sumB2, f2_pack(e0, e1));
+              else
+                sumA2 = f2_add(sumA2, f2_pack(e0, e1));
+              pk[2 * k + rw] = pack_bf16x2(e0, e1);
             }
-            sum2 = f2_add(sum2, f2_pack(e0, e1));
-            pk[i] = pack_bf16x2(e0, e1);
           }
         };
         uint32_t pk[16];
-        chunk(sa, pk);
+        exps(sb, pk);
         if (tt > 0) {
           // the previous P V must be done before P is overwritten (and, inside
           // a segment, before O is rescaled)
@@ -840,34 +859,33 @@ __global__ void __launch_bounds__(kPairThreads, 1) attn_pair_kernel(const __grid
             break;
           }
           tc_fence_after();
-          if (jj > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+          if (jj > 0 && __any_sync(0xffffffffu, alA != 1.f || alB != 1.f)) {
+            uint32_t o[32];
+            tmem_ld16x256_x8(tO, o);
+            tmem_wait_ld();
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-              uint32_t o[32];
-              tmem_ld32(tO + 32 * hf, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-              tmem_st32(tO + 32 * hf, o);
+            for (int k = 0; k < 8; ++k) {
+              o[4 * k] = __float_as_uint(__uint_as_float(o[4 * k]) * alA);
+              o[4 * k + 1] = __float_as_uint(__uint_as_float(o[4 * k + 1]) * alA);
+              o[4 * k + 2] = __float_as_uint(__uint_as_float(o[4 * k + 2]) * alB);
+              o[4 * k + 3] = __float_as_uint(__uint_as_float(o[4 * k + 3]) * alB);
             }
+            tmem_st16x256_x8(tO, o);
           }
         }
-        tmem_st16(tP + 32, pk);
-        chunk(sb, pk);
-        tmem_st16(tP + 48, pk);
-        tmem_ld32(tS, sa);
-        tmem_ld32(tS + 32, sb);
+        tmem_st16x128_x8(tP + 32, pk);
+        tmem_ld16x256_x8(tS, sa);
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_free[tile]);   // S(j+1) may now be computed
-        chunk(sa, pk);
-        tmem_st16(tP, pk);
-        chunk(sb, pk);
-        tmem_st16(tP + 16, pk);
-        float rs0, rs1;
-        f2_unpack(sum2, rs0, rs1);
-        l = l * alpha + (rs0 + rs1);
+        exps(sa, pk);
+        tmem_st16x128_x8(tP, pk);
+        float s0, s1;
+        f2_unpack(sumA2, s0, s1);
+        lA = lA * alA + (s0 + s1);
+        f2_unpack(sumB2, s0, s1);
+        lB = lB * alB + (s0 + s1);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -880,25 +898,24 @@ __global__ void __launch_bounds__(kPairThreads, 1) attn_pair_kernel(const __grid
         break;
       }
       tc_fence_after();
-      float acc[64];
-      {
-        uint32_t o[2][32];
-        tmem_ld32(tO, o[0]);
-        tmem_ld32(tO + 32, o[1]);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          acc[i] = __uint_as_float(o[0][i]);
-          acc[32 + i] = __uint_as_float(o[1][i]);
-        }
-      }
+      uint32_t ob[32];
+      tmem_ld16x256_x8(tO, ob);
+      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&o_free[tile]);
+      lA += __shfl_xor_sync(0xffffffffu, lA, 1);
+      lB += __shfl_xor_sync(0xffffffffu, lB, 1);
+      lA += __shfl_xor_sync(0xffffffffu, lA, 2);
+      lB += __shfl_xor_sync(0xffffffffu, lB, 2);
+      float acc[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) acc[i] = __uint_as_float(ob[i]);
       const int h = sg.u / p.n_qt, q0 = (sg.u - h * p.n_qt) * 256;
-      float inv;
+      float invA, invB;
       if (sg.k0 == 0 && sg.k1 == p.n_kv) {
-        inv = 1.f / l;
+        invA = 1.f / lA;
+        invB = 1.f / lB;
       } else {
         // A unit cut between CTAs b_lo..b_hi: each part stores its rows
         // (unnormalised O, row max m in the log2 domain, row sum l); the part
@@ -906,21 +923,20 @@ __global__ void __launch_bounds__(kPairThreads, 1) attn_pair_kernel(const __grid
         // another CTA.
         const int b_lo = (sg.u * p.n_kv) / p.L, b_hi = ((sg.u + 1) * p.n_kv - 1) / p.L;
         const int me = blockIdx.x;
-        const int wslice = warp - 2;
         auto slice = [&](int b) {
           return reinterpret_cast<float4*>(p.part + static_cast<size_t>(2 * b + (b == b_lo ? 1 : 0)) * kPairSlotFloats +
                                            static_cast<size_t>(wslice) * kPairSliceFloats) + lane;
         };
         float4* mine = slice(me);
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
+        for (int i = 0; i < 8; ++i)
           mine[32 * i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
-        mine[32 * 16] = make_float4(m_used, l, 0.f, 0.f);
+        mine[32 * 8] = make_float4(mA, lA, mB, lB);
         __syncwarp();
         unsigned last = 0;
         if (lane == 0) {
           __threadfence();
-          last = atomicAdd(p.count + b_lo * 8 + wslice, 1u) == static_cast<unsigned>(b_hi - b_lo);
+          last = atomicAdd(p.count + b_lo * 16 + wslice, 1u) == static_cast<unsigned>(b_hi - b_lo);
         }
         last = __shfl_sync(0xffffffffu, last, 0);
         if (!last) {
@@ -929,46 +945,49 @@ __global__ void __launch_bounds__(kPairThreads, 1) attn_pair_kernel(const __grid
           continue;
         }
         __threadfence();
-        float m = m_used, ls = l;
+        float ma = mA, la = lA, mb = mB, lb = lB;
         for (int b = b_lo; b <= b_hi; ++b) {
           if (b == me) continue;
           const float4* pc = slice(b);
-          const float4 ml = __ldcg(pc + 32 * 16);
-          float4 v[16];
+          const float4 ml = __ldcg(pc + 32 * 8);
+          float4 v[8];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) v[i] = __ldcg(pc + 32 * i);
-          const float mn = fmaxf(m, ml.x);
-          const float a0 = ex2_approx(m - mn), a1 = ex2_approx(ml.x - mn);
+          for (int i = 0; i < 8; ++i) v[i] = __ldcg(pc + 32 * i);
+          const float na = fmaxf(ma, ml.x), nb = fmaxf(mb, ml.z);
+          const float a0 = ex2_approx(ma - na), a1 = ex2_approx(ml.x - na);
+          const float b0 = ex2_approx(mb - nb), b1 = ex2_approx(ml.z - nb);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
+          for (int i = 0; i < 8; ++i) {
             acc[4 * i] = fmaf(acc[4 * i], a0, v[i].x * a1);
             acc[4 * i + 1] = fmaf(acc[4 * i + 1], a0, v[i].y * a1);
-            acc[4 * i + 2] = fmaf(acc[4 * i + 2], a0, v[i].z * a1);
-            acc[4 * i + 3] = fmaf(acc[4 * i + 3], a0, v[i].w * a1);
+            acc[4 * i + 2] = fmaf(acc[4 * i + 2], b0, v[i].z * b1);
+            acc[4 * i + 3] = fmaf(acc[4 * i + 3], b0, v[i].w * b1);
           }
-          ls = fmaf(ls, a0, ml.y * a1);
-          m = mn;
+          la = fmaf(la, a0, ml.y * a1);
+          lb = fmaf(lb, b0, ml.w * b1);
+          ma = na;
+          mb = nb;
         }
-        if (lane == 0) p.count[b_lo * 8 + wslice] = 0u;   // ready for the next call
-        inv = 1.f / ls;
+        if (lane == 0) p.count[b_lo * 16 + wslice] = 0u;   // ready for the next call
+        invA = 1.f / la;
+        invB = 1.f / lb;
       }
-      // O / l as bf16: each lane writes its row into the warp's staging rows
-      // (16-byte chunks rotated by the row, so 8 lanes cover all banks), then
+      // O / l as bf16 through the warp's 16 staging rows of 128 bytes (16-byte
+      // chunks rotated by the row, so a quarter-warp covers all banks), then
       // 8 lanes per row store 128 contiguous bytes
-      uint8_t* stage_rows = sOut + (warp - 2) * 4096;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        uint4 u;
-        u.x = pack_bf16x2(acc[8 * i] * inv, acc[8 * i + 1] * inv);
-        u.y = pack_bf16x2(acc[8 * i + 2] * inv, acc[8 * i + 3] * inv);
-        u.z = pack_bf16x2(acc[8 * i + 4] * inv, acc[8 * i + 5] * inv);
-        u.w = pack_bf16x2(acc[8 * i + 6] * inv, acc[8 * i + 7] * inv);
-        *reinterpret_cast<uint4*>(stage_rows + lane * 128 + ((i ^ (lane & 7)) << 4)) = u;
-      }
-      __syncwarp();
-      const int row0 = q0 + 128 * tile + q * 32;
+      uint8_t* stage_rows = sOut + wslice * 2048;
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
+        const int off = ((k ^ r) << 4) + 4 * cq;
+        *reinterpret_cast<uint32_t*>(stage_rows + r * 128 + off) =
+            pack_bf16x2(acc[4 * k] * invA, acc[4 * k + 1] * invA);
+        *reinterpret_cast<uint32_t*>(stage_rows + (r + 8) * 128 + off) =
+            pack_bf16x2(acc[4 * k + 2] * invB, acc[4 * k + 3] * invB);
+      }
+      __syncwarp();
+      const int row0 = q0 + 128 * tile + rbase;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
         const int rr = 4 * k + (lane >> 3), ch = lane & 7;
         const uint4 u = *reinterpret_cast<const uint4*>(stage_rows + rr * 128 + ((ch ^ (rr & 7)) << 4));
         *reinterpret_cast<uint4*>(p.o + static_cast<size_t>(row0 + rr) * p.ld + h * 64 + ch * 8) = u;
@@ -978,7 +997,6 @@ __global__ void __launch_bounds__(kPairThreads, 1) attn_pair_kernel(const __grid
       ++si;
     }
   }
-
   tc_fence_before();
   __syncthreads();
   __syncwarp();
