@@ -849,8 +849,16 @@ __global__ void __launch_bounds__(kPairThreads, 1) attn_pair_kernel(const __grid
             }
           }
         };
-        uint32_t pk[16];
-        exps(sb, pk);
+        // Both halves are exponentiated before P is written, so the previous
+        // P V (which frees the P columns) has the whole softmax to complete.
+        uint32_t pk_hi[16], pk_lo[16];
+        exps(sb, pk_hi);
+        tmem_ld16x256_x8(tS, sa);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_free[tile]);   // S(j+1) may now be computed
+        exps(sa, pk_lo);
         if (tt > 0) {
           // the previous P V must be done before P is overwritten (and, inside
           // a segment, before O is rescaled)
@@ -873,14 +881,8 @@ __global__ void __launch_bounds__(kPairThreads, 1) attn_pair_kernel(const __grid
             tmem_st16x256_x8(tO, o);
           }
         }
-        tmem_st16x128_x8(tP + 32, pk);
-        tmem_ld16x256_x8(tS, sa);
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_free[tile]);   // S(j+1) may now be computed
-        exps(sa, pk);
-        tmem_st16x128_x8(tP, pk);
+        tmem_st16x128_x8(tP + 32, pk_hi);
+        tmem_st16x128_x8(tP, pk_lo);
         float s0, s1;
         f2_unpack(sumA2, s0, s1);
         lA = lA * alA + (s0 + s1);
