@@ -36,6 +36,10 @@ sys.path.insert(0, ROOT)
 
 METRIC = "displaced U-Net block step latency & TFLOP/s; GroupNorm GB/s; % of roofline"
 FLUSH_BYTES = 256 << 20
+# GroupNorm statistics of the displaced steps (--gn-stats): the method's
+# corrected statistics (default) or one of its ablation alternatives
+GN_STATS_NAMES = ["corrected", "local", "stale", "sync"]
+GN_STATS = 0
 
 
 def load_peaks():
@@ -148,9 +152,11 @@ def block_kind(B, wl):
 
 
 def block_desc(B, wl, H=None):
-    return B.dp_block_desc_init(block_kind(B, wl), H or wl.H, wl.W, wl.C, wl.cout, wl.G, wl.P,
-                                wl.heads, B.BF16 if wl.dtype == "bf16" else B.FP32, wl.silu,
-                                wl.eps, 1.0)
+    d = B.dp_block_desc_init(block_kind(B, wl), H or wl.H, wl.W, wl.C, wl.cout, wl.G, wl.P,
+                             wl.heads, B.BF16 if wl.dtype == "bf16" else B.FP32, wl.silu,
+                             wl.eps, 1.0)
+    B.dp_block_desc_set_gn_stats(d, GN_STATS)
+    return d
 
 
 def launch_plan(B, wl, mode):
@@ -173,7 +179,7 @@ def cpu_baseline_ours(wl, seconds):
     reps, t0 = 0, time.perf_counter()
     while True:
         O.block_step(wl.kind, st, x1, wts, wl.P, wl.G, wl.eps, 1.0, synth.DISPLACED, wl.dtype,
-                     heads=wl.heads, silu=wl.silu)
+                     heads=wl.heads, silu=wl.silu, gn_stats=GN_STATS)
         reps += 1
         el = time.perf_counter() - t0
         if el >= seconds:
@@ -206,7 +212,7 @@ def run_reference(args, wl):
                      heads=w.heads, silu=w.silu)
         t0 = time.perf_counter()
         O.block_step(w.kind, st, xs.x(1)[0], wts, w.P, w.G, w.eps, 1.0, synth.DISPLACED, w.dtype,
-                     heads=w.heads, silu=w.silu)
+                     heads=w.heads, silu=w.silu, gn_stats=GN_STATS)
         return time.perf_counter() - t0, wts, st, xs
 
     hb = wl.H // wl.P
@@ -222,11 +228,11 @@ def run_reference(args, wl):
     x = xs.x(2)[0]
     for _ in range(args.warmup):
         O.block_step(w.kind, st, x, wts, w.P, w.G, w.eps, 1.0, synth.DISPLACED, w.dtype,
-                     heads=w.heads, silu=w.silu)
+                     heads=w.heads, silu=w.silu, gn_stats=GN_STATS)
     t0 = time.perf_counter()
     for _ in range(args.steps):
         O.block_step(w.kind, st, x, wts, w.P, w.G, w.eps, 1.0, synth.DISPLACED, w.dtype,
-                     heads=w.heads, silu=w.silu)
+                     heads=w.heads, silu=w.silu, gn_stats=GN_STATS)
     el = time.perf_counter() - t0
     flops = wl_flops(wl, w.H)
     value = flops * args.steps / el / 1e12
@@ -236,7 +242,8 @@ def run_reference(args, wl):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name, "sample": sample},
+            "config": {"workload": wl.name, "shape_nchw": [1, wl.C, wl.H, wl.W], "P": wl.P,
+                       "mode": "displaced", "gn_stats": GN_STATS_NAMES[GN_STATS], "sample": sample},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -265,7 +272,8 @@ def run_ours(args, wl):
     wts = synth.make_weights(wl)
     dw = block_weights(wl.kind, wts, tdt, dev)
     blk = B.Block(block_kind(B, wl), wl.H, wl.W, wl.C, wl.cout, wl.G, wl.P, wl.heads,
-                  B.BF16 if wl.dtype == "bf16" else B.FP32, wl.silu, wl.eps, 1.0, device=dev)
+                  B.BF16 if wl.dtype == "bf16" else B.FP32, wl.silu, wl.eps, 1.0, device=dev,
+                  gn_stats=GN_STATS)
     xs = synth.InputStream(wl)
     pool = 4
     host_x = [synth.nchw_to_nhwc(xs.x(k)).to(tdt).pin_memory() for k in range(pool)]
@@ -428,7 +436,8 @@ def run_ours(args, wl):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
             "data": "synthetic",
             "config": {"workload": wl.name, "shape_nchw": [1, wl.C, wl.H, wl.W], "P": wl.P,
-                       "mode": "displaced", "l2": "flushed between steps (256 MiB write, untimed)",
+                       "mode": "displaced", "gn_stats": GN_STATS_NAMES[GN_STATS],
+                       "l2": "flushed between steps (256 MiB write, untimed)",
                        "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
             "roofline": roof, "kernels": kernels, "groupnorm": gn,
             "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s",
@@ -459,7 +468,11 @@ def main():
     ap.add_argument("--workload", default="resblock_320x128x128")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--gn-stats", choices=GN_STATS_NAMES, default="corrected",
+                    help="GroupNorm statistics of the displaced steps")
     args = ap.parse_args()
+    global GN_STATS
+    GN_STATS = GN_STATS_NAMES.index(args.gn_stats)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     from displaced_patch_parallelism_b200 import synth

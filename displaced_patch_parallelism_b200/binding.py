@@ -19,6 +19,7 @@ DP_OK, DP_ERR_INVALID_ARG, DP_ERR_UNSUPPORTED, DP_ERR_STATE, DP_ERR_CUDA, DP_ERR
 SYNC, DISPLACED, NAIVE = 0, 1, 2
 BF16, FP32 = 0, 1
 GN_CONV, RESBLOCK, ATTN, UNET_MINI = 0, 1, 2, 3
+GN_STATS_CORRECTED, GN_STATS_LOCAL, GN_STATS_STALE, GN_STATS_SYNC = 0, 1, 2, 3
 
 ERR_NAMES = {DP_ERR_INVALID_ARG: "DP_ERR_INVALID_ARG", DP_ERR_UNSUPPORTED: "DP_ERR_UNSUPPORTED",
              DP_ERR_STATE: "DP_ERR_STATE", DP_ERR_CUDA: "DP_ERR_CUDA",
@@ -35,7 +36,8 @@ class BlockDesc(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int),
                 ("C", ctypes.c_int), ("Cout", ctypes.c_int), ("G", ctypes.c_int),
                 ("P", ctypes.c_int), ("heads", ctypes.c_int), ("dtype", ctypes.c_int),
-                ("silu", ctypes.c_int), ("eps", ctypes.c_float), ("w", ctypes.c_float)]
+                ("silu", ctypes.c_int), ("eps", ctypes.c_float), ("w", ctypes.c_float),
+                ("gn_stats", ctypes.c_int)]
 
 
 class BlockState(ctypes.Structure):
@@ -63,6 +65,7 @@ _SIGS = {
     "dp_refresh_stale": ([_V, _V, _SZ, _I, _I, _I, _V], _I),
     "dp_refresh_stats": ([_V, _V, _V, _I, _I, _V], _I),
     "dp_block_desc_init": ([ctypes.POINTER(BlockDesc), _I, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _F], _I),
+    "dp_block_desc_set_gn_stats": ([ctypes.POINTER(BlockDesc), _I], _I),
     "dp_block_workspace_size": ([ctypes.POINTER(BlockDesc)], _SZ),
     "dp_block_state_init": ([ctypes.POINTER(BlockDesc), ctypes.POINTER(BlockState), _V, _SZ, _V], _I),
     "dp_block_step": ([ctypes.POINTER(BlockDesc), ctypes.POINTER(BlockState), _V, _V,
@@ -212,6 +215,10 @@ def dp_block_desc_init(kind, H, W, C, Cout, G, P, heads, dtype, silu, eps, w) ->
     return d
 
 
+def dp_block_desc_set_gn_stats(d: BlockDesc, variant: int):
+    return _check(lib().dp_block_desc_set_gn_stats(ctypes.byref(d), variant))
+
+
 def dp_block_workspace_size(d: BlockDesc) -> int:
     n = lib().dp_block_workspace_size(ctypes.byref(d))
     if n == 0:
@@ -281,9 +288,11 @@ class Block:
     """A block descriptor, its device workspace (a torch uint8 tensor) and its state."""
 
     def __init__(self, kind, H, W, C, Cout=0, G=32, P=4, heads=0, dtype=BF16, silu=True,
-                 eps=1e-5, w=1.0, device="cuda", stream=None):
+                 eps=1e-5, w=1.0, device="cuda", stream=None, gn_stats=GN_STATS_CORRECTED):
         import torch
         self.desc = dp_block_desc_init(kind, H, W, C, Cout, G, P, heads, dtype, silu, eps, w)
+        if gn_stats != GN_STATS_CORRECTED:
+            dp_block_desc_set_gn_stats(self.desc, gn_stats)
         self.ws_bytes = dp_block_workspace_size(self.desc)
         self.workspace = torch.empty(self.ws_bytes, dtype=torch.uint8, device=device)
         self.state = dp_block_state_init(self.desc, self.workspace, self.ws_bytes, stream)

@@ -153,6 +153,8 @@ int desc_check(const dp_block_desc* d) {
   if (d->dtype == DP_FP32 && d->kind != DP_BLOCK_GN_CONV)
     return set_error(DP_ERR_UNSUPPORTED, "block: fp32 storage is only built for GN_CONV");
   if (!(d->eps > 0.f)) return set_error(DP_ERR_INVALID_ARG, "block: eps must be > 0");
+  if (d->gn_stats < DP_GN_STATS_CORRECTED || d->gn_stats > DP_GN_STATS_SYNC)
+    return set_error(DP_ERR_INVALID_ARG, "block: unknown GroupNorm statistics variant %d", d->gn_stats);
   if (d->H % d->P) return set_error(DP_ERR_UNSUPPORTED, "block: H %% P != 0");
   if (d->kind == DP_BLOCK_UNET_MINI) {
     if (d->C > 16 || d->C % 2)
@@ -231,13 +233,22 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
   const double e = d->dtype == DP_FP32 ? 4.0 : 2.0;
   const int f = cur ^ 1, o = cur;
   const int H = d->H, W = d->W, C = d->C, Co = d->Cout, G = d->G, P = d->P;
+  // statistics of this step's GroupNorms: a displaced step takes the
+  // descriptor's variant (corrected, band-local, stale-only or exact)
+  int gn_mode = mode;
+  float gn_w = d->w;
+  if (mode == DP_MODE_DISPLACED) {
+    if (d->gn_stats == DP_GN_STATS_LOCAL) gn_mode = DP_MODE_NAIVE;
+    if (d->gn_stats == DP_GN_STATS_STALE) gn_w = 0.0f;
+    if (d->gn_stats == DP_GN_STATS_SYNC) gn_mode = DP_MODE_SYNC;
+  }
   auto gn = [&](const GnSlots& g, const void* in, void* y, const void* gamma, const void* beta,
                 int ch, int silu) {
     if (plan) {
       const double bytes = static_cast<double>(H) * W * ch * e;
       int nb, chunk, th;
       size_t sm;
-      if (gn_cluster_plan(H, W, ch, G, P, d->dtype, mode, &nb, &chunk, &th, &sm)) {
+      if (gn_cluster_plan(H, W, ch, G, P, d->dtype, gn_mode, &nb, &chunk, &th, &sm)) {
         plan->push(DP_KERNEL_GN_CLUSTER, 0.0, 2.0 * bytes);
       } else if (gn_fused_plan(H, W, ch, G, P, d->dtype, &nb, &chunk, &th, &sm)) {
         plan->push(DP_KERNEL_GN_FUSED, 0.0, 2.0 * bytes);
@@ -248,7 +259,7 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
       return DP_OK;
     }
     return gn_launch(in, y, static_cast<const float*>(gamma), static_cast<const float*>(beta), H,
-                     W, ch, G, P, d->eps, d->w, silu, mode, d->dtype, at<float>(ws, g.global[o]),
+                     W, ch, G, P, d->eps, gn_w, silu, gn_mode, d->dtype, at<float>(ws, g.global[o]),
                      at<float>(ws, g.local[o]), at<float>(ws, g.local[f]),
                      at<float>(ws, g.global[f]), at<float>(ws, g.used), at<void>(ws, g.ws),
                      gn_workspace_bytes(P, G), st);
@@ -443,7 +454,16 @@ int dp_block_desc_init(dp_block_desc* d, int kind, int H, int W, int C, int Cout
   d->silu = silu;
   d->eps = eps;
   d->w = w;
+  d->gn_stats = DP_GN_STATS_CORRECTED;
   return dp::desc_check(d);
+}
+
+int dp_block_desc_set_gn_stats(dp_block_desc* d, int variant) {
+  if (!d) return dp::set_error(DP_ERR_INVALID_ARG, "block: null descriptor");
+  if (variant < DP_GN_STATS_CORRECTED || variant > DP_GN_STATS_SYNC)
+    return dp::set_error(DP_ERR_INVALID_ARG, "block: unknown GroupNorm statistics variant %d", variant);
+  d->gn_stats = variant;
+  return DP_OK;
 }
 
 size_t dp_block_workspace_size(const dp_block_desc* d) {

@@ -299,6 +299,7 @@ typedef struct dp_block_desc {
   int silu;       /* GN_CONV: SiLU after GroupNorm                */
   float eps;      /* GroupNorm epsilon                            */
   float w;        /* weight of the corrected-statistics drift term */
+  int gn_stats;   /* DP_GN_STATS_*: statistics of displaced steps  */
 } dp_block_desc;
 
 typedef struct dp_block_state {
@@ -310,6 +311,27 @@ typedef struct dp_block_state {
 
 DP_API int dp_block_desc_init(dp_block_desc* d, int kind, int H, int W, int C, int Cout, int G,
                        int P, int heads, int dtype, int silu, float eps, float w);
+
+/*
+ * GroupNorm statistics of the displaced steps of a block: the method's
+ * corrected asynchronous statistics, or one of the alternatives its GroupNorm
+ * ablation compares ("DistriFusion", atlas.scime.ai summary, Approach and the
+ * GroupNorm ablation rows: statistics of the device's own patch only, stale
+ * statistics only, and a synchronous exact pass).  Only DISPLACED steps are
+ * affected; SYNC and NAIVE steps keep their own statistics.  The halo rows
+ * and the keys and values stay stale in every variant.
+ *   DP_GN_STATS_CORRECTED  stale_global + w (fresh_local - stale_local)  (default)
+ *   DP_GN_STATS_LOCAL      the band's own fresh moments
+ *   DP_GN_STATS_STALE      the previous step's whole-image moments (w = 0)
+ *   DP_GN_STATS_SYNC       the exact whole-image moments of this step
+ * dp_block_desc_init sets DP_GN_STATS_CORRECTED.  Returns DP_ERR_INVALID_ARG
+ * for an unknown variant or a null descriptor.
+ */
+#define DP_GN_STATS_CORRECTED 0
+#define DP_GN_STATS_LOCAL 1
+#define DP_GN_STATS_STALE 2
+#define DP_GN_STATS_SYNC 3
+DP_API int dp_block_desc_set_gn_stats(dp_block_desc* d, int variant);
 DP_API size_t dp_block_workspace_size(const dp_block_desc* d);
 DP_API int dp_block_state_init(const dp_block_desc* d, dp_block_state* s, void* workspace,
                         size_t workspace_bytes, void* stream);

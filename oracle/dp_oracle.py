@@ -312,8 +312,35 @@ class GNState:
         self.stale_global, self.stale_local = refresh_stats(f)
 
 
-def _gn(st: GNState, x, gamma, beta, P, G, eps, w, silu, mode, trace, key):
-    y, f, used, nneg = groupnorm_async(x, gamma, beta, P, G, eps, w, silu, mode,
+# GroupNorm statistics variants of a displaced step ("DistriFusion",
+# atlas.scime.ai summary, the GroupNorm ablation rows): the method's corrected
+# statistics, statistics of the band alone, the stale statistics alone, or an
+# exact synchronous pass.  Only displaced steps change; the halos and the
+# keys/values stay stale.
+GN_STATS_CORRECTED, GN_STATS_LOCAL, GN_STATS_STALE, GN_STATS_SYNC = 0, 1, 2, 3
+
+
+def gn_variant_mode(mode: int, w: float, gn_stats: int) -> Tuple[int, float]:
+    """(statistics mode, drift weight) a GroupNorm of a step in ``mode`` uses.
+
+    corrected: displaced statistics with weight w; band-local: the band's own
+    moments (as in a naive step); stale-only: displaced with w = 0, i.e. the
+    previous step's whole-image moments; sync: the exact whole-image moments.
+    """
+    if mode != DISPLACED or gn_stats == GN_STATS_CORRECTED:
+        return mode, w
+    if gn_stats == GN_STATS_LOCAL:
+        return NAIVE, w
+    if gn_stats == GN_STATS_STALE:
+        return DISPLACED, 0.0
+    if gn_stats == GN_STATS_SYNC:
+        return SYNC, w
+    raise ValueError(gn_stats)
+
+
+def _gn(st: GNState, x, gamma, beta, P, G, eps, w, silu, mode, trace, key, gn_stats=GN_STATS_CORRECTED):
+    gmode, gw = gn_variant_mode(mode, w, gn_stats)
+    y, f, used, nneg = groupnorm_async(x, gamma, beta, P, G, eps, gw, silu, gmode,
                                        st.stale_global, st.stale_local)
     if trace is not None:
         trace[key + ".fresh_local"] = f
@@ -330,12 +357,12 @@ def _a(x) -> np.ndarray:
 
 def gn_conv_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float,
                  silu: bool, mode: int, storage: str, trace: Optional[Dict] = None,
-                 final_storage: Optional[str] = None):
+                 final_storage: Optional[str] = None, gn_stats: int = GN_STATS_CORRECTED):
     """GroupNorm (+SiLU) -> 3x3 conv with stale halo.  x: (C, H, W)."""
     x = _a(x)
     gn = state.setdefault("gn", GNState())
     a, f = _gn(gn, x, _a(wts["gn_gamma"]), _a(wts["gn_beta"]), P, G, eps, w, silu, mode,
-               trace, "gn")
+               trace, "gn", gn_stats)
     a = store(a, storage)
     out = conv3x3_halo(a, state.get("a_stale"), _a(wts["conv_w"]), _a(wts["conv_b"]), None,
                        P, mode)
@@ -349,19 +376,19 @@ def gn_conv_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float
 
 def resblock_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float,
                   mode: int, storage: str, trace: Optional[Dict] = None, prefix: str = "",
-                  final_storage: Optional[str] = None):
+                  final_storage: Optional[str] = None, gn_stats: int = GN_STATS_CORRECTED):
     """GN -> SiLU -> conv1 -> GN -> SiLU -> conv2 -> + x (or + 1x1 shortcut(x))."""
     x = _a(x)
     W_ = lambda n: _a(wts[prefix + n])
     gn1 = state.setdefault("gn1", GNState())
     gn2 = state.setdefault("gn2", GNState())
     a1, f1 = _gn(gn1, x, W_("gn1_gamma"), W_("gn1_beta"), P, G, eps, w, True, mode, trace,
-                 prefix + "gn1")
+                 prefix + "gn1", gn_stats)
     a1 = store(a1, storage)
     h = store(conv3x3_halo(a1, state.get("a1_stale"), W_("conv1_w"), W_("conv1_b"), None, P,
                            mode), storage)
     a2, f2 = _gn(gn2, h, W_("gn2_gamma"), W_("gn2_beta"), P, G, eps, w, True, mode, trace,
-                 prefix + "gn2")
+                 prefix + "gn2", gn_stats)
     a2 = store(a2, storage)
     if (prefix + "short_w") in wts:
         res = store(conv1x1(x, W_("short_w"), W_("short_b")), storage)
@@ -379,7 +406,7 @@ def resblock_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: floa
 
 def attn_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float, heads: int,
               mode: int, storage: str, trace: Optional[Dict] = None, prefix: str = "",
-              final_storage: Optional[str] = None):
+              final_storage: Optional[str] = None, gn_stats: int = GN_STATS_CORRECTED):
     """GN (no SiLU) -> q, k, v projections -> stale-K/V attention -> out proj + bias -> + x.
 
     x: (C, H, W); tokens are pixels in raster order, so band p's tokens are
@@ -390,7 +417,7 @@ def attn_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float, h
     W_ = lambda n: _a(wts[prefix + n])
     gn = state.setdefault("gn", GNState())
     a, f = _gn(gn, x, W_("gn_gamma"), W_("gn_beta"), P, G, eps, w, False, mode, trace,
-               prefix + "gn")
+               prefix + "gn", gn_stats)
     a = store(a, storage)
     tok = a.reshape(C, H * Wd).T                       # (T, C)
     q = store(linear(tok, W_("wq"), W_("bq")), storage)
@@ -411,7 +438,7 @@ def attn_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float, h
 
 def unet_mini_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float,
                    mode: int, storage: str, trace: Optional[Dict] = None,
-                   final_storage: Optional[str] = None):
+                   final_storage: Optional[str] = None, gn_stats: int = GN_STATS_CORRECTED):
     """conv_in -> ResBlock(320) -> down -> ResBlock(320->640) -> Attn(640, 10 heads)
     -> down -> ResBlock(640->1280) -> Attn(1280, 20 heads)   (reading R6/R7).
 
@@ -429,20 +456,25 @@ def unet_mini_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: flo
         return store(y, storage)
 
     h = conv_layer("conv_in", x, "conv_in_w", "conv_in_b", 1)
-    h = resblock_step(sub("rb1"), h, wts, P, G, eps, w, mode, storage, trace, "rb1.")
+    h = resblock_step(sub("rb1"), h, wts, P, G, eps, w, mode, storage, trace, "rb1.",
+                      gn_stats=gn_stats)
     h = conv_layer("down1", h, "down1_w", "down1_b", 2)
-    h = resblock_step(sub("rb2"), h, wts, P, G, eps, w, mode, storage, trace, "rb2.")
-    h = attn_step(sub("at2"), h, wts, P, G, eps, w, 10, mode, storage, trace, "at2.")
+    h = resblock_step(sub("rb2"), h, wts, P, G, eps, w, mode, storage, trace, "rb2.",
+                      gn_stats=gn_stats)
+    h = attn_step(sub("at2"), h, wts, P, G, eps, w, 10, mode, storage, trace, "at2.",
+                  gn_stats=gn_stats)
     h = conv_layer("down2", h, "down2_w", "down2_b", 2)
-    h = resblock_step(sub("rb3"), h, wts, P, G, eps, w, mode, storage, trace, "rb3.")
+    h = resblock_step(sub("rb3"), h, wts, P, G, eps, w, mode, storage, trace, "rb3.",
+                      gn_stats=gn_stats)
     h = attn_step(sub("at3"), h, wts, P, G, eps, w, 20, mode, storage, trace, "at3.",
-                  final_storage)
+                  final_storage, gn_stats=gn_stats)
     return h
 
 
 def block_step(kind: str, state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float,
                mode: int, storage: str, heads: int = 0, silu: bool = True,
-               trace: Optional[Dict] = None, final_storage: Optional[str] = None):
+               trace: Optional[Dict] = None, final_storage: Optional[str] = None,
+               gn_stats: int = GN_STATS_CORRECTED):
     """Dispatch one block step by kind; x is (C, H, W) (a leading batch of 1 is dropped).
 
     ``final_storage`` (default: ``storage``) is the rounding of the block's
@@ -453,13 +485,14 @@ def block_step(kind: str, state: Dict, x, wts: Dict, P: int, G: int, eps: float,
         x = x[0]
     if kind == "gn_conv":
         return gn_conv_step(state, x, wts, P, G, eps, w, silu, mode, storage, trace,
-                            final_storage)
+                            final_storage, gn_stats)
     if kind == "resblock":
         return resblock_step(state, x, wts, P, G, eps, w, mode, storage, trace,
-                             final_storage=final_storage)
+                             final_storage=final_storage, gn_stats=gn_stats)
     if kind == "attn":
         return attn_step(state, x, wts, P, G, eps, w, heads, mode, storage, trace,
-                         final_storage=final_storage)
+                         final_storage=final_storage, gn_stats=gn_stats)
     if kind == "unet_mini":
-        return unet_mini_step(state, x, wts, P, G, eps, w, mode, storage, trace, final_storage)
+        return unet_mini_step(state, x, wts, P, G, eps, w, mode, storage, trace, final_storage,
+                              gn_stats)
     raise ValueError(kind)

@@ -159,3 +159,25 @@ def test_kernel_calls_reject_bad_arguments_on_the_host(B):
 def test_groupnorm_workspace_size(B):
     assert B.dp_groupnorm_workspace_size(128, 128, 320, 32, 4) >= 256 + 4 * 32 * 2 * 8
     assert B.dp_groupnorm_workspace_size(128, 128, 320, 32, 0) == 0
+
+
+def test_gn_stats_variants_on_the_host(B):
+    """GroupNorm statistics variants of displaced steps: the default is the corrected statistics;
+    the exact variant needs the whole image, so its GroupNorms take the grid-wide pass even in a
+    displaced step; unknown variants are refused before any launch."""
+    kinds = lambda d, m: [B.dp_block_launch_info(d, m, i)[0] for i in range(B.dp_block_launch_count(d))]
+    d = B.dp_block_desc_init(B.RESBLOCK, 128, 128, 320, 320, 32, 4, 0, B.BF16, 1, 1e-5, 1.0)
+    assert d.gn_stats == B.GN_STATS_CORRECTED
+    B.dp_block_desc_set_gn_stats(d, B.GN_STATS_SYNC)
+    assert kinds(d, B.DISPLACED) == ["gn_fused", "conv", "gn_fused", "conv"]
+    for v in (B.GN_STATS_LOCAL, B.GN_STATS_STALE, B.GN_STATS_CORRECTED):
+        B.dp_block_desc_set_gn_stats(d, v)
+        assert kinds(d, B.DISPLACED) == ["gn_cluster", "conv", "gn_cluster", "conv"]
+    with pytest.raises(B.DPError):
+        B.dp_block_desc_set_gn_stats(d, 4)
+    with pytest.raises(B.DPError):
+        B.dp_block_desc_set_gn_stats(d, -1)
+    d.gn_stats = 7                      # a descriptor edited by hand is checked too
+    with pytest.raises(B.DPError, match="statistics variant"):
+        B.dp_block_workspace_size(d)
+    assert B.lib().dp_block_desc_set_gn_stats(None, 0) == -1

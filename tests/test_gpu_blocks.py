@@ -20,16 +20,18 @@ pytestmark = pytest.mark.gpu
 KIND = {"gn_conv": B.GN_CONV, "resblock": B.RESBLOCK, "attn": B.ATTN, "unet_mini": B.UNET_MINI}
 
 
-def make_block(wl):
+def make_block(wl, gn_stats=B.GN_STATS_CORRECTED):
     return B.Block(KIND[wl.kind], wl.H, wl.W, wl.C, wl.cout, wl.G, wl.P, wl.heads,
-                   B.BF16 if wl.dtype == "bf16" else B.FP32, wl.silu, wl.eps, 1.0)
+                   B.BF16 if wl.dtype == "bf16" else B.FP32, wl.silu, wl.eps, 1.0,
+                   gn_stats=gn_stats)
 
 
-def run_chain(wl, modes, random_affine, storage_rel=0.0, rl2=RL2, scale_rel=0.0):
+def run_chain(wl, modes, random_affine, storage_rel=0.0, rl2=RL2, scale_rel=0.0,
+              gn_stats=B.GN_STATS_CORRECTED):
     wts = synth.make_weights(wl, random_affine=random_affine)
     tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
     dev_w = block_weights(wl.kind, wts, tdt)
-    blk = make_block(wl)
+    blk = make_block(wl, gn_stats)
     xs = synth.InputStream(wl)
     st = {}
     for k, mode in enumerate(modes):
@@ -40,7 +42,7 @@ def run_chain(wl, modes, random_affine, storage_rel=0.0, rl2=RL2, scale_rel=0.0)
         blk.step(xd, out, dev_w, mode)
         ref = O.block_step(wl.kind, st, x, {n: v.double().numpy() for n, v in wts.items()}, wl.P,
                            wl.G, wl.eps, 1.0, mode, wl.dtype, heads=wl.heads, silu=wl.silu,
-                           final_storage="none")
+                           final_storage="none", gn_stats=gn_stats)
         torch.cuda.synchronize()
         check(host_img(out), ref, what=f"{wl.name} step {k} mode {mode}", storage_rel=storage_rel,
               rl2=rl2, scale_rel=scale_rel)
@@ -67,6 +69,21 @@ def test_resblock_channel_change():
     wl = synth.Workload(name="resblock_320to640x64x64", kind="resblock", C=320, Cout=640, H=64, W=64,
                         P=4)
     run_chain(wl, [B.SYNC, B.DISPLACED], True, storage_rel=BF16_HALF_ULP, scale_rel=2.0 ** -7)
+
+
+@pytest.mark.parametrize("gn_stats", [B.GN_STATS_LOCAL, B.GN_STATS_STALE, B.GN_STATS_SYNC],
+                         ids=["local", "stale", "sync"])
+@pytest.mark.parametrize("kind", ["resblock", "attn"])
+def test_gn_statistics_variants(kind, gn_stats):
+    """The GroupNorm ablation variants of displaced steps (band-local, stale-only and exact
+    statistics; halos and keys/values stale in all of them), against the oracle."""
+    if kind == "resblock":
+        wl = synth.Workload(name="resblock_320x64x64", kind="resblock", C=320, H=64, W=64, P=4)
+    else:
+        wl = synth.Workload(name="attn_640x32x32", kind="attn", C=640, H=32, W=32, P=4, heads=10,
+                            silu=False)
+    run_chain(wl, [B.SYNC, B.DISPLACED, B.DISPLACED], True, storage_rel=BF16_HALF_ULP,
+              gn_stats=gn_stats)
 
 
 def test_attn_640x64x64():

@@ -474,3 +474,100 @@ def test_conv_rows_matches_whole_image(mode, stride):
     rows = list(range(full.shape[1]))
     np.testing.assert_allclose(O.conv3x3_halo_rows(af, ast, wt, b, P, mode, rows, stride), full,
                                rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- GroupNorm ablation variants
+def _two_step_gn_used(kind, x0, x1, w, P, G, gn_stats, heads=0):
+    """GroupNorm statistics of a displaced step after a sync step, per variant."""
+    st = {}
+    O.block_step(kind, st, x0, w, P, G, 1e-5, 1.0, SYNC, "none", heads=heads)
+    tr = {}
+    y = O.block_step(kind, st, x1, w, P, G, 1e-5, 1.0, DISPLACED, "none", heads=heads, trace=tr,
+                     gn_stats=gn_stats)
+    return y, tr
+
+
+def _library_moments(x, P, G, bands):
+    """(mean, var) per (band, group): over the whole image (bands=False) or each band's rows."""
+    C, H, W = x.shape
+    hb, cg = H // P, C // G
+    out = np.empty((P, G, 2))
+    for p in range(P):
+        for g in range(G):
+            v = T64(x[g * cg:(g + 1) * cg, p * hb:(p + 1) * hb, :] if bands else x[g * cg:(g + 1) * cg])
+            out[p, g] = (v.mean().item(), v.var(unbiased=False).item())
+    return out
+
+
+def test_gn_variant_sync_uses_exact_whole_image_moments():
+    """The synchronous variant normalises a displaced step with this step's exact moments: its
+    GroupNorm output is the library's full-image GroupNorm, while the halos stay stale."""
+    r = rng(70)
+    C, H, W, P, G = 8, 8, 5, 4, 4
+    w = rand_gn_conv_weights(r, C, C)
+    x0 = r.standard_normal((C, H, W))
+    x1 = x0 + 0.3 * r.standard_normal((C, H, W))
+    _, tr = _two_step_gn_used("gn_conv", x0, x1, w, P, G, O.GN_STATS_SYNC)
+    np.testing.assert_allclose(tr["gn.used"], _library_moments(x1, P, G, bands=False), rtol=0, atol=1e-12)
+    a = F.silu(F.group_norm(T64(x1)[None], G, T64(w["gn_gamma"]), T64(w["gn_beta"]), 1e-5))[0].numpy()
+    np.testing.assert_allclose(tr["a"], a, rtol=0, atol=1e-12)
+
+
+def test_gn_variant_local_uses_each_bands_own_moments():
+    """The band-local variant normalises each band with its own rows' moments (the library's
+    GroupNorm of the band crop)."""
+    r = rng(71)
+    C, H, W, P, G = 8, 8, 5, 4, 4
+    w = rand_gn_conv_weights(r, C, C)
+    x0 = r.standard_normal((C, H, W))
+    x1 = x0 + 0.3 * r.standard_normal((C, H, W))
+    _, tr = _two_step_gn_used("gn_conv", x0, x1, w, P, G, O.GN_STATS_LOCAL)
+    np.testing.assert_allclose(tr["gn.used"], _library_moments(x1, P, G, bands=True), rtol=0, atol=1e-12)
+    hb = H // P
+    for p in range(P):
+        crop = x1[:, p * hb:(p + 1) * hb, :]
+        a = F.silu(F.group_norm(T64(crop)[None], G, T64(w["gn_gamma"]), T64(w["gn_beta"]), 1e-5))[0].numpy()
+        np.testing.assert_allclose(tr["a"][:, p * hb:(p + 1) * hb, :], a, rtol=0, atol=1e-12)
+
+
+def test_gn_variant_stale_uses_previous_steps_moments():
+    """The stale-only variant normalises with the previous step's whole-image moments, whatever
+    this step's input is."""
+    r = rng(72)
+    C, H, W, P, G = 8, 8, 5, 4, 4
+    w = rand_res_weights(r, C, C)
+    x0 = r.standard_normal((C, H, W))
+    x1 = 1.5 * x0 + 0.7 + 0.3 * r.standard_normal((C, H, W))
+    _, tr = _two_step_gn_used("resblock", x0, x1, w, P, G, O.GN_STATS_STALE)
+    np.testing.assert_allclose(tr["gn1.used"], _library_moments(x0, P, G, bands=False), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("variant", [O.GN_STATS_CORRECTED, O.GN_STATS_LOCAL, O.GN_STATS_STALE,
+                                     O.GN_STATS_SYNC])
+def test_gn_variants_agree_when_nothing_changes_and_p1(variant):
+    """With one band and an unchanged input every variant is the library's block; the variants
+    differ from each other once the input drifts."""
+    r = rng(73)
+    C, H, W, G = 8, 6, 5, 4
+    w = rand_res_weights(r, C, C)
+    x = r.standard_normal((C, H, W))
+    y, _ = _two_step_gn_used("resblock", x, x, w, 1, G, variant)
+    np.testing.assert_allclose(y, lib_resblock(x, w, G, 1e-5), rtol=0, atol=1e-11)
+
+
+def test_gn_variants_differ_under_drift():
+    r = rng(74)
+    C, H, W, P, G = 8, 8, 5, 4, 4
+    w = rand_res_weights(r, C, C)
+    x0 = r.standard_normal((C, H, W))
+    x1 = x0 + 0.4 * r.standard_normal((C, H, W)) + 0.2
+    ys = [_two_step_gn_used("resblock", x0, x1, w, P, G, v)[0]
+          for v in (O.GN_STATS_CORRECTED, O.GN_STATS_LOCAL, O.GN_STATS_STALE, O.GN_STATS_SYNC)]
+    for i in range(4):
+        for j in range(i + 1, 4):
+            assert np.linalg.norm(ys[i] - ys[j]) / np.linalg.norm(ys[j]) > 1e-4, (i, j)
+    # sync and naive-step modes ignore the variant
+    st = {}
+    a = O.block_step("resblock", st, x0, w, P, G, 1e-5, 1.0, NAIVE, "none", gn_stats=O.GN_STATS_STALE)
+    b = O.block_step("resblock", {}, x0, w, P, G, 1e-5, 1.0, NAIVE, "none")
+    np.testing.assert_array_equal(a, b)
