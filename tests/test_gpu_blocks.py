@@ -86,6 +86,30 @@ def test_gn_statistics_variants(kind, gn_stats):
               gn_stats=gn_stats)
 
 
+@pytest.mark.parametrize("kind", ["resblock", "attn"])
+def test_one_band(kind):
+    """With one band no context is stale: against the oracle, and a displaced step of an
+    unchanged input gives the synchronous step's output (to bf16 storage of the output)."""
+    if kind == "resblock":
+        wl = synth.Workload(name="resblock_320x32x32_p1", kind="resblock", C=320, H=32, W=32, P=1)
+    else:
+        wl = synth.Workload(name="attn_640x32x32_p1", kind="attn", C=640, H=32, W=32, P=1, heads=10,
+                            silu=False)
+    run_chain(wl, [B.SYNC, B.DISPLACED, B.DISPLACED], True, storage_rel=BF16_HALF_ULP)
+    wts = synth.make_weights(wl, random_affine=True)
+    dev_w = block_weights(wl.kind, wts, torch.bfloat16)
+    x = dev_img(synth.InputStream(wl).x(0)[0].double().numpy(), "bf16")
+    outs = []
+    for modes in ([B.SYNC], [B.SYNC, B.DISPLACED]):
+        blk = make_block(wl)
+        out = torch.empty(wl.H, wl.W, wl.cout, dtype=torch.bfloat16, device="cuda")
+        for m in modes:
+            blk.step(x, out, dev_w, m)
+        outs.append(host_img(out))
+    torch.cuda.synchronize()
+    check(outs[1], outs[0], what=f"{wl.name} displaced vs sync", storage_rel=2 * BF16_HALF_ULP)
+
+
 def test_attn_640x64x64():
     wl = synth.WORKLOADS["attn_640x64x64"]
     run_chain(wl, [B.SYNC, B.DISPLACED], True)

@@ -32,6 +32,7 @@ GN_CASES = [
     (1280, 8, 8, 2, 32, "bf16", True),
     (320, 256, 240, 4, 32, "bf16", True),    # too big for shared memory: two-pass kernels
     (64, 512, 384, 8, 32, "fp32", False),    # two-pass, fp32
+    (320, 32, 32, 1, 32, "bf16", True),      # one band: displaced == sync
 ]
 
 
@@ -149,6 +150,8 @@ CONV_CASES = [
     (320, 160, 6, 240, 3, 1, "bf16", False),    # halo-row pair kernel, 256x160, ragged row
     (64, 64, 16, 16, 2, 1, "fp32", False),
     (64, 128, 8, 10, 2, 1, "fp32", True),
+    (320, 320, 32, 48, 1, 1, "bf16", True),     # one band: no halo from other bands
+    (64, 64, 16, 16, 1, 2, "bf16", False),      # one band, stride 2
 ]
 
 
@@ -274,7 +277,8 @@ def test_linear_parity(M, N, K, split, use_res):
 
 # ---------------------------------------------------------------- attention
 @pytest.mark.parametrize("T,heads,P,qscale", [(512, 2, 2, 1.0), (512, 2, 4, 3.0), (1024, 3, 2, 1.0),
-                                              (1536, 5, 2, 2.0), (2048, 4, 16, 1.0), (4096, 10, 4, 1.0)])
+                                              (1536, 5, 2, 2.0), (2048, 4, 16, 1.0), (4096, 10, 4, 1.0),
+                                              (512, 3, 1, 1.0), (384, 2, 1, 2.0)])
 @pytest.mark.parametrize("mode", MODES)
 @pytest.mark.parametrize("split", [True, False], ids=["split", "whole_tiles"])
 def test_attention_parity(T, heads, P, qscale, mode, split):
