@@ -63,6 +63,7 @@ _SIGS = {
     "dp_attn_workspace_size": ([], _SZ),
     "dp_attn_stale_kv": ([_V, _V, _V, _V, _V, _V, _I, _I, _I, _I, _F, _I, _V, _SZ, _V], _I),
     "dp_refresh_stale": ([_V, _V, _SZ, _I, _I, _I, _V], _I),
+    "dp_refresh_halo": ([_V, _V, _SZ, _I, _I, _I, _I, _V], _I),
     "dp_refresh_stats": ([_V, _V, _V, _I, _I, _V], _I),
     "dp_block_desc_init": ([ctypes.POINTER(BlockDesc), _I, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _F], _I),
     "dp_block_desc_set_gn_stats": ([ctypes.POINTER(BlockDesc), _I], _I),
@@ -201,6 +202,11 @@ def dp_attn_stale_kv(q, k_fresh, v_fresh, k_stale, v_stale, o, T, heads, head_di
 def dp_refresh_stale(fresh, stale, row_bytes, rows, P, band=-1, stream=None):
     return _check(lib().dp_refresh_stale(_p(fresh), _p(stale), row_bytes, rows, P, band,
                                          _s(stream)))
+
+
+def dp_refresh_halo(fresh, stale, row_bytes, rows, P, above, below, stream=None):
+    return _check(lib().dp_refresh_halo(_p(fresh), _p(stale), row_bytes, rows, P, above, below,
+                                        _s(stream)))
 
 
 def dp_refresh_stats(fresh_local, stale_local, stale_global, P, G, stream=None):

@@ -30,6 +30,20 @@ __global__ void __launch_bounds__(256) copy16_kernel(const uint4* __restrict__ s
   for (; i < n16; i += stride) dst[i] = __ldcs(src + i);
 }
 
+// Halo refresh: edge e (between bands e and e+1) owns the contiguous rows
+// [(e+1) hb - above, (e+1) hb + below); blockIdx.y is the edge, the x blocks
+// stride over that range's 16-byte vectors.
+__global__ void __launch_bounds__(256) halo_copy_kernel(const uint4* __restrict__ src,
+                                                        uint4* __restrict__ dst, size_t edge0_16,
+                                                        size_t band16, size_t range16) {
+  griddep_wait();
+  griddep_trigger();
+  const size_t base = edge0_16 + static_cast<size_t>(blockIdx.y) * band16;
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < range16;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    dst[base + i] = __ldcs(src + base + i);
+}
+
 __global__ void refresh_stats_kernel(const float* __restrict__ fresh_local,
                                      float* __restrict__ stale_local,
                                      float* __restrict__ stale_global, int P, int G) {
@@ -75,6 +89,36 @@ int dp_refresh_stale(const void* fresh, void* stale, size_t row_bytes, int rows,
   if ((f < s + total) && (s < f + total))
     return dp::set_error(DP_ERR_INVALID_ARG, "refresh: fresh and stale overlap");
   return dp::copy_launch(f, s, total, static_cast<cudaStream_t>(stream));
+}
+
+int dp_refresh_halo(const void* fresh, void* stale, size_t row_bytes, int rows, int P, int above,
+                    int below, void* stream) {
+  if (!fresh || !stale) return dp::set_error(DP_ERR_INVALID_ARG, "refresh_halo: null buffer");
+  if (rows < 0 || P <= 0 || above < 0 || below < 0)
+    return dp::set_error(DP_ERR_INVALID_ARG, "refresh_halo: bad rows/P/above/below");
+  if (rows % P) return dp::set_error(DP_ERR_UNSUPPORTED, "refresh_halo: rows %% P != 0");
+  const int hb = rows / P;
+  if (above > hb || below > hb)
+    return dp::set_error(DP_ERR_INVALID_ARG, "refresh_halo: halo deeper than a band (%d rows)", hb);
+  if (row_bytes % 16 || !dp::aligned16(fresh) || !dp::aligned16(stale))
+    return dp::set_error(DP_ERR_UNSUPPORTED, "refresh_halo: rows and pointers must be 16-byte aligned");
+  const size_t total = row_bytes * static_cast<size_t>(rows);
+  const char* f = static_cast<const char*>(fresh);
+  char* s = static_cast<char*>(stale);
+  if ((f < s + total) && (s < f + total))
+    return dp::set_error(DP_ERR_INVALID_ARG, "refresh_halo: fresh and stale overlap");
+  if (P == 1 || above + below == 0 || row_bytes == 0) return DP_OK;   // no band edge to refresh
+  const size_t row16 = row_bytes / 16;
+  const size_t range16 = static_cast<size_t>(above + below) * row16;
+  const size_t edge0_16 = (static_cast<size_t>(hb) - above) * row16;
+  size_t bx = (range16 + 255) / 256;   // about one vector per thread
+  if (bx > 1024) bx = 1024;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  dp::mark_launch(st);
+  return dp::launch_kernel(dp::halo_copy_kernel, dim3(static_cast<unsigned>(bx), P - 1), dim3(256), 0,
+                           st, false, "refresh_halo launch", static_cast<const uint4*>(fresh),
+                           static_cast<uint4*>(stale), edge0_16, static_cast<size_t>(hb) * row16,
+                           range16);
 }
 
 int dp_refresh_stats(const float* fresh_local, float* stale_local, float* stale_global, int P,

@@ -274,6 +274,22 @@ DP_API int dp_attn_stale_kv(const void* q, const void* k_fresh, const void* v_fr
 DP_API int dp_refresh_stale(const void* fresh, void* stale, size_t row_bytes, int rows, int P,
                      int band, void* stream);
 
+/*
+ * Halo-only refresh.  A 3x3 conv reads other bands only at band edges: band p
+ * takes the `above` rows just above its first row (the end of band p-1) and
+ * the `below` rows just below its last row (the start of band p+1) from the
+ * stale buffer.  For a layer whose stale buffer feeds only such a conv, this
+ * copies just those rows, [(e+1) hb - above, (e+1) hb + below) for every
+ * band edge e (hb = rows/P), from `fresh` to `stale`; the other rows of
+ * `stale` are left as they are.  A stride-1 3x3 conv needs above = below = 1;
+ * a stride-2 one with even band heights needs above = 1, below = 0.
+ * Same buffer rules as dp_refresh_stale; above, below <= rows/P.  The pages
+ * have no counterpart beyond the AllGather it replaces (atlas.scime.ai
+ * summary, Approach): that gather sends whole patches.
+ */
+DP_API int dp_refresh_halo(const void* fresh, void* stale, size_t row_bytes, int rows, int P,
+                    int above, int below, void* stream);
+
 /* Statistics refresh: stale_local = fresh_local; stale_global[g] = mean over
  * bands of fresh_local[p][g].  All [.][2] fp32 device arrays. */
 DP_API int dp_refresh_stats(const float* fresh_local, float* stale_local, float* stale_global,

@@ -181,3 +181,19 @@ def test_gn_stats_variants_on_the_host(B):
     with pytest.raises(B.DPError, match="statistics variant"):
         B.dp_block_workspace_size(d)
     assert B.lib().dp_block_desc_set_gn_stats(None, 0) == -1
+
+
+def test_refresh_halo_rejects_bad_arguments_on_the_host(B):
+    with pytest.raises(B.DPError) as e:   # halo deeper than a band
+        B.dp_refresh_halo(16, 4096, 64, 8, 4, 3, 0, stream=0)
+    assert e.value.code == B.DP_ERR_INVALID_ARG
+    with pytest.raises(B.DPError) as e:   # rows not a multiple of P
+        B.dp_refresh_halo(16, 4096, 64, 9, 4, 1, 1, stream=0)
+    assert e.value.code == B.DP_ERR_UNSUPPORTED
+    with pytest.raises(B.DPError) as e:   # overlapping buffers
+        B.dp_refresh_halo(16, 32, 64, 8, 4, 1, 1, stream=0)
+    assert e.value.code == B.DP_ERR_INVALID_ARG
+    with pytest.raises(B.DPError) as e:   # row bytes not a multiple of 16
+        B.dp_refresh_halo(16, 4096, 40, 8, 4, 1, 1, stream=0)
+    assert e.value.code == B.DP_ERR_UNSUPPORTED
+    assert B.dp_refresh_halo(16, 4096, 64, 8, 1, 1, 1, stream=0) == B.DP_OK   # one band: nothing to do

@@ -320,6 +320,47 @@ def test_refresh_is_an_exact_copy():
     assert torch.equal(stale, fresh)
 
 
+@pytest.mark.parametrize("H,W,C,P,above,below", [(480, 480, 320, 8, 1, 1), (128, 128, 320, 4, 1, 0),
+                                                  (12, 8, 64, 3, 2, 3), (16, 8, 64, 1, 1, 1),
+                                                  (16, 8, 64, 4, 4, 4)])
+def test_refresh_halo_copies_exactly_the_band_edge_rows(H, W, C, P, above, below):
+    g = torch.Generator(device="cpu").manual_seed(4)
+    fresh = torch.randint(-2 ** 15, 2 ** 15, (H, W, C), generator=g, dtype=torch.int16).cuda()
+    stale = torch.randint(-2 ** 15, 2 ** 15, (H, W, C), generator=g, dtype=torch.int16).cuda()
+    want = stale.clone()
+    hb = H // P
+    for e in range(P - 1):
+        r0, r1 = (e + 1) * hb - above, (e + 1) * hb + below
+        want[r0:r1] = fresh[r0:r1]
+    B.dp_refresh_halo(fresh, stale, W * C * 2, H, P, above, below)
+    torch.cuda.synchronize()
+    assert torch.equal(stale, want)
+
+
+@pytest.mark.parametrize("stride", [1, 2])
+def test_halo_refresh_is_all_a_displaced_conv_reads(stride):
+    """A displaced conv gives the same bits whether its stale buffer was refreshed whole or only
+    at the band-edge rows it reads (1 above and 1 below for stride 1, 1 above for stride 2)."""
+    r = rng(77 + stride)
+    H, W, C, P = 64, 48, 128, 4
+    prev = torch.from_numpy(r.standard_normal((H, W, C)).astype(np.float32)).to(torch.bfloat16).cuda()
+    cur = torch.from_numpy(r.standard_normal((H, W, C)).astype(np.float32)).to(torch.bfloat16).cuda()
+    wt = torch.from_numpy(0.05 * r.standard_normal((C, 3, 3, C)).astype(np.float32)).to(torch.bfloat16).cuda()
+    b = torch.zeros(C, device="cuda")
+    full = prev.clone()
+    halo = torch.from_numpy(r.standard_normal((H, W, C)).astype(np.float32)).to(torch.bfloat16).cuda()
+    B.dp_refresh_stale(prev, full, W * C * 2, H, P, -1)
+    B.dp_refresh_halo(prev, halo, W * C * 2, H, P, 1, 1 if stride == 1 else 0)
+    Ho, Wo = (H - 1) // stride + 1, (W - 1) // stride + 1
+    o_full = torch.empty(Ho, Wo, C, dtype=torch.bfloat16, device="cuda")
+    o_halo = torch.empty_like(o_full)
+    B.dp_conv3x3_halo(cur, full, wt, b, None, o_full, H, W, C, C, stride, P, B.DISPLACED, B.BF16)
+    B.dp_conv3x3_halo(cur, halo, wt, b, None, o_halo, H, W, C, C, stride, P, B.DISPLACED, B.BF16)
+    torch.cuda.synchronize()
+    assert torch.equal(o_full, o_halo)
+    assert not torch.equal(full, halo)   # the interiors really differ
+
+
 def test_refresh_stats():
     P, G = 4, 32
     f = torch.randn(P * G * 2, device="cuda")
