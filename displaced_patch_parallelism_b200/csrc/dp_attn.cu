@@ -38,18 +38,22 @@ namespace dp {
 struct AttnParams {
   CUtensorMap tmQ, tmKf, tmVf, tmKs, tmVs;
   int T, heads, P, tb, mode;
-  // Work split: a unit is 128 queries of one head (units ordered head-major);
-  // it takes n_kv key tiles.  CTA b owns the iterations [b L, (b+1) L) of the
-  // W = units x n_kv (unit, key tile) iterations.
+  // Work split: a unit is 128 queries of one head (256 in the two-tile
+  // kernel; units ordered head-major, n_qt units per head); it takes n_kv key
+  // tiles.  CTA b owns the iterations [b L, (b+1) L) of the W = units x n_kv
+  // (unit, key tile) iterations.
   int n_qt, n_kv, W, L;
   float scale_log2;
   __nv_bfloat16* o;
   int ld;
   // Partials of units cut between CTAs: slot 2b + 1 holds CTA b's last
-  // segment when it is a unit's start, slot 2b its first segment otherwise;
-  // each slot is 8 warp slices of 32 rows x (32 O columns, m, l, 2 pad).
+  // segment when it is a unit's start, slot 2b its first segment otherwise.
+  // One-tile kernel: each slot is 8 warp slices of 32 rows x (32 O columns,
+  // m, l, 2 pad); two-tile kernel: 16 lane-contiguous warp slices (see
+  // kPairSliceFloats).
   float* part;
-  unsigned* count;          // [grid][8]: parts of the unit starting in CTA b done so far
+  unsigned* count;          // per CTA 8 (one-tile) or 16 (two-tile) counters: parts of the unit
+                            // starting in that CTA done so far
   int* status;
 };
 
