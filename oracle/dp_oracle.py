@@ -31,14 +31,18 @@ Readings of what the pages leave open (each also listed in the design notes):
       ``unet_mini_step``
   R7  every 3x3 conv, stride 1 or 2, pads by one and takes halo rows from
       other bands per mode; stride-2 output bands are Ho/P rows
+  R12 the GroupNorm ablation's alternatives for displaced steps (band-local,
+      stale-only and exact statistics): see ``gn_variant_mode``
 
 Parity pins (the tests under tests/test_oracle_*.py): P = 1 reduces to the
 library full-image block (torch group_norm / conv2d / softmax attention);
 brute-force loops on tiny inputs; naive mode equals independent crops; an
 unchanged input makes displaced equal sync; a uniform drift makes the
 corrected statistics exact; halo and attention locality; zero warm-up differs
-from sync.  ``unet_mini_step`` is pinned only through its parts and the P = 1
-reduction of the whole chain.
+from sync; the GroupNorm variants equal the library GroupNorm of the whole
+image, of each band's crop and of the previous step's image.
+``unet_mini_step`` is pinned only through its parts and the P = 1 reduction of
+the whole chain.
 """
 from __future__ import annotations
 
