@@ -197,3 +197,42 @@ def test_refresh_halo_rejects_bad_arguments_on_the_host(B):
         B.dp_refresh_halo(16, 4096, 40, 8, 4, 1, 1, stream=0)
     assert e.value.code == B.DP_ERR_UNSUPPORTED
     assert B.dp_refresh_halo(16, 4096, 64, 8, 1, 1, 1, stream=0) == B.DP_OK   # one band: nothing to do
+
+
+def test_plain_c_caller(B, tmp_path):
+    """The header is plain C99, and a C program links against libdp and uses the host-side
+    calls (descriptor set-up, validation, the step-mode helper) with no Python in between."""
+    import shutil
+    import subprocess
+    if not shutil.which("gcc"):
+        pytest.skip("no C compiler")
+    src = tmp_path / "caller.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include <string.h>
+#include "dp.h"
+int main(void) {
+  dp_block_desc d;
+  if (dp_block_desc_init(&d, DP_BLOCK_RESBLOCK, 128, 128, 320, 320, 32, 4, 0, DP_BF16, 1,
+                         1e-5f, 1.0f) != DP_OK) return 1;
+  if (d.gn_stats != DP_GN_STATS_CORRECTED) return 2;
+  if (dp_block_desc_set_gn_stats(&d, DP_GN_STATS_SYNC) != DP_OK) return 3;
+  if (dp_block_desc_set_gn_stats(&d, 9) != DP_ERR_INVALID_ARG) return 4;
+  if (strstr(dp_last_error(), "variant") == NULL) return 5;
+  if (dp_block_workspace_size(&d) == 0) return 6;
+  if (dp_mode_for_step(0, 0) != DP_MODE_NAIVE || dp_mode_for_step(3, 4) != DP_MODE_SYNC ||
+      dp_mode_for_step(4, 4) != DP_MODE_DISPLACED) return 7;
+  if (dp_block_desc_init(&d, DP_BLOCK_RESBLOCK, 130, 128, 320, 320, 32, 4, 0, DP_BF16, 1,
+                         1e-5f, 1.0f) != DP_ERR_UNSUPPORTED) return 8;
+  printf("%s\n", dp_version());
+  return 0;
+}
+''')
+    exe = tmp_path / "caller"
+    libdir = os.path.dirname(B.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                    "-I" + os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                    "-L" + libdir, "-l:libdp.so", "-Wl,-rpath," + libdir], check=True)
+    run = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert run.returncode == 0, (run.returncode, run.stdout, run.stderr)
+    assert run.stdout.strip()
