@@ -62,6 +62,7 @@ _SIGS = {
     "dp_linear": ([_V, _V, _V, _V, _V, _V, _V, _I, _I, _I, _I, _V, _SZ, _V], _I),
     "dp_attn_workspace_size": ([], _SZ),
     "dp_attn_stale_kv": ([_V, _V, _V, _V, _V, _V, _I, _I, _I, _I, _F, _I, _V, _SZ, _V], _I),
+    "dp_attn_cross": ([_V, _V, _V, _V, _I, _I, _I, _I, _F, _V, _SZ, _V], _I),
     "dp_refresh_stale": ([_V, _V, _SZ, _I, _I, _I, _V], _I),
     "dp_refresh_halo": ([_V, _V, _SZ, _I, _I, _I, _I, _V], _I),
     "dp_refresh_stats": ([_V, _V, _V, _I, _I, _V], _I),
@@ -197,6 +198,12 @@ def dp_attn_stale_kv(q, k_fresh, v_fresh, k_stale, v_stale, o, T, heads, head_di
     return _check(lib().dp_attn_stale_kv(_p(q), _p(k_fresh), _p(v_fresh), _p(k_stale),
                                          _p(v_stale), _p(o), T, heads, head_dim, P, scale, mode,
                                          _p(workspace), workspace_bytes, _s(stream)))
+
+
+def dp_attn_cross(q, k, v, o, Tq, Tk, heads, head_dim, scale, workspace=None, workspace_bytes=0,
+                  stream=None):
+    return _check(lib().dp_attn_cross(_p(q), _p(k), _p(v), _p(o), Tq, Tk, heads, head_dim, scale,
+                                      _p(workspace), workspace_bytes, _s(stream)))
 
 
 def dp_refresh_stale(fresh, stale, row_bytes, rows, P, band=-1, stream=None):

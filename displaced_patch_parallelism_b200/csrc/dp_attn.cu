@@ -43,6 +43,9 @@ struct AttnParams {
   // tiles.  CTA b owns the iterations [b L, (b+1) L) of the W = units x n_kv
   // (unit, key tile) iterations.
   int n_qt, n_kv, W, L;
+  // keys in the last key tile (128 unless the key count is ragged, as for
+  // cross-attention over a text context; the rest of that tile is masked)
+  int kv_last;
   float scale_log2;
   __nv_bfloat16* o;
   int ld;
@@ -793,6 +796,19 @@ __global__ void __launch_bounds__(kPairThreads, 1) attn_pair_kernel(const __grid
         tmem_ld16x256_x8(tS, sa);
         tmem_ld16x256_x8(tS + 64, sb);
         tmem_wait_ld();
+        // a ragged last key tile: its missing keys (zero rows from the
+        // tensor map's bounds) get score -inf, i.e. weight 0
+        const bool ragged = sg.k0 + jj == p.n_kv - 1 && p.kv_last < 128;
+        if (ragged) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int col = 8 * k + 2 * cq + (e & 1);
+              if (col >= p.kv_last) sa[4 * k + e] = 0xff800000u;
+              if (col + 64 >= p.kv_last) sb[4 * k + e] = 0xff800000u;
+            }
+        }
         float xa0 = fmaxf(__uint_as_float(sa[0]), __uint_as_float(sa[1]));
         float xa1 = fmaxf(__uint_as_float(sb[0]), __uint_as_float(sb[1]));
         float xb0 = fmaxf(__uint_as_float(sa[2]), __uint_as_float(sa[3]));
@@ -859,6 +875,13 @@ __global__ void __launch_bounds__(kPairThreads, 1) attn_pair_kernel(const __grid
         exps(sb, pk_hi);
         tmem_ld16x256_x8(tS, sa);
         tmem_wait_ld();
+        if (ragged) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (8 * k + 2 * cq + (e & 1) >= p.kv_last) sa[4 * k + e] = 0xff800000u;
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_free[tile]);   // S(j+1) may now be computed
@@ -1023,18 +1046,20 @@ size_t attn_workspace_bytes() {
   return attn_count_bytes(2 * sms) + (one > pair ? one : pair) * sizeof(float);
 }
 
-int attn_launch(const void* q, const void* kf, const void* vf, const void* ks, const void* vs,
-                void* o, int T, int heads, int P, float scale, int mode, void* workspace,
-                size_t workspace_bytes, cudaStream_t stream) {
+// Self-attention (Tk = T) or, with Tk != T, attention of T queries over Tk
+// keys that are all visible (mode SYNC, P = 1: cross-attention).
+static int attn_launch_tk(const void* q, const void* kf, const void* vf, const void* ks, const void* vs,
+                          void* o, int T, int Tk, int heads, int P, float scale, int mode,
+                          void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   AttnParams a;
   memset(&a, 0, sizeof(a));
   const int ld = heads * 64;
-  uint64_t dims[2] = {static_cast<uint64_t>(ld), static_cast<uint64_t>(T)};
   uint64_t str[1] = {static_cast<uint64_t>(ld) * 2};
   uint32_t box[2] = {64, 128};
   const void* ptrs[5] = {q, kf, vf, ks ? ks : kf, vs ? vs : vf};
   CUtensorMap* maps[5] = {&a.tmQ, &a.tmKf, &a.tmVf, &a.tmKs, &a.tmVs};
   for (int i = 0; i < 5; ++i) {
+    uint64_t dims[2] = {static_cast<uint64_t>(ld), static_cast<uint64_t>(i == 0 ? T : Tk)};
     int rc = encode_tmap(maps[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptrs[i]),
                          dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc) return rc;
@@ -1066,7 +1091,9 @@ int attn_launch(const void* q, const void* kf, const void* vf, const void* ks, c
     attr_mask |= 1 << (dev & 31);
   }
   a.n_qt = T / (pair ? 256 : 128);
-  a.n_kv = mode == DP_MODE_NAIVE ? a.tb / 128 : T / 128;
+  a.n_kv = mode == DP_MODE_NAIVE ? a.tb / 128 : (Tk + 127) / 128;
+  a.kv_last = Tk - (a.n_kv - 1) * 128;
+  if (mode == DP_MODE_NAIVE) a.kv_last = 128;
   const int units = a.n_qt * heads;
   a.W = units * a.n_kv;
   // Balanced split: every CTA takes an equal run of (unit, key tile)
@@ -1100,6 +1127,13 @@ int attn_launch(const void* q, const void* kf, const void* vf, const void* ks, c
                        "attention launch", a);
 }
 
+int attn_launch(const void* q, const void* kf, const void* vf, const void* ks, const void* vs,
+                void* o, int T, int heads, int P, float scale, int mode, void* workspace,
+                size_t workspace_bytes, cudaStream_t stream) {
+  return attn_launch_tk(q, kf, vf, ks, vs, o, T, T, heads, P, scale, mode, workspace,
+                        workspace_bytes, stream);
+}
+
 int attn_validate(const void* q, const void* kf, const void* vf, const void* ks, const void* vs,
                   const void* o, int T, int heads, int head_dim, int P, int mode) {
   if (!q || !kf || !vf || !o) return set_error(DP_ERR_INVALID_ARG, "attention: null pointer");
@@ -1123,6 +1157,25 @@ int attn_validate(const void* q, const void* kf, const void* vf, const void* ks,
 }  // namespace dp
 
 extern "C" size_t dp_attn_workspace_size(void) { return dp::attn_workspace_bytes(); }
+
+extern "C" int dp_attn_cross(const void* q, const void* k, const void* v, void* o, int Tq, int Tk,
+                             int heads, int head_dim, float scale, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !o) return dp::set_error(DP_ERR_INVALID_ARG, "cross-attention: null pointer");
+  if (Tq <= 0 || Tk <= 0 || heads <= 0) return dp::set_error(DP_ERR_INVALID_ARG, "cross-attention: bad size");
+  if (head_dim != 64) return dp::set_error(DP_ERR_UNSUPPORTED, "cross-attention: head_dim must be 64");
+  if (Tq % 256) return dp::set_error(DP_ERR_UNSUPPORTED, "cross-attention: Tq must be a multiple of 256");
+  const void* ins[3] = {q, k, v};
+  for (int i = 0; i < 3; ++i) {
+    if (!dp::aligned16(ins[i])) return dp::set_error(DP_ERR_UNSUPPORTED, "cross-attention: pointer not 16-byte aligned");
+    if (ins[i] == o) return dp::set_error(DP_ERR_INVALID_ARG, "cross-attention: o aliases an input");
+  }
+  if (!dp::aligned16(o)) return dp::set_error(DP_ERR_UNSUPPORTED, "cross-attention: o not 16-byte aligned");
+  if (workspace && !dp::aligned16(workspace))
+    return dp::set_error(DP_ERR_UNSUPPORTED, "cross-attention: workspace not 16-byte aligned");
+  return dp::attn_launch_tk(q, k, v, nullptr, nullptr, o, Tq, Tk, heads, 1, scale, DP_MODE_SYNC,
+                            workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
 
 extern "C" int dp_attn_stale_kv(const void* q, const void* k_fresh, const void* v_fresh,
                                 const void* k_stale, const void* v_stale, void* o, int T,

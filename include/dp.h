@@ -264,6 +264,24 @@ DP_API int dp_attn_stale_kv(const void* q, const void* k_fresh, const void* v_fr
                      size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Cross-attention: Tq queries attend over Tk keys and values that every band
+ * sees whole and fresh, as the text context of an SDXL transformer block
+ * (the keys and values come from the prompt, not from the image, so they are
+ * the same for every patch and need no stale copy).  The SDXL-shaped U-Net
+ * step with cross-attention is a "next" extension; the pages do not discuss
+ * it beyond naming SDXL as the model.
+ *
+ *  q  [Tq][heads*64] bf16, device;   k, v  [Tk][heads*64] bf16, device
+ *  o  [Tq][heads*64] bf16, device, written;   o[t] = softmax(q k^T scale) v per head
+ *  workspace: as for dp_attn_stale_kv (NULL: whole query tiles per CTA)
+ * Needs head_dim == 64 and Tq % 256 == 0; any Tk >= 1 (a ragged last key
+ * tile is masked).
+ * ---------------------------------------------------------------------- */
+DP_API int dp_attn_cross(const void* q, const void* k, const void* v, void* o, int Tq, int Tk,
+                  int heads, int head_dim, float scale, void* workspace, size_t workspace_bytes,
+                  void* stream);
+
+/* ------------------------------------------------------------------------
  * Stale-buffer refresh: the device-local replacement of the paper's
  * per-layer AllGather (atlas.scime.ai summary, Approach: AllGather overlaps
  * computation; limitations: NCCL kernels take SMs).  Copies the rows of band

@@ -298,6 +298,22 @@ def attention_stale_kv(q: np.ndarray, k_fresh: np.ndarray, v_fresh: np.ndarray,
     return o
 
 
+def attention_cross(q: np.ndarray, k: np.ndarray, v: np.ndarray, heads: int,
+                    scale: float) -> np.ndarray:
+    """Cross-attention over a context every band sees whole (an SDXL block's text keys and
+    values): per head, softmax(q K^T * scale) V.  q: (Tq, heads*d); k, v: (Tk, heads*d)."""
+    Tq, Cq = q.shape
+    d = Cq // heads
+    o = np.zeros((Tq, Cq))
+    for h in range(heads):
+        hs = slice(h * d, (h + 1) * d)
+        s = (q[:, hs] @ k[:, hs].T) * scale
+        s = s - s.max(axis=1, keepdims=True)
+        e = np.exp(s)
+        o[:, hs] = (e / e.sum(axis=1, keepdims=True)) @ v[:, hs]
+    return o
+
+
 def linear(x: np.ndarray, w: np.ndarray, b: Optional[np.ndarray]) -> np.ndarray:
     """x @ w.T + b with w stored (out, in)."""
     y = x @ w.T

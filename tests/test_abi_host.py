@@ -236,3 +236,18 @@ int main(void) {
     run = subprocess.run([str(exe)], capture_output=True, text=True)
     assert run.returncode == 0, (run.returncode, run.stdout, run.stderr)
     assert run.stdout.strip()
+
+
+def test_cross_attention_rejects_bad_arguments_on_the_host(B):
+    with pytest.raises(B.DPError) as e:   # query count not a multiple of 256
+        B.dp_attn_cross(16, 32, 48, 64, 300, 77, 2, 64, 0.125, stream=0)
+    assert e.value.code == B.DP_ERR_UNSUPPORTED
+    with pytest.raises(B.DPError) as e:   # head_dim 128
+        B.dp_attn_cross(16, 32, 48, 64, 256, 77, 2, 128, 0.125, stream=0)
+    assert e.value.code == B.DP_ERR_UNSUPPORTED
+    with pytest.raises(B.DPError) as e:   # output aliases the queries
+        B.dp_attn_cross(16, 32, 48, 16, 256, 77, 2, 64, 0.125, stream=0)
+    assert e.value.code == B.DP_ERR_INVALID_ARG
+    with pytest.raises(B.DPError) as e:
+        B.dp_attn_cross(None, 32, 48, 64, 256, 77, 2, 64, 0.125, stream=0)
+    assert e.value.code == B.DP_ERR_INVALID_ARG

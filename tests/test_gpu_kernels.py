@@ -304,6 +304,29 @@ def test_attention_parity(T, heads, P, qscale, mode, split):
     assert B.dp_device_status() == 0
 
 
+@pytest.mark.parametrize("Tq,Tk,heads", [(1024, 77, 10), (4096, 77, 10), (256, 128, 2), (512, 200, 4),
+                                          (256, 1, 2), (768, 300, 3)])
+@pytest.mark.parametrize("split", [True, False], ids=["split", "whole_tiles"])
+def test_cross_attention_parity(Tq, Tk, heads, split):
+    """Queries over a context of Tk keys every band sees whole (77 = an SDXL text context); a
+    ragged last key tile is masked."""
+    r = rng(Tq + Tk + heads)
+    C = heads * 64
+    q = rounded(r.standard_normal((Tq, C)), "bf16")
+    k, v = (rounded(r.standard_normal((Tk, C)), "bf16") for _ in range(2))
+    ref = O.attention_cross(q, k, v, heads, 0.125)
+    o = torch.empty(Tq, C, dtype=torch.bfloat16, device="cuda")
+    nws = B.dp_attn_workspace_size()
+    ws = torch.zeros(nws, dtype=torch.uint8, device="cuda") if split else None
+    for _ in range(2):   # the second call reuses the workspace's flags
+        o.zero_()
+        B.dp_attn_cross(dev_mat(q), dev_mat(k), dev_mat(v), o, Tq, Tk, heads, 64, 0.125, ws,
+                        nws if split else 0)
+        torch.cuda.synchronize()
+        check(host(o), ref, what=f"cross-attention Tq={Tq} Tk={Tk} split={split}")
+    assert B.dp_device_status() == 0
+
+
 # ---------------------------------------------------------------- refresh
 def test_refresh_is_an_exact_copy():
     g = torch.Generator(device="cpu").manual_seed(3)

@@ -571,3 +571,22 @@ def test_gn_variants_differ_under_drift():
     a = O.block_step("resblock", st, x0, w, P, G, 1e-5, 1.0, NAIVE, "none", gn_stats=O.GN_STATS_STALE)
     b = O.block_step("resblock", {}, x0, w, P, G, 1e-5, 1.0, NAIVE, "none")
     np.testing.assert_array_equal(a, b)
+
+
+# ---------------------------------------------------------------- cross-attention
+@pytest.mark.parametrize("Tq,Tk,heads", [(6, 5, 2), (8, 77, 3), (16, 1, 1)])
+def test_cross_attention_equals_library_and_brute_force(Tq, Tk, heads):
+    r = rng(80 + Tk)
+    d = 4
+    q, k, v = (r.standard_normal((T, heads * d)) for T in (Tq, Tk, Tk))
+    o = O.attention_cross(q, k, v, heads, 0.37)
+    sh = lambda z, T: T64(z).reshape(T, heads, d).permute(1, 0, 2)
+    ref = F.scaled_dot_product_attention(sh(q, Tq), sh(k, Tk), sh(v, Tk), scale=0.37)
+    np.testing.assert_allclose(o, ref.permute(1, 0, 2).reshape(Tq, heads * d).numpy(), rtol=0, atol=1e-12)
+    # brute force: one query, one head at a time
+    for t in range(Tq):
+        for h in range(heads):
+            w = [math.exp(0.37 * sum(q[t, h * d + i] * k[j, h * d + i] for i in range(d))) for j in range(Tk)]
+            z = sum(w)
+            for i in range(d):
+                assert abs(o[t, h * d + i] - sum(w[j] * v[j, h * d + i] for j in range(Tk)) / z) < 1e-10
