@@ -396,8 +396,13 @@ def gn_conv_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float
 
 def resblock_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float,
                   mode: int, storage: str, trace: Optional[Dict] = None, prefix: str = "",
-                  final_storage: Optional[str] = None, gn_stats: int = GN_STATS_CORRECTED):
-    """GN -> SiLU -> conv1 -> GN -> SiLU -> conv2 -> + x (or + 1x1 shortcut(x))."""
+                  final_storage: Optional[str] = None, gn_stats: int = GN_STATS_CORRECTED,
+                  temb: Optional[np.ndarray] = None):
+    """GN -> SiLU -> conv1 -> GN -> SiLU -> conv2 -> + x (or + 1x1 shortcut(x)).
+
+    With a time embedding ``temb`` (and weights temb_w (Cout, Ct), temb_b), conv1's output
+    gets the per-channel term temb_w silu(temb) + temb_b, as in an SDXL ResBlock (reading R13):
+    a step-dependent bias that is the same for every band."""
     x = _a(x)
     W_ = lambda n: _a(wts[prefix + n])
     gn1 = state.setdefault("gn1", GNState())
@@ -405,8 +410,11 @@ def resblock_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: floa
     a1, f1 = _gn(gn1, x, W_("gn1_gamma"), W_("gn1_beta"), P, G, eps, w, True, mode, trace,
                  prefix + "gn1", gn_stats)
     a1 = store(a1, storage)
-    h = store(conv3x3_halo(a1, state.get("a1_stale"), W_("conv1_w"), W_("conv1_b"), None, P,
-                           mode), storage)
+    b1 = W_("conv1_b")
+    if temb is not None:
+        tv = _a(temb)
+        b1 = b1 + linear((tv / (1.0 + np.exp(-tv)))[None, :], W_("temb_w"), W_("temb_b"))[0]
+    h = store(conv3x3_halo(a1, state.get("a1_stale"), W_("conv1_w"), b1, None, P, mode), storage)
     a2, f2 = _gn(gn2, h, W_("gn2_gamma"), W_("gn2_beta"), P, G, eps, w, True, mode, trace,
                  prefix + "gn2", gn_stats)
     a2 = store(a2, storage)
@@ -451,6 +459,83 @@ def attn_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float, h
     if trace is not None:
         trace[prefix + "a"], trace[prefix + "q"] = a, q
         trace[prefix + "k"], trace[prefix + "v"], trace[prefix + "o"] = k, v, o
+    gn.refresh(f)
+    state["k_stale"], state["v_stale"] = k, v
+    return out
+
+
+# --------------------------------------------------------------------------
+# SDXL-shaped transformer block (a "next" extension beyond the hot path)
+# --------------------------------------------------------------------------
+# The pages name SDXL as the model DistriFusion runs but do not spell out its
+# blocks.  Reading (R13): the plainest SDXL transformer block --
+#   GroupNorm -> proj_in -> [LN -> self-attention] + -> [LN -> cross-attention
+#   over the text context] + -> [LN -> GEGLU feed-forward] + -> proj_out -> + x
+# Only the GroupNorm statistics and the self-attention keys/values cross
+# bands, so only they are stale in displaced steps; LayerNorm, the
+# cross-attention (the same text context for every band) and the feed-forward
+# act on each token alone.
+
+def layer_norm(x: np.ndarray, gamma: np.ndarray, beta: np.ndarray, eps: float) -> np.ndarray:
+    """Per token (row of x: (T, C)): (x - mean) / sqrt(var + eps) * gamma + beta."""
+    m = x.mean(axis=1, keepdims=True)
+    v = ((x - m) ** 2).mean(axis=1, keepdims=True)
+    return (x - m) / np.sqrt(v + eps) * gamma + beta
+
+
+def gelu(x: np.ndarray) -> np.ndarray:
+    """Exact GELU, x * Phi(x) = x (1 + erf(x / sqrt 2)) / 2."""
+    return 0.5 * x * (1.0 + torch.special.erf(torch.from_numpy(np.asarray(x, dtype=np.float64)
+                                                                / math.sqrt(2.0))).numpy())
+
+
+def geglu_ff(x: np.ndarray, w1: np.ndarray, b1: np.ndarray, w2: np.ndarray,
+             b2: np.ndarray) -> np.ndarray:
+    """Feed-forward with a GELU-gated linear unit: [a | g] = x W1^T + b1 (two halves of the
+    inner width), then (a * gelu(g)) W2^T + b2."""
+    h = linear(x, w1, b1)
+    inner = h.shape[1] // 2
+    return linear(h[:, :inner] * gelu(h[:, inner:]), w2, b2)
+
+
+def transformer_step(state: Dict, x, ctx, wts: Dict, P: int, G: int, eps: float, w: float,
+                     heads: int, mode: int, storage: str, trace: Optional[Dict] = None,
+                     prefix: str = "", final_storage: Optional[str] = None,
+                     gn_stats: int = GN_STATS_CORRECTED, ln_eps: float = 1e-5):
+    """One SDXL-shaped transformer block (R13).  x: (C, H, W) image; ctx: (Tk, Cctx) text
+    context.  Tokens are pixels in raster order; band p's tokens are its rows."""
+    x = _a(x)
+    ctx = _a(ctx)
+    C, H, Wd = x.shape
+    W_ = lambda n: _a(wts[prefix + n])
+    gn = state.setdefault("gn", GNState())
+    a, f = _gn(gn, x, W_("gn_gamma"), W_("gn_beta"), P, G, eps, w, False, mode, trace,
+               prefix + "gn", gn_stats)
+    a = store(a, storage)
+    h = store(linear(a.reshape(C, H * Wd).T, W_("proj_in_w"), W_("proj_in_b")), storage)
+    d = C // heads
+    # self-attention: keys and values of other bands are the previous step's
+    t = store(layer_norm(h, W_("ln1_g"), W_("ln1_b"), ln_eps), storage)
+    q = store(linear(t, W_("wq"), W_("bq")), storage)
+    k = store(linear(t, W_("wk"), W_("bk")), storage)
+    v = store(linear(t, W_("wv"), W_("bv")), storage)
+    o = store(attention_stale_kv(q, k, v, state.get("k_stale"), state.get("v_stale"), P, heads,
+                                 1.0 / math.sqrt(d), mode), storage)
+    h = store(h + linear(o, W_("wo"), W_("bo")), storage)
+    # cross-attention over the text context: the same for every band
+    t = store(layer_norm(h, W_("ln2_g"), W_("ln2_b"), ln_eps), storage)
+    q2 = store(linear(t, W_("cq_w"), None), storage)
+    k2 = store(linear(ctx, W_("ck_w"), None), storage)
+    v2 = store(linear(ctx, W_("cv_w"), None), storage)
+    o2 = store(attention_cross(q2, k2, v2, heads, 1.0 / math.sqrt(d)), storage)
+    h = store(h + linear(o2, W_("co_w"), W_("co_b")), storage)
+    # feed-forward
+    t = store(layer_norm(h, W_("ln3_g"), W_("ln3_b"), ln_eps), storage)
+    h = store(h + geglu_ff(t, W_("ff1_w"), W_("ff1_b"), W_("ff2_w"), W_("ff2_b")), storage)
+    out_tok = linear(h, W_("proj_out_w"), W_("proj_out_b")) + x.reshape(C, H * Wd).T
+    out = store(out_tok.T.reshape(C, H, Wd), final_storage or storage)
+    if trace is not None:
+        trace[prefix + "k"], trace[prefix + "v"] = k, v
     gn.refresh(f)
     state["k_stale"], state["v_stale"] = k, v
     return out

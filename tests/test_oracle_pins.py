@@ -590,3 +590,125 @@ def test_cross_attention_equals_library_and_brute_force(Tq, Tk, heads):
             z = sum(w)
             for i in range(d):
                 assert abs(o[t, h * d + i] - sum(w[j] * v[j, h * d + i] for j in range(Tk)) / z) < 1e-10
+
+
+# ---------------------------------------------------------------- SDXL-shaped transformer block
+def rand_transformer_weights(r, C, Cctx, heads, mult=2):
+    s = lambda *shape: r.standard_normal(shape) * (1.0 / math.sqrt(shape[-1]))
+    w = {"gn_gamma": 1 + 0.3 * r.standard_normal(C), "gn_beta": 0.3 * r.standard_normal(C),
+         "proj_in_w": s(C, C), "proj_in_b": 0.3 * r.standard_normal(C),
+         "proj_out_w": s(C, C), "proj_out_b": 0.3 * r.standard_normal(C)}
+    for i in (1, 2, 3):
+        w[f"ln{i}_g"], w[f"ln{i}_b"] = 1 + 0.3 * r.standard_normal(C), 0.3 * r.standard_normal(C)
+    for n in ("wq", "wk", "wv", "wo"):
+        w[n] = s(C, C)
+    for n in ("bq", "bk", "bv", "bo", "co_b"):
+        w[n] = 0.3 * r.standard_normal(C)
+    w["cq_w"], w["co_w"] = s(C, C), s(C, C)
+    w["ck_w"], w["cv_w"] = s(C, Cctx), s(C, Cctx)
+    w["ff1_w"], w["ff1_b"] = s(2 * mult * C, C), 0.3 * r.standard_normal(2 * mult * C)
+    w["ff2_w"], w["ff2_b"] = s(C, mult * C), 0.3 * r.standard_normal(C)
+    return w
+
+
+def lib_transformer(x, ctx, w, G, eps, heads):
+    """The same block composed from library operators, on the whole image."""
+    g = lambda n: T64(w[n])
+    C, H, W = x.shape
+    d = C // heads
+    sh = lambda z: z.reshape(z.shape[0], heads, d).permute(1, 0, 2)
+    un = lambda z: z.permute(1, 0, 2).reshape(-1, C)
+    a = F.group_norm(T64(x)[None], G, g("gn_gamma"), g("gn_beta"), eps)[0].reshape(C, H * W).T
+    h = F.linear(a, g("proj_in_w"), g("proj_in_b"))
+    t = F.layer_norm(h, (C,), g("ln1_g"), g("ln1_b"), 1e-5)
+    o = F.scaled_dot_product_attention(sh(F.linear(t, g("wq"), g("bq"))), sh(F.linear(t, g("wk"), g("bk"))),
+                                       sh(F.linear(t, g("wv"), g("bv"))))
+    h = h + F.linear(un(o), g("wo"), g("bo"))
+    t = F.layer_norm(h, (C,), g("ln2_g"), g("ln2_b"), 1e-5)
+    c = T64(ctx)
+    o = F.scaled_dot_product_attention(sh(F.linear(t, g("cq_w"))), sh(F.linear(c, g("ck_w"))),
+                                       sh(F.linear(c, g("cv_w"))))
+    h = h + F.linear(un(o), g("co_w"), g("co_b"))
+    t = F.layer_norm(h, (C,), g("ln3_g"), g("ln3_b"), 1e-5)
+    a2, gate = F.linear(t, g("ff1_w"), g("ff1_b")).chunk(2, dim=-1)
+    h = h + F.linear(a2 * F.gelu(gate), g("ff2_w"), g("ff2_b"))
+    out = F.linear(h, g("proj_out_w"), g("proj_out_b")) + T64(x).reshape(C, H * W).T
+    return out.T.reshape(C, H, W).numpy()
+
+
+def test_layer_norm_gelu_geglu_equal_library():
+    r = rng(90)
+    x = r.standard_normal((7, 12)) * 2 + 0.3
+    gm, bt = 1 + 0.3 * r.standard_normal(12), 0.3 * r.standard_normal(12)
+    np.testing.assert_allclose(O.layer_norm(x, gm, bt, 1e-5),
+                               F.layer_norm(T64(x), (12,), T64(gm), T64(bt), 1e-5).numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(O.gelu(x), F.gelu(T64(x)).numpy(), rtol=0, atol=1e-14)
+    w1, b1 = r.standard_normal((16, 12)), r.standard_normal(16)
+    w2, b2 = r.standard_normal((12, 8)), r.standard_normal(12)
+    a, g = F.linear(T64(x), T64(w1), T64(b1)).chunk(2, dim=-1)
+    ref = F.linear(a * F.gelu(g), T64(w2), T64(b2)).numpy()
+    np.testing.assert_allclose(O.geglu_ff(x, w1, b1, w2, b2), ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("mode", [SYNC, DISPLACED, NAIVE])
+def test_p1_transformer_equals_library(mode):
+    r = rng(91)
+    C, H, W, G, heads, Cctx, Tk = 8, 4, 6, 4, 2, 6, 5
+    w = rand_transformer_weights(r, C, Cctx, heads)
+    x, ctx = r.standard_normal((C, H, W)), r.standard_normal((Tk, Cctx))
+    st = {}
+    O.transformer_step(st, x, ctx, w, 1, G, 1e-5, 1.0, heads, SYNC, "none")
+    y = O.transformer_step(st, x, ctx, w, 1, G, 1e-5, 1.0, heads, mode, "none")
+    np.testing.assert_allclose(y, lib_transformer(x, ctx, w, G, 1e-5, heads), rtol=0, atol=1e-11)
+
+
+def test_transformer_displaced_and_naive_invariants():
+    """Unchanged input: displaced equals sync.  Naive: each band is an independent image."""
+    r = rng(92)
+    C, H, W, P, G, heads, Cctx, Tk = 8, 8, 4, 4, 4, 2, 6, 5
+    w = rand_transformer_weights(r, C, Cctx, heads)
+    x, ctx = r.standard_normal((C, H, W)), r.standard_normal((Tk, Cctx))
+    outs = {}
+    for m in (SYNC, DISPLACED):
+        st = {}
+        O.transformer_step(st, x, ctx, w, P, G, 1e-5, 1.0, heads, SYNC, "none")
+        outs[m] = O.transformer_step(st, x, ctx, w, P, G, 1e-5, 1.0, heads, m, "none")
+    np.testing.assert_allclose(outs[DISPLACED], outs[SYNC], rtol=0, atol=1e-11)
+    y = O.transformer_step({}, x, ctx, w, P, G, 1e-5, 1.0, heads, NAIVE, "none")
+    hb = H // P
+    for p in range(P):
+        crop = x[:, p * hb:(p + 1) * hb, :]
+        np.testing.assert_allclose(y[:, p * hb:(p + 1) * hb, :], lib_transformer(crop, ctx, w, G, 1e-5, heads),
+                                   rtol=0, atol=1e-11)
+    # drift: displaced differs from sync, and from naive by more
+    x1 = x + 0.3 * r.standard_normal(x.shape)
+    res = {}
+    for m in (SYNC, DISPLACED, NAIVE):
+        st = {}
+        O.transformer_step(st, x, ctx, w, P, G, 1e-5, 1.0, heads, SYNC, "none")
+        res[m] = O.transformer_step(st, x1, ctx, w, P, G, 1e-5, 1.0, heads, m, "none")
+    err = lambda m: np.linalg.norm(res[m] - res[SYNC]) / np.linalg.norm(res[SYNC])
+    assert 0 < err(DISPLACED) < err(NAIVE)
+
+
+@pytest.mark.parametrize("mode", [SYNC, DISPLACED])
+def test_p1_resblock_time_embedding_equals_library(mode):
+    """A time embedding adds temb_w silu(temb) + temb_b to every pixel of conv1's output."""
+    r = rng(93)
+    C, H, W, G, Ct = 8, 5, 6, 4, 10
+    w = rand_res_weights(r, C, C)
+    w["temb_w"], w["temb_b"] = r.standard_normal((C, Ct)) / math.sqrt(Ct), 0.3 * r.standard_normal(C)
+    x, temb = r.standard_normal((C, H, W)), r.standard_normal(Ct)
+    st = {}
+    O.resblock_step(st, x, w, 1, G, 1e-5, 1.0, SYNC, "none", temb=temb)
+    y = O.resblock_step(st, x, w, 1, G, 1e-5, 1.0, mode, "none", temb=temb)
+    g = lambda n: T64(w[n])
+    t = F.silu(F.group_norm(T64(x)[None], G, g("gn1_gamma"), g("gn1_beta"), 1e-5))
+    h = F.conv2d(t, g("conv1_w"), g("conv1_b"), padding=1)
+    h = h + F.linear(F.silu(T64(temb)), g("temb_w"), g("temb_b"))[None, :, None, None]
+    t = F.silu(F.group_norm(h, G, g("gn2_gamma"), g("gn2_beta"), 1e-5))
+    ref = (F.conv2d(t, g("conv2_w"), g("conv2_b"), padding=1) + T64(x)[None])[0].numpy()
+    np.testing.assert_allclose(y, ref, rtol=0, atol=1e-11)
+    # without the embedding the block is the plain ResBlock
+    np.testing.assert_allclose(O.resblock_step({}, x, w, 1, G, 1e-5, 1.0, SYNC, "none"),
+                               lib_resblock(x, w, G, 1e-5), rtol=0, atol=1e-11)
