@@ -63,6 +63,8 @@ _SIGS = {
     "dp_attn_workspace_size": ([], _SZ),
     "dp_attn_stale_kv": ([_V, _V, _V, _V, _V, _V, _I, _I, _I, _I, _F, _I, _V, _SZ, _V], _I),
     "dp_attn_cross": ([_V, _V, _V, _V, _I, _I, _I, _I, _F, _V, _SZ, _V], _I),
+    "dp_layernorm": ([_V, _V, _V, _V, _I, _I, _F, _V], _I),
+    "dp_geglu": ([_V, _V, _I, _I, _V], _I),
     "dp_refresh_stale": ([_V, _V, _SZ, _I, _I, _I, _V], _I),
     "dp_refresh_halo": ([_V, _V, _SZ, _I, _I, _I, _I, _V], _I),
     "dp_refresh_stats": ([_V, _V, _V, _I, _I, _V], _I),
@@ -204,6 +206,14 @@ def dp_attn_cross(q, k, v, o, Tq, Tk, heads, head_dim, scale, workspace=None, wo
                   stream=None):
     return _check(lib().dp_attn_cross(_p(q), _p(k), _p(v), _p(o), Tq, Tk, heads, head_dim, scale,
                                       _p(workspace), workspace_bytes, _s(stream)))
+
+
+def dp_layernorm(x, y, gamma, beta, T, C, eps, stream=None):
+    return _check(lib().dp_layernorm(_p(x), _p(y), _p(gamma), _p(beta), T, C, eps, _s(stream)))
+
+
+def dp_geglu(h, y, T, F, stream=None):
+    return _check(lib().dp_geglu(_p(h), _p(y), T, F, _s(stream)))
 
 
 def dp_refresh_stale(fresh, stale, row_bytes, rows, P, band=-1, stream=None):

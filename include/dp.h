@@ -282,6 +282,23 @@ DP_API int dp_attn_cross(const void* q, const void* k, const void* v, void* o, i
                   void* stream);
 
 /* ------------------------------------------------------------------------
+ * Per-token operators of an SDXL-shaped transformer block ("next" item: the
+ * pages name SDXL as the model; they act on each token alone, so every band
+ * runs them on its fresh tokens with no stale context).
+ *
+ * dp_layernorm: y[t] = (x[t] - mean_t) / sqrt(var_t + eps) * gamma + beta
+ *   over the C channels of token t (biased variance).
+ *   x, y [T][C] bf16, device (y may not alias x); gamma, beta [C] fp32,
+ *   device.  C % 8 == 0, C <= 2048, 16-byte aligned pointers.
+ * dp_geglu: y[t][c] = a * gelu(g), a = h[t][c], g = h[t][F + c], exact GELU
+ *   x (1 + erf(x / sqrt 2)) / 2 (the gated feed-forward's middle step).
+ *   h [T][2F] bf16, y [T][F] bf16, device, not overlapping; F % 8 == 0.
+ * ---------------------------------------------------------------------- */
+DP_API int dp_layernorm(const void* x, void* y, const float* gamma, const float* beta, int T,
+                 int C, float eps, void* stream);
+DP_API int dp_geglu(const void* h, void* y, int T, int F, void* stream);
+
+/* ------------------------------------------------------------------------
  * Stale-buffer refresh: the device-local replacement of the paper's
  * per-layer AllGather (atlas.scime.ai summary, Approach: AllGather overlaps
  * computation; limitations: NCCL kernels take SMs).  Copies the rows of band

@@ -251,3 +251,21 @@ def test_cross_attention_rejects_bad_arguments_on_the_host(B):
     with pytest.raises(B.DPError) as e:
         B.dp_attn_cross(None, 32, 48, 64, 256, 77, 2, 64, 0.125, stream=0)
     assert e.value.code == B.DP_ERR_INVALID_ARG
+
+
+def test_token_operators_reject_bad_arguments_on_the_host(B):
+    with pytest.raises(B.DPError) as e:   # C not a multiple of 8
+        B.dp_layernorm(16, 4096, 32, 48, 4, 12, 1e-5, stream=0)
+    assert e.value.code == B.DP_ERR_UNSUPPORTED
+    with pytest.raises(B.DPError) as e:   # C too large for one warp's registers
+        B.dp_layernorm(16, 1 << 20, 32, 48, 4, 4096, 1e-5, stream=0)
+    assert e.value.code == B.DP_ERR_UNSUPPORTED
+    with pytest.raises(B.DPError) as e:   # y aliases x
+        B.dp_layernorm(16, 16, 32, 48, 4, 64, 1e-5, stream=0)
+    assert e.value.code == B.DP_ERR_INVALID_ARG
+    with pytest.raises(B.DPError) as e:   # F not a multiple of 8
+        B.dp_geglu(16, 4096, 4, 12, stream=0)
+    assert e.value.code == B.DP_ERR_UNSUPPORTED
+    with pytest.raises(B.DPError) as e:   # y overlaps h
+        B.dp_geglu(16, 32, 4, 64, stream=0)
+    assert e.value.code == B.DP_ERR_INVALID_ARG

@@ -327,6 +327,28 @@ def test_cross_attention_parity(Tq, Tk, heads, split):
     assert B.dp_device_status() == 0
 
 
+# ---------------------------------------------------------------- per-token operators
+@pytest.mark.parametrize("T,C", [(4096, 640), (1024, 1280), (300, 320), (7, 8), (33, 2048)])
+def test_layernorm_parity(T, C):
+    r = rng(T + C)
+    x = rounded(1.5 * r.standard_normal((T, C)) + 0.4, "bf16")
+    g, b = 1 + 0.3 * r.standard_normal(C), 0.3 * r.standard_normal(C)
+    y = torch.empty(T, C, dtype=torch.bfloat16, device="cuda")
+    B.dp_layernorm(dev_mat(x), y, dev_f32(g), dev_f32(b), T, C, 1e-5)
+    torch.cuda.synchronize()
+    check(host(y), O.layer_norm(x, g, b, 1e-5), what=f"layernorm T={T} C={C}", storage_rel=BF16_HALF_ULP)
+
+
+@pytest.mark.parametrize("T,F", [(4096, 2560), (1024, 5120), (77, 8), (5, 24)])
+def test_geglu_parity(T, F):
+    r = rng(T + F)
+    h = rounded(2.0 * r.standard_normal((T, 2 * F)), "bf16")
+    y = torch.empty(T, F, dtype=torch.bfloat16, device="cuda")
+    B.dp_geglu(dev_mat(h), y, T, F)
+    torch.cuda.synchronize()
+    check(host(y), h[:, :F] * O.gelu(h[:, F:]), what=f"geglu T={T} F={F}", storage_rel=BF16_HALF_ULP)
+
+
 # ---------------------------------------------------------------- refresh
 def test_refresh_is_an_exact_copy():
     g = torch.Generator(device="cpu").manual_seed(3)
