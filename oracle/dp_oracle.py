@@ -531,7 +531,10 @@ def transformer_step(state: Dict, x, ctx, wts: Dict, P: int, G: int, eps: float,
     h = store(h + linear(o2, W_("co_w"), W_("co_b")), storage)
     # feed-forward
     t = store(layer_norm(h, W_("ln3_g"), W_("ln3_b"), ln_eps), storage)
-    h = store(h + geglu_ff(t, W_("ff1_w"), W_("ff1_b"), W_("ff2_w"), W_("ff2_b")), storage)
+    hf = store(linear(t, W_("ff1_w"), W_("ff1_b")), storage)     # geglu_ff, stored where the GPU stores
+    inner = hf.shape[1] // 2
+    gf = store(hf[:, :inner] * gelu(hf[:, inner:]), storage)
+    h = store(h + linear(gf, W_("ff2_w"), W_("ff2_b")), storage)
     out_tok = linear(h, W_("proj_out_w"), W_("proj_out_b")) + x.reshape(C, H * Wd).T
     out = store(out_tok.T.reshape(C, H, Wd), final_storage or storage)
     if trace is not None:
