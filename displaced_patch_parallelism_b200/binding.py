@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(PKG_DIR, "libdp.so")
 DP_OK, DP_ERR_INVALID_ARG, DP_ERR_UNSUPPORTED, DP_ERR_STATE, DP_ERR_CUDA, DP_ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
 SYNC, DISPLACED, NAIVE = 0, 1, 2
 BF16, FP32 = 0, 1
-GN_CONV, RESBLOCK, ATTN, UNET_MINI = 0, 1, 2, 3
+GN_CONV, RESBLOCK, ATTN, UNET_MINI, TRANSFORMER = 0, 1, 2, 3, 4
 GN_STATS_CORRECTED, GN_STATS_LOCAL, GN_STATS_STALE, GN_STATS_SYNC = 0, 1, 2, 3
 
 ERR_NAMES = {DP_ERR_INVALID_ARG: "DP_ERR_INVALID_ARG", DP_ERR_UNSUPPORTED: "DP_ERR_UNSUPPORTED",
@@ -37,7 +37,8 @@ class BlockDesc(ctypes.Structure):
                 ("C", ctypes.c_int), ("Cout", ctypes.c_int), ("G", ctypes.c_int),
                 ("P", ctypes.c_int), ("heads", ctypes.c_int), ("dtype", ctypes.c_int),
                 ("silu", ctypes.c_int), ("eps", ctypes.c_float), ("w", ctypes.c_float),
-                ("gn_stats", ctypes.c_int)]
+                ("gn_stats", ctypes.c_int), ("ctx_len", ctypes.c_int), ("ctx_dim", ctypes.c_int),
+                ("ff_inner", ctypes.c_int)]
 
 
 class BlockState(ctypes.Structure):
@@ -70,6 +71,7 @@ _SIGS = {
     "dp_refresh_stats": ([_V, _V, _V, _I, _I, _V], _I),
     "dp_block_desc_init": ([ctypes.POINTER(BlockDesc), _I, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _F], _I),
     "dp_block_desc_set_gn_stats": ([ctypes.POINTER(BlockDesc), _I], _I),
+    "dp_block_desc_set_context": ([ctypes.POINTER(BlockDesc), _I, _I, _I], _I),
     "dp_block_workspace_size": ([ctypes.POINTER(BlockDesc)], _SZ),
     "dp_block_state_init": ([ctypes.POINTER(BlockDesc), ctypes.POINTER(BlockState), _V, _SZ, _V], _I),
     "dp_block_step": ([ctypes.POINTER(BlockDesc), ctypes.POINTER(BlockState), _V, _V,
@@ -242,6 +244,10 @@ def dp_block_desc_set_gn_stats(d: BlockDesc, variant: int):
     return _check(lib().dp_block_desc_set_gn_stats(ctypes.byref(d), variant))
 
 
+def dp_block_desc_set_context(d: BlockDesc, ctx_len: int, ctx_dim: int, ff_inner: int):
+    return _check(lib().dp_block_desc_set_context(ctypes.byref(d), ctx_len, ctx_dim, ff_inner))
+
+
 def dp_block_workspace_size(d: BlockDesc) -> int:
     n = lib().dp_block_workspace_size(ctypes.byref(d))
     if n == 0:
@@ -285,7 +291,7 @@ def dp_block_step_timed(d: BlockDesc, s: BlockState, x, out, weights: Sequence, 
 
 KERNEL_NAMES = {0: "gn_stats", 1: "gn_apply", 2: "gn_fused", 3: "conv", 4: "linear", 5: "attn",
                 6: "copy", 7: "conv_small", 8: "splitk_finish",
-                9: "gn_cluster"}
+                9: "gn_cluster", 10: "layernorm", 11: "geglu"}
 
 
 def dp_block_launch_info(d: BlockDesc, mode: int, i: int):
@@ -311,9 +317,13 @@ class Block:
     """A block descriptor, its device workspace (a torch uint8 tensor) and its state."""
 
     def __init__(self, kind, H, W, C, Cout=0, G=32, P=4, heads=0, dtype=BF16, silu=True,
-                 eps=1e-5, w=1.0, device="cuda", stream=None, gn_stats=GN_STATS_CORRECTED):
+                 eps=1e-5, w=1.0, device="cuda", stream=None, gn_stats=GN_STATS_CORRECTED,
+                 context=None):
+        """``context`` = (ctx_len, ctx_dim, ff_inner) for TRANSFORMER blocks."""
         import torch
         self.desc = dp_block_desc_init(kind, H, W, C, Cout, G, P, heads, dtype, silu, eps, w)
+        if context is not None:
+            dp_block_desc_set_context(self.desc, *context)
         if gn_stats != GN_STATS_CORRECTED:
             dp_block_desc_set_gn_stats(self.desc, gn_stats)
         self.ws_bytes = dp_block_workspace_size(self.desc)

@@ -1048,9 +1048,9 @@ size_t attn_workspace_bytes() {
 
 // Self-attention (Tk = T) or, with Tk != T, attention of T queries over Tk
 // keys that are all visible (mode SYNC, P = 1: cross-attention).
-static int attn_launch_tk(const void* q, const void* kf, const void* vf, const void* ks, const void* vs,
-                          void* o, int T, int Tk, int heads, int P, float scale, int mode,
-                          void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+int attn_launch_tk(const void* q, const void* kf, const void* vf, const void* ks, const void* vs,
+                   void* o, int T, int Tk, int heads, int P, float scale, int mode,
+                   void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   AttnParams a;
   memset(&a, 0, sizeof(a));
   const int ld = heads * 64;

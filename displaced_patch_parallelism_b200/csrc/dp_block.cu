@@ -10,7 +10,10 @@
 // output of the layer feeding a conv) and reads the stale half; the refresh
 // that replaces the paper's AllGather is a flip of `cur`, so no byte moves.
 //
-// Kinds: GN_CONV, RESBLOCK, ATTN, and UNET_MINI, a chain of the others with
+// Kinds: GN_CONV, RESBLOCK, ATTN, TRANSFORMER (SDXL-shaped: GroupNorm and
+// self-attention with stale context, then per-token LayerNorms, a
+// cross-attention over the text context and a gated feed-forward, none of
+// which need context from other bands), and UNET_MINI, a chain of the others with
 // two stride-2 downsampling convs (conv_in -> ResBlock(320) -> down ->
 // ResBlock(320->640) -> Attn(640) -> down -> ResBlock(640->1280) ->
 // Attn(1280)).  Composite kinds run their sub-blocks with the parent's
@@ -48,6 +51,7 @@ struct Layout {
   GnSlots gn1, gn2;
   size_t a1[2], a2[2], h, sc;        // conv inputs (pairs), conv1 output, shortcut output
   size_t act, q, k[2], v[2], o;      // attention buffers
+  size_t ha, hb, tn, q2, k2, v2, o2, ffh, ffg;   // TRANSFORMER: residual stream, LN output, cross, FF
   size_t attn_ws;                     // balanced attention split: counters + partials
   size_t gemm_ws;                     // split-K partials of the convs and projections
   // UNET_MINI: sub-block workspaces and the buffers between them
@@ -112,6 +116,24 @@ Layout layout_of(const dp_block_desc* d) {
     for (int i = 0; i < 2; ++i) L.a2[i] = b.take(hw * d->Cout * e);
     L.h = b.take(hw * d->Cout * e);
     if (d->C != d->Cout) L.sc = b.take(hw * d->Cout * e);
+  } else if (d->kind == DP_BLOCK_TRANSFORMER) {
+    const size_t C = d->C, Tk = d->ctx_len, F = d->ff_inner;
+    L.gn1 = gn_slots(b, d->P, d->G);
+    L.act = b.take(hw * C * e);
+    L.ha = b.take(hw * C * e);
+    L.hb = b.take(hw * C * e);
+    L.tn = b.take(hw * C * e);
+    L.q = b.take(hw * C * e);
+    for (int i = 0; i < 2; ++i) L.k[i] = b.take(hw * C * e);
+    for (int i = 0; i < 2; ++i) L.v[i] = b.take(hw * C * e);
+    L.o = b.take(hw * C * e);
+    L.q2 = b.take(hw * C * e);
+    L.k2 = b.take(Tk * C * e);
+    L.v2 = b.take(Tk * C * e);
+    L.o2 = b.take(hw * C * e);
+    L.ffh = b.take(hw * 2 * F * e);
+    L.ffg = b.take(hw * F * e);
+    L.attn_ws = b.take(attn_workspace_bytes());
   } else if (d->kind == DP_BLOCK_ATTN) {
     L.gn1 = gn_slots(b, d->P, d->G);
     L.act = b.take(hw * d->C * e);
@@ -144,7 +166,7 @@ Layout layout_of(const dp_block_desc* d) {
 
 int desc_check(const dp_block_desc* d) {
   if (!d) return set_error(DP_ERR_INVALID_ARG, "block: null descriptor");
-  if (d->kind < DP_BLOCK_GN_CONV || d->kind > DP_BLOCK_UNET_MINI)
+  if (d->kind < DP_BLOCK_GN_CONV || d->kind > DP_BLOCK_TRANSFORMER)
     return set_error(DP_ERR_INVALID_ARG, "block: bad kind %d", d->kind);
   if (d->H <= 0 || d->W <= 0 || d->C <= 0 || d->Cout <= 0 || d->G <= 0 || d->P <= 0)
     return set_error(DP_ERR_INVALID_ARG, "block: non-positive size");
@@ -170,6 +192,17 @@ int desc_check(const dp_block_desc* d) {
     return DP_OK;
   }
   if (d->C % d->G || d->Cout % d->G) return set_error(DP_ERR_UNSUPPORTED, "block: channels %% G != 0");
+  if (d->kind == DP_BLOCK_TRANSFORMER) {
+    if (d->Cout != d->C) return set_error(DP_ERR_INVALID_ARG, "block: transformer keeps C");
+    if (d->heads <= 0 || d->C != d->heads * 64)
+      return set_error(DP_ERR_UNSUPPORTED, "block: transformer needs C == heads * 64");
+    const int T = d->H * d->W;
+    if ((T / d->P) % 128 || T % 256)
+      return set_error(DP_ERR_UNSUPPORTED, "block: transformer needs (H*W/P) %% 128 == 0 and H*W %% 256 == 0");
+    if (d->ctx_len < 1 || d->ctx_dim <= 0 || d->ctx_dim % 64 || d->ff_inner <= 0 || d->ff_inner % 64)
+      return set_error(DP_ERR_INVALID_ARG, "block: transformer needs dp_block_desc_set_context "
+                                           "(ctx_len >= 1, ctx_dim and ff_inner multiples of 64)");
+  }
   if (d->kind == DP_BLOCK_ATTN) {
     if (d->Cout != d->C) return set_error(DP_ERR_INVALID_ARG, "block: attention keeps C");
     if (d->heads <= 0 || d->C != d->heads * 64)
@@ -184,6 +217,7 @@ int weight_count(const dp_block_desc* d) {
   if (d->kind == DP_BLOCK_GN_CONV) return 4;
   if (d->kind == DP_BLOCK_RESBLOCK) return d->C != d->Cout ? 10 : 8;
   if (d->kind == DP_BLOCK_ATTN) return 6;
+  if (d->kind == DP_BLOCK_TRANSFORMER) return 25;
   const MiniDescs m = mini_descs(d);
   return 2 + weight_count(&m.rb1) + 2 + weight_count(&m.rb2) + weight_count(&m.at2) + 2 +
          weight_count(&m.rb3) + weight_count(&m.at3);
@@ -197,6 +231,13 @@ double flops_of(const dp_block_desc* d) {
     return 2.0 * hw * Co * 9.0 * C + 2.0 * hw * Co * 9.0 * Co + (C != Co ? 2.0 * hw * Co * C : 0.0);
   if (d->kind == DP_BLOCK_ATTN)
     return 2.0 * hw * 3.0 * C * C + 4.0 * hw * hw * C + 2.0 * hw * C * C;
+  if (d->kind == DP_BLOCK_TRANSFORMER) {
+    const double Tk = d->ctx_len, Cc = d->ctx_dim, F = d->ff_inner;
+    return 2.0 * hw * C * C * 5.0 +                       // proj_in, wo, cq, co, proj_out
+           2.0 * hw * 3.0 * C * C + 4.0 * hw * hw * C +   // q/k/v, self-attention
+           2.0 * Tk * 2.0 * C * Cc + 4.0 * hw * Tk * C +  // context k/v, cross-attention
+           2.0 * hw * 2.0 * F * C + 2.0 * hw * C * F;     // ff1, ff2
+  }
   const MiniDescs m = mini_descs(d);
   return 2.0 * hw * kU1 * 9.0 * C + flops_of(&m.rb1) + 2.0 * (hw / 4) * kU1 * 9.0 * kU1 +
          flops_of(&m.rb2) + flops_of(&m.at2) + 2.0 * (hw / 16) * kU2 * 9.0 * kU2 +
@@ -303,8 +344,10 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
   if (d->kind != DP_BLOCK_UNET_MINI && !plan) {
     // biases (conv_b, conv1_b, conv2_b, short_b; bqkv, bo) may be NULL
     for (int i = 0; i < weight_count(d); ++i) {
-      const bool bias = d->kind == DP_BLOCK_ATTN ? (i == 3 || i == 5)
-                                                 : (i == 3 || i == 7 || i == 9);
+      const bool bias = d->kind == DP_BLOCK_ATTN          ? (i == 3 || i == 5)
+                        : d->kind == DP_BLOCK_TRANSFORMER ? (i == 3 || i == 7 || i == 9 || i == 15 ||
+                                                             i == 19 || i == 21 || i == 23)
+                                                          : (i == 3 || i == 7 || i == 9);
       if (!w[i] && !bias) return set_error(DP_ERR_INVALID_ARG, "block: weight %d is NULL", i);
     }
   }
@@ -342,6 +385,79 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
       res = sc;
     }
     return conv(a2f, at<void>(ws, L.a2[o]), w[6], w[7], res, out, H, W, Co, Co, 1);
+  }
+  if (d->kind == DP_BLOCK_TRANSFORMER) {
+    const int T = H * W, Tk = d->ctx_len, Cc = d->ctx_dim, Fi = d->ff_inner;
+    void* act = at<void>(ws, L.act);
+    void* ha = at<void>(ws, L.ha);
+    void* hb = at<void>(ws, L.hb);
+    void* tn = at<void>(ws, L.tn);
+    void* q = at<void>(ws, L.q);
+    void* kf = at<void>(ws, L.k[f]);
+    void* vf = at<void>(ws, L.v[f]);
+    void* ob = at<void>(ws, L.o);
+    void* q2 = at<void>(ws, L.q2);
+    void* k2 = at<void>(ws, L.k2);
+    void* v2 = at<void>(ws, L.v2);
+    void* o2 = at<void>(ws, L.o2);
+    void* ffh = at<void>(ws, L.ffh);
+    void* ffg = at<void>(ws, L.ffg);
+    auto ln = [&](const void* in, void* y, const void* g, const void* b) {
+      if (plan) {
+        plan->push(DP_KERNEL_LAYERNORM, 0.0, 2.0 * T * C * e);
+        return DP_OK;
+      }
+      return dp_layernorm(in, y, static_cast<const float*>(g), static_cast<const float*>(b), T, C, 1e-5f, st);
+    };
+    rc = gn(L.gn1, x, act, w[0], w[1], C, 0);
+    if (rc) return rc;
+    rc = lin(act, w[2], w[3], nullptr, ha, nullptr, nullptr, T, C, C, C);   // proj_in
+    if (rc) return rc;
+    // self-attention: other bands' keys and values are the previous step's
+    rc = ln(ha, tn, w[4], w[5]);
+    if (rc) return rc;
+    rc = lin(tn, w[6], w[7], nullptr, q, kf, vf, T, 3 * C, C, C);
+    if (rc) return rc;
+    if (plan) {
+      const double keys = mode == DP_MODE_NAIVE ? static_cast<double>(T) / P : T;
+      plan->push(DP_KERNEL_ATTN, 4.0 * T * keys * C, 4.0 * T * C * e);
+    } else {
+      rc = attn_launch(q, kf, vf, at<void>(ws, L.k[o]), at<void>(ws, L.v[o]), ob, T, d->heads, P,
+                       0.125f, mode, at<void>(ws, L.attn_ws), attn_workspace_bytes(), st);
+      if (rc) return rc;
+    }
+    rc = lin(ob, w[8], w[9], ha, hb, nullptr, nullptr, T, C, C, C);
+    if (rc) return rc;
+    // cross-attention over the step's text context (w[24]): the same for every band
+    rc = ln(hb, tn, w[10], w[11]);
+    if (rc) return rc;
+    rc = lin(tn, w[12], nullptr, nullptr, q2, nullptr, nullptr, T, C, C, C);
+    if (rc) return rc;
+    rc = lin(w[24], w[13], nullptr, nullptr, k2, v2, nullptr, Tk, 2 * C, Cc, C);
+    if (rc) return rc;
+    if (plan) {
+      plan->push(DP_KERNEL_ATTN, 4.0 * T * static_cast<double>(Tk) * C, (2.0 * T * C + 2.0 * Tk * C) * e);
+    } else {
+      rc = attn_launch_tk(q2, k2, v2, nullptr, nullptr, o2, T, Tk, d->heads, 1, 0.125f, DP_MODE_SYNC,
+                          at<void>(ws, L.attn_ws), attn_workspace_bytes(), st);
+      if (rc) return rc;
+    }
+    rc = lin(o2, w[14], w[15], hb, ha, nullptr, nullptr, T, C, C, C);
+    if (rc) return rc;
+    // gated feed-forward
+    rc = ln(ha, tn, w[16], w[17]);
+    if (rc) return rc;
+    rc = lin(tn, w[18], w[19], nullptr, ffh, nullptr, nullptr, T, 2 * Fi, C, 2 * Fi);
+    if (rc) return rc;
+    if (plan) {
+      plan->push(DP_KERNEL_GEGLU, 0.0, 3.0 * T * Fi * e);
+    } else {
+      rc = dp_geglu(ffh, ffg, T, Fi, st);
+      if (rc) return rc;
+    }
+    rc = lin(ffg, w[20], w[21], ha, hb, nullptr, nullptr, T, C, Fi, C);
+    if (rc) return rc;
+    return lin(hb, w[22], w[23], x, out, nullptr, nullptr, T, C, C, C);   // proj_out + x
   }
   if (d->kind == DP_BLOCK_ATTN) {
     const int T = H * W;
@@ -455,6 +571,20 @@ int dp_block_desc_init(dp_block_desc* d, int kind, int H, int W, int C, int Cout
   d->eps = eps;
   d->w = w;
   d->gn_stats = DP_GN_STATS_CORRECTED;
+  d->ctx_len = 0;
+  d->ctx_dim = 0;
+  d->ff_inner = 0;
+  if (kind == DP_BLOCK_TRANSFORMER) return DP_OK;   // checked once dp_block_desc_set_context is called
+  return dp::desc_check(d);
+}
+
+int dp_block_desc_set_context(dp_block_desc* d, int ctx_len, int ctx_dim, int ff_inner) {
+  if (!d) return dp::set_error(DP_ERR_INVALID_ARG, "block: null descriptor");
+  if (d->kind != DP_BLOCK_TRANSFORMER)
+    return dp::set_error(DP_ERR_INVALID_ARG, "block: a context is only for TRANSFORMER blocks");
+  d->ctx_len = ctx_len;
+  d->ctx_dim = ctx_dim;
+  d->ff_inner = ff_inner;
   return dp::desc_check(d);
 }
 

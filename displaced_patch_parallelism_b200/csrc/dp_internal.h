@@ -35,6 +35,11 @@ int linear_launch(const void* x, const void* weight, const float* bias, const vo
 int attn_validate(const void* q, const void* kf, const void* vf, const void* ks, const void* vs,
                   const void* o, int T, int heads, int head_dim, int P, int mode);
 size_t attn_workspace_bytes();
+// attention of T queries over Tk keys (Tk = T: self-attention; with mode SYNC
+// and P = 1 and Tk != T: cross-attention over a context every band sees)
+int attn_launch_tk(const void* q, const void* kf, const void* vf, const void* ks, const void* vs,
+                   void* o, int T, int Tk, int heads, int P, float scale, int mode, void* workspace,
+                   size_t workspace_bytes, cudaStream_t stream);
 int attn_launch(const void* q, const void* kf, const void* vf, const void* ks, const void* vs,
                 void* o, int T, int heads, int P, float scale, int mode, void* workspace,
                 size_t workspace_bytes, cudaStream_t stream);

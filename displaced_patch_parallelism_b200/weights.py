@@ -24,7 +24,8 @@ def _conv(w, dtype, device):
 
 def block_weights(kind: str, wts: Dict, dtype: torch.dtype = torch.bfloat16, device="cuda",
                   prefix: str = "") -> List[torch.Tensor]:
-    """Device tensors in the order ``dp_block_step`` documents for ``kind``."""
+    """Device tensors in the order ``dp_block_step`` documents for ``kind`` (a TRANSFORMER
+    block's per-step text context, its 25th pointer, is appended by the caller)."""
     g = lambda n: wts[prefix + n]
     f32 = torch.float32
     if kind == "gn_conv":
@@ -47,6 +48,16 @@ def block_weights(kind: str, wts: Dict, dtype: torch.dtype = torch.bfloat16, dev
                 _t(cat(g("wq"), g("wk"), g("wv")), dtype, device),
                 _t(cat(g("bq"), g("bk"), g("bv")), f32, device),
                 _t(g("wo"), dtype, device), _t(g("bo"), f32, device)]
+    if kind == "transformer":
+        cat = lambda *xs: torch.cat([x if isinstance(x, torch.Tensor) else torch.as_tensor(x) for x in xs])
+        v = lambda n: _t(g(n), f32, device)
+        m = lambda n: _t(g(n), dtype, device)
+        return [v("gn_gamma"), v("gn_beta"), m("proj_in_w"), v("proj_in_b"), v("ln1_g"), v("ln1_b"),
+                _t(cat(g("wq"), g("wk"), g("wv")), dtype, device),
+                _t(cat(g("bq"), g("bk"), g("bv")), f32, device), m("wo"), v("bo"),
+                v("ln2_g"), v("ln2_b"), m("cq_w"), _t(cat(g("ck_w"), g("cv_w")), dtype, device),
+                m("co_w"), v("co_b"), v("ln3_g"), v("ln3_b"), m("ff1_w"), v("ff1_b"), m("ff2_w"),
+                v("ff2_b"), m("proj_out_w"), v("proj_out_b")]
     if kind == "unet_mini":
         out = [_conv(g("conv_in_w"), dtype, device), _t(g("conv_in_b"), f32, device)]
         out += block_weights("resblock", wts, dtype, device, prefix + "rb1.")

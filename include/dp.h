@@ -72,6 +72,9 @@ extern "C" {
 #define DP_BLOCK_ATTN 2     /* GN -> q,k,v proj -> stale-K/V attention -> out proj -> + x   */
 #define DP_BLOCK_UNET_MINI 3 /* conv_in -> ResBlock(320) -> down -> ResBlock(320->640) ->   */
                              /* Attn(640) -> down -> ResBlock(640->1280) -> Attn(1280)      */
+#define DP_BLOCK_TRANSFORMER 4 /* SDXL-shaped: GN -> proj_in -> [LN -> self-attention] + ->   */
+                               /* [LN -> cross-attention] + -> [LN -> GEGLU FF] + ->          */
+                               /* proj_out -> + x (dp_block_desc_set_context first)           */
 
 /* Message for the calling thread's last failed call ("" if none). */
 DP_API const char* dp_last_error(void);
@@ -351,7 +354,19 @@ typedef struct dp_block_desc {
   float eps;      /* GroupNorm epsilon                            */
   float w;        /* weight of the corrected-statistics drift term */
   int gn_stats;   /* DP_GN_STATS_*: statistics of displaced steps  */
+  int ctx_len;    /* TRANSFORMER: text context tokens (Tk)        */
+  int ctx_dim;    /* TRANSFORMER: text context width (Cctx)       */
+  int ff_inner;   /* TRANSFORMER: feed-forward inner width (F)    */
 } dp_block_desc;
+
+/*
+ * TRANSFORMER blocks: the text context's length and width and the
+ * feed-forward's inner width (SDXL: 77, 2048, 4C).  The context is an input of
+ * every step (the last weight pointer); it is the same for every band, so it
+ * has no stale copy.  Needs ctx_len >= 1, ctx_dim % 64 == 0, ff_inner % 64 ==
+ * 0.  DP_ERR_INVALID_ARG on a null descriptor or bad sizes.
+ */
+DP_API int dp_block_desc_set_context(dp_block_desc* d, int ctx_len, int ctx_dim, int ff_inner);
 
 typedef struct dp_block_state {
   void* workspace;        /* device memory of dp_block_workspace_size() bytes */
@@ -398,6 +413,15 @@ DP_API int dp_block_state_init(const dp_block_desc* d, dp_block_state* s, void* 
  *             conv2_b[Cout], then if C != Cout: short_w[Cout][C], short_b[Cout]
  *   ATTN:     gn_gamma[C], gn_beta[C], wqkv[3C][C] (the q, k and v (out, in)
  *             matrices stacked), bqkv[3C], wo[C][C], bo[C]
+ *   TRANSFORMER (C == heads * 64, (H*W/P) % 128 == 0, (H*W) % 256 == 0):
+ *             gn_gamma[C], gn_beta[C], proj_in_w[C][C], proj_in_b[C], ln1_g[C],
+ *             ln1_b[C], wqkv[3C][C], bqkv[3C], wo[C][C], bo[C], ln2_g[C], ln2_b[C],
+ *             cq_w[C][C], ckv_w[2C][Cctx] (the context's k and v matrices
+ *             stacked), co_w[C][C], co_b[C], ln3_g[C], ln3_b[C],
+ *             ff1_w[2F][C] (value half, then gate half), ff1_b[2F], ff2_w[C][F],
+ *             ff2_b[C], proj_out_w[C][C], proj_out_b[C], and the step's context
+ *             [ctx_len][ctx_dim] bf16 (25 pointers; matrices bf16, vectors fp32;
+ *             the biases may be NULL)
  *   UNET_MINI (latent [H][W][C], C even <= 16, H % 4P == 0, W % 4 == 0; output
  *             [H/4][W/4][1280]): conv_in_w[320][3][3][C], conv_in_b[320], the
  *             RESBLOCK list for 320->320 at HxW, down1_w[320][3][3][320],
@@ -425,6 +449,8 @@ DP_API int dp_block_step(const dp_block_desc* d, dp_block_state* s, const void* 
 #define DP_KERNEL_CONV_SMALL 7 /* direct 3x3 conv for few input channels        */
 #define DP_KERNEL_SPLITK_FINISH 8 /* sum of split-K partials + bias + residual   */
 #define DP_KERNEL_GN_CLUSTER 9  /* GroupNorm, one thread-block cluster per band */
+#define DP_KERNEL_LAYERNORM 10  /* per-token LayerNorm                          */
+#define DP_KERNEL_GEGLU 11      /* gated GELU unit of the feed-forward          */
 
 /*
  * Number of kernel launches one displaced dp_block_step makes for this
@@ -434,6 +460,9 @@ DP_API int dp_block_step(const dp_block_desc* d, dp_block_state* s, const void* 
  *   RESBLOCK: GN1, conv1, GN2, [1x1 shortcut if C != Cout], conv2
  *   ATTN:     GN, q/k/v projection, attention, out projection
  *   UNET_MINI: input copy, conv_in, then its blocks and downsamplers in order
+ *   TRANSFORMER: GN, proj_in, LN, q/k/v projection, attention, out projection,
+ *             LN, query projection, context k/v projection, cross-attention,
+ *             out projection, LN, ff1, GEGLU, ff2, proj_out
  * Negative status on a bad descriptor.
  */
 DP_API int dp_block_launch_count(const dp_block_desc* d);

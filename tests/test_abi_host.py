@@ -269,3 +269,25 @@ def test_token_operators_reject_bad_arguments_on_the_host(B):
     with pytest.raises(B.DPError) as e:   # y overlaps h
         B.dp_geglu(16, 32, 4, 64, stream=0)
     assert e.value.code == B.DP_ERR_INVALID_ARG
+
+
+def test_transformer_block_plan_on_the_host(B):
+    """An SDXL-shaped transformer block: it needs its context sizes, takes 25 pointers, and its
+    launches follow the documented order; the launches' flops add up to the block's."""
+    d = B.dp_block_desc_init(B.TRANSFORMER, 64, 64, 640, 640, 32, 4, 10, B.BF16, 0, 1e-5, 1.0)
+    with pytest.raises(B.DPError, match="set_context"):
+        B.dp_block_workspace_size(d)
+    with pytest.raises(B.DPError):
+        B.dp_block_desc_set_context(d, 77, 100, 2560)     # context width not a multiple of 64
+    B.dp_block_desc_set_context(d, 77, 2048, 2560)
+    assert B.dp_block_weight_count(d) == 25
+    kinds = [B.dp_block_launch_info(d, B.DISPLACED, i)[0] for i in range(B.dp_block_launch_count(d))]
+    assert [k for k in kinds if k != "splitk_finish"] == [
+        "gn_cluster", "linear", "layernorm", "linear", "attn", "linear", "layernorm", "linear", "linear",
+        "attn", "linear", "layernorm", "linear", "geglu", "linear", "linear"]
+    fl = sum(B.dp_block_launch_info(d, B.DISPLACED, i)[1] for i in range(B.dp_block_launch_count(d)))
+    assert abs(fl - B.dp_block_flops(d)) < 1e-6 * fl
+    assert B.dp_block_workspace_size(d) > 64 * 64 * 2560 * 2 * 2
+    dr = B.dp_block_desc_init(B.RESBLOCK, 64, 64, 320, 320, 32, 4, 0, B.BF16, 1, 1e-5, 1.0)
+    with pytest.raises(B.DPError, match="only for TRANSFORMER"):
+        B.dp_block_desc_set_context(dr, 77, 2048, 1280)
