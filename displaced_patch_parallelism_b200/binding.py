@@ -38,7 +38,7 @@ class BlockDesc(ctypes.Structure):
                 ("P", ctypes.c_int), ("heads", ctypes.c_int), ("dtype", ctypes.c_int),
                 ("silu", ctypes.c_int), ("eps", ctypes.c_float), ("w", ctypes.c_float),
                 ("gn_stats", ctypes.c_int), ("ctx_len", ctypes.c_int), ("ctx_dim", ctypes.c_int),
-                ("ff_inner", ctypes.c_int)]
+                ("ff_inner", ctypes.c_int), ("temb_dim", ctypes.c_int)]
 
 
 class BlockState(ctypes.Structure):
@@ -66,12 +66,14 @@ _SIGS = {
     "dp_attn_cross": ([_V, _V, _V, _V, _I, _I, _I, _I, _F, _V, _SZ, _V], _I),
     "dp_layernorm": ([_V, _V, _V, _V, _I, _I, _F, _V], _I),
     "dp_geglu": ([_V, _V, _I, _I, _V], _I),
+    "dp_time_embedding_bias": ([_V, _V, _V, _V, _V, _I, _I, _V], _I),
     "dp_refresh_stale": ([_V, _V, _SZ, _I, _I, _I, _V], _I),
     "dp_refresh_halo": ([_V, _V, _SZ, _I, _I, _I, _I, _V], _I),
     "dp_refresh_stats": ([_V, _V, _V, _I, _I, _V], _I),
     "dp_block_desc_init": ([ctypes.POINTER(BlockDesc), _I, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _F], _I),
     "dp_block_desc_set_gn_stats": ([ctypes.POINTER(BlockDesc), _I], _I),
     "dp_block_desc_set_context": ([ctypes.POINTER(BlockDesc), _I, _I, _I], _I),
+    "dp_block_desc_set_time_embedding": ([ctypes.POINTER(BlockDesc), _I], _I),
     "dp_block_workspace_size": ([ctypes.POINTER(BlockDesc)], _SZ),
     "dp_block_state_init": ([ctypes.POINTER(BlockDesc), ctypes.POINTER(BlockState), _V, _SZ, _V], _I),
     "dp_block_step": ([ctypes.POINTER(BlockDesc), ctypes.POINTER(BlockState), _V, _V,
@@ -218,6 +220,11 @@ def dp_geglu(h, y, T, F, stream=None):
     return _check(lib().dp_geglu(_p(h), _p(y), T, F, _s(stream)))
 
 
+def dp_time_embedding_bias(temb, temb_w, temb_b, conv_b, bias, Ct, Cout, stream=None):
+    return _check(lib().dp_time_embedding_bias(_p(temb), _p(temb_w), _p(temb_b), _p(conv_b),
+                                               _p(bias), Ct, Cout, _s(stream)))
+
+
 def dp_refresh_stale(fresh, stale, row_bytes, rows, P, band=-1, stream=None):
     return _check(lib().dp_refresh_stale(_p(fresh), _p(stale), row_bytes, rows, P, band,
                                          _s(stream)))
@@ -246,6 +253,10 @@ def dp_block_desc_set_gn_stats(d: BlockDesc, variant: int):
 
 def dp_block_desc_set_context(d: BlockDesc, ctx_len: int, ctx_dim: int, ff_inner: int):
     return _check(lib().dp_block_desc_set_context(ctypes.byref(d), ctx_len, ctx_dim, ff_inner))
+
+
+def dp_block_desc_set_time_embedding(d: BlockDesc, temb_dim: int):
+    return _check(lib().dp_block_desc_set_time_embedding(ctypes.byref(d), temb_dim))
 
 
 def dp_block_workspace_size(d: BlockDesc) -> int:
@@ -291,7 +302,7 @@ def dp_block_step_timed(d: BlockDesc, s: BlockState, x, out, weights: Sequence, 
 
 KERNEL_NAMES = {0: "gn_stats", 1: "gn_apply", 2: "gn_fused", 3: "conv", 4: "linear", 5: "attn",
                 6: "copy", 7: "conv_small", 8: "splitk_finish",
-                9: "gn_cluster", 10: "layernorm", 11: "geglu"}
+                9: "gn_cluster", 10: "layernorm", 11: "geglu", 12: "temb"}
 
 
 def dp_block_launch_info(d: BlockDesc, mode: int, i: int):
@@ -318,12 +329,15 @@ class Block:
 
     def __init__(self, kind, H, W, C, Cout=0, G=32, P=4, heads=0, dtype=BF16, silu=True,
                  eps=1e-5, w=1.0, device="cuda", stream=None, gn_stats=GN_STATS_CORRECTED,
-                 context=None):
-        """``context`` = (ctx_len, ctx_dim, ff_inner) for TRANSFORMER blocks."""
+                 context=None, temb_dim=0):
+        """``context`` = (ctx_len, ctx_dim, ff_inner) for TRANSFORMER blocks; ``temb_dim`` the
+        time-embedding width of a RESBLOCK (0: none)."""
         import torch
         self.desc = dp_block_desc_init(kind, H, W, C, Cout, G, P, heads, dtype, silu, eps, w)
         if context is not None:
             dp_block_desc_set_context(self.desc, *context)
+        if temb_dim:
+            dp_block_desc_set_time_embedding(self.desc, temb_dim)
         if gn_stats != GN_STATS_CORRECTED:
             dp_block_desc_set_gn_stats(self.desc, gn_stats)
         self.ws_bytes = dp_block_workspace_size(self.desc)

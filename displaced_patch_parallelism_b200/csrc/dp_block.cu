@@ -10,7 +10,8 @@
 // output of the layer feeding a conv) and reads the stale half; the refresh
 // that replaces the paper's AllGather is a flip of `cur`, so no byte moves.
 //
-// Kinds: GN_CONV, RESBLOCK, ATTN, TRANSFORMER (SDXL-shaped: GroupNorm and
+// Kinds: GN_CONV, RESBLOCK (optionally with an SDXL time embedding added to
+// conv1's output), ATTN, TRANSFORMER (SDXL-shaped: GroupNorm and
 // self-attention with stale context, then per-token LayerNorms, a
 // cross-attention over the text context and a gated feed-forward, none of
 // which need context from other bands), and UNET_MINI, a chain of the others with
@@ -53,6 +54,7 @@ struct Layout {
   size_t act, q, k[2], v[2], o;      // attention buffers
   size_t ha, hb, tn, q2, k2, v2, o2, ffh, ffg;   // TRANSFORMER: residual stream, LN output, cross, FF
   size_t attn_ws;                     // balanced attention split: counters + partials
+  size_t tbias;                       // RESBLOCK with a time embedding: conv1's step bias
   size_t gemm_ws;                     // split-K partials of the convs and projections
   // UNET_MINI: sub-block workspaces and the buffers between them
   size_t xin[2], h0, rb1, d1[2], h1, rb2, h2, at2, d2[2], h3, rb3, h4, at3;
@@ -116,6 +118,7 @@ Layout layout_of(const dp_block_desc* d) {
     for (int i = 0; i < 2; ++i) L.a2[i] = b.take(hw * d->Cout * e);
     L.h = b.take(hw * d->Cout * e);
     if (d->C != d->Cout) L.sc = b.take(hw * d->Cout * e);
+    if (d->temb_dim > 0) L.tbias = b.take(static_cast<size_t>(d->Cout) * sizeof(float));
   } else if (d->kind == DP_BLOCK_TRANSFORMER) {
     const size_t C = d->C, Tk = d->ctx_len, F = d->ff_inner;
     L.gn1 = gn_slots(b, d->P, d->G);
@@ -178,6 +181,10 @@ int desc_check(const dp_block_desc* d) {
   if (d->gn_stats < DP_GN_STATS_CORRECTED || d->gn_stats > DP_GN_STATS_SYNC)
     return set_error(DP_ERR_INVALID_ARG, "block: unknown GroupNorm statistics variant %d", d->gn_stats);
   if (d->H % d->P) return set_error(DP_ERR_UNSUPPORTED, "block: H %% P != 0");
+  if (d->temb_dim < 0 || d->temb_dim > 8192)
+    return set_error(DP_ERR_INVALID_ARG, "block: time-embedding width %d outside [0, 8192]", d->temb_dim);
+  if (d->temb_dim && d->kind != DP_BLOCK_RESBLOCK)
+    return set_error(DP_ERR_INVALID_ARG, "block: a time embedding is only for RESBLOCK blocks");
   if (d->kind == DP_BLOCK_UNET_MINI) {
     if (d->C > 16 || d->C % 2)
       return set_error(DP_ERR_UNSUPPORTED, "block: mini U-Net latent needs an even C <= 16");
@@ -215,7 +222,7 @@ int desc_check(const dp_block_desc* d) {
 
 int weight_count(const dp_block_desc* d) {
   if (d->kind == DP_BLOCK_GN_CONV) return 4;
-  if (d->kind == DP_BLOCK_RESBLOCK) return d->C != d->Cout ? 10 : 8;
+  if (d->kind == DP_BLOCK_RESBLOCK) return (d->C != d->Cout ? 10 : 8) + (d->temb_dim > 0 ? 3 : 0);
   if (d->kind == DP_BLOCK_ATTN) return 6;
   if (d->kind == DP_BLOCK_TRANSFORMER) return 25;
   const MiniDescs m = mini_descs(d);
@@ -228,7 +235,8 @@ double flops_of(const dp_block_desc* d) {
   const double C = d->C, Co = d->Cout;
   if (d->kind == DP_BLOCK_GN_CONV) return 2.0 * hw * Co * 9.0 * C;
   if (d->kind == DP_BLOCK_RESBLOCK)
-    return 2.0 * hw * Co * 9.0 * C + 2.0 * hw * Co * 9.0 * Co + (C != Co ? 2.0 * hw * Co * C : 0.0);
+    return 2.0 * hw * Co * 9.0 * C + 2.0 * hw * Co * 9.0 * Co + (C != Co ? 2.0 * hw * Co * C : 0.0) +
+           2.0 * Co * d->temb_dim;
   if (d->kind == DP_BLOCK_ATTN)
     return 2.0 * hw * 3.0 * C * C + 4.0 * hw * hw * C + 2.0 * hw * C * C;
   if (d->kind == DP_BLOCK_TRANSFORMER) {
@@ -342,12 +350,14 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
   };
   int rc;
   if (d->kind != DP_BLOCK_UNET_MINI && !plan) {
-    // biases (conv_b, conv1_b, conv2_b, short_b; bqkv, bo) may be NULL
+    // biases (conv_b, conv1_b, conv2_b, short_b, temb_b; bqkv, bo, ...) may be NULL
+    const int temb_b = weight_count(d) - 2;   // RESBLOCK with a time embedding: temb_b
     for (int i = 0; i < weight_count(d); ++i) {
       const bool bias = d->kind == DP_BLOCK_ATTN          ? (i == 3 || i == 5)
                         : d->kind == DP_BLOCK_TRANSFORMER ? (i == 3 || i == 7 || i == 9 || i == 15 ||
                                                              i == 19 || i == 21 || i == 23)
-                                                          : (i == 3 || i == 7 || i == 9);
+                                                          : (i == 3 || i == 7 || i == 9 ||
+                                                             (d->temb_dim > 0 && i == temb_b));
       if (!w[i] && !bias) return set_error(DP_ERR_INVALID_ARG, "block: weight %d is NULL", i);
     }
   }
@@ -371,9 +381,28 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
     void* a1f = at<void>(ws, L.a1[f]);
     void* a2f = at<void>(ws, L.a2[f]);
     void* h = at<void>(ws, L.h);
+    const void* b1 = w[3];
+    if (d->temb_dim > 0) {
+      // the step's time embedding (temb_w, temb_b, then temb), folded with
+      // conv1_b into conv1's bias
+      const int t0 = C != Co ? 10 : 8;
+      const int Ct = d->temb_dim;
+      if (plan) {
+        plan->push(DP_KERNEL_TEMB, 2.0 * Co * Ct, (static_cast<double>(Co) * Ct + Ct + 3.0 * Co) * 4.0);
+      } else {
+        float* tb = at<float>(ws, L.tbias);
+        rc = temb_bias_validate(w[t0 + 2], w[t0], w[t0 + 1], w[3], tb, Ct, Co);
+        if (rc) return rc;
+        rc = temb_bias_launch(static_cast<const float*>(w[t0 + 2]), static_cast<const float*>(w[t0]),
+                              static_cast<const float*>(w[t0 + 1]), static_cast<const float*>(w[3]), tb,
+                              Ct, Co, st);
+        if (rc) return rc;
+        b1 = tb;
+      }
+    }
     rc = gn(L.gn1, x, a1f, w[0], w[1], C, 1);
     if (rc) return rc;
-    rc = conv(a1f, at<void>(ws, L.a1[o]), w[2], w[3], nullptr, h, H, W, C, Co, 1);
+    rc = conv(a1f, at<void>(ws, L.a1[o]), w[2], b1, nullptr, h, H, W, C, Co, 1);
     if (rc) return rc;
     rc = gn(L.gn2, h, a2f, w[4], w[5], Co, 1);
     if (rc) return rc;
@@ -574,6 +603,7 @@ int dp_block_desc_init(dp_block_desc* d, int kind, int H, int W, int C, int Cout
   d->ctx_len = 0;
   d->ctx_dim = 0;
   d->ff_inner = 0;
+  d->temb_dim = 0;
   if (kind == DP_BLOCK_TRANSFORMER) return DP_OK;   // checked once dp_block_desc_set_context is called
   return dp::desc_check(d);
 }
@@ -585,6 +615,16 @@ int dp_block_desc_set_context(dp_block_desc* d, int ctx_len, int ctx_dim, int ff
   d->ctx_len = ctx_len;
   d->ctx_dim = ctx_dim;
   d->ff_inner = ff_inner;
+  return dp::desc_check(d);
+}
+
+int dp_block_desc_set_time_embedding(dp_block_desc* d, int temb_dim) {
+  if (!d) return dp::set_error(DP_ERR_INVALID_ARG, "block: null descriptor");
+  if (d->kind != DP_BLOCK_RESBLOCK)
+    return dp::set_error(DP_ERR_INVALID_ARG, "block: a time embedding is only for RESBLOCK blocks");
+  if (temb_dim < 0 || temb_dim > 8192)
+    return dp::set_error(DP_ERR_INVALID_ARG, "block: time-embedding width %d outside [0, 8192]", temb_dim);
+  d->temb_dim = temb_dim;
   return dp::desc_check(d);
 }
 

@@ -35,6 +35,12 @@ int linear_launch(const void* x, const void* weight, const float* bias, const vo
 int attn_validate(const void* q, const void* kf, const void* vf, const void* ks, const void* vs,
                   const void* o, int T, int heads, int head_dim, int P, int mode);
 size_t attn_workspace_bytes();
+// bias[c] = conv_b[c] + temb_b[c] + temb_w[c] . silu(temb) (fp32; temb_b and
+// conv_b may be null); the validate call checks sizes, nulls and aliasing
+int temb_bias_validate(const void* temb, const void* temb_w, const void* temb_b, const void* conv_b,
+                       const void* bias, int Ct, int Cout);
+int temb_bias_launch(const float* temb, const float* temb_w, const float* temb_b, const float* conv_b,
+                     float* bias, int Ct, int Cout, cudaStream_t st);
 // attention of T queries over Tk keys (Tk = T: self-attention; with mode SYNC
 // and P = 1 and Tk != T: cross-attention over a context every band sees)
 int attn_launch_tk(const void* q, const void* kf, const void* vf, const void* ks, const void* vs,

@@ -25,7 +25,8 @@ def _conv(w, dtype, device):
 def block_weights(kind: str, wts: Dict, dtype: torch.dtype = torch.bfloat16, device="cuda",
                   prefix: str = "") -> List[torch.Tensor]:
     """Device tensors in the order ``dp_block_step`` documents for ``kind`` (a TRANSFORMER
-    block's per-step text context, its 25th pointer, is appended by the caller)."""
+    block's per-step text context, its 25th pointer, and a RESBLOCK's per-step time
+    embedding, its last pointer, are appended by the caller)."""
     g = lambda n: wts[prefix + n]
     f32 = torch.float32
     if kind == "gn_conv":
@@ -41,6 +42,8 @@ def block_weights(kind: str, wts: Dict, dtype: torch.dtype = torch.bfloat16, dev
             sw = sw if isinstance(sw, torch.Tensor) else torch.as_tensor(sw)
             out += [_t(sw.reshape(sw.shape[0], sw.shape[1]), dtype, device),
                     _t(g("short_b"), f32, device)]
+        if (prefix + "temb_w") in wts:   # the step's time embedding is appended by the caller
+            out += [_t(g("temb_w"), f32, device), _t(g("temb_b"), f32, device)]
         return out
     if kind == "attn":
         cat = lambda *xs: torch.cat([x if isinstance(x, torch.Tensor) else torch.as_tensor(x) for x in xs])

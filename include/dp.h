@@ -285,6 +285,22 @@ DP_API int dp_attn_cross(const void* q, const void* k, const void* v, void* o, i
                   void* stream);
 
 /* ------------------------------------------------------------------------
+ * Time-embedding term of an SDXL-shaped ResBlock ("next" item: the pages name
+ * SDXL as the model; its ResBlocks add a projection of the step's time
+ * embedding to the first conv's output, one vector per step that every band
+ * shares, so it has no stale copy):
+ *   bias[c] = conv_b[c] + temb_b[c] + sum_j temb_w[c][j] * silu(temb[j])
+ * The result is the first conv's bias for the step.
+ *  temb    [Ct] fp32, device;   temb_w [Cout][Ct] fp32 row-major, device;
+ *  temb_b, conv_b [Cout] fp32, device, or NULL (taken as 0);
+ *  bias    [Cout] fp32, device, written; may not overlap any input.
+ *  1 <= Ct <= 8192, Cout >= 1.  fp32 arithmetic; asynchronous on `stream`.
+ *  DP_ERR_INVALID_ARG on a null temb / temb_w / bias, bad sizes or overlap.
+ * ---------------------------------------------------------------------- */
+DP_API int dp_time_embedding_bias(const float* temb, const float* temb_w, const float* temb_b,
+                                  const float* conv_b, float* bias, int Ct, int Cout, void* stream);
+
+/* ------------------------------------------------------------------------
  * Per-token operators of an SDXL-shaped transformer block ("next" item: the
  * pages name SDXL as the model; they act on each token alone, so every band
  * runs them on its fresh tokens with no stale context).
@@ -357,6 +373,7 @@ typedef struct dp_block_desc {
   int ctx_len;    /* TRANSFORMER: text context tokens (Tk)        */
   int ctx_dim;    /* TRANSFORMER: text context width (Cctx)       */
   int ff_inner;   /* TRANSFORMER: feed-forward inner width (F)    */
+  int temb_dim;   /* RESBLOCK: time-embedding width (0: none)     */
 } dp_block_desc;
 
 /*
@@ -367,6 +384,17 @@ typedef struct dp_block_desc {
  * 0.  DP_ERR_INVALID_ARG on a null descriptor or bad sizes.
  */
 DP_API int dp_block_desc_set_context(dp_block_desc* d, int ctx_len, int ctx_dim, int ff_inner);
+
+/*
+ * RESBLOCK blocks: the width Ct of the step's time embedding (0 switches it
+ * off, the default).  With Ct > 0 the block takes three more weight pointers,
+ * temb_w[Cout][Ct], temb_b[Cout] and the step's temb[Ct] (fp32; temb_b may be
+ * NULL), and
+ * adds temb_w silu(temb) + temb_b to every pixel of conv1's output (one extra
+ * launch, dp_time_embedding_bias).  DP_ERR_INVALID_ARG on a null descriptor,
+ * another kind, or Ct outside [0, 8192].
+ */
+DP_API int dp_block_desc_set_time_embedding(dp_block_desc* d, int temb_dim);
 
 typedef struct dp_block_state {
   void* workspace;        /* device memory of dp_block_workspace_size() bytes */
@@ -410,7 +438,9 @@ DP_API int dp_block_state_init(const dp_block_desc* d, dp_block_state* s, void* 
  *   GN_CONV:  gn_gamma[C], gn_beta[C], conv_w[Cout][3][3][C], conv_b[Cout]
  *   RESBLOCK: gn1_gamma[C], gn1_beta[C], conv1_w[Cout][3][3][C], conv1_b[Cout],
  *             gn2_gamma[Cout], gn2_beta[Cout], conv2_w[Cout][3][3][Cout],
- *             conv2_b[Cout], then if C != Cout: short_w[Cout][C], short_b[Cout]
+ *             conv2_b[Cout], then if C != Cout: short_w[Cout][C], short_b[Cout],
+ *             then if temb_dim > 0: temb_w[Cout][temb_dim], temb_b[Cout] and the
+ *             step's time embedding temb[temb_dim] (fp32; temb_b may be NULL)
  *   ATTN:     gn_gamma[C], gn_beta[C], wqkv[3C][C] (the q, k and v (out, in)
  *             matrices stacked), bqkv[3C], wo[C][C], bo[C]
  *   TRANSFORMER (C == heads * 64, (H*W/P) % 128 == 0, (H*W) % 256 == 0):
@@ -451,6 +481,7 @@ DP_API int dp_block_step(const dp_block_desc* d, dp_block_state* s, const void* 
 #define DP_KERNEL_GN_CLUSTER 9  /* GroupNorm, one thread-block cluster per band */
 #define DP_KERNEL_LAYERNORM 10  /* per-token LayerNorm                          */
 #define DP_KERNEL_GEGLU 11      /* gated GELU unit of the feed-forward          */
+#define DP_KERNEL_TEMB 12       /* time-embedding bias of a ResBlock's conv1     */
 
 /*
  * Number of kernel launches one displaced dp_block_step makes for this

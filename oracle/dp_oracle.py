@@ -33,6 +33,10 @@ Readings of what the pages leave open (each also listed in the design notes):
       other bands per mode; stride-2 output bands are Ho/P rows
   R12 the GroupNorm ablation's alternatives for displaced steps (band-local,
       stale-only and exact statistics): see ``gn_variant_mode``
+  R13 the pages name SDXL but not its blocks' insides: the plainest SDXL
+      transformer block (``transformer_step``) and ResBlock time embedding
+      (``resblock_step``'s ``temb``); only GroupNorm statistics and
+      self-attention keys/values cross bands
 
 Parity pins (the tests under tests/test_oracle_*.py): P = 1 reduces to the
 library full-image block (torch group_norm / conv2d / softmax attention);
@@ -394,6 +398,14 @@ def gn_conv_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float
     return out
 
 
+def time_embedding_term(temb, temb_w, temb_b) -> np.ndarray:
+    """temb_w silu(temb) + temb_b: the per-channel term an SDXL ResBlock adds to its first
+    conv's output (reading R13), with temb_w stored (out, in); temb_b may be None."""
+    tv = _a(temb)
+    return linear((tv / (1.0 + np.exp(-tv)))[None, :], _a(temb_w),
+                  None if temb_b is None else _a(temb_b))[0]
+
+
 def resblock_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float,
                   mode: int, storage: str, trace: Optional[Dict] = None, prefix: str = "",
                   final_storage: Optional[str] = None, gn_stats: int = GN_STATS_CORRECTED,
@@ -412,8 +424,7 @@ def resblock_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: floa
     a1 = store(a1, storage)
     b1 = W_("conv1_b")
     if temb is not None:
-        tv = _a(temb)
-        b1 = b1 + linear((tv / (1.0 + np.exp(-tv)))[None, :], W_("temb_w"), W_("temb_b"))[0]
+        b1 = b1 + time_embedding_term(temb, W_("temb_w"), W_("temb_b"))
     h = store(conv3x3_halo(a1, state.get("a1_stale"), W_("conv1_w"), b1, None, P, mode), storage)
     a2, f2 = _gn(gn2, h, W_("gn2_gamma"), W_("gn2_beta"), P, G, eps, w, True, mode, trace,
                  prefix + "gn2", gn_stats)

@@ -291,3 +291,44 @@ def test_transformer_block_plan_on_the_host(B):
     dr = B.dp_block_desc_init(B.RESBLOCK, 64, 64, 320, 320, 32, 4, 0, B.BF16, 1, 1e-5, 1.0)
     with pytest.raises(B.DPError, match="only for TRANSFORMER"):
         B.dp_block_desc_set_context(dr, 77, 2048, 1280)
+
+
+def test_time_embedding_rejects_bad_arguments_on_the_host(B):
+    A = 1 << 20                                   # fake, never dereferenced: checks run first
+    for args in [(0, A, 0, 0, 2 * A, 8, 4),      # null temb
+                 (A, A, 0, 0, 0, 8, 4),           # null bias
+                 (A, 2 * A, 0, 0, 3 * A, 0, 4),   # Ct = 0
+                 (A, 2 * A, 0, 0, 3 * A, 8193, 4),
+                 (A, 2 * A, 0, 0, 3 * A, 8, 0),   # Cout = 0
+                 (A, 2 * A, 0, 0, A + 16, 8, 4),  # bias overlaps temb
+                 (A, 2 * A, 0, 3 * A, 3 * A + 8, 8, 4)]:   # bias overlaps conv_b
+        with pytest.raises(B.DPError) as e:
+            B.dp_time_embedding_bias(*args, stream=0)
+        assert e.value.code == B.DP_ERR_INVALID_ARG, args
+
+
+def test_resblock_time_embedding_plan_on_the_host(B):
+    """A RESBLOCK with a time embedding takes temb_w, temb_b and temb after its other
+    weights, launches the bias kernel first, and counts its flops."""
+    d = B.dp_block_desc_init(B.RESBLOCK, 64, 64, 320, 640, 32, 4, 0, B.BF16, 1, 1e-5, 1.0)
+    n0, f0, w0 = B.dp_block_launch_count(d), B.dp_block_flops(d), B.dp_block_workspace_size(d)
+    assert B.dp_block_weight_count(d) == 10
+    B.dp_block_desc_set_time_embedding(d, 1280)
+    assert B.dp_block_weight_count(d) == 13
+    assert B.dp_block_launch_count(d) == n0 + 1
+    assert B.dp_block_launch_info(d, B.DISPLACED, 0)[:2] == ("temb", 2.0 * 640 * 1280)
+    assert B.dp_block_flops(d) == f0 + 2.0 * 640 * 1280
+    fl = sum(B.dp_block_launch_info(d, B.DISPLACED, i)[1] for i in range(B.dp_block_launch_count(d)))
+    assert abs(fl - B.dp_block_flops(d)) < 1e-6 * fl
+    assert B.dp_block_workspace_size(d) >= w0 + 640 * 4
+    B.dp_block_desc_set_time_embedding(d, 0)       # off again: the plain ResBlock
+    assert B.dp_block_weight_count(d) == 10 and B.dp_block_launch_count(d) == n0
+    for bad in (-1, 8193):
+        with pytest.raises(B.DPError):
+            B.dp_block_desc_set_time_embedding(d, bad)
+    da = B.dp_block_desc_init(B.ATTN, 64, 64, 640, 640, 32, 4, 10, B.BF16, 0, 1e-5, 1.0)
+    with pytest.raises(B.DPError, match="only for RESBLOCK"):
+        B.dp_block_desc_set_time_embedding(da, 1280)
+    da.temb_dim = 1280                              # set behind the setter's back
+    with pytest.raises(B.DPError, match="only for RESBLOCK"):
+        B.dp_block_workspace_size(da)

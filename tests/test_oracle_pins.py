@@ -691,6 +691,18 @@ def test_transformer_displaced_and_naive_invariants():
     assert 0 < err(DISPLACED) < err(NAIVE)
 
 
+def test_time_embedding_term_equals_library():
+    """temb_w silu(temb) + temb_b is the library's linear of the library's SiLU; without
+    temb_b it is the bare product, and a zero embedding leaves only temb_b (silu(0) = 0)."""
+    r = rng(94)
+    Ct, Co = 37, 11
+    tw, tb, t = r.standard_normal((Co, Ct)), r.standard_normal(Co), 3 * r.standard_normal(Ct)
+    ref = F.linear(F.silu(T64(t)), T64(tw), T64(tb)).numpy()
+    np.testing.assert_allclose(O.time_embedding_term(t, tw, tb), ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(O.time_embedding_term(t, tw, None), ref - tb, rtol=0, atol=1e-12)
+    np.testing.assert_array_equal(O.time_embedding_term(np.zeros(Ct), tw, tb), tb)
+
+
 @pytest.mark.parametrize("mode", [SYNC, DISPLACED])
 def test_p1_resblock_time_embedding_equals_library(mode):
     """A time embedding adds temb_w silu(temb) + temb_b to every pixel of conv1's output."""
