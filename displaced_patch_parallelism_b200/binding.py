@@ -67,6 +67,7 @@ _SIGS = {
     "dp_layernorm": ([_V, _V, _V, _V, _I, _I, _F, _V], _I),
     "dp_geglu": ([_V, _V, _I, _I, _V], _I),
     "dp_time_embedding_bias": ([_V, _V, _V, _V, _V, _I, _I, _V], _I),
+    "dp_ddim_step": ([_V, _V, _V, _SZ, ctypes.c_double, ctypes.c_double, _I, _V], _I),
     "dp_refresh_stale": ([_V, _V, _SZ, _I, _I, _I, _V], _I),
     "dp_refresh_halo": ([_V, _V, _SZ, _I, _I, _I, _I, _V], _I),
     "dp_refresh_stats": ([_V, _V, _V, _I, _I, _V], _I),
@@ -223,6 +224,11 @@ def dp_geglu(h, y, T, F, stream=None):
 def dp_time_embedding_bias(temb, temb_w, temb_b, conv_b, bias, Ct, Cout, stream=None):
     return _check(lib().dp_time_embedding_bias(_p(temb), _p(temb_w), _p(temb_b), _p(conv_b),
                                                _p(bias), Ct, Cout, _s(stream)))
+
+
+def dp_ddim_step(x, eps, x_prev, n, abar_t, abar_prev, dtype, stream=None):
+    return _check(lib().dp_ddim_step(_p(x), _p(eps), _p(x_prev), n, abar_t, abar_prev, dtype,
+                                     _s(stream)))
 
 
 def dp_refresh_stale(fresh, stale, row_bytes, rows, P, band=-1, stream=None):

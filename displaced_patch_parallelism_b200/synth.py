@@ -2,7 +2,8 @@
 
 This module is shared by the CPU oracle's tests, the CUDA parity tests and the
 benchmark.  It holds no arithmetic of the method itself: only random draws, the
-bf16 storage rounding of those draws, and the workload shapes.
+bf16 storage rounding of those draws, the workload shapes and the sampler's noise
+schedule (``ddim_alpha_bars``, an input of the sampler update).
 
 The shapes stand in for the SDXL workloads that "DistriFusion: Distributed
 Parallel Inference for High-Resolution Diffusion Models" (study.space summary,
@@ -238,6 +239,24 @@ class InputStream:
             j = len(self._chain)
             self._chain.append(self._chain[-1] + randn(self.shape, self.wl.drift_seed(j), self.wl.drift))
         return store(self._chain[k], self.wl.dtype)
+
+
+def ddim_alpha_bars(steps: int = 50, train_steps: int = 1000, beta_start: float = 0.00085,
+                    beta_end: float = 0.012) -> List[Tuple[float, float]]:
+    """(abar_t, abar_prev) of each sampler step, first to last: the scaled-linear noise
+    schedule of the Stable Diffusion family (betas evenly spaced in sqrt between beta_start
+    and beta_end over train_steps, abar = cumulative product of 1 - beta) at `steps` evenly
+    spaced timesteps from the noisiest down; the last step's previous level is abar = 1
+    (the clean sample).  Sampler inputs only."""
+    betas = torch.linspace(beta_start ** 0.5, beta_end ** 0.5, train_steps, dtype=torch.float64) ** 2
+    abar = torch.cumprod(1.0 - betas, dim=0)
+    stride = train_steps // steps
+    ts = [train_steps - 1 - k * stride for k in range(steps)]
+    out = []
+    for k, t in enumerate(ts):
+        prev = abar[ts[k + 1]] if k + 1 < steps else 1.0
+        out.append((float(abar[t]), float(prev)))
+    return out
 
 
 def nchw_to_nhwc(t: torch.Tensor) -> torch.Tensor:

@@ -301,6 +301,26 @@ DP_API int dp_time_embedding_bias(const float* temb, const float* temb_w, const 
                                   const float* conv_b, float* bias, int Ct, int Cout, void* stream);
 
 /* ------------------------------------------------------------------------
+ * The sampler update between two denoising steps ("next" item: the pages'
+ * results use a 50-step DDIM sampler; the update is deterministic DDIM, eta =
+ * 0, of Song, Meng and Ermon, "Denoising Diffusion Implicit Models"):
+ *   x_prev = sqrt(abar_prev) (x - sqrt(1 - abar_t) eps) / sqrt(abar_t)
+ *            + sqrt(1 - abar_prev) eps
+ * elementwise over n values; the host folds the schedule into two fp32
+ * coefficients (computed in double) and the kernel does one fp32 FMA per
+ * element.
+ *  x, eps, x_prev  n values of `dtype` (DP_BF16 or DP_FP32), device, 16-byte
+ *                  aligned; x_prev may BE x (in place) but may not otherwise
+ *                  overlap x or eps.  Any n (a ragged tail is handled).
+ *  abar_t, abar_prev  cumulative alpha products of the current and the
+ *                  previous timestep, each in (0, 1].
+ * DP_ERR_INVALID_ARG on null pointers, bad dtype, abar out of range or
+ * overlap; DP_ERR_UNSUPPORTED on misalignment.  n == 0 launches nothing.
+ * ---------------------------------------------------------------------- */
+DP_API int dp_ddim_step(const void* x, const void* eps, void* x_prev, size_t n, double abar_t,
+                        double abar_prev, int dtype, void* stream);
+
+/* ------------------------------------------------------------------------
  * Per-token operators of an SDXL-shaped transformer block ("next" item: the
  * pages name SDXL as the model; they act on each token alone, so every band
  * runs them on its fresh tokens with no stale context).

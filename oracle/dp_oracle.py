@@ -33,6 +33,8 @@ Readings of what the pages leave open (each also listed in the design notes):
       other bands per mode; stride-2 output bands are Ho/P rows
   R12 the GroupNorm ablation's alternatives for displaced steps (band-local,
       stale-only and exact statistics): see ``gn_variant_mode``
+  R15 the pages' sampler is "50-step DDIM" with no update printed: the
+      deterministic DDIM step (``ddim_step``), alpha-bar values from the caller
   R13 the pages name SDXL but not its blocks' insides: the plainest SDXL
       transformer block (``transformer_step``) and ResBlock time embedding
       (``resblock_step``'s ``temb``); only GroupNorm statistics and
@@ -404,6 +406,17 @@ def time_embedding_term(temb, temb_w, temb_b) -> np.ndarray:
     tv = _a(temb)
     return linear((tv / (1.0 + np.exp(-tv)))[None, :], _a(temb_w),
                   None if temb_b is None else _a(temb_b))[0]
+
+
+def ddim_step(x, eps, abar_t: float, abar_prev: float) -> np.ndarray:
+    """The sampler update between two denoising steps (reading R15): deterministic DDIM,
+    eta = 0 (Song, Meng and Ermon, "Denoising Diffusion Implicit Models", section 4.1 with
+    sigma = 0), the sampler of the pages' 50-step DDIM results (atlas.scime.ai summary, Key
+    results).  The clean sample is predicted from x and the noise estimate, then put back at
+    the previous timestep's noise level with the same noise estimate."""
+    x, eps = _a(x), _a(eps)
+    x0 = (x - math.sqrt(1.0 - abar_t) * eps) / math.sqrt(abar_t)
+    return math.sqrt(abar_prev) * x0 + math.sqrt(1.0 - abar_prev) * eps
 
 
 def resblock_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float,

@@ -332,3 +332,20 @@ def test_resblock_time_embedding_plan_on_the_host(B):
     da.temb_dim = 1280                              # set behind the setter's back
     with pytest.raises(B.DPError, match="only for RESBLOCK"):
         B.dp_block_workspace_size(da)
+
+
+def test_ddim_step_rejects_bad_arguments_on_the_host(B):
+    A = 1 << 20                                   # fake, never dereferenced: checks run first
+    bad = [((0, 2 * A, 3 * A, 64, 0.5, 0.6, B.BF16), B.DP_ERR_INVALID_ARG),    # null x
+           ((A, 2 * A, 3 * A, 64, 0.5, 0.6, 7), B.DP_ERR_INVALID_ARG),         # dtype
+           ((A, 2 * A, 3 * A, 64, 0.0, 0.6, B.BF16), B.DP_ERR_INVALID_ARG),    # abar_t = 0
+           ((A, 2 * A, 3 * A, 64, 0.5, 1.5, B.BF16), B.DP_ERR_INVALID_ARG),    # abar_prev > 1
+           ((A, 2 * A, 3 * A, 64, float("nan"), 0.6, B.BF16), B.DP_ERR_INVALID_ARG),
+           ((A, 2 * A, 3 * A + 8, 64, 0.5, 0.6, B.BF16), B.DP_ERR_UNSUPPORTED),  # misaligned
+           ((A, 2 * A, 2 * A + 64, 64, 0.5, 0.6, B.BF16), B.DP_ERR_INVALID_ARG),  # overlaps eps
+           ((A, 2 * A, A + 64, 64, 0.5, 0.6, B.FP32), B.DP_ERR_INVALID_ARG)]      # partly overlaps x
+    for args, code in bad:
+        with pytest.raises(B.DPError) as e:
+            B.dp_ddim_step(*args, stream=0)
+        assert e.value.code == code, args
+    B.dp_ddim_step(A, 2 * A, A, 0, 0.5, 0.6, B.BF16, stream=0)   # in place, n = 0: nothing to do

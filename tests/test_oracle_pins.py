@@ -724,3 +724,33 @@ def test_p1_resblock_time_embedding_equals_library(mode):
     # without the embedding the block is the plain ResBlock
     np.testing.assert_allclose(O.resblock_step({}, x, w, 1, G, 1e-5, 1.0, SYNC, "none"),
                                lib_resblock(x, w, G, 1e-5), rtol=0, atol=1e-11)
+
+
+def test_ddim_step_moves_exact_noise_to_the_previous_level():
+    """With the exact noise of x_t = sqrt(abar_t) x0 + sqrt(1 - abar_t) e, the deterministic
+    DDIM step lands exactly on sqrt(abar_prev) x0 + sqrt(1 - abar_prev) e: the defining
+    property of the update (the same x0 and the same noise, one level less noisy)."""
+    r = rng(95)
+    x0, e = r.standard_normal((3, 5, 7)), r.standard_normal((3, 5, 7))
+    for abar_t, abar_prev in [(0.0047, 0.0059), (0.3, 0.5), (0.98, 1.0)]:
+        xt = math.sqrt(abar_t) * x0 + math.sqrt(1 - abar_t) * e
+        want = math.sqrt(abar_prev) * x0 + math.sqrt(1 - abar_prev) * e
+        np.testing.assert_allclose(O.ddim_step(xt, e, abar_t, abar_prev), want, rtol=0, atol=1e-12)
+    # abar_prev = 1: the step returns the predicted clean sample itself
+    np.testing.assert_allclose(O.ddim_step(math.sqrt(0.4) * x0 + math.sqrt(0.6) * e, e, 0.4, 1.0), x0,
+                               rtol=0, atol=1e-12)
+
+
+def test_ddim_step_identity_and_composition():
+    """No change of level leaves x unchanged for any noise estimate; with a fixed noise
+    estimate, two steps t -> s -> r equal the one step t -> r (the update is a change of
+    noise level along one line); the step is affine in (x, eps)."""
+    r = rng(96)
+    x, e = r.standard_normal(40), r.standard_normal(40)
+    np.testing.assert_allclose(O.ddim_step(x, e, 0.37, 0.37), x, rtol=0, atol=1e-13)
+    two = O.ddim_step(O.ddim_step(x, e, 0.1, 0.25), e, 0.25, 0.7)
+    np.testing.assert_allclose(two, O.ddim_step(x, e, 0.1, 0.7), rtol=0, atol=1e-12)
+    x2, e2 = r.standard_normal(40), r.standard_normal(40)
+    lin = O.ddim_step(2 * x - x2, 2 * e - e2, 0.2, 0.3)
+    np.testing.assert_allclose(lin, 2 * O.ddim_step(x, e, 0.2, 0.3) - O.ddim_step(x2, e2, 0.2, 0.3),
+                               rtol=0, atol=1e-12)
