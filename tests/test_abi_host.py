@@ -349,3 +349,30 @@ def test_ddim_step_rejects_bad_arguments_on_the_host(B):
             B.dp_ddim_step(*args, stream=0)
         assert e.value.code == code, args
     B.dp_ddim_step(A, 2 * A, A, 0, 0.5, 0.6, B.BF16, stream=0)   # in place, n = 0: nothing to do
+
+
+def test_binding_structs_match_the_header(B, tmp_path):
+    """Every field of dp_block_desc and dp_block_state sits at the same offset, and each struct
+    has the same size, in the C header (compiled by gcc) and in the ctypes binding."""
+    import shutil
+    import subprocess
+    if not shutil.which("gcc"):
+        pytest.skip("no C compiler")
+    structs = {"dp_block_desc": B.BlockDesc, "dp_block_state": B.BlockState}
+    lines = []
+    for cname, py in structs.items():
+        lines.append(f'  printf("{cname} sizeof %zu\\n", sizeof({cname}));')
+        for field, _ in py._fields_:
+            lines.append(f'  printf("{cname} {field} %zu\\n", offsetof({cname}, {field}));')
+    src = tmp_path / "layout.c"
+    src.write_text("#include <stddef.h>\n#include <stdio.h>\n#include \"dp.h\"\nint main(void) {\n" +
+                   "\n".join(lines) + "\n  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I" + os.path.join(ROOT, "include"),
+                    str(src), "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
+    for row in filter(None, out):
+        cname, field, value = row.split()
+        py = structs[cname]
+        want = ctypes.sizeof(py) if field == "sizeof" else getattr(py, field).offset
+        assert int(value) == want, (cname, field, int(value), want)
