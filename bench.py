@@ -148,13 +148,26 @@ def job_tflops(world_size, flops_per_step, steps, total_ms):
 
 def block_kind(B, wl):
     return {"gn_conv": B.GN_CONV, "resblock": B.RESBLOCK, "attn": B.ATTN,
-            "unet_mini": B.UNET_MINI}[wl.kind]
+            "unet_mini": B.UNET_MINI, "transformer": B.TRANSFORMER}[wl.kind]
+
+
+def wl_context(wl):
+    """(ctx_len, ctx_dim, ff_inner) of a transformer workload, else None."""
+    return (wl.ctx_len, wl.ctx_dim, wl.ff_inner) if wl.kind == "transformer" else None
+
+
+def oracle_context(wl):
+    """A transformer workload's text context for the oracle (fp64), else None."""
+    from displaced_patch_parallelism_b200 import synth
+    return synth.context(wl).double().numpy() if wl.kind == "transformer" else None
 
 
 def block_desc(B, wl, H=None):
     d = B.dp_block_desc_init(block_kind(B, wl), H or wl.H, wl.W, wl.C, wl.cout, wl.G, wl.P,
                              wl.heads, B.BF16 if wl.dtype == "bf16" else B.FP32, wl.silu,
                              wl.eps, 1.0)
+    if wl_context(wl):
+        B.dp_block_desc_set_context(d, *wl_context(wl))
     B.dp_block_desc_set_gn_stats(d, GN_STATS)
     return d
 
@@ -172,14 +185,15 @@ def cpu_baseline_ours(wl, seconds):
     from oracle import dp_oracle as O
     wts = {n: v.double().numpy() for n, v in synth.make_weights(wl).items()}
     xs = synth.InputStream(wl)
+    ctx = oracle_context(wl)
     st = {}
     O.block_step(wl.kind, st, xs.x(0)[0], wts, wl.P, wl.G, wl.eps, 1.0, synth.SYNC, wl.dtype,
-                 heads=wl.heads, silu=wl.silu)
+                 heads=wl.heads, silu=wl.silu, ctx=ctx)
     x1 = xs.x(1)[0]
     reps, t0 = 0, time.perf_counter()
     while True:
         O.block_step(wl.kind, st, x1, wts, wl.P, wl.G, wl.eps, 1.0, synth.DISPLACED, wl.dtype,
-                     heads=wl.heads, silu=wl.silu, gn_stats=GN_STATS)
+                     heads=wl.heads, silu=wl.silu, gn_stats=GN_STATS, ctx=ctx)
         reps += 1
         el = time.perf_counter() - t0
         if el >= seconds:
@@ -200,6 +214,7 @@ def run_reference(args, wl):
     from oracle import dp_oracle as O
     budget = 150.0
     cores = len(os.sched_getaffinity(0))
+    ctx = oracle_context(wl)
 
     def crop(rows_per_band):
         return dataclasses.replace(wl, H=wl.P * rows_per_band)
@@ -209,14 +224,14 @@ def run_reference(args, wl):
         xs = synth.InputStream(w)
         st = {}
         O.block_step(w.kind, st, xs.x(0)[0], wts, w.P, w.G, w.eps, 1.0, synth.SYNC, w.dtype,
-                     heads=w.heads, silu=w.silu)
+                     heads=w.heads, silu=w.silu, ctx=ctx)
         t0 = time.perf_counter()
         O.block_step(w.kind, st, xs.x(1)[0], wts, w.P, w.G, w.eps, 1.0, synth.DISPLACED, w.dtype,
-                     heads=w.heads, silu=w.silu, gn_stats=GN_STATS)
+                     heads=w.heads, silu=w.silu, gn_stats=GN_STATS, ctx=ctx)
         return time.perf_counter() - t0, wts, st, xs
 
     hb = wl.H // wl.P
-    if wl.kind == "attn":
+    if wl.kind in ("attn", "transformer"):
         rows = hb  # attention blocks need whole 128-token tiles: keep the full image
     else:
         t_small, *_ = one_step_time(crop(2))
@@ -228,11 +243,11 @@ def run_reference(args, wl):
     x = xs.x(2)[0]
     for _ in range(args.warmup):
         O.block_step(w.kind, st, x, wts, w.P, w.G, w.eps, 1.0, synth.DISPLACED, w.dtype,
-                     heads=w.heads, silu=w.silu, gn_stats=GN_STATS)
+                     heads=w.heads, silu=w.silu, gn_stats=GN_STATS, ctx=ctx)
     t0 = time.perf_counter()
     for _ in range(args.steps):
         O.block_step(w.kind, st, x, wts, w.P, w.G, w.eps, 1.0, synth.DISPLACED, w.dtype,
-                     heads=w.heads, silu=w.silu, gn_stats=GN_STATS)
+                     heads=w.heads, silu=w.silu, gn_stats=GN_STATS, ctx=ctx)
     el = time.perf_counter() - t0
     flops = wl_flops(wl, w.H)
     value = flops * args.steps / el / 1e12
@@ -271,9 +286,11 @@ def run_ours(args, wl):
     tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
     wts = synth.make_weights(wl)
     dw = block_weights(wl.kind, wts, tdt, dev)
+    if wl.kind == "transformer":     # the step's text context is the last pointer
+        dw.append(synth.context(wl).to(tdt).to(dev))
     blk = B.Block(block_kind(B, wl), wl.H, wl.W, wl.C, wl.cout, wl.G, wl.P, wl.heads,
                   B.BF16 if wl.dtype == "bf16" else B.FP32, wl.silu, wl.eps, 1.0, device=dev,
-                  gn_stats=GN_STATS)
+                  gn_stats=GN_STATS, context=wl_context(wl))
     xs = synth.InputStream(wl)
     pool = 4
     host_x = [synth.nchw_to_nhwc(xs.x(k)).to(tdt).pin_memory() for k in range(pool)]

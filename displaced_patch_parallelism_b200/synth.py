@@ -91,6 +91,9 @@ class Workload:
     drift_seed_base: int = 1000
     weight_seed: int = 2
     first_drift_seed: Optional[int] = None  # overrides drift_seed_base + 1
+    ctx_len: int = 0          # transformer: text context tokens
+    ctx_dim: int = 0          # transformer: text context width
+    ff_inner: int = 0         # transformer: feed-forward inner width
 
     @property
     def cout(self) -> int:
@@ -117,6 +120,12 @@ class Workload:
                     ("wv", (C, C), 0.02), ("wo", (C, C), 0.02)]
         if self.kind == "unet_mini":
             return unet_mini_weight_specs(self.C)
+        if self.kind == "transformer":
+            Cc, F = self.ctx_dim, self.ff_inner
+            sq = [(n, (C, C), C ** -0.5) for n in ("proj_in_w", "wq", "wk", "wv", "wo", "cq_w")]
+            return sq + [("ck_w", (C, Cc), Cc ** -0.5), ("cv_w", (C, Cc), Cc ** -0.5),
+                         ("co_w", (C, C), C ** -0.5), ("ff1_w", (2 * F, C), C ** -0.5),
+                         ("ff2_w", (C, F), F ** -0.5), ("proj_out_w", (C, C), C ** -0.5)]
         raise ValueError(self.kind)
 
 
@@ -153,6 +162,12 @@ WORKLOADS: Dict[str, Workload] = {
     "attn_640x64x64": Workload(
         name="attn_640x64x64", kind="attn", C=640, H=64, W=64, P=4, heads=10,
         head_dim=64, silu=False, steps=50, warmup=4, drift=0.05),
+    # SDXL 1024 px transformer block shape ("next" item; not a headline workload): 640
+    # channels at 64x64, 10 heads, a 77-token text context of width 2048, feed-forward 4C
+    "transformer_640x64x64": Workload(
+        name="transformer_640x64x64", kind="transformer", C=640, H=64, W=64, P=4, heads=10,
+        head_dim=64, silu=False, steps=50, warmup=4, drift=0.05, ctx_len=77, ctx_dim=2048,
+        ff_inner=2560),
     "gn_conv_320x480x480": Workload(
         name="gn_conv_320x480x480", kind="gn_conv", C=320, H=480, W=480, P=8,
         steps=50, warmup=4, drift=0.05),
@@ -218,7 +233,19 @@ def affine_specs(wl: Workload) -> List[Tuple[str, int, str]]:
                   (pre + ".bq", c, "bias"), (pre + ".bk", c, "bias"),
                   (pre + ".bv", c, "bias"), (pre + ".bo", c, "bias")]
         return s
+    if wl.kind == "transformer":
+        return [("gn_gamma", C, "gamma"), ("gn_beta", C, "beta"), ("proj_in_b", C, "bias"),
+                ("ln1_g", C, "gamma"), ("ln1_b", C, "beta"), ("bq", C, "bias"), ("bk", C, "bias"),
+                ("bv", C, "bias"), ("bo", C, "bias"), ("ln2_g", C, "gamma"), ("ln2_b", C, "beta"),
+                ("co_b", C, "bias"), ("ln3_g", C, "gamma"), ("ln3_b", C, "beta"),
+                ("ff1_b", 2 * wl.ff_inner, "bias"), ("ff2_b", C, "bias"), ("proj_out_b", C, "bias")]
     raise ValueError(wl.kind)
+
+
+def context(wl: Workload) -> torch.Tensor:
+    """A transformer workload's text context (ctx_len, ctx_dim): N(0, 1), storage-rounded,
+    drawn with seed ``seed + 500``; the same for every step, as a prompt's encoding is."""
+    return store(randn((wl.ctx_len, wl.ctx_dim), wl.seed + 500), wl.dtype)
 
 
 class InputStream:

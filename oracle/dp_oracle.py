@@ -606,8 +606,9 @@ def unet_mini_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: flo
 def block_step(kind: str, state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float,
                mode: int, storage: str, heads: int = 0, silu: bool = True,
                trace: Optional[Dict] = None, final_storage: Optional[str] = None,
-               gn_stats: int = GN_STATS_CORRECTED):
-    """Dispatch one block step by kind; x is (C, H, W) (a leading batch of 1 is dropped).
+               gn_stats: int = GN_STATS_CORRECTED, ctx=None):
+    """Dispatch one block step by kind; x is (C, H, W) (a leading batch of 1 is dropped);
+    ``ctx`` is a transformer block's (Tk, Cctx) text context.
 
     ``final_storage`` (default: ``storage``) is the rounding of the block's
     output alone; intermediates always use ``storage``.
@@ -624,6 +625,9 @@ def block_step(kind: str, state: Dict, x, wts: Dict, P: int, G: int, eps: float,
     if kind == "attn":
         return attn_step(state, x, wts, P, G, eps, w, heads, mode, storage, trace,
                          final_storage=final_storage, gn_stats=gn_stats)
+    if kind == "transformer":
+        return transformer_step(state, x, ctx, wts, P, G, eps, w, heads, mode, storage, trace,
+                                final_storage=final_storage, gn_stats=gn_stats)
     if kind == "unet_mini":
         return unet_mini_step(state, x, wts, P, G, eps, w, mode, storage, trace, final_storage,
                               gn_stats)

@@ -376,3 +376,24 @@ def test_binding_structs_match_the_header(B, tmp_path):
         py = structs[cname]
         want = ctypes.sizeof(py) if field == "sizeof" else getattr(py, field).offset
         assert int(value) == want, (cname, field, int(value), want)
+
+
+def test_transformer_workload_marshals_to_the_block(B):
+    """The benchmark's SDXL transformer workload: its seeded weights marshal into the 24
+    pointers the block documents (the context is the 25th), with the documented shapes."""
+    import torch
+
+    from displaced_patch_parallelism_b200 import synth
+    from displaced_patch_parallelism_b200.weights import block_weights
+    wl = synth.WORKLOADS["transformer_640x64x64"]
+    C, F, Cc, Tk = wl.C, wl.ff_inner, wl.ctx_dim, wl.ctx_len
+    d = B.dp_block_desc_init(B.TRANSFORMER, wl.H, wl.W, C, C, wl.G, wl.P, wl.heads, B.BF16, 0,
+                             wl.eps, 1.0)
+    B.dp_block_desc_set_context(d, Tk, Cc, F)
+    w = block_weights("transformer", synth.make_weights(wl), torch.bfloat16, "cpu")
+    assert len(w) + 1 == B.dp_block_weight_count(d)
+    shapes = [(C,), (C,), (C, C), (C,), (C,), (C,), (3 * C, C), (3 * C,), (C, C), (C,), (C,), (C,),
+              (C, C), (2 * C, Cc), (C, C), (C,), (C,), (C,), (2 * F, C), (2 * F,), (C, F), (C,),
+              (C, C), (C,)]
+    assert [tuple(t.shape) for t in w] == shapes
+    assert tuple(synth.context(wl).shape) == (Tk, Cc)
