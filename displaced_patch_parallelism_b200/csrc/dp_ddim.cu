@@ -83,6 +83,7 @@ int dp_ddim_step(const void* x, const void* eps, void* x_prev, size_t n, double 
   if (!dp::aligned16(x) || !dp::aligned16(eps) || !dp::aligned16(x_prev))
     return dp::set_error(DP_ERR_UNSUPPORTED, "ddim: pointers must be 16-byte aligned");
   const size_t es = dtype == DP_FP32 ? 4 : 2;
+  if (n > (static_cast<size_t>(-1) >> 3)) return dp::set_error(DP_ERR_INVALID_ARG, "ddim: n too large");
   const size_t bytes = n * es;
   const char* xb = static_cast<const char*>(x);
   const char* eb = static_cast<const char*>(eps);

@@ -343,7 +343,8 @@ def test_ddim_step_rejects_bad_arguments_on_the_host(B):
            ((A, 2 * A, 3 * A, 64, float("nan"), 0.6, B.BF16), B.DP_ERR_INVALID_ARG),
            ((A, 2 * A, 3 * A + 8, 64, 0.5, 0.6, B.BF16), B.DP_ERR_UNSUPPORTED),  # misaligned
            ((A, 2 * A, 2 * A + 64, 64, 0.5, 0.6, B.BF16), B.DP_ERR_INVALID_ARG),  # overlaps eps
-           ((A, 2 * A, A + 64, 64, 0.5, 0.6, B.FP32), B.DP_ERR_INVALID_ARG)]      # partly overlaps x
+           ((A, 2 * A, A + 64, 64, 0.5, 0.6, B.FP32), B.DP_ERR_INVALID_ARG),      # partly overlaps x
+           ((A, 2 * A, 3 * A, 1 << 62, 0.5, 0.6, B.FP32), B.DP_ERR_INVALID_ARG)]  # byte count overflows
     for args, code in bad:
         with pytest.raises(B.DPError) as e:
             B.dp_ddim_step(*args, stream=0)
