@@ -46,7 +46,11 @@ brute-force loops on tiny inputs; naive mode equals independent crops; an
 unchanged input makes displaced equal sync; a uniform drift makes the
 corrected statistics exact; halo and attention locality; zero warm-up differs
 from sync; the GroupNorm variants equal the library GroupNorm of the whole
-image, of each band's crop and of the previous step's image.
+image, of each band's crop and of the previous step's image; the transformer
+block and the time-embedding ResBlock equal the same blocks composed from
+library operators at P = 1; ``time_embedding_term`` is the library linear of
+the library SiLU; ``ddim_step`` moves an exactly known noise to the previous
+level, is the identity at an unchanged level, composes, and is affine.
 ``unet_mini_step`` is pinned only through its parts and the P = 1 reduction of
 the whole chain.
 """
