@@ -662,6 +662,32 @@ def test_p1_transformer_equals_library(mode):
     np.testing.assert_allclose(y, lib_transformer(x, ctx, w, G, 1e-5, heads), rtol=0, atol=1e-11)
 
 
+def test_transformer_displaced_band_locality():
+    """A displaced step needs nothing of the current step from other bands: changing one
+    band's input leaves every other band's output bit for bit the same (their GroupNorm
+    statistics take only their own fresh moments, their self-attention the other bands'
+    stale keys and values, and LayerNorm, cross-attention and the feed-forward act per
+    token), while in a sync step the change reaches every band."""
+    r = rng(97)
+    C, H, W, P, G, heads, Cctx, Tk = 8, 8, 4, 4, 4, 2, 6, 5
+    w = rand_transformer_weights(r, C, Cctx, heads)
+    x0, ctx = r.standard_normal((C, H, W)), r.standard_normal((Tk, Cctx))
+    x1 = x0 + 0.3 * r.standard_normal(x0.shape)
+    hb, q = H // P, 2
+    x1b = x1.copy()
+    x1b[:, q * hb:(q + 1) * hb, :] += r.standard_normal((C, hb, W))
+    for mode in (DISPLACED, SYNC):
+        ys = []
+        for xin in (x1, x1b):
+            st = {}
+            O.transformer_step(st, x0, ctx, w, P, G, 1e-5, 1.0, heads, SYNC, "none")
+            ys.append(O.transformer_step(st, xin, ctx, w, P, G, 1e-5, 1.0, heads, mode, "none"))
+        for p in range(P):
+            rows = slice(p * hb, (p + 1) * hb)
+            same = np.array_equal(ys[0][:, rows, :], ys[1][:, rows, :])
+            assert same == (mode == DISPLACED and p != q), (mode, p)
+
+
 def test_transformer_displaced_and_naive_invariants():
     """Unchanged input: displaced equals sync.  Naive: each band is an independent image."""
     r = rng(92)
