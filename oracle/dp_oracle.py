@@ -20,7 +20,7 @@ bf16 (GroupNorm output, conv output feeding the next GroupNorm, q/k/v, the
 attention output, block outputs) the oracle rounds to bf16 at the same point
 (``store``); pass ``storage="none"`` to keep everything unrounded.
 
-Readings of what the pages leave open (each also listed in the design notes):
+Readings of what the pages leave open:
   R1  corrected statistics on raw moments (E[x], E[x^2]):
         used = stale_global + w * (fresh_local - stale_local),  w = 1 by default
   R2  a negative corrected variance falls back to the patch's fresh variance
@@ -51,8 +51,11 @@ block and the time-embedding ResBlock equal the same blocks composed from
 library operators at P = 1; ``time_embedding_term`` is the library linear of
 the library SiLU; ``ddim_step`` moves an exactly known noise to the previous
 level, is the identity at an unchanged level, composes, and is affine.
-``unet_mini_step`` is pinned only through its parts and the P = 1 reduction of
-the whole chain.
+``unet_mini_step`` at P = 1 equals the same chain composed from library
+operators (conv2d with stride 1 and 2, the library ResBlock and attention with
+10 and 20 heads); its naive step at P = 4 equals that library chain on each
+band's crop; and at P = 4 an unchanged input makes its displaced step equal its
+synchronous one.
 """
 from __future__ import annotations
 

@@ -161,23 +161,98 @@ def test_conv1x1_equals_library():
     np.testing.assert_allclose(O.conv1x1(a, wt, b), ref, rtol=0, atol=1e-12)
 
 
-def test_p1_unet_mini_displaced_equals_sync():
-    """The whole chain with one band: displacement changes nothing."""
+def _unet_mini_weights(seed):
+    """Random weights of the mini U-Net chain (the workload's own names and shapes, random
+    affine parameters and biases so that no term hides behind a zero)."""
     from displaced_patch_parallelism_b200 import synth
     wl = synth.WORKLOADS["unet_mini_4x128x128"]
-    # shrink: the chain's structure with tiny spatial size
-    r = rng(6)
+    r = rng(seed)
     wts = {}
     for name, shape, std in synth.unet_mini_weight_specs(4):
         wts[name] = r.standard_normal(shape) * std
     for name, c, kind in synth.affine_specs(wl):
         wts[name] = (1 + 0.2 * r.standard_normal(c)) if kind == "gamma" else 0.2 * r.standard_normal(c)
+    return wts
+
+
+def lib_unet_mini(x, w, G=32, eps=1e-5, heads=(10, 20)):
+    """The mini U-Net chain composed from library operators only: conv2d (stride 1 and 2,
+    padding 1), the library ResBlock and the library attention block with 10 and 20 heads."""
+    conv = lambda t, n, s: F.conv2d(T64(t)[None], T64(w[n + "_w"]), T64(w[n + "_b"]), stride=s,
+                                    padding=1)[0].numpy()
+    h = conv(x, "conv_in", 1)
+    h = lib_resblock(h, w, G, eps, "rb1.")
+    h = conv(h, "down1", 2)
+    h = lib_resblock(h, w, G, eps, "rb2.")
+    h = lib_attn(h, w, G, eps, heads[0], "at2.")
+    h = conv(h, "down2", 2)
+    h = lib_resblock(h, w, G, eps, "rb3.")
+    return lib_attn(h, w, G, eps, heads[1], "at3.")
+
+
+@pytest.mark.parametrize("mode", [SYNC, DISPLACED])
+def test_p1_unet_mini_equals_library(mode):
+    """With one band the whole chain is the ordinary network: conv_in, ResBlock(320), a
+    stride-2 downsampler, ResBlock(320->640) with its 1x1 shortcut, attention with 10 heads,
+    a second downsampler, ResBlock(640->1280), attention with 20 heads -- composed here
+    from library operators.  A wrong head count, stage order, stride or shortcut fails."""
+    w = _unet_mini_weights(6)
+    r = rng(7)
+    x0, x1 = r.standard_normal((4, 8, 8)), r.standard_normal((4, 8, 8))
+    st = {}
+    O.unet_mini_step(st, x0, w, 1, 32, 1e-5, 1.0, SYNC, "none")
+    y = O.unet_mini_step(st, x1, w, 1, 32, 1e-5, 1.0, mode, "none")
+    assert y.shape == (1280, 2, 2)
+    ref = lib_unet_mini(x1, w)
+    tol = 1e-9 * np.abs(ref).max()
+    np.testing.assert_allclose(y, ref, rtol=0, atol=tol)
+    # the pin has teeth: other head counts give results far outside the tolerance
+    for heads in ((20, 20), (10, 10)):
+        assert np.abs(lib_unet_mini(x1, w, heads=heads) - ref).max() > 1e3 * tol
+
+
+def test_unet_mini_naive_equals_independent_crops():
+    """Zero warm-up's step 0 (naive) at P = 4: every band runs the whole chain as an image of
+    its own -- its own GroupNorm statistics, zero rows beyond its edges in every conv (the
+    stride-2 downsamplers included) and only its own tokens as keys -- so the output is the
+    library chain of each band's crop, stacked."""
+    w = _unet_mini_weights(8)
+    x = rng(9).standard_normal((4, 16, 8))
+    y = O.unet_mini_step({}, x, w, 4, 32, 1e-5, 1.0, NAIVE, "none")
+    assert y.shape == (1280, 4, 2)
+    ref = np.concatenate([lib_unet_mini(x[:, 4 * p:4 * (p + 1)], w) for p in range(4)], axis=1)
+    np.testing.assert_allclose(y, ref, rtol=0, atol=1e-9 * np.abs(ref).max())
+
+
+def test_unet_mini_unchanged_input_displaced_equals_sync():
+    """P = 4, an unchanged input after a synchronous step: every stale buffer (the halo rows
+    of each conv, the downsamplers' own inputs, the keys and values of both attentions, the
+    GroupNorm statistics) equals the fresh one, so the displaced chain gives the synchronous
+    chain.  A stage that took its stale rows or keys from another layer's buffer fails."""
+    w = _unet_mini_weights(10)
+    x = rng(11).standard_normal((4, 16, 16))
+    st = {}
+    y_sync = O.unet_mini_step(st, x, w, 4, 32, 1e-5, 1.0, SYNC, "none")
+    y_disp = O.unet_mini_step(st, x, w, 4, 32, 1e-5, 1.0, DISPLACED, "none")
+    np.testing.assert_allclose(y_disp, y_sync, rtol=0, atol=1e-9 * np.abs(y_sync).max())
+    # and with a changed input the displaced chain differs from the synchronous one
+    x2 = x + 0.3 * rng(12).standard_normal(x.shape)
+    st2 = {k: dict(v) if isinstance(v, dict) else v for k, v in st.items()}
+    y2_sync = O.unet_mini_step({}, x2, w, 4, 32, 1e-5, 1.0, SYNC, "none")
+    y2_disp = O.unet_mini_step(st2, x2, w, 4, 32, 1e-5, 1.0, DISPLACED, "none")
+    assert np.abs(y2_disp - y2_sync).max() > 1e-4 * np.abs(y2_sync).max()
+
+
+def test_p1_unet_mini_displaced_equals_sync():
+    """The whole chain with one band: displacement changes nothing."""
+    w = _unet_mini_weights(6)
+    r = rng(6)
     x0, x1 = r.standard_normal((4, 8, 8)), r.standard_normal((4, 8, 8))
     outs = {}
     for m in (SYNC, DISPLACED):
         st = {}
-        O.unet_mini_step(st, x0, wts, 1, 32, 1e-5, 1.0, SYNC, "none")
-        outs[m] = O.unet_mini_step(st, x1, wts, 1, 32, 1e-5, 1.0, m, "none")
+        O.unet_mini_step(st, x0, w, 1, 32, 1e-5, 1.0, SYNC, "none")
+        outs[m] = O.unet_mini_step(st, x1, w, 1, 32, 1e-5, 1.0, m, "none")
     np.testing.assert_allclose(outs[DISPLACED], outs[SYNC], rtol=0, atol=1e-10)
     assert outs[SYNC].shape == (1280, 2, 2)
 
