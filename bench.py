@@ -3,13 +3,17 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
-A step is one ``dp_block_step`` of the workload (default: the SDXL 1024 px
-top-resolution ResBlock, latent 1x320x128x128, P = 4 bands) in displaced mode,
-on synthetic inputs already resident in HBM.  Each step is timed with CUDA
-events recorded on the launching stream just before and after it; L2 is
-flushed (a 256 MiB write) between steps, outside the timed events.  A second
-pass with an event before every kernel (``dp_block_step_timed``) gives the
-per-kernel breakdown and the roofline of the dominant kernel.
+A step is one ``dp_block_step`` of the workload in displaced mode, on
+synthetic inputs already resident in HBM.  The default workload is the largest
+single-GPU one: the 3840x3840-shaped GroupNorm + SiLU + 3x3 conv block, latent
+1x320x480x480, P = 8 bands of 60 rows.  Each step is timed with CUDA events
+recorded on the launching stream just before and after it.  Between steps L2
+is flushed (a 256 MiB write, outside the timed events) unless the step's input
+alone is larger than L2, in which case the inputs themselves evict it.  A
+second pass with an event before every kernel (``dp_block_step_timed``) gives
+the per-kernel breakdown and the roofline of the dominant kernel.  The other
+workloads are then timed the same way (device time and breakdown, no
+end-to-end pass) and reported under ``workloads``.
 With N > 1 (torchrun) every rank runs an independent replica on its own GPU:
 the path has no data exchange on one GPU per image, so there is no
 collective; the time is the max over ranks.
@@ -179,67 +183,106 @@ def launch_plan(B, wl, mode):
     return [B.dp_block_launch_info(d, mode, i) for i in range(B.dp_block_launch_count(d))]
 
 
-def cpu_baseline_ours(wl, seconds):
-    """The oracle, as it stands, timed on this host: full displaced steps until `seconds` pass."""
+L2_BYTES = 126 << 20          # B200 L2
+
+
+def wl_flops(wl, H=None):
+    """Algorithmic flops of one displaced step of workload ``wl`` (rows ``H`` if given): the
+    convolutions, projections and attention contractions, multiply-adds counted twice.
+    Computed from the shapes alone, so the oracle arm never loads the CUDA library."""
+    H = H or wl.H
+    hw = float(H) * wl.W
+    C, Co = float(wl.C), float(wl.cout)
+
+    def conv(hw_out, ci, co):
+        return 2.0 * hw_out * co * 9.0 * ci
+
+    def resblock(hw_, ci, co):
+        return conv(hw_, ci, co) + conv(hw_, co, co) + (2.0 * hw_ * co * ci if ci != co else 0.0)
+
+    def attn(t, c):
+        return 2.0 * t * 3.0 * c * c + 4.0 * t * t * c + 2.0 * t * c * c
+
+    if wl.kind == "gn_conv":
+        return conv(hw, C, Co)
+    if wl.kind == "resblock":
+        return resblock(hw, C, Co)
+    if wl.kind == "attn":
+        return attn(hw, C)
+    if wl.kind == "transformer":
+        Tk, Cc, F = float(wl.ctx_len), float(wl.ctx_dim), float(wl.ff_inner)
+        return (2.0 * hw * C * C * 5.0 + 2.0 * hw * 3.0 * C * C + 4.0 * hw * hw * C +
+                2.0 * Tk * 2.0 * C * Cc + 4.0 * hw * Tk * C + 2.0 * hw * 2.0 * F * C +
+                2.0 * hw * C * F)
+    if wl.kind == "unet_mini":
+        return (conv(hw, C, 320) + resblock(hw, 320, 320) + conv(hw / 4, 320, 320) +
+                resblock(hw / 4, 320, 640) + attn(hw / 4, 640) + conv(hw / 16, 640, 640) +
+                resblock(hw / 16, 640, 1280) + attn(hw / 16, 1280))
+    raise ValueError(wl.kind)
+
+
+def crop_rows_for(wl, seconds_per_step):
+    """Rows per band of a row crop whose displaced oracle step takes about
+    ``seconds_per_step`` on this host (attention blocks keep the whole image: their
+    tiles need every token)."""
+    import dataclasses
+    hb = wl.H // wl.P
+    if wl.kind in ("attn", "transformer"):
+        return wl, hb
+    t_small = oracle_step_time(dataclasses.replace(wl, H=wl.P * 2))[0]
+    per_row = t_small / (2 * wl.P)
+    rows = max(2, min(hb, int(seconds_per_step / max(per_row, 1e-6) / wl.P)))
+    return dataclasses.replace(wl, H=wl.P * rows), rows
+
+
+def oracle_step_time(w):
+    """One sync step, then one timed displaced step of the oracle on workload ``w``."""
     from displaced_patch_parallelism_b200 import synth
     from oracle import dp_oracle as O
-    wts = {n: v.double().numpy() for n, v in synth.make_weights(wl).items()}
-    xs = synth.InputStream(wl)
-    ctx = oracle_context(wl)
+    ctx = oracle_context(w)
+    wts = {n: v.double().numpy() for n, v in synth.make_weights(w).items()}
+    xs = synth.InputStream(w)
     st = {}
-    O.block_step(wl.kind, st, xs.x(0)[0], wts, wl.P, wl.G, wl.eps, 1.0, synth.SYNC, wl.dtype,
-                 heads=wl.heads, silu=wl.silu, ctx=ctx)
-    x1 = xs.x(1)[0]
+    O.block_step(w.kind, st, xs.x(0)[0], wts, w.P, w.G, w.eps, 1.0, synth.SYNC, w.dtype,
+                 heads=w.heads, silu=w.silu, ctx=ctx)
+    t0 = time.perf_counter()
+    O.block_step(w.kind, st, xs.x(1)[0], wts, w.P, w.G, w.eps, 1.0, synth.DISPLACED, w.dtype,
+                 heads=w.heads, silu=w.silu, gn_stats=GN_STATS, ctx=ctx)
+    return time.perf_counter() - t0, wts, st, xs, ctx
+
+
+def cpu_baseline_ours(wl, seconds):
+    """The oracle, as it stands, on this host: displaced steps of a row crop of the workload
+    (each about a quarter of ``seconds``) until ``seconds`` pass.  Returns the line's
+    ``cpu_baseline`` object."""
+    from displaced_patch_parallelism_b200 import synth
+    from oracle import dp_oracle as O
+    w, rows = crop_rows_for(wl, seconds / 4)
+    _, wts, st, xs, ctx = oracle_step_time(w)
+    x = xs.x(2)[0]
     reps, t0 = 0, time.perf_counter()
     while True:
-        O.block_step(wl.kind, st, x1, wts, wl.P, wl.G, wl.eps, 1.0, synth.DISPLACED, wl.dtype,
-                     heads=wl.heads, silu=wl.silu, gn_stats=GN_STATS, ctx=ctx)
+        O.block_step(w.kind, st, x, wts, w.P, w.G, w.eps, 1.0, synth.DISPLACED, w.dtype,
+                     heads=w.heads, silu=w.silu, gn_stats=GN_STATS, ctx=ctx)
         reps += 1
         el = time.perf_counter() - t0
         if el >= seconds:
             break
-    return reps, el
-
-
-def wl_flops(wl, H=None):
-    from displaced_patch_parallelism_b200 import binding as B
-    return B.dp_block_flops(block_desc(B, wl, H))
+    fl = wl_flops(wl, w.H)
+    return {"value": round(fl * reps / el / 1e12, 6), "unit": "TFLOP/s",
+            "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+            "sample": (f"{reps} displaced steps of {wl.name} on a {w.C}x{w.H}x{w.W} row crop "
+                       f"({rows} rows per band, {fl / 1e9:.2f} GFLOP each) in {el:.1f} s")}
 
 
 def run_reference(args, wl):
     """The CPU oracle on the host cores: each step a displaced step of a row crop of the block."""
-    import dataclasses
-
     from displaced_patch_parallelism_b200 import synth
     from oracle import dp_oracle as O
     budget = 150.0
     cores = len(os.sched_getaffinity(0))
-    ctx = oracle_context(wl)
-
-    def crop(rows_per_band):
-        return dataclasses.replace(wl, H=wl.P * rows_per_band)
-
-    def one_step_time(w):
-        wts = {n: v.double().numpy() for n, v in synth.make_weights(w).items()}
-        xs = synth.InputStream(w)
-        st = {}
-        O.block_step(w.kind, st, xs.x(0)[0], wts, w.P, w.G, w.eps, 1.0, synth.SYNC, w.dtype,
-                     heads=w.heads, silu=w.silu, ctx=ctx)
-        t0 = time.perf_counter()
-        O.block_step(w.kind, st, xs.x(1)[0], wts, w.P, w.G, w.eps, 1.0, synth.DISPLACED, w.dtype,
-                     heads=w.heads, silu=w.silu, gn_stats=GN_STATS, ctx=ctx)
-        return time.perf_counter() - t0, wts, st, xs
-
-    hb = wl.H // wl.P
-    if wl.kind in ("attn", "transformer"):
-        rows = hb  # attention blocks need whole 128-token tiles: keep the full image
-    else:
-        t_small, *_ = one_step_time(crop(2))
-        per_row = t_small / (2 * wl.P)
-        fit = int((budget / max(1, args.steps + args.warmup)) / max(per_row, 1e-6) / wl.P)
-        rows = max(2, min(hb, fit))
-    w = crop(rows)
-    _, wts, st, xs = one_step_time(w)
+    w, rows = crop_rows_for(wl, budget / max(1, args.steps + args.warmup))
+    _, wts, st, xs, ctx = oracle_step_time(w)
     x = xs.x(2)[0]
     for _ in range(args.warmup):
         O.block_step(w.kind, st, x, wts, w.P, w.G, w.eps, 1.0, synth.DISPLACED, w.dtype,
@@ -257,8 +300,7 @@ def run_reference(args, wl):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name, "shape_nchw": [1, wl.C, wl.H, wl.W], "P": wl.P,
-                       "mode": "displaced", "gn_stats": GN_STATS_NAMES[GN_STATS], "sample": sample},
+            "config": workload_config(wl, ws=1, extra={"sample": sample}),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -266,80 +308,102 @@ def run_reference(args, wl):
     print(json.dumps(line), flush=True)
 
 
-def run_ours(args, wl):
+def input_bytes(wl):
+    return wl.C * wl.H * wl.W * (2 if wl.dtype == "bf16" else 4)
+
+
+def l2_policy(wl):
+    """(flush between steps?, description): a step whose input alone exceeds L2 evicts it
+    by itself; smaller ones get a 256 MiB write between steps, outside the timed events."""
+    if input_bytes(wl) > L2_BYTES:
+        return False, (f"inputs larger than L2 ({input_bytes(wl) / 1e6:.1f} MB input per step, "
+                       f"4 inputs in rotation); no flush")
+    return True, "flushed between steps (256 MiB write, outside the timed events)"
+
+
+def workload_config(wl, ws, extra=None):
+    cfg = {"workload": wl.name, "shape_nchw": [1, wl.C, wl.H, wl.W], "P": wl.P,
+           "mode": "displaced", "gn_stats": GN_STATS_NAMES[GN_STATS],
+           "l2": l2_policy(wl)[1],
+           "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"}
+    if wl.dtype == "fp32":
+        cfg["arithmetic"] = "fp32 storage, conv on tf32 tensor cores with fp32 accumulation"
+    cfg.update(extra or {})
+    return cfg
+
+
+class Run:
+    """One workload's block, weights and inputs on the device."""
+
+    def __init__(self, wl, dev, pool=4):
+        import torch
+
+        from displaced_patch_parallelism_b200 import binding as B
+        from displaced_patch_parallelism_b200 import synth
+        from displaced_patch_parallelism_b200.weights import block_weights
+        self.wl, self.B = wl, B
+        self.tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+        wts = synth.make_weights(wl)
+        self.dw = block_weights(wl.kind, wts, self.tdt, dev)
+        if wl.kind == "transformer":     # the step's text context is the last pointer
+            self.dw.append(synth.context(wl).to(self.tdt).to(dev))
+        self.blk = B.Block(block_kind(B, wl), wl.H, wl.W, wl.C, wl.cout, wl.G, wl.P, wl.heads,
+                           B.BF16 if wl.dtype == "bf16" else B.FP32, wl.silu, wl.eps, 1.0,
+                           device=dev, gn_stats=GN_STATS, context=wl_context(wl))
+        xs = synth.InputStream(wl)
+        self.pool = pool
+        self.host_x = [synth.nchw_to_nhwc(xs.x(k)).to(self.tdt).pin_memory() for k in range(pool)]
+        self.dev_x = [h.to(dev) for h in self.host_x]
+        Ho, Wo = (wl.H // 4, wl.W // 4) if wl.kind == "unet_mini" else (wl.H, wl.W)
+        self.out = torch.empty(Ho, Wo, wl.cout, dtype=self.tdt, device=dev)
+        self.flush_between = l2_policy(wl)[0]
+        self.plan = launch_plan(B, wl, B.DISPLACED)
+        assert len(self.plan) == self.blk.launches
+        self.flops = wl_flops(wl)
+
+    def warm(self, n):
+        import torch
+        for i in range(n):
+            self.blk.step(self.dev_x[i % self.pool], self.out, self.dw,
+                          self.B.dp_mode_for_step(i, self.wl.warmup))
+        torch.cuda.synchronize()
+
+
+def time_steps(run, steps, flush, dist, sampler=None):
+    """Device time (ms) of each of ``steps`` displaced steps, an event pair around each."""
     import torch
-
-    from displaced_patch_parallelism_b200 import binding as B
-    from displaced_patch_parallelism_b200 import synth
-    from displaced_patch_parallelism_b200.weights import block_weights
-
-    ws, rank, local = dist_env()
-    torch.cuda.set_device(local)
-    dist = None
-    if ws > 1:
-        import datetime
-
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    dev = torch.device("cuda", local)
-    tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
-    wts = synth.make_weights(wl)
-    dw = block_weights(wl.kind, wts, tdt, dev)
-    if wl.kind == "transformer":     # the step's text context is the last pointer
-        dw.append(synth.context(wl).to(tdt).to(dev))
-    blk = B.Block(block_kind(B, wl), wl.H, wl.W, wl.C, wl.cout, wl.G, wl.P, wl.heads,
-                  B.BF16 if wl.dtype == "bf16" else B.FP32, wl.silu, wl.eps, 1.0, device=dev,
-                  gn_stats=GN_STATS, context=wl_context(wl))
-    xs = synth.InputStream(wl)
-    pool = 4
-    host_x = [synth.nchw_to_nhwc(xs.x(k)).to(tdt).pin_memory() for k in range(pool)]
-    dev_x = [h.to(dev) for h in host_x]
-    Ho, Wo = (wl.H // 4, wl.W // 4) if wl.kind == "unet_mini" else (wl.H, wl.W)
-    out = torch.empty(Ho, Wo, wl.cout, dtype=tdt, device=dev)
-    host_out = torch.empty(out.shape, dtype=tdt).pin_memory()
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    n_launch = blk.launches
-    plan = launch_plan(B, wl, B.DISPLACED)
-    assert len(plan) == n_launch
-    roles = [r for r, _, _ in plan]
-
-    warm = max(args.warmup, wl.warmup + 1)
-    for i in range(warm):
-        blk.step(dev_x[i % pool], out, dw, B.dp_mode_for_step(i, wl.warmup))
-    torch.cuda.synchronize()
-
-    # Timed region: one event before and one after each step, so that the
-    # kernels of a step follow one another as they do in use (dependent
-    # launches overlap a kernel's set-up with its predecessor).
-    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     for e in ev0 + ev1:          # torch creates the CUDA event on its first record
         e.record()
     torch.cuda.synchronize()
-    sampler = ClockSampler(local)
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
-    sampler.start()
+    if sampler:
+        sampler.start()
     wall0 = time.perf_counter()
-    for k in range(args.steps):
-        flush.zero_()
+    for k in range(steps):
+        if run.flush_between:
+            flush.zero_()
         ev0[k].record()
-        blk.step(dev_x[k % pool], out, dw, B.DISPLACED)
+        run.blk.step(run.dev_x[k % run.pool], run.out, run.dw, run.B.DISPLACED)
         ev1[k].record()
     torch.cuda.synchronize()
     wall = time.perf_counter() - wall0
-    clocks = sampler.stop()
+    clocks = sampler.stop() if sampler else None
     if dist:
         dist.barrier()
-    step_ms = [ev0[k].elapsed_time(ev1[k]) for k in range(args.steps)]
-    total_ms = sum(step_ms)
+    return [ev0[k].elapsed_time(ev1[k]) for k in range(steps)], wall, clocks
 
-    # Per-kernel breakdown: a separate pass with an event before every launch
-    # (dp_block_step_timed); those events keep kernels from overlapping, so the
-    # per-kernel times add up to a little more than the step above.
-    n_bd = min(args.steps, 50)
+
+def breakdown(run, steps, flush, peaks):
+    """Per-kernel roles of the step: mean duration, share, rate; and the dominant role's
+    roofline.  An event before every launch (dp_block_step_timed) keeps kernels from
+    overlapping, so these times add up to a little more than the step."""
+    import torch
+    n_launch = run.blk.launches
+    n_bd = min(steps, 50)
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_launch + 1)]
               for _ in range(n_bd)]
     for row in events:
@@ -347,66 +411,14 @@ def run_ours(args, wl):
             e.record()
     torch.cuda.synchronize()
     for k in range(n_bd):
-        flush.zero_()
-        blk.step_timed(dev_x[k % pool], out, dw, B.DISPLACED, events[k])
+        if run.flush_between:
+            flush.zero_()
+        run.blk.step_timed(run.dev_x[k % run.pool], run.out, run.dw, run.B.DISPLACED, events[k])
     torch.cuda.synchronize()
     per_launch = [[events[k][i].elapsed_time(events[k][i + 1]) for i in range(n_launch)]
                   for k in range(n_bd)]
-    total_ms = max_over_ranks(total_ms, dist, dev)
-
-    # end-to-end: every step copies its input from pinned host memory, runs the
-    # block step and copies its result back to pinned host memory.  The copies
-    # run on their own streams (the copy engines), so step k+1's input and step
-    # k's result move while a neighbouring step computes; the L2 flush stays in
-    # front of every step's compute.  Timed on the device from the first copy
-    # to the last.
-    s_comp, s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
-    xin = [torch.empty_like(dev_x[0]) for _ in range(2)]
-    outb = [torch.empty_like(out) for _ in range(2)]
-    host_o = [host_out, torch.empty_like(host_out).pin_memory()]
-    ev_in = [torch.cuda.Event() for _ in range(args.steps)]
-    ev_comp = [torch.cuda.Event() for _ in range(args.steps)]
-    ev_out = [torch.cuda.Event() for _ in range(args.steps)]
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize()
-    t_start.record(s_comp)
-    s_in.wait_event(t_start)
-    for k in range(args.steps):
-        b = k & 1
-        if k >= 2:
-            s_in.wait_event(ev_comp[k - 2])      # step k-2 has read xin[b]
-        with torch.cuda.stream(s_in):
-            xin[b].copy_(host_x[k % pool], non_blocking=True)
-            ev_in[k].record(s_in)
-        with torch.cuda.stream(s_comp):
-            flush.zero_()
-            s_comp.wait_event(ev_in[k])
-            if k >= 2:
-                s_comp.wait_event(ev_out[k - 2])  # outb[b] has reached the host
-            blk.step(xin[b], outb[b], dw, B.DISPLACED)
-            ev_comp[k].record(s_comp)
-        s_out.wait_event(ev_comp[k])
-        with torch.cuda.stream(s_out):
-            host_o[b].copy_(outb[b], non_blocking=True)
-            ev_out[k].record(s_out)
-    s_comp.wait_event(ev_out[args.steps - 1])
-    t_end.record(s_comp)
-    torch.cuda.synchronize()
-    e2e_ms = t_start.elapsed_time(t_end)
-    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
-    if dist:
-        dist.barrier()
-    status = B.dp_device_status()
-
-    flops = blk.flops
-    value = job_tflops(ws, flops, args.steps, total_ms)
-    e2e_value = job_tflops(ws, flops, args.steps, e2e_ms)
-
-    # per-kernel roles: mean duration, share, roofline of the dominant one
-    work = [(f, b) for _, f, b in plan]
-    peaks = load_peaks()
+    roles = [r for r, _, _ in run.plan]
+    work = [(f, b) for _, f, b in run.plan]
     role_ms, role_n = {}, {}
     for k in range(n_bd):
         for i, r in enumerate(roles):
@@ -426,9 +438,10 @@ def run_ours(args, wl):
     dk = kernels[dominant]
     src = {"conv": ["dp_gemm.cu"], "linear": ["dp_gemm.cu"], "attn": ["dp_attn.cu"],
            "gn_stats": ["dp_gn.cu"], "gn_apply": ["dp_gn.cu"], "gn_fused": ["dp_gn.cu"],
-           "gn_cluster": ["dp_gn.cu"],
-           "copy": ["dp_refresh.cu"], "conv_small": ["dp_conv_small.cu"], "splitk_finish": ["dp_gemm.cu"]}[dominant]
-    traffic = load_traffic(f"{dominant}:{wl.name}", kernel_source_hash(src))
+           "gn_cluster": ["dp_gn.cu"], "copy": ["dp_refresh.cu"],
+           "conv_small": ["dp_conv_small.cu"], "splitk_finish": ["dp_gemm.cu"],
+           "layernorm": ["dp_token.cu"], "geglu": ["dp_token.cu"], "temb": ["dp_temb.cu"]}
+    traffic = load_traffic(f"{dominant}:{run.wl.name}", kernel_source_hash(src[dominant]))
     if dk["tflops"]:
         roof = {"bound": "tensor", "achieved": dk["tflops"], "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": round(dk["tflops"] / peaks["bf16_tflops"], 4),
@@ -436,6 +449,8 @@ def run_ours(args, wl):
                 "peak_source": f"{peaks['source']} bf16 burst",
                 "frac_of_sustained": round(dk["tflops"] / peaks["bf16_tflops_sustained"], 4)
                 if peaks.get("bf16_tflops_sustained") else None}
+        if run.wl.dtype == "fp32":
+            roof["note"] = "tf32 contraction measured against the bf16 peak"
     else:
         roof = {"bound": "hbm", "achieved": dk["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(dk["gbs"] / peaks["hbm_gbs"], 4), "traffic": traffic,
@@ -447,28 +462,133 @@ def run_ours(args, wl):
           "bytes_model": "single pass: read x + write y; two passes: stats read x, apply read x + write y"}
     if gn["achieved_gbs"]:
         gn["frac"] = round(gn["achieved_gbs"] / peaks["hbm_gbs"], 4)
+    return kernels, roof, gn
 
-    line = {"metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": ws,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 5),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
-            "data": "synthetic",
-            "config": {"workload": wl.name, "shape_nchw": [1, wl.C, wl.H, wl.W], "P": wl.P,
-                       "mode": "displaced", "gn_stats": GN_STATS_NAMES[GN_STATS],
-                       "l2": "flushed between steps (256 MiB write, untimed)",
-                       "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
+
+def time_e2e(run, steps, dist, dev):
+    """End to end through the public call: every step copies its input from pinned host
+    memory, runs the block step and copies its result back to pinned host memory.  The
+    copies run on their own streams (the copy engines), so step k+1's input and step k's
+    result move while a neighbouring step computes.  Timed on the device from the first
+    copy to the last; nothing else (no L2 flush) runs in the timed region."""
+    import torch
+    s_comp, s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    xin = [torch.empty_like(run.dev_x[0]) for _ in range(2)]
+    outb = [torch.empty_like(run.out) for _ in range(2)]
+    host_o = [torch.empty(run.out.shape, dtype=run.tdt).pin_memory() for _ in range(2)]
+    ev_in = [torch.cuda.Event() for _ in range(steps)]
+    ev_comp = [torch.cuda.Event() for _ in range(steps)]
+    ev_out = [torch.cuda.Event() for _ in range(steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_start.record(s_comp)
+    s_in.wait_event(t_start)
+    for k in range(steps):
+        b = k & 1
+        if k >= 2:
+            s_in.wait_event(ev_comp[k - 2])      # step k-2 has read xin[b]
+        with torch.cuda.stream(s_in):
+            xin[b].copy_(run.host_x[k % run.pool], non_blocking=True)
+            ev_in[k].record(s_in)
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(ev_in[k])
+            if k >= 2:
+                s_comp.wait_event(ev_out[k - 2])  # outb[b] has reached the host
+            run.blk.step(xin[b], outb[b], run.dw, run.B.DISPLACED)
+            ev_comp[k].record(s_comp)
+        s_out.wait_event(ev_comp[k])
+        with torch.cuda.stream(s_out):
+            host_o[b].copy_(outb[b], non_blocking=True)
+            ev_out[k].record(s_out)
+    s_comp.wait_event(ev_out[steps - 1])
+    t_end.record(s_comp)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(t_start.elapsed_time(t_end), dist, dev)
+    if dist:
+        dist.barrier()
+    return e2e_ms, (run.dev_x[0].numel() * run.dev_x[0].element_size(),
+                    run.out.numel() * run.out.element_size())
+
+
+EXTRA_WORKLOADS = ["tiny_fp32_gn_conv", "resblock_320x128x128", "attn_640x64x64",
+                   "unet_mini_4x128x128", "transformer_640x64x64"]
+
+
+def run_ours(args, wl):
+    import torch
+
+    from displaced_patch_parallelism_b200 import binding as B
+    from displaced_patch_parallelism_b200 import synth
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dist = None
+    if ws > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    peaks = load_peaks()
+
+    run = Run(wl, dev)
+    run.warm(max(args.warmup, wl.warmup + 1))
+    step_ms, wall, clocks = time_steps(run, args.steps, flush, dist, ClockSampler(local))
+    total_ms = max_over_ranks(sum(step_ms), dist, dev)
+    kernels, roof, gn = breakdown(run, args.steps, flush, peaks)
+    e2e_ms, (h2d, d2h) = time_e2e(run, args.steps, dist, dev)
+    status = B.dp_device_status()
+    n_launch = run.blk.launches
+    line = {"metric": METRIC, "value": round(job_tflops(ws, run.flops, args.steps, total_ms), 3),
+            "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(total_ms / args.steps, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
+            "config": workload_config(wl, ws),
             "roofline": roof, "kernels": kernels, "groupnorm": gn,
-            "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s",
+            "e2e": {"value": round(job_tflops(ws, run.flops, args.steps, e2e_ms), 3),
+                    "unit": "TFLOP/s", "ms_per_step": round(e2e_ms / args.steps, 5),
                     "copies": "input and result copies on their own streams, overlapping "
-                              "neighbouring steps; L2 flushed before every step's compute",
-                    "h2d_bytes_per_step": dev_x[0].numel() * dev_x[0].element_size(),
-                    "d2h_bytes_per_step": out.numel() * out.element_size()},
+                              "neighbouring steps; no L2 flush in the timed region",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": n_launch * args.steps, "clocks": clocks,
             "wall_s_timed_region": round(wall, 4), "device_status": status}
+    del run
+    torch.cuda.empty_cache()
+
+    # the other workloads: device-timed steps and the per-kernel breakdown
+    if not args.headline_only:
+        extra = {}
+        for name in EXTRA_WORKLOADS:
+            if name == wl.name:
+                continue
+            w = synth.WORKLOADS[name]
+            try:
+                r = Run(w, dev)
+                r.warm(max(args.warmup, w.warmup + 1))
+                ms, _, _ = time_steps(r, args.steps, flush, dist)
+                t_ms = max_over_ranks(sum(ms), dist, dev)
+                k, rf, g = breakdown(r, args.steps, flush, peaks)
+            except B.DPError as e:          # a host-side rejection; recorded, not fatal
+                extra[name] = {"error": str(e)}
+                continue
+            extra[name] = {"ms_per_step": round(t_ms / args.steps, 5),
+                           "value": round(job_tflops(ws, r.flops, args.steps, t_ms), 3),
+                           "unit": "TFLOP/s", "gflop_per_step": round(r.flops / 1e9, 3),
+                           "dtype": w.dtype, "config": workload_config(w, ws),
+                           "roofline": {kk: rf[kk] for kk in ("bound", "kernel", "achieved",
+                                                              "peak", "unit", "frac")},
+                           "kernels": k, "groupnorm": g,
+                           "gpu_launches": r.blk.launches * args.steps}
+            del r
+            torch.cuda.empty_cache()
+        line["workloads"] = extra
+        line["device_status"] = line["device_status"] or B.dp_device_status()
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        reps, el = cpu_baseline_ours(wl, args.cpu_seconds)
-        line["cpu_baseline"] = {"value": round(wl_flops(wl) * reps / el / 1e12, 6), "unit": "TFLOP/s",
-                                "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
-                                "sample": f"{reps} full displaced steps of {wl.name} in {el:.1f} s"}
+        line["cpu_baseline"] = cpu_baseline_ours(wl, args.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist:
@@ -479,10 +599,12 @@ def run_ours(args, wl):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="resblock_320x128x128")
+    ap.add_argument("--workload", default="gn_conv_320x480x480")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="time only --workload (skip the other workloads' lines)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--gn-stats", choices=GN_STATS_NAMES, default="corrected",

@@ -203,6 +203,10 @@ int desc_check(const dp_block_desc* d) {
     if (d->Cout != d->C) return set_error(DP_ERR_INVALID_ARG, "block: transformer keeps C");
     if (d->heads <= 0 || d->C != d->heads * 64)
       return set_error(DP_ERR_UNSUPPORTED, "block: transformer needs C == heads * 64");
+    // the block's LayerNorms hold a token in one warp's registers; reject wider
+    // tokens here, before a step has launched anything
+    if (d->C > kLnMaxC)
+      return set_error(DP_ERR_UNSUPPORTED, "block: transformer needs C <= %d (LayerNorm width)", kLnMaxC);
     const int T = d->H * d->W;
     if ((T / d->P) % 128 || T % 256)
       return set_error(DP_ERR_UNSUPPORTED, "block: transformer needs (H*W/P) %% 128 == 0 and H*W %% 256 == 0");

@@ -6,6 +6,10 @@
 
 namespace dp {
 
+// Widest token dp_layernorm takes: a warp holds one token, 8 bf16 per lane
+// per 16-byte vector, at most 8 vectors per lane.
+constexpr int kLnMaxC = 32 * 8 * 8;
+
 size_t gn_acc_bytes(int P, int G);
 size_t gn_workspace_bytes(int P, int G);
 bool gn_cluster_plan(int H, int W, int C, int G, int P, int dtype, int mode, int* cpb, int* chunk,

@@ -20,7 +20,7 @@
 
 namespace dp {
 
-constexpr int kLnMaxVec = 8;   // 16-byte vectors per lane: C <= 32 * 8 * 8 = 2048
+constexpr int kLnMaxVec = kLnMaxC / (32 * 8);   // 16-byte vectors per lane
 
 template <int NV>
 __global__ void __launch_bounds__(256) layernorm_kernel(const __nv_bfloat16* __restrict__ x,
@@ -127,7 +127,15 @@ int dp_layernorm(const void* x, void* y, const float* gamma, const float* beta, 
   if (!(eps > 0.f)) return dp::set_error(DP_ERR_INVALID_ARG, "layernorm: eps must be > 0");
   if (!dp::aligned16(x) || !dp::aligned16(y) || !dp::aligned16(gamma) || !dp::aligned16(beta))
     return dp::set_error(DP_ERR_UNSUPPORTED, "layernorm: pointers must be 16-byte aligned");
-  if (x == y) return dp::set_error(DP_ERR_INVALID_ARG, "layernorm: y aliases x");
+  {
+    // each warp reads its token before writing it, but another warp's rows may be
+    // read after this one's are written: y may not overlap x at all
+    const char* xb8 = static_cast<const char*>(x);
+    const char* yb8 = static_cast<const char*>(y);
+    const size_t bytes = static_cast<size_t>(T) * C * 2;
+    if (xb8 < yb8 + bytes && yb8 < xb8 + bytes)
+      return dp::set_error(DP_ERR_INVALID_ARG, "layernorm: y overlaps x");
+  }
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   const unsigned blocks = static_cast<unsigned>((static_cast<long>(T) * 32 + 255) / 256);
   const int nv = (C / 8 + 31) / 32;

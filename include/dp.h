@@ -159,7 +159,10 @@ DP_API int dp_groupnorm_async(const void* x, void* y, const float* gamma, const 
  *  - Every GPU that loads the library holds those 64 KiB until the process
  *    exits.
  *  - The first call on a device looks the array's device address up
- *    (cudaGetSymbolAddress); make that first call before any stream capture.
+ *    (cudaGetSymbolAddress) and keeps it for the life of the process; make
+ *    that first call before any stream capture.  The kept address does not
+ *    survive cudaDeviceReset (or any re-creation of the device's primary
+ *    context): do not call this entry point on a device after resetting it.
  *  - Each call clears the part of the scratch it uses (a cudaMemsetAsync of
  *    256 + 128 * P * G bytes on `stream`) before its kernels; nothing is
  *    allocated.

@@ -263,6 +263,9 @@ def test_token_operators_reject_bad_arguments_on_the_host(B):
     with pytest.raises(B.DPError) as e:   # y aliases x
         B.dp_layernorm(16, 16, 32, 48, 4, 64, 1e-5, stream=0)
     assert e.value.code == B.DP_ERR_INVALID_ARG
+    with pytest.raises(B.DPError) as e:   # y overlaps x in part (4 tokens x 64 x 2 bytes = 512)
+        B.dp_layernorm(4096, 4096 + 256, 32, 48, 4, 64, 1e-5, stream=0)
+    assert e.value.code == B.DP_ERR_INVALID_ARG
     with pytest.raises(B.DPError) as e:   # F not a multiple of 8
         B.dp_geglu(16, 4096, 4, 12, stream=0)
     assert e.value.code == B.DP_ERR_UNSUPPORTED
@@ -288,6 +291,12 @@ def test_transformer_block_plan_on_the_host(B):
     fl = sum(B.dp_block_launch_info(d, B.DISPLACED, i)[1] for i in range(B.dp_block_launch_count(d)))
     assert abs(fl - B.dp_block_flops(d)) < 1e-6 * fl
     assert B.dp_block_workspace_size(d) > 64 * 64 * 2560 * 2 * 2
+    # tokens wider than one LayerNorm warp holds are rejected before any step runs
+    dw = B.dp_block_desc_init(B.TRANSFORMER, 32, 32, 2112, 2112, 32, 4, 33, B.BF16, 0, 1e-5, 1.0)
+    with pytest.raises(B.DPError, match="LayerNorm width") as e:
+        B.dp_block_desc_set_context(dw, 77, 2048, 4 * 2112)
+        B.dp_block_workspace_size(dw)
+    assert e.value.code in (B.DP_ERR_UNSUPPORTED, B.DP_ERR_INVALID_ARG)
     dr = B.dp_block_desc_init(B.RESBLOCK, 64, 64, 320, 320, 32, 4, 0, B.BF16, 1, 1e-5, 1.0)
     with pytest.raises(B.DPError, match="only for TRANSFORMER"):
         B.dp_block_desc_set_context(dr, 77, 2048, 1280)

@@ -1,4 +1,4 @@
-"""The GroupNorm entry point that allocates nothing, against the workspace one.
+"""The GroupNorm entry point that allocates nothing, against the workspace one and the oracle.
 
 dp_groupnorm_async_noalloc serves callers that cannot allocate device memory
 (code that must not trigger cudaMalloc's device synchronisation, hosts with a
@@ -50,6 +50,13 @@ def test_groupnorm_noalloc_matches_workspace_call_twice_in_a_row():
         np.testing.assert_allclose(host(f), host(f_ref), rtol=0, atol=STATS_ATOL)
         np.testing.assert_allclose(host(u), host(u_ref), rtol=0, atol=STATS_ATOL)
         check(host_img(y), host_img(y_ref), what=f"noalloc call {call}", storage_rel=BF16_HALF_ULP)
+        # and against the oracle itself: output, fresh moments and the moments used
+        f32 = lambda a: np.asarray(a, dtype=np.float32).astype(np.float64)   # as the device holds them
+        y_o, f_o, u_o, _ = O.groupnorm_async(x, f32(gamma), f32(beta), P, G, 1e-5, 1.0, True, mode,
+                                             f32(sg), f32(sl))
+        np.testing.assert_allclose(host(f), f_o.reshape(-1), rtol=0, atol=STATS_ATOL)
+        np.testing.assert_allclose(host(u), u_o.reshape(-1), rtol=0, atol=STATS_ATOL)
+        check(host_img(y), y_o, what=f"noalloc call {call} vs oracle", storage_rel=BF16_HALF_ULP)
     assert B.dp_device_status() == 0
 
 
