@@ -52,6 +52,9 @@ _SIGS = {
     "dp_version": ([], ctypes.c_char_p),
     "dp_mode_for_step": ([_I, _I], _I),
     "dp_device_status": ([_V, ctypes.POINTER(_I)], _I),
+    "dp_selftest_bounded_wait": ([_I, ctypes.c_uint, _V], _I),
+    "dp_block_status": ([ctypes.POINTER(BlockDesc), ctypes.POINTER(BlockState), _V,
+                         ctypes.POINTER(_I)], _I),
     "dp_groupnorm_workspace_size": ([_I, _I, _I, _I, _I], _SZ),
     "dp_groupnorm_async": ([_V, _V, _V, _V, _I, _I, _I, _I, _I, _F, _F, _I, _I, _I, _V, _V, _V, _V,
                             _V, _SZ, _V], _I),
@@ -147,6 +150,19 @@ def dp_mode_for_step(step: int, warmup: int) -> int:
 def dp_device_status(stream=None) -> int:
     st = ctypes.c_int(0)
     _check(lib().dp_device_status(_s(stream), ctypes.byref(st)))
+    return st.value
+
+
+SELFTEST_WAIT_MBARRIER, SELFTEST_WAIT_FLAG = 0, 1
+
+
+def dp_selftest_bounded_wait(kind, limit_us, stream=None):
+    return _check(lib().dp_selftest_bounded_wait(kind, limit_us, _s(stream)))
+
+
+def dp_block_status(d: "BlockDesc", s: "BlockState", stream=None) -> int:
+    st = ctypes.c_int(0)
+    _check(lib().dp_block_status(ctypes.byref(d), ctypes.byref(s), _s(stream), ctypes.byref(st)))
     return st.value
 
 
@@ -355,6 +371,10 @@ class Block:
 
     def step_timed(self, x, out, weights, mode, events, stream=None):
         return dp_block_step_timed(self.desc, self.state, x, out, weights, mode, events, stream)
+
+    def status(self, stream=None) -> int:
+        """Reads and clears this block's own device status word (DP_OK or DP_ERR_TIMEOUT)."""
+        return dp_block_status(self.desc, self.state, stream)
 
     @property
     def launches(self) -> int:

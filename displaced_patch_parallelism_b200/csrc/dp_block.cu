@@ -49,6 +49,7 @@ struct GnSlots {
 constexpr int kU1 = 320, kU2 = 640, kU3 = 1280;
 
 struct Layout {
+  size_t status;                      // the block state's device status word
   GnSlots gn1, gn2;
   size_t a1[2], a2[2], h, sc;        // conv inputs (pairs), conv1 output, shortcut output
   size_t act, q, k[2], v[2], o;      // attention buffers
@@ -108,6 +109,7 @@ Layout layout_of(const dp_block_desc* d) {
   Bump b;
   const size_t e = d->dtype == DP_FP32 ? 4 : 2;
   const size_t hw = static_cast<size_t>(d->H) * d->W;
+  L.status = b.take(sizeof(int));
   if (d->kind == DP_BLOCK_GN_CONV) {
     L.gn1 = gn_slots(b, d->P, d->G);
     for (int i = 0; i < 2; ++i) L.a1[i] = b.take(hw * d->C * e);
@@ -694,12 +696,27 @@ int dp_block_step(const dp_block_desc* d, dp_block_state* s, const void* x, void
                          dp::weight_count(d));
   if (s->workspace_bytes < dp::layout_of(d).total)
     return dp::set_error(DP_ERR_INVALID_ARG, "block: workspace too small");
-  rc = dp::step_impl(d, s->workspace, s->cur, x, out, weights, mode,
-                     static_cast<cudaStream_t>(stream), nullptr);
+  {
+    // every kernel of this step reports a timed-out wait in the state's own word
+    dp::StatusScope scope(reinterpret_cast<int*>(static_cast<char*>(s->workspace) +
+                                                 dp::layout_of(d).status));
+    rc = dp::step_impl(d, s->workspace, s->cur, x, out, weights, mode,
+                       static_cast<cudaStream_t>(stream), nullptr);
+  }
   if (rc) return rc;
   s->cur ^= 1;
   s->steps_done += 1;
   return DP_OK;
+}
+
+int dp_block_status(const dp_block_desc* d, const dp_block_state* s, void* stream, int* status) {
+  int rc = dp::desc_check(d);
+  if (rc) return rc;
+  if (!s || !s->workspace || !status) return dp::set_error(DP_ERR_INVALID_ARG, "block: null argument");
+  const dp::Layout L = dp::layout_of(d);
+  if (s->workspace_bytes < L.total) return dp::set_error(DP_ERR_INVALID_ARG, "block: workspace too small");
+  return dp::read_clear_status(reinterpret_cast<int*>(static_cast<char*>(s->workspace) + L.status),
+                               static_cast<cudaStream_t>(stream), status);
 }
 
 int dp_block_launch_count(const dp_block_desc* d) {

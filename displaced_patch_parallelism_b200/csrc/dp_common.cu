@@ -18,6 +18,11 @@ namespace dp {
 __device__ int g_status_word = 0;
 
 static thread_local char t_last_error[512] = "";
+// The status word of the block step running on this thread (null: none).
+static thread_local int* t_status_word = nullptr;
+
+StatusScope::StatusScope(int* word) : prev_(t_status_word) { t_status_word = word; }
+StatusScope::~StatusScope() { t_status_word = prev_; }
 
 struct LaunchRecorder {
   void* const* events = nullptr;
@@ -67,6 +72,7 @@ int cuda_check(cudaError_t e, const char* what) {
 }
 
 int* device_status_ptr() {
+  if (t_status_word) return t_status_word;
   static int* ptrs[64] = {nullptr};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
@@ -119,6 +125,23 @@ int encode_tmap(CUtensorMap* map, CUtensorMapDataType dt, int rank, void* base,
   return DP_OK;
 }
 
+int read_clear_status(int* word, cudaStream_t s, int* out) {
+  int host = 0;
+  int rc = cuda_check(cudaMemcpyAsync(&host, word, sizeof(int), cudaMemcpyDeviceToHost, s),
+                      "read status");
+  if (rc) return rc;
+  rc = cuda_check(cudaStreamSynchronize(s), "sync for status");
+  if (rc) return rc;
+  if (host != 0) {
+    rc = cuda_check(cudaMemsetAsync(word, 0, sizeof(int), s), "clear status");
+    if (rc) return rc;
+    rc = cuda_check(cudaStreamSynchronize(s), "sync after clear");
+    if (rc) return rc;
+  }
+  *out = host;
+  return DP_OK;
+}
+
 }  // namespace dp
 
 extern "C" {
@@ -136,23 +159,9 @@ int dp_mode_for_step(int step, int warmup) {
 
 int dp_device_status(void* stream, int* status) {
   if (!status) return dp::set_error(DP_ERR_INVALID_ARG, "status is NULL");
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* p = dp::device_status_ptr();
   if (!p) return dp::set_error(DP_ERR_CUDA, "status word address unavailable");
-  int host = 0;
-  int rc = dp::cuda_check(cudaMemcpyAsync(&host, p, sizeof(int), cudaMemcpyDeviceToHost, s),
-                          "read status");
-  if (rc) return rc;
-  rc = dp::cuda_check(cudaStreamSynchronize(s), "sync for status");
-  if (rc) return rc;
-  if (host != 0) {
-    rc = dp::cuda_check(cudaMemsetAsync(p, 0, sizeof(int), s), "clear status");
-    if (rc) return rc;
-    rc = dp::cuda_check(cudaStreamSynchronize(s), "sync after clear");
-    if (rc) return rc;
-  }
-  *status = host;
-  return DP_OK;
+  return dp::read_clear_status(p, static_cast<cudaStream_t>(stream), status);
 }
 
 }  // extern "C"

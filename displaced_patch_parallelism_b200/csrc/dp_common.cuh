@@ -2,10 +2,11 @@
 //
 // PTX wrappers for mbarriers, TMA tile loads and the 5th-generation tensor
 // core (tcgen05: tensor-memory allocation, MMA, commit, loads), plus the
-// bounded wait every kernel uses: no spin in this library is unbounded; a
+// bounded waits every kernel uses: no spin in this library is unbounded; a
 // wait that runs out sets an abort flag in shared memory, records
-// DP_ERR_TIMEOUT in the library's device status word and lets every role of
-// the block fall through to its teardown.
+// DP_ERR_TIMEOUT in the status word the launch was given (the block state's
+// own word during a block step, else the library's word for the device) and
+// lets every role of the block fall through to its teardown.
 #pragma once
 
 #include <cuda.h>
@@ -20,7 +21,25 @@ namespace dp {
 // ---------------------------------------------------------------- host side
 int set_error(int code, const char* fmt, ...);
 int cuda_check(cudaError_t e, const char* what);
-int* device_status_ptr();         // device address of the status word (current device)
+// Device address of the status word kernels launched now should write: the
+// word of the block step running on this thread, else the library's word for
+// the current device.
+int* device_status_ptr();
+// While alive, launches made by this thread write their timeouts to `word`
+// (a block state's own status word) instead of the library's word.
+class StatusScope {
+ public:
+  explicit StatusScope(int* word);
+  ~StatusScope();
+  StatusScope(const StatusScope&) = delete;
+  StatusScope& operator=(const StatusScope&) = delete;
+
+ private:
+  int* prev_;
+};
+// Reads the device status word `word` into *out after `s` has drained, and
+// clears it if it was set.
+int read_clear_status(int* word, cudaStream_t s, int* out);
 int num_sms();                    // SM count of the current device
 int encode_tmap(CUtensorMap* map, CUtensorMapDataType dt, int rank, void* base,
                 const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
@@ -119,10 +138,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase of `bar` with parity `parity` to complete.  Returns
-// false if the block is aborting or the wait ran past kWaitLimitNs (then it
+// false if the block is aborting or the wait ran past `limit_ns` (then it
 // raises the abort flag and records DP_ERR_TIMEOUT in *status).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int* status) {
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity,
+                                                volatile int* abort_flag, int* status,
+                                                unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   uint32_t n = 0;
@@ -130,13 +150,49 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_try_wait(bar, parity)) return true;
     if ((++n & 63u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         if (status) atomicExch(status, DP_ERR_TIMEOUT);
         return false;
       }
     }
   }
+}
+
+// The wait every kernel's pipeline uses: limit kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          int* status) {
+  return mbar_wait_limit(bar, parity, abort_flag, status, kWaitLimitNs);
+}
+
+// Global-memory flags between blocks: release arrival, acquire polling.
+__device__ __forceinline__ unsigned atom_add_release_gpu(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.add.release.gpu.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(unsigned* p, unsigned v) {
+  asm volatile("st.release.gpu.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Waits (acquire) until the flag at `p` no longer holds `v`.  Returns false,
+// recording DP_ERR_TIMEOUT in *status, if that takes longer than `limit_ns`.
+__device__ __forceinline__ bool flag_wait_change(const unsigned* p, unsigned v, int* status,
+                                                 unsigned long long limit_ns) {
+  const unsigned long long t0 = globaltimer_ns();
+  uint32_t n = 0;
+  while (ld_acquire_gpu(p) == v) {
+    if ((++n & 63u) == 0 && globaltimer_ns() - t0 > limit_ns) {
+      if (status) atomicExch(status, DP_ERR_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
 }
 
 // ---- TMA tile loads (plain tiled loads only: every CTA fetches its own tiles)

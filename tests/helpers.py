@@ -14,8 +14,10 @@ the other four workloads' own chains keep the plain 2e-2 bound.
 Blocks with a channel-changing shortcut add a bf16-stored shortcut tensor
 whose elements can be larger than the output element they feed; a one-ulp
 storage flip there is bounded by 2^-7 * max|ref| rather than by the output
-element (``scale_rel``).  The 8-stage mini U-Net chain is held end to end to
-a bound derived from its depth (see tests/test_gpu_blocks.py).
+element (``scale_rel``).
+
+Chains of bf16-stored stages (the 8-stage mini U-Net, the transformer block)
+are held end to end by ``check_chain``: see its docstring.
 """
 import numpy as np
 import torch
@@ -86,3 +88,30 @@ def check(gpu: np.ndarray, ref: np.ndarray, atol=ATOL, rl2=RL2, what="", storage
                              f"rel-L2 {rel:.2e}")
     assert rel <= rl2, f"{what}: rel-L2 {rel:.3e} > {rl2:.1e} (max-abs {maxabs:.2e})"
     return maxabs, rel
+
+
+# A chain of stages that each store their output in bf16 drifts from the exact
+# (unrounded fp64) method by an amount set by that storage alone.  The oracle
+# measures it in the same test: its result with bf16 storage at the GPU's
+# storage points, against its exact result.  For the 8-stage mini U-Net that
+# floor is 5.5e-3 rel-L2, above the 5e-3 bar, so no bf16 chain can meet the
+# bar there; the GPU is then held to the floor instead, allowed to exceed the
+# oracle's own storage-only distance by 10 % (rel-L2) and 50 % (largest
+# element).  Where the floor is below the bar, the bar applies.
+CHAIN_RL2_RATIO = 1.10
+CHAIN_MAX_RATIO = 1.5
+
+
+def check_chain(gpu, exact, stored, what=""):
+    """Holds ``gpu`` against the oracle's ``exact`` result (no storage rounding) with the
+    stated bar, or -- where the oracle's own bf16-stored result ``stored`` is already further
+    from ``exact`` than the bar -- with the floor that storage sets (see above)."""
+    exact = np.asarray(exact, dtype=np.float64)
+    stored = np.asarray(stored, dtype=np.float64)
+    nref = float(np.linalg.norm(exact))
+    floor_rl2 = float(np.linalg.norm(stored - exact)) / nref
+    floor_max = float(np.abs(stored - exact).max())
+    rl2 = max(RL2, CHAIN_RL2_RATIO * floor_rl2)
+    atol = max(ATOL, CHAIN_MAX_RATIO * floor_max)
+    maxabs, rel = check(gpu, exact, atol=atol, rl2=rl2, what=what, storage_rel=BF16_HALF_ULP)
+    return {"rel_l2": rel, "max_abs": maxabs, "floor_rel_l2": floor_rl2, "floor_max_abs": floor_max}

@@ -407,3 +407,14 @@ def test_transformer_workload_marshals_to_the_block(B):
               (C, C), (C,)]
     assert [tuple(t.shape) for t in w] == shapes
     assert tuple(synth.context(wl).shape) == (Tk, Cc)
+
+
+def test_selftest_and_block_status_reject_bad_arguments_on_the_host(B):
+    for kind, limit in [(2, 100), (-1, 100), (0, 0), (1, 2000000)]:
+        with pytest.raises(B.DPError) as e:
+            B.dp_selftest_bounded_wait(kind, limit, stream=0)
+        assert e.value.code == B.DP_ERR_INVALID_ARG
+    d = B.dp_block_desc_init(B.GN_CONV, 16, 16, 64, 64, 32, 2, 0, B.BF16, 1, 1e-5, 1.0)
+    with pytest.raises(B.DPError) as e:   # a state never initialised has no workspace
+        B.dp_block_status(d, B.BlockState(), stream=0)
+    assert e.value.code == B.DP_ERR_INVALID_ARG
