@@ -8,7 +8,8 @@ synthetic inputs already resident in HBM.  The default workload is the largest
 single-GPU one: the 3840x3840-shaped GroupNorm + SiLU + 3x3 conv block, latent
 1x320x480x480, P = 8 bands of 60 rows.  Each step is timed with CUDA events
 recorded on the launching stream just before and after it.  Between steps L2
-is flushed (a 256 MiB write, outside the timed events) unless the step's input
+is flushed (a 256 MiB write, then a 256 MiB read that writes its dirty lines back,
+both outside the timed events) unless the step's input
 alone is larger than L2, in which case the inputs themselves evict it.  A
 second pass with an event before every kernel (``dp_block_step_timed``) gives
 the per-kernel breakdown and the roofline of the dominant kernel.  The other
@@ -40,10 +41,28 @@ sys.path.insert(0, ROOT)
 
 METRIC = "displaced U-Net block step latency & TFLOP/s; GroupNorm GB/s; % of roofline"
 FLUSH_BYTES = 256 << 20
+
+
+class L2Flush:
+    """Empties L2 between timed steps, outside the timed events: a 256 MiB write (evicting
+    everything), then a 256 MiB read of a second buffer, which writes the first buffer's dirty
+    lines back and leaves L2 holding clean lines only.  The next step then starts with a cold
+    cache and pays for no write-back of the flush itself."""
+
+    def __init__(self, dev):
+        import torch
+        self.w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        self.r = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def __call__(self):
+        self.w.zero_()
+        self.r.sum()
 # GroupNorm statistics of the displaced steps (--gn-stats): the method's
 # corrected statistics (default) or one of its ablation alternatives
 GN_STATS_NAMES = ["corrected", "local", "stale", "sync"]
 GN_STATS = 0
+# --gn-fuse: GroupNorm -> conv pairs through the conv that normalises its own input
+GN_FUSE = False
 
 
 def load_peaks():
@@ -173,6 +192,8 @@ def block_desc(B, wl, H=None):
     if wl_context(wl):
         B.dp_block_desc_set_context(d, *wl_context(wl))
     B.dp_block_desc_set_gn_stats(d, GN_STATS)
+    if GN_FUSE:
+        B.dp_block_desc_set_gn_fusion(d, 1)
     return d
 
 
@@ -318,12 +339,14 @@ def l2_policy(wl):
     if input_bytes(wl) > L2_BYTES:
         return False, (f"inputs larger than L2 ({input_bytes(wl) / 1e6:.1f} MB input per step, "
                        f"4 inputs in rotation); no flush")
-    return True, "flushed between steps (256 MiB write, outside the timed events)"
+    return True, ("flushed between steps (256 MiB write, then a 256 MiB read that writes the dirty "
+                  "lines back; both outside the timed events)")
 
 
 def workload_config(wl, ws, extra=None):
     cfg = {"workload": wl.name, "shape_nchw": [1, wl.C, wl.H, wl.W], "P": wl.P,
            "mode": "displaced", "gn_stats": GN_STATS_NAMES[GN_STATS],
+           "gn_conv": "fused (conv normalises its input)" if GN_FUSE else "separate passes",
            "l2": l2_policy(wl)[1],
            "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"}
     if wl.dtype == "fp32":
@@ -349,7 +372,7 @@ class Run:
             self.dw.append(synth.context(wl).to(self.tdt).to(dev))
         self.blk = B.Block(block_kind(B, wl), wl.H, wl.W, wl.C, wl.cout, wl.G, wl.P, wl.heads,
                            B.BF16 if wl.dtype == "bf16" else B.FP32, wl.silu, wl.eps, 1.0,
-                           device=dev, gn_stats=GN_STATS, context=wl_context(wl))
+                           device=dev, gn_stats=GN_STATS, context=wl_context(wl), gn_fuse=GN_FUSE)
         xs = synth.InputStream(wl)
         self.pool = pool
         self.host_x = [synth.nchw_to_nhwc(xs.x(k)).to(self.tdt).pin_memory() for k in range(pool)]
@@ -385,7 +408,7 @@ def time_steps(run, steps, flush, dist, sampler=None):
     wall0 = time.perf_counter()
     for k in range(steps):
         if run.flush_between:
-            flush.zero_()
+            flush()
         ev0[k].record()
         run.blk.step(run.dev_x[k % run.pool], run.out, run.dw, run.B.DISPLACED)
         ev1[k].record()
@@ -412,7 +435,7 @@ def breakdown(run, steps, flush, peaks):
     torch.cuda.synchronize()
     for k in range(n_bd):
         if run.flush_between:
-            flush.zero_()
+            flush()
         run.blk.step_timed(run.dev_x[k % run.pool], run.out, run.dw, run.B.DISPLACED, events[k])
     torch.cuda.synchronize()
     per_launch = [[events[k][i].elapsed_time(events[k][i + 1]) for i in range(n_launch)]
@@ -436,7 +459,8 @@ def breakdown(run, steps, flush, peaks):
                       "gbs": round(by / (avg_us * 1e-6) / 1e9, 1)}
     dominant = max(role_ms, key=lambda r: role_ms[r])
     dk = kernels[dominant]
-    src = {"conv": ["dp_gemm.cu"], "linear": ["dp_gemm.cu"], "attn": ["dp_attn.cu"],
+    src = {"conv": ["dp_gemm.cu"], "conv_gn": ["dp_gemm.cu"], "linear": ["dp_gemm.cu"],
+           "attn": ["dp_attn.cu"],
            "gn_stats": ["dp_gn.cu"], "gn_apply": ["dp_gn.cu"], "gn_fused": ["dp_gn.cu"],
            "gn_cluster": ["dp_gn.cu"], "copy": ["dp_refresh.cu"],
            "conv_small": ["dp_conv_small.cu"], "splitk_finish": ["dp_gemm.cu"],
@@ -532,7 +556,7 @@ def run_ours(args, wl):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     dev = torch.device("cuda", local)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     peaks = load_peaks()
 
     run = Run(wl, dev)
@@ -609,9 +633,12 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--gn-stats", choices=GN_STATS_NAMES, default="corrected",
                     help="GroupNorm statistics of the displaced steps")
+    ap.add_argument("--gn-fuse", action="store_true",
+                    help="GroupNorm -> conv pairs through the conv that normalises its own input")
     args = ap.parse_args()
-    global GN_STATS
+    global GN_STATS, GN_FUSE
     GN_STATS = GN_STATS_NAMES.index(args.gn_stats)
+    GN_FUSE = args.gn_fuse
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     from displaced_patch_parallelism_b200 import synth

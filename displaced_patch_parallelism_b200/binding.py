@@ -38,7 +38,7 @@ class BlockDesc(ctypes.Structure):
                 ("P", ctypes.c_int), ("heads", ctypes.c_int), ("dtype", ctypes.c_int),
                 ("silu", ctypes.c_int), ("eps", ctypes.c_float), ("w", ctypes.c_float),
                 ("gn_stats", ctypes.c_int), ("ctx_len", ctypes.c_int), ("ctx_dim", ctypes.c_int),
-                ("ff_inner", ctypes.c_int), ("temb_dim", ctypes.c_int)]
+                ("ff_inner", ctypes.c_int), ("temb_dim", ctypes.c_int), ("gn_fuse", ctypes.c_int)]
 
 
 class BlockState(ctypes.Structure):
@@ -61,6 +61,9 @@ _SIGS = {
     "dp_groupnorm_async_noalloc": ([_V, _V, _V, _V, _I, _I, _I, _I, _I, _F, _F, _I, _I, _I, _V, _V,
                                     _V, _V, _V], _I),
     "dp_gemm_workspace_size": ([], _SZ),
+    "dp_groupnorm_stats": ([_V, _I, _I, _I, _I, _I, _F, _I, _I, _V, _V, _V, _V, _V, _SZ, _V], _I),
+    "dp_conv3x3_halo_gn": ([_V, _V, _V, _V, _V, _V, _I, _F, _I, _V, _V, _V, _V, _I, _I, _I, _I, _I, _I,
+                            _V], _I),
     "dp_conv3x3_halo": ([_V, _V, _V, _V, _V, _V, _I, _I, _I, _I, _I, _I, _I, _I, _V, _SZ, _V], _I),
     "dp_conv3x3_halo_small": ([_V, _V, _V, _V, _V, _I, _I, _I, _I, _I, _I, _V], _I),
     "dp_linear": ([_V, _V, _V, _V, _V, _V, _V, _I, _I, _I, _I, _V, _SZ, _V], _I),
@@ -76,6 +79,7 @@ _SIGS = {
     "dp_refresh_stats": ([_V, _V, _V, _I, _I, _V], _I),
     "dp_block_desc_init": ([ctypes.POINTER(BlockDesc), _I, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _F], _I),
     "dp_block_desc_set_gn_stats": ([ctypes.POINTER(BlockDesc), _I], _I),
+    "dp_block_desc_set_gn_fusion": ([ctypes.POINTER(BlockDesc), _I], _I),
     "dp_block_desc_set_context": ([ctypes.POINTER(BlockDesc), _I, _I, _I], _I),
     "dp_block_desc_set_time_embedding": ([ctypes.POINTER(BlockDesc), _I], _I),
     "dp_block_workspace_size": ([ctypes.POINTER(BlockDesc)], _SZ),
@@ -205,6 +209,22 @@ def dp_conv3x3_halo_small(a_fresh, a_stale, weight, bias, out, H, W, Cin, Cout, 
                                               _p(out), H, W, Cin, Cout, P, mode, _s(stream)))
 
 
+def dp_groupnorm_stats(x, H, W, C, G, P, w, mode, dtype, stale_global, stale_local, fresh_local,
+                       used_stats, workspace, workspace_bytes=None, stream=None):
+    if workspace_bytes is None:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    return _check(lib().dp_groupnorm_stats(_p(x), H, W, C, G, P, w, mode, dtype, _p(stale_global),
+                                           _p(stale_local), _p(fresh_local), _p(used_stats),
+                                           _p(workspace), workspace_bytes, _s(stream)))
+
+
+def dp_conv3x3_halo_gn(x, a_stale, a_next, used_stats, gamma, beta, G, eps, silu, weight, bias,
+                       residual, out, H, W, Cin, Cout, P, mode, stream=None):
+    return _check(lib().dp_conv3x3_halo_gn(_p(x), _p(a_stale), _p(a_next), _p(used_stats), _p(gamma),
+                                           _p(beta), G, eps, int(silu), _p(weight), _p(bias),
+                                           _p(residual), _p(out), H, W, Cin, Cout, P, mode, _s(stream)))
+
+
 def dp_linear(x, weight, bias, residual, out0, out1, out2, M, N, K, split, workspace=None,
               workspace_bytes=0, stream=None):
     return _check(lib().dp_linear(_p(x), _p(weight), _p(bias), _p(residual), _p(out0), _p(out1),
@@ -273,6 +293,10 @@ def dp_block_desc_set_gn_stats(d: BlockDesc, variant: int):
     return _check(lib().dp_block_desc_set_gn_stats(ctypes.byref(d), variant))
 
 
+def dp_block_desc_set_gn_fusion(d: BlockDesc, on: int):
+    return _check(lib().dp_block_desc_set_gn_fusion(ctypes.byref(d), int(on)))
+
+
 def dp_block_desc_set_context(d: BlockDesc, ctx_len: int, ctx_dim: int, ff_inner: int):
     return _check(lib().dp_block_desc_set_context(ctypes.byref(d), ctx_len, ctx_dim, ff_inner))
 
@@ -324,7 +348,7 @@ def dp_block_step_timed(d: BlockDesc, s: BlockState, x, out, weights: Sequence, 
 
 KERNEL_NAMES = {0: "gn_stats", 1: "gn_apply", 2: "gn_fused", 3: "conv", 4: "linear", 5: "attn",
                 6: "copy", 7: "conv_small", 8: "splitk_finish",
-                9: "gn_cluster", 10: "layernorm", 11: "geglu", 12: "temb"}
+                9: "gn_cluster", 10: "layernorm", 11: "geglu", 12: "temb", 13: "conv_gn"}
 
 
 def dp_block_launch_info(d: BlockDesc, mode: int, i: int):
@@ -351,7 +375,7 @@ class Block:
 
     def __init__(self, kind, H, W, C, Cout=0, G=32, P=4, heads=0, dtype=BF16, silu=True,
                  eps=1e-5, w=1.0, device="cuda", stream=None, gn_stats=GN_STATS_CORRECTED,
-                 context=None, temb_dim=0):
+                 context=None, temb_dim=0, gn_fuse=False):
         """``context`` = (ctx_len, ctx_dim, ff_inner) for TRANSFORMER blocks; ``temb_dim`` the
         time-embedding width of a RESBLOCK (0: none)."""
         import torch
@@ -362,6 +386,8 @@ class Block:
             dp_block_desc_set_time_embedding(self.desc, temb_dim)
         if gn_stats != GN_STATS_CORRECTED:
             dp_block_desc_set_gn_stats(self.desc, gn_stats)
+        if gn_fuse:
+            dp_block_desc_set_gn_fusion(self.desc, 1)
         self.ws_bytes = dp_block_workspace_size(self.desc)
         self.workspace = torch.empty(self.ws_bytes, dtype=torch.uint8, device=device)
         self.state = dp_block_state_init(self.desc, self.workspace, self.ws_bytes, stream)

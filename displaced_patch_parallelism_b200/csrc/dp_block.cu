@@ -170,6 +170,8 @@ Layout layout_of(const dp_block_desc* d) {
 }
 
 int desc_check(const dp_block_desc* d) {
+  if (d && d->gn_fuse != 0 && d->gn_fuse != 1)
+    return set_error(DP_ERR_INVALID_ARG, "block: gn fusion flag %d is not 0 or 1", d->gn_fuse);
   if (!d) return set_error(DP_ERR_INVALID_ARG, "block: null descriptor");
   if (d->kind < DP_BLOCK_GN_CONV || d->kind > DP_BLOCK_TRANSFORMER)
     return set_error(DP_ERR_INVALID_ARG, "block: bad kind %d", d->kind);
@@ -282,6 +284,13 @@ struct Plan {
 
 // One step of the block described by `d` whose state lives at `ws`; `cur`
 // selects the stale half of every ping-pong pair (the fresh half is cur ^ 1).
+// Whether a GroupNorm -> 3x3 conv pair of this block runs as the statistics
+// pass plus the conv that normalises its own input tiles: when the descriptor
+// asks for it (dp_block_desc_set_gn_fusion) and the shapes allow it.
+bool gn_conv_fused(const dp_block_desc* d, int ch, int co) {
+  return d->gn_fuse == 1 && conv3x3_gn_eligible(d->H, d->W, ch, co, d->G, d->dtype);
+}
+
 int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* out,
               const void* const* w, int mode, cudaStream_t st, Plan* plan) {
   const Layout L = layout_of(d);
@@ -354,6 +363,39 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
     return linear_launch(in, wt, static_cast<const float*>(b), res, o0, o1, o2, M, N, K, split,
                          at<void>(ws, L.gemm_ws), gemm_workspace_bytes(), st);
   };
+  // GroupNorm (+SiLU) -> 3x3 conv, in two calls: gn_part, then conv_part.
+  // Where the conv can normalise its own input tiles (gn_conv_fused), the
+  // GroupNorm runs as its statistics pass only and the conv reads x itself:
+  // the normalised activations never go through HBM, and the ping-pong
+  // buffer `a` receives only the band-edge rows, the rows the next step's
+  // displaced conv reads from other bands.  Otherwise the GroupNorm writes
+  // `a` whole and the conv reads it.
+  auto gn_part = [&](const GnSlots& g, const void* in, const size_t a_off[2], const void* gamma,
+                     const void* beta, int ch, int co, int silu) {
+    if (!gn_conv_fused(d, ch, co)) return gn(g, in, at<void>(ws, a_off[f]), gamma, beta, ch, silu);
+    if (plan) {
+      plan->push(DP_KERNEL_GN_STATS, 0.0, static_cast<double>(H) * W * ch * e);
+      return DP_OK;
+    }
+    return gn_stats_launch(in, H, W, ch, G, P, gn_w, gn_mode, d->dtype, at<float>(ws, g.global[o]),
+                           at<float>(ws, g.local[o]), at<float>(ws, g.local[f]),
+                           at<float>(ws, g.global[f]), at<float>(ws, g.used), at<void>(ws, g.ws), st);
+  };
+  auto conv_part = [&](const GnSlots& g, const void* in, const size_t a_off[2], const void* gamma,
+                       const void* beta, int ch, int co, int silu, const void* wt, const void* b,
+                       const void* res, void* y) {
+    if (!gn_conv_fused(d, ch, co))
+      return conv(at<void>(ws, a_off[f]), at<void>(ws, a_off[o]), wt, b, res, y, H, W, ch, co, 1);
+    if (plan) {
+      const double hw = static_cast<double>(H) * W;
+      plan->push(DP_KERNEL_CONV_GN, 2.0 * hw * co * 9.0 * ch,
+                 (hw * ch + hw * co * (res ? 2 : 1) + 2.0 * P * W * ch) * e);
+      return DP_OK;
+    }
+    return conv3x3_gn_launch(in, at<void>(ws, a_off[o]), at<void>(ws, a_off[f]), at<float>(ws, g.used),
+                             static_cast<const float*>(gamma), static_cast<const float*>(beta), G, d->eps,
+                             silu, wt, static_cast<const float*>(b), res, y, H, W, ch, co, P, mode, st);
+  };
   int rc;
   if (d->kind != DP_BLOCK_UNET_MINI && !plan) {
     // biases (conv_b, conv1_b, conv2_b, short_b, temb_b; bqkv, bo, ...) may be NULL
@@ -372,10 +414,10 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
       rc = conv3x3_validate(x, x, w[2], nullptr, out, H, W, C, Co, 1, P, mode, d->dtype);
       if (rc) return rc;
     }
-    rc = gn(L.gn1, x, at<void>(ws, L.a1[f]), w[0], w[1], C, d->silu);
+    const size_t a1[2] = {L.a1[0], L.a1[1]};
+    rc = gn_part(L.gn1, x, a1, w[0], w[1], C, Co, d->silu);
     if (rc) return rc;
-    return conv(at<void>(ws, L.a1[f]), at<void>(ws, L.a1[o]), w[2], w[3], nullptr, out, H, W, C, Co,
-                1);
+    return conv_part(L.gn1, x, a1, w[0], w[1], C, Co, d->silu, w[2], w[3], nullptr, out);
   }
   if (d->kind == DP_BLOCK_RESBLOCK) {
     if (!plan) {
@@ -384,8 +426,6 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
       rc = conv3x3_validate(x, x, w[6], nullptr, out, H, W, Co, Co, 1, P, mode, d->dtype);
       if (rc) return rc;
     }
-    void* a1f = at<void>(ws, L.a1[f]);
-    void* a2f = at<void>(ws, L.a2[f]);
     void* h = at<void>(ws, L.h);
     const void* b1 = w[3];
     if (d->temb_dim > 0) {
@@ -406,11 +446,12 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
         b1 = tb;
       }
     }
-    rc = gn(L.gn1, x, a1f, w[0], w[1], C, 1);
+    const size_t a1[2] = {L.a1[0], L.a1[1]}, a2[2] = {L.a2[0], L.a2[1]};
+    rc = gn_part(L.gn1, x, a1, w[0], w[1], C, Co, 1);
     if (rc) return rc;
-    rc = conv(a1f, at<void>(ws, L.a1[o]), w[2], b1, nullptr, h, H, W, C, Co, 1);
+    rc = conv_part(L.gn1, x, a1, w[0], w[1], C, Co, 1, w[2], b1, nullptr, h);
     if (rc) return rc;
-    rc = gn(L.gn2, h, a2f, w[4], w[5], Co, 1);
+    rc = gn_part(L.gn2, h, a2, w[4], w[5], Co, Co, 1);
     if (rc) return rc;
     const void* res = x;
     if (C != Co) {
@@ -419,7 +460,7 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
       if (rc) return rc;
       res = sc;
     }
-    return conv(a2f, at<void>(ws, L.a2[o]), w[6], w[7], res, out, H, W, Co, Co, 1);
+    return conv_part(L.gn2, h, a2, w[4], w[5], Co, Co, 1, w[6], w[7], res, out);
   }
   if (d->kind == DP_BLOCK_TRANSFORMER) {
     const int T = H * W, Tk = d->ctx_len, Cc = d->ctx_dim, Fi = d->ff_inner;
@@ -610,6 +651,7 @@ int dp_block_desc_init(dp_block_desc* d, int kind, int H, int W, int C, int Cout
   d->ctx_dim = 0;
   d->ff_inner = 0;
   d->temb_dim = 0;
+  d->gn_fuse = 0;
   if (kind == DP_BLOCK_TRANSFORMER) return DP_OK;   // checked once dp_block_desc_set_context is called
   return dp::desc_check(d);
 }
@@ -632,6 +674,13 @@ int dp_block_desc_set_time_embedding(dp_block_desc* d, int temb_dim) {
     return dp::set_error(DP_ERR_INVALID_ARG, "block: time-embedding width %d outside [0, 8192]", temb_dim);
   d->temb_dim = temb_dim;
   return dp::desc_check(d);
+}
+
+int dp_block_desc_set_gn_fusion(dp_block_desc* d, int on) {
+  if (!d) return dp::set_error(DP_ERR_INVALID_ARG, "block: null descriptor");
+  if (on != 0 && on != 1) return dp::set_error(DP_ERR_INVALID_ARG, "block: gn fusion must be 0 or 1");
+  d->gn_fuse = on;
+  return DP_OK;
 }
 
 int dp_block_desc_set_gn_stats(dp_block_desc* d, int variant) {

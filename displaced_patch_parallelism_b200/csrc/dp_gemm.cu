@@ -32,6 +32,7 @@
 #include <type_traits>
 
 #include "dp_common.cuh"
+#include "dp_gn_apply.cuh"
 #include "dp_internal.h"
 
 namespace dp {
@@ -61,6 +62,16 @@ struct GemmParams {
   // and residual and stores the outputs.
   int splits;
   float* part;
+  // GroupNorm-fused conv only (igemm_gn_pair_kernel): tmA0 maps the raw input
+  // x, tmA1 the previous step's normalised activations; the kernel normalises
+  // each staged input row in shared memory.
+  const float* gn_used;    // [P][G][2]: (mean, var) band p normalises group g with
+  const float* gn_gamma;   // [Cin]
+  const float* gn_beta;    // [Cin]
+  float gn_eps;
+  int gn_cg;               // channels per group
+  int gn_silu;
+  void* a_next;            // [H][W][Cin]: receives the normalised band-edge rows, or null
 };
 
 // k-blocks [*kb0, *kb1) of run `r` of `splits` over `kb` k-blocks.
@@ -495,6 +506,14 @@ __device__ __forceinline__ bool pair_epilogue_tile(const GemmParams& p, uint32_t
   constexpr int NCH = BN / 32;
   static_assert(NCH >= 2, "chunks");
   const int last_ch = ((NCH - 1 - half) / 2) * 2 + half;   // this warp's last chunk
+  // hands the accumulator back after this warp's last chunk has been read
+  auto release = [&](int ch) {
+    if (ch == last_ch) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
+    }
+  };
   const int tile = item / p.splits;
   // Split K: this run's accumulator goes to its fp32 partial, rows at their
   // output pixels; bias, residual and the cast are the finish kernel's.
@@ -513,11 +532,7 @@ __device__ __forceinline__ bool pair_epilogue_tile(const GemmParams& p, uint32_t
       uint32_t r[32];
       tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + ch * 32, r);
       tmem_wait_ld();
-      if (ch == last_ch) {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
-      }
+      release(ch);
       if (!valid) continue;
       float4* d4 = reinterpret_cast<float4*>(dst + ch * 32);
 #pragma unroll
@@ -556,11 +571,7 @@ __device__ __forceinline__ bool pair_epilogue_tile(const GemmParams& p, uint32_t
       uint32_t r[32];
       tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + ch * 32, r);
       tmem_wait_ld();
-      if (ch == last_ch) {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
-      }
+      release(ch);
       if (!b.ok) continue;
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
@@ -859,6 +870,422 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
         break;
     }
     if (lane == 0) bulk_wait_all();   // every store has finished reading its slot
+  }
+
+  tc_fence_before();
+  cluster_sync_all();
+  __syncwarp();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// GroupNorm-fused pair conv: the 3x3 conv of GroupNorm(x) (+SiLU) whose A
+// operand is normalised in shared memory, so the normalised activations are
+// never written to or read back from HBM ("DistriFusion", atlas.scime.ai
+// summary, Approach: the corrected GroupNorm feeds the next layer; study.space
+// summary, Method: other bands' rows are the previous step's activations).
+//
+// Tiles are one output row r x 128 columns (stride 1).  K runs channel block
+// by channel block (64 channels), and for each block the three input rows
+// r-1, r, r+1 are staged once by TMA, 130 pixels each (the tile plus one
+// column of halo on each side), in 128-byte-swizzled rows 136 pixels apart.
+// The nine taps are then nine shifted views of that one staging: tap (kh, kw)
+// starts kh rows and kw pixels in, and the tensor core applies the swizzle to
+// the absolute shared-memory address, so a shifted view reads the bytes the
+// TMA wrote.  Each staged row comes from
+//   * x, the raw input, when it lies in the tile's band (or in any band in a
+//     sync step): the transform warps normalise it in place with that band's
+//     scale and shift (exactly the GroupNorm apply pass's arithmetic);
+//   * the stale normalised activations, when it lies in another band in a
+//     displaced step (already normalised: left as loaded);
+//   * nowhere (zero fill) outside the image or for another band in a naive
+//     step; zero-filled columns outside the image stay zero.
+// The transform warps also write the tile's own row, normalised, to a_next
+// when it is the first or last row of its band: those are the only rows the
+// next step's displaced conv reads from another band, so a_next serves as the
+// next step's stale buffer without a full write.
+//
+// Cost on B200 at the SDXL shapes: every input row is normalised three times
+// (once in each row window that reads it), and the in-place pass adds a read
+// and a write of every staged byte to a shared memory whose bandwidth the
+// tensor core's operand reads and the weight loads already nearly fill.  The
+// separate GroupNorm pass plus the plain conv is faster there, so the block
+// step takes this kernel only when asked to (dp_block_desc_set_gn_fusion).
+//
+// Roles (576 threads): warp 0 B producer, warp 1 MMA issuer (leader CTA),
+// warps 2-9 epilogue (as in igemm_pair_kernel), warps 10-17 transform (warp
+// 10 lane 0 also issues the A row loads).
+template <int NJ>
+struct GnConvCfg {
+  static constexpr int NI = 160;
+  static constexpr int BN = NI * NJ;
+  static constexpr int ROW_PX = 130;                 // staged pixels per row
+  static constexpr int ROW_PITCH = 136 * 128;        // bytes between staged rows (1 KiB multiple)
+  static constexpr int A_BYTES = 3 * ROW_PITCH;      // one stage: rows r-1, r, r+1
+  static constexpr int A_TX = 3 * ROW_PX * 128;      // bytes the three row loads deliver
+  static constexpr int A_STAGES = 2;
+  static constexpr int XF_WARPS = 8;                 // staging / transform warps per CTA
+  static constexpr int BSUB_BYTES = (NI / 2) * 128;  // this CTA's half of one B slice
+  static constexpr int B_BYTES = NJ * BSUB_BYTES;
+  static constexpr int B_STAGES = NJ == 2 ? 4 : 6;
+  static constexpr int ACC = 2 * BN <= 512 ? 2 : 1;
+  static constexpr int TMEM_COLS = ACC * BN <= 256 ? 256 : 512;
+  static constexpr int EPI_BYTES = 8 * 2 * kEpiSlot;
+  static constexpr int BIAS_BYTES = 8 * BN * 4;
+  static constexpr int THREADS = 320 + 32 * XF_WARPS;
+  static constexpr int SMEM =
+      A_STAGES * A_BYTES + B_STAGES * B_BYTES + EPI_BYTES + BIAS_BYTES + 1024 + 512;
+  static_assert(SMEM <= 227 * 1024, "shared memory");
+  static_assert(ROW_PITCH % 1024 == 0 && A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "alignment");
+};
+
+// Where staged row kh (input row r - 1 + kh) of M tile mt comes from: 0 zero
+// fill, 1 the raw input (normalised with band *band), 2 the stale normalised
+// activations.  *rho is the input row.
+__device__ __forceinline__ int gn_row_source(const GemmParams& p, int mt, int kh, int* rho, int* band) {
+  if (mt >= p.m_tiles) return 0;
+  const int r = mt / p.tiles_w;
+  const int rr = r + kh - 1;
+  *rho = rr;
+  if (rr < 0 || rr >= p.H) return 0;
+  const int own = r / p.hb_in, other = rr / p.hb_in;
+  *band = other;
+  if (other == own || p.mode == DP_MODE_SYNC) return 1;
+  return p.mode == DP_MODE_DISPLACED ? 2 : 0;
+}
+
+// Scale and shift of the eight channels [c_base, c_base + 8) for band `band`
+// (gamma and beta read as 16-byte vectors; c_base is a multiple of 8).
+__device__ __forceinline__ void gn_chunk_scale_shift(const GemmParams& p, int band, int c_base,
+                                                     float (&sc)[8], float (&sh)[8]) {
+  const float4 g0 = __ldg(reinterpret_cast<const float4*>(p.gn_gamma + c_base));
+  const float4 g1 = __ldg(reinterpret_cast<const float4*>(p.gn_gamma + c_base) + 1);
+  const float4 b0 = __ldg(reinterpret_cast<const float4*>(p.gn_beta + c_base));
+  const float4 b1 = __ldg(reinterpret_cast<const float4*>(p.gn_beta + c_base) + 1);
+  const float gm[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+  const float bt[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+  const float* u = p.gn_used + 2 * band * (p.Cin / p.gn_cg);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const int g = (c_base + e) / p.gn_cg;
+    gn_scale_shift(__ldg(u + 2 * g), __ldg(u + 2 * g + 1), p.gn_eps, gm[e], bt[e], &sc[e], &sh[e]);
+  }
+}
+
+template <int NJ>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GnConvCfg<NJ>::THREADS, 1)
+    igemm_gn_pair_kernel(const __grid_constant__ GemmParams p) {
+  using C = GnConvCfg<NJ>;
+  constexpr int NI = C::NI;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + C::A_STAGES * C::A_BYTES;
+  uint8_t* sEpi = sB + C::B_STAGES * C::B_BYTES;
+  float* sBias = reinterpret_cast<float*>(sEpi + C::EPI_BYTES);
+  uint64_t* a_loaded = reinterpret_cast<uint64_t*>(sEpi + C::EPI_BYTES + C::BIAS_BYTES);  // [A_STAGES]
+  uint64_t* a_ready = a_loaded + C::A_STAGES;   // [A_STAGES], the leader's count both CTAs
+  uint64_t* a_empty = a_ready + C::A_STAGES;    // [A_STAGES]
+  uint64_t* b_full = a_empty + C::A_STAGES;     // [B_STAGES], the leader's count both CTAs
+  uint64_t* b_empty = b_full + C::B_STAGES;     // [B_STAGES]
+  uint64_t* acc_full = b_empty + C::B_STAGES;   // [2]
+  uint64_t* acc_empty = acc_full + 2;           // [2]
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = warp_id(), lane = lane_id();
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int num_items = ((p.m_tiles + 1) >> 1) * p.n_tiles;
+  const int kc = p.kc;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::A_STAGES; ++s) {
+      mbar_init(&a_loaded[s], 1);
+      mbar_init(&a_ready[s], 2 * C::XF_WARPS);   // the transform warps of both CTAs
+      mbar_init(&a_empty[s], 1);
+    }
+    for (int s = 0; s < C::B_STAGES; ++s) {
+      mbar_init(&b_full[s], 1);
+      mbar_init(&b_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 16);  // 8 epilogue warps in each CTA
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&p.tmA0);
+    prefetch_tmap(&p.tmA1);
+    prefetch_tmap(&p.tmB);
+    prefetch_tmap(&p.tmO[0]);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  griddep_wait();
+  griddep_trigger();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ B producer (both CTAs)
+      int stage = 0;
+      uint32_t phase = 0;
+      const uint32_t full0 = mapa_shared(smem_u32(b_full), 0);   // leader's b_full[0]
+      for (int item = pair; item < num_items && !*abort_flag; item += npairs) {
+        const int nt = item % p.n_tiles;
+        for (int cb = 0; cb < kc; ++cb) {
+          for (int tap = 0; tap < 9; ++tap) {
+            if (!mbar_wait(&b_empty[stage], phase ^ 1u, abort_flag, p.status)) goto b_done;
+            if (leader) mbar_arrive_expect_tx(&b_full[stage], 2 * C::B_BYTES);
+            const uint32_t fb = full0 + stage * 8;
+            uint8_t* b_dst = sB + stage * C::B_BYTES;
+#pragma unroll
+            for (int j = 0; j < NJ; ++j)
+              tma_load_2d_pair(b_dst + j * C::BSUB_BYTES, &p.tmB, fb, tap * p.Cin + cb * 64,
+                               nt * C::BN + j * NI + static_cast<int>(rank) * (NI / 2));
+            if (++stage == C::B_STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+      }
+    b_done:;
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ------------------------------------------------------------ MMA issuer (leader CTA)
+      constexpr uint32_t idesc = idesc_dense(256, NI, 1, 0, 0);
+      const uint64_t b_desc0 = sdesc_sw128(smem_u32(sB), 1024);
+      const uint32_t a_base = smem_u32(sA);
+      const uint32_t bempty_own = smem_u32(b_empty), bempty_peer = mapa_shared(smem_u32(b_empty), 1);
+      const uint32_t aempty_own = smem_u32(a_empty), aempty_peer = mapa_shared(smem_u32(a_empty), 1);
+      const uint32_t accf_own = smem_u32(acc_full), accf_peer = mapa_shared(smem_u32(acc_full), 1);
+      int bs = 0, as = 0;
+      uint32_t bph = 0, aph = 0;
+      int it = 0;
+      for (int item = pair; item < num_items; item += npairs, ++it) {
+        const int buf = C::ACC == 2 ? (it & 1) : 0;
+        const int use = C::ACC == 2 ? (it >> 1) : it;
+        if (!mbar_wait(&acc_empty[buf], (use & 1) ^ 1, abort_flag, p.status)) goto mma_done;
+        tc_fence_after();
+        const uint32_t dacc = tmem + buf * C::BN;
+        for (int cb = 0; cb < kc; ++cb) {
+          if (!mbar_wait(&a_ready[as], aph, abort_flag, p.status)) goto mma_done;
+          tc_fence_after();
+          const uint32_t a_stage = a_base + as * C::A_BYTES;
+          // taps in pairs (0,1) (2,3) (4,5) (6,7), then 8: one wait for two
+          // B stages keeps enough MMAs queued behind the wait
+          for (int tap = 0; tap < 9;) {
+            const int nb = tap < 8 ? 2 : 1;
+            int bs2 = bs + 1;
+            uint32_t bph2 = bph;
+            if (bs2 == C::B_STAGES) {
+              bs2 = 0;
+              bph2 ^= 1u;
+            }
+            if (!mbar_wait(&b_full[bs], bph, abort_flag, p.status) ||
+                (nb == 2 && !mbar_wait(&b_full[bs2], bph2, abort_flag, p.status)))
+              goto mma_done;
+            tc_fence_after();
+#pragma unroll 1
+            for (int t = 0; t < nb; ++t) {
+              const int tp = tap + t;
+              const int kh = tp / 3, kw = tp - 3 * (tp / 3);
+              const uint64_t ad = sdesc_sw128(a_stage + kh * C::ROW_PITCH + kw * 128, 1024);
+              const int sb = t == 0 ? bs : bs2;
+              const uint64_t bd = b_desc0 + static_cast<uint64_t>((sb * C::B_BYTES) >> 4);
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+#pragma unroll
+                for (int j = 0; j < NJ; ++j)
+                  umma_f16_ss_pair(dacc + j * NI, ad + 2 * k,
+                                   bd + static_cast<uint64_t>((j * C::BSUB_BYTES) >> 4) + 2 * k, idesc,
+                                   (cb != 0 || tp != 0 || k != 0));
+            }
+            umma_commit_pair(bempty_own + bs * 8);
+            umma_commit_pair(bempty_peer + bs * 8);
+            if (nb == 2) {
+              umma_commit_pair(bempty_own + bs2 * 8);
+              umma_commit_pair(bempty_peer + bs2 * 8);
+            }
+            tap += nb;
+            bs = nb == 2 ? bs2 : bs;
+            bph = nb == 2 ? bph2 : bph;
+            if (++bs == C::B_STAGES) {
+              bs = 0;
+              bph ^= 1u;
+            }
+          }
+          umma_commit_pair(aempty_own + as * 8);
+          umma_commit_pair(aempty_peer + as * 8);
+          if (++as == C::A_STAGES) {
+            as = 0;
+            aph ^= 1u;
+          }
+        }
+        umma_commit_pair(accf_own + buf * 8);
+        umma_commit_pair(accf_peer + buf * 8);
+      }
+    mma_done:
+      if (*abort_flag) {
+        umma_commit_pair(smem_u32(drain));
+        mbar_wait_teardown(drain, 0);
+      }
+    }
+  } else if (warp < 10) {
+    // -------------------------------------------------------------- epilogue (both CTAs)
+    const int q = warp & 3;
+    const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
+    const int ew = warp - 2, half = ew >> 2;
+    PairEpi e;
+    e.out = sEpi + ew * 2 * kEpiSlot;
+    e.bias = sBias + ew * C::BN;
+    e.oi = 0;
+    int it = 0;
+    for (int item = pair; item < num_items; item += npairs, ++it) {
+      const int buf = C::ACC == 2 ? (it & 1) : 0;
+      const int use = C::ACC == 2 ? (it >> 1) : it;
+      if (!pair_epilogue_tile<C::BN>(p, tmem + buf * C::BN, q, half, lane, rank, item,
+                                     static_cast<uint32_t>(use & 1), &acc_full[buf],
+                                     acc_empty_leader + buf * 8, abort_flag, e))
+        break;
+    }
+    if (lane == 0) bulk_wait_all();
+  } else {
+    // -------------------------------------------------------------- A staging + transform (both CTAs)
+    const int t = threadIdx.x - 320;             // 0 .. 32 * XF_WARPS - 1
+    constexpr int PXL = 4 * C::XF_WARPS;         // pixel lanes: 8 chunk lanes x PXL = the threads
+    const int j = t & 7, pl = t >> 3;            // 16-byte channel chunk, pixel lane
+    const uint32_t ready_leader = mapa_shared(smem_u32(a_ready), 0);
+    constexpr int NPX = (C::ROW_PX + PXL - 1) / PXL;   // chunks of one staged row per thread
+    // the three row loads of step (item, cb) into stage s (warp 10, lane 0)
+    auto issue = [&](int item, int cb, int st) {
+      const int mt = 2 * (item / p.n_tiles) + static_cast<int>(rank);
+      const int c0 = (mt % p.tiles_w) * 128;
+      uint8_t* dst = sA + st * C::A_BYTES;
+      mbar_arrive_expect_tx(&a_loaded[st], C::A_TX);
+      for (int kh = 0; kh < 3; ++kh) {
+        int rho = -1, band = 0;
+        const int src = gn_row_source(p, mt, kh, &rho, &band);
+        tma_load_3d(dst + kh * C::ROW_PITCH, src == 2 ? &p.tmA1 : &p.tmA0, &a_loaded[st], cb * 64,
+                    c0 - 1, src == 0 ? -1 : rho);
+      }
+    };
+    // the first A_STAGES steps go out at once; later ones when the MMA frees
+    // the stage of the step before the one being transformed
+    int pre_item = pair, pre_cb = 0;
+    auto advance = [&]() {
+      if (++pre_cb == kc) {
+        pre_cb = 0;
+        pre_item += npairs;
+      }
+    };
+    if (warp == 10 && lane == 0) {
+      for (int k = 0; k < C::A_STAGES && pre_item < num_items; ++k) {
+        issue(pre_item, pre_cb, k);
+        advance();
+      }
+    }
+    int s = 0;
+    uint32_t ph = 0;
+    int seq = 0;   // (item, cb) steps transformed so far
+    for (int item = pair; item < num_items && !*abort_flag; item += npairs) {
+      const int mt = 2 * (item / p.n_tiles) + static_cast<int>(rank);
+      const int nt = item % p.n_tiles;
+      const int r = mt / p.tiles_w, c0 = (mt % p.tiles_w) * 128;
+      const bool edge = p.a_next && nt == 0 && mt < p.m_tiles &&
+                        (r % p.hb_in == 0 || r % p.hb_in == p.hb_in - 1);
+      const int own_band = r / p.hb_in;
+      for (int cb = 0; cb < kc; ++cb) {
+        const int c_base = cb * 64 + j * 8;      // first channel of this thread's chunk
+        // the own band's scale and shift, fetched while the rows arrive
+        VecApply<__nv_bfloat16> ap_own;
+        {
+          float sc[8], sh[8];
+          gn_chunk_scale_shift(p, own_band, c_base, sc, sh);
+          ap_own = VecApply<__nv_bfloat16>(sc, sh);
+        }
+        if (!mbar_wait(&a_loaded[s], ph, abort_flag, p.status)) goto xf_done;
+        uint8_t* stage = sA + s * C::A_BYTES;
+#pragma unroll 1
+        for (int kh = 0; kh < 3; ++kh) {
+          int rho = -1, band = 0;
+          if (gn_row_source(p, mt, kh, &rho, &band) != 1) continue;   // stale or zero: as loaded
+          VecApply<__nv_bfloat16> ap = ap_own;
+          if (band != own_band) {                           // a sync step's halo row
+            float osc[8], osh[8];
+            gn_chunk_scale_shift(p, band, c_base, osc, osh);
+            ap = VecApply<__nv_bfloat16>(osc, osh);
+          }
+          uint8_t* row = stage + kh * C::ROW_PITCH;
+          const bool write_edge = edge && kh == 1;
+          __nv_bfloat16* nrow = write_edge ? static_cast<__nv_bfloat16*>(p.a_next) +
+                                                 static_cast<size_t>(r) * p.W * p.Cin + c_base
+                                           : nullptr;
+          // this thread's chunks of the row: all loads first, then normalise
+          // in place (zero-filled padding columns stay zero)
+          uint4 v[NPX];
+#pragma unroll
+          for (int i = 0; i < NPX; ++i) {
+            const int px = pl + PXL * i;
+            if (px < C::ROW_PX) v[i] = *reinterpret_cast<const uint4*>(row + px * 128 + ((j ^ (px & 7)) << 4));
+          }
+#pragma unroll
+          for (int i = 0; i < NPX; ++i) {
+            const int px = pl + PXL * i, c = c0 - 1 + px;
+            if (px >= C::ROW_PX || c < 0 || c >= p.W) continue;
+            const uint4 y = ap.apply(v[i], p.gn_silu);
+            *reinterpret_cast<uint4*>(row + px * 128 + ((j ^ (px & 7)) << 4)) = y;
+            if (write_edge && px >= 1 && px <= 128)
+              *reinterpret_cast<uint4*>(nrow + static_cast<size_t>(c) * p.Cin) = y;
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(ready_leader + s * 8);
+        // the next load goes into the stage of the step before this one, once
+        // the MMA (running while this step was transformed) is done with it;
+        // warp 10 leaves together if that wait gives up
+        if (warp == 10 && seq >= 1) {
+          int ok = 1;
+          if (lane == 0 && pre_item < num_items) {
+            const int st = (seq + 1) % C::A_STAGES;
+            ok = mbar_wait(&a_empty[st], static_cast<uint32_t>(((seq + 1) / C::A_STAGES - 1) & 1),
+                           abort_flag, p.status);
+            if (ok) {
+              issue(pre_item, pre_cb, st);
+              advance();
+            }
+          }
+          if (!__shfl_sync(0xffffffffu, ok, 0)) goto xf_done;
+        }
+        ++seq;
+        if (++s == C::A_STAGES) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+    }
+  xf_done:
+    if (*abort_flag && warp == 10 && lane == 0) {
+      // row loads in flight land in this CTA's stages: give them time
+      const unsigned long long t0 = globaltimer_ns();
+      while (globaltimer_ns() - t0 < 2000000ull) {
+      }
+    }
   }
 
   tc_fence_before();
@@ -1239,6 +1666,111 @@ int conv3x3_launch(const void* a_fresh, const void* a_stale, const void* weight,
   return launch_gemm(p, BN, tf32, stream);
 }
 
+bool conv3x3_gn_eligible(int H, int W, int Cin, int Cout, int G, int dtype) {
+  return dtype == DP_BF16 && W >= 128 && Cin % 64 == 0 && G > 0 && Cin % G == 0 && Cout % 160 == 0 &&
+         H >= 1;
+}
+
+template <int NJ>
+static int launch_gn_pair(const GemmParams& p, cudaStream_t s) {
+  using C = GnConvCfg<NJ>;
+  static int grid_cache[32] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int& maxg = grid_cache[dev & 31];
+  if (!maxg) {
+    int rc = cuda_check(cudaFuncSetAttribute(igemm_gn_pair_kernel<NJ>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM),
+                        "groupnorm conv smem attribute");
+    if (rc) return rc;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * num_sms());
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, igemm_gn_pair_kernel<NJ>, &cfg) != cudaSuccess ||
+        clusters <= 0) {
+      cudaGetLastError();
+      clusters = num_sms() / 2;
+    }
+    maxg = 2 * clusters;
+  }
+  const int pair_tiles = ((p.m_tiles + 1) / 2) * p.n_tiles;
+  const int grid = std::min(2 * pair_tiles, maxg);
+  mark_launch(s);
+  return launch_kernel(igemm_gn_pair_kernel<NJ>, dim3(grid), dim3(C::THREADS), C::SMEM, s, false,
+                       "groupnorm conv launch", p);
+}
+
+int conv3x3_gn_launch(const void* x, const void* a_stale, void* a_next, const float* used,
+                      const float* gamma, const float* beta, int G, float eps, int silu,
+                      const void* weight, const float* bias, const void* residual, void* out, int H,
+                      int W, int Cin, int Cout, int P, int mode, cudaStream_t stream) {
+  if (!conv3x3_gn_eligible(H, W, Cin, Cout, G, DP_BF16))
+    return set_error(DP_ERR_UNSUPPORTED, "groupnorm conv: needs bf16, W >= 128, Cin %% 64 == 0, "
+                                         "Cout %% 160 == 0 (H=%d W=%d Cin=%d Cout=%d)", H, W, Cin, Cout);
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  p.splits = 1;
+  p.a_mode = 1;
+  p.H = H;
+  p.W = W;
+  p.Ho = H;
+  p.Wo = W;
+  p.Cin = Cin;
+  p.stride = 1;
+  p.hb_in = H / P;
+  p.hb_out = H / P;
+  p.mode = mode;
+  p.Wt = 128;
+  p.R = 1;
+  p.tiles_w = (W + 127) / 128;
+  p.m_tiles = p.tiles_w * H;
+  p.kc = Cin / 64;
+  p.k_blocks = 9 * p.kc;
+  p.N = Cout;
+  p.split = Cout;
+  p.ld_out = Cout;
+  p.bias = bias;
+  p.residual = residual;
+  p.out0 = out;
+  p.status = device_status_ptr();
+  p.gn_used = used;
+  p.gn_gamma = gamma;
+  p.gn_beta = beta;
+  p.gn_eps = eps;
+  p.gn_cg = Cin / G;
+  p.gn_silu = silu;
+  p.a_next = a_next;
+  const int NJ = Cout % 320 == 0 ? 2 : 1;
+  p.n_tiles = Cout / (160 * NJ);
+  uint64_t dims[3] = {static_cast<uint64_t>(Cin), static_cast<uint64_t>(W), static_cast<uint64_t>(H)};
+  uint64_t str[2] = {static_cast<uint64_t>(Cin) * 2, static_cast<uint64_t>(W) * Cin * 2};
+  uint32_t box[3] = {64, static_cast<uint32_t>(GnConvCfg<1>::ROW_PX), 1};
+  int rc = encode_tmap(&p.tmA0, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), dims, str, box,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc) return rc;
+  rc = encode_tmap(&p.tmA1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(a_stale ? a_stale : x),
+                   dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc) return rc;
+  uint64_t bdims[2] = {9 * static_cast<uint64_t>(Cin), static_cast<uint64_t>(Cout)};
+  uint64_t bstr[1] = {9 * static_cast<uint64_t>(Cin) * 2};
+  uint32_t bbox[2] = {64, 80};
+  rc = encode_tmap(&p.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(weight), bdims, bstr,
+                   bbox, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc) return rc;
+  rc = encode_conv_epilogue(p, out, Cout);
+  if (rc) return rc;
+  return NJ == 2 ? launch_gn_pair<2>(p, stream) : launch_gn_pair<1>(p, stream);
+}
+
 int linear_launch(const void* x, const void* weight, const float* bias, const void* residual,
                   void* out0, void* out1, void* out2, int M, int N, int K, int split,
                   void* workspace, size_t workspace_bytes, cudaStream_t stream) {
@@ -1327,6 +1859,37 @@ int conv3x3_validate(const void* a_fresh, const void* a_stale, const void* weigh
 extern "C" {
 
 size_t dp_gemm_workspace_size(void) { return dp::gemm_workspace_bytes(); }
+
+int dp_conv3x3_halo_gn(const void* x, const void* a_stale, void* a_next, const float* used_stats,
+                       const float* gamma, const float* beta, int G, float eps, int silu,
+                       const void* weight, const float* bias, const void* residual, void* out, int H,
+                       int W, int Cin, int Cout, int P, int mode, void* stream) {
+  int rc = dp::conv3x3_validate(x, a_stale, weight, residual, out, H, W, Cin, Cout, 1, P, mode, DP_BF16);
+  if (rc) return rc;
+  if (!used_stats || !gamma || !beta)
+    return dp::set_error(DP_ERR_INVALID_ARG, "groupnorm conv: null used_stats/gamma/beta");
+  if (!dp::aligned16(gamma) || !dp::aligned16(beta))
+    return dp::set_error(DP_ERR_UNSUPPORTED, "groupnorm conv: gamma/beta not 16-byte aligned");
+  if (G <= 0 || Cin % G) return dp::set_error(DP_ERR_UNSUPPORTED, "groupnorm conv: Cin %% G != 0");
+  if (!(eps > 0.f)) return dp::set_error(DP_ERR_INVALID_ARG, "groupnorm conv: eps must be > 0");
+  if (!dp::conv3x3_gn_eligible(H, W, Cin, Cout, G, DP_BF16))
+    return dp::set_error(DP_ERR_UNSUPPORTED, "groupnorm conv: needs W >= 128, Cin %% 64 == 0 and "
+                                             "Cout %% 160 == 0");
+  if (a_next) {
+    if (!dp::aligned16(a_next)) return dp::set_error(DP_ERR_UNSUPPORTED, "groupnorm conv: a_next not aligned");
+    const size_t bytes = static_cast<size_t>(H) * W * Cin * 2;
+    const char* n = static_cast<const char*>(a_next);
+    auto hit = [&](const void* q, size_t qb) {
+      const char* c = static_cast<const char*>(q);
+      return q && n < c + qb && c < n + bytes;
+    };
+    const size_t ob = static_cast<size_t>(H) * W * Cout * 2;
+    if (hit(x, bytes) || hit(a_stale, bytes) || hit(out, ob) || hit(residual, ob))
+      return dp::set_error(DP_ERR_INVALID_ARG, "groupnorm conv: a_next overlaps an input or the output");
+  }
+  return dp::conv3x3_gn_launch(x, a_stale, a_next, used_stats, gamma, beta, G, eps, silu, weight, bias,
+                               residual, out, H, W, Cin, Cout, P, mode, static_cast<cudaStream_t>(stream));
+}
 
 int dp_conv3x3_halo(const void* a_fresh, const void* a_stale, const void* weight,
                     const float* bias, const void* residual, void* out, int H, int W, int Cin,

@@ -1073,6 +1073,75 @@ static bool gn_fused_launch(const void* x, void* y, const float* gamma, const fl
   return true;
 }
 
+// Shared memory of the two-kernel path's kernels, with the opt-in above
+// 48 KiB set (kept per dtype and device at the largest size so far).
+static int gn_two_pass_setup(const GnArgs& a, int C, int G, int P, int dtype, size_t* smem_stats,
+                             size_t* smem_apply) {
+  const size_t ring = static_cast<size_t>(kGnStages) * a.piece * C * (dtype == DP_BF16 ? 2 : 4);
+  size_t red = static_cast<size_t>(a.lanes) * C * 2 * sizeof(float);
+  const size_t fin = static_cast<size_t>(P) * G * 2 * sizeof(double);
+  if (fin > ring + red) red = fin - ring;
+  *smem_stats = ring + red;
+  *smem_apply = ring + static_cast<size_t>(C) * 2 * sizeof(float);
+  if (*smem_stats > 220 * 1024 || *smem_apply > 220 * 1024)
+    return set_error(DP_ERR_UNSUPPORTED, "groupnorm: C = %d needs too much shared memory", C);
+  static size_t attr_set[2][32] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  size_t& done = attr_set[dtype][dev & 31];
+  const size_t need = *smem_stats > *smem_apply ? *smem_stats : *smem_apply;
+  if (need > done) {
+    const int lim = static_cast<int>(need);
+    int rc = 0;
+    if (dtype == DP_BF16) {
+      rc = cuda_check(cudaFuncSetAttribute(gn_stats_kernel<__nv_bfloat16>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, lim),
+                      "groupnorm stats smem attribute");
+      if (!rc)
+        rc = cuda_check(cudaFuncSetAttribute(gn_apply_kernel<__nv_bfloat16>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, lim),
+                        "groupnorm apply smem attribute");
+    } else {
+      rc = cuda_check(cudaFuncSetAttribute(gn_stats_kernel<float>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, lim),
+                      "groupnorm stats smem attribute");
+      if (!rc)
+        rc = cuda_check(cudaFuncSetAttribute(gn_apply_kernel<float>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, lim),
+                        "groupnorm apply smem attribute");
+    }
+    if (rc) return rc;
+    done = need;
+  }
+  return DP_OK;
+}
+
+int gn_stats_launch(const void* x, int H, int W, int C, int G, int P, float w, int mode, int dtype,
+                    const float* stale_global, const float* stale_local, float* fresh_local,
+                    float* fresh_global, float* used, void* workspace, cudaStream_t stream) {
+  GnArgs a;
+  gn_plan(H, W, C, G, P, dtype, &a);
+  a.eps = 1.0f;   // unused by the statistics pass
+  a.w = w;
+  a.silu = 0;
+  a.mode = mode;
+  size_t smem_stats = 0, smem_apply = 0;
+  int rc = gn_two_pass_setup(a, C, G, P, dtype, &smem_stats, &smem_apply);
+  if (rc) return rc;
+  unsigned* counter = static_cast<unsigned*>(workspace);
+  double* acc = reinterpret_cast<double*>(static_cast<char*>(workspace) + 256);
+  int* status = device_status_ptr();
+  mark_launch(stream);
+  if (dtype == DP_BF16)
+    return launch_kernel(gn_stats_kernel<__nv_bfloat16>, dim3(a.P * a.S), dim3(a.vpp * a.lanes),
+                         smem_stats, stream, false, "groupnorm stats launch",
+                         static_cast<const __nv_bfloat16*>(x), a, acc, counter, stale_global, stale_local,
+                         fresh_local, fresh_global, used, status);
+  return launch_kernel(gn_stats_kernel<float>, dim3(a.P * a.S), dim3(a.vpp * a.lanes), smem_stats, stream,
+                       false, "groupnorm stats launch", static_cast<const float*>(x), a, acc, counter,
+                       stale_global, stale_local, fresh_local, fresh_global, used, status);
+}
+
 // Internal entry shared by the ABI call and the block step.
 int gn_launch(const void* x, void* y, const float* gamma, const float* beta, int H, int W, int C,
               int G, int P, float eps, float w, int silu, int mode, int dtype,
@@ -1099,46 +1168,11 @@ int gn_launch(const void* x, void* y, const float* gamma, const float* beta, int
                         &rc))
       return rc;
   }
+  size_t smem_stats = 0, smem_apply = 0;
+  int rc0 = gn_two_pass_setup(a, C, G, P, dtype, &smem_stats, &smem_apply);
+  if (rc0) return rc0;
   const int threads = a.vpp * a.lanes;
   const int blocks = a.P * a.S;
-  const size_t ring = static_cast<size_t>(kGnStages) * a.piece * C * (dtype == DP_BF16 ? 2 : 4);
-  size_t red = static_cast<size_t>(a.lanes) * C * 2 * sizeof(float);
-  const size_t fin = static_cast<size_t>(P) * G * 2 * sizeof(double);
-  if (fin > ring + red) red = fin - ring;
-  const size_t smem_stats = ring + red;
-  const size_t smem_apply = ring + static_cast<size_t>(C) * 2 * sizeof(float);
-  if (smem_stats > 220 * 1024 || smem_apply > 220 * 1024)
-    return set_error(DP_ERR_UNSUPPORTED, "groupnorm: C = %d needs too much shared memory", C);
-  // dynamic shared memory above 48 KiB must be opted into; keep the largest
-  // size set so far per (dtype, device)
-  static size_t attr_set[2][32] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  size_t& done = attr_set[dtype][dev & 31];
-  const size_t need = smem_stats > smem_apply ? smem_stats : smem_apply;
-  if (need > done) {
-    const int lim = static_cast<int>(need);
-    int rc = 0;
-    if (dtype == DP_BF16) {
-      rc = cuda_check(cudaFuncSetAttribute(gn_stats_kernel<__nv_bfloat16>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, lim),
-                      "groupnorm stats smem attribute");
-      if (!rc)
-        rc = cuda_check(cudaFuncSetAttribute(gn_apply_kernel<__nv_bfloat16>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, lim),
-                        "groupnorm apply smem attribute");
-    } else {
-      rc = cuda_check(cudaFuncSetAttribute(gn_stats_kernel<float>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, lim),
-                      "groupnorm stats smem attribute");
-      if (!rc)
-        rc = cuda_check(cudaFuncSetAttribute(gn_apply_kernel<float>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, lim),
-                        "groupnorm apply smem attribute");
-    }
-    if (rc) return rc;
-    done = need;
-  }
   int* status = device_status_ptr();
   const float* cgl = stale_global;
   const float* cll = stale_local;
@@ -1205,6 +1239,22 @@ size_t dp_groupnorm_workspace_size(int H, int W, int C, int G, int P) {
   (void)C;
   if (P <= 0 || G <= 0) return 0;
   return dp::gn_workspace_bytes(P, G);
+}
+
+int dp_groupnorm_stats(const void* x, int H, int W, int C, int G, int P, float w, int mode, int dtype,
+                       const float* stale_global, const float* stale_local, float* fresh_local,
+                       float* used_stats, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = dp::gn_validate(x, x, H, W, C, G, P, dtype, mode);   // no output tensor: x stands in
+  if (rc) return rc;
+  if (!fresh_local || !used_stats || !workspace)
+    return dp::set_error(DP_ERR_INVALID_ARG, "groupnorm stats: null fresh_local/used/workspace");
+  if (mode == DP_MODE_DISPLACED && (!stale_global || !stale_local))
+    return dp::set_error(DP_ERR_INVALID_ARG, "groupnorm stats: displaced mode needs stale statistics");
+  if (workspace_bytes < dp::gn_acc_bytes(P, G))
+    return dp::set_error(DP_ERR_INVALID_ARG, "groupnorm stats: workspace too small (%zu < %zu)",
+                         workspace_bytes, dp::gn_acc_bytes(P, G));
+  return dp::gn_stats_launch(x, H, W, C, G, P, w, mode, dtype, stale_global, stale_local, fresh_local,
+                             nullptr, used_stats, workspace, static_cast<cudaStream_t>(stream));
 }
 
 int dp_groupnorm_async(const void* x, void* y, const float* gamma, const float* beta, int H,

@@ -42,6 +42,7 @@ struct VecApply;
 template <>
 struct VecApply<__nv_bfloat16> {
   uint64_t sc[4], sh[4];
+  VecApply() = default;
   __device__ __forceinline__ VecApply(const float* scale, const float* shift) {
 #pragma unroll
     for (int k = 0; k < 4; ++k) {

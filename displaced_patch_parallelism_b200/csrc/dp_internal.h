@@ -25,6 +25,19 @@ int conv3x3_validate(const void* a_fresh, const void* a_stale, const void* weigh
                      const void* residual, const void* out, int H, int W, int Cin, int Cout,
                      int stride, int P, int mode, int dtype);
 size_t gemm_workspace_bytes();
+// GroupNorm statistics alone (the first kernel of the two-kernel path): fresh
+// moments, used moments and (if given) the whole-image moments; no apply.
+int gn_stats_launch(const void* x, int H, int W, int C, int G, int P, float w, int mode, int dtype,
+                    const float* stale_global, const float* stale_local, float* fresh_local,
+                    float* fresh_global, float* used, void* workspace, cudaStream_t stream);
+// 3x3 conv (stride 1) of GroupNorm(x) (+SiLU), normalised in the conv's
+// operand path from the used moments; the band-edge rows of the normalised
+// input go to a_next (if not null).  Eligible shapes: conv3x3_gn_eligible.
+bool conv3x3_gn_eligible(int H, int W, int Cin, int Cout, int G, int dtype);
+int conv3x3_gn_launch(const void* x, const void* a_stale, void* a_next, const float* used,
+                      const float* gamma, const float* beta, int G, float eps, int silu,
+                      const void* weight, const float* bias, const void* residual, void* out, int H,
+                      int W, int Cin, int Cout, int P, int mode, cudaStream_t stream);
 // K runs of a conv / projection (1: no split; more: the GEMM is followed by
 // the split-K finish kernel).
 int conv3x3_splits(int H, int W, int Cin, int Cout, int stride, int dtype, bool can_split);

@@ -236,6 +236,54 @@ DP_API int dp_conv3x3_halo(const void* a_fresh, const void* a_stale, const void*
                     void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * The GroupNorm -> 3x3 conv pair of a block as two calls that never store the
+ * normalised activations whole: dp_groupnorm_stats computes the moments each
+ * band normalises with (the statistics half of dp_groupnorm_async), and
+ * dp_conv3x3_halo_gn convolves GroupNorm(x) (+SiLU), normalising each input
+ * tile in shared memory on its way to the tensor cores ("DistriFusion",
+ * atlas.scime.ai summary, Approach: the corrected GroupNorm feeds the conv;
+ * study.space summary, Method: other bands' rows are the previous step's
+ * activations).
+ *
+ * dp_groupnorm_stats: arguments, statistics, workspace rules and errors as
+ *   dp_groupnorm_async, without y, gamma, beta, eps and silu; writes
+ *   fresh_local and used_stats only.
+ *
+ * dp_conv3x3_halo_gn: out = conv3x3(a) + bias (+ residual), stride 1, where a
+ *   is x normalised per band with used_stats (scale = rsqrt(var + eps) *
+ *   gamma_c, shift = beta_c - mean * scale, then SiLU if silu != 0, then the
+ *   bf16 cast -- the same arithmetic as dp_groupnorm_async's output), and the
+ *   halo rule of dp_conv3x3_halo: an input row of another band is a row of x
+ *   normalised with that band's moments (SYNC), the row of a_stale
+ *   (DISPLACED; a_stale holds normalised activations) or zero (NAIVE).
+ *    x         [H][W][Cin] bf16, device: the GroupNorm's input
+ *    a_stale   [H][W][Cin] bf16, device: the previous step's normalised
+ *              activations; read in DISPLACED mode only, and only rows just
+ *              outside a band (the first and last row of every band)
+ *    a_next    [H][W][Cin] bf16, device, or NULL: receives the normalised
+ *              first and last row of every band (the rows the next step's
+ *              displaced call reads as its a_stale); other rows untouched.
+ *              May not overlap x, a_stale, residual or out.
+ *    used_stats [P][G][2] fp32 (mean, var), device (dp_groupnorm_stats)
+ *    gamma, beta [Cin] fp32, device, 16-byte aligned;  weight, bias, residual, out as
+ *              dp_conv3x3_halo (Ho = H, Wo = W).
+ *   Needs bf16, W >= 128, Cin % 64 == 0, Cin % G == 0, Cout % 160 == 0,
+ *   H % P == 0.  Tiles are one output row x 128 columns; the three input rows
+ *   a tile reads are staged once per 64 input channels and the nine taps read
+ *   shifted views of them.  Errors as dp_conv3x3_halo, plus DP_ERR_INVALID_ARG
+ *   for null used_stats/gamma/beta, eps <= 0 or an overlapping a_next.
+ * ---------------------------------------------------------------------- */
+DP_API int dp_groupnorm_stats(const void* x, int H, int W, int C, int G, int P, float w, int mode,
+                              int dtype, const float* stale_global, const float* stale_local,
+                              float* fresh_local, float* used_stats, void* workspace,
+                              size_t workspace_bytes, void* stream);
+DP_API int dp_conv3x3_halo_gn(const void* x, const void* a_stale, void* a_next,
+                              const float* used_stats, const float* gamma, const float* beta, int G,
+                              float eps, int silu, const void* weight, const float* bias,
+                              const void* residual, void* out, int H, int W, int Cin, int Cout,
+                              int P, int mode, void* stream);
+
+/* ------------------------------------------------------------------------
  * Direct 3x3 conv for few input channels (the latent input conv), same
  * halo rule and layouts as dp_conv3x3_halo, stride 1, bf16 only.
  * Needs Cin <= 16, Cout % 32 == 0.  Runs on the CUDA cores.
@@ -420,6 +468,7 @@ typedef struct dp_block_desc {
   int ctx_dim;    /* TRANSFORMER: text context width (Cctx)       */
   int ff_inner;   /* TRANSFORMER: feed-forward inner width (F)    */
   int temb_dim;   /* RESBLOCK: time-embedding width (0: none)     */
+  int gn_fuse;    /* 1: GroupNorm -> conv through dp_conv3x3_halo_gn */
 } dp_block_desc;
 
 /*
@@ -472,6 +521,19 @@ DP_API int dp_block_desc_init(dp_block_desc* d, int kind, int H, int W, int C, i
 #define DP_GN_STATS_STALE 2
 #define DP_GN_STATS_SYNC 3
 DP_API int dp_block_desc_set_gn_stats(dp_block_desc* d, int variant);
+
+/*
+ * GN_CONV and RESBLOCK blocks (and the mini U-Net's ResBlocks): with on = 1,
+ * every GroupNorm -> 3x3 conv pair whose shapes dp_conv3x3_halo_gn takes runs
+ * as dp_groupnorm_stats + dp_conv3x3_halo_gn, so the normalised activations
+ * are never stored whole and the state keeps only their band-edge rows.  Off
+ * (0) by default: on B200 the separate GroupNorm pass plus the plain conv is
+ * the faster pair at the SDXL shapes (the fused conv redoes the normalisation
+ * for each of the three row windows that read an input row, and its
+ * shared-memory traffic slows the tensor core's operand reads).
+ * DP_ERR_INVALID_ARG for a null descriptor or on not 0/1.
+ */
+DP_API int dp_block_desc_set_gn_fusion(dp_block_desc* d, int on);
 DP_API size_t dp_block_workspace_size(const dp_block_desc* d);
 DP_API int dp_block_state_init(const dp_block_desc* d, dp_block_state* s, void* workspace,
                         size_t workspace_bytes, void* stream);
@@ -538,13 +600,18 @@ DP_API int dp_block_status(const dp_block_desc* d, const dp_block_state* s, void
 #define DP_KERNEL_LAYERNORM 10  /* per-token LayerNorm                          */
 #define DP_KERNEL_GEGLU 11      /* gated GELU unit of the feed-forward          */
 #define DP_KERNEL_TEMB 12       /* time-embedding bias of a ResBlock's conv1     */
+#define DP_KERNEL_CONV_GN 13    /* 3x3 conv of GroupNorm(x), normalised in-kernel */
 
 /*
  * Number of kernel launches one displaced dp_block_step makes for this
  * descriptor.  A GroupNorm is one launch when its tensor fits in the GPU's
- * shared memory and two (statistics, apply) otherwise.  Launch order --
+ * shared memory and two (statistics, apply) otherwise; a GroupNorm that feeds
+ * a 3x3 conv dp_conv3x3_halo_gn can take (bf16, W >= 128, Cin % 64 == 0,
+ * Cout % 160 == 0) is its statistics pass alone, and the conv that follows
+ * normalises its own input (DP_KERNEL_CONV_GN).  Launch order --
  *   GN_CONV:  GN, conv
  *   RESBLOCK: GN1, conv1, GN2, [1x1 shortcut if C != Cout], conv2
+ *             (each GN and conv a statistics pass and a CONV_GN when fused)
  *   ATTN:     GN, q/k/v projection, attention, out projection
  *   UNET_MINI: input copy, conv_in, then its blocks and downsamplers in order
  *   TRANSFORMER: GN, proj_in, LN, q/k/v projection, attention, out projection,

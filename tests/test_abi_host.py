@@ -173,6 +173,12 @@ def test_gn_stats_variants_on_the_host(B):
     for v in (B.GN_STATS_LOCAL, B.GN_STATS_STALE, B.GN_STATS_CORRECTED):
         B.dp_block_desc_set_gn_stats(d, v)
         assert kinds(d, B.DISPLACED) == ["gn_cluster", "conv", "gn_cluster", "conv"]
+    # with fusion on, the conv normalises its own input under every variant
+    d1 = B.dp_block_desc_init(B.RESBLOCK, 128, 128, 320, 320, 32, 4, 0, B.BF16, 1, 1e-5, 1.0)
+    B.dp_block_desc_set_gn_fusion(d1, 1)
+    for v in (B.GN_STATS_SYNC, B.GN_STATS_LOCAL, B.GN_STATS_STALE, B.GN_STATS_CORRECTED):
+        B.dp_block_desc_set_gn_stats(d1, v)
+        assert kinds(d1, B.DISPLACED) == ["gn_stats", "conv_gn", "gn_stats", "conv_gn"]
     with pytest.raises(B.DPError):
         B.dp_block_desc_set_gn_stats(d, 4)
     with pytest.raises(B.DPError):
@@ -417,4 +423,59 @@ def test_selftest_and_block_status_reject_bad_arguments_on_the_host(B):
     d = B.dp_block_desc_init(B.GN_CONV, 16, 16, 64, 64, 32, 2, 0, B.BF16, 1, 1e-5, 1.0)
     with pytest.raises(B.DPError) as e:   # a state never initialised has no workspace
         B.dp_block_status(d, B.BlockState(), stream=0)
+    assert e.value.code == B.DP_ERR_INVALID_ARG
+
+
+def test_groupnorm_fusion_plan(B):
+    """dp_block_desc_set_gn_fusion(d, 1): every GroupNorm -> conv pair the fused conv takes is a
+    statistics pass plus a conv that normalises its own input; others stay as they are; the
+    flag reaches the mini U-Net's ResBlocks; it is checked."""
+    kinds = lambda d, m: [B.dp_block_launch_info(d, m, i)[0] for i in range(B.dp_block_launch_count(d))]
+    d = B.dp_block_desc_init(B.RESBLOCK, 128, 128, 320, 320, 32, 4, 0, B.BF16, 1, 1e-5, 1.0)
+    B.dp_block_desc_set_gn_fusion(d, 1)
+    assert kinds(d, B.DISPLACED) == ["gn_stats", "conv_gn", "gn_stats", "conv_gn"]
+    assert kinds(d, B.SYNC) == ["gn_stats", "conv_gn", "gn_stats", "conv_gn"]
+    fl = sum(B.dp_block_launch_info(d, B.DISPLACED, i)[1] for i in range(4))
+    assert abs(fl - B.dp_block_flops(d)) < 1
+    d4 = B.dp_block_desc_init(B.GN_CONV, 480, 480, 320, 320, 32, 8, 0, B.BF16, 1, 1e-5, 1.0)
+    B.dp_block_desc_set_gn_fusion(d4, 1)
+    assert kinds(d4, B.DISPLACED) == ["gn_stats", "conv_gn"]
+    d2 = B.dp_block_desc_init(B.RESBLOCK, 64, 64, 320, 640, 32, 4, 0, B.BF16, 1, 1e-5, 1.0)
+    B.dp_block_desc_set_gn_fusion(d2, 1)                  # 64 columns: not eligible
+    assert kinds(d2, B.DISPLACED) == ["gn_cluster", "conv", "gn_cluster", "linear", "conv"]
+    du = B.dp_block_desc_init(B.UNET_MINI, 128, 128, 4, 0, 32, 4, 0, B.BF16, 1, 1e-5, 1.0)
+    B.dp_block_desc_set_gn_fusion(du, 1)
+    assert kinds(du, B.DISPLACED).count("conv_gn") == 2   # the 128x128 ResBlock's two convs
+    with pytest.raises(B.DPError):
+        B.dp_block_desc_set_gn_fusion(d, 2)
+    d.gn_fuse = 5                                         # edited by hand: checked too
+    with pytest.raises(B.DPError, match="fusion"):
+        B.dp_block_workspace_size(d)
+
+
+def test_groupnorm_conv_rejects_bad_arguments_on_the_host(B):
+    A = 1 << 20                                   # fake, never dereferenced: checks run first
+    base = dict(x=A, a_stale=2 * A, a_next=0, used=3 * A, gamma=4 * A, beta=5 * A, G=32, eps=1e-5,
+                silu=1, weight=6 * A, bias=0, residual=0, out=7 * A, H=16, W=128, Cin=64, Cout=160,
+                P=2, mode=B.DISPLACED)
+
+    def call(**kw):
+        a = dict(base, **kw)
+        B.dp_conv3x3_halo_gn(a["x"], a["a_stale"], a["a_next"], a["used"], a["gamma"], a["beta"],
+                             a["G"], a["eps"], a["silu"], a["weight"], a["bias"], a["residual"],
+                             a["out"], a["H"], a["W"], a["Cin"], a["Cout"], a["P"], a["mode"], stream=0)
+
+    for kw, code in [(dict(W=64), B.DP_ERR_UNSUPPORTED),          # tiles need 128 columns
+                     (dict(Cout=96), B.DP_ERR_UNSUPPORTED),       # Cout % 160
+                     (dict(used=0), B.DP_ERR_INVALID_ARG),
+                     (dict(eps=0.0), B.DP_ERR_INVALID_ARG),
+                     (dict(a_stale=0), B.DP_ERR_INVALID_ARG),     # displaced needs a_stale
+                     (dict(a_next=A + 64), B.DP_ERR_INVALID_ARG),  # a_next overlaps x
+                     (dict(H=15), B.DP_ERR_UNSUPPORTED)]:         # H % P
+        with pytest.raises(B.DPError) as e:
+            call(**kw)
+        assert e.value.code == code, kw
+    with pytest.raises(B.DPError) as e:                           # stats: displaced needs stale moments
+        B.dp_groupnorm_stats(A, 16, 128, 64, 32, 2, 1.0, B.DISPLACED, B.BF16, 0, 0, 2 * A, 3 * A, 4 * A,
+                             1 << 16, stream=0)
     assert e.value.code == B.DP_ERR_INVALID_ARG

@@ -20,21 +20,21 @@ pytestmark = pytest.mark.gpu
 KIND = {"gn_conv": B.GN_CONV, "resblock": B.RESBLOCK, "attn": B.ATTN, "unet_mini": B.UNET_MINI}
 
 
-def make_block(wl, gn_stats=B.GN_STATS_CORRECTED):
+def make_block(wl, gn_stats=B.GN_STATS_CORRECTED, gn_fuse=False):
     return B.Block(KIND[wl.kind], wl.H, wl.W, wl.C, wl.cout, wl.G, wl.P, wl.heads,
                    B.BF16 if wl.dtype == "bf16" else B.FP32, wl.silu, wl.eps, 1.0,
-                   gn_stats=gn_stats)
+                   gn_stats=gn_stats, gn_fuse=gn_fuse)
 
 
 def run_chain(wl, modes, random_affine, storage_rel=0.0, rl2=RL2, scale_rel=0.0,
-              gn_stats=B.GN_STATS_CORRECTED, chain=False):
+              gn_stats=B.GN_STATS_CORRECTED, chain=False, gn_fuse=False):
     """Steps the block through ``modes`` on the GPU and in the oracle and compares every
     step's output.  With ``chain`` the oracle also runs without storage rounding and the
     output is held by ``check_chain`` (the stated bar, or the floor bf16 storage sets)."""
     wts = synth.make_weights(wl, random_affine=random_affine)
     tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
     dev_w = block_weights(wl.kind, wts, tdt)
-    blk = make_block(wl, gn_stats)
+    blk = make_block(wl, gn_stats, gn_fuse)
     xs = synth.InputStream(wl)
     w64 = {n: v.double().numpy() for n, v in wts.items()}
     st, st_exact = {}, {}
@@ -70,6 +70,20 @@ def test_resblock_320x128x128():
     displaced steps whose stale state has been refreshed by every earlier step."""
     wl = synth.WORKLOADS["resblock_320x128x128"]
     run_chain(wl, [B.SYNC] * wl.warmup + [B.DISPLACED] * 2, True)
+
+
+@pytest.mark.parametrize("gn_stats", [B.GN_STATS_CORRECTED, B.GN_STATS_SYNC], ids=["corrected", "sync"])
+def test_resblock_320x128x128_gn_fusion(gn_stats):
+    """The same schedule with every GroupNorm -> conv pair through dp_groupnorm_stats +
+    dp_conv3x3_halo_gn: the state keeps only the band-edge rows of the normalised activations,
+    and every displaced step's halo comes from them."""
+    wl = synth.WORKLOADS["resblock_320x128x128"]
+    run_chain(wl, [B.SYNC] * wl.warmup + [B.DISPLACED] * 2, True, gn_stats=gn_stats, gn_fuse=True)
+
+
+def test_resblock_fusion_zero_warmup():
+    wl = synth.WORKLOADS["resblock_320x128x128"]
+    run_chain(wl, [B.NAIVE, B.DISPLACED, B.DISPLACED], False, gn_fuse=True)
 
 
 def test_resblock_zero_warmup():
@@ -200,15 +214,17 @@ def test_unet_mini_stages():
         h = O.store(ref, S)
 
 
-def test_gn_conv_320x480x480_sampled_rows():
+@pytest.mark.parametrize("gn_fuse", [False, True], ids=["separate", "fused"])
+def test_gn_conv_320x480x480_sampled_rows(gn_fuse):
     """The 3840x3840-shaped workload at full size over a sync step and two displaced steps:
     every band's first two and last two rows (the rows whose 3x3 window reaches another
-    band) and one interior row per band, computed by the oracle row by row."""
+    band) and one interior row per band, computed by the oracle row by row; with the
+    GroupNorm in its own passes, and fused into the conv's operand path."""
     wl = synth.WORKLOADS["gn_conv_320x480x480"]
     wts = synth.make_weights(wl, random_affine=True)
     dev_w = block_weights(wl.kind, wts, torch.bfloat16)
     W64 = {n: v.double().numpy() for n, v in wts.items()}
-    blk = make_block(wl)
+    blk = make_block(wl, gn_fuse=gn_fuse)
     xs = synth.InputStream(wl)
     hb = wl.H // wl.P
     rows = sorted({hb * p + i for p in range(wl.P) for i in (0, 1, hb // 2, hb - 2, hb - 1)})
