@@ -71,9 +71,16 @@ def load_peaks():
         with open(p) as f:
             d = json.load(f)
         return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
-                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"),
+                "sm_max_mhz": d.get("sm_max_mhz"), "source": "measured"}
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
             "source": "fallback"}
+
+
+# fp32 fused multiply-adds per clock per SM (4 sub-partitions x 32 lanes) and the SM
+# count of a B200: the peak of a kernel bound by fp32 CUDA-core arithmetic is
+# 148 * 128 * 2 flops * the SM clock (74.4 TFLOP/s at 1965 MHz)
+FP32_FMA_PER_CLK_PER_SM, B200_SMS = 128, 148
 
 
 def kernel_source_hash(files):
@@ -350,7 +357,7 @@ def workload_config(wl, ws, extra=None):
            "l2": l2_policy(wl)[1],
            "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"}
     if wl.dtype == "fp32":
-        cfg["arithmetic"] = "fp32 storage, conv on tf32 tensor cores with fp32 accumulation"
+        cfg["arithmetic"] = "fp32 storage and arithmetic; the conv on the CUDA cores"
     cfg.update(extra or {})
     return cfg
 
@@ -464,17 +471,22 @@ def breakdown(run, steps, flush, peaks):
            "gn_stats": ["dp_gn.cu"], "gn_apply": ["dp_gn.cu"], "gn_fused": ["dp_gn.cu"],
            "gn_cluster": ["dp_gn.cu"], "copy": ["dp_refresh.cu"],
            "conv_small": ["dp_conv_small.cu"], "splitk_finish": ["dp_gemm.cu"],
+           "conv_f32": ["dp_conv_f32.cu"],
            "layernorm": ["dp_token.cu"], "geglu": ["dp_token.cu"], "temb": ["dp_temb.cu"]}
     traffic = load_traffic(f"{dominant}:{run.wl.name}", kernel_source_hash(src[dominant]))
-    if dk["tflops"]:
+    if dk["tflops"] and dominant in ("conv_f32", "conv_small"):
+        sm_mhz = peaks.get("sm_max_mhz") or 1965.0
+        alu_peak = B200_SMS * FP32_FMA_PER_CLK_PER_SM * 2 * sm_mhz * 1e6 / 1e12
+        roof = {"bound": "alu", "achieved": dk["tflops"], "peak": round(alu_peak, 1), "unit": "TFLOP/s",
+                "frac": round(dk["tflops"] / alu_peak, 4), "traffic": traffic, "kernel": dominant,
+                "peak_source": "derived: 148 SMs x 128 fp32 FMA/clk x 2 flops x max SM clock"}
+    elif dk["tflops"]:
         roof = {"bound": "tensor", "achieved": dk["tflops"], "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": round(dk["tflops"] / peaks["bf16_tflops"], 4),
                 "traffic": traffic, "kernel": dominant,
                 "peak_source": f"{peaks['source']} bf16 burst",
                 "frac_of_sustained": round(dk["tflops"] / peaks["bf16_tflops_sustained"], 4)
                 if peaks.get("bf16_tflops_sustained") else None}
-        if run.wl.dtype == "fp32":
-            roof["note"] = "tf32 contraction measured against the bf16 peak"
     else:
         roof = {"bound": "hbm", "achieved": dk["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(dk["gbs"] / peaks["hbm_gbs"], 4), "traffic": traffic,

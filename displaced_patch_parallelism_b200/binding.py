@@ -348,7 +348,7 @@ def dp_block_step_timed(d: BlockDesc, s: BlockState, x, out, weights: Sequence, 
 
 KERNEL_NAMES = {0: "gn_stats", 1: "gn_apply", 2: "gn_fused", 3: "conv", 4: "linear", 5: "attn",
                 6: "copy", 7: "conv_small", 8: "splitk_finish",
-                9: "gn_cluster", 10: "layernorm", 11: "geglu", 12: "temb", 13: "conv_gn"}
+                9: "gn_cluster", 10: "layernorm", 11: "geglu", 12: "temb", 13: "conv_gn", 14: "conv_f32"}
 
 
 def dp_block_launch_info(d: BlockDesc, mode: int, i: int):

@@ -334,7 +334,10 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
     if (plan) {
       const double ho = (h - 1) / stride + 1, wo = (wd - 1) / stride + 1;
       const int S = conv3x3_splits(h, wd, ci, co, stride, d->dtype, true);
-      if (S == 1) {
+      if (d->dtype == DP_FP32) {
+        plan->push(DP_KERNEL_CONV_F32, 2.0 * ho * wo * co * 9.0 * ci,
+                   (static_cast<double>(h) * wd * ci + ho * wo * co * (res ? 2 : 1)) * e);
+      } else if (S == 1) {
         plan->push(DP_KERNEL_CONV, 2.0 * ho * wo * co * 9.0 * ci,
                    (static_cast<double>(h) * wd * ci + ho * wo * co * (res ? 2 : 1)) * e);
       } else {

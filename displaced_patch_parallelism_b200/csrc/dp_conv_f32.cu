@@ -1,0 +1,120 @@
+// dp_conv_f32.cu -- the stale-halo 3x3 conv in fp32 on the CUDA cores.
+//
+// Same operation and halo rule as the bf16 tensor-core conv ("DistriFusion",
+// study.space summary, Method): output row r of band p reads input row
+// rho = stride*r + kh - 1 from the fresh buffer when it lies in band p,
+// otherwise from the fresh buffer (sync), the stale buffer (displaced) or
+// nowhere (naive: zeros); outside the image it is zero padding.  Storage and
+// arithmetic are fp32 (fp32 fused multiply-adds, no narrower operand format):
+// the fp32 workloads state fp32, and at their sizes (tens of MFLOP) the
+// launch, not the math, sets the time.
+//
+// A block computes one output row x 32 columns x 32 output channels.  It
+// walks the input channels 16 at a time: the three input rows the row
+// window needs ([kh][ci][column], zero where the halo rule or the image edge
+// says so) and the filter slice ([tap][ci][co]) go to shared memory, then
+// each thread accumulates 4 output channels of one column (lane = column,
+// warp = channel quad): one input load per (tap, ci) that neighbouring lanes
+// take from neighbouring banks, and one 16-byte filter load that every lane
+// of the warp shares.
+#include "dp_common.cuh"
+#include "dp_internal.h"
+
+namespace dp {
+
+constexpr int kF32Px = 32;    // output columns of a block
+constexpr int kF32Co = 32;    // output channels of a block
+constexpr int kF32Ci = 16;    // input channels staged at a time
+
+__global__ void __launch_bounds__(256) conv3x3_f32_kernel(
+    const float* __restrict__ af, const float* __restrict__ as, const float* __restrict__ w,
+    const float* __restrict__ bias, const float* __restrict__ residual, float* __restrict__ out,
+    int H, int W, int Ho, int Wo, int Cin, int Cout, int stride, int hb_in, int hb_out, int mode) {
+  constexpr int kMaxSpan = 2 * (kF32Px - 1) + 3;            // input columns of a window, stride <= 2
+  __shared__ float s_in[3][kF32Ci][kMaxSpan + 1];
+  __shared__ __align__(16) float s_w[9][kF32Ci][kF32Co];
+  griddep_wait();
+  griddep_trigger();
+  const int c0 = blockIdx.x * kF32Px, r = blockIdx.y, co0 = blockIdx.z * kF32Co;
+  const int lane = threadIdx.x & 31, quad = threadIdx.x >> 5;
+  const int span = stride * (kF32Px - 1) + 3;
+  const int band = r / hb_out;
+  // the source of each of the three input rows: fresh, stale or none
+  const float* src[3];
+  int rows[3];
+#pragma unroll
+  for (int kh = 0; kh < 3; ++kh) {
+    const int rho = stride * r + kh - 1;
+    rows[kh] = rho;
+    src[kh] = nullptr;
+    if (rho < 0 || rho >= H) continue;
+    if (rho / hb_in == band || mode == DP_MODE_SYNC) src[kh] = af;
+    else if (mode == DP_MODE_DISPLACED) src[kh] = as;
+  }
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int ci0 = 0; ci0 < Cin; ci0 += kF32Ci) {
+    // input window: consecutive threads take consecutive channels of a pixel
+    for (int i = threadIdx.x; i < 3 * span * kF32Ci; i += blockDim.x) {
+      const int ci = i % kF32Ci, rest = i / kF32Ci;
+      const int px = rest % span, kh = rest / span;
+      const int col = stride * c0 + px - 1;
+      float v = 0.f;
+      if (src[kh] && col >= 0 && col < W)
+        v = __ldg(src[kh] + (static_cast<size_t>(rows[kh]) * W + col) * Cin + ci0 + ci);
+      s_in[kh][ci][px] = v;
+    }
+    // filter slice [tap][ci][co] of this block's 32 output channels
+    for (int i = threadIdx.x; i < 9 * kF32Ci * kF32Co; i += blockDim.x) {
+      const int ci = i % kF32Ci, rest = i / kF32Ci;
+      const int tap = rest % 9, co = rest / 9;
+      s_w[tap][ci][co] = __ldg(w + (static_cast<size_t>(co0 + co) * 9 + tap) * Cin + ci0 + ci);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kh = 0; kh < 3; ++kh)
+#pragma unroll
+      for (int kw = 0; kw < 3; ++kw) {
+        const int px = stride * lane + kw;
+#pragma unroll 4
+        for (int ci = 0; ci < kF32Ci; ++ci) {
+          const float v = s_in[kh][ci][px];
+          const float4 wq = *reinterpret_cast<const float4*>(&s_w[kh * 3 + kw][ci][4 * quad]);
+          acc[0] = fmaf(v, wq.x, acc[0]);
+          acc[1] = fmaf(v, wq.y, acc[1]);
+          acc[2] = fmaf(v, wq.z, acc[2]);
+          acc[3] = fmaf(v, wq.w, acc[3]);
+        }
+      }
+    __syncthreads();   // the next channel slice overwrites the staging
+  }
+  const int c = c0 + lane;
+  if (c >= Wo) return;
+  const int co = co0 + 4 * quad;
+  const size_t o = (static_cast<size_t>(r) * Wo + c) * Cout + co;
+  float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (residual) res = *reinterpret_cast<const float4*>(residual + o);
+  float4 b4 = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (bias) b4 = *reinterpret_cast<const float4*>(bias + co);
+  *reinterpret_cast<float4*>(out + o) =
+      make_float4(acc[0] + b4.x + res.x, acc[1] + b4.y + res.y, acc[2] + b4.z + res.z,
+                  acc[3] + b4.w + res.w);
+}
+
+int conv3x3_f32_launch(const void* a_fresh, const void* a_stale, const void* weight, const float* bias,
+                       const void* residual, void* out, int H, int W, int Cin, int Cout, int stride, int P,
+                       int mode, cudaStream_t stream) {
+  if (Cin % kF32Ci || Cout % kF32Co)
+    return set_error(DP_ERR_UNSUPPORTED, "fp32 conv: needs Cin %% %d == 0 and Cout %% %d == 0", kF32Ci,
+                     kF32Co);
+  if (bias && !aligned16(bias)) return set_error(DP_ERR_UNSUPPORTED, "fp32 conv: bias not 16-byte aligned");
+  const int Ho = (H - 1) / stride + 1, Wo = (W - 1) / stride + 1;
+  const dim3 grid((Wo + kF32Px - 1) / kF32Px, Ho, Cout / kF32Co);
+  mark_launch(stream);
+  return launch_kernel(conv3x3_f32_kernel, grid, dim3(256), 0, stream, false, "fp32 conv launch",
+                       static_cast<const float*>(a_fresh),
+                       static_cast<const float*>(a_stale ? a_stale : a_fresh),
+                       static_cast<const float*>(weight), bias, static_cast<const float*>(residual),
+                       static_cast<float*>(out), H, W, Ho, Wo, Cin, Cout, stride, H / P, Ho / P, mode);
+}
+
+}  // namespace dp

@@ -26,7 +26,7 @@
 //  * stride 2 views the image as [H][W/2][2*Cin] (two neighbouring columns
 //    side by side in the channel axis): the three column taps become two
 //    channel halves of pairs c-1 and c, and the same TMA boxes serve.
-//  * tf32 (fp32 storage) uses the same tiles with 32 fp32 per 128-byte row.
+//  * fp32 storage runs in fp32 on the CUDA cores instead (dp_conv_f32.cu).
 #include <algorithm>
 #include <cstring>
 #include <type_traits>
@@ -1382,13 +1382,7 @@ static int launch_t(const GemmParams& p, cudaStream_t s) {
 }
 
 static int launch_gemm(const GemmParams& p, int BN, bool tf32, cudaStream_t s) {
-  if (tf32) {
-    switch (BN) {
-      case 64: return launch_t<64, true>(p, s);
-      case 128: return launch_t<128, true>(p, s);
-      default: break;
-    }
-  } else {
+  if (!tf32) {
     switch (BN) {
       case 32: return launch_t<32, false>(p, s);
       case 64: return launch_t<64, false>(p, s);
@@ -1592,7 +1586,11 @@ int conv3x3_launch(const void* a_fresh, const void* a_stale, const void* weight,
                    const float* bias, const void* residual, void* out, int H, int W, int Cin,
                    int Cout, int stride, int P, int mode, int dtype, void* workspace,
                    size_t workspace_bytes, cudaStream_t stream) {
-  const bool tf32 = dtype == DP_FP32;
+  // fp32 storage: fp32 arithmetic on the CUDA cores (dp_conv_f32.cu)
+  if (dtype == DP_FP32)
+    return conv3x3_f32_launch(a_fresh, a_stale, weight, bias, residual, out, H, W, Cin, Cout, stride, P,
+                              mode, stream);
+  const bool tf32 = false;
   const int e = tf32 ? 4 : 2;
   const int BK = 128 / e;
   const int Ho = (H - 1) / stride + 1, Wo = (W - 1) / stride + 1;
@@ -1839,10 +1837,9 @@ int conv3x3_validate(const void* a_fresh, const void* a_stale, const void* weigh
   if (stride != 1 && stride != 2) return set_error(DP_ERR_UNSUPPORTED, "conv: stride must be 1 or 2");
   if (mode == DP_MODE_DISPLACED && !a_stale)
     return set_error(DP_ERR_INVALID_ARG, "conv: displaced mode needs the stale buffer");
-  const int BK = dtype == DP_FP32 ? 32 : 64;
+  const int BK = dtype == DP_FP32 ? 16 : 64;
   if (Cin % BK) return set_error(DP_ERR_UNSUPPORTED, "conv: Cin must be a multiple of %d", BK);
   if (Cout % 32) return set_error(DP_ERR_UNSUPPORTED, "conv: Cout must be a multiple of 32");
-  if (dtype == DP_FP32 && Cout % 64) return set_error(DP_ERR_UNSUPPORTED, "conv: fp32 needs Cout %% 64 == 0");
   const int Ho = (H - 1) / stride + 1;
   if (H % P || Ho % P) return set_error(DP_ERR_UNSUPPORTED, "conv: rows not divisible by P");
   if (stride == 2 && (W % 2)) return set_error(DP_ERR_UNSUPPORTED, "conv: stride 2 needs even W");

@@ -25,6 +25,10 @@ int conv3x3_validate(const void* a_fresh, const void* a_stale, const void* weigh
                      const void* residual, const void* out, int H, int W, int Cin, int Cout,
                      int stride, int P, int mode, int dtype);
 size_t gemm_workspace_bytes();
+// the 3x3 halo conv in fp32 on the CUDA cores (fp32 storage)
+int conv3x3_f32_launch(const void* a_fresh, const void* a_stale, const void* weight, const float* bias,
+                       const void* residual, void* out, int H, int W, int Cin, int Cout, int stride, int P,
+                       int mode, cudaStream_t stream);
 // GroupNorm statistics alone (the first kernel of the two-kernel path): fresh
 // moments, used moments and (if given) the whole-image moments; no apply.
 int gn_stats_launch(const void* x, int H, int W, int C, int G, int P, float w, int mode, int dtype,

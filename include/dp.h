@@ -29,8 +29,9 @@
  *  - Modes: DP_MODE_SYNC (warm-up step: every band sees fresh context),
  *    DP_MODE_DISPLACED (other bands' context is the stale previous step),
  *    DP_MODE_NAIVE (other bands are invisible: zero halo, own keys only).
- *  - dtype: DP_BF16 (bf16 storage, fp32 accumulation) or DP_FP32 (fp32
- *    storage; the 3x3 conv then multiplies in tf32 with fp32 accumulation).
+ *  - dtype: DP_BF16 (bf16 storage, bf16 tensor-core products, fp32
+ *    accumulation) or DP_FP32 (fp32 storage and fp32 arithmetic throughout;
+ *    the 3x3 conv then runs on the CUDA cores).
  *    Statistics, GroupNorm scale/shift and biases are always fp32.
  */
 #ifndef DP_H
@@ -222,10 +223,10 @@ DP_API int dp_groupnorm_async_noalloc(const void* x, void* y, const float* gamma
  *                    separate SM pairs; each run stores an fp32 partial and
  *                    the last run of a tile sums them in run order.  Calls
  *                    that overlap on the GPU must not share it.
- * Ho = (H-1)/stride + 1.  Needs Cin % 64 == 0 (bf16) or % 32 == 0 (fp32),
- * Cout % 32 == 0 (fp32: Cout % 64 == 0), H % P == 0, Ho % P == 0, W even when
- * stride 2.  Any W works; ragged tiles are masked.
- * Runs on the tensor cores (tcgen05, operands staged by TMA).
+ * Ho = (H-1)/stride + 1.  Needs Cin % 64 == 0 (bf16) or % 16 == 0 (fp32),
+ * Cout % 32 == 0, H % P == 0, Ho % P == 0, W even when stride 2.  Any W works;
+ * ragged tiles are masked.  bf16 runs on the tensor cores (tcgen05, operands
+ * staged by TMA); fp32 runs in fp32 on the CUDA cores (bias 16-byte aligned).
  * Errors: DP_ERR_INVALID_ARG (null pointers, bad mode/dtype, aliasing,
  * missing stale buffer in DISPLACED), DP_ERR_UNSUPPORTED (shape, alignment).
  * ---------------------------------------------------------------------- */
@@ -601,6 +602,7 @@ DP_API int dp_block_status(const dp_block_desc* d, const dp_block_state* s, void
 #define DP_KERNEL_GEGLU 11      /* gated GELU unit of the feed-forward          */
 #define DP_KERNEL_TEMB 12       /* time-embedding bias of a ResBlock's conv1     */
 #define DP_KERNEL_CONV_GN 13    /* 3x3 conv of GroupNorm(x), normalised in-kernel */
+#define DP_KERNEL_CONV_F32 14   /* 3x3 halo conv in fp32 on the CUDA cores       */
 
 /*
  * Number of kernel launches one displaced dp_block_step makes for this

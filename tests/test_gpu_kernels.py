@@ -11,7 +11,7 @@ import torch
 
 from displaced_patch_parallelism_b200 import binding as B
 from oracle import dp_oracle as O
-from tests.helpers import (BF16_HALF_ULP, STATS_ATOL, check, conv_w_dev, dev_f32, dev_img,
+from tests.helpers import (F32_ATOL, F32_RL2, BF16_HALF_ULP, STATS_ATOL, check, conv_w_dev, dev_f32, dev_img,
                            dev_mat, host, host_img, rounded)
 
 pytestmark = pytest.mark.gpu
@@ -150,6 +150,9 @@ CONV_CASES = [
     (320, 160, 6, 240, 3, 1, "bf16", False),    # halo-row pair kernel, 256x160, ragged row
     (64, 64, 16, 16, 2, 1, "fp32", False),
     (64, 128, 8, 10, 2, 1, "fp32", True),
+    (32, 64, 9, 40, 3, 1, "fp32", True),        # fp32: ragged 32-column block, 16-channel slices
+    (64, 32, 16, 20, 2, 2, "fp32", True),       # fp32, stride 2
+    (16, 96, 8, 8, 1, 1, "fp32", False),        # fp32, one band
     (320, 320, 32, 48, 1, 1, "bf16", True),     # one band: no halo from other bands
     (64, 64, 16, 16, 1, 2, "bf16", False),      # one band, stride 2
 ]
@@ -173,8 +176,10 @@ def test_conv3x3_halo_parity(case, mode):
                       dev_img(res, dtype) if use_res else None, out, H, W, Cin, Cout, stride, P,
                       mode, B.BF16 if dtype == "bf16" else B.FP32)
     torch.cuda.synchronize()
-    check(host_img(out), ref, what=f"conv {case} mode {mode}",
-          storage_rel=BF16_HALF_ULP if dtype == "bf16" else 0.0)
+    if dtype == "fp32":
+        check(host_img(out), ref, atol=F32_ATOL, rl2=F32_RL2, what=f"conv {case} mode {mode}")
+    else:
+        check(host_img(out), ref, what=f"conv {case} mode {mode}", storage_rel=BF16_HALF_ULP)
     assert B.dp_device_status() == 0
 
 
