@@ -35,6 +35,8 @@ Readings of what the pages leave open:
       stale-only and exact statistics): see ``gn_variant_mode``
   R15 the pages' sampler is "50-step DDIM" with no update printed: the
       deterministic DDIM step (``ddim_step``), alpha-bar values from the caller
+  R16 the pages' warm-up ablation names a "10-step DPM-Solver" with no update
+      printed: the multistep second-order DPM-Solver++ (``dpm_solver_2m_step``)
   R13 the pages name SDXL but not its blocks' insides: the plainest SDXL
       transformer block (``transformer_step``) and ResBlock time embedding
       (``resblock_step``'s ``temb``); only GroupNorm statistics and
@@ -51,6 +53,10 @@ block and the time-embedding ResBlock equal the same blocks composed from
 library operators at P = 1; ``time_embedding_term`` is the library linear of
 the library SiLU; ``ddim_step`` moves an exactly known noise to the previous
 level, is the identity at an unchanged level, composes, and is affine.
+``dpm_solver_2m_step`` in its first-order form equals the DDIM step, its
+second-order form equals the first when the data prediction does not change,
+and on an ODE whose exact solution is known it converges at second order (the
+first-order form at first order).
 ``unet_mini_step`` at P = 1 equals the same chain composed from library
 operators (conv2d with stride 1 and 2, the library ResBlock and attention with
 10 and 20 heads); its naive step at P = 4 equals that library chain on each
@@ -424,6 +430,35 @@ def ddim_step(x, eps, abar_t: float, abar_prev: float) -> np.ndarray:
     x, eps = _a(x), _a(eps)
     x0 = (x - math.sqrt(1.0 - abar_t) * eps) / math.sqrt(abar_t)
     return math.sqrt(abar_prev) * x0 + math.sqrt(1.0 - abar_prev) * eps
+
+
+def dpm_solver_2m_step(x, eps, x0_prev, abar_prev: float, abar_s: float, abar_t: float):
+    """One step of the multistep second-order DPM-Solver++ (reading R16; Lu, Zhou, Bao, Chen,
+    Li and Zhu, "DPM-Solver++: Fast Solver for Guided Sampling of Diffusion Probabilistic
+    Models", the multistep second-order solver in data prediction), the sampler of the pages'
+    "10-step DPM-Solver" warm-up ablation (atlas.scime.ai summary).  Moves the latent x from
+    the level abar_s to the less noisy level abar_t.  Returns (x_t, x0), x0 being this step's
+    data prediction, which the next step takes as its x0_prev.
+
+    With alpha = sqrt(abar), sigma = sqrt(1 - abar), lambda = log(alpha / sigma), h = lambda_t -
+    lambda_s:  x0 = (x - sigma_s eps) / alpha_s;  D = x0 for a first-order step (x0_prev None or
+    abar_prev <= 0, and the final step to abar_t = 1), otherwise D = x0 + (x0 - x0_prev) / (2 r)
+    with r = (lambda_s - lambda_prev) / h;  x_t = (sigma_t / sigma_s) x - alpha_t (exp(-h) - 1) D.
+    """
+    x, eps = _a(x), _a(eps)
+    a_s, s_s = math.sqrt(abar_s), math.sqrt(1.0 - abar_s)
+    x0 = (x - s_s * eps) / a_s
+    if abar_t >= 1.0:                      # the final step: the clean sample, first order
+        return x0.copy(), x0
+    a_t, s_t = math.sqrt(abar_t), math.sqrt(1.0 - abar_t)
+    lam_s, lam_t = math.log(a_s / s_s), math.log(a_t / s_t)
+    h = lam_t - lam_s
+    D = x0
+    if x0_prev is not None and abar_prev > 0.0:
+        lam_p = math.log(math.sqrt(abar_prev) / math.sqrt(1.0 - abar_prev))
+        r = (lam_s - lam_p) / h
+        D = x0 + (x0 - _a(x0_prev)) / (2.0 * r)
+    return (s_t / s_s) * x - a_t * (math.exp(-h) - 1.0) * D, x0
 
 
 def resblock_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float,

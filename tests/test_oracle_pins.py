@@ -855,3 +855,66 @@ def test_ddim_step_identity_and_composition():
     lin = O.ddim_step(2 * x - x2, 2 * e - e2, 0.2, 0.3)
     np.testing.assert_allclose(lin, 2 * O.ddim_step(x, e, 0.2, 0.3) - O.ddim_step(x2, e2, 0.2, 0.3),
                                rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- DPM-Solver++ (2M)
+def test_dpm_solver_first_order_is_ddim():
+    """The first-order step of DPM-Solver++ is the deterministic DDIM step: with
+    exp(-h) = sigma_t alpha_s / (alpha_t sigma_s) the update becomes alpha_t x0 + sigma_t eps."""
+    r = rng(120)
+    x, e = r.standard_normal((3, 6, 5)), r.standard_normal((3, 6, 5))
+    for abar_s, abar_t in [(0.0047, 0.0066), (0.3, 0.45), (0.9, 0.97), (0.6, 1.0)]:
+        got, x0 = O.dpm_solver_2m_step(x, e, None, 0.0, abar_s, abar_t)
+        np.testing.assert_allclose(got, O.ddim_step(x, e, abar_s, abar_t), rtol=0, atol=1e-11)
+        np.testing.assert_allclose(x0, (x - math.sqrt(1 - abar_s) * e) / math.sqrt(abar_s), rtol=0,
+                                   atol=1e-12)
+
+
+def test_dpm_solver_second_order_with_constant_prediction_is_first_order():
+    """D = x0 + (x0 - x0_prev) / (2r): an unchanged data prediction leaves the first-order step."""
+    r = rng(121)
+    x, e = r.standard_normal(30), r.standard_normal(30)
+    _, x0 = O.dpm_solver_2m_step(x, e, None, 0.0, 0.2, 0.3)
+    got, _ = O.dpm_solver_2m_step(x, e, x0, 0.12, 0.2, 0.3)
+    np.testing.assert_allclose(got, O.dpm_solver_2m_step(x, e, None, 0.0, 0.2, 0.3)[0], rtol=0, atol=1e-12)
+    # and a changed one moves it by alpha_t (1 - e^{-h}) (x0 - x0_prev) / (2r), the sign included
+    got2, _ = O.dpm_solver_2m_step(x, e, x0 - 1.0, 0.12, 0.2, 0.3)
+    lam = lambda ab: math.log(math.sqrt(ab) / math.sqrt(1 - ab))
+    h, hp = lam(0.3) - lam(0.2), lam(0.2) - lam(0.12)
+    shift = math.sqrt(0.3) * (1 - math.exp(-h)) * 1.0 / (2 * hp / h)
+    np.testing.assert_allclose(got2 - got, shift, rtol=1e-12, atol=1e-12)
+
+
+def _ode_errors(order, n_steps):
+    """Integrates the data-prediction ODE x' = x + ... along lambda from -2 to 1, whose exact
+    solution for the data prediction x0(lambda) = cos(lambda) is known in closed form:
+    x(l) = (sigma_l / sigma_a) x(a) + sigma_l * integral_a^l e^u cos(u) du.  The solver sees
+    eps = (x - alpha x0(lambda)) / sigma, i.e. an exact model.  Returns the final error."""
+    lam = np.linspace(-2.0, 1.0, n_steps + 1)
+    ab = lambda l: 1.0 / (1.0 + math.exp(-2.0 * l))          # alpha^2 with lambda = log(alpha/sigma)
+    sig = lambda l: math.sqrt(1.0 - ab(l))
+    prim = lambda u: math.exp(u) * (math.cos(u) + math.sin(u)) / 2.0
+    exact = lambda l, x_a, a: sig(l) / sig(a) * x_a + sig(l) * (prim(l) - prim(a))
+    x_a = 0.7
+    x, x0_prev, ab_prev = x_a, None, 0.0
+    for i in range(n_steps):
+        l_s, l_t = lam[i], lam[i + 1]
+        e = (x - math.sqrt(ab(l_s)) * math.cos(l_s)) / sig(l_s)
+        use_prev = x0_prev if order == 2 else None
+        x, x0_prev = O.dpm_solver_2m_step(np.array(x), np.array(e), use_prev, ab_prev if order == 2 else 0.0,
+                                          ab(l_s), ab(l_t))
+        x = float(x)
+        ab_prev = ab(l_s)
+    return abs(x - exact(lam[-1], x_a, lam[0]))
+
+
+def test_dpm_solver_convergence_order():
+    """Halving the step halves the first-order error and quarters the second-order one: the
+    multistep correction has the published coefficient and sign."""
+    e1 = [_ode_errors(1, n) for n in (20, 40, 80)]
+    e2 = [_ode_errors(2, n) for n in (20, 40, 80)]
+    for a, b in zip(e1, e1[1:]):
+        assert 1.8 < a / b < 2.2, e1
+    for a, b in zip(e2, e2[1:]):
+        assert 3.5 < a / b < 4.5, e2
+    assert e2[-1] < e1[-1] / 5      # and more accurate at the same step count
