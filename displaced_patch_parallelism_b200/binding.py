@@ -74,6 +74,8 @@ _SIGS = {
     "dp_geglu": ([_V, _V, _I, _I, _V], _I),
     "dp_time_embedding_bias": ([_V, _V, _V, _V, _V, _I, _I, _V], _I),
     "dp_ddim_step": ([_V, _V, _V, _SZ, ctypes.c_double, ctypes.c_double, _I, _V], _I),
+    "dp_dpm_solver_step": ([_V, _V, _V, _V, _SZ, ctypes.c_double, ctypes.c_double, ctypes.c_double, _I, _V],
+                           _I),
     "dp_refresh_stale": ([_V, _V, _SZ, _I, _I, _I, _V], _I),
     "dp_refresh_halo": ([_V, _V, _SZ, _I, _I, _I, _I, _V], _I),
     "dp_refresh_stats": ([_V, _V, _V, _I, _I, _V], _I),
@@ -265,6 +267,11 @@ def dp_time_embedding_bias(temb, temb_w, temb_b, conv_b, bias, Ct, Cout, stream=
 def dp_ddim_step(x, eps, x_prev, n, abar_t, abar_prev, dtype, stream=None):
     return _check(lib().dp_ddim_step(_p(x), _p(eps), _p(x_prev), n, abar_t, abar_prev, dtype,
                                      _s(stream)))
+
+
+def dp_dpm_solver_step(x, eps, x0_buf, x_next, n, abar_prev, abar_s, abar_t, dtype, stream=None):
+    return _check(lib().dp_dpm_solver_step(_p(x), _p(eps), _p(x0_buf), _p(x_next), n, abar_prev, abar_s,
+                                           abar_t, dtype, _s(stream)))
 
 
 def dp_refresh_stale(fresh, stale, row_bytes, rows, P, band=-1, stream=None):

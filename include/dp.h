@@ -396,6 +396,32 @@ DP_API int dp_ddim_step(const void* x, const void* eps, void* x_prev, size_t n, 
                         double abar_prev, int dtype, void* stream);
 
 /* ------------------------------------------------------------------------
+ * The multistep second-order DPM-Solver++ update ("next" item: the pages'
+ * warm-up ablation uses a "10-step DPM-Solver"; Lu, Zhou, Bao, Chen, Li and
+ * Zhu, "DPM-Solver++", the multistep second-order solver in data prediction),
+ * elementwise over n values, from level abar_s to the less noisy abar_t:
+ *   x0     = (x - sqrt(1 - abar_s) eps) / sqrt(abar_s)
+ *   D      = x0 + (x0 - x0_prev) h / (2 (lambda_s - lambda_prev))   (2nd order)
+ *   D      = x0                                  (1st order: abar_prev == 0)
+ *   x_next = (sigma_t / sigma_s) x + alpha_t (1 - exp(-h)) D
+ * with alpha = sqrt(abar), sigma = sqrt(1 - abar), lambda = log(alpha / sigma),
+ * h = lambda_t - lambda_s; abar_t == 1 (the final step) gives x_next = x0.
+ *  x, eps     n values of `dtype` (DP_BF16 or DP_FP32), device, 16-byte aligned
+ *  x0_buf     n values: on entry the previous step's x0 (read only when
+ *             abar_prev > 0), on exit this step's x0 for the next step
+ *  x_next     n values, written; may BE x, may not otherwise overlap x, eps or
+ *             x0_buf (x0_buf may not overlap any of the others)
+ *  abar_prev  alpha-bar of the previous step's level (0 for a first-order step),
+ *             0 < abar_prev < abar_s < abar_t <= 1 otherwise
+ * The host folds the schedule into five fp32 coefficients (in double); the
+ * kernel does three fp32 fused multiply-adds per element.  DP_ERR_INVALID_ARG
+ * on null pointers, bad dtype, levels out of order or overlap;
+ * DP_ERR_UNSUPPORTED on misalignment.  n == 0 launches nothing.
+ * ---------------------------------------------------------------------- */
+DP_API int dp_dpm_solver_step(const void* x, const void* eps, void* x0_buf, void* x_next, size_t n,
+                              double abar_prev, double abar_s, double abar_t, int dtype, void* stream);
+
+/* ------------------------------------------------------------------------
  * Per-token operators of an SDXL-shaped transformer block ("next" item: the
  * pages name SDXL as the model; they act on each token alone, so every band
  * runs them on its fresh tokens with no stale context).

@@ -479,3 +479,17 @@ def test_groupnorm_conv_rejects_bad_arguments_on_the_host(B):
         B.dp_groupnorm_stats(A, 16, 128, 64, 32, 2, 1.0, B.DISPLACED, B.BF16, 0, 0, 2 * A, 3 * A, 4 * A,
                              1 << 16, stream=0)
     assert e.value.code == B.DP_ERR_INVALID_ARG
+
+
+def test_dpm_solver_rejects_bad_arguments_on_the_host(B):
+    A = 1 << 20                                   # fake, never dereferenced: checks run first
+    good = (A, 2 * A, 3 * A, 4 * A, 64, 0.1, 0.2, 0.3, B.FP32)
+    for args, code in [((0,) + good[1:], B.DP_ERR_INVALID_ARG),                       # null x
+                       (good[:5] + (0.1, 0.3, 0.2, B.FP32), B.DP_ERR_INVALID_ARG),   # abar_t < abar_s
+                       (good[:5] + (0.25, 0.2, 0.3, B.FP32), B.DP_ERR_INVALID_ARG),  # abar_prev > abar_s
+                       (good[:8] + (7,), B.DP_ERR_INVALID_ARG),                       # dtype
+                       ((A, 2 * A, A + 64, 4 * A) + good[4:], B.DP_ERR_INVALID_ARG),  # x0_buf overlaps x
+                       ((A + 8,) + good[1:], B.DP_ERR_UNSUPPORTED)]:                  # misaligned
+        with pytest.raises(B.DPError) as e:
+            B.dp_dpm_solver_step(*args, stream=0)
+        assert e.value.code == code, args
