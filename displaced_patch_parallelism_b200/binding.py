@@ -38,7 +38,8 @@ class BlockDesc(ctypes.Structure):
                 ("P", ctypes.c_int), ("heads", ctypes.c_int), ("dtype", ctypes.c_int),
                 ("silu", ctypes.c_int), ("eps", ctypes.c_float), ("w", ctypes.c_float),
                 ("gn_stats", ctypes.c_int), ("ctx_len", ctypes.c_int), ("ctx_dim", ctypes.c_int),
-                ("ff_inner", ctypes.c_int), ("temb_dim", ctypes.c_int), ("gn_fuse", ctypes.c_int)]
+                ("ff_inner", ctypes.c_int), ("temb_dim", ctypes.c_int), ("gn_fuse", ctypes.c_int),
+                ("depth", ctypes.c_int)]
 
 
 class BlockState(ctypes.Structure):
@@ -83,6 +84,7 @@ _SIGS = {
     "dp_block_desc_set_gn_stats": ([ctypes.POINTER(BlockDesc), _I], _I),
     "dp_block_desc_set_gn_fusion": ([ctypes.POINTER(BlockDesc), _I], _I),
     "dp_block_desc_set_context": ([ctypes.POINTER(BlockDesc), _I, _I, _I], _I),
+    "dp_block_desc_set_depth": ([ctypes.POINTER(BlockDesc), _I], _I),
     "dp_block_desc_set_time_embedding": ([ctypes.POINTER(BlockDesc), _I], _I),
     "dp_block_workspace_size": ([ctypes.POINTER(BlockDesc)], _SZ),
     "dp_block_state_init": ([ctypes.POINTER(BlockDesc), ctypes.POINTER(BlockState), _V, _SZ, _V], _I),
@@ -308,6 +310,10 @@ def dp_block_desc_set_context(d: BlockDesc, ctx_len: int, ctx_dim: int, ff_inner
     return _check(lib().dp_block_desc_set_context(ctypes.byref(d), ctx_len, ctx_dim, ff_inner))
 
 
+def dp_block_desc_set_depth(d: BlockDesc, depth: int):
+    return _check(lib().dp_block_desc_set_depth(ctypes.byref(d), depth))
+
+
 def dp_block_desc_set_time_embedding(d: BlockDesc, temb_dim: int):
     return _check(lib().dp_block_desc_set_time_embedding(ctypes.byref(d), temb_dim))
 
@@ -382,13 +388,15 @@ class Block:
 
     def __init__(self, kind, H, W, C, Cout=0, G=32, P=4, heads=0, dtype=BF16, silu=True,
                  eps=1e-5, w=1.0, device="cuda", stream=None, gn_stats=GN_STATS_CORRECTED,
-                 context=None, temb_dim=0, gn_fuse=False):
+                 context=None, temb_dim=0, gn_fuse=False, depth=1):
         """``context`` = (ctx_len, ctx_dim, ff_inner) for TRANSFORMER blocks; ``temb_dim`` the
         time-embedding width of a RESBLOCK (0: none)."""
         import torch
         self.desc = dp_block_desc_init(kind, H, W, C, Cout, G, P, heads, dtype, silu, eps, w)
         if context is not None:
             dp_block_desc_set_context(self.desc, *context)
+        if depth != 1:
+            dp_block_desc_set_depth(self.desc, depth)
         if temb_dim:
             dp_block_desc_set_time_embedding(self.desc, temb_dim)
         if gn_stats != GN_STATS_CORRECTED:

@@ -54,6 +54,7 @@ struct Layout {
   size_t a1[2], a2[2], h, sc;        // conv inputs (pairs), conv1 output, shortcut output
   size_t act, q, k[2], v[2], o;      // attention buffers
   size_t ha, hb, tn, q2, k2, v2, o2, ffh, ffg;   // TRANSFORMER: residual stream, LN output, cross, FF
+  size_t kv_layer;                    // TRANSFORMER: bytes between layers' k/v ping-pong pairs
   size_t attn_ws;                     // balanced attention split: counters + partials
   size_t tbias;                       // RESBLOCK with a time embedding: conv1's step bias
   size_t gemm_ws;                     // split-K partials of the convs and projections
@@ -129,8 +130,11 @@ Layout layout_of(const dp_block_desc* d) {
     L.hb = b.take(hw * C * e);
     L.tn = b.take(hw * C * e);
     L.q = b.take(hw * C * e);
+    // each layer's self-attention keeps its own stale keys and values
+    L.kv_layer = 4 * ((hw * C * e + 255) & ~static_cast<size_t>(255));
     for (int i = 0; i < 2; ++i) L.k[i] = b.take(hw * C * e);
     for (int i = 0; i < 2; ++i) L.v[i] = b.take(hw * C * e);
+    for (int l = 1; l < d->depth; ++l) b.take(L.kv_layer);
     L.o = b.take(hw * C * e);
     L.q2 = b.take(hw * C * e);
     L.k2 = b.take(Tk * C * e);
@@ -170,6 +174,9 @@ Layout layout_of(const dp_block_desc* d) {
 }
 
 int desc_check(const dp_block_desc* d) {
+  if (d && (d->depth < 1 || d->depth > 16 || (d->depth != 1 && d->kind != DP_BLOCK_TRANSFORMER)))
+    return set_error(DP_ERR_INVALID_ARG, "block: depth %d (1..16, and above 1 only for TRANSFORMER)",
+                     d->depth);
   if (d && d->gn_fuse != 0 && d->gn_fuse != 1)
     return set_error(DP_ERR_INVALID_ARG, "block: gn fusion flag %d is not 0 or 1", d->gn_fuse);
   if (!d) return set_error(DP_ERR_INVALID_ARG, "block: null descriptor");
@@ -232,7 +239,7 @@ int weight_count(const dp_block_desc* d) {
   if (d->kind == DP_BLOCK_GN_CONV) return 4;
   if (d->kind == DP_BLOCK_RESBLOCK) return (d->C != d->Cout ? 10 : 8) + (d->temb_dim > 0 ? 3 : 0);
   if (d->kind == DP_BLOCK_ATTN) return 6;
-  if (d->kind == DP_BLOCK_TRANSFORMER) return 25;
+  if (d->kind == DP_BLOCK_TRANSFORMER) return 7 + 18 * d->depth;
   const MiniDescs m = mini_descs(d);
   return 2 + weight_count(&m.rb1) + 2 + weight_count(&m.rb2) + weight_count(&m.at2) + 2 +
          weight_count(&m.rb3) + weight_count(&m.at3);
@@ -249,10 +256,11 @@ double flops_of(const dp_block_desc* d) {
     return 2.0 * hw * 3.0 * C * C + 4.0 * hw * hw * C + 2.0 * hw * C * C;
   if (d->kind == DP_BLOCK_TRANSFORMER) {
     const double Tk = d->ctx_len, Cc = d->ctx_dim, F = d->ff_inner;
-    return 2.0 * hw * C * C * 5.0 +                       // proj_in, wo, cq, co, proj_out
-           2.0 * hw * 3.0 * C * C + 4.0 * hw * hw * C +   // q/k/v, self-attention
-           2.0 * Tk * 2.0 * C * Cc + 4.0 * hw * Tk * C +  // context k/v, cross-attention
-           2.0 * hw * 2.0 * F * C + 2.0 * hw * C * F;     // ff1, ff2
+    return 2.0 * hw * C * C * 2.0 +                        // proj_in, proj_out
+           d->depth * (2.0 * hw * C * C * 3.0 +             // wo, cq, co
+                       2.0 * hw * 3.0 * C * C + 4.0 * hw * hw * C +   // q/k/v, self-attention
+                       2.0 * Tk * 2.0 * C * Cc + 4.0 * hw * Tk * C +  // context k/v, cross-attention
+                       2.0 * hw * 2.0 * F * C + 2.0 * hw * C * F);    // ff1, ff2
   }
   const MiniDescs m = mini_descs(d);
   return 2.0 * hw * kU1 * 9.0 * C + flops_of(&m.rb1) + 2.0 * (hw / 4) * kU1 * 9.0 * kU1 +
@@ -404,9 +412,12 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
     // biases (conv_b, conv1_b, conv2_b, short_b, temb_b; bqkv, bo, ...) may be NULL
     const int temb_b = weight_count(d) - 2;   // RESBLOCK with a time embedding: temb_b
     for (int i = 0; i < weight_count(d); ++i) {
+      const int tl = (i - 4) % 18;   // TRANSFORMER: index within a layer's 18 pointers
       const bool bias = d->kind == DP_BLOCK_ATTN          ? (i == 3 || i == 5)
-                        : d->kind == DP_BLOCK_TRANSFORMER ? (i == 3 || i == 7 || i == 9 || i == 15 ||
-                                                             i == 19 || i == 21 || i == 23)
+                        : d->kind == DP_BLOCK_TRANSFORMER ? (i == 3 || i == 5 + 18 * d->depth ||
+                                                             (i >= 4 && i < 4 + 18 * d->depth &&
+                                                              (tl == 3 || tl == 5 || tl == 11 || tl == 15 ||
+                                                               tl == 17)))
                                                           : (i == 3 || i == 7 || i == 9 ||
                                                              (d->temb_dim > 0 && i == temb_b));
       if (!w[i] && !bias) return set_error(DP_ERR_INVALID_ARG, "block: weight %d is NULL", i);
@@ -472,8 +483,6 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
     void* hb = at<void>(ws, L.hb);
     void* tn = at<void>(ws, L.tn);
     void* q = at<void>(ws, L.q);
-    void* kf = at<void>(ws, L.k[f]);
-    void* vf = at<void>(ws, L.v[f]);
     void* ob = at<void>(ws, L.o);
     void* q2 = at<void>(ws, L.q2);
     void* k2 = at<void>(ws, L.k2);
@@ -492,51 +501,62 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
     if (rc) return rc;
     rc = lin(act, w[2], w[3], nullptr, ha, nullptr, nullptr, T, C, C, C);   // proj_in
     if (rc) return rc;
-    // self-attention: other bands' keys and values are the previous step's
-    rc = ln(ha, tn, w[4], w[5]);
-    if (rc) return rc;
-    rc = lin(tn, w[6], w[7], nullptr, q, kf, vf, T, 3 * C, C, C);
-    if (rc) return rc;
-    if (plan) {
-      const double keys = mode == DP_MODE_NAIVE ? static_cast<double>(T) / P : T;
-      plan->push(DP_KERNEL_ATTN, 4.0 * T * keys * C, 4.0 * T * C * e);
-    } else {
-      rc = attn_launch(q, kf, vf, at<void>(ws, L.k[o]), at<void>(ws, L.v[o]), ob, T, d->heads, P,
-                       0.125f, mode, at<void>(ws, L.attn_ws), attn_workspace_bytes(), st);
+    const void* ctx = w[6 + 18 * d->depth];
+    void* cur = ha;     // the residual stream entering the layer
+    void* other = hb;
+    for (int l = 0; l < d->depth; ++l) {
+      const void* const* lw = w + 4 + 18 * l;   // this layer's 18 pointers
+      void* kf = at<void>(ws, L.k[f] + l * L.kv_layer);
+      void* vf = at<void>(ws, L.v[f] + l * L.kv_layer);
+      // self-attention: other bands' keys and values are the previous step's
+      rc = ln(cur, tn, lw[0], lw[1]);
       if (rc) return rc;
-    }
-    rc = lin(ob, w[8], w[9], ha, hb, nullptr, nullptr, T, C, C, C);
-    if (rc) return rc;
-    // cross-attention over the step's text context (w[24]): the same for every band
-    rc = ln(hb, tn, w[10], w[11]);
-    if (rc) return rc;
-    rc = lin(tn, w[12], nullptr, nullptr, q2, nullptr, nullptr, T, C, C, C);
-    if (rc) return rc;
-    rc = lin(w[24], w[13], nullptr, nullptr, k2, v2, nullptr, Tk, 2 * C, Cc, C);
-    if (rc) return rc;
-    if (plan) {
-      plan->push(DP_KERNEL_ATTN, 4.0 * T * static_cast<double>(Tk) * C, (2.0 * T * C + 2.0 * Tk * C) * e);
-    } else {
-      rc = attn_launch_tk(q2, k2, v2, nullptr, nullptr, o2, T, Tk, d->heads, 1, 0.125f, DP_MODE_SYNC,
-                          at<void>(ws, L.attn_ws), attn_workspace_bytes(), st);
+      rc = lin(tn, lw[2], lw[3], nullptr, q, kf, vf, T, 3 * C, C, C);
       if (rc) return rc;
-    }
-    rc = lin(o2, w[14], w[15], hb, ha, nullptr, nullptr, T, C, C, C);
-    if (rc) return rc;
-    // gated feed-forward
-    rc = ln(ha, tn, w[16], w[17]);
-    if (rc) return rc;
-    rc = lin(tn, w[18], w[19], nullptr, ffh, nullptr, nullptr, T, 2 * Fi, C, 2 * Fi);
-    if (rc) return rc;
-    if (plan) {
-      plan->push(DP_KERNEL_GEGLU, 0.0, 3.0 * T * Fi * e);
-    } else {
-      rc = dp_geglu(ffh, ffg, T, Fi, st);
+      if (plan) {
+        const double keys = mode == DP_MODE_NAIVE ? static_cast<double>(T) / P : T;
+        plan->push(DP_KERNEL_ATTN, 4.0 * T * keys * C, 4.0 * T * C * e);
+      } else {
+        rc = attn_launch(q, kf, vf, at<void>(ws, L.k[o] + l * L.kv_layer), at<void>(ws, L.v[o] + l * L.kv_layer),
+                         ob, T, d->heads, P, 0.125f, mode, at<void>(ws, L.attn_ws), attn_workspace_bytes(), st);
+        if (rc) return rc;
+      }
+      rc = lin(ob, lw[4], lw[5], cur, other, nullptr, nullptr, T, C, C, C);
       if (rc) return rc;
+      // cross-attention over the step's text context: the same for every band
+      rc = ln(other, tn, lw[6], lw[7]);
+      if (rc) return rc;
+      rc = lin(tn, lw[8], nullptr, nullptr, q2, nullptr, nullptr, T, C, C, C);
+      if (rc) return rc;
+      rc = lin(ctx, lw[9], nullptr, nullptr, k2, v2, nullptr, Tk, 2 * C, Cc, C);
+      if (rc) return rc;
+      if (plan) {
+        plan->push(DP_KERNEL_ATTN, 4.0 * T * static_cast<double>(Tk) * C, (2.0 * T * C + 2.0 * Tk * C) * e);
+      } else {
+        rc = attn_launch_tk(q2, k2, v2, nullptr, nullptr, o2, T, Tk, d->heads, 1, 0.125f, DP_MODE_SYNC,
+                            at<void>(ws, L.attn_ws), attn_workspace_bytes(), st);
+        if (rc) return rc;
+      }
+      rc = lin(o2, lw[10], lw[11], other, cur, nullptr, nullptr, T, C, C, C);
+      if (rc) return rc;
+      // gated feed-forward
+      rc = ln(cur, tn, lw[12], lw[13]);
+      if (rc) return rc;
+      rc = lin(tn, lw[14], lw[15], nullptr, ffh, nullptr, nullptr, T, 2 * Fi, C, 2 * Fi);
+      if (rc) return rc;
+      if (plan) {
+        plan->push(DP_KERNEL_GEGLU, 0.0, 3.0 * T * Fi * e);
+      } else {
+        rc = dp_geglu(ffh, ffg, T, Fi, st);
+        if (rc) return rc;
+      }
+      rc = lin(ffg, lw[16], lw[17], cur, other, nullptr, nullptr, T, C, Fi, C);
+      if (rc) return rc;
+      void* t = cur;   // the layer's output is the next layer's input
+      cur = other;
+      other = t;
     }
-    rc = lin(ffg, w[20], w[21], ha, hb, nullptr, nullptr, T, C, Fi, C);
-    if (rc) return rc;
-    return lin(hb, w[22], w[23], x, out, nullptr, nullptr, T, C, C, C);   // proj_out + x
+    return lin(cur, w[4 + 18 * d->depth], w[5 + 18 * d->depth], x, out, nullptr, nullptr, T, C, C, C);   // proj_out + x
   }
   if (d->kind == DP_BLOCK_ATTN) {
     const int T = H * W;
@@ -655,6 +675,7 @@ int dp_block_desc_init(dp_block_desc* d, int kind, int H, int W, int C, int Cout
   d->ff_inner = 0;
   d->temb_dim = 0;
   d->gn_fuse = 0;
+  d->depth = 1;
   if (kind == DP_BLOCK_TRANSFORMER) return DP_OK;   // checked once dp_block_desc_set_context is called
   return dp::desc_check(d);
 }
@@ -667,6 +688,15 @@ int dp_block_desc_set_context(dp_block_desc* d, int ctx_len, int ctx_dim, int ff
   d->ctx_dim = ctx_dim;
   d->ff_inner = ff_inner;
   return dp::desc_check(d);
+}
+
+int dp_block_desc_set_depth(dp_block_desc* d, int depth) {
+  if (!d) return dp::set_error(DP_ERR_INVALID_ARG, "block: null descriptor");
+  if (d->kind != DP_BLOCK_TRANSFORMER)
+    return dp::set_error(DP_ERR_INVALID_ARG, "block: a depth is only for TRANSFORMER blocks");
+  if (depth < 1 || depth > 16) return dp::set_error(DP_ERR_INVALID_ARG, "block: depth %d outside [1, 16]", depth);
+  d->depth = depth;
+  return DP_OK;
 }
 
 int dp_block_desc_set_time_embedding(dp_block_desc* d, int temb_dim) {

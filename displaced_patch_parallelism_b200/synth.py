@@ -94,6 +94,7 @@ class Workload:
     ctx_len: int = 0          # transformer: text context tokens
     ctx_dim: int = 0          # transformer: text context width
     ff_inner: int = 0         # transformer: feed-forward inner width
+    depth: int = 1            # transformer: basic layers between proj_in and proj_out
 
     @property
     def cout(self) -> int:
@@ -122,10 +123,17 @@ class Workload:
             return unet_mini_weight_specs(self.C)
         if self.kind == "transformer":
             Cc, F = self.ctx_dim, self.ff_inner
-            sq = [(n, (C, C), C ** -0.5) for n in ("proj_in_w", "wq", "wk", "wv", "wo", "cq_w")]
-            return sq + [("ck_w", (C, Cc), Cc ** -0.5), ("cv_w", (C, Cc), Cc ** -0.5),
-                         ("co_w", (C, C), C ** -0.5), ("ff1_w", (2 * F, C), C ** -0.5),
-                         ("ff2_w", (C, F), F ** -0.5), ("proj_out_w", (C, C), C ** -0.5)]
+
+            def layer(pre):
+                sq = [(pre + n, (C, C), C ** -0.5) for n in ("wq", "wk", "wv", "wo", "cq_w")]
+                return sq + [(pre + "ck_w", (C, Cc), Cc ** -0.5), (pre + "cv_w", (C, Cc), Cc ** -0.5),
+                             (pre + "co_w", (C, C), C ** -0.5), (pre + "ff1_w", (2 * F, C), C ** -0.5),
+                             (pre + "ff2_w", (C, F), F ** -0.5)]
+            # layers after the first are drawn after proj_out, so depth 1 draws what it always did
+            s = [("proj_in_w", (C, C), C ** -0.5)] + layer("") + [("proj_out_w", (C, C), C ** -0.5)]
+            for i in range(1, self.depth):
+                s += layer(f"l{i}.")
+            return s
         raise ValueError(self.kind)
 
 
@@ -234,11 +242,17 @@ def affine_specs(wl: Workload) -> List[Tuple[str, int, str]]:
                   (pre + ".bv", c, "bias"), (pre + ".bo", c, "bias")]
         return s
     if wl.kind == "transformer":
-        return [("gn_gamma", C, "gamma"), ("gn_beta", C, "beta"), ("proj_in_b", C, "bias"),
-                ("ln1_g", C, "gamma"), ("ln1_b", C, "beta"), ("bq", C, "bias"), ("bk", C, "bias"),
-                ("bv", C, "bias"), ("bo", C, "bias"), ("ln2_g", C, "gamma"), ("ln2_b", C, "beta"),
-                ("co_b", C, "bias"), ("ln3_g", C, "gamma"), ("ln3_b", C, "beta"),
-                ("ff1_b", 2 * wl.ff_inner, "bias"), ("ff2_b", C, "bias"), ("proj_out_b", C, "bias")]
+        def layer(pre):
+            return [(pre + "ln1_g", C, "gamma"), (pre + "ln1_b", C, "beta"), (pre + "bq", C, "bias"),
+                    (pre + "bk", C, "bias"), (pre + "bv", C, "bias"), (pre + "bo", C, "bias"),
+                    (pre + "ln2_g", C, "gamma"), (pre + "ln2_b", C, "beta"), (pre + "co_b", C, "bias"),
+                    (pre + "ln3_g", C, "gamma"), (pre + "ln3_b", C, "beta"),
+                    (pre + "ff1_b", 2 * wl.ff_inner, "bias"), (pre + "ff2_b", C, "bias")]
+        s = [("gn_gamma", C, "gamma"), ("gn_beta", C, "beta"), ("proj_in_b", C, "bias")]
+        s += layer("") + [("proj_out_b", C, "bias")]
+        for i in range(1, wl.depth):
+            s += layer(f"l{i}.")
+        return s
     raise ValueError(wl.kind)
 
 

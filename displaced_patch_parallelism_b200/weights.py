@@ -23,10 +23,11 @@ def _conv(w, dtype, device):
 
 
 def block_weights(kind: str, wts: Dict, dtype: torch.dtype = torch.bfloat16, device="cuda",
-                  prefix: str = "") -> List[torch.Tensor]:
+                  prefix: str = "", depth: int = 1) -> List[torch.Tensor]:
     """Device tensors in the order ``dp_block_step`` documents for ``kind`` (a TRANSFORMER
-    block's per-step text context, its 25th pointer, and a RESBLOCK's per-step time
-    embedding, its last pointer, are appended by the caller)."""
+    block's per-step text context, its last pointer, and a RESBLOCK's per-step time
+    embedding, its last pointer, are appended by the caller).  ``depth`` is a TRANSFORMER
+    block's number of basic layers; layer l >= 1 has its weights named "l<l>.<name>"."""
     g = lambda n: wts[prefix + n]
     f32 = torch.float32
     if kind == "gn_conv":
@@ -55,12 +56,17 @@ def block_weights(kind: str, wts: Dict, dtype: torch.dtype = torch.bfloat16, dev
         cat = lambda *xs: torch.cat([x if isinstance(x, torch.Tensor) else torch.as_tensor(x) for x in xs])
         v = lambda n: _t(g(n), f32, device)
         m = lambda n: _t(g(n), dtype, device)
-        return [v("gn_gamma"), v("gn_beta"), m("proj_in_w"), v("proj_in_b"), v("ln1_g"), v("ln1_b"),
-                _t(cat(g("wq"), g("wk"), g("wv")), dtype, device),
-                _t(cat(g("bq"), g("bk"), g("bv")), f32, device), m("wo"), v("bo"),
-                v("ln2_g"), v("ln2_b"), m("cq_w"), _t(cat(g("ck_w"), g("cv_w")), dtype, device),
-                m("co_w"), v("co_b"), v("ln3_g"), v("ln3_b"), m("ff1_w"), v("ff1_b"), m("ff2_w"),
-                v("ff2_b"), m("proj_out_w"), v("proj_out_b")]
+        out = [v("gn_gamma"), v("gn_beta"), m("proj_in_w"), v("proj_in_b")]
+        for i in range(depth):
+            p = "" if i == 0 else f"l{i}."     # layer i's weight names
+            out += [v(p + "ln1_g"), v(p + "ln1_b"),
+                    _t(cat(g(p + "wq"), g(p + "wk"), g(p + "wv")), dtype, device),
+                    _t(cat(g(p + "bq"), g(p + "bk"), g(p + "bv")), f32, device), m(p + "wo"), v(p + "bo"),
+                    v(p + "ln2_g"), v(p + "ln2_b"), m(p + "cq_w"),
+                    _t(cat(g(p + "ck_w"), g(p + "cv_w")), dtype, device), m(p + "co_w"), v(p + "co_b"),
+                    v(p + "ln3_g"), v(p + "ln3_b"), m(p + "ff1_w"), v(p + "ff1_b"), m(p + "ff2_w"),
+                    v(p + "ff2_b")]
+        return out + [m("proj_out_w"), v("proj_out_b")]
     if kind == "unet_mini":
         out = [_conv(g("conv_in_w"), dtype, device), _t(g("conv_in_b"), f32, device)]
         out += block_weights("resblock", wts, dtype, device, prefix + "rb1.")

@@ -496,6 +496,7 @@ typedef struct dp_block_desc {
   int ff_inner;   /* TRANSFORMER: feed-forward inner width (F)    */
   int temb_dim;   /* RESBLOCK: time-embedding width (0: none)     */
   int gn_fuse;    /* 1: GroupNorm -> conv through dp_conv3x3_halo_gn */
+  int depth;      /* TRANSFORMER: basic transformer layers (default 1) */
 } dp_block_desc;
 
 /*
@@ -506,6 +507,16 @@ typedef struct dp_block_desc {
  * 0.  DP_ERR_INVALID_ARG on a null descriptor or bad sizes.
  */
 DP_API int dp_block_desc_set_context(dp_block_desc* d, int ctx_len, int ctx_dim, int ff_inner);
+
+/*
+ * TRANSFORMER blocks: the number of basic transformer layers (LN + self-
+ * attention, LN + cross-attention, LN + feed-forward, each with its residual)
+ * between the one GroupNorm / proj_in and the one proj_out (SDXL: 2 at the
+ * 640-channel level, 10 at the 1280-channel level; default 1).  Every layer's
+ * self-attention keeps its own stale keys and values.  1 <= depth <= 16;
+ * DP_ERR_INVALID_ARG otherwise or for another kind.
+ */
+DP_API int dp_block_desc_set_depth(dp_block_desc* d, int depth);
 
 /*
  * RESBLOCK blocks: the width Ct of the step's time embedding (0 switches it
@@ -579,14 +590,15 @@ DP_API int dp_block_state_init(const dp_block_desc* d, dp_block_state* s, void* 
  *   ATTN:     gn_gamma[C], gn_beta[C], wqkv[3C][C] (the q, k and v (out, in)
  *             matrices stacked), bqkv[3C], wo[C][C], bo[C]
  *   TRANSFORMER (C == heads * 64, (H*W/P) % 128 == 0, (H*W) % 256 == 0):
- *             gn_gamma[C], gn_beta[C], proj_in_w[C][C], proj_in_b[C], ln1_g[C],
- *             ln1_b[C], wqkv[3C][C], bqkv[3C], wo[C][C], bo[C], ln2_g[C], ln2_b[C],
- *             cq_w[C][C], ckv_w[2C][Cctx] (the context's k and v matrices
- *             stacked), co_w[C][C], co_b[C], ln3_g[C], ln3_b[C],
- *             ff1_w[2F][C] (value half, then gate half), ff1_b[2F], ff2_w[C][F],
- *             ff2_b[C], proj_out_w[C][C], proj_out_b[C], and the step's context
- *             [ctx_len][ctx_dim] bf16 (25 pointers; matrices bf16, vectors fp32;
- *             the biases may be NULL)
+ *             gn_gamma[C], gn_beta[C], proj_in_w[C][C], proj_in_b[C], then for each
+ *             of the `depth` layers: ln1_g[C], ln1_b[C], wqkv[3C][C], bqkv[3C],
+ *             wo[C][C], bo[C], ln2_g[C], ln2_b[C], cq_w[C][C], ckv_w[2C][Cctx]
+ *             (the context's k and v matrices stacked), co_w[C][C], co_b[C],
+ *             ln3_g[C], ln3_b[C], ff1_w[2F][C] (value half, then gate half),
+ *             ff1_b[2F], ff2_w[C][F], ff2_b[C]; then proj_out_w[C][C],
+ *             proj_out_b[C], and the step's context [ctx_len][ctx_dim] bf16
+ *             (7 + 18 depth pointers; matrices bf16, vectors fp32; the biases may
+ *             be NULL)
  *   UNET_MINI (latent [H][W][C], C even <= 16, H % 4P == 0, W % 4 == 0; output
  *             [H/4][W/4][1280]): conv_in_w[320][3][3][C], conv_in_b[320], the
  *             RESBLOCK list for 320->320 at HxW, down1_w[320][3][3][320],
@@ -642,9 +654,9 @@ DP_API int dp_block_status(const dp_block_desc* d, const dp_block_state* s, void
  *             (each GN and conv a statistics pass and a CONV_GN when fused)
  *   ATTN:     GN, q/k/v projection, attention, out projection
  *   UNET_MINI: input copy, conv_in, then its blocks and downsamplers in order
- *   TRANSFORMER: GN, proj_in, LN, q/k/v projection, attention, out projection,
- *             LN, query projection, context k/v projection, cross-attention,
- *             out projection, LN, ff1, GEGLU, ff2, proj_out
+ *   TRANSFORMER: GN, proj_in, then per layer LN, q/k/v projection, attention,
+ *             out projection, LN, query projection, context k/v projection,
+ *             cross-attention, out projection, LN, ff1, GEGLU, ff2; then proj_out
  * Negative status on a bad descriptor.
  */
 DP_API int dp_block_launch_count(const dp_block_desc* d);

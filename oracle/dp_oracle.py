@@ -564,12 +564,21 @@ def geglu_ff(x: np.ndarray, w1: np.ndarray, b1: np.ndarray, w2: np.ndarray,
     return linear(h[:, :inner] * gelu(h[:, inner:]), w2, b2)
 
 
+def transformer_layer_name(layer: int, name: str) -> str:
+    """Weight name of ``name`` in basic layer ``layer`` of a transformer block: the first
+    layer's weights keep their plain names, layer l >= 1 prefixes them with "l<l>."."""
+    return name if layer == 0 else f"l{layer}.{name}"
+
+
 def transformer_step(state: Dict, x, ctx, wts: Dict, P: int, G: int, eps: float, w: float,
                      heads: int, mode: int, storage: str, trace: Optional[Dict] = None,
                      prefix: str = "", final_storage: Optional[str] = None,
-                     gn_stats: int = GN_STATS_CORRECTED, ln_eps: float = 1e-5):
-    """One SDXL-shaped transformer block (R13).  x: (C, H, W) image; ctx: (Tk, Cctx) text
-    context.  Tokens are pixels in raster order; band p's tokens are its rows."""
+                     gn_stats: int = GN_STATS_CORRECTED, ln_eps: float = 1e-5, depth: int = 1):
+    """One SDXL-shaped transformer block (R13): GroupNorm, proj_in, ``depth`` basic layers
+    (self-attention, cross-attention, gated feed-forward, each with a residual), proj_out
+    and the block's residual.  x: (C, H, W) image; ctx: (Tk, Cctx) text context.  Tokens
+    are pixels in raster order; band p's tokens are its rows.  Each layer's
+    self-attention keeps its own stale keys and values."""
     x = _a(x)
     ctx = _a(ctx)
     C, H, Wd = x.shape
@@ -580,33 +589,40 @@ def transformer_step(state: Dict, x, ctx, wts: Dict, P: int, G: int, eps: float,
     a = store(a, storage)
     h = store(linear(a.reshape(C, H * Wd).T, W_("proj_in_w"), W_("proj_in_b")), storage)
     d = C // heads
-    # self-attention: keys and values of other bands are the previous step's
-    t = store(layer_norm(h, W_("ln1_g"), W_("ln1_b"), ln_eps), storage)
-    q = store(linear(t, W_("wq"), W_("bq")), storage)
-    k = store(linear(t, W_("wk"), W_("bk")), storage)
-    v = store(linear(t, W_("wv"), W_("bv")), storage)
-    o = store(attention_stale_kv(q, k, v, state.get("k_stale"), state.get("v_stale"), P, heads,
-                                 1.0 / math.sqrt(d), mode), storage)
-    h = store(h + linear(o, W_("wo"), W_("bo")), storage)
-    # cross-attention over the text context: the same for every band
-    t = store(layer_norm(h, W_("ln2_g"), W_("ln2_b"), ln_eps), storage)
-    q2 = store(linear(t, W_("cq_w"), None), storage)
-    k2 = store(linear(ctx, W_("ck_w"), None), storage)
-    v2 = store(linear(ctx, W_("cv_w"), None), storage)
-    o2 = store(attention_cross(q2, k2, v2, heads, 1.0 / math.sqrt(d)), storage)
-    h = store(h + linear(o2, W_("co_w"), W_("co_b")), storage)
-    # feed-forward
-    t = store(layer_norm(h, W_("ln3_g"), W_("ln3_b"), ln_eps), storage)
-    hf = store(linear(t, W_("ff1_w"), W_("ff1_b")), storage)     # geglu_ff, stored where the GPU stores
-    inner = hf.shape[1] // 2
-    gf = store(hf[:, :inner] * gelu(hf[:, inner:]), storage)
-    h = store(h + linear(gf, W_("ff2_w"), W_("ff2_b")), storage)
+    fresh_kv = []
+    for layer in range(depth):
+        L = lambda n: W_(transformer_layer_name(layer, n))
+        kv_key = transformer_layer_name(layer, "")
+        # self-attention: keys and values of other bands are the previous step's
+        t = store(layer_norm(h, L("ln1_g"), L("ln1_b"), ln_eps), storage)
+        q = store(linear(t, L("wq"), L("bq")), storage)
+        k = store(linear(t, L("wk"), L("bk")), storage)
+        v = store(linear(t, L("wv"), L("bv")), storage)
+        o = store(attention_stale_kv(q, k, v, state.get(kv_key + "k_stale"),
+                                     state.get(kv_key + "v_stale"), P, heads,
+                                     1.0 / math.sqrt(d), mode), storage)
+        h = store(h + linear(o, L("wo"), L("bo")), storage)
+        # cross-attention over the text context: the same for every band
+        t = store(layer_norm(h, L("ln2_g"), L("ln2_b"), ln_eps), storage)
+        q2 = store(linear(t, L("cq_w"), None), storage)
+        k2 = store(linear(ctx, L("ck_w"), None), storage)
+        v2 = store(linear(ctx, L("cv_w"), None), storage)
+        o2 = store(attention_cross(q2, k2, v2, heads, 1.0 / math.sqrt(d)), storage)
+        h = store(h + linear(o2, L("co_w"), L("co_b")), storage)
+        # feed-forward
+        t = store(layer_norm(h, L("ln3_g"), L("ln3_b"), ln_eps), storage)
+        hf = store(linear(t, L("ff1_w"), L("ff1_b")), storage)   # geglu_ff, stored where the GPU stores
+        inner = hf.shape[1] // 2
+        gf = store(hf[:, :inner] * gelu(hf[:, inner:]), storage)
+        h = store(h + linear(gf, L("ff2_w"), L("ff2_b")), storage)
+        fresh_kv.append((kv_key, k, v))
     out_tok = linear(h, W_("proj_out_w"), W_("proj_out_b")) + x.reshape(C, H * Wd).T
     out = store(out_tok.T.reshape(C, H, Wd), final_storage or storage)
-    if trace is not None:
-        trace[prefix + "k"], trace[prefix + "v"] = k, v
     gn.refresh(f)
-    state["k_stale"], state["v_stale"] = k, v
+    for kv_key, k, v in fresh_kv:
+        if trace is not None:
+            trace[prefix + kv_key + "k"], trace[prefix + kv_key + "v"] = k, v
+        state[kv_key + "k_stale"], state[kv_key + "v_stale"] = k, v
     return out
 
 
@@ -648,9 +664,10 @@ def unet_mini_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: flo
 def block_step(kind: str, state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float,
                mode: int, storage: str, heads: int = 0, silu: bool = True,
                trace: Optional[Dict] = None, final_storage: Optional[str] = None,
-               gn_stats: int = GN_STATS_CORRECTED, ctx=None):
+               gn_stats: int = GN_STATS_CORRECTED, ctx=None, depth: int = 1):
     """Dispatch one block step by kind; x is (C, H, W) (a leading batch of 1 is dropped);
-    ``ctx`` is a transformer block's (Tk, Cctx) text context.
+    ``ctx`` is a transformer block's (Tk, Cctx) text context and ``depth`` its number of
+    basic layers.
 
     ``final_storage`` (default: ``storage``) is the rounding of the block's
     output alone; intermediates always use ``storage``.
@@ -669,7 +686,7 @@ def block_step(kind: str, state: Dict, x, wts: Dict, P: int, G: int, eps: float,
                          final_storage=final_storage, gn_stats=gn_stats)
     if kind == "transformer":
         return transformer_step(state, x, ctx, wts, P, G, eps, w, heads, mode, storage, trace,
-                                final_storage=final_storage, gn_stats=gn_stats)
+                                final_storage=final_storage, gn_stats=gn_stats, depth=depth)
     if kind == "unet_mini":
         return unet_mini_step(state, x, wts, P, G, eps, w, mode, storage, trace, final_storage,
                               gn_stats)

@@ -394,6 +394,56 @@ def test_binding_structs_match_the_header(B, tmp_path):
         assert int(value) == want, (cname, field, int(value), want)
 
 
+def test_transformer_depth_on_the_host(B):
+    """A transformer block of depth 3: 7 + 18 * 3 pointers, the layer launches three times
+    between proj_in and proj_out, flops three layers' worth; a depth is for TRANSFORMER
+    blocks only and lies in [1, 16]."""
+    d = B.dp_block_desc_init(B.TRANSFORMER, 32, 32, 320, 320, 32, 4, 5, B.BF16, 0, 1e-5, 1.0)
+    B.dp_block_desc_set_context(d, 77, 128, 1280)
+    one = B.dp_block_flops(d)
+    ws1 = B.dp_block_workspace_size(d)
+    for bad in (0, 17, -1):
+        with pytest.raises(B.DPError):
+            B.dp_block_desc_set_depth(d, bad)
+    B.dp_block_desc_set_depth(d, 3)
+    assert B.dp_block_weight_count(d) == 7 + 18 * 3
+    kinds = [B.dp_block_launch_info(d, B.DISPLACED, i)[0] for i in range(B.dp_block_launch_count(d))]
+    layer = ["layernorm", "linear", "attn", "linear", "layernorm", "linear", "linear", "attn", "linear",
+             "layernorm", "linear", "geglu", "linear"]
+    assert [k for k in kinds if k != "splitk_finish"] == ["gn_cluster", "linear"] + 3 * layer + ["linear"]
+    T, C = 32 * 32, 320
+    proj = 2 * 2.0 * T * C * C
+    assert abs(B.dp_block_flops(d) - (proj + 3 * (one - proj))) < 1e-9 * one
+    # two more layers' stale key/value ping-pong pairs
+    assert B.dp_block_workspace_size(d) - ws1 >= 2 * 4 * T * C * 2
+    r = B.dp_block_desc_init(B.RESBLOCK, 32, 32, 320, 320, 32, 4, 0, B.BF16, 1, 1e-5, 1.0)
+    with pytest.raises(B.DPError, match="TRANSFORMER"):
+        B.dp_block_desc_set_depth(r, 2)
+    r.depth = 2                                     # written past the setter: rejected at use
+    with pytest.raises(B.DPError, match="depth"):
+        B.dp_block_workspace_size(r)
+
+
+def test_transformer_depth_workload_marshals(B):
+    """Seeded weights of a depth-2 transformer workload marshal into 7 + 18 * 2 pointers (the
+    context last), and its first layer's weights are those of the depth-1 workload."""
+    import dataclasses
+
+    import torch
+
+    from displaced_patch_parallelism_b200 import synth
+    from displaced_patch_parallelism_b200.weights import block_weights
+    wl1 = dataclasses.replace(synth.WORKLOADS["transformer_640x64x64"], C=64, ctx_dim=64, ff_inner=256, heads=1)
+    wl2 = dataclasses.replace(wl1, depth=2)
+    w1 = block_weights("transformer", synth.make_weights(wl1, True), torch.bfloat16, "cpu")
+    w2 = block_weights("transformer", synth.make_weights(wl2, True), torch.bfloat16, "cpu", depth=2)
+    assert len(w2) + 1 == 7 + 18 * 2
+    for a, b in zip(w1[:22], w2[:22]):
+        assert torch.equal(a, b)
+    assert torch.equal(w1[22], w2[40]) and torch.equal(w1[23], w2[41])   # proj_out
+    assert not torch.equal(w2[6], w2[24])                                 # the layers' wqkv differ
+
+
 def test_transformer_workload_marshals_to_the_block(B):
     """The benchmark's SDXL transformer workload: its seeded weights marshal into the 24
     pointers the block documents (the context is the 25th), with the documented shapes."""

@@ -21,9 +21,10 @@ from tests.helpers import (BF16_HALF_ULP, check, check_chain, dev_f32, dev_img, 
 pytestmark = pytest.mark.gpu
 
 
-def _transformer_case():
+def _transformer_case(depth=1):
     """Sizes, weights (matrices storage-rounded to bf16) and text context of a 320-channel
-    transformer block with 5 heads, a 77-token context of width 128 and F = 1280."""
+    transformer block with 5 heads, a 77-token context of width 128, F = 1280 and ``depth``
+    basic layers (layer l >= 1 named "l<l>.<name>")."""
     dims = dict(C=320, H=32, W=32, P=4, G=32, heads=5, Tk=77, Cc=128, F=1280)
     C, Cc, F, Tk = dims["C"], dims["Cc"], dims["F"], dims["Tk"]
     g = torch.Generator().manual_seed(11)
@@ -43,6 +44,17 @@ def _transformer_case():
     for i in (1, 2, 3):
         wts[f"ln{i}_g"], wts[f"ln{i}_b"] = 1 + 0.2 * rnd(C), 0.2 * rnd(C)
     ctx = bf(rnd(Tk, Cc))
+    for layer in range(1, depth):
+        p = f"l{layer}."
+        for n in ("wq", "wk", "wv", "wo", "cq_w", "co_w"):
+            wts[p + n] = bf(rnd(C, C, std=C ** -0.5))
+        wts[p + "ck_w"], wts[p + "cv_w"] = bf(rnd(C, Cc, std=Cc ** -0.5)), bf(rnd(C, Cc, std=Cc ** -0.5))
+        wts[p + "ff1_w"], wts[p + "ff2_w"] = bf(rnd(2 * F, C, std=C ** -0.5)), bf(rnd(C, F, std=F ** -0.5))
+        for n in ("bq", "bk", "bv", "bo", "co_b", "ff2_b"):
+            wts[p + n] = 0.1 * rnd(C)
+        wts[p + "ff1_b"] = 0.1 * rnd(2 * F)
+        for i in (1, 2, 3):
+            wts[f"{p}ln{i}_g"], wts[f"{p}ln{i}_b"] = 1 + 0.2 * rnd(C), 0.2 * rnd(C)
     return dims, wts, ctx, g, rnd, bf
 
 
@@ -73,6 +85,34 @@ def test_transformer_block():
         exact = O.transformer_step(st_exact, xr, c64, w64, P, G, 1e-5, 1.0, heads, mode, "none")
         torch.cuda.synchronize()
         print(check_chain(host_img(out), exact, ref, what=f"transformer step {k} mode {mode}"))
+    assert blk.status() == 0 and B.dp_device_status() == 0
+
+
+def test_transformer_block_depth2():
+    """The same block with two basic layers, each with its own stale keys and values: a sync
+    step and three displaced steps of a drifting input against the oracle, held end to end by
+    check_chain (the chain of bf16-stored stages is twice as long)."""
+    d, wts, ctx, g, rnd, bf = _transformer_case(depth=2)
+    C, H, W, P, G, heads = d["C"], d["H"], d["W"], d["P"], d["G"], d["heads"]
+    dev_w = block_weights("transformer", wts, depth=2) + [ctx.to(torch.bfloat16).cuda()]
+    blk = B.Block(B.TRANSFORMER, H, W, C, C, G, P, heads, B.BF16, False, 1e-5, 1.0,
+                  context=(d["Tk"], d["Cc"], d["F"]), depth=2)
+    assert len(dev_w) == B.dp_block_weight_count(blk.desc)
+    w64 = {n: v.double().numpy() for n, v in wts.items()}
+    c64 = ctx.double().numpy()
+    st, st_exact = {}, {}
+    x = rnd(C, H, W)
+    for k, mode in enumerate([B.SYNC, B.DISPLACED, B.DISPLACED, B.DISPLACED]):
+        if k:
+            x = x + 0.05 * rnd(C, H, W)
+        xr = bf(x).double().numpy()
+        out = torch.empty(H, W, C, dtype=torch.bfloat16, device="cuda")
+        blk.step(dev_img(xr, "bf16"), out, dev_w, mode)
+        ref = O.transformer_step(st, xr, c64, w64, P, G, 1e-5, 1.0, heads, mode, "bf16",
+                                 final_storage="none", depth=2)
+        exact = O.transformer_step(st_exact, xr, c64, w64, P, G, 1e-5, 1.0, heads, mode, "none", depth=2)
+        torch.cuda.synchronize()
+        print(check_chain(host_img(out), exact, ref, what=f"depth-2 transformer step {k} mode {mode}"))
     assert blk.status() == 0 and B.dp_device_status() == 0
 
 

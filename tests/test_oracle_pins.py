@@ -668,46 +668,51 @@ def test_cross_attention_equals_library_and_brute_force(Tq, Tk, heads):
 
 
 # ---------------------------------------------------------------- SDXL-shaped transformer block
-def rand_transformer_weights(r, C, Cctx, heads, mult=2):
+def rand_transformer_weights(r, C, Cctx, heads, mult=2, depth=1):
     s = lambda *shape: r.standard_normal(shape) * (1.0 / math.sqrt(shape[-1]))
     w = {"gn_gamma": 1 + 0.3 * r.standard_normal(C), "gn_beta": 0.3 * r.standard_normal(C),
          "proj_in_w": s(C, C), "proj_in_b": 0.3 * r.standard_normal(C),
          "proj_out_w": s(C, C), "proj_out_b": 0.3 * r.standard_normal(C)}
-    for i in (1, 2, 3):
-        w[f"ln{i}_g"], w[f"ln{i}_b"] = 1 + 0.3 * r.standard_normal(C), 0.3 * r.standard_normal(C)
-    for n in ("wq", "wk", "wv", "wo"):
-        w[n] = s(C, C)
-    for n in ("bq", "bk", "bv", "bo", "co_b"):
-        w[n] = 0.3 * r.standard_normal(C)
-    w["cq_w"], w["co_w"] = s(C, C), s(C, C)
-    w["ck_w"], w["cv_w"] = s(C, Cctx), s(C, Cctx)
-    w["ff1_w"], w["ff1_b"] = s(2 * mult * C, C), 0.3 * r.standard_normal(2 * mult * C)
-    w["ff2_w"], w["ff2_b"] = s(C, mult * C), 0.3 * r.standard_normal(C)
+    for layer in range(depth):
+        p = "" if layer == 0 else f"l{layer}."
+        for i in (1, 2, 3):
+            w[f"{p}ln{i}_g"], w[f"{p}ln{i}_b"] = 1 + 0.3 * r.standard_normal(C), 0.3 * r.standard_normal(C)
+        for n in ("wq", "wk", "wv", "wo"):
+            w[p + n] = s(C, C)
+        for n in ("bq", "bk", "bv", "bo", "co_b"):
+            w[p + n] = 0.3 * r.standard_normal(C)
+        w[p + "cq_w"], w[p + "co_w"] = s(C, C), s(C, C)
+        w[p + "ck_w"], w[p + "cv_w"] = s(C, Cctx), s(C, Cctx)
+        w[p + "ff1_w"], w[p + "ff1_b"] = s(2 * mult * C, C), 0.3 * r.standard_normal(2 * mult * C)
+        w[p + "ff2_w"], w[p + "ff2_b"] = s(C, mult * C), 0.3 * r.standard_normal(C)
     return w
 
 
-def lib_transformer(x, ctx, w, G, eps, heads):
-    """The same block composed from library operators, on the whole image."""
-    g = lambda n: T64(w[n])
+def lib_transformer(x, ctx, w, G, eps, heads, depth=1):
+    """The same block composed from library operators, on the whole image: ``depth`` basic
+    layers (the first named plainly, layer l >= 1 with an "l<l>." prefix)."""
     C, H, W = x.shape
     d = C // heads
     sh = lambda z: z.reshape(z.shape[0], heads, d).permute(1, 0, 2)
     un = lambda z: z.permute(1, 0, 2).reshape(-1, C)
-    a = F.group_norm(T64(x)[None], G, g("gn_gamma"), g("gn_beta"), eps)[0].reshape(C, H * W).T
-    h = F.linear(a, g("proj_in_w"), g("proj_in_b"))
-    t = F.layer_norm(h, (C,), g("ln1_g"), g("ln1_b"), 1e-5)
-    o = F.scaled_dot_product_attention(sh(F.linear(t, g("wq"), g("bq"))), sh(F.linear(t, g("wk"), g("bk"))),
-                                       sh(F.linear(t, g("wv"), g("bv"))))
-    h = h + F.linear(un(o), g("wo"), g("bo"))
-    t = F.layer_norm(h, (C,), g("ln2_g"), g("ln2_b"), 1e-5)
+    g0 = lambda n: T64(w[n])
+    a = F.group_norm(T64(x)[None], G, g0("gn_gamma"), g0("gn_beta"), eps)[0].reshape(C, H * W).T
+    h = F.linear(a, g0("proj_in_w"), g0("proj_in_b"))
     c = T64(ctx)
-    o = F.scaled_dot_product_attention(sh(F.linear(t, g("cq_w"))), sh(F.linear(c, g("ck_w"))),
-                                       sh(F.linear(c, g("cv_w"))))
-    h = h + F.linear(un(o), g("co_w"), g("co_b"))
-    t = F.layer_norm(h, (C,), g("ln3_g"), g("ln3_b"), 1e-5)
-    a2, gate = F.linear(t, g("ff1_w"), g("ff1_b")).chunk(2, dim=-1)
-    h = h + F.linear(a2 * F.gelu(gate), g("ff2_w"), g("ff2_b"))
-    out = F.linear(h, g("proj_out_w"), g("proj_out_b")) + T64(x).reshape(C, H * W).T
+    for layer in range(depth):
+        g = lambda n: T64(w[n if layer == 0 else f"l{layer}.{n}"])
+        t = F.layer_norm(h, (C,), g("ln1_g"), g("ln1_b"), 1e-5)
+        o = F.scaled_dot_product_attention(sh(F.linear(t, g("wq"), g("bq"))), sh(F.linear(t, g("wk"), g("bk"))),
+                                           sh(F.linear(t, g("wv"), g("bv"))))
+        h = h + F.linear(un(o), g("wo"), g("bo"))
+        t = F.layer_norm(h, (C,), g("ln2_g"), g("ln2_b"), 1e-5)
+        o = F.scaled_dot_product_attention(sh(F.linear(t, g("cq_w"))), sh(F.linear(c, g("ck_w"))),
+                                           sh(F.linear(c, g("cv_w"))))
+        h = h + F.linear(un(o), g("co_w"), g("co_b"))
+        t = F.layer_norm(h, (C,), g("ln3_g"), g("ln3_b"), 1e-5)
+        a2, gate = F.linear(t, g("ff1_w"), g("ff1_b")).chunk(2, dim=-1)
+        h = h + F.linear(a2 * F.gelu(gate), g("ff2_w"), g("ff2_b"))
+    out = F.linear(h, g0("proj_out_w"), g0("proj_out_b")) + T64(x).reshape(C, H * W).T
     return out.T.reshape(C, H, W).numpy()
 
 
@@ -735,6 +740,56 @@ def test_p1_transformer_equals_library(mode):
     O.transformer_step(st, x, ctx, w, 1, G, 1e-5, 1.0, heads, SYNC, "none")
     y = O.transformer_step(st, x, ctx, w, 1, G, 1e-5, 1.0, heads, mode, "none")
     np.testing.assert_allclose(y, lib_transformer(x, ctx, w, G, 1e-5, heads), rtol=0, atol=1e-11)
+
+
+@pytest.mark.parametrize("mode", [SYNC, DISPLACED, NAIVE])
+def test_p1_transformer_depth3_equals_library(mode):
+    """Three basic layers at one band equal the library's composition of three layers, and
+    neither one nor two layers of the same weights give that result (so every layer runs,
+    each with its own weights)."""
+    r = rng(93)
+    C, H, W, G, heads, Cctx, Tk = 8, 4, 6, 4, 2, 6, 5
+    w = rand_transformer_weights(r, C, Cctx, heads, depth=3)
+    x, ctx = r.standard_normal((C, H, W)), r.standard_normal((Tk, Cctx))
+    st = {}
+    O.transformer_step(st, x, ctx, w, 1, G, 1e-5, 1.0, heads, SYNC, "none", depth=3)
+    y = O.transformer_step(st, x, ctx, w, 1, G, 1e-5, 1.0, heads, mode, "none", depth=3)
+    np.testing.assert_allclose(y, lib_transformer(x, ctx, w, G, 1e-5, heads, depth=3), rtol=0, atol=1e-11)
+    for fewer in (1, 2):
+        assert np.abs(y - lib_transformer(x, ctx, w, G, 1e-5, heads, depth=fewer)).max() > 1e-3
+
+
+def test_transformer_depth2_keeps_each_layers_stale_keys():
+    """Two layers over four bands: with an unchanged input a displaced step equals a sync step
+    (each layer's stale keys and values are its own, from the step before), the state holds
+    one stale pair per layer, and band locality holds through both layers."""
+    r = rng(96)
+    C, H, W, P, G, heads, Cctx, Tk = 8, 8, 4, 4, 4, 2, 6, 5
+    w = rand_transformer_weights(r, C, Cctx, heads, depth=2)
+    x0, ctx = r.standard_normal((C, H, W)), r.standard_normal((Tk, Cctx))
+    st = {}
+    ys = O.transformer_step(st, x0, ctx, w, P, G, 1e-5, 1.0, heads, SYNC, "none", depth=2)
+    assert {"k_stale", "v_stale", "l1.k_stale", "l1.v_stale"} <= set(st)
+    assert not np.allclose(st["k_stale"], st["l1.k_stale"])
+    yd = O.transformer_step(st, x0, ctx, w, P, G, 1e-5, 1.0, heads, DISPLACED, "none", depth=2)
+    np.testing.assert_allclose(yd, ys, rtol=0, atol=1e-11)
+    # a displaced step that took layer 0's stale pair for layer 1 would not equal sync
+    bad = dict(st)
+    bad["l1.k_stale"], bad["l1.v_stale"] = st["k_stale"], st["v_stale"]
+    yb = O.transformer_step(bad, x0, ctx, w, P, G, 1e-5, 1.0, heads, DISPLACED, "none", depth=2)
+    assert np.abs(yb - ys).max() > 1e-3
+    x1 = x0 + 0.3 * r.standard_normal(x0.shape)
+    hb, q = H // P, 1
+    x1b = x1.copy()
+    x1b[:, q * hb:(q + 1) * hb, :] += r.standard_normal((C, hb, W))
+    outs = []
+    for xin in (x1, x1b):
+        s2 = {}
+        O.transformer_step(s2, x0, ctx, w, P, G, 1e-5, 1.0, heads, SYNC, "none", depth=2)
+        outs.append(O.transformer_step(s2, xin, ctx, w, P, G, 1e-5, 1.0, heads, DISPLACED, "none", depth=2))
+    for p in range(P):
+        rows = slice(p * hb, (p + 1) * hb)
+        assert np.array_equal(outs[0][:, rows, :], outs[1][:, rows, :]) == (p != q), p
 
 
 def test_transformer_displaced_band_locality():
