@@ -72,7 +72,7 @@ class Workload:
     """One synthetic workload: a block kind, its shapes and its seeds."""
 
     name: str
-    kind: str                 # "gn_conv" | "resblock" | "attn" | "unet_mini"
+    kind: str                 # "gn_conv" | "resblock" | "attn" | "transformer" | "unet_mini" | "unet_sdxl"
     C: int                    # channels of the block input
     H: int
     W: int
@@ -95,6 +95,9 @@ class Workload:
     ctx_dim: int = 0          # transformer: text context width
     ff_inner: int = 0         # transformer: feed-forward inner width
     depth: int = 1            # transformer: basic layers between proj_in and proj_out
+    base: int = 320           # unet_sdxl: level widths base, 2 base, 4 base
+    depths: Tuple[int, int, int] = (0, 2, 10)   # unet_sdxl: transformer depth of each level
+    temb_dim: int = 0         # unet_sdxl: time-embedding width
 
     @property
     def cout(self) -> int:
@@ -122,19 +125,106 @@ class Workload:
         if self.kind == "unet_mini":
             return unet_mini_weight_specs(self.C)
         if self.kind == "transformer":
-            Cc, F = self.ctx_dim, self.ff_inner
-
-            def layer(pre):
-                sq = [(pre + n, (C, C), C ** -0.5) for n in ("wq", "wk", "wv", "wo", "cq_w")]
-                return sq + [(pre + "ck_w", (C, Cc), Cc ** -0.5), (pre + "cv_w", (C, Cc), Cc ** -0.5),
-                             (pre + "co_w", (C, C), C ** -0.5), (pre + "ff1_w", (2 * F, C), C ** -0.5),
-                             (pre + "ff2_w", (C, F), F ** -0.5)]
-            # layers after the first are drawn after proj_out, so depth 1 draws what it always did
-            s = [("proj_in_w", (C, C), C ** -0.5)] + layer("") + [("proj_out_w", (C, C), C ** -0.5)]
-            for i in range(1, self.depth):
-                s += layer(f"l{i}.")
-            return s
+            return transformer_weight_specs("", C, self.ctx_dim, self.ff_inner, self.depth)
+        if self.kind == "unet_sdxl":
+            return sdxl_unet_specs(self)[0]
         raise ValueError(self.kind)
+
+
+def transformer_weight_specs(pre: str, C: int, Cc: int, F: int,
+                             depth: int) -> List[Tuple[str, Tuple[int, ...], float]]:
+    """Matrices of a transformer block (names prefixed by ``pre``), in draw order; layers
+    after the first are drawn after proj_out, so depth 1 draws what it always did."""
+    def layer(lp):
+        sq = [(lp + n, (C, C), C ** -0.5) for n in ("wq", "wk", "wv", "wo", "cq_w")]
+        return sq + [(lp + "ck_w", (C, Cc), Cc ** -0.5), (lp + "cv_w", (C, Cc), Cc ** -0.5),
+                     (lp + "co_w", (C, C), C ** -0.5), (lp + "ff1_w", (2 * F, C), C ** -0.5),
+                     (lp + "ff2_w", (C, F), F ** -0.5)]
+    s = [(pre + "proj_in_w", (C, C), C ** -0.5)] + layer(pre) + [(pre + "proj_out_w", (C, C), C ** -0.5)]
+    for i in range(1, depth):
+        s += layer(f"{pre}l{i}.")
+    return s
+
+
+def transformer_affine_specs(pre: str, C: int, F: int, depth: int) -> List[Tuple[str, int, str]]:
+    def layer(lp):
+        return [(lp + "ln1_g", C, "gamma"), (lp + "ln1_b", C, "beta"), (lp + "bq", C, "bias"),
+                (lp + "bk", C, "bias"), (lp + "bv", C, "bias"), (lp + "bo", C, "bias"),
+                (lp + "ln2_g", C, "gamma"), (lp + "ln2_b", C, "beta"), (lp + "co_b", C, "bias"),
+                (lp + "ln3_g", C, "gamma"), (lp + "ln3_b", C, "beta"),
+                (lp + "ff1_b", 2 * F, "bias"), (lp + "ff2_b", C, "bias")]
+    s = [(pre + "gn_gamma", C, "gamma"), (pre + "gn_beta", C, "beta"), (pre + "proj_in_b", C, "bias")]
+    s += layer(pre) + [(pre + "proj_out_b", C, "bias")]
+    for i in range(1, depth):
+        s += layer(f"{pre}l{i}.")
+    return s
+
+
+def sdxl_unet_stages(base: int, depths) -> List[Tuple[str, str, int, int]]:
+    """The SDXL-shaped U-Net's stages in execution order: (kind, weight prefix, input channels,
+    output channels), kind one of "conv_in", "resblock", "transformer", "down", "up", "out".
+    Names only: the weight names a caller draws and marshals (the latent's channel count is
+    filled in as 0 here)."""
+    ch = (base, 2 * base, 4 * base)
+    s = [("conv_in", "conv_in", 0, ch[0])]
+    skips = [ch[0]]
+    c = ch[0]
+    for lvl in range(3):
+        for i in range(2):
+            s.append(("resblock", f"d{lvl}.r{i}.", c, ch[lvl]))
+            c = ch[lvl]
+            if depths[lvl]:
+                s.append(("transformer", f"d{lvl}.t{i}.", c, c))
+            skips.append(c)
+        if lvl < 2:
+            s.append(("down", f"d{lvl}.down", c, c))
+            skips.append(c)
+    s += [("resblock", "mid.r0.", c, c), ("transformer", "mid.t.", c, c), ("resblock", "mid.r1.", c, c)]
+    for lvl in (2, 1, 0):
+        for i in range(3):
+            s.append(("resblock", f"u{lvl}.r{i}.", c + skips.pop(), ch[lvl]))
+            c = ch[lvl]
+            if depths[lvl]:
+                s.append(("transformer", f"u{lvl}.t{i}.", c, c))
+        if lvl > 0:
+            s.append(("up", f"u{lvl}.up", c, c))
+    s.append(("out", "out.", c, 0))
+    return s
+
+
+def sdxl_unet_specs(wl: "Workload"):
+    """(matrix specs, affine specs) of an SDXL-shaped U-Net workload, in draw order."""
+    mats: List[Tuple[str, Tuple[int, ...], float]] = []
+    aff: List[Tuple[str, int, str]] = []
+    depth_of = {"d0": wl.depths[0], "d1": wl.depths[1], "d2": wl.depths[2], "mid": wl.depths[2],
+                "u2": wl.depths[2], "u1": wl.depths[1], "u0": wl.depths[0]}
+    conv = lambda name, co, ci: (name, (co, ci, 3, 3), math.sqrt(2.0 / (ci * 9)))
+    for kind, pre, ci, co in sdxl_unet_stages(wl.base, wl.depths):
+        if kind == "conv_in":
+            mats.append(conv("conv_in_w", co, wl.C))
+            aff.append(("conv_in_b", co, "bias"))
+        elif kind in ("down", "up"):
+            mats.append(conv(pre + "_w", co, ci))
+            aff.append((pre + "_b", co, "bias"))
+        elif kind == "resblock":
+            mats += [conv(pre + "conv1_w", co, ci), conv(pre + "conv2_w", co, co)]
+            if ci != co:
+                mats.append((pre + "short_w", (co, ci, 1, 1), math.sqrt(2.0 / ci)))
+            mats.append((pre + "temb_w", (co, wl.temb_dim), wl.temb_dim ** -0.5))
+            aff += [(pre + "gn1_gamma", ci, "gamma"), (pre + "gn1_beta", ci, "beta"),
+                    (pre + "conv1_b", co, "bias"), (pre + "gn2_gamma", co, "gamma"),
+                    (pre + "gn2_beta", co, "beta"), (pre + "conv2_b", co, "bias")]
+            if ci != co:
+                aff.append((pre + "short_b", co, "bias"))
+            aff.append((pre + "temb_b", co, "bias"))
+        elif kind == "transformer":
+            depth = depth_of[pre.split(".")[0]]
+            mats += transformer_weight_specs(pre, ci, wl.ctx_dim, 4 * ci, depth)
+            aff += transformer_affine_specs(pre, ci, 4 * ci, depth)
+        else:   # out: GroupNorm + SiLU + conv_out back to the latent's channels
+            mats.append(conv("out.conv_w", wl.C, ci))
+            aff += [("out.gn_gamma", ci, "gamma"), ("out.gn_beta", ci, "beta"), ("out.conv_b", wl.C, "bias")]
+    return mats, aff
 
 
 def unet_mini_weight_specs(cin: int) -> List[Tuple[str, Tuple[int, ...], float]]:
@@ -242,17 +332,9 @@ def affine_specs(wl: Workload) -> List[Tuple[str, int, str]]:
                   (pre + ".bv", c, "bias"), (pre + ".bo", c, "bias")]
         return s
     if wl.kind == "transformer":
-        def layer(pre):
-            return [(pre + "ln1_g", C, "gamma"), (pre + "ln1_b", C, "beta"), (pre + "bq", C, "bias"),
-                    (pre + "bk", C, "bias"), (pre + "bv", C, "bias"), (pre + "bo", C, "bias"),
-                    (pre + "ln2_g", C, "gamma"), (pre + "ln2_b", C, "beta"), (pre + "co_b", C, "bias"),
-                    (pre + "ln3_g", C, "gamma"), (pre + "ln3_b", C, "beta"),
-                    (pre + "ff1_b", 2 * wl.ff_inner, "bias"), (pre + "ff2_b", C, "bias")]
-        s = [("gn_gamma", C, "gamma"), ("gn_beta", C, "beta"), ("proj_in_b", C, "bias")]
-        s += layer("") + [("proj_out_b", C, "bias")]
-        for i in range(1, wl.depth):
-            s += layer(f"l{i}.")
-        return s
+        return transformer_affine_specs("", C, wl.ff_inner, wl.depth)
+    if wl.kind == "unet_sdxl":
+        return sdxl_unet_specs(wl)[1]
     raise ValueError(wl.kind)
 
 

@@ -396,18 +396,19 @@ def _a(x) -> np.ndarray:
 
 def gn_conv_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float,
                  silu: bool, mode: int, storage: str, trace: Optional[Dict] = None,
-                 final_storage: Optional[str] = None, gn_stats: int = GN_STATS_CORRECTED):
+                 final_storage: Optional[str] = None, gn_stats: int = GN_STATS_CORRECTED,
+                 prefix: str = ""):
     """GroupNorm (+SiLU) -> 3x3 conv with stale halo.  x: (C, H, W)."""
     x = _a(x)
     gn = state.setdefault("gn", GNState())
-    a, f = _gn(gn, x, _a(wts["gn_gamma"]), _a(wts["gn_beta"]), P, G, eps, w, silu, mode,
-               trace, "gn", gn_stats)
+    a, f = _gn(gn, x, _a(wts[prefix + "gn_gamma"]), _a(wts[prefix + "gn_beta"]), P, G, eps, w, silu,
+               mode, trace, prefix + "gn", gn_stats)
     a = store(a, storage)
-    out = conv3x3_halo(a, state.get("a_stale"), _a(wts["conv_w"]), _a(wts["conv_b"]), None,
-                       P, mode)
+    out = conv3x3_halo(a, state.get("a_stale"), _a(wts[prefix + "conv_w"]), _a(wts[prefix + "conv_b"]),
+                       None, P, mode)
     out = store(out, final_storage or storage)
     if trace is not None:
-        trace["a"] = a
+        trace[prefix + "a"] = a
     gn.refresh(f)
     state["a_stale"] = a
     return out
@@ -659,6 +660,89 @@ def unet_mini_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: flo
     h = attn_step(sub("at3"), h, wts, P, G, eps, w, 20, mode, storage, trace, "at3.",
                   final_storage, gn_stats=gn_stats)
     return h
+
+
+# ---------------------------------------------------------------- SDXL-shaped U-Net step
+# Reading R18: the whole denoising network of the pages' SDXL experiments
+# ("DistriFusion", atlas.scime.ai summary, Key results: SDXL at 1024 px and
+# above), shaped as SDXL's U-Net: conv_in; three down levels of two ResBlocks
+# (level widths base, 2 base, 4 base), the ResBlocks of levels with a nonzero
+# transformer depth each followed by a transformer block of that depth, levels
+# 0 and 1 ending in a stride-2 conv; a middle ResBlock -> transformer ->
+# ResBlock; three up levels of three ResBlocks, each taking the channel
+# concatenation [h, skip] of the running tensor and the latest unused skip
+# (the outputs of conv_in, of every down ResBlock/transformer pair and of the
+# down convs), levels 2 and 1 ending in a nearest-neighbour 2x upsample and a
+# 3x3 conv; then GroupNorm -> SiLU -> conv_out to the latent's channels.
+# Every ResBlock adds the step's time embedding term.  Every 3x3 conv (conv_in,
+# down, up and conv_out included) takes its halo rows from the previous step's
+# copy of its own input; upsampling and concatenation act on each pixel's rows
+# within its band, so they need no context.
+
+def upsample_nearest2x(x) -> np.ndarray:
+    """Nearest-neighbour 2x upsampling of (C, H, W): out[:, i, j] = x[:, i // 2, j // 2]."""
+    x = _a(x)
+    return np.repeat(np.repeat(x, 2, axis=1), 2, axis=2)
+
+
+def concat_channels(a, b) -> np.ndarray:
+    """Channel concatenation [a, b] of (Ca, H, W) and (Cb, H, W)."""
+    return np.concatenate([_a(a), _a(b)], axis=0)
+
+
+def sdxl_unet_step(state: Dict, x, ctx, temb, wts: Dict, P: int, G: int, eps: float, w: float,
+                   mode: int, storage: str, base: int = 320, depths=(0, 2, 10), head_dim: int = 64,
+                   ff_mult: int = 4, trace: Optional[Dict] = None, final_storage: Optional[str] = None,
+                   gn_stats: int = GN_STATS_CORRECTED) -> np.ndarray:
+    """One step of the SDXL-shaped U-Net (R18).  x: (Cl, H, W) latent; ctx: (Tk, Cctx) text
+    context; temb: (Ct,) the step's time embedding.  Weight names: conv_in_*; d<l>.r<i>. and
+    d<l>.t<i>. (down ResBlock / transformer i of level l), d<l>.down_*; mid.r0., mid.t.,
+    mid.r1.; u<l>.r<i>., u<l>.t<i>., u<l>.up_*; out. (GroupNorm + conv_out).  Transformers
+    have C / head_dim heads and a feed-forward inner width ff_mult * C."""
+    x = _a(x)
+    A = lambda n: _a(wts[n])
+    sub = lambda n: state.setdefault(n, {})
+    chans = (base, 2 * base, 4 * base)
+
+    def conv_layer(name, inp, stride):
+        st = sub(name)
+        y = conv3x3_halo(inp, st.get("a_stale"), A(name + "_w"), A(name + "_b"), None, P, mode, stride)
+        st["a_stale"] = inp
+        return store(y, storage)
+
+    def resblock(pre, h):
+        return resblock_step(sub(pre), h, wts, P, G, eps, w, mode, storage, trace, pre,
+                             gn_stats=gn_stats, temb=temb)
+
+    def transformer(pre, h, depth):
+        c = h.shape[0]
+        return transformer_step(sub(pre), h, ctx, wts, P, G, eps, w, c // head_dim, mode, storage,
+                                trace, pre, gn_stats=gn_stats, depth=depth)
+
+    h = conv_layer("conv_in", x, 1)
+    skips = [h]
+    for lvl in range(3):
+        for i in range(2):
+            h = resblock(f"d{lvl}.r{i}.", h)
+            if depths[lvl]:
+                h = transformer(f"d{lvl}.t{i}.", h, depths[lvl])
+            skips.append(h)
+        if lvl < 2:
+            h = conv_layer(f"d{lvl}.down", h, 2)
+            skips.append(h)
+    h = resblock("mid.r0.", h)
+    h = transformer("mid.t.", h, depths[2])
+    h = resblock("mid.r1.", h)
+    for lvl in (2, 1, 0):
+        for i in range(3):
+            h = resblock(f"u{lvl}.r{i}.", concat_channels(h, skips.pop()))
+            if depths[lvl]:
+                h = transformer(f"u{lvl}.t{i}.", h, depths[lvl])
+        if lvl > 0:
+            h = conv_layer(f"u{lvl}.up", upsample_nearest2x(h), 1)
+    assert not skips
+    return gn_conv_step(sub("out."), h, wts, P, G, eps, w, True, mode, storage, trace,
+                        final_storage, gn_stats, prefix="out.")
 
 
 def block_step(kind: str, state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: float,

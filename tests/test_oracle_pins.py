@@ -73,10 +73,12 @@ def lib_gn_conv(x, w, G, eps, silu=True):
     return F.conv2d(t, T64(w["conv_w"]), T64(w["conv_b"]), padding=1)[0].numpy()
 
 
-def lib_resblock(x, w, G, eps, prefix=""):
+def lib_resblock(x, w, G, eps, prefix="", temb=None):
     g = lambda n: T64(w[prefix + n])
     t = F.silu(F.group_norm(T64(x)[None], G, g("gn1_gamma"), g("gn1_beta"), eps))
     h = F.conv2d(t, g("conv1_w"), g("conv1_b"), padding=1)
+    if temb is not None:
+        h = h + F.linear(F.silu(T64(temb)), g("temb_w"), g("temb_b"))[None, :, None, None]
     t = F.silu(F.group_norm(h, G, g("gn2_gamma"), g("gn2_beta"), eps))
     res = T64(x)[None]
     if prefix + "short_w" in w:
@@ -688,19 +690,19 @@ def rand_transformer_weights(r, C, Cctx, heads, mult=2, depth=1):
     return w
 
 
-def lib_transformer(x, ctx, w, G, eps, heads, depth=1):
+def lib_transformer(x, ctx, w, G, eps, heads, depth=1, prefix=""):
     """The same block composed from library operators, on the whole image: ``depth`` basic
     layers (the first named plainly, layer l >= 1 with an "l<l>." prefix)."""
     C, H, W = x.shape
     d = C // heads
     sh = lambda z: z.reshape(z.shape[0], heads, d).permute(1, 0, 2)
     un = lambda z: z.permute(1, 0, 2).reshape(-1, C)
-    g0 = lambda n: T64(w[n])
+    g0 = lambda n: T64(w[prefix + n])
     a = F.group_norm(T64(x)[None], G, g0("gn_gamma"), g0("gn_beta"), eps)[0].reshape(C, H * W).T
     h = F.linear(a, g0("proj_in_w"), g0("proj_in_b"))
     c = T64(ctx)
     for layer in range(depth):
-        g = lambda n: T64(w[n if layer == 0 else f"l{layer}.{n}"])
+        g = lambda n: T64(w[prefix + (n if layer == 0 else f"l{layer}.{n}")])
         t = F.layer_norm(h, (C,), g("ln1_g"), g("ln1_b"), 1e-5)
         o = F.scaled_dot_product_attention(sh(F.linear(t, g("wq"), g("bq"))), sh(F.linear(t, g("wk"), g("bk"))),
                                            sh(F.linear(t, g("wv"), g("bv"))))
@@ -973,3 +975,146 @@ def test_dpm_solver_convergence_order():
     for a, b in zip(e2, e2[1:]):
         assert 3.5 < a / b < 4.5, e2
     assert e2[-1] < e1[-1] / 5      # and more accurate at the same step count
+
+
+# ---------------------------------------------------------------- SDXL-shaped U-Net step
+UNET_TINY = dict(Cl=4, base=8, depths=(0, 1, 2), head_dim=4, G=4, Tk=3, Cc=8, Ct=6)
+
+
+def _sdxl_unet_case(seed, H, W, P, depths=UNET_TINY["depths"]):
+    """Weights drawn from the workload's own names and shapes (random affine parameters and
+    biases, so that no term hides behind a zero), a text context and a time embedding."""
+    from displaced_patch_parallelism_b200 import synth
+    t = UNET_TINY
+    wl = synth.Workload(name="tiny_unet", kind="unet_sdxl", C=t["Cl"], H=H, W=W, P=P, G=t["G"],
+                        base=t["base"], depths=depths, ctx_len=t["Tk"], ctx_dim=t["Cc"],
+                        temb_dim=t["Ct"])
+    r = rng(seed)
+    mats, aff = synth.sdxl_unet_specs(wl)
+    w = {n: r.standard_normal(shape) * std for n, shape, std in mats}
+    for n, c, kind in aff:
+        w[n] = (1 + 0.2 * r.standard_normal(c)) if kind == "gamma" else 0.2 * r.standard_normal(c)
+    return w, r.standard_normal((t["Tk"], t["Cc"])), r.standard_normal(t["Ct"])
+
+
+def lib_sdxl_unet(x, ctx, temb, w, depths=UNET_TINY["depths"], skip_first=False):
+    """The SDXL-shaped U-Net composed from library operators on the whole image: conv2d
+    (stride 1 and 2, padding 1), nearest interpolation, channel concatenation, the library
+    ResBlock with its time-embedding term and the library transformer block.
+    ``skip_first`` concatenates [skip, h] instead of [h, skip] (a plausible slip)."""
+    t = UNET_TINY
+    G, eps, hd = t["G"], 1e-5, t["head_dim"]
+    conv = lambda z, n, s: F.conv2d(T64(z)[None], T64(w[n + "_w"]), T64(w[n + "_b"]), stride=s,
+                                    padding=1)[0].numpy()
+    res = lambda z, pre: lib_resblock(z, w, G, eps, pre, temb)
+    tf = lambda z, pre, dp: lib_transformer(z, ctx, w, G, eps, z.shape[0] // hd, dp, pre)
+    h = conv(x, "conv_in", 1)
+    skips = [h]
+    for lvl in range(3):
+        for i in range(2):
+            h = res(h, f"d{lvl}.r{i}.")
+            if depths[lvl]:
+                h = tf(h, f"d{lvl}.t{i}.", depths[lvl])
+            skips.append(h)
+        if lvl < 2:
+            h = conv(h, f"d{lvl}.down", 2)
+            skips.append(h)
+    h = res(h, "mid.r0.")
+    h = tf(h, "mid.t.", depths[2])
+    h = res(h, "mid.r1.")
+    for lvl in (2, 1, 0):
+        for i in range(3):
+            sk = skips.pop()
+            h = res(np.concatenate([sk, h] if skip_first else [h, sk]), f"u{lvl}.r{i}.")
+            if depths[lvl]:
+                h = tf(h, f"u{lvl}.t{i}.", depths[lvl])
+        if lvl > 0:
+            up = F.interpolate(T64(h)[None], scale_factor=2, mode="nearest")[0].numpy()
+            h = conv(up, f"u{lvl}.up", 1)
+    a = F.silu(F.group_norm(T64(h)[None], G, T64(w["out.gn_gamma"]), T64(w["out.gn_beta"]), eps))
+    return F.conv2d(a, T64(w["out.conv_w"]), T64(w["out.conv_b"]), padding=1)[0].numpy()
+
+
+def _unet(st, x, ctx, temb, w, P, mode, depths=UNET_TINY["depths"]):
+    t = UNET_TINY
+    return O.sdxl_unet_step(st, x, ctx, temb, w, P, t["G"], 1e-5, 1.0, mode, "none", base=t["base"],
+                            depths=depths, head_dim=t["head_dim"])
+
+
+def test_upsample_and_concat_are_the_library_ops():
+    r = rng(120)
+    x, y = r.standard_normal((3, 4, 5)), r.standard_normal((2, 4, 5))
+    np.testing.assert_array_equal(O.upsample_nearest2x(x),
+                                  F.interpolate(T64(x)[None], scale_factor=2, mode="nearest")[0].numpy())
+    np.testing.assert_array_equal(O.concat_channels(x, y), torch.cat([T64(x), T64(y)]).numpy())
+
+
+@pytest.mark.parametrize("mode", [SYNC, DISPLACED, NAIVE])
+def test_p1_sdxl_unet_equals_library(mode):
+    """One band: the whole U-Net step is the ordinary network composed from library operators
+    (after a sync step, so a displaced step has stale state).  Swapping the skip order, or
+    the transformer depths of the two deeper levels, changes the result."""
+    w, ctx, temb = _sdxl_unet_case(121, 8, 8, 1)
+    x = rng(122).standard_normal((UNET_TINY["Cl"], 8, 8))
+    st = {}
+    _unet(st, x, ctx, temb, w, 1, SYNC)
+    y = _unet(st, x, ctx, temb, w, 1, mode)
+    ref = lib_sdxl_unet(x, ctx, temb, w)
+    np.testing.assert_allclose(y, ref, rtol=0, atol=1e-10 * np.abs(ref).max())
+    assert np.abs(y - lib_sdxl_unet(x, ctx, temb, w, skip_first=True)).max() > 1e-3 * np.abs(ref).max()
+    w2, _, _ = _sdxl_unet_case(121, 8, 8, 1, depths=(0, 2, 2))
+    assert np.abs(_unet({}, x, ctx, temb, w2, 1, SYNC, depths=(0, 2, 2)) - ref).max() > 1e-3 * np.abs(ref).max()
+
+
+def test_sdxl_unet_naive_equals_independent_crops():
+    """Naive patches: every band is an independent image through the whole network."""
+    P, H, W = 2, 16, 8
+    w, ctx, temb = _sdxl_unet_case(123, H, W, P)
+    x = rng(124).standard_normal((UNET_TINY["Cl"], H, W))
+    y = _unet({}, x, ctx, temb, w, P, NAIVE)
+    hb = H // P
+    for p in range(P):
+        ref = lib_sdxl_unet(x[:, p * hb:(p + 1) * hb], ctx, temb, w)
+        np.testing.assert_allclose(y[:, p * hb:(p + 1) * hb], ref, rtol=0, atol=1e-10 * np.abs(ref).max())
+
+
+def test_sdxl_unet_unchanged_input_displaced_equals_sync():
+    """With the same input as the step before, every stale buffer (conv inputs, keys and
+    values, GroupNorm statistics) holds what a sync step computes, so displaced equals sync."""
+    P, H, W = 4, 16, 8
+    w, ctx, temb = _sdxl_unet_case(125, H, W, P)
+    x = rng(126).standard_normal((UNET_TINY["Cl"], H, W))
+    st = {}
+    ys = _unet(st, x, ctx, temb, w, P, SYNC)
+    yd = _unet(st, x, ctx, temb, w, P, DISPLACED)
+    np.testing.assert_allclose(yd, ys, rtol=0, atol=1e-10 * np.abs(ys).max())
+
+
+def test_sdxl_unet_displaced_band_locality():
+    """A displaced step takes nothing of the current step from other bands, through all
+    levels, skips and up/down sampling: changing band q's input leaves every other band's
+    output bit for bit the same; a sync step carries the change to every band; and a
+    displaced step after drift lies closer to sync than naive does."""
+    P, H, W, q = 4, 16, 8, 2
+    w, ctx, temb = _sdxl_unet_case(127, H, W, P)
+    r = rng(128)
+    x0 = r.standard_normal((UNET_TINY["Cl"], H, W))
+    x1 = x0 + 0.2 * r.standard_normal(x0.shape)
+    hb = H // P
+    x1b = x1.copy()
+    x1b[:, q * hb:(q + 1) * hb] += r.standard_normal((UNET_TINY["Cl"], hb, W))
+    res = {}
+    for mode in (SYNC, DISPLACED, NAIVE):
+        outs = []
+        for xin in (x1, x1b):
+            st = {}
+            _unet(st, x0, ctx, temb, w, P, SYNC)
+            outs.append(_unet(st, xin, ctx, temb, w, P, mode))
+        res[mode] = outs[0]
+        if mode == NAIVE:
+            continue
+        for p in range(P):
+            rows = slice(p * hb, (p + 1) * hb)
+            assert np.array_equal(outs[0][:, rows], outs[1][:, rows]) == (mode == DISPLACED and p != q), (mode, p)
+    err = lambda m: np.linalg.norm(res[m] - res[SYNC]) / np.linalg.norm(res[SYNC])
+    assert 0 < err(DISPLACED) < err(NAIVE)
