@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(PKG_DIR, "libdp.so")
 DP_OK, DP_ERR_INVALID_ARG, DP_ERR_UNSUPPORTED, DP_ERR_STATE, DP_ERR_CUDA, DP_ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
 SYNC, DISPLACED, NAIVE = 0, 1, 2
 BF16, FP32 = 0, 1
-GN_CONV, RESBLOCK, ATTN, UNET_MINI, TRANSFORMER = 0, 1, 2, 3, 4
+GN_CONV, RESBLOCK, ATTN, UNET_MINI, TRANSFORMER, UNET_SDXL = 0, 1, 2, 3, 4, 5
 GN_STATS_CORRECTED, GN_STATS_LOCAL, GN_STATS_STALE, GN_STATS_SYNC = 0, 1, 2, 3
 
 ERR_NAMES = {DP_ERR_INVALID_ARG: "DP_ERR_INVALID_ARG", DP_ERR_UNSUPPORTED: "DP_ERR_UNSUPPORTED",
@@ -39,7 +39,8 @@ class BlockDesc(ctypes.Structure):
                 ("silu", ctypes.c_int), ("eps", ctypes.c_float), ("w", ctypes.c_float),
                 ("gn_stats", ctypes.c_int), ("ctx_len", ctypes.c_int), ("ctx_dim", ctypes.c_int),
                 ("ff_inner", ctypes.c_int), ("temb_dim", ctypes.c_int), ("gn_fuse", ctypes.c_int),
-                ("depth", ctypes.c_int)]
+                ("depth", ctypes.c_int), ("unet_base", ctypes.c_int),
+                ("unet_depth", ctypes.c_int * 3)]
 
 
 class BlockState(ctypes.Structure):
@@ -73,6 +74,8 @@ _SIGS = {
     "dp_attn_cross": ([_V, _V, _V, _V, _I, _I, _I, _I, _F, _V, _SZ, _V], _I),
     "dp_layernorm": ([_V, _V, _V, _V, _I, _I, _F, _V], _I),
     "dp_geglu": ([_V, _V, _I, _I, _V], _I),
+    "dp_concat_channels": ([_V, _V, _V, ctypes.c_size_t, _I, _I, _I, _V], _I),
+    "dp_upsample_nearest2x": ([_V, _V, _I, _I, _I, _I, _V], _I),
     "dp_time_embedding_bias": ([_V, _V, _V, _V, _V, _I, _I, _V], _I),
     "dp_ddim_step": ([_V, _V, _V, _SZ, ctypes.c_double, ctypes.c_double, _I, _V], _I),
     "dp_dpm_solver_step": ([_V, _V, _V, _V, _SZ, ctypes.c_double, ctypes.c_double, ctypes.c_double, _I, _V],
@@ -85,6 +88,7 @@ _SIGS = {
     "dp_block_desc_set_gn_fusion": ([ctypes.POINTER(BlockDesc), _I], _I),
     "dp_block_desc_set_context": ([ctypes.POINTER(BlockDesc), _I, _I, _I], _I),
     "dp_block_desc_set_depth": ([ctypes.POINTER(BlockDesc), _I], _I),
+    "dp_block_desc_set_unet": ([ctypes.POINTER(BlockDesc), _I, _I, _I, _I], _I),
     "dp_block_desc_set_time_embedding": ([ctypes.POINTER(BlockDesc), _I], _I),
     "dp_block_workspace_size": ([ctypes.POINTER(BlockDesc)], _SZ),
     "dp_block_state_init": ([ctypes.POINTER(BlockDesc), ctypes.POINTER(BlockState), _V, _SZ, _V], _I),
@@ -261,6 +265,14 @@ def dp_geglu(h, y, T, F, stream=None):
     return _check(lib().dp_geglu(_p(h), _p(y), T, F, _s(stream)))
 
 
+def dp_concat_channels(a, b, out, npix, Ca, Cb, dtype=BF16, stream=None):
+    return _check(lib().dp_concat_channels(_p(a), _p(b), _p(out), npix, Ca, Cb, dtype, _s(stream)))
+
+
+def dp_upsample_nearest2x(x, out, H, W, C, dtype=BF16, stream=None):
+    return _check(lib().dp_upsample_nearest2x(_p(x), _p(out), H, W, C, dtype, _s(stream)))
+
+
 def dp_time_embedding_bias(temb, temb_w, temb_b, conv_b, bias, Ct, Cout, stream=None):
     return _check(lib().dp_time_embedding_bias(_p(temb), _p(temb_w), _p(temb_b), _p(conv_b),
                                                _p(bias), Ct, Cout, _s(stream)))
@@ -314,6 +326,10 @@ def dp_block_desc_set_depth(d: BlockDesc, depth: int):
     return _check(lib().dp_block_desc_set_depth(ctypes.byref(d), depth))
 
 
+def dp_block_desc_set_unet(d: BlockDesc, base: int, depth0: int, depth1: int, depth2: int):
+    return _check(lib().dp_block_desc_set_unet(ctypes.byref(d), base, depth0, depth1, depth2))
+
+
 def dp_block_desc_set_time_embedding(d: BlockDesc, temb_dim: int):
     return _check(lib().dp_block_desc_set_time_embedding(ctypes.byref(d), temb_dim))
 
@@ -361,7 +377,8 @@ def dp_block_step_timed(d: BlockDesc, s: BlockState, x, out, weights: Sequence, 
 
 KERNEL_NAMES = {0: "gn_stats", 1: "gn_apply", 2: "gn_fused", 3: "conv", 4: "linear", 5: "attn",
                 6: "copy", 7: "conv_small", 8: "splitk_finish",
-                9: "gn_cluster", 10: "layernorm", 11: "geglu", 12: "temb", 13: "conv_gn", 14: "conv_f32"}
+                9: "gn_cluster", 10: "layernorm", 11: "geglu", 12: "temb", 13: "conv_gn", 14: "conv_f32",
+                15: "conv_narrow", 16: "concat", 17: "upsample"}
 
 
 def dp_block_launch_info(d: BlockDesc, mode: int, i: int):
@@ -388,11 +405,14 @@ class Block:
 
     def __init__(self, kind, H, W, C, Cout=0, G=32, P=4, heads=0, dtype=BF16, silu=True,
                  eps=1e-5, w=1.0, device="cuda", stream=None, gn_stats=GN_STATS_CORRECTED,
-                 context=None, temb_dim=0, gn_fuse=False, depth=1):
-        """``context`` = (ctx_len, ctx_dim, ff_inner) for TRANSFORMER blocks; ``temb_dim`` the
-        time-embedding width of a RESBLOCK (0: none)."""
+                 context=None, temb_dim=0, gn_fuse=False, depth=1, unet=None):
+        """``context`` = (ctx_len, ctx_dim, ff_inner) for TRANSFORMER and UNET_SDXL blocks;
+        ``temb_dim`` the time-embedding width of a RESBLOCK or UNET_SDXL (0: none); ``unet`` =
+        (base, depth0, depth1, depth2) of a UNET_SDXL block."""
         import torch
         self.desc = dp_block_desc_init(kind, H, W, C, Cout, G, P, heads, dtype, silu, eps, w)
+        if unet is not None:
+            dp_block_desc_set_unet(self.desc, *unet)
         if context is not None:
             dp_block_desc_set_context(self.desc, *context)
         if depth != 1:

@@ -17,9 +17,13 @@
 // which need context from other bands), and UNET_MINI, a chain of the others with
 // two stride-2 downsampling convs (conv_in -> ResBlock(320) -> down ->
 // ResBlock(320->640) -> Attn(640) -> down -> ResBlock(640->1280) ->
-// Attn(1280)).  Composite kinds run their sub-blocks with the parent's
-// ping-pong parity.
+// Attn(1280)), and UNET_SDXL, a whole SDXL-shaped U-Net step (conv_in, three
+// down levels of ResBlocks and transformers, a middle, three up levels whose
+// ResBlocks take the running tensor concatenated with a skip connection, and
+// GroupNorm -> SiLU -> conv_out).  Composite kinds run their sub-blocks with
+// the parent's ping-pong parity.
 #include <cstring>
+#include <vector>
 
 #include "dp_common.cuh"
 #include "dp_internal.h"
@@ -73,8 +77,94 @@ dp_block_desc sub_desc(const dp_block_desc* d, int kind, int H, int W, int C, in
   s.Cout = Cout;
   s.heads = heads;
   s.silu = silu;
+  // kind-specific settings start from their defaults
+  s.ctx_len = s.ctx_dim = s.ff_inner = s.temb_dim = 0;
+  s.depth = 1;
+  s.unet_base = 0;
+  s.unet_depth[0] = s.unet_depth[1] = s.unet_depth[2] = 0;
   return s;
 }
+
+// UNET_SDXL: the stages of one step in execution order.
+enum { US_CONV_IN, US_RES, US_TF, US_DOWN, US_UP, US_OUT };
+struct UStage {
+  int kind;
+  int H, W;            // the stage's input rows and columns (UP: before upsampling)
+  int ci, co;          // input / output channels (RES in the up path: ci includes the skip)
+  bool cat;            // RES: input = [h, latest unused skip]
+  bool skip;           // the stage's output is a skip connection of the up path
+  dp_block_desc sub;   // RES, TF, OUT: the sub-block
+};
+
+std::vector<UStage> unet_stages(const dp_block_desc* d) {
+  std::vector<UStage> s;
+  const int base = d->unet_base;
+  const int ch[3] = {base, 2 * base, 4 * base};
+  int H = d->H, W = d->W, c = base;
+  std::vector<int> skips;
+  auto add = [&](int kind, int ci, int co, bool cat) -> UStage& {
+    UStage u;
+    memset(&u, 0, sizeof(u));
+    u.kind = kind;
+    u.H = H;
+    u.W = W;
+    u.ci = ci;
+    u.co = co;
+    u.cat = cat;
+    if (kind == US_RES) {
+      u.sub = sub_desc(d, DP_BLOCK_RESBLOCK, H, W, ci, co, 0, 1);
+      u.sub.temb_dim = d->temb_dim;
+    } else if (kind == US_TF) {
+      u.sub = sub_desc(d, DP_BLOCK_TRANSFORMER, H, W, ci, ci, ci / 64, 0);
+      u.sub.ctx_len = d->ctx_len;
+      u.sub.ctx_dim = d->ctx_dim;
+      u.sub.ff_inner = 4 * ci;
+    } else if (kind == US_OUT) {
+      u.sub = sub_desc(d, DP_BLOCK_GN_CONV, H, W, ci, co, 0, 1);
+    }
+    s.push_back(u);
+    return s.back();
+  };
+  add(US_CONV_IN, d->C, base, false).skip = true;
+  skips.push_back(base);
+  for (int lvl = 0; lvl < 3; ++lvl) {
+    for (int i = 0; i < 2; ++i) {
+      add(US_RES, c, ch[lvl], false);
+      c = ch[lvl];
+      if (d->unet_depth[lvl] > 0) add(US_TF, c, c, false).sub.depth = d->unet_depth[lvl];
+      s.back().skip = true;
+      skips.push_back(c);
+    }
+    if (lvl < 2) {
+      add(US_DOWN, c, c, false).skip = true;
+      skips.push_back(c);
+      H /= 2;
+      W /= 2;
+    }
+  }
+  add(US_RES, c, c, false);
+  if (d->unet_depth[2] > 0) add(US_TF, c, c, false).sub.depth = d->unet_depth[2];
+  add(US_RES, c, c, false);
+  for (int lvl = 2; lvl >= 0; --lvl) {
+    for (int i = 0; i < 3; ++i) {
+      add(US_RES, c + skips.back(), ch[lvl], true);
+      skips.pop_back();
+      c = ch[lvl];
+      if (d->unet_depth[lvl] > 0) add(US_TF, c, c, false).sub.depth = d->unet_depth[lvl];
+    }
+    if (lvl > 0) {
+      add(US_UP, c, c, false);
+      H *= 2;
+      W *= 2;
+    }
+  }
+  add(US_OUT, c, d->C, false);
+  return s;
+}
+
+// Weight pointers of a stage in the composite's list (a ResBlock's temb vector
+// and a transformer's context are the composite's last two pointers).
+int stage_weight_count(const UStage& u);
 
 struct MiniDescs {
   dp_block_desc rb1, rb2, at2, rb3, at3;
@@ -89,6 +179,46 @@ MiniDescs mini_descs(const dp_block_desc* d) {
   m.rb3 = sub_desc(d, DP_BLOCK_RESBLOCK, H / 4, W / 4, kU2, kU3, 0, 1);
   m.at3 = sub_desc(d, DP_BLOCK_ATTN, H / 4, W / 4, kU3, kU3, kU3 / 64, 0);
   return m;
+}
+
+// UNET_SDXL workspace: per stage its sub-block's workspace (RES, TF, OUT),
+// the ping-pong pair of its conv's input (CONV_IN: a copy of x; DOWN: written
+// by the stage before; UP: the upsampled tensor) and its output buffer; one
+// buffer for the concatenated input of the up path's ResBlocks.
+struct ULayout {
+  std::vector<UStage> st;
+  std::vector<size_t> ws, pair0, pair1, out;
+  size_t cat = 0;
+};
+
+size_t layout_total(const dp_block_desc* d);
+
+ULayout unet_layout(const dp_block_desc* d, Bump& b) {
+  ULayout U;
+  U.st = unet_stages(d);
+  const size_t n = U.st.size();
+  U.ws.assign(n, 0);
+  U.pair0.assign(n, 0);
+  U.pair1.assign(n, 0);
+  U.out.assign(n, 0);
+  size_t cat = 0;
+  for (size_t i = 0; i < n; ++i) {
+    const UStage& u = U.st[i];
+    const size_t hw = static_cast<size_t>(u.H) * u.W;
+    if (u.kind == US_RES || u.kind == US_TF || u.kind == US_OUT) U.ws[i] = b.take(layout_total(&u.sub));
+    if (u.kind == US_CONV_IN || u.kind == US_DOWN || u.kind == US_UP) {
+      const size_t pb = hw * u.ci * 2 * (u.kind == US_UP ? 4 : 1);
+      U.pair0[i] = b.take(pb);
+      U.pair1[i] = b.take(pb);
+    }
+    if (u.kind == US_RES && u.cat) cat = cat > hw * u.ci * 2 ? cat : hw * u.ci * 2;
+    const size_t ob = u.kind == US_DOWN ? hw / 4 * u.co * 2 : u.kind == US_UP ? 4 * hw * u.co * 2 : hw * u.co * 2;
+    // the stage before a down conv writes into that conv's input pair instead
+    const bool to_down = i + 1 < n && U.st[i + 1].kind == US_DOWN;
+    if (u.kind != US_OUT && !to_down) U.out[i] = b.take(ob);
+  }
+  U.cat = b.take(cat);
+  return U;
 }
 
 GnSlots gn_slots(Bump& b, int P, int G) {
@@ -151,6 +281,8 @@ Layout layout_of(const dp_block_desc* d) {
     for (int i = 0; i < 2; ++i) L.v[i] = b.take(hw * d->C * e);
     L.o = b.take(hw * d->C * e);
     L.attn_ws = b.take(attn_workspace_bytes());
+  } else if (d->kind == DP_BLOCK_UNET_SDXL) {
+    unet_layout(d, b);
   } else {
     const MiniDescs m = mini_descs(d);
     const size_t hw2 = hw / 4, hw3 = hw / 16;
@@ -173,6 +305,8 @@ Layout layout_of(const dp_block_desc* d) {
   return L;
 }
 
+size_t layout_total(const dp_block_desc* d) { return layout_of(d).total; }
+
 int desc_check(const dp_block_desc* d) {
   if (d && (d->depth < 1 || d->depth > 16 || (d->depth != 1 && d->kind != DP_BLOCK_TRANSFORMER)))
     return set_error(DP_ERR_INVALID_ARG, "block: depth %d (1..16, and above 1 only for TRANSFORMER)",
@@ -180,7 +314,7 @@ int desc_check(const dp_block_desc* d) {
   if (d && d->gn_fuse != 0 && d->gn_fuse != 1)
     return set_error(DP_ERR_INVALID_ARG, "block: gn fusion flag %d is not 0 or 1", d->gn_fuse);
   if (!d) return set_error(DP_ERR_INVALID_ARG, "block: null descriptor");
-  if (d->kind < DP_BLOCK_GN_CONV || d->kind > DP_BLOCK_TRANSFORMER)
+  if (d->kind < DP_BLOCK_GN_CONV || d->kind > DP_BLOCK_UNET_SDXL)
     return set_error(DP_ERR_INVALID_ARG, "block: bad kind %d", d->kind);
   if (d->H <= 0 || d->W <= 0 || d->C <= 0 || d->Cout <= 0 || d->G <= 0 || d->P <= 0)
     return set_error(DP_ERR_INVALID_ARG, "block: non-positive size");
@@ -194,8 +328,32 @@ int desc_check(const dp_block_desc* d) {
   if (d->H % d->P) return set_error(DP_ERR_UNSUPPORTED, "block: H %% P != 0");
   if (d->temb_dim < 0 || d->temb_dim > 8192)
     return set_error(DP_ERR_INVALID_ARG, "block: time-embedding width %d outside [0, 8192]", d->temb_dim);
-  if (d->temb_dim && d->kind != DP_BLOCK_RESBLOCK)
-    return set_error(DP_ERR_INVALID_ARG, "block: a time embedding is only for RESBLOCK blocks");
+  if (d->temb_dim && d->kind != DP_BLOCK_RESBLOCK && d->kind != DP_BLOCK_UNET_SDXL)
+    return set_error(DP_ERR_INVALID_ARG, "block: a time embedding is only for RESBLOCK and UNET_SDXL blocks");
+  if (d->kind == DP_BLOCK_UNET_SDXL) {
+    if (d->C < 2 || d->C > 8 || d->C % 2)
+      return set_error(DP_ERR_UNSUPPORTED, "block: SDXL U-Net latent needs an even C <= 8");
+    if (d->Cout != d->C) return set_error(DP_ERR_INVALID_ARG, "block: SDXL U-Net needs Cout == C");
+    if (d->unet_base <= 0 || d->unet_base % 64 || d->unet_base > 512)
+      return set_error(DP_ERR_UNSUPPORTED, "block: SDXL U-Net base width %d (a multiple of 64, <= 512)",
+                       d->unet_base);
+    for (int l = 0; l < 3; ++l)
+      if (d->unet_depth[l] < 0 || d->unet_depth[l] > 16)
+        return set_error(DP_ERR_INVALID_ARG, "block: SDXL U-Net depth %d outside [0, 16]", d->unet_depth[l]);
+    if (d->H % (4 * d->P) || d->W % 4)
+      return set_error(DP_ERR_UNSUPPORTED, "block: SDXL U-Net needs H %% 4P == 0 and W %% 4 == 0");
+    if (d->ctx_len < 1 || d->ctx_dim <= 0 || d->ctx_dim % 64 || d->ff_inner != 0)
+      return set_error(DP_ERR_INVALID_ARG, "block: SDXL U-Net needs dp_block_desc_set_context "
+                                           "(ctx_len >= 1, ctx_dim a multiple of 64, ff_inner 0)");
+    if (d->temb_dim <= 0)
+      return set_error(DP_ERR_INVALID_ARG, "block: SDXL U-Net needs dp_block_desc_set_time_embedding");
+    for (const UStage& u : unet_stages(d)) {
+      if (u.kind != US_RES && u.kind != US_TF && u.kind != US_OUT) continue;
+      int rc = desc_check(&u.sub);
+      if (rc) return rc;
+    }
+    return DP_OK;
+  }
   if (d->kind == DP_BLOCK_UNET_MINI) {
     if (d->C > 16 || d->C % 2)
       return set_error(DP_ERR_UNSUPPORTED, "block: mini U-Net latent needs an even C <= 16");
@@ -209,7 +367,9 @@ int desc_check(const dp_block_desc* d) {
     }
     return DP_OK;
   }
-  if (d->C % d->G || d->Cout % d->G) return set_error(DP_ERR_UNSUPPORTED, "block: channels %% G != 0");
+  // GroupNorms act on the input channels (and on Cout inside a RESBLOCK)
+  if (d->C % d->G || (d->kind != DP_BLOCK_GN_CONV && d->Cout % d->G))
+    return set_error(DP_ERR_UNSUPPORTED, "block: channels %% G != 0");
   if (d->kind == DP_BLOCK_TRANSFORMER) {
     if (d->Cout != d->C) return set_error(DP_ERR_INVALID_ARG, "block: transformer keeps C");
     if (d->heads <= 0 || d->C != d->heads * 64)
@@ -240,9 +400,20 @@ int weight_count(const dp_block_desc* d) {
   if (d->kind == DP_BLOCK_RESBLOCK) return (d->C != d->Cout ? 10 : 8) + (d->temb_dim > 0 ? 3 : 0);
   if (d->kind == DP_BLOCK_ATTN) return 6;
   if (d->kind == DP_BLOCK_TRANSFORMER) return 7 + 18 * d->depth;
+  if (d->kind == DP_BLOCK_UNET_SDXL) {
+    int n = 2;   // context, time embedding
+    for (const UStage& u : unet_stages(d)) n += stage_weight_count(u);
+    return n;
+  }
   const MiniDescs m = mini_descs(d);
   return 2 + weight_count(&m.rb1) + 2 + weight_count(&m.rb2) + weight_count(&m.at2) + 2 +
          weight_count(&m.rb3) + weight_count(&m.at3);
+}
+
+int stage_weight_count(const UStage& u) {
+  if (u.kind == US_RES || u.kind == US_TF) return weight_count(&u.sub) - 1;
+  if (u.kind == US_OUT) return weight_count(&u.sub);
+  return 2;
 }
 
 double flops_of(const dp_block_desc* d) {
@@ -261,6 +432,17 @@ double flops_of(const dp_block_desc* d) {
                        2.0 * hw * 3.0 * C * C + 4.0 * hw * hw * C +   // q/k/v, self-attention
                        2.0 * Tk * 2.0 * C * Cc + 4.0 * hw * Tk * C +  // context k/v, cross-attention
                        2.0 * hw * 2.0 * F * C + 2.0 * hw * C * F);    // ff1, ff2
+  }
+  if (d->kind == DP_BLOCK_UNET_SDXL) {
+    double f = 0.0;
+    for (const UStage& u : unet_stages(d)) {
+      const double uhw = static_cast<double>(u.H) * u.W;
+      if (u.kind == US_CONV_IN) f += 2.0 * uhw * u.co * 9.0 * u.ci;
+      else if (u.kind == US_DOWN) f += 2.0 * (uhw / 4) * u.co * 9.0 * u.ci;
+      else if (u.kind == US_UP) f += 2.0 * (4 * uhw) * u.co * 9.0 * u.ci;
+      else f += flops_of(&u.sub);
+    }
+    return f;
   }
   const MiniDescs m = mini_descs(d);
   return 2.0 * hw * kU1 * 9.0 * C + flops_of(&m.rb1) + 2.0 * (hw / 4) * kU1 * 9.0 * kU1 +
@@ -282,10 +464,10 @@ struct LaunchRec {
   double flops, bytes;
 };
 struct Plan {
-  LaunchRec rec[128];
+  std::vector<LaunchRec> rec;
   int n = 0;
   void push(int kind, double flops, double bytes) {
-    if (n < 128) rec[n] = {kind, flops, bytes};
+    rec.push_back({kind, flops, bytes});
     ++n;
   }
 };
@@ -342,7 +524,10 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
     if (plan) {
       const double ho = (h - 1) / stride + 1, wo = (wd - 1) / stride + 1;
       const int S = conv3x3_splits(h, wd, ci, co, stride, d->dtype, true);
-      if (d->dtype == DP_FP32) {
+      if (conv3x3_is_narrow(co)) {
+        plan->push(DP_KERNEL_CONV_NARROW, 2.0 * ho * wo * co * 9.0 * ci,
+                   (static_cast<double>(h) * wd * ci + ho * wo * co * (res ? 2 : 1)) * e);
+      } else if (d->dtype == DP_FP32) {
         plan->push(DP_KERNEL_CONV_F32, 2.0 * ho * wo * co * 9.0 * ci,
                    (static_cast<double>(h) * wd * ci + ho * wo * co * (res ? 2 : 1)) * e);
       } else if (S == 1) {
@@ -408,7 +593,7 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
                              silu, wt, static_cast<const float*>(b), res, y, H, W, ch, co, P, mode, st);
   };
   int rc;
-  if (d->kind != DP_BLOCK_UNET_MINI && !plan) {
+  if (d->kind != DP_BLOCK_UNET_MINI && d->kind != DP_BLOCK_UNET_SDXL && !plan) {
     // biases (conv_b, conv1_b, conv2_b, short_b, temb_b; bqkv, bo, ...) may be NULL
     const int temb_b = weight_count(d) - 2;   // RESBLOCK with a time embedding: temb_b
     for (int i = 0; i < weight_count(d); ++i) {
@@ -579,6 +764,92 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
     }
     return lin(ob, w[4], w[5], x, out, nullptr, nullptr, T, C, C, C);
   }
+  if (d->kind == DP_BLOCK_UNET_SDXL) {
+    Bump b;
+    b.take(sizeof(int));   // the status word, as layout_of
+    const ULayout U = unet_layout(d, b);
+    const int nw = weight_count(d);
+    const void* ctx = w[nw - 2];
+    const void* temb = w[nw - 1];
+    std::vector<const void*> skips, sw;
+    const void* h = nullptr;
+    int wi = 0;
+    for (size_t i = 0; i < U.st.size(); ++i) {
+      const UStage& u = U.st[i];
+      const void* const* uw = w + wi;
+      wi += stage_weight_count(u);
+      void* sub_ws = at<void>(ws, U.ws[i]);
+      // the output of a stage that feeds a down conv goes into that conv's input pair
+      const bool to_down = i + 1 < U.st.size() && U.st[i + 1].kind == US_DOWN;
+      void* dst = to_down ? at<void>(ws, f ? U.pair1[i + 1] : U.pair0[i + 1]) : at<void>(ws, U.out[i]);
+      void* pf = at<void>(ws, f ? U.pair1[i] : U.pair0[i]);
+      void* po = at<void>(ws, o ? U.pair1[i] : U.pair0[i]);
+      const size_t uhw = static_cast<size_t>(u.H) * u.W;
+      if ((u.kind == US_CONV_IN || u.kind == US_DOWN || u.kind == US_UP) && !plan && !uw[0])
+        return set_error(DP_ERR_INVALID_ARG, "block: conv weight of U-Net stage %zu is NULL", i);
+      if (u.kind == US_CONV_IN) {
+        const size_t xb = uhw * u.ci * 2;
+        if (plan) {
+          plan->push(DP_KERNEL_COPY, 0.0, 2.0 * xb);
+          plan->push(DP_KERNEL_CONV_SMALL, 2.0 * uhw * u.co * 9.0 * u.ci, static_cast<double>(uhw) * (u.ci + u.co) * 2.0);
+        } else {
+          rc = copy_launch(x, pf, xb, st);
+          if (rc) return rc;
+          rc = conv3x3_small_launch(pf, po, uw[0], static_cast<const float*>(uw[1]), dst, u.H, u.W, u.ci, u.co, P,
+                                    mode, st);
+          if (rc) return rc;
+        }
+      } else if (u.kind == US_DOWN || u.kind == US_UP) {
+        int hc = u.H, wc = u.W, stride = 2;
+        if (u.kind == US_UP) {
+          hc = 2 * u.H;
+          wc = 2 * u.W;
+          stride = 1;
+          if (plan) {
+            plan->push(DP_KERNEL_UPSAMPLE, 0.0, 5.0 * uhw * u.ci * 2.0);
+          } else {
+            rc = upsample2x_launch(h, pf, u.H, u.W, u.ci, DP_BF16, st);
+            if (rc) return rc;
+          }
+        }
+        if (!plan) {
+          rc = conv3x3_validate(pf, po, uw[0], nullptr, dst, hc, wc, u.ci, u.co, stride, P, mode, DP_BF16);
+          if (rc) return rc;
+        }
+        rc = conv(pf, po, uw[0], uw[1], nullptr, dst, hc, wc, u.ci, u.co, stride);
+        if (rc) return rc;
+      } else if (u.kind == US_RES) {
+        const void* in = h;
+        if (u.cat) {
+          void* cat = at<void>(ws, U.cat);
+          const int ch = U.st[i - 1].co;   // the running tensor's channels; the skip has the rest
+          const int ck = u.ci - ch;
+          if (plan) {
+            plan->push(DP_KERNEL_CONCAT, 0.0, 2.0 * uhw * u.ci * 2.0);
+          } else {
+            rc = concat_launch(h, skips.back(), cat, uhw, ch, ck, DP_BF16, st);
+            if (rc) return rc;
+          }
+          skips.pop_back();
+          in = cat;
+        }
+        sw.assign(uw, uw + stage_weight_count(u));
+        sw.push_back(temb);
+        rc = step_impl(&u.sub, sub_ws, cur, in, dst, sw.data(), mode, st, plan);
+        if (rc) return rc;
+      } else if (u.kind == US_TF) {
+        sw.assign(uw, uw + stage_weight_count(u));
+        sw.push_back(ctx);
+        rc = step_impl(&u.sub, sub_ws, cur, h, dst, sw.data(), mode, st, plan);
+        if (rc) return rc;
+      } else {   // US_OUT
+        return step_impl(&u.sub, sub_ws, cur, h, out, uw, mode, st, plan);
+      }
+      h = dst;
+      if (u.skip) skips.push_back(h);
+    }
+    return set_error(DP_ERR_INVALID_ARG, "block: SDXL U-Net without an output stage");
+  }
   // UNET_MINI
   const MiniDescs m = mini_descs(d);
   const int H2 = H / 2, W2 = W / 2, H3 = H / 4, W3 = W / 4;
@@ -645,8 +916,8 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
 
 // Records the launches of one step of `d` in `mode`.
 int plan_of(const dp_block_desc* d, int mode, Plan* plan) {
-  static const void* const null_w[128] = {nullptr};
-  return step_impl(d, nullptr, 0, nullptr, nullptr, null_w, mode, nullptr, plan);
+  const std::vector<const void*> null_w(weight_count(d) + 1, nullptr);
+  return step_impl(d, nullptr, 0, nullptr, nullptr, null_w.data(), mode, nullptr, plan);
 }
 
 }  // namespace
@@ -676,17 +947,30 @@ int dp_block_desc_init(dp_block_desc* d, int kind, int H, int W, int C, int Cout
   d->temb_dim = 0;
   d->gn_fuse = 0;
   d->depth = 1;
-  if (kind == DP_BLOCK_TRANSFORMER) return DP_OK;   // checked once dp_block_desc_set_context is called
+  d->unet_base = kind == DP_BLOCK_UNET_SDXL ? 320 : 0;
+  d->unet_depth[0] = kind == DP_BLOCK_UNET_SDXL ? 0 : 0;
+  d->unet_depth[1] = kind == DP_BLOCK_UNET_SDXL ? 2 : 0;
+  d->unet_depth[2] = kind == DP_BLOCK_UNET_SDXL ? 10 : 0;
+  if (kind == DP_BLOCK_UNET_SDXL) d->Cout = C;
+  // checked once dp_block_desc_set_context (and, for UNET_SDXL, _set_time_embedding) is called
+  if (kind == DP_BLOCK_TRANSFORMER || kind == DP_BLOCK_UNET_SDXL) return DP_OK;
   return dp::desc_check(d);
 }
 
 int dp_block_desc_set_context(dp_block_desc* d, int ctx_len, int ctx_dim, int ff_inner) {
   if (!d) return dp::set_error(DP_ERR_INVALID_ARG, "block: null descriptor");
-  if (d->kind != DP_BLOCK_TRANSFORMER)
-    return dp::set_error(DP_ERR_INVALID_ARG, "block: a context is only for TRANSFORMER blocks");
+  if (d->kind != DP_BLOCK_TRANSFORMER && d->kind != DP_BLOCK_UNET_SDXL)
+    return dp::set_error(DP_ERR_INVALID_ARG, "block: a context is only for TRANSFORMER and UNET_SDXL blocks");
   d->ctx_len = ctx_len;
   d->ctx_dim = ctx_dim;
   d->ff_inner = ff_inner;
+  if (d->kind == DP_BLOCK_UNET_SDXL) {
+    // the time embedding may still be unset: check the context alone
+    if (ctx_len < 1 || ctx_dim <= 0 || ctx_dim % 64 || ff_inner != 0)
+      return dp::set_error(DP_ERR_INVALID_ARG, "block: SDXL U-Net context needs ctx_len >= 1, ctx_dim a "
+                                               "multiple of 64 and ff_inner 0");
+    return d->temb_dim > 0 ? dp::desc_check(d) : DP_OK;
+  }
   return dp::desc_check(d);
 }
 
@@ -701,11 +985,28 @@ int dp_block_desc_set_depth(dp_block_desc* d, int depth) {
 
 int dp_block_desc_set_time_embedding(dp_block_desc* d, int temb_dim) {
   if (!d) return dp::set_error(DP_ERR_INVALID_ARG, "block: null descriptor");
-  if (d->kind != DP_BLOCK_RESBLOCK)
-    return dp::set_error(DP_ERR_INVALID_ARG, "block: a time embedding is only for RESBLOCK blocks");
+  if (d->kind != DP_BLOCK_RESBLOCK && d->kind != DP_BLOCK_UNET_SDXL)
+    return dp::set_error(DP_ERR_INVALID_ARG, "block: a time embedding is only for RESBLOCK and UNET_SDXL blocks");
   if (temb_dim < 0 || temb_dim > 8192)
     return dp::set_error(DP_ERR_INVALID_ARG, "block: time-embedding width %d outside [0, 8192]", temb_dim);
   d->temb_dim = temb_dim;
+  if (d->kind == DP_BLOCK_UNET_SDXL && d->ctx_len == 0) return DP_OK;   // context still to come
+  return dp::desc_check(d);
+}
+
+int dp_block_desc_set_unet(dp_block_desc* d, int base, int depth0, int depth1, int depth2) {
+  if (!d) return dp::set_error(DP_ERR_INVALID_ARG, "block: null descriptor");
+  if (d->kind != DP_BLOCK_UNET_SDXL)
+    return dp::set_error(DP_ERR_INVALID_ARG, "block: U-Net widths and depths are only for UNET_SDXL blocks");
+  if (base <= 0 || base % 64 || base > 512)
+    return dp::set_error(DP_ERR_INVALID_ARG, "block: SDXL U-Net base width %d (a multiple of 64, <= 512)", base);
+  const int dep[3] = {depth0, depth1, depth2};
+  for (int l = 0; l < 3; ++l)
+    if (dep[l] < 0 || dep[l] > 16)
+      return dp::set_error(DP_ERR_INVALID_ARG, "block: SDXL U-Net depth %d outside [0, 16]", dep[l]);
+  d->unet_base = base;
+  for (int l = 0; l < 3; ++l) d->unet_depth[l] = dep[l];
+  if (d->ctx_len == 0 || d->temb_dim == 0) return DP_OK;   // checked once both are set
   return dp::desc_check(d);
 }
 
@@ -819,7 +1120,7 @@ int dp_block_launch_info(const dp_block_desc* d, int mode, int i, int* kind, dou
   dp::Plan plan;
   rc = dp::plan_of(d, mode, &plan);
   if (rc) return rc;
-  if (i < 0 || i >= plan.n || i >= 128)
+  if (i < 0 || i >= plan.n)
     return dp::set_error(DP_ERR_INVALID_ARG, "block: launch %d of %d", i, plan.n);
   if (kind) *kind = plan.rec[i].kind;
   if (flops) *flops = plan.rec[i].flops;

@@ -1565,7 +1565,7 @@ static int conv_tile_width(int Wo) {
 }
 
 int conv3x3_splits(int H, int W, int Cin, int Cout, int stride, int dtype, bool can_split) {
-  if (dtype == DP_FP32) return 1;
+  if (dtype == DP_FP32 || conv3x3_is_narrow(Cout)) return 1;
   const int Ho = (H - 1) / stride + 1, Wo = (W - 1) / stride + 1;
   const int Wt = conv_tile_width(Wo), R = 128 / Wt;
   const int m_tiles = ((Wo + Wt - 1) / Wt) * ((Ho + R - 1) / R);
@@ -1586,6 +1586,10 @@ int conv3x3_launch(const void* a_fresh, const void* a_stale, const void* weight,
                    const float* bias, const void* residual, void* out, int H, int W, int Cin,
                    int Cout, int stride, int P, int mode, int dtype, void* workspace,
                    size_t workspace_bytes, cudaStream_t stream) {
+  // a few output channels: the CUDA-core conv (dp_conv_narrow.cu)
+  if (conv3x3_is_narrow(Cout))
+    return conv3x3_narrow_launch(a_fresh, a_stale, weight, bias, residual, out, H, W, Cin, Cout, stride, P, mode,
+                                 dtype, stream);
   // fp32 storage: fp32 arithmetic on the CUDA cores (dp_conv_f32.cu)
   if (dtype == DP_FP32)
     return conv3x3_f32_launch(a_fresh, a_stale, weight, bias, residual, out, H, W, Cin, Cout, stride, P,
@@ -1839,7 +1843,8 @@ int conv3x3_validate(const void* a_fresh, const void* a_stale, const void* weigh
     return set_error(DP_ERR_INVALID_ARG, "conv: displaced mode needs the stale buffer");
   const int BK = dtype == DP_FP32 ? 16 : 64;
   if (Cin % BK) return set_error(DP_ERR_UNSUPPORTED, "conv: Cin must be a multiple of %d", BK);
-  if (Cout % 32) return set_error(DP_ERR_UNSUPPORTED, "conv: Cout must be a multiple of 32");
+  if (Cout % 32 && !conv3x3_is_narrow(Cout))
+    return set_error(DP_ERR_UNSUPPORTED, "conv: Cout must be a multiple of 32 or at most 16");
   const int Ho = (H - 1) / stride + 1;
   if (H % P || Ho % P) return set_error(DP_ERR_UNSUPPORTED, "conv: rows not divisible by P");
   if (stride == 2 && (W % 2)) return set_error(DP_ERR_UNSUPPORTED, "conv: stride 2 needs even W");

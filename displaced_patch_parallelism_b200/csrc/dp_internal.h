@@ -29,6 +29,15 @@ size_t gemm_workspace_bytes();
 int conv3x3_f32_launch(const void* a_fresh, const void* a_stale, const void* weight, const float* bias,
                        const void* residual, void* out, int H, int W, int Cin, int Cout, int stride, int P,
                        int mode, cudaStream_t stream);
+// the 3x3 halo conv to Cout <= 16 channels on the CUDA cores (any storage type)
+bool conv3x3_is_narrow(int Cout);
+int conv3x3_narrow_launch(const void* a_fresh, const void* a_stale, const void* weight, const float* bias,
+                          const void* residual, void* out, int H, int W, int Cin, int Cout, int stride, int P,
+                          int mode, int dtype, cudaStream_t stream);
+// the up path's copies: channel concatenation and nearest 2x upsampling
+int concat_launch(const void* a, const void* b, void* out, size_t npix, int Ca, int Cb, int dtype,
+                  cudaStream_t st);
+int upsample2x_launch(const void* x, void* out, int H, int W, int C, int dtype, cudaStream_t st);
 // GroupNorm statistics alone (the first kernel of the two-kernel path): fresh
 // moments, used moments and (if given) the whole-image moments; no apply.
 int gn_stats_launch(const void* x, int H, int W, int C, int G, int P, float w, int mode, int dtype,

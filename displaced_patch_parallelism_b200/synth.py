@@ -179,7 +179,10 @@ def sdxl_unet_stages(base: int, depths) -> List[Tuple[str, str, int, int]]:
         if lvl < 2:
             s.append(("down", f"d{lvl}.down", c, c))
             skips.append(c)
-    s += [("resblock", "mid.r0.", c, c), ("transformer", "mid.t.", c, c), ("resblock", "mid.r1.", c, c)]
+    s.append(("resblock", "mid.r0.", c, c))
+    if depths[2]:
+        s.append(("transformer", "mid.t.", c, c))
+    s.append(("resblock", "mid.r1.", c, c))
     for lvl in (2, 1, 0):
         for i in range(3):
             s.append(("resblock", f"u{lvl}.r{i}.", c + skips.pop(), ch[lvl]))

@@ -67,6 +67,8 @@ def block_weights(kind: str, wts: Dict, dtype: torch.dtype = torch.bfloat16, dev
                     v(p + "ln3_g"), v(p + "ln3_b"), m(p + "ff1_w"), v(p + "ff1_b"), m(p + "ff2_w"),
                     v(p + "ff2_b")]
         return out + [m("proj_out_w"), v("proj_out_b")]
+    if kind == "unet_sdxl":
+        raise ValueError("use unet_sdxl_weights for a UNET_SDXL block")
     if kind == "unet_mini":
         out = [_conv(g("conv_in_w"), dtype, device), _t(g("conv_in_b"), f32, device)]
         out += block_weights("resblock", wts, dtype, device, prefix + "rb1.")
@@ -78,3 +80,27 @@ def block_weights(kind: str, wts: Dict, dtype: torch.dtype = torch.bfloat16, dev
         out += block_weights("attn", wts, dtype, device, prefix + "at3.")
         return out
     raise ValueError(kind)
+
+
+def unet_sdxl_weights(wts: Dict, stages, depths, dtype: torch.dtype = torch.bfloat16,
+                      device="cuda") -> List[torch.Tensor]:
+    """Device tensors of a UNET_SDXL block in the order ``dp_block_step`` documents, from
+    ``stages`` (the (kind, prefix, cin, cout) list of ``synth.sdxl_unet_stages``) and the
+    levels' transformer ``depths``; the step's context and time embedding, its last two
+    pointers, are appended by the caller."""
+    f32 = torch.float32
+    depth_of = {"d0": depths[0], "d1": depths[1], "d2": depths[2], "mid": depths[2],
+                "u2": depths[2], "u1": depths[1], "u0": depths[0]}
+    out: List[torch.Tensor] = []
+    for kind, pre, _ci, _co in stages:
+        if kind == "conv_in":
+            out += [_conv(wts["conv_in_w"], dtype, device), _t(wts["conv_in_b"], f32, device)]
+        elif kind in ("down", "up"):
+            out += [_conv(wts[pre + "_w"], dtype, device), _t(wts[pre + "_b"], f32, device)]
+        elif kind == "resblock":
+            out += block_weights("resblock", wts, dtype, device, pre)
+        elif kind == "transformer":
+            out += block_weights("transformer", wts, dtype, device, pre, depth_of[pre.split(".")[0]])
+        else:
+            out += block_weights("gn_conv", wts, dtype, device, pre)
+    return out

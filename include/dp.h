@@ -76,6 +76,9 @@ extern "C" {
 #define DP_BLOCK_TRANSFORMER 4 /* SDXL-shaped: GN -> proj_in -> [LN -> self-attention] + ->   */
                                /* [LN -> cross-attention] + -> [LN -> GEGLU FF] + ->          */
                                /* proj_out -> + x (dp_block_desc_set_context first)           */
+#define DP_BLOCK_UNET_SDXL 5   /* SDXL-shaped U-Net step: conv_in, 3 down levels, middle,      */
+                               /* 3 up levels with skips, GN -> SiLU -> conv_out               */
+                               /* (dp_block_desc_set_context, _set_time_embedding first)       */
 
 /* Message for the calling thread's last failed call ("" if none). */
 DP_API const char* dp_last_error(void);
@@ -224,9 +227,12 @@ DP_API int dp_groupnorm_async_noalloc(const void* x, void* y, const float* gamma
  *                    the last run of a tile sums them in run order.  Calls
  *                    that overlap on the GPU must not share it.
  * Ho = (H-1)/stride + 1.  Needs Cin % 64 == 0 (bf16) or % 16 == 0 (fp32),
- * Cout % 32 == 0, H % P == 0, Ho % P == 0, W even when stride 2.  Any W works;
- * ragged tiles are masked.  bf16 runs on the tensor cores (tcgen05, operands
- * staged by TMA); fp32 runs in fp32 on the CUDA cores (bias 16-byte aligned).
+ * Cout % 32 == 0 or Cout <= 16, H % P == 0, Ho % P == 0, W even when stride
+ * 2.  Any W works; ragged tiles are masked.  bf16 runs on the tensor cores
+ * (tcgen05, operands staged by TMA); fp32 runs in fp32 on the CUDA cores (bias
+ * 16-byte aligned); Cout <= 16 (a U-Net's conv_out back to the latent's
+ * channels) runs as fp32 multiply-adds on the CUDA cores for either dtype,
+ * rounded once to the output type.
  * Errors: DP_ERR_INVALID_ARG (null pointers, bad mode/dtype, aliasing,
  * missing stale buffer in DISPLACED), DP_ERR_UNSUPPORTED (shape, alignment).
  * ---------------------------------------------------------------------- */
@@ -439,6 +445,29 @@ DP_API int dp_layernorm(const void* x, void* y, const float* gamma, const float*
 DP_API int dp_geglu(const void* h, void* y, int T, int F, void* stream);
 
 /* ------------------------------------------------------------------------
+ * The up path of an SDXL-shaped U-Net (the pages' SDXL model, "DistriFusion",
+ * atlas.scime.ai summary, Key results): each up ResBlock takes the running
+ * tensor concatenated with a skip connection, and each up level ends in a
+ * nearest-neighbour 2x upsample before its conv.  Both act on a pixel's own
+ * rows, inside its band, so a displaced step runs them on fresh data with no
+ * stale context.  Pure copies, HBM-bound.
+ *
+ * dp_concat_channels: out[pix] = [a[pix] | b[pix]] for npix pixels.
+ *   a [npix][Ca], b [npix][Cb], out [npix][Ca + Cb], dtype (DP_BF16 or
+ *   DP_FP32), device, 16-byte aligned; Ca and Cb multiples of 8 (bf16) or 4
+ *   (fp32); out must not overlap a or b.  npix == 0 is a no-op.
+ * dp_upsample_nearest2x: out[2i + di][2j + dj][c] = x[i][j][c], di, dj in {0, 1}.
+ *   x [H][W][C], out [2H][2W][C], dtype, device, 16-byte aligned, not
+ *   overlapping; C a multiple of 8 (bf16) or 4 (fp32).
+ * Errors: DP_ERR_INVALID_ARG (null pointer, bad dtype or size, overlap),
+ * DP_ERR_UNSUPPORTED (channel count or alignment).
+ * ---------------------------------------------------------------------- */
+DP_API int dp_concat_channels(const void* a, const void* b, void* out, size_t npix, int Ca, int Cb,
+                              int dtype, void* stream);
+DP_API int dp_upsample_nearest2x(const void* x, void* out, int H, int W, int C, int dtype,
+                                 void* stream);
+
+/* ------------------------------------------------------------------------
  * Stale-buffer refresh: the device-local replacement of the paper's
  * per-layer AllGather (atlas.scime.ai summary, Approach: AllGather overlaps
  * computation; limitations: NCCL kernels take SMs).  Copies the rows of band
@@ -497,6 +526,8 @@ typedef struct dp_block_desc {
   int temb_dim;   /* RESBLOCK: time-embedding width (0: none)     */
   int gn_fuse;    /* 1: GroupNorm -> conv through dp_conv3x3_halo_gn */
   int depth;      /* TRANSFORMER: basic transformer layers (default 1) */
+  int unet_base;  /* UNET_SDXL: level widths base, 2 base, 4 base (320) */
+  int unet_depth[3]; /* UNET_SDXL: transformer depth per level (0, 2, 10) */
 } dp_block_desc;
 
 /*
@@ -504,7 +535,9 @@ typedef struct dp_block_desc {
  * feed-forward's inner width (SDXL: 77, 2048, 4C).  The context is an input of
  * every step (the last weight pointer); it is the same for every band, so it
  * has no stale copy.  Needs ctx_len >= 1, ctx_dim % 64 == 0, ff_inner % 64 ==
- * 0.  DP_ERR_INVALID_ARG on a null descriptor or bad sizes.
+ * 0.  UNET_SDXL blocks: the context of all their transformers, with
+ * ff_inner 0 (each transformer's inner width is 4 C).  DP_ERR_INVALID_ARG on
+ * a null descriptor or bad sizes.
  */
 DP_API int dp_block_desc_set_context(dp_block_desc* d, int ctx_len, int ctx_dim, int ff_inner);
 
@@ -519,13 +552,45 @@ DP_API int dp_block_desc_set_context(dp_block_desc* d, int ctx_len, int ctx_dim,
 DP_API int dp_block_desc_set_depth(dp_block_desc* d, int depth);
 
 /*
+ * UNET_SDXL blocks: one whole denoising step of an SDXL-shaped U-Net over all
+ * bands (the pages' SDXL model, "DistriFusion", atlas.scime.ai summary, Key
+ * results; SDXL's layout):
+ *   conv_in (C -> base)
+ *   down level l = 0, 1, 2 (width base << l): 2 x [ResBlock, then a
+ *     transformer of depth unet_depth[l] when it is > 0]; levels 0 and 1 end
+ *     in a 3x3 stride-2 conv
+ *   middle: ResBlock, transformer (depth unet_depth[2], if > 0), ResBlock
+ *   up level l = 2, 1, 0: 3 x [concatenate [h, skip] (the latest unused skip:
+ *     the outputs of conv_in, of each down ResBlock/transformer pair and of
+ *     the down convs), ResBlock, transformer as above]; levels 2 and 1 end in a
+ *     nearest 2x upsample and a 3x3 conv
+ *   GroupNorm -> SiLU -> conv_out (base -> C)
+ * Every ResBlock adds the step's time embedding term; every transformer has
+ * C/64 heads and a feed-forward inner width of 4 C; every 3x3 conv takes its
+ * halo rows from the previous step's copy of its own input.  The descriptor's
+ * C is the latent's channel count (even, <= 8) and Cout = C; bf16 only;
+ * base % 64 == 0, base <= 512; 0 <= unet_depth[l] <= 16; H % 4P == 0,
+ * W % 4 == 0, and each level's transformer needs its tokens per band to be a
+ * multiple of 128.  dp_block_desc_set_context(d, Tk, Cctx, 0) and
+ * dp_block_desc_set_time_embedding(d, Ct) are required.  The weight list is
+ * the stages' lists in execution order (conv_in: w, b; ResBlock: its RESBLOCK
+ * list without the temb vector; transformer: its TRANSFORMER list without the
+ * context; down/up conv: w, b; output: gn_gamma, gn_beta, conv_w, conv_b),
+ * then the step's context [Tk][Cctx] bf16 and time embedding [Ct] fp32.
+ * DP_ERR_INVALID_ARG for another kind or a bad value.
+ */
+DP_API int dp_block_desc_set_unet(dp_block_desc* d, int base, int depth0, int depth1, int depth2);
+
+/*
  * RESBLOCK blocks: the width Ct of the step's time embedding (0 switches it
  * off, the default).  With Ct > 0 the block takes three more weight pointers,
  * temb_w[Cout][Ct], temb_b[Cout] and the step's temb[Ct] (fp32; temb_b may be
  * NULL), and
  * adds temb_w silu(temb) + temb_b to every pixel of conv1's output (one extra
- * launch, dp_time_embedding_bias).  DP_ERR_INVALID_ARG on a null descriptor,
- * another kind, or Ct outside [0, 8192].
+ * launch, dp_time_embedding_bias).  UNET_SDXL blocks: the width of the
+ * step's time embedding every ResBlock takes (> 0 before a step).
+ * DP_ERR_INVALID_ARG on a null descriptor, another kind, or Ct outside
+ * [0, 8192].
  */
 DP_API int dp_block_desc_set_time_embedding(dp_block_desc* d, int temb_dim);
 
@@ -641,6 +706,9 @@ DP_API int dp_block_status(const dp_block_desc* d, const dp_block_state* s, void
 #define DP_KERNEL_TEMB 12       /* time-embedding bias of a ResBlock's conv1     */
 #define DP_KERNEL_CONV_GN 13    /* 3x3 conv of GroupNorm(x), normalised in-kernel */
 #define DP_KERNEL_CONV_F32 14   /* 3x3 halo conv in fp32 on the CUDA cores       */
+#define DP_KERNEL_CONV_NARROW 15 /* 3x3 halo conv to <= 16 channels, CUDA cores  */
+#define DP_KERNEL_CONCAT 16     /* channel concatenation [h, skip]               */
+#define DP_KERNEL_UPSAMPLE 17   /* nearest-neighbour 2x upsampling               */
 
 /*
  * Number of kernel launches one displaced dp_block_step makes for this

@@ -41,6 +41,10 @@ Readings of what the pages leave open:
       transformer block (``transformer_step``) and ResBlock time embedding
       (``resblock_step``'s ``temb``); only GroupNorm statistics and
       self-attention keys/values cross bands
+  R18 the whole SDXL-shaped U-Net (``sdxl_unet_step``): SDXL's level layout
+      (widths base, 2 base, 4 base; transformer depths per level), [h, skip]
+      concatenation, nearest 2x upsampling; one GroupNorm epsilon for all
+      GroupNorms; the caller gives the step's time embedding vector
 
 Parity pins (the tests under tests/test_oracle_*.py): P = 1 reduces to the
 library full-image block (torch group_norm / conv2d / softmax attention);
@@ -57,6 +61,10 @@ level, is the identity at an unchanged level, composes, and is affine.
 second-order form equals the first when the data prediction does not change,
 and on an ODE whose exact solution is known it converges at second order (the
 first-order form at first order).
+``sdxl_unet_step`` at P = 1 equals the U-Net composed from library operators
+(and differs from it with the skip order swapped or other depths), equals
+independent crops in naive mode, equals sync under an unchanged input, and a
+displaced step keeps every other band bit for bit when one band's input changes.
 ``unet_mini_step`` at P = 1 equals the same chain composed from library
 operators (conv2d with stride 1 and 2, the library ResBlock and attention with
 10 and 20 heads); its naive step at P = 4 equals that library chain on each
@@ -669,7 +677,9 @@ def unet_mini_step(state: Dict, x, wts: Dict, P: int, G: int, eps: float, w: flo
 # (level widths base, 2 base, 4 base), the ResBlocks of levels with a nonzero
 # transformer depth each followed by a transformer block of that depth, levels
 # 0 and 1 ending in a stride-2 conv; a middle ResBlock -> transformer ->
-# ResBlock; three up levels of three ResBlocks, each taking the channel
+# ResBlock (no transformer when the deepest level's depth is 0, as no
+# transformer follows a ResBlock at a level of depth 0); three up levels of
+# three ResBlocks, each taking the channel
 # concatenation [h, skip] of the running tensor and the latest unused skip
 # (the outputs of conv_in, of every down ResBlock/transformer pair and of the
 # down convs), levels 2 and 1 ending in a nearest-neighbour 2x upsample and a
@@ -731,7 +741,8 @@ def sdxl_unet_step(state: Dict, x, ctx, temb, wts: Dict, P: int, G: int, eps: fl
             h = conv_layer(f"d{lvl}.down", h, 2)
             skips.append(h)
     h = resblock("mid.r0.", h)
-    h = transformer("mid.t.", h, depths[2])
+    if depths[2]:
+        h = transformer("mid.t.", h, depths[2])
     h = resblock("mid.r1.", h)
     for lvl in (2, 1, 0):
         for i in range(3):

@@ -444,6 +444,77 @@ def test_transformer_depth_workload_marshals(B):
     assert not torch.equal(w2[6], w2[24])                                 # the layers' wqkv differ
 
 
+def test_unet_sdxl_descriptor_on_the_host(B):
+    """An SDXL-shaped U-Net step: it needs its context and time embedding; at SDXL's own sizes
+    (latent 4x128x128, base 320, depths 0 / 2 / 10) it takes 1534 pointers and 6.76 TFLOP;
+    its launches follow the stage order and add up to its flops; the seeded small workload's
+    marshalled weights fill its list."""
+    import torch
+
+    from displaced_patch_parallelism_b200 import synth
+    from displaced_patch_parallelism_b200.weights import unet_sdxl_weights
+    d = B.dp_block_desc_init(B.UNET_SDXL, 128, 128, 4, 0, 32, 8, 0, B.BF16, 1, 1e-5, 1.0)
+    assert d.Cout == 4 and d.unet_base == 320 and list(d.unet_depth) == [0, 2, 10]
+    with pytest.raises(B.DPError, match="set_context"):
+        B.dp_block_workspace_size(d)
+    B.dp_block_desc_set_context(d, 77, 2048, 0)
+    with pytest.raises(B.DPError, match="set_time_embedding"):
+        B.dp_block_workspace_size(d)
+    B.dp_block_desc_set_time_embedding(d, 1280)
+    assert B.dp_block_weight_count(d) == 1534
+    assert abs(B.dp_block_flops(d) - 6.7612e12) < 1e-3 * 6.76e12
+    kinds = [B.dp_block_launch_info(d, B.DISPLACED, i)[0] for i in range(B.dp_block_launch_count(d))]
+    assert kinds[:2] == ["copy", "conv_small"] and kinds[-1] == "conv_narrow"
+    assert kinds.count("concat") == 9 and kinds.count("upsample") == 2
+    fl = sum(B.dp_block_launch_info(d, B.DISPLACED, i)[1] for i in range(len(kinds)))
+    assert abs(fl - B.dp_block_flops(d)) < 1e-9 * fl
+    for bad in [(320, -1, 2, 10), (96, 0, 2, 10), (320, 0, 17, 10), (1024, 0, 2, 10)]:
+        with pytest.raises(B.DPError):
+            B.dp_block_desc_set_unet(d, *bad)
+    with pytest.raises(B.DPError):
+        B.dp_block_desc_set_context(d, 77, 2048, 5120)   # the inner width is 4C per level
+    r = B.dp_block_desc_init(B.RESBLOCK, 32, 32, 320, 320, 32, 4, 0, B.BF16, 1, 1e-5, 1.0)
+    with pytest.raises(B.DPError, match="UNET_SDXL"):
+        B.dp_block_desc_set_unet(r, 320, 0, 2, 10)
+    # a small U-Net: the marshalled seeded weights fill the list, the context and temb follow
+    wl = synth.Workload(name="u", kind="unet_sdxl", C=4, H=64, W=64, P=2, base=64, depths=(0, 1, 1),
+                        ctx_len=77, ctx_dim=128, temb_dim=128)
+    s = B.dp_block_desc_init(B.UNET_SDXL, 64, 64, 4, 4, 32, 2, 0, B.BF16, 1, 1e-5, 1.0)
+    B.dp_block_desc_set_unet(s, 64, 0, 1, 1)
+    B.dp_block_desc_set_context(s, 77, 128, 0)
+    B.dp_block_desc_set_time_embedding(s, 128)
+    w = unet_sdxl_weights(synth.make_weights(wl), synth.sdxl_unet_stages(64, (0, 1, 1)), (0, 1, 1),
+                          torch.bfloat16, "cpu")
+    assert len(w) + 2 == B.dp_block_weight_count(s)
+    # too few tokens per band at the deepest level for its transformer
+    with pytest.raises(B.DPError):
+        B.dp_block_desc_set_unet(d, 320, 0, 2, 10)
+        t = B.dp_block_desc_init(B.UNET_SDXL, 32, 32, 4, 4, 32, 2, 0, B.BF16, 1, 1e-5, 1.0)
+        B.dp_block_desc_set_context(t, 77, 2048, 0)
+        B.dp_block_desc_set_time_embedding(t, 1280)
+
+
+def test_concat_upsample_reject_bad_arguments_on_the_host(B):
+    """Argument checks run before any launch: null pointers, channel counts that are not whole
+    16-byte vectors, overlapping output, misalignment, bad sizes."""
+    A = 1 << 20                                   # fake, never dereferenced: checks run first
+    for args, code in [((0, 2 * A, 3 * A, 4, 64, 64), B.DP_ERR_INVALID_ARG),            # null a
+                       ((A, 2 * A, 3 * A, 4, 60, 68), B.DP_ERR_UNSUPPORTED),           # channels
+                       ((3 * A, 2 * A, 3 * A, 4, 64, 64), B.DP_ERR_INVALID_ARG),       # out overlaps a
+                       ((A, 2 * A, 3 * A + 8, 4, 64, 64), B.DP_ERR_UNSUPPORTED),       # misaligned
+                       ((A, 2 * A, 3 * A, 4, 0, 64), B.DP_ERR_INVALID_ARG)]:           # empty channels
+        with pytest.raises(B.DPError) as e:
+            B.dp_concat_channels(*args, stream=0)
+        assert e.value.code == code, args
+    for args, code in [((0, 2 * A, 2, 2, 64), B.DP_ERR_INVALID_ARG),                   # null x
+                       ((A, 2 * A, 2, 2, 12), B.DP_ERR_UNSUPPORTED),                   # C not whole vectors
+                       ((A, A + 64, 1, 1, 64), B.DP_ERR_INVALID_ARG),                  # out overlaps x
+                       ((A, 2 * A, 0, 2, 64), B.DP_ERR_INVALID_ARG)]:                  # empty image
+        with pytest.raises(B.DPError) as e:
+            B.dp_upsample_nearest2x(*args, stream=0)
+        assert e.value.code == code, args
+
+
 def test_transformer_workload_marshals_to_the_block(B):
     """The benchmark's SDXL transformer workload: its seeded weights marshal into the 24
     pointers the block documents (the context is the 25th), with the documented shapes."""

@@ -1020,7 +1020,8 @@ def lib_sdxl_unet(x, ctx, temb, w, depths=UNET_TINY["depths"], skip_first=False)
             h = conv(h, f"d{lvl}.down", 2)
             skips.append(h)
     h = res(h, "mid.r0.")
-    h = tf(h, "mid.t.", depths[2])
+    if depths[2]:
+        h = tf(h, "mid.t.", depths[2])
     h = res(h, "mid.r1.")
     for lvl in (2, 1, 0):
         for i in range(3):
