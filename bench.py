@@ -178,12 +178,14 @@ def job_tflops(world_size, flops_per_step, steps, total_ms):
 
 def block_kind(B, wl):
     return {"gn_conv": B.GN_CONV, "resblock": B.RESBLOCK, "attn": B.ATTN,
-            "unet_mini": B.UNET_MINI, "transformer": B.TRANSFORMER}[wl.kind]
+            "unet_mini": B.UNET_MINI, "transformer": B.TRANSFORMER, "unet_sdxl": B.UNET_SDXL}[wl.kind]
 
 
 def wl_context(wl):
-    """(ctx_len, ctx_dim, ff_inner) of a transformer workload, else None."""
-    return (wl.ctx_len, wl.ctx_dim, wl.ff_inner) if wl.kind == "transformer" else None
+    """(ctx_len, ctx_dim, ff_inner) of a transformer or whole-U-Net workload, else None."""
+    if wl.kind == "transformer":
+        return (wl.ctx_len, wl.ctx_dim, wl.ff_inner)
+    return (wl.ctx_len, wl.ctx_dim, 0) if wl.kind == "unet_sdxl" else None
 
 
 def oracle_context(wl):
@@ -196,6 +198,9 @@ def block_desc(B, wl, H=None):
     d = B.dp_block_desc_init(block_kind(B, wl), H or wl.H, wl.W, wl.C, wl.cout, wl.G, wl.P,
                              wl.heads, B.BF16 if wl.dtype == "bf16" else B.FP32, wl.silu,
                              wl.eps, 1.0)
+    if wl.kind == "unet_sdxl":
+        B.dp_block_desc_set_unet(d, wl.base, *wl.depths)
+        B.dp_block_desc_set_time_embedding(d, wl.temb_dim)
     if wl_context(wl):
         B.dp_block_desc_set_context(d, *wl_context(wl))
     B.dp_block_desc_set_gn_stats(d, GN_STATS)
@@ -237,11 +242,36 @@ def wl_flops(wl, H=None):
         return resblock(hw, C, Co)
     if wl.kind == "attn":
         return attn(hw, C)
+    def transformer(t, c, f, depth):
+        Tk, Cc = float(wl.ctx_len), float(wl.ctx_dim)
+        layer = (2.0 * t * c * c * 3.0 + 2.0 * t * 3.0 * c * c + 4.0 * t * t * c + 2.0 * Tk * 2.0 * c * Cc +
+                 4.0 * t * Tk * c + 2.0 * t * 2.0 * f * c + 2.0 * t * c * f)
+        return 2.0 * t * c * c * 2.0 + depth * layer
+
     if wl.kind == "transformer":
-        Tk, Cc, F = float(wl.ctx_len), float(wl.ctx_dim), float(wl.ff_inner)
-        return (2.0 * hw * C * C * 5.0 + 2.0 * hw * 3.0 * C * C + 4.0 * hw * hw * C +
-                2.0 * Tk * 2.0 * C * Cc + 4.0 * hw * Tk * C + 2.0 * hw * 2.0 * F * C +
-                2.0 * hw * C * F)
+        return transformer(hw, C, float(wl.ff_inner), wl.depth)
+    if wl.kind == "unet_sdxl":
+        from displaced_patch_parallelism_b200 import synth
+        level = {"d0": 0, "u0": 0, "d1": 1, "u1": 1, "d2": 2, "u2": 2, "mid": 2}
+        depth = {"d0": wl.depths[0], "u0": wl.depths[0], "d1": wl.depths[1], "u1": wl.depths[1],
+                 "d2": wl.depths[2], "u2": wl.depths[2], "mid": wl.depths[2]}
+        total = 0.0
+        for kind, pre, ci, co in synth.sdxl_unet_stages(wl.base, wl.depths):
+            key = pre.split(".")[0]
+            t = hw / 4 ** level.get(key, 0)          # the stage's pixels (its input's, for down/up)
+            if kind == "conv_in":
+                total += conv(hw, C, co)
+            elif kind == "out":
+                total += conv(hw, ci, C)
+            elif kind == "down":
+                total += conv(t / 4, ci, co)
+            elif kind == "up":
+                total += conv(t * 4, ci, co)
+            elif kind == "resblock":
+                total += resblock(t, ci, co) + 2.0 * co * wl.temb_dim
+            else:
+                total += transformer(t, ci, 4.0 * ci, depth[key])
+        return total
     if wl.kind == "unet_mini":
         return (conv(hw, C, 320) + resblock(hw, 320, 320) + conv(hw / 4, 320, 320) +
                 resblock(hw / 4, 320, 640) + attn(hw / 4, 640) + conv(hw / 16, 640, 640) +
@@ -370,16 +400,28 @@ class Run:
 
         from displaced_patch_parallelism_b200 import binding as B
         from displaced_patch_parallelism_b200 import synth
-        from displaced_patch_parallelism_b200.weights import block_weights
+        from displaced_patch_parallelism_b200.weights import block_weights, unet_sdxl_weights
         self.wl, self.B = wl, B
         self.tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
-        wts = synth.make_weights(wl)
-        self.dw = block_weights(wl.kind, wts, self.tdt, dev)
-        if wl.kind == "transformer":     # the step's text context is the last pointer
-            self.dw.append(synth.context(wl).to(self.tdt).to(dev))
+        if wl.kind == "unet_sdxl":
+            # 2.56 billion parameters: drawn on the device; the step's context and time
+            # embedding are its last two pointers
+            wts = synth.make_weights(wl, device=dev)
+            self.dw = unet_sdxl_weights(wts, synth.sdxl_unet_stages(wl.base, wl.depths), wl.depths,
+                                        self.tdt, dev)
+            del wts
+            self.dw += [synth.context(wl).to(self.tdt).to(dev),
+                        synth.randn((wl.temb_dim,), wl.seed + 600).to(dev)]
+        else:
+            wts = synth.make_weights(wl)
+            self.dw = block_weights(wl.kind, wts, self.tdt, dev)
+            if wl.kind == "transformer":     # the step's text context is the last pointer
+                self.dw.append(synth.context(wl).to(self.tdt).to(dev))
+        unet = (wl.base,) + tuple(wl.depths) if wl.kind == "unet_sdxl" else None
         self.blk = B.Block(block_kind(B, wl), wl.H, wl.W, wl.C, wl.cout, wl.G, wl.P, wl.heads,
                            B.BF16 if wl.dtype == "bf16" else B.FP32, wl.silu, wl.eps, 1.0,
-                           device=dev, gn_stats=GN_STATS, context=wl_context(wl), gn_fuse=GN_FUSE)
+                           device=dev, gn_stats=GN_STATS, context=wl_context(wl), gn_fuse=GN_FUSE,
+                           temb_dim=wl.temb_dim if wl.kind == "unet_sdxl" else 0, unet=unet)
         xs = synth.InputStream(wl)
         self.pool = pool
         self.host_x = [synth.nchw_to_nhwc(xs.x(k)).to(self.tdt).pin_memory() for k in range(pool)]
@@ -472,7 +514,9 @@ def breakdown(run, steps, flush, peaks):
            "gn_cluster": ["dp_gn.cu"], "copy": ["dp_refresh.cu"],
            "conv_small": ["dp_conv_small.cu"], "splitk_finish": ["dp_gemm.cu"],
            "conv_f32": ["dp_conv_f32.cu"],
-           "layernorm": ["dp_token.cu"], "geglu": ["dp_token.cu"], "temb": ["dp_temb.cu"]}
+           "layernorm": ["dp_token.cu"], "geglu": ["dp_token.cu"], "temb": ["dp_temb.cu"],
+           "conv_narrow": ["dp_conv_narrow.cu"], "concat": ["dp_resample.cu"],
+           "upsample": ["dp_resample.cu"]}
     traffic = load_traffic(f"{dominant}:{run.wl.name}", kernel_source_hash(src[dominant]))
     if dk["tflops"] and dominant in ("conv_f32", "conv_small"):
         sm_mhz = peaks.get("sm_max_mhz") or 1965.0
@@ -549,7 +593,7 @@ def time_e2e(run, steps, dist, dev):
 
 
 EXTRA_WORKLOADS = ["tiny_fp32_gn_conv", "resblock_320x128x128", "attn_640x64x64",
-                   "unet_mini_4x128x128", "transformer_640x64x64"]
+                   "unet_mini_4x128x128", "transformer_640x64x64", "unet_sdxl_4x128x128"]
 
 
 def run_ours(args, wl):

@@ -251,7 +251,7 @@ def unet_mini_weight_specs(cin: int) -> List[Tuple[str, Tuple[int, ...], float]]
     return s
 
 
-# The five synthetic workloads (logical NCHW shapes, N = 1).
+# The synthetic workloads (logical NCHW shapes, N = 1).
 WORKLOADS: Dict[str, Workload] = {
     "tiny_fp32_gn_conv": Workload(
         name="tiny_fp32_gn_conv", kind="gn_conv", C=64, H=32, W=32, P=2,
@@ -272,25 +272,41 @@ WORKLOADS: Dict[str, Workload] = {
     "gn_conv_320x480x480": Workload(
         name="gn_conv_320x480x480", kind="gn_conv", C=320, H=480, W=480, P=8,
         steps=50, warmup=4, drift=0.05),
+    # SDXL's whole U-Net at 1024 px (latent 4x128x128), one step of batch 1, over 8 bands:
+    # base width 320, transformer depths 0 / 2 / 10, 77-token context of width 2048, time
+    # embedding of width 1280 (2.56 billion parameters)
+    "unet_sdxl_4x128x128": Workload(
+        name="unet_sdxl_4x128x128", kind="unet_sdxl", C=4, H=128, W=128, P=8, steps=10, warmup=2,
+        drift=0.03, weight_seed=21, base=320, depths=(0, 2, 10), ctx_len=77, ctx_dim=2048,
+        temb_dim=1280),
     "unet_mini_4x128x128": Workload(
         name="unet_mini_4x128x128", kind="unet_mini", C=4, H=128, W=128, P=4, Cout=1280,
         steps=10, warmup=2, drift=0.03, weight_seed=7),
 }
 
 
+# The five block workloads the parity and benchmark configurations are built on; the
+# transformer block and the whole SDXL U-Net are the wider SDXL-shaped workloads.
+CONFIG_WORKLOADS = ("tiny_fp32_gn_conv", "resblock_320x128x128", "attn_640x64x64",
+                    "gn_conv_320x480x480", "unet_mini_4x128x128")
+
+
 def make_weights(wl: Workload, random_affine: bool = False,
-                 affine_seed: int = 99) -> Dict[str, torch.Tensor]:
+                 affine_seed: int = 99, device=None) -> Dict[str, torch.Tensor]:
     """All weights of ``wl`` as fp32 tensors holding storage-rounded values.
 
     GroupNorm scale/shift are 1/0 and biases 0 as the workloads state; with
     ``random_affine`` they are drawn instead (unit tests use this so that an
-    indexing slip in gamma, beta or a bias cannot hide behind zeros).
+    indexing slip in gamma, beta or a bias cannot hide behind zeros).  With a
+    ``device`` the matrices are drawn there by that device's generator, seeded
+    the same way (the benchmark's whole-U-Net workload: 2.56 billion parameters),
+    so their values differ from the CPU draw; the rules are the same.
     """
-    g = torch.Generator(device="cpu")
+    g = torch.Generator(device=device or "cpu")
     g.manual_seed(int(wl.weight_seed))
     out: Dict[str, torch.Tensor] = {}
     for name, shape, std in wl.weight_specs():
-        out[name] = store(torch.randn(*shape, generator=g) * std, wl.dtype)
+        out[name] = store(torch.randn(*shape, generator=g, device=device) * std, wl.dtype)
     # affine parameters and biases
     ga = torch.Generator(device="cpu")
     ga.manual_seed(int(affine_seed))
