@@ -40,7 +40,7 @@ class BlockDesc(ctypes.Structure):
                 ("gn_stats", ctypes.c_int), ("ctx_len", ctypes.c_int), ("ctx_dim", ctypes.c_int),
                 ("ff_inner", ctypes.c_int), ("temb_dim", ctypes.c_int), ("gn_fuse", ctypes.c_int),
                 ("depth", ctypes.c_int), ("unet_base", ctypes.c_int),
-                ("unet_depth", ctypes.c_int * 3)]
+                ("unet_depth", ctypes.c_int * 3), ("ctx_fixed", ctypes.c_int)]
 
 
 class BlockState(ctypes.Structure):
@@ -89,6 +89,7 @@ _SIGS = {
     "dp_block_desc_set_context": ([ctypes.POINTER(BlockDesc), _I, _I, _I], _I),
     "dp_block_desc_set_depth": ([ctypes.POINTER(BlockDesc), _I], _I),
     "dp_block_desc_set_unet": ([ctypes.POINTER(BlockDesc), _I, _I, _I, _I], _I),
+    "dp_block_desc_set_context_fixed": ([ctypes.POINTER(BlockDesc), _I], _I),
     "dp_block_desc_set_time_embedding": ([ctypes.POINTER(BlockDesc), _I], _I),
     "dp_block_workspace_size": ([ctypes.POINTER(BlockDesc)], _SZ),
     "dp_block_state_init": ([ctypes.POINTER(BlockDesc), ctypes.POINTER(BlockState), _V, _SZ, _V], _I),
@@ -326,6 +327,10 @@ def dp_block_desc_set_depth(d: BlockDesc, depth: int):
     return _check(lib().dp_block_desc_set_depth(ctypes.byref(d), depth))
 
 
+def dp_block_desc_set_context_fixed(d: BlockDesc, on: bool):
+    return _check(lib().dp_block_desc_set_context_fixed(ctypes.byref(d), int(on)))
+
+
 def dp_block_desc_set_unet(d: BlockDesc, base: int, depth0: int, depth1: int, depth2: int):
     return _check(lib().dp_block_desc_set_unet(ctypes.byref(d), base, depth0, depth1, depth2))
 
@@ -405,7 +410,7 @@ class Block:
 
     def __init__(self, kind, H, W, C, Cout=0, G=32, P=4, heads=0, dtype=BF16, silu=True,
                  eps=1e-5, w=1.0, device="cuda", stream=None, gn_stats=GN_STATS_CORRECTED,
-                 context=None, temb_dim=0, gn_fuse=False, depth=1, unet=None):
+                 context=None, temb_dim=0, gn_fuse=False, depth=1, unet=None, context_fixed=False):
         """``context`` = (ctx_len, ctx_dim, ff_inner) for TRANSFORMER and UNET_SDXL blocks;
         ``temb_dim`` the time-embedding width of a RESBLOCK or UNET_SDXL (0: none); ``unet`` =
         (base, depth0, depth1, depth2) of a UNET_SDXL block."""
@@ -417,6 +422,8 @@ class Block:
             dp_block_desc_set_context(self.desc, *context)
         if depth != 1:
             dp_block_desc_set_depth(self.desc, depth)
+        if context_fixed:
+            dp_block_desc_set_context_fixed(self.desc, True)
         if temb_dim:
             dp_block_desc_set_time_embedding(self.desc, temb_dim)
         if gn_stats != GN_STATS_CORRECTED:

@@ -59,6 +59,7 @@ struct Layout {
   size_t act, q, k[2], v[2], o;      // attention buffers
   size_t ha, hb, tn, q2, k2, v2, o2, ffh, ffg;   // TRANSFORMER: residual stream, LN output, cross, FF
   size_t kv_layer;                    // TRANSFORMER: bytes between layers' k/v ping-pong pairs
+  size_t kv2_layer;                   // TRANSFORMER: bytes between layers' context k/v
   size_t attn_ws;                     // balanced attention split: counters + partials
   size_t tbias;                       // RESBLOCK with a time embedding: conv1's step bias
   size_t gemm_ws;                     // split-K partials of the convs and projections
@@ -78,7 +79,7 @@ dp_block_desc sub_desc(const dp_block_desc* d, int kind, int H, int W, int C, in
   s.heads = heads;
   s.silu = silu;
   // kind-specific settings start from their defaults
-  s.ctx_len = s.ctx_dim = s.ff_inner = s.temb_dim = 0;
+  s.ctx_len = s.ctx_dim = s.ff_inner = s.temb_dim = s.ctx_fixed = 0;
   s.depth = 1;
   s.unet_base = 0;
   s.unet_depth[0] = s.unet_depth[1] = s.unet_depth[2] = 0;
@@ -118,6 +119,7 @@ std::vector<UStage> unet_stages(const dp_block_desc* d) {
       u.sub = sub_desc(d, DP_BLOCK_TRANSFORMER, H, W, ci, ci, ci / 64, 0);
       u.sub.ctx_len = d->ctx_len;
       u.sub.ctx_dim = d->ctx_dim;
+      u.sub.ctx_fixed = d->ctx_fixed;
       u.sub.ff_inner = 4 * ci;
     } else if (kind == US_OUT) {
       u.sub = sub_desc(d, DP_BLOCK_GN_CONV, H, W, ci, co, 0, 1);
@@ -267,8 +269,11 @@ Layout layout_of(const dp_block_desc* d) {
     for (int l = 1; l < d->depth; ++l) b.take(L.kv_layer);
     L.o = b.take(hw * C * e);
     L.q2 = b.take(hw * C * e);
+    // each layer's context keys and values (kept across steps when the context is fixed)
+    L.kv2_layer = 2 * ((Tk * C * e + 255) & ~static_cast<size_t>(255));
     L.k2 = b.take(Tk * C * e);
     L.v2 = b.take(Tk * C * e);
+    for (int l = 1; l < d->depth; ++l) b.take(L.kv2_layer);
     L.o2 = b.take(hw * C * e);
     L.ffh = b.take(hw * 2 * F * e);
     L.ffg = b.take(hw * F * e);
@@ -311,6 +316,8 @@ int desc_check(const dp_block_desc* d) {
   if (d && (d->depth < 1 || d->depth > 16 || (d->depth != 1 && d->kind != DP_BLOCK_TRANSFORMER)))
     return set_error(DP_ERR_INVALID_ARG, "block: depth %d (1..16, and above 1 only for TRANSFORMER)",
                      d->depth);
+  if (d && (d->ctx_fixed != 0 && d->ctx_fixed != 1))
+    return set_error(DP_ERR_INVALID_ARG, "block: fixed-context flag %d is not 0 or 1", d->ctx_fixed);
   if (d && d->gn_fuse != 0 && d->gn_fuse != 1)
     return set_error(DP_ERR_INVALID_ARG, "block: gn fusion flag %d is not 0 or 1", d->gn_fuse);
   if (!d) return set_error(DP_ERR_INVALID_ARG, "block: null descriptor");
@@ -430,7 +437,8 @@ double flops_of(const dp_block_desc* d) {
     return 2.0 * hw * C * C * 2.0 +                        // proj_in, proj_out
            d->depth * (2.0 * hw * C * C * 3.0 +             // wo, cq, co
                        2.0 * hw * 3.0 * C * C + 4.0 * hw * hw * C +   // q/k/v, self-attention
-                       2.0 * Tk * 2.0 * C * Cc + 4.0 * hw * Tk * C +  // context k/v, cross-attention
+                       (d->ctx_fixed ? 0.0 : 2.0 * Tk * 2.0 * C * Cc) +   // context k/v (kept when fixed)
+                       4.0 * hw * Tk * C +                             // cross-attention
                        2.0 * hw * 2.0 * F * C + 2.0 * hw * C * F);    // ff1, ff2
   }
   if (d->kind == DP_BLOCK_UNET_SDXL) {
@@ -482,7 +490,7 @@ bool gn_conv_fused(const dp_block_desc* d, int ch, int co) {
 }
 
 int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* out,
-              const void* const* w, int mode, cudaStream_t st, Plan* plan) {
+              const void* const* w, int mode, int first, cudaStream_t st, Plan* plan) {
   const Layout L = layout_of(d);
   const double e = d->dtype == DP_FP32 ? 4.0 : 2.0;
   const int f = cur ^ 1, o = cur;
@@ -670,8 +678,6 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
     void* q = at<void>(ws, L.q);
     void* ob = at<void>(ws, L.o);
     void* q2 = at<void>(ws, L.q2);
-    void* k2 = at<void>(ws, L.k2);
-    void* v2 = at<void>(ws, L.v2);
     void* o2 = at<void>(ws, L.o2);
     void* ffh = at<void>(ws, L.ffh);
     void* ffg = at<void>(ws, L.ffg);
@@ -713,8 +719,13 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
       if (rc) return rc;
       rc = lin(tn, lw[8], nullptr, nullptr, q2, nullptr, nullptr, T, C, C, C);
       if (rc) return rc;
-      rc = lin(ctx, lw[9], nullptr, nullptr, k2, v2, nullptr, Tk, 2 * C, Cc, C);
-      if (rc) return rc;
+      void* k2 = at<void>(ws, L.k2 + l * L.kv2_layer);
+      void* v2 = at<void>(ws, L.v2 + l * L.kv2_layer);
+      // a fixed context's keys and values are computed at the state's first step and kept
+      if (!d->ctx_fixed || first) {
+        rc = lin(ctx, lw[9], nullptr, nullptr, k2, v2, nullptr, Tk, 2 * C, Cc, C);
+        if (rc) return rc;
+      }
       if (plan) {
         plan->push(DP_KERNEL_ATTN, 4.0 * T * static_cast<double>(Tk) * C, (2.0 * T * C + 2.0 * Tk * C) * e);
       } else {
@@ -835,15 +846,15 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
         }
         sw.assign(uw, uw + stage_weight_count(u));
         sw.push_back(temb);
-        rc = step_impl(&u.sub, sub_ws, cur, in, dst, sw.data(), mode, st, plan);
+        rc = step_impl(&u.sub, sub_ws, cur, in, dst, sw.data(), mode, first, st, plan);
         if (rc) return rc;
       } else if (u.kind == US_TF) {
         sw.assign(uw, uw + stage_weight_count(u));
         sw.push_back(ctx);
-        rc = step_impl(&u.sub, sub_ws, cur, h, dst, sw.data(), mode, st, plan);
+        rc = step_impl(&u.sub, sub_ws, cur, h, dst, sw.data(), mode, first, st, plan);
         if (rc) return rc;
       } else {   // US_OUT
-        return step_impl(&u.sub, sub_ws, cur, h, out, uw, mode, st, plan);
+        return step_impl(&u.sub, sub_ws, cur, h, out, uw, mode, first, st, plan);
       }
       h = dst;
       if (u.skip) skips.push_back(h);
@@ -877,7 +888,7 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
     if (rc) return rc;
   }
   rc = step_impl(&m.rb1, at<void>(ws, L.rb1), cur, at<void>(ws, L.h0), at<void>(ws, L.d1[f]),
-                 take(weight_count(&m.rb1)), mode, st, plan);
+                 take(weight_count(&m.rb1)), mode, first, st, plan);
   if (rc) return rc;
   wc = take(2);
   if (!plan) {
@@ -890,10 +901,10 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
             H, W, kU1, kU1, 2);
   if (rc) return rc;
   rc = step_impl(&m.rb2, at<void>(ws, L.rb2), cur, at<void>(ws, L.h1), at<void>(ws, L.h2),
-                 take(weight_count(&m.rb2)), mode, st, plan);
+                 take(weight_count(&m.rb2)), mode, first, st, plan);
   if (rc) return rc;
   rc = step_impl(&m.at2, at<void>(ws, L.at2), cur, at<void>(ws, L.h2), at<void>(ws, L.d2[f]),
-                 take(weight_count(&m.at2)), mode, st, plan);
+                 take(weight_count(&m.at2)), mode, first, st, plan);
   if (rc) return rc;
   wc = take(2);
   if (!plan) {
@@ -906,18 +917,18 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
             H2, W2, kU2, kU2, 2);
   if (rc) return rc;
   rc = step_impl(&m.rb3, at<void>(ws, L.rb3), cur, at<void>(ws, L.h3), at<void>(ws, L.h4),
-                 take(weight_count(&m.rb3)), mode, st, plan);
+                 take(weight_count(&m.rb3)), mode, first, st, plan);
   if (rc) return rc;
   (void)H3;
   (void)W3;
   return step_impl(&m.at3, at<void>(ws, L.at3), cur, at<void>(ws, L.h4), out,
-                   take(weight_count(&m.at3)), mode, st, plan);
+                   take(weight_count(&m.at3)), mode, first, st, plan);
 }
 
 // Records the launches of one step of `d` in `mode`.
 int plan_of(const dp_block_desc* d, int mode, Plan* plan) {
   const std::vector<const void*> null_w(weight_count(d) + 1, nullptr);
-  return step_impl(d, nullptr, 0, nullptr, nullptr, null_w.data(), mode, nullptr, plan);
+  return step_impl(d, nullptr, 0, nullptr, nullptr, null_w.data(), mode, 0, nullptr, plan);
 }
 
 }  // namespace
@@ -947,6 +958,7 @@ int dp_block_desc_init(dp_block_desc* d, int kind, int H, int W, int C, int Cout
   d->temb_dim = 0;
   d->gn_fuse = 0;
   d->depth = 1;
+  d->ctx_fixed = 0;
   d->unet_base = kind == DP_BLOCK_UNET_SDXL ? 320 : 0;
   d->unet_depth[0] = kind == DP_BLOCK_UNET_SDXL ? 0 : 0;
   d->unet_depth[1] = kind == DP_BLOCK_UNET_SDXL ? 2 : 0;
@@ -1008,6 +1020,15 @@ int dp_block_desc_set_unet(dp_block_desc* d, int base, int depth0, int depth1, i
   for (int l = 0; l < 3; ++l) d->unet_depth[l] = dep[l];
   if (d->ctx_len == 0 || d->temb_dim == 0) return DP_OK;   // checked once both are set
   return dp::desc_check(d);
+}
+
+int dp_block_desc_set_context_fixed(dp_block_desc* d, int on) {
+  if (!d) return dp::set_error(DP_ERR_INVALID_ARG, "block: null descriptor");
+  if (d->kind != DP_BLOCK_TRANSFORMER && d->kind != DP_BLOCK_UNET_SDXL)
+    return dp::set_error(DP_ERR_INVALID_ARG, "block: a fixed context is only for TRANSFORMER and UNET_SDXL blocks");
+  if (on != 0 && on != 1) return dp::set_error(DP_ERR_INVALID_ARG, "block: fixed context must be 0 or 1");
+  d->ctx_fixed = on;
+  return DP_OK;
 }
 
 int dp_block_desc_set_gn_fusion(dp_block_desc* d, int on) {
@@ -1083,7 +1104,7 @@ int dp_block_step(const dp_block_desc* d, dp_block_state* s, const void* x, void
     // every kernel of this step reports a timed-out wait in the state's own word
     dp::StatusScope scope(reinterpret_cast<int*>(static_cast<char*>(s->workspace) +
                                                  dp::layout_of(d).status));
-    rc = dp::step_impl(d, s->workspace, s->cur, x, out, weights, mode,
+    rc = dp::step_impl(d, s->workspace, s->cur, x, out, weights, mode, s->steps_done == 0 ? 1 : 0,
                        static_cast<cudaStream_t>(stream), nullptr);
   }
   if (rc) return rc;

@@ -528,6 +528,7 @@ typedef struct dp_block_desc {
   int depth;      /* TRANSFORMER: basic transformer layers (default 1) */
   int unet_base;  /* UNET_SDXL: level widths base, 2 base, 4 base (320) */
   int unet_depth[3]; /* UNET_SDXL: transformer depth per level (0, 2, 10) */
+  int ctx_fixed;  /* TRANSFORMER, UNET_SDXL: 1 = the context is the same every step */
 } dp_block_desc;
 
 /*
@@ -550,6 +551,19 @@ DP_API int dp_block_desc_set_context(dp_block_desc* d, int ctx_len, int ctx_dim,
  * DP_ERR_INVALID_ARG otherwise or for another kind.
  */
 DP_API int dp_block_desc_set_depth(dp_block_desc* d, int depth);
+
+/*
+ * TRANSFORMER and UNET_SDXL blocks: on = 1 declares that the text context is
+ * the same at every step of the state (a prompt's encoding is, for all the
+ * denoising steps of one image).  Each layer's context keys and values are
+ * then computed at the state's first step (steps_done == 0) and kept in the
+ * workspace; later steps skip those projections (one launch per layer fewer;
+ * the launch plan and dp_block_flops describe the later steps).  The caller
+ * must not change the context's contents until dp_block_state_init starts a
+ * new state; a changed context is not detected.  Default 0 (recomputed every
+ * step).  DP_ERR_INVALID_ARG for another kind or on not in {0, 1}.
+ */
+DP_API int dp_block_desc_set_context_fixed(dp_block_desc* d, int on);
 
 /*
  * UNET_SDXL blocks: one whole denoising step of an SDXL-shaped U-Net over all

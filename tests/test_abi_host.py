@@ -424,6 +424,23 @@ def test_transformer_depth_on_the_host(B):
         B.dp_block_workspace_size(r)
 
 
+def test_fixed_context_on_the_host(B):
+    """A fixed context drops each layer's context k/v projection from the (later) steps' plan
+    and flops, and is only for TRANSFORMER and UNET_SDXL blocks."""
+    d = B.dp_block_desc_init(B.TRANSFORMER, 32, 32, 320, 320, 32, 4, 5, B.BF16, 0, 1e-5, 1.0)
+    B.dp_block_desc_set_context(d, 77, 128, 1280)
+    B.dp_block_desc_set_depth(d, 3)
+    n, fl = B.dp_block_launch_count(d), B.dp_block_flops(d)
+    B.dp_block_desc_set_context_fixed(d, True)
+    assert B.dp_block_launch_count(d) == n - 3
+    assert abs(fl - B.dp_block_flops(d) - 3 * 2.0 * 77 * 2 * 320 * 128) < 1e-6 * fl
+    with pytest.raises(B.DPError):
+        B.dp_block_desc_set_context_fixed(d, 2)
+    r = B.dp_block_desc_init(B.RESBLOCK, 32, 32, 320, 320, 32, 4, 0, B.BF16, 1, 1e-5, 1.0)
+    with pytest.raises(B.DPError, match="TRANSFORMER"):
+        B.dp_block_desc_set_context_fixed(r, True)
+
+
 def test_transformer_depth_workload_marshals(B):
     """Seeded weights of a depth-2 transformer workload marshal into 7 + 18 * 2 pointers (the
     context last), and its first layer's weights are those of the depth-1 workload."""

@@ -88,15 +88,18 @@ def test_transformer_block():
     assert blk.status() == 0 and B.dp_device_status() == 0
 
 
-def test_transformer_block_depth2():
+@pytest.mark.parametrize("context_fixed", [False, True])
+def test_transformer_block_depth2(context_fixed):
     """The same block with two basic layers, each with its own stale keys and values: a sync
     step and three displaced steps of a drifting input against the oracle, held end to end by
-    check_chain (the chain of bf16-stored stages is twice as long)."""
+    check_chain (the chain of bf16-stored stages is twice as long).  With a fixed context the
+    layers' context keys and values come from the first step (the oracle recomputes them every
+    step: the same values, as the context does not change)."""
     d, wts, ctx, g, rnd, bf = _transformer_case(depth=2)
     C, H, W, P, G, heads = d["C"], d["H"], d["W"], d["P"], d["G"], d["heads"]
     dev_w = block_weights("transformer", wts, depth=2) + [ctx.to(torch.bfloat16).cuda()]
     blk = B.Block(B.TRANSFORMER, H, W, C, C, G, P, heads, B.BF16, False, 1e-5, 1.0,
-                  context=(d["Tk"], d["Cc"], d["F"]), depth=2)
+                  context=(d["Tk"], d["Cc"], d["F"]), depth=2, context_fixed=context_fixed)
     assert len(dev_w) == B.dp_block_weight_count(blk.desc)
     w64 = {n: v.double().numpy() for n, v in wts.items()}
     c64 = ctx.double().numpy()

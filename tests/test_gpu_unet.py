@@ -89,9 +89,12 @@ def test_unet_sdxl_plan_matches_the_stages():
     assert len(dw) + 2 == B.dp_block_weight_count(blk.desc)
 
 
-def test_unet_sdxl_step():
+@pytest.mark.parametrize("context_fixed", [False, True])
+def test_unet_sdxl_step(context_fixed):
     """The whole U-Net step on the GPU against the oracle: a sync step, three displaced steps
-    of a drifting latent and a naive step of a fresh state, every output compared."""
+    of a drifting latent and a naive step of a fresh state, every output compared (with a
+    fixed context, every transformer layer's context keys and values come from the first
+    step)."""
     u = UNET
     wl = _unet_workload()
     wts = synth.make_weights(wl, random_affine=True)
@@ -111,7 +114,7 @@ def test_unet_sdxl_step():
     def make_block():
         return B.Block(B.UNET_SDXL, u["H"], u["W"], u["C"], u["C"], u["G"], u["P"], 0, B.BF16, True,
                        1e-5, 1.0, context=(u["Tk"], u["Cc"], 0), temb_dim=u["Ct"],
-                       unet=(u["base"],) + u["depths"])
+                       unet=(u["base"],) + u["depths"], context_fixed=context_fixed)
 
     blk = make_block()
     st, st_exact = {}, {}
