@@ -75,6 +75,7 @@ _SIGS = {
     "dp_layernorm": ([_V, _V, _V, _V, _I, _I, _F, _V], _I),
     "dp_geglu": ([_V, _V, _I, _I, _V], _I),
     "dp_concat_channels": ([_V, _V, _V, ctypes.c_size_t, _I, _I, _I, _V], _I),
+    "dp_linear_geglu": ([_V, _V, _V, _V, _I, _I, _I, _V], _I),
     "dp_upsample_nearest2x": ([_V, _V, _I, _I, _I, _I, _V], _I),
     "dp_time_embedding_bias": ([_V, _V, _V, _V, _V, _I, _I, _V], _I),
     "dp_ddim_step": ([_V, _V, _V, _SZ, ctypes.c_double, ctypes.c_double, _I, _V], _I),
@@ -264,6 +265,10 @@ def dp_layernorm(x, y, gamma, beta, T, C, eps, stream=None):
 
 def dp_geglu(h, y, T, F, stream=None):
     return _check(lib().dp_geglu(_p(h), _p(y), T, F, _s(stream)))
+
+
+def dp_linear_geglu(x, weight, bias, y, M, F, K, stream=None):
+    return _check(lib().dp_linear_geglu(_p(x), _p(weight), _p(bias), _p(y), M, F, K, _s(stream)))
 
 
 def dp_concat_channels(a, b, out, npix, Ca, Cb, dtype=BF16, stream=None):

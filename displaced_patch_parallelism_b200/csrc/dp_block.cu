@@ -738,13 +738,24 @@ int step_impl(const dp_block_desc* d, void* ws, int cur, const void* x, void* ou
       // gated feed-forward
       rc = ln(cur, tn, lw[12], lw[13]);
       if (rc) return rc;
-      rc = lin(tn, lw[14], lw[15], nullptr, ffh, nullptr, nullptr, T, 2 * Fi, C, 2 * Fi);
-      if (rc) return rc;
-      if (plan) {
-        plan->push(DP_KERNEL_GEGLU, 0.0, 3.0 * T * Fi * e);
+      // ff1 with the gated GELU in its epilogue when the pair kernel tiles it;
+      // otherwise ff1, then the interleaved GEGLU pass
+      if (linear_geglu_fusable(T, Fi, C)) {
+        if (plan) {
+          plan->push(DP_KERNEL_LINEAR, 2.0 * T * 2.0 * Fi * C, (static_cast<double>(T) * C + 1.0 * T * Fi) * e);
+        } else {
+          rc = linear_geglu_launch(tn, lw[14], static_cast<const float*>(lw[15]), ffg, T, Fi, C, st);
+          if (rc) return rc;
+        }
       } else {
-        rc = dp_geglu(ffh, ffg, T, Fi, st);
+        rc = lin(tn, lw[14], lw[15], nullptr, ffh, nullptr, nullptr, T, 2 * Fi, C, 2 * Fi);
         if (rc) return rc;
+        if (plan) {
+          plan->push(DP_KERNEL_GEGLU, 0.0, 3.0 * T * Fi * e);
+        } else {
+          rc = geglu_launch(ffh, ffg, T, Fi, true, st);
+          if (rc) return rc;
+        }
       }
       rc = lin(ffg, lw[16], lw[17], cur, other, nullptr, nullptr, T, C, Fi, C);
       if (rc) return rc;

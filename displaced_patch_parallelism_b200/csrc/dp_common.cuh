@@ -516,6 +516,11 @@ __device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t w) {
   return f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
 }
 
+// Exact GELU, x * Phi(x) = x (1 + erf(x / sqrt 2)) / 2: the gated feed-forward's
+// activation, in the stand-alone GEGLU kernel and in the projection epilogue
+// that fuses it.
+__device__ __forceinline__ float gelu_exact(float x) { return 0.5f * x * (1.f + erff(x * 0.70710678118654752f)); }
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

@@ -72,6 +72,11 @@ struct GemmParams {
   int gn_cg;               // channels per group
   int gn_silu;
   void* a_next;            // [H][W][Cin]: receives the normalised band-edge rows, or null
+  // Pair kernels, plain A only: the epilogue applies the gated GELU.  The N =
+  // 2F accumulator columns hold value and gate interleaved in blocks of 16
+  // (each 32-column chunk: 16 values, then their 16 gates); tmO[0] maps the
+  // [M][F] output as 16-column boxes of 32 rows, unswizzled.
+  int geglu;
 };
 
 // k-blocks [*kb0, *kb1) of run `r` of `splits` over `kb` k-blocks.
@@ -579,6 +584,26 @@ __device__ __forceinline__ bool pair_epilogue_tile(const GemmParams& p, uint32_t
     const float* bb = e.bias + ch * 32;
 #pragma unroll
     for (int j = 0; j < 32; ++j) v[j] += bb[j];
+    if (p.geglu) {
+      // 16 outputs a * gelu(g) of this row: 32 bytes, one 16-column box
+      uint8_t* ob = e.out + (e.oi & 1u) * kEpiSlot;
+      if (lane == 0) bulk_wait_read_1();   // the store that last used this slot has read it
+      __syncwarp();
+      uint32_t o[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        o[j] = pack_bf16x2(v[2 * j] * gelu_exact(v[16 + 2 * j]), v[2 * j + 1] * gelu_exact(v[17 + 2 * j]));
+      *reinterpret_cast<uint4*>(ob + lane * 32) = make_uint4(o[0], o[1], o[2], o[3]);
+      *reinterpret_cast<uint4*>(ob + lane * 32 + 16) = make_uint4(o[4], o[5], o[6], o[7]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(om, ob, (b.x + ch * 32) / 2, b.y);
+        bulk_commit();
+      }
+      ++e.oi;
+      continue;
+    }
     if (rrow) {
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj) {
@@ -1829,6 +1854,54 @@ int linear_launch(const void* x, const void* weight, const float* bias, const vo
   return launch_gemm(p, BN, false, stream);
 }
 
+bool linear_geglu_fusable(int M, int F, int K) {
+  return M > 0 && F > 0 && K > 0 && K % 64 == 0 && F % 16 == 0 && (2 * F) % 160 == 0;
+}
+
+// y = a * gelu(g) of the projection [a|g] = x W^T + b, in one pair-kernel launch
+// whose epilogue applies the gated GELU (W's rows interleaved in blocks of 16).
+int linear_geglu_launch(const void* x, const void* weight, const float* bias, void* y, int M, int F, int K,
+                        cudaStream_t stream) {
+  if (!linear_geglu_fusable(M, F, K)) return set_error(DP_ERR_UNSUPPORTED, "linear geglu: shape not fusable");
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  const int N = 2 * F;
+  p.splits = 1;
+  p.a_mode = 0;
+  p.M = M;
+  p.m_tiles = (M + 127) / 128;
+  p.k_blocks = K / 64;
+  p.N = N;
+  p.split = N;
+  p.ld_out = F;
+  p.bias = bias;
+  p.out0 = y;
+  p.geglu = 1;
+  p.status = device_status_ptr();
+  int bn_single = 0, splits = 1;
+  int pw = pick_pair(p.m_tiles, N, N, p.k_blocks, false, &bn_single, &splits);
+  if (!pw) pw = N % 320 == 0 ? 320 : 160;   // the single-CTA kernel has no gated epilogue
+  p.n_tiles = N / pw;
+  uint64_t adims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
+  uint64_t astr[1] = {static_cast<uint64_t>(K) * 2};
+  uint32_t abox[2] = {64, 128};
+  int rc = encode_tmap(&p.tmA0, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), adims, astr, abox,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc) return rc;
+  uint64_t bdims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N)};
+  uint32_t bbox[2] = {64, 80};
+  rc = encode_tmap(&p.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(weight), bdims, astr, bbox,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc) return rc;
+  uint64_t odims[2] = {static_cast<uint64_t>(F), static_cast<uint64_t>(M)};
+  uint64_t ostr[1] = {static_cast<uint64_t>(F) * 2};
+  uint32_t obox[2] = {16, 32};
+  rc = encode_tmap(&p.tmO[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, y, odims, ostr, obox,
+                   CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (rc) return rc;
+  return pw == 320 ? launch_pair<160, 2>(p, stream) : launch_pair<160, 1>(p, stream);
+}
+
 int conv3x3_validate(const void* a_fresh, const void* a_stale, const void* weight,
                      const void* residual, const void* out, int H, int W, int Cin, int Cout,
                      int stride, int P, int mode, int dtype) {
@@ -1906,6 +1979,21 @@ int dp_conv3x3_halo(const void* a_fresh, const void* a_stale, const void* weight
   return dp::conv3x3_launch(a_fresh, a_stale, weight, bias, residual, out, H, W, Cin, Cout, stride,
                             P, mode, dtype, workspace, workspace_bytes,
                             static_cast<cudaStream_t>(stream));
+}
+
+int dp_linear_geglu(const void* x, const void* weight, const float* bias, void* y, int M, int F, int K,
+                    void* stream) {
+  if (!x || !weight || !y) return dp::set_error(DP_ERR_INVALID_ARG, "linear geglu: null pointer");
+  if (M <= 0 || F <= 0 || K <= 0) return dp::set_error(DP_ERR_INVALID_ARG, "linear geglu: bad size");
+  if (!dp::linear_geglu_fusable(M, F, K))
+    return dp::set_error(DP_ERR_UNSUPPORTED, "linear geglu: needs K %% 64 == 0, F %% 16 == 0 and 2F %% 160 == 0");
+  if (!dp::aligned16(x) || !dp::aligned16(weight) || !dp::aligned16(y) || (bias && !dp::aligned16(bias)))
+    return dp::set_error(DP_ERR_UNSUPPORTED, "linear geglu: pointers must be 16-byte aligned");
+  const char* xb = static_cast<const char*>(x);
+  const char* yb = static_cast<const char*>(y);
+  const size_t xbytes = static_cast<size_t>(M) * K * 2, ybytes = static_cast<size_t>(M) * F * 2;
+  if (xb < yb + ybytes && yb < xb + xbytes) return dp::set_error(DP_ERR_INVALID_ARG, "linear geglu: y overlaps x");
+  return dp::linear_geglu_launch(x, weight, bias, y, M, F, K, static_cast<cudaStream_t>(stream));
 }
 
 int dp_linear(const void* x, const void* weight, const float* bias, const void* residual,

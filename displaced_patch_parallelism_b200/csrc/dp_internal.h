@@ -79,6 +79,12 @@ int attn_launch_tk(const void* q, const void* kf, const void* vf, const void* ks
 int attn_launch(const void* q, const void* kf, const void* vf, const void* ks, const void* vs,
                 void* o, int T, int heads, int P, float scale, int mode, void* workspace,
                 size_t workspace_bytes, cudaStream_t stream);
+// the feed-forward's projection with the gated GELU in its epilogue (weight and
+// bias rows interleaved in blocks of 16), and the stand-alone gated GELU
+bool linear_geglu_fusable(int M, int F, int K);
+int linear_geglu_launch(const void* x, const void* weight, const float* bias, void* y, int M, int F, int K,
+                        cudaStream_t stream);
+int geglu_launch(const void* h, void* y, int T, int F, bool interleaved, cudaStream_t st);
 void recorder_begin(void* const* events, int n);
 int recorder_end();
 int copy_launch(const void* src, void* dst, size_t bytes, cudaStream_t stream);

@@ -88,8 +88,11 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const __nv_bfloat16* __r
   }
 }
 
-__device__ __forceinline__ float gelu_exact(float x) { return 0.5f * x * (1.f + erff(x * 0.70710678118654752f)); }
-
+// IL = false: h's row is [a (F values) | g (F values)].  IL = true: value and
+// gate columns interleaved in blocks of 16 (columns 32k..32k+15 are a for
+// outputs 16k..16k+15, columns 32k+16..32k+31 the matching g), the layout a
+// transformer block's feed-forward projection writes.
+template <bool IL>
 __global__ void __launch_bounds__(256) geglu_kernel(const __nv_bfloat16* __restrict__ h,
                                                     __nv_bfloat16* __restrict__ y, int T, int F) {
   griddep_wait();
@@ -100,7 +103,9 @@ __global__ void __launch_bounds__(256) geglu_kernel(const __nv_bfloat16* __restr
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
     const size_t t = i / fv, c = i - t * fv;
     const uint4* row = reinterpret_cast<const uint4*>(h + t * 2 * F);
-    const uint4 a = row[c], g = row[fv + c];
+    // 8 outputs per vector: IL takes the half-block c & 1 of block c / 2
+    const uint4 a = IL ? row[4 * (c >> 1) + (c & 1)] : row[c];
+    const uint4 g = IL ? row[4 * (c >> 1) + 2 + (c & 1)] : row[fv + c];
     const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wg[4] = {g.x, g.y, g.z, g.w};
     uint32_t o[4];
 #pragma unroll
@@ -111,6 +116,22 @@ __global__ void __launch_bounds__(256) geglu_kernel(const __nv_bfloat16* __restr
     }
     reinterpret_cast<uint4*>(y + t * F)[c] = make_uint4(o[0], o[1], o[2], o[3]);
   }
+}
+
+int geglu_launch(const void* h, void* y, int T, int F, bool interleaved, cudaStream_t st) {
+  const size_t n = static_cast<size_t>(T) * (F / 8);
+  size_t blocks = (n + 255) / 256;
+  const size_t cap = static_cast<size_t>(num_sms()) * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks == 0) blocks = 1;
+  mark_launch(st);
+  const auto* hb = static_cast<const __nv_bfloat16*>(h);
+  auto* yb = static_cast<__nv_bfloat16*>(y);
+  if (interleaved)
+    return launch_kernel(geglu_kernel<true>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, false,
+                         "geglu launch", hb, yb, T, F);
+  return launch_kernel(geglu_kernel<false>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, false,
+                       "geglu launch", hb, yb, T, F);
 }
 
 }  // namespace dp
@@ -162,15 +183,7 @@ int dp_geglu(const void* h, void* y, int T, int F, void* stream) {
   const char* yb = static_cast<const char*>(y);
   const size_t hbytes = static_cast<size_t>(T) * 2 * F * 2, ybytes = static_cast<size_t>(T) * F * 2;
   if (hb < yb + ybytes && yb < hb + hbytes) return dp::set_error(DP_ERR_INVALID_ARG, "geglu: y overlaps h");
-  const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t n = static_cast<size_t>(T) * (F / 8);
-  size_t blocks = (n + 255) / 256;
-  const size_t cap = static_cast<size_t>(dp::num_sms()) * 8;
-  if (blocks > cap) blocks = cap;
-  dp::mark_launch(st);
-  return dp::launch_kernel(dp::geglu_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, false,
-                           "geglu launch", static_cast<const __nv_bfloat16*>(h),
-                           static_cast<__nv_bfloat16*>(y), T, F);
+  return dp::geglu_launch(h, y, T, F, false, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

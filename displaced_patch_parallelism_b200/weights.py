@@ -2,8 +2,9 @@
 
 Layout changes only (no arithmetic of the method): conv filters go from
 (Cout, Cin, 3, 3) to [Cout][3][3][Cin]; the q, k and v projection matrices are
-stacked into one [3C][C] matrix so a single GEMM produces all three; GroupNorm
-scale/shift and biases are fp32.
+stacked into one [3C][C] matrix so a single GEMM produces all three; a
+transformer's gated feed-forward projection has its value and gate rows
+interleaved in blocks of 16; GroupNorm scale/shift and biases are fp32.
 """
 from __future__ import annotations
 
@@ -15,6 +16,15 @@ import torch
 def _t(a, dtype, device):
     t = a if isinstance(a, torch.Tensor) else torch.as_tensor(a)
     return t.to(torch.float32).to(dtype).contiguous().to(device)
+
+
+def _interleave16(w):
+    """Rows [a (F rows) | g (F rows)] of a gated feed-forward projection -> blocks of 16:
+    rows 32k..32k+15 are a rows 16k..16k+15, rows 32k+16..32k+31 the matching g rows."""
+    t = w if isinstance(w, torch.Tensor) else torch.as_tensor(w)
+    F = t.shape[0] // 2
+    rest = tuple(t.shape[1:])
+    return t.reshape(2, F // 16, 16, *rest).transpose(0, 1).reshape(2 * F, *rest)
 
 
 def _conv(w, dtype, device):
@@ -64,8 +74,8 @@ def block_weights(kind: str, wts: Dict, dtype: torch.dtype = torch.bfloat16, dev
                     _t(cat(g(p + "bq"), g(p + "bk"), g(p + "bv")), f32, device), m(p + "wo"), v(p + "bo"),
                     v(p + "ln2_g"), v(p + "ln2_b"), m(p + "cq_w"),
                     _t(cat(g(p + "ck_w"), g(p + "cv_w")), dtype, device), m(p + "co_w"), v(p + "co_b"),
-                    v(p + "ln3_g"), v(p + "ln3_b"), m(p + "ff1_w"), v(p + "ff1_b"), m(p + "ff2_w"),
-                    v(p + "ff2_b")]
+                    v(p + "ln3_g"), v(p + "ln3_b"), _t(_interleave16(g(p + "ff1_w")), dtype, device),
+                    _t(_interleave16(g(p + "ff1_b")), f32, device), m(p + "ff2_w"), v(p + "ff2_b")]
         return out + [m("proj_out_w"), v("proj_out_b")]
     if kind == "unet_sdxl":
         raise ValueError("use unet_sdxl_weights for a UNET_SDXL block")

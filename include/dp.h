@@ -445,6 +445,21 @@ DP_API int dp_layernorm(const void* x, void* y, const float* gamma, const float*
 DP_API int dp_geglu(const void* h, void* y, int T, int F, void* stream);
 
 /* ------------------------------------------------------------------------
+ * The gated feed-forward's first projection with the gated GELU applied in
+ * its epilogue: y[t][c] = a * gelu(g), [a | g] = x W^T + b, without storing
+ * the 2F-wide projection.  W's rows (and b's entries) come interleaved in
+ * blocks of 16: rows 32k..32k+15 are the value rows 16k..16k+15 and rows
+ * 32k+16..32k+31 the matching gate rows (the layout of a TRANSFORMER block's
+ * ff1_w and ff1_b).
+ *   x [M][K] bf16, W [2F][K] bf16, b [2F] fp32 or NULL, y [M][F] bf16, device,
+ *   16-byte aligned; y must not overlap x.  Needs K % 64 == 0, F % 16 == 0 and
+ *   2F % 160 == 0 (the 2-SM tensor-core tiles); DP_ERR_UNSUPPORTED otherwise
+ *   (a block then runs the projection and an interleaved GEGLU pass).
+ * ---------------------------------------------------------------------- */
+DP_API int dp_linear_geglu(const void* x, const void* weight, const float* bias, void* y, int M,
+                           int F, int K, void* stream);
+
+/* ------------------------------------------------------------------------
  * The up path of an SDXL-shaped U-Net (the pages' SDXL model, "DistriFusion",
  * atlas.scime.ai summary, Key results): each up ResBlock takes the running
  * tensor concatenated with a skip connection, and each up level ends in a
@@ -673,8 +688,11 @@ DP_API int dp_block_state_init(const dp_block_desc* d, dp_block_state* s, void* 
  *             of the `depth` layers: ln1_g[C], ln1_b[C], wqkv[3C][C], bqkv[3C],
  *             wo[C][C], bo[C], ln2_g[C], ln2_b[C], cq_w[C][C], ckv_w[2C][Cctx]
  *             (the context's k and v matrices stacked), co_w[C][C], co_b[C],
- *             ln3_g[C], ln3_b[C], ff1_w[2F][C] (value half, then gate half),
- *             ff1_b[2F], ff2_w[C][F], ff2_b[C]; then proj_out_w[C][C],
+ *             ln3_g[C], ln3_b[C], ff1_w[2F][C] and ff1_b[2F] (value and gate
+ *             rows interleaved in blocks of 16, as dp_linear_geglu takes them:
+ *             the block fuses the gated GELU into ff1 when dp_linear_geglu's
+ *             shape rule holds and otherwise runs ff1 and a GEGLU pass over the
+ *             same layout), ff2_w[C][F], ff2_b[C]; then proj_out_w[C][C],
  *             proj_out_b[C], and the step's context [ctx_len][ctx_dim] bf16
  *             (7 + 18 depth pointers; matrices bf16, vectors fp32; the biases may
  *             be NULL)

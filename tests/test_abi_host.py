@@ -291,9 +291,10 @@ def test_transformer_block_plan_on_the_host(B):
     B.dp_block_desc_set_context(d, 77, 2048, 2560)
     assert B.dp_block_weight_count(d) == 25
     kinds = [B.dp_block_launch_info(d, B.DISPLACED, i)[0] for i in range(B.dp_block_launch_count(d))]
+    # ff1 carries the gated GELU in its epilogue (2F = 5120 is a whole number of pair tiles)
     assert [k for k in kinds if k != "splitk_finish"] == [
         "gn_cluster", "linear", "layernorm", "linear", "attn", "linear", "layernorm", "linear", "linear",
-        "attn", "linear", "layernorm", "linear", "geglu", "linear", "linear"]
+        "attn", "linear", "layernorm", "linear", "linear", "linear"]
     fl = sum(B.dp_block_launch_info(d, B.DISPLACED, i)[1] for i in range(B.dp_block_launch_count(d)))
     assert abs(fl - B.dp_block_flops(d)) < 1e-6 * fl
     assert B.dp_block_workspace_size(d) > 64 * 64 * 2560 * 2 * 2
@@ -409,7 +410,7 @@ def test_transformer_depth_on_the_host(B):
     assert B.dp_block_weight_count(d) == 7 + 18 * 3
     kinds = [B.dp_block_launch_info(d, B.DISPLACED, i)[0] for i in range(B.dp_block_launch_count(d))]
     layer = ["layernorm", "linear", "attn", "linear", "layernorm", "linear", "linear", "attn", "linear",
-             "layernorm", "linear", "geglu", "linear"]
+             "layernorm", "linear", "linear"]
     assert [k for k in kinds if k != "splitk_finish"] == ["gn_cluster", "linear"] + 3 * layer + ["linear"]
     T, C = 32 * 32, 320
     proj = 2 * 2.0 * T * C * C
@@ -422,6 +423,26 @@ def test_transformer_depth_on_the_host(B):
     r.depth = 2                                     # written past the setter: rejected at use
     with pytest.raises(B.DPError, match="depth"):
         B.dp_block_workspace_size(r)
+
+
+def test_feed_forward_fusion_rule_on_the_host(B):
+    """The gated GELU rides in ff1's epilogue when 2F is a whole number of 160-column pair
+    tiles (SDXL: F = 4C, C a multiple of 320 here); otherwise ff1 and a GEGLU pass run; the
+    fused call rejects other shapes before any launch."""
+    def kinds(C, F):
+        d = B.dp_block_desc_init(B.TRANSFORMER, 32, 32, C, C, 32, 2, C // 64, B.BF16, 0, 1e-5, 1.0)
+        B.dp_block_desc_set_context(d, 77, 128, F)
+        return [B.dp_block_launch_info(d, B.DISPLACED, i)[0] for i in range(B.dp_block_launch_count(d))]
+    assert "geglu" not in kinds(640, 2560) and "geglu" not in kinds(320, 1280)
+    assert kinds(128, 512).count("geglu") == 1 and kinds(256, 1024).count("geglu") == 1
+    A = 1 << 20
+    for args, code in [((0, 2 * A, 0, 3 * A, 128, 1280, 320), B.DP_ERR_INVALID_ARG),   # null x
+                       ((A, 2 * A, 0, 3 * A, 128, 512, 320), B.DP_ERR_UNSUPPORTED),   # 2F % 160
+                       ((A, 2 * A, 0, 3 * A, 128, 1280, 96), B.DP_ERR_UNSUPPORTED),   # K % 64
+                       ((A, 2 * A, 0, A + 64, 128, 1280, 320), B.DP_ERR_INVALID_ARG)]:  # y overlaps x
+        with pytest.raises(B.DPError) as e:
+            B.dp_linear_geglu(*args, stream=0)
+        assert e.value.code == code, args
 
 
 def test_fixed_context_on_the_host(B):

@@ -119,6 +119,25 @@ def test_transformer_block_depth2(context_fixed):
     assert blk.status() == 0 and B.dp_device_status() == 0
 
 
+@pytest.mark.parametrize("M,F,K", [(1000, 1280, 320), (333, 80, 64), (1024, 2560, 640), (77, 160, 128)])
+def test_linear_geglu_fused(M, F, K):
+    """ff1 with the gated GELU in its epilogue (value and gate rows interleaved in blocks of
+    16): against the oracle's projection followed by a * gelu(g), at the stated bar; ragged M,
+    both pair-tile widths, one and several k-blocks."""
+    from displaced_patch_parallelism_b200.weights import _interleave16
+    r = np.random.default_rng(150 + M + F)
+    x = O.store(r.standard_normal((M, K)), "bf16")
+    w1 = O.store(r.standard_normal((2 * F, K)) * K ** -0.5, "bf16")
+    b1 = (0.2 * r.standard_normal(2 * F)).astype(np.float32).astype(np.float64)
+    y = torch.empty(M, F, dtype=torch.bfloat16, device="cuda")
+    B.dp_linear_geglu(dev_mat(x), dev_mat(_interleave16(torch.from_numpy(w1)).numpy()),
+                      dev_f32(_interleave16(torch.from_numpy(b1)).numpy()), y, M, F, K)
+    torch.cuda.synchronize()
+    h = O.linear(x, w1, b1)
+    ref = h[:, :F] * O.gelu(h[:, F:])
+    check(host(y), ref, what=f"fused ff1 + GEGLU {M}x{F}x{K}", storage_rel=BF16_HALF_ULP)
+
+
 def test_transformer_stages():
     """Every stage of the transformer block on its own: the GPU call of that stage fed the
     oracle's bf16-stored output of the stage before, against the oracle's unrounded output of
