@@ -479,6 +479,28 @@ def time_steps(run, steps, flush, dist, sampler=None):
     return [ev0[k].elapsed_time(ev1[k]) for k in range(steps)], wall, clocks
 
 
+def time_graph(run, steps, flush):
+    """Device time (ms) of ``steps`` displaced steps replayed from the library's CUDA graphs
+    (dp_block_graph_*: one captured step per ping-pong parity, the first input buffer fixed in
+    them), an event pair around each, L2 flushed between steps as in time_steps."""
+    import torch
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    with torch.cuda.stream(s):
+        g = run.blk.graph(run.dev_x[0], run.out, run.dw, run.B.DISPLACED, s)
+        g.launch(s)                      # first replay: uploads the graphs
+        for k in range(steps):
+            if run.flush_between:
+                flush()
+            ev[k][0].record(s)
+            g.launch(s)
+            ev[k][1].record(s)
+    torch.cuda.synchronize()
+    g.close()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
 def breakdown(run, steps, flush, peaks):
     """Per-kernel roles of the step: mean duration, share, rate; and the dominant role's
     roofline.  An event before every launch (dp_block_step_timed) keeps kernels from
@@ -662,6 +684,7 @@ def run_ours(args, wl):
                 ms, _, _ = time_steps(r, args.steps, flush, dist)
                 t_ms = max_over_ranks(sum(ms), dist, dev)
                 k, rf, g = breakdown(r, args.steps, flush, peaks)
+                g_ms = max_over_ranks(sum(time_graph(r, args.steps, flush)), dist, dev)
             except B.DPError as e:          # a host-side rejection; recorded, not fatal
                 extra[name] = {"error": str(e)}
                 continue
@@ -672,6 +695,10 @@ def run_ours(args, wl):
                            "roofline": {kk: rf[kk] for kk in ("bound", "kernel", "achieved",
                                                               "peak", "unit", "frac")},
                            "kernels": k, "groupnorm": g,
+                           "graph": {"ms_per_step": round(g_ms / args.steps, 5),
+                                     "value": round(job_tflops(ws, r.flops, args.steps, g_ms), 3),
+                                     "unit": "TFLOP/s",
+                                     "how": "the same steps replayed from dp_block_graph_* CUDA graphs"},
                            "gpu_launches": r.blk.launches * args.steps}
             del r
             torch.cuda.empty_cache()

@@ -94,6 +94,10 @@ _SIGS = {
     "dp_block_desc_set_time_embedding": ([ctypes.POINTER(BlockDesc), _I], _I),
     "dp_block_workspace_size": ([ctypes.POINTER(BlockDesc)], _SZ),
     "dp_block_state_init": ([ctypes.POINTER(BlockDesc), ctypes.POINTER(BlockState), _V, _SZ, _V], _I),
+    "dp_block_graph_create": ([ctypes.POINTER(BlockDesc), ctypes.POINTER(BlockState), _V, _V,
+                               ctypes.POINTER(ctypes.c_void_p), _I, _I, _V, ctypes.POINTER(ctypes.c_void_p)], _I),
+    "dp_block_graph_launch": ([_V, ctypes.POINTER(BlockState), _V], _I),
+    "dp_block_graph_destroy": ([_V], _I),
     "dp_block_step": ([ctypes.POINTER(BlockDesc), ctypes.POINTER(BlockState), _V, _V,
                        ctypes.POINTER(_V), _I, _I, _V], _I),
     "dp_block_flops": ([ctypes.POINTER(BlockDesc)], ctypes.c_double),
@@ -366,6 +370,24 @@ def dp_block_step(d: BlockDesc, s: BlockState, x, out, weights: Sequence, mode: 
                                       len(weights), mode, _s(stream)))
 
 
+def dp_block_graph_create(d: BlockDesc, s: BlockState, x, out, weights: Sequence, mode: int,
+                          stream=None) -> int:
+    """The opaque graph handle (an address) of one captured step per ping-pong parity."""
+    arr = (ctypes.c_void_p * len(weights))(*[_p(w) for w in weights])
+    h = ctypes.c_void_p(0)
+    _check(lib().dp_block_graph_create(ctypes.byref(d), ctypes.byref(s), _p(x), _p(out), arr, len(weights),
+                                       mode, _s(stream), ctypes.byref(h)))
+    return h.value
+
+
+def dp_block_graph_launch(graph: int, s: BlockState, stream=None):
+    return _check(lib().dp_block_graph_launch(graph, ctypes.byref(s), _s(stream)))
+
+
+def dp_block_graph_destroy(graph: int):
+    return _check(lib().dp_block_graph_destroy(graph))
+
+
 def dp_block_launch_count(d: BlockDesc) -> int:
     n = lib().dp_block_launch_count(ctypes.byref(d))
     if n < 0:
@@ -442,6 +464,11 @@ class Block:
     def step(self, x, out, weights, mode, stream=None):
         return dp_block_step(self.desc, self.state, x, out, weights, mode, stream)
 
+    def graph(self, x, out, weights, mode, stream):
+        """One captured step per ping-pong parity with these arguments; launch() runs the
+        state's next step from it (see dp_block_graph_create)."""
+        return BlockGraph(self, dp_block_graph_create(self.desc, self.state, x, out, weights, mode, stream))
+
     def step_timed(self, x, out, weights, mode, events, stream=None):
         return dp_block_step_timed(self.desc, self.state, x, out, weights, mode, events, stream)
 
@@ -456,3 +483,24 @@ class Block:
     @property
     def flops(self) -> float:
         return dp_block_flops(self.desc)
+
+
+class BlockGraph:
+    """A block's captured steps; launch() replays the state's next one."""
+
+    def __init__(self, block: Block, handle: int):
+        self.block, self.handle = block, handle
+
+    def launch(self, stream=None):
+        return dp_block_graph_launch(self.handle, self.block.state, stream)
+
+    def close(self):
+        if self.handle:
+            dp_block_graph_destroy(self.handle)
+            self.handle = 0
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

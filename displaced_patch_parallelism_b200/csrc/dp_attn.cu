@@ -467,8 +467,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_kernel(const __grid_cons
       } else {
         // A unit cut between CTAs b_lo..b_hi.  Each part stores this warp's
         // slice (unnormalised O, row max m in the log2 domain, row sum l);
-        // the part that finishes last merges the others into its registers
-        // and writes O.  Nothing waits on another CTA.
+        // the part that finishes last merges all parts in part order (the
+        // same bits whichever finishes last) and writes O.  Nothing waits on
+        // another CTA.
         const int b_lo = (sg.u * p.n_kv) / p.L, b_hi = ((sg.u + 1) * p.n_kv - 1) / p.L;
         const int me = blockIdx.x;
         const int wslice = warp - 2;
@@ -493,9 +494,22 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_kernel(const __grid_cons
           continue;
         }
         __threadfence();
-        float m = m_used, ls = lsum;
-        for (int b = b_lo; b <= b_hi; ++b) {
-          if (b == me) continue;
+        float m, ls;
+        {
+          const float* p0 = slice(b_lo);
+          const float2 ml = __ldcg(reinterpret_cast<const float2*>(p0 + 32));
+          m = ml.x;
+          ls = ml.y;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(p0) + i);
+            acc[4 * i] = v.x;
+            acc[4 * i + 1] = v.y;
+            acc[4 * i + 2] = v.z;
+            acc[4 * i + 3] = v.w;
+          }
+        }
+        for (int b = b_lo + 1; b <= b_hi; ++b) {
           const float* pc = slice(b);
           const float2 ml = __ldcg(reinterpret_cast<const float2*>(pc + 32));
           const float mn = fmaxf(m, ml.x);
@@ -948,8 +962,8 @@ __global__ void __launch_bounds__(kPairThreads, 1) attn_pair_kernel(const __grid
       } else {
         // A unit cut between CTAs b_lo..b_hi: each part stores its rows
         // (unnormalised O, row max m in the log2 domain, row sum l); the part
-        // that finishes last merges the others and writes O.  Nothing waits on
-        // another CTA.
+        // that finishes last merges all parts in part order (the same bits
+        // whichever finishes last) and writes O.  Nothing waits on another CTA.
         const int b_lo = (sg.u * p.n_kv) / p.L, b_hi = ((sg.u + 1) * p.n_kv - 1) / p.L;
         const int me = blockIdx.x;
         auto slice = [&](int b) {
@@ -974,9 +988,24 @@ __global__ void __launch_bounds__(kPairThreads, 1) attn_pair_kernel(const __grid
           continue;
         }
         __threadfence();
-        float ma = mA, la = lA, mb = mB, lb = lB;
-        for (int b = b_lo; b <= b_hi; ++b) {
-          if (b == me) continue;
+        float ma, la, mb, lb;
+        {
+          const float4* p0 = slice(b_lo);
+          const float4 ml = __ldcg(p0 + 32 * 8);
+          ma = ml.x;
+          la = ml.y;
+          mb = ml.z;
+          lb = ml.w;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 v = __ldcg(p0 + 32 * i);
+            acc[4 * i] = v.x;
+            acc[4 * i + 1] = v.y;
+            acc[4 * i + 2] = v.z;
+            acc[4 * i + 3] = v.w;
+          }
+        }
+        for (int b = b_lo + 1; b <= b_hi; ++b) {
           const float4* pc = slice(b);
           const float4 ml = __ldcg(pc + 32 * 8);
           float4 v[8];

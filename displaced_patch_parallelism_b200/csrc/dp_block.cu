@@ -23,6 +23,7 @@
 // GroupNorm -> SiLU -> conv_out).  Composite kinds run their sub-blocks with
 // the parent's ping-pong parity.
 #include <cstring>
+#include <new>
 #include <vector>
 
 #include "dp_common.cuh"
@@ -1122,6 +1123,84 @@ int dp_block_step(const dp_block_desc* d, dp_block_state* s, const void* x, void
   s->cur ^= 1;
   s->steps_done += 1;
   return DP_OK;
+}
+
+// A captured block step per ping-pong parity: exec[c] is the step whose stale
+// halves are the `c` halves.
+struct dp_block_graph {
+  cudaGraphExec_t exec[2];
+  void* workspace;   // the state the graphs were captured on
+};
+
+int dp_block_graph_create(const dp_block_desc* d, dp_block_state* s, const void* x, void* out,
+                          const void* const* weights, int n_weights, int mode, void* stream,
+                          dp_block_graph** graph) {
+  int rc = dp::desc_check(d);
+  if (rc) return rc;
+  if (!graph) return dp::set_error(DP_ERR_INVALID_ARG, "block graph: null handle pointer");
+  *graph = nullptr;
+  if (!s || !s->workspace || !x || !out || !weights)
+    return dp::set_error(DP_ERR_INVALID_ARG, "block graph: null argument");
+  if (!stream) return dp::set_error(DP_ERR_INVALID_ARG, "block graph: capture needs a stream other than the default one");
+  if (mode < DP_MODE_SYNC || mode > DP_MODE_NAIVE)
+    return dp::set_error(DP_ERR_INVALID_ARG, "block graph: bad mode %d", mode);
+  if (s->steps_done == 0)
+    return dp::set_error(DP_ERR_STATE, "block graph: capture after the state's first step");
+  if (x == out) return dp::set_error(DP_ERR_INVALID_ARG, "block graph: out aliases x");
+  if (!dp::aligned16(x) || !dp::aligned16(out))
+    return dp::set_error(DP_ERR_UNSUPPORTED, "block graph: x/out not 16-byte aligned");
+  if (n_weights < dp::weight_count(d))
+    return dp::set_error(DP_ERR_INVALID_ARG, "block graph: %d weights given, %d needed", n_weights,
+                         dp::weight_count(d));
+  const dp::Layout L = dp::layout_of(d);
+  if (s->workspace_bytes < L.total) return dp::set_error(DP_ERR_INVALID_ARG, "block graph: workspace too small");
+  auto* g = new (std::nothrow) dp_block_graph;
+  if (!g) return dp::set_error(DP_ERR_INVALID_ARG, "block graph: out of host memory");
+  g->exec[0] = g->exec[1] = nullptr;
+  g->workspace = s->workspace;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  for (int par = 0; par < 2 && !rc; ++par) {
+    rc = dp::cuda_check(cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal), "block graph: begin capture");
+    if (rc) break;
+    {
+      dp::StatusScope scope(reinterpret_cast<int*>(static_cast<char*>(s->workspace) + L.status));
+      rc = dp::step_impl(d, s->workspace, par, x, out, weights, mode, 0, st, nullptr);
+    }
+    cudaGraph_t cg = nullptr;
+    const int rc_end = dp::cuda_check(cudaStreamEndCapture(st, &cg), "block graph: end capture");
+    if (!rc) rc = rc_end;
+    if (!rc) rc = dp::cuda_check(cudaGraphInstantiate(&g->exec[par], cg, 0), "block graph: instantiate");
+    if (cg) cudaGraphDestroy(cg);
+  }
+  if (rc) {
+    for (int par = 0; par < 2; ++par)
+      if (g->exec[par]) cudaGraphExecDestroy(g->exec[par]);
+    delete g;
+    return rc;
+  }
+  *graph = g;
+  return DP_OK;
+}
+
+int dp_block_graph_launch(dp_block_graph* graph, dp_block_state* s, void* stream) {
+  if (!graph || !s) return dp::set_error(DP_ERR_INVALID_ARG, "block graph: null argument");
+  if (s->workspace != graph->workspace)
+    return dp::set_error(DP_ERR_INVALID_ARG, "block graph: launched on another state than it was captured on");
+  int rc = dp::cuda_check(cudaGraphLaunch(graph->exec[s->cur & 1], static_cast<cudaStream_t>(stream)),
+                          "block graph: launch");
+  if (rc) return rc;
+  s->cur ^= 1;
+  s->steps_done += 1;
+  return DP_OK;
+}
+
+int dp_block_graph_destroy(dp_block_graph* graph) {
+  if (!graph) return DP_OK;
+  int rc = DP_OK;
+  for (int par = 0; par < 2; ++par)
+    if (graph->exec[par] && !rc) rc = dp::cuda_check(cudaGraphExecDestroy(graph->exec[par]), "block graph: destroy");
+  delete graph;
+  return rc;
 }
 
 int dp_block_status(const dp_block_desc* d, const dp_block_state* s, void* stream, int* status) {

@@ -719,6 +719,35 @@ DP_API int dp_block_step(const dp_block_desc* d, dp_block_state* s, const void* 
  * step timed out.  Synchronises `stream` first; *status receives DP_OK or
  * DP_ERR_TIMEOUT.  DP_ERR_INVALID_ARG on a null or uninitialised state.
  */
+/*
+ * Block steps as CUDA graphs (a step of a large block is hundreds of launches;
+ * replaying them as one graph removes their host-side launch cost and part of
+ * the gaps between them).  dp_block_graph_create captures one step of `d` in
+ * `mode` for each ping-pong parity, on the caller's (non-default) `stream`,
+ * with the given x, out and weight pointers fixed in the graphs; nothing runs
+ * and the state does not change.  dp_block_graph_launch then runs the step of
+ * the state's current parity on `stream`, flips the parity and counts the
+ * step, exactly as dp_block_step with those arguments would: new inputs are
+ * copied into the captured x before a launch, and anything the caller does
+ * between steps (a sampler update) runs between launches.
+ *   - Capture after the state's first step (DP_ERR_STATE before it): the
+ *     graphs are later steps (a fixed context's keys and values, computed at
+ *     the first step, are not in them).
+ *   - A graph runs only on the state it was captured on (DP_ERR_INVALID_ARG
+ *     otherwise) and while the weights, x, out and workspace stay where they
+ *     were at capture.
+ *   - DP_ERR_CUDA if the capture or instantiation fails; nothing is left
+ *     allocated then.  dp_block_graph_destroy frees the graphs (NULL is a no-op).
+ * Handles are opaque and owned by the caller; one handle per state at a time
+ * and stream order between its launches and other calls on the state.
+ */
+typedef struct dp_block_graph dp_block_graph;
+DP_API int dp_block_graph_create(const dp_block_desc* d, dp_block_state* s, const void* x, void* out,
+                                 const void* const* weights, int n_weights, int mode, void* stream,
+                                 dp_block_graph** graph);
+DP_API int dp_block_graph_launch(dp_block_graph* graph, dp_block_state* s, void* stream);
+DP_API int dp_block_graph_destroy(dp_block_graph* graph);
+
 DP_API int dp_block_status(const dp_block_desc* d, const dp_block_state* s, void* stream,
                            int* status);
 

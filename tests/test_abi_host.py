@@ -445,6 +445,29 @@ def test_feed_forward_fusion_rule_on_the_host(B):
         assert e.value.code == code, args
 
 
+def test_block_graph_rejects_bad_arguments_on_the_host(B):
+    """Graph capture checks its arguments before any CUDA call: a state before its first
+    step, the default stream, a null handle pointer; launch and destroy of a null handle."""
+    import ctypes
+    d = B.dp_block_desc_init(B.RESBLOCK, 32, 32, 320, 320, 32, 4, 0, B.BF16, 1, 1e-5, 1.0)
+    A = 1 << 20
+    st = B.BlockState(A, B.dp_block_workspace_size(d), 0, 0)
+    w = (ctypes.c_void_p * 8)(*([A] * 8))
+    h = ctypes.c_void_p(0)
+    L = B.lib()
+    assert L.dp_block_graph_create(ctypes.byref(d), ctypes.byref(st), A, 2 * A, w, 8, B.DISPLACED, A,
+                                   ctypes.byref(h)) == B.DP_ERR_STATE
+    st.steps_done = 1
+    assert L.dp_block_graph_create(ctypes.byref(d), ctypes.byref(st), A, 2 * A, w, 8, B.DISPLACED, None,
+                                   ctypes.byref(h)) == B.DP_ERR_INVALID_ARG       # default stream
+    assert L.dp_block_graph_create(ctypes.byref(d), ctypes.byref(st), A, 2 * A, w, 8, B.DISPLACED, A,
+                                   None) == B.DP_ERR_INVALID_ARG                  # no handle pointer
+    assert L.dp_block_graph_create(ctypes.byref(d), ctypes.byref(st), A, 2 * A, w, 7, B.DISPLACED, A,
+                                   ctypes.byref(h)) == B.DP_ERR_INVALID_ARG       # too few weights
+    assert L.dp_block_graph_launch(None, ctypes.byref(st), A) == B.DP_ERR_INVALID_ARG
+    assert L.dp_block_graph_destroy(None) == B.DP_OK
+
+
 def test_fixed_context_on_the_host(B):
     """A fixed context drops each layer's context k/v projection from the (later) steps' plan
     and flops, and is only for TRANSFORMER and UNET_SDXL blocks."""
