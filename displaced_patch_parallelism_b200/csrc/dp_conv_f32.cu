@@ -52,22 +52,42 @@ __global__ void __launch_bounds__(256) conv3x3_f32_kernel(
     else if (mode == DP_MODE_DISPLACED) src[kh] = as;
   }
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  constexpr int kInIter = (3 * kMaxSpan * kF32Ci + 255) / 256;   // staging loads per thread
+  constexpr int kWIter = 9 * kF32Ci * kF32Co / 256;
   for (int ci0 = 0; ci0 < Cin; ci0 += kF32Ci) {
-    // input window: consecutive threads take consecutive channels of a pixel
-    for (int i = threadIdx.x; i < 3 * span * kF32Ci; i += blockDim.x) {
+    // input window and filter slice: every load of a thread is issued before
+    // the first store, so the loads overlap instead of waiting one by one
+    float vin[kInIter], vw[kWIter];
+#pragma unroll
+    for (int j = 0; j < kInIter; ++j) {
+      const int i = threadIdx.x + 256 * j;   // consecutive threads: consecutive channels of a pixel
       const int ci = i % kF32Ci, rest = i / kF32Ci;
       const int px = rest % span, kh = rest / span;
       const int col = stride * c0 + px - 1;
-      float v = 0.f;
-      if (src[kh] && col >= 0 && col < W)
-        v = __ldg(src[kh] + (static_cast<size_t>(rows[kh]) * W + col) * Cin + ci0 + ci);
-      s_in[kh][ci][px] = v;
+      vin[j] = 0.f;
+      if (kh < 3 && src[kh] && col >= 0 && col < W)
+        vin[j] = __ldg(src[kh] + (static_cast<size_t>(rows[kh]) * W + col) * Cin + ci0 + ci);
     }
-    // filter slice [tap][ci][co] of this block's 32 output channels
-    for (int i = threadIdx.x; i < 9 * kF32Ci * kF32Co; i += blockDim.x) {
+#pragma unroll
+    for (int j = 0; j < kWIter; ++j) {
+      const int i = threadIdx.x + 256 * j;   // filter slice [tap][ci][co] of this block's channels
       const int ci = i % kF32Ci, rest = i / kF32Ci;
       const int tap = rest % 9, co = rest / 9;
-      s_w[tap][ci][co] = __ldg(w + (static_cast<size_t>(co0 + co) * 9 + tap) * Cin + ci0 + ci);
+      vw[j] = __ldg(w + (static_cast<size_t>(co0 + co) * 9 + tap) * Cin + ci0 + ci);
+    }
+#pragma unroll
+    for (int j = 0; j < kInIter; ++j) {
+      const int i = threadIdx.x + 256 * j;
+      const int ci = i % kF32Ci, rest = i / kF32Ci;
+      const int px = rest % span, kh = rest / span;
+      if (kh < 3) s_in[kh][ci][px] = vin[j];
+    }
+#pragma unroll
+    for (int j = 0; j < kWIter; ++j) {
+      const int i = threadIdx.x + 256 * j;
+      const int ci = i % kF32Ci, rest = i / kF32Ci;
+      const int tap = rest % 9, co = rest / 9;
+      s_w[tap][ci][co] = vw[j];
     }
     __syncthreads();
 #pragma unroll

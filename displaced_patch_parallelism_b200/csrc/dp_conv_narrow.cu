@@ -68,11 +68,22 @@ __global__ void __launch_bounds__(256) conv3x3_narrow_kernel(
 #pragma unroll
   for (int j = 0; j < CO; ++j) acc[j] = 0.f;
   for (int ci0 = 0; ci0 < Cin; ci0 += kNarrowCi) {
-    for (int i = threadIdx.x; i < 9 * kNarrowCi * CO; i += blockDim.x) {
+    // the filter slice: all of a thread's loads issued before its stores
+    constexpr int kWIter = (9 * kNarrowCi * CO + 255) / 256;
+    float vw[kWIter];
+#pragma unroll
+    for (int j = 0; j < kWIter; ++j) {
+      const int i = threadIdx.x + 256 * j;
       const int co = i % CO, rest = i / CO;
       const int ci = rest % kNarrowCi, tap = rest / kNarrowCi;
-      s_w[tap][ci][co] =
-          co < Cout ? to_f(w[(static_cast<size_t>(co) * 9 + tap) * Cin + ci0 + ci]) : 0.f;
+      vw[j] = co < Cout && tap < 9 ? to_f(w[(static_cast<size_t>(co) * 9 + tap) * Cin + ci0 + ci]) : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < kWIter; ++j) {
+      const int i = threadIdx.x + 256 * j;
+      const int co = i % CO, rest = i / CO;
+      const int ci = rest % kNarrowCi, tap = rest / kNarrowCi;
+      if (tap < 9) s_w[tap][ci][co] = vw[j];
     }
     __syncthreads();
     if (c < Wo) {

@@ -647,6 +647,8 @@ __global__ void __launch_bounds__(1024, 1) gn_cluster_kernel(
   float* sscale = reinterpret_cast<float*>(f + 2 * a.G);                 // [C]: gamma, then the scale
   float* sshift = sscale + a.C;                                          // [C]: beta, then the shift
   float* sstale = sshift + a.C;                                          // [G][2] global, [G][2] band
+  float* gremote = sstale + 4 * a.G;                                     // [cpb][G][2]: the cluster's sums
+  float* gbands = gremote + 2 * a.cpb * a.G;                             // [P][G][2]: every band's moments
   __shared__ __align__(8) uint64_t load_bar;
   __shared__ int s_last;
 
@@ -745,16 +747,21 @@ __global__ void __launch_bounds__(1024, 1) gn_cluster_kernel(
   }
   cluster_sync_all();   // every CTA of the band has its sums in shared memory
 
-  // ---- the band's fresh moments, added over the cluster in rank order
+  // ---- the band's fresh moments, added over the cluster in rank order: each
+  // (rank, moment) is read by its own thread, so the remote reads overlap
   const double n = static_cast<double>(a.HWp) * cg;
-  for (int i = threadIdx.x; i < 2 * a.G; i += blockDim.x) {
-    const uint32_t local = smem_u32(gpart + i);
-    double s = 0.0;
-    for (int k = 0; k < a.cpb; ++k) s += ld_dsmem_f32(mapa_shared(local, static_cast<uint32_t>(k)));
-    f[i] = s / n;
+  for (int t = threadIdx.x; t < 2 * a.G * a.cpb; t += blockDim.x) {
+    const int k = t / (2 * a.G), i = t - k * 2 * a.G;
+    gremote[t] = ld_dsmem_f32(mapa_shared(smem_u32(gpart + i), static_cast<uint32_t>(k)));
   }
+  __syncthreads();
   // no more reads of other CTAs' shared memory: arrive now, wait at exit
   cluster_arrive();
+  for (int i = threadIdx.x; i < 2 * a.G; i += blockDim.x) {
+    double s = 0.0;
+    for (int k = 0; k < a.cpb; ++k) s += gremote[k * 2 * a.G + i];
+    f[i] = s / n;
+  }
   __syncthreads();
   for (int c = threadIdx.x; c < a.C; c += blockDim.x) {
     const int g = c / cg;
@@ -810,9 +817,12 @@ __global__ void __launch_bounds__(1024, 1) gn_cluster_kernel(
     __syncthreads();
     if (s_last) {
       __threadfence();
+      // every band's moments read by their own threads, then added in band order
+      for (int t = threadIdx.x; t < 2 * a.G * a.P; t += blockDim.x) gbands[t] = __ldcg(fresh_local + t);
+      __syncthreads();
       for (int i = threadIdx.x; i < 2 * a.G; i += blockDim.x) {
         double s = 0.0;
-        for (int q = 0; q < a.P; ++q) s += __ldcg(fresh_local + q * a.G * 2 + i);
+        for (int q = 0; q < a.P; ++q) s += gbands[q * a.G * 2 + i];
         fresh_global[i] = static_cast<float>(s / a.P);
       }
       if (threadIdx.x == 0) *ticket = 0u;
@@ -917,7 +927,7 @@ bool gn_cluster_plan(int H, int W, int C, int G, int P, int dtype, int mode, int
   const size_t data = ((static_cast<size_t>(ch) * C * e) + 127) & ~size_t(127);
   const size_t need = data + static_cast<size_t>(slanes) * C * 8 + static_cast<size_t>(G) * 8 + 16 +
                       static_cast<size_t>(G) * 16 + static_cast<size_t>(C) * 8 +
-                      static_cast<size_t>(G) * 16;
+                      static_cast<size_t>(G) * 16 + static_cast<size_t>(n + P) * G * 8;
   if (need > 220 * 1024) return false;
   *cpb = n;
   *chunk = static_cast<int>(ch);
