@@ -28,11 +28,19 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const __nv_bfloat16* __r
                                                         const float* __restrict__ gamma,
                                                         const float* __restrict__ beta, int T,
                                                         int C, float eps) {
+  // gamma and beta are weights, never written by the kernel before this one:
+  // staged while that kernel finishes, so the token's end needs no memory trip
+  __shared__ __align__(16) float sg[kLnMaxC], sb[kLnMaxC];
+  for (int c = 4 * threadIdx.x; c < C; c += 4 * blockDim.x) {
+    *reinterpret_cast<float4*>(sg + c) = __ldg(reinterpret_cast<const float4*>(gamma + c));
+    *reinterpret_cast<float4*>(sb + c) = __ldg(reinterpret_cast<const float4*>(beta + c));
+  }
+  __syncthreads();
   griddep_wait();
   griddep_trigger();
   const int warp = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   const int lane = lane_id();
-  if (warp >= T) return;
+  if (warp >= T) return;   // after the block's only barrier
   const int nvec = C / 8;
   const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(warp) * C);
   float v[NV][8];
@@ -73,10 +81,10 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const __nv_bfloat16* __r
   for (int i = 0; i < NV; ++i) {
     const int e = lane + 32 * i;
     if (e < nvec) {
-      const float4 g0 = __ldg(reinterpret_cast<const float4*>(gamma) + 2 * e);
-      const float4 g1 = __ldg(reinterpret_cast<const float4*>(gamma) + 2 * e + 1);
-      const float4 b0 = __ldg(reinterpret_cast<const float4*>(beta) + 2 * e);
-      const float4 b1 = __ldg(reinterpret_cast<const float4*>(beta) + 2 * e + 1);
+      const float4 g0 = reinterpret_cast<const float4*>(sg)[2 * e];
+      const float4 g1 = reinterpret_cast<const float4*>(sg)[2 * e + 1];
+      const float4 b0 = reinterpret_cast<const float4*>(sb)[2 * e];
+      const float4 b1 = reinterpret_cast<const float4*>(sb)[2 * e + 1];
       const float g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
       const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
       float o[8];

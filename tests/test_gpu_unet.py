@@ -137,3 +137,55 @@ def test_unet_sdxl_step(context_fixed):
     exact = oracle({}, xr, B.NAIVE, "none", None)
     torch.cuda.synchronize()
     print(check_chain(host_img(out), exact, ref, what="SDXL U-Net naive step"))
+
+
+def test_unet_sdxl_full_size_properties():
+    """SDXL's whole U-Net at 1024 px (latent 4x128x128, 8 bands, depths 0 / 2 / 10, the
+    benchmark's workload), beyond the oracle's reach at this size, held to properties that hold
+    at any size: a displaced step of an unchanged latent reproduces the sync step (every stale
+    buffer then holds what a sync step computes; only rounding differs), both are finite, and a
+    naive step (no context between bands) lies much further from them; graph replays of the
+    displaced step agree with it as well; no bounded wait ran out."""
+    wl = synth.WORKLOADS["unet_sdxl_4x128x128"]
+    dev = torch.device("cuda")
+    wts = synth.make_weights(wl, device=dev)
+    dw = unet_sdxl_weights(wts, synth.sdxl_unet_stages(wl.base, wl.depths), wl.depths, torch.bfloat16, dev)
+    del wts
+    dw += [synth.context(wl).to(torch.bfloat16).to(dev), synth.randn((wl.temb_dim,), wl.seed + 600).to(dev)]
+
+    def block():
+        return B.Block(B.UNET_SDXL, wl.H, wl.W, wl.C, wl.C, wl.G, wl.P, 0, B.BF16, True, wl.eps, 1.0,
+                       context=(wl.ctx_len, wl.ctx_dim, 0), temb_dim=wl.temb_dim,
+                       unet=(wl.base,) + tuple(wl.depths), context_fixed=True)
+
+    x = synth.nchw_to_nhwc(synth.InputStream(wl).x(0)).to(torch.bfloat16).to(dev)
+    outs = {m: torch.empty(wl.H, wl.W, wl.C, dtype=torch.bfloat16, device=dev) for m in ("s", "d", "n", "g")}
+    blk = block()
+    blk.step(x, outs["s"], dw, B.SYNC)
+    blk.step(x, outs["d"], dw, B.DISPLACED)
+    naive = block()
+    naive.step(x, outs["n"], dw, B.NAIVE)
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        g = blk.graph(x, outs["g"], dw, B.DISPLACED, stream)
+        # the plain step above ran at one parity: replay twice so one replay has that parity
+        g.launch(stream)
+        first = outs["g"].clone()
+        g.launch(stream)
+    torch.cuda.synchronize()
+    g.close()
+    s, d, n = (outs[k].double() for k in "sdn")
+    assert torch.isfinite(s).all() and torch.isfinite(d).all() and torch.isfinite(n).all()
+    rel = lambda a, b: float(torch.linalg.norm(a - b) / torch.linalg.norm(b))
+    r_d, r_n = rel(d, s), rel(n, s)
+    print({"displaced_vs_sync": r_d, "naive_vs_sync": r_n})
+    # measured on B200: 1.5e-2 (the sync step's grid-wide GroupNorm and the displaced step's
+    # cluster GroupNorm add in different orders; over ~150 bf16-stored stages, ten-layer
+    # transformers included, those last-bit differences grow) against 0.59 for naive patches
+    assert r_d < 5e-2, r_d
+    assert r_n > 10 * r_d, (r_n, r_d)
+    # every displaced step of this unchanged latent computes the same thing, so the graph
+    # replays agree with the sync step as closely as the plain displaced step does
+    assert rel(first.double(), s) < 5e-2 and rel(outs["g"].double(), s) < 5e-2
+    assert blk.status() == 0 and naive.status() == 0 and B.dp_device_status() == 0
