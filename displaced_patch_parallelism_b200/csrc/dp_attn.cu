@@ -494,8 +494,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2) attn_kernel(const __grid_cons
           continue;
         }
         __threadfence();
-        float m, ls;
-        {
+        float m = m_used, ls = lsum;   // the first part's state: this CTA's own when it is the first
+        if (me != b_lo) {
           const float* p0 = slice(b_lo);
           const float2 ml = __ldcg(reinterpret_cast<const float2*>(p0 + 32));
           m = ml.x;
@@ -988,8 +988,8 @@ __global__ void __launch_bounds__(kPairThreads, 1) attn_pair_kernel(const __grid
           continue;
         }
         __threadfence();
-        float ma, la, mb, lb;
-        {
+        float ma = mA, la = lA, mb = mB, lb = lB;   // the first part's state: this CTA's own when it is the first
+        if (me != b_lo) {
           const float4* p0 = slice(b_lo);
           const float4 ml = __ldcg(p0 + 32 * 8);
           ma = ml.x;

@@ -139,6 +139,40 @@ def test_unet_sdxl_step(context_fixed):
     print(check_chain(host_img(out), exact, ref, what="SDXL U-Net naive step"))
 
 
+def test_unet_sdxl_step_eight_bands():
+    """The U-Net step over 8 bands of a 4x128x128 latent (base 64, depths 0 / 1 / 1): 16-row
+    bands at the first level, 8 at the second and 4 (128 tokens) at the third, so every conv
+    halo and every down / up sampling crosses band edges at every level.  A sync step and two
+    displaced steps of a drifting latent against the oracle, end to end (check_chain)."""
+    wl = synth.Workload(name="unet_sdxl_p8", kind="unet_sdxl", C=4, H=128, W=128, P=8, G=32, base=64,
+                        depths=(0, 1, 1), ctx_len=77, ctx_dim=128, temb_dim=128, weight_seed=19)
+    wts = synth.make_weights(wl, random_affine=True)
+    dev_w = unet_sdxl_weights(wts, synth.sdxl_unet_stages(wl.base, wl.depths), wl.depths)
+    g = torch.Generator().manual_seed(20)
+    ctx = torch.randn(wl.ctx_len, wl.ctx_dim, generator=g).to(torch.bfloat16).to(torch.float32)
+    temb = torch.randn(wl.temb_dim, generator=g)
+    dev_w += [ctx.to(torch.bfloat16).cuda(), temb.cuda()]
+    w64 = {n: v.double().numpy() for n, v in wts.items()}
+    c64, t64 = ctx.double().numpy(), temb.double().numpy()
+    blk = B.Block(B.UNET_SDXL, wl.H, wl.W, wl.C, wl.C, wl.G, wl.P, 0, B.BF16, True, 1e-5, 1.0,
+                  context=(wl.ctx_len, wl.ctx_dim, 0), temb_dim=wl.temb_dim, unet=(wl.base,) + wl.depths,
+                  context_fixed=True)
+    st, st_exact = {}, {}
+    x = torch.randn(wl.C, wl.H, wl.W, generator=g)
+    for k, mode in enumerate([B.SYNC, B.DISPLACED, B.DISPLACED]):
+        if k:
+            x = x + 0.05 * torch.randn(x.shape, generator=g)
+        xr = x.to(torch.bfloat16).double().numpy()
+        out = torch.empty(wl.H, wl.W, wl.C, dtype=torch.bfloat16, device="cuda")
+        blk.step(dev_img(xr, "bf16"), out, dev_w, mode)
+        kw = dict(base=wl.base, depths=wl.depths)
+        ref = O.sdxl_unet_step(st, xr, c64, t64, w64, wl.P, wl.G, 1e-5, 1.0, mode, "bf16", final_storage="none", **kw)
+        exact = O.sdxl_unet_step(st_exact, xr, c64, t64, w64, wl.P, wl.G, 1e-5, 1.0, mode, "none", **kw)
+        torch.cuda.synchronize()
+        print(check_chain(host_img(out), exact, ref, what=f"SDXL U-Net P=8 step {k} mode {mode}"))
+    assert blk.status() == 0 and B.dp_device_status() == 0
+
+
 def test_unet_sdxl_full_size_properties():
     """SDXL's whole U-Net at 1024 px (latent 4x128x128, 8 bands, depths 0 / 2 / 10, the
     benchmark's workload), beyond the oracle's reach at this size, held to properties that hold
