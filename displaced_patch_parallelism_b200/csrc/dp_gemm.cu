@@ -72,6 +72,9 @@ struct GemmParams {
   int gn_cg;               // channels per group
   int gn_silu;
   void* a_next;            // [H][W][Cin]: receives the normalised band-edge rows, or null
+  // Pair kernels, 3x3 conv: stores under an L2 evict-first policy (an output
+  // larger than L2 is written back while the kernel runs).
+  int out_evict_first;
   // Pair kernels, plain A only: the epilogue applies the gated GELU.  The N =
   // 2F accumulator columns hold value and gate interleaved in blocks of 16
   // (each 32-column chunk: 16 values, then their 16 gates); tmO[0] maps the
@@ -636,6 +639,7 @@ __device__ __forceinline__ bool pair_epilogue_tile(const GemmParams& p, uint32_t
     __syncwarp();
     if (lane == 0) {
       if (p.a_mode == 0) tma_store_2d(om, ob, b.x + ch * 32, b.y);
+      else if (p.out_evict_first) tma_store_3d_evict_first(om, ob, b.x + ch * 32, b.y, b.z, l2_evict_first_policy());
       else tma_store_3d(om, ob, b.x + ch * 32, b.y, b.z);
       bulk_commit();
     }
@@ -1650,6 +1654,8 @@ int conv3x3_launch(const void* a_fresh, const void* a_stale, const void* weight,
   p.residual = residual;
   p.out0 = out;
   p.status = device_status_ptr();
+  // an output of more than three quarters of L2 (126 MB) leaves L2 as it is written
+  p.out_evict_first = static_cast<size_t>(Ho) * Wo * Cout * e > (static_cast<size_t>(96) << 20);
   int bn_single = 0, splits = 1;
   const bool can_split = workspace && workspace_bytes >= gemm_workspace_bytes();
   const int pw = tf32 ? 0 : pick_pair(p.m_tiles, Cout, Cout, p.k_blocks, can_split, &bn_single, &splits);
