@@ -306,3 +306,30 @@ def test_resblock_time_embedding():
         check(host_img(out), ref, what=f"temb resblock step {k} mode {mode}", storage_rel=BF16_HALF_ULP,
               scale_rel=2.0 ** -7)
     assert B.dp_device_status() == 0
+
+
+def test_transformer_640x64x64_workload():
+    """The benchmark's transformer workload at its own sizes and settings (640 channels at
+    64x64 over 4 bands, 10 heads, a 77x2048 context kept from the first step, F = 2560 with the
+    gated GELU in ff1's epilogue, the workload's seeded weights): a sync step and a displaced
+    step of the workload's drifting input against the oracle, end to end (check_chain)."""
+    wl = synth.WORKLOADS["transformer_640x64x64"]
+    wts = synth.make_weights(wl, random_affine=True)
+    ctx = synth.context(wl)
+    dev_w = block_weights("transformer", wts) + [ctx.to(torch.bfloat16).cuda()]
+    blk = B.Block(B.TRANSFORMER, wl.H, wl.W, wl.C, wl.C, wl.G, wl.P, wl.heads, B.BF16, False, wl.eps, 1.0,
+                  context=(wl.ctx_len, wl.ctx_dim, wl.ff_inner), context_fixed=True)
+    w64 = {n: v.double().numpy() for n, v in wts.items()}
+    c64 = ctx.double().numpy()
+    xs = synth.InputStream(wl)
+    st, st_exact = {}, {}
+    for k, mode in enumerate([B.SYNC, B.DISPLACED]):
+        xr = xs.x(k)[0].double().numpy()
+        out = torch.empty(wl.H, wl.W, wl.C, dtype=torch.bfloat16, device="cuda")
+        blk.step(dev_img(xr, "bf16"), out, dev_w, mode)
+        ref = O.transformer_step(st, xr, c64, w64, wl.P, wl.G, wl.eps, 1.0, wl.heads, mode, "bf16",
+                                 final_storage="none")
+        exact = O.transformer_step(st_exact, xr, c64, w64, wl.P, wl.G, wl.eps, 1.0, wl.heads, mode, "none")
+        torch.cuda.synchronize()
+        print(check_chain(host_img(out), exact, ref, what=f"transformer_640x64x64 step {k} mode {mode}"))
+    assert blk.status() == 0 and B.dp_device_status() == 0
