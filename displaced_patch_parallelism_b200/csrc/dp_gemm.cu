@@ -88,11 +88,10 @@ __device__ __forceinline__ void split_range(int kb, int splits, int r, int* kb0,
   *kb1 = ((r + 1) * kb) / splits;
 }
 
-template <int BN, bool TF32>
+template <int BN>
 struct GemmCfg {
   static constexpr int BM = 128;
-  static constexpr int ELEM = TF32 ? 4 : 2;
-  static constexpr int BK = 128 / ELEM;          // elements per 128-byte row
+  static constexpr int BK = 64;                  // bf16 elements per 128-byte row
   static constexpr int A_BYTES = BM * 128;
   static constexpr int B_BYTES = BN * 128;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -117,10 +116,10 @@ __device__ __forceinline__ void mbar_wait_teardown(uint64_t* bar, uint32_t parit
   }
 }
 
-template <int BN, bool TF32>
+template <int BN>
 __global__ void __launch_bounds__(192, 1) igemm_kernel(const __grid_constant__ GemmParams p) {
-  using C = GemmCfg<BN, TF32>;
-  using OutT = typename std::conditional<TF32, float, __nv_bfloat16>::type;
+  using C = GemmCfg<BN>;
+  using OutT = __nv_bfloat16;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -248,7 +247,7 @@ __global__ void __launch_bounds__(192, 1) igemm_kernel(const __grid_constant__ G
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------------ MMA issuer
-      constexpr uint32_t idesc = idesc_dense(128, BN, TF32 ? 2 : 1, 0, 0);
+      constexpr uint32_t idesc = idesc_dense(128, BN, 1, 0, 0);
       const uint64_t a_desc0 = sdesc_sw128(smem_u32(sA), 1024);
       const uint64_t b_desc0 = sdesc_sw128(smem_u32(sB), 1024);
       int stage = 0;
@@ -280,12 +279,7 @@ __global__ void __launch_bounds__(192, 1) igemm_kernel(const __grid_constant__ G
             const uint64_t ad = a_desc0 + static_cast<uint64_t>((st * C::A_BYTES) >> 4);
             const uint64_t bd = b_desc0 + static_cast<uint64_t>((st * C::B_BYTES) >> 4);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              if (TF32)
-                umma_tf32_ss(d, ad + 2 * k, bd + 2 * k, idesc, ((kb + h) | k) != 0);
-              else
-                umma_f16_ss(d, ad + 2 * k, bd + 2 * k, idesc, ((kb + h) | k) != 0);
-            }
+            for (int k = 0; k < 4; ++k) umma_f16_ss(d, ad + 2 * k, bd + 2 * k, idesc, ((kb + h) | k) != 0);
             if (++st == C::STAGES) st = 0;
           }
           for (int h = 0; h < g; ++h) {
@@ -360,47 +354,29 @@ __global__ void __launch_bounds__(192, 1) igemm_kernel(const __grid_constant__ G
             v[4 * j + 3] += b.w;
           }
         }
-        if (TF32) {
-          if (rrow) {
-            const float4* r4 = reinterpret_cast<const float4*>(rrow + ch * 32);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const float4 x = r4[j];
-              v[4 * j] += x.x;
-              v[4 * j + 1] += x.y;
-              v[4 * j + 2] += x.z;
-              v[4 * j + 3] += x.w;
-            }
-          }
-          float4* o4 = reinterpret_cast<float4*>(orow + ch * 32);
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            o4[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-        } else {
-          if (rrow) {
-            const uint4* r4 = reinterpret_cast<const uint4*>(rrow + ch * 32);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              uint4 u = r4[j];
-              const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float2 f = __bfloat1622float2(h[e]);
-                v[8 * j + 2 * e] += f.x;
-                v[8 * j + 2 * e + 1] += f.y;
-              }
-            }
-          }
-          uint4* o4 = reinterpret_cast<uint4*>(orow + ch * 32);
+        if (rrow) {
+          const uint4* r4 = reinterpret_cast<const uint4*>(rrow + ch * 32);
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            uint4 u;
-            u.x = pack_bf16x2(v[8 * j], v[8 * j + 1]);
-            u.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
-            u.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
-            u.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
-            o4[j] = u;
+            uint4 u = r4[j];
+            const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __bfloat1622float2(h[e]);
+              v[8 * j + 2 * e] += f.x;
+              v[8 * j + 2 * e + 1] += f.y;
+            }
           }
+        }
+        uint4* o4 = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint4 u;
+          u.x = pack_bf16x2(v[8 * j], v[8 * j + 1]);
+          u.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
+          u.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
+          u.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
+          o4[j] = u;
         }
       }
     }
@@ -1390,14 +1366,14 @@ static int launch_pair(const GemmParams& p, cudaStream_t s) {
                        "pair gemm launch", p);
 }
 
-template <int BN, bool TF32>
+template <int BN>
 static int launch_t(const GemmParams& p, cudaStream_t s) {
-  using C = GemmCfg<BN, TF32>;
+  using C = GemmCfg<BN>;
   static int attr_dev_mask = 0;
   int dev = 0;
   cudaGetDevice(&dev);
   if (!(attr_dev_mask & (1 << (dev & 31)))) {
-    int rc = cuda_check(cudaFuncSetAttribute(igemm_kernel<BN, TF32>,
+    int rc = cuda_check(cudaFuncSetAttribute(igemm_kernel<BN>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM),
                         "gemm smem attribute");
     if (rc) return rc;
@@ -1406,33 +1382,29 @@ static int launch_t(const GemmParams& p, cudaStream_t s) {
   const int tiles = p.m_tiles * p.n_tiles;
   const int grid = std::min(tiles, num_sms());
   mark_launch(s);
-  return launch_kernel(igemm_kernel<BN, TF32>, dim3(grid), dim3(192), C::SMEM, s, false,
+  return launch_kernel(igemm_kernel<BN>, dim3(grid), dim3(192), C::SMEM, s, false,
                        "gemm launch", p);
 }
 
-static int launch_gemm(const GemmParams& p, int BN, bool tf32, cudaStream_t s) {
-  if (!tf32) {
-    switch (BN) {
-      case 32: return launch_t<32, false>(p, s);
-      case 64: return launch_t<64, false>(p, s);
-      case 96: return launch_t<96, false>(p, s);
-      case 128: return launch_t<128, false>(p, s);
-      case 160: return launch_t<160, false>(p, s);
-      case 192: return launch_t<192, false>(p, s);
-      case 256: return launch_t<256, false>(p, s);
-      default: break;
-    }
+static int launch_gemm(const GemmParams& p, int BN, cudaStream_t s) {
+  switch (BN) {
+    case 32: return launch_t<32>(p, s);
+    case 64: return launch_t<64>(p, s);
+    case 96: return launch_t<96>(p, s);
+    case 128: return launch_t<128>(p, s);
+    case 160: return launch_t<160>(p, s);
+    case 192: return launch_t<192>(p, s);
+    case 256: return launch_t<256>(p, s);
+    default: break;
   }
   return set_error(DP_ERR_UNSUPPORTED, "gemm: no kernel for BN=%d", BN);
 }
 
 // Tile width in N: the candidate that divides `split` with the fewest
 // wave-quantised columns per SM (a small per-tile cost favours wider tiles).
-static int pick_bn(int m_tiles, int N, int split, bool tf32) {
-  static const int bf16_c[] = {256, 192, 160, 128, 96, 64, 32};
-  static const int tf32_c[] = {128, 64};
-  const int* c = tf32 ? tf32_c : bf16_c;
-  const int nc = tf32 ? 2 : 7;
+static int pick_bn(int m_tiles, int N, int split) {
+  static const int c[] = {256, 192, 160, 128, 96, 64, 32};
+  const int nc = 7;
   int best = 0;
   long best_cost = 0;
   for (int i = 0; i < nc; ++i) {
@@ -1489,7 +1461,7 @@ static int pick_pair(int m_tiles, int N, int split, int kb, bool can_split, int*
       }
     }
   }
-  *bn_single = pick_bn(m_tiles, N, split, false);
+  *bn_single = pick_bn(m_tiles, N, split);
   if (*bn_single) {
     const long tiles = static_cast<long>(m_tiles) * (N / *bn_single);
     const double t = static_cast<double>((tiles + sms - 1) / sms) *
@@ -1623,8 +1595,7 @@ int conv3x3_launch(const void* a_fresh, const void* a_stale, const void* weight,
   if (dtype == DP_FP32)
     return conv3x3_f32_launch(a_fresh, a_stale, weight, bias, residual, out, H, W, Cin, Cout, stride, P,
                               mode, stream);
-  const bool tf32 = false;
-  const int e = tf32 ? 4 : 2;
+  const int e = 2;   // bf16
   const int BK = 128 / e;
   const int Ho = (H - 1) / stride + 1, Wo = (W - 1) / stride + 1;
   GemmParams p;
@@ -1658,13 +1629,13 @@ int conv3x3_launch(const void* a_fresh, const void* a_stale, const void* weight,
   p.out_evict_first = static_cast<size_t>(Ho) * Wo * Cout * e > (static_cast<size_t>(96) << 20);
   int bn_single = 0, splits = 1;
   const bool can_split = workspace && workspace_bytes >= gemm_workspace_bytes();
-  const int pw = tf32 ? 0 : pick_pair(p.m_tiles, Cout, Cout, p.k_blocks, can_split, &bn_single, &splits);
+  const int pw = pick_pair(p.m_tiles, Cout, Cout, p.k_blocks, can_split, &bn_single, &splits);
   const bool pair = pw != 0;
-  const int BN = pair ? pw : pick_bn(p.m_tiles, Cout, Cout, tf32);
+  const int BN = pair ? pw : pick_bn(p.m_tiles, Cout, Cout);
   if (!BN) return set_error(DP_ERR_UNSUPPORTED, "conv: no N tile divides Cout=%d", Cout);
   p.n_tiles = Cout / BN;
   const CUtensorMapDataType dt =
-      tf32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+      CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   uint64_t dims[3], str[2];
   uint32_t box[3] = {static_cast<uint32_t>(BK), static_cast<uint32_t>(Wt), 1};
   if (stride == 1) {
@@ -1696,7 +1667,7 @@ int conv3x3_launch(const void* a_fresh, const void* a_stale, const void* weight,
     if (rc || splits == 1) return rc;
     return launch_finish(p, Ho * Wo, stream);
   }
-  return launch_gemm(p, BN, tf32, stream);
+  return launch_gemm(p, BN, stream);
 }
 
 bool conv3x3_gn_eligible(int H, int W, int Cin, int Cout, int G, int dtype) {
@@ -1832,7 +1803,7 @@ int linear_launch(const void* x, const void* weight, const float* bias, const vo
   const int pw = p.k_blocks >= 8
                      ? pick_pair(p.m_tiles, N, split, p.k_blocks, can_split, &bn_single, &splits)
                      : 0;
-  if (!pw) bn_single = pick_bn(p.m_tiles, N, split, false);
+  if (!pw) bn_single = pick_bn(p.m_tiles, N, split);
   const bool pair = pw != 0;
   const int BN = pair ? pw : bn_single;
   if (!BN) return set_error(DP_ERR_UNSUPPORTED, "linear: no N tile divides split=%d", split);
@@ -1857,7 +1828,7 @@ int linear_launch(const void* x, const void* weight, const float* bias, const vo
     if (rc || splits == 1) return rc;
     return launch_finish(p, M, stream);
   }
-  return launch_gemm(p, BN, false, stream);
+  return launch_gemm(p, BN, stream);
 }
 
 bool linear_geglu_fusable(int M, int F, int K) {
