@@ -93,3 +93,37 @@ def test_graph_runs_only_on_its_own_state():
     stream.synchronize()
     g.close()
     assert a.status() == 0
+
+
+@pytest.mark.parametrize("name", ["resblock_320x128x128", "tiny_fp32_gn_conv"])
+def test_sync_graph_steps_equal_plain_steps(name):
+    """Graphs of sync steps (whose GroupNorm takes the grid-wide cooperative single pass) capture
+    and replay the plain steps' bits, in bf16 and in fp32."""
+    wl = synth.WORKLOADS[name]
+    tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    dw = block_weights(wl.kind, synth.make_weights(wl, random_affine=True), tdt)
+    kind = {"resblock": B.RESBLOCK, "gn_conv": B.GN_CONV}[wl.kind]
+
+    def make():
+        return B.Block(kind, wl.H, wl.W, wl.C, wl.cout, wl.G, wl.P, 0, B.BF16 if wl.dtype == "bf16" else B.FP32,
+                       wl.silu, wl.eps, 1.0)
+    xs = synth.InputStream(wl)
+    xin = [synth.nchw_to_nhwc(xs.x(k)).to(tdt).cuda() for k in range(4)]
+    plain, replay = make(), make()
+    out_p = torch.empty(wl.H, wl.W, wl.cout, dtype=tdt, device="cuda")
+    out_g = torch.empty_like(out_p)
+    xbuf = xin[0].clone()
+    plain.step(xin[0], out_p, dw, B.SYNC)
+    replay.step(xbuf, out_g, dw, B.SYNC)
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        graph = replay.graph(xbuf, out_g, dw, B.SYNC, stream)
+        for k in range(1, 4):
+            plain.step(xin[k], out_p, dw, B.SYNC, stream)
+            xbuf.copy_(xin[k])
+            graph.launch(stream)
+            stream.synchronize()
+            assert torch.equal(out_p, out_g), f"{name}: sync step {k} differs"
+    graph.close()
+    assert plain.status() == 0 and replay.status() == 0 and B.dp_device_status() == 0
