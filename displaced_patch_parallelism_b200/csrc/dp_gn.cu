@@ -317,8 +317,6 @@ __global__ void __launch_bounds__(1024) gn_apply_kernel(const T* __restrict__ x,
     fence_mbar_init();
   }
   __syncthreads();
-  griddep_wait();
-  griddep_trigger();
   const int b = gridDim.x - 1 - blockIdx.x;   // reverse walk: L2-hot tail first
   const int p = b / a.S, s = b % a.S;
   const int chunk = (a.HWp + a.S - 1) / a.S;
@@ -327,8 +325,15 @@ __global__ void __launch_bounds__(1024) gn_apply_kernel(const T* __restrict__ x,
   const size_t off = (static_cast<size_t>(p) * a.HWp + beg) * a.C;
   GnRing<T> rg{ring, full, x + off, end - beg, a.piece, a.C};
   const int np = rg.pieces();
+  // The first pieces of x are fetched before the wait: this kernel always
+  // follows the statistics kernel on the stream, which lets it start only
+  // after every one of its blocks has passed its own wait, so the kernel that
+  // wrote x has completed.  Only the moments (written by the statistics
+  // kernel) and y need the wait.
   if (threadIdx.x == 0)
     for (int k = 0; k < min(np, kGnStages); ++k) rg.issue(k);
+  griddep_wait();
+  griddep_trigger();
   const int cg = a.C / a.G;
   for (int c = threadIdx.x; c < a.C; c += blockDim.x) {
     const int g = c / cg;
