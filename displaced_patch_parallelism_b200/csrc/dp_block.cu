@@ -8,7 +8,7 @@
 // ping-pong pair inside the caller's workspace: a step writes the fresh half
 // (GroupNorm output, fused q/k/v projection output, fresh statistics, or the
 // output of the layer feeding a conv) and reads the stale half; the refresh
-// that replaces the paper's AllGather is a flip of `cur`, so no byte moves.
+// that replaces DistriFusion's AllGather is a flip of `cur`, so no byte moves.
 //
 // Kinds: GN_CONV, RESBLOCK (optionally with an SDXL time embedding added to
 // conv1's output), ATTN, TRANSFORMER (SDXL-shaped: GroupNorm and

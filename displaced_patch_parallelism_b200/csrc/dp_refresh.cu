@@ -1,6 +1,6 @@
 // dp_refresh.cu -- the stale-buffer refresh.
 //
-// In the paper every device AllGathers its fresh activations asynchronously
+// In DistriFusion every device AllGathers its fresh activations asynchronously
 // so that the next step can use them as stale context ("DistriFusion",
 // atlas.scime.ai summary, Approach; its limitations note that the NCCL
 // kernels doing so occupy SMs).  With all bands on one GPU the gathered

@@ -7,7 +7,7 @@
  * latent is split into P row patches ("bands"); every band computes its own
  * rows with fresh activations and takes the context it needs from the other
  * bands out of the previous denoising step's activations.  Here all P bands
- * live on one GPU and are computed in one launch per layer; the paper's
+ * live on one GPU and are computed in one launch per layer; DistriFusion's
  * per-layer AllGather becomes a device-local refresh of the stale buffers.
  *
  * Conventions shared by every call
@@ -171,8 +171,8 @@ DP_API int dp_groupnorm_async(const void* x, void* y, const float* gamma, const 
                        void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
- * dp_groupnorm_async for callers that cannot allocate device memory.  The
- * paper has no counterpart of this call; it exists for integration only.
+ * dp_groupnorm_async for callers that cannot allocate device memory.
+ * DistriFusion has no counterpart of this call; it exists for integration only.
  *
  * Some callers have no way to obtain a workspace: code that runs where
  * cudaMalloc is off limits (it can synchronise the device, which a latency-
@@ -483,7 +483,7 @@ DP_API int dp_upsample_nearest2x(const void* x, void* out, int H, int W, int C, 
                                  void* stream);
 
 /* ------------------------------------------------------------------------
- * Stale-buffer refresh: the device-local replacement of the paper's
+ * Stale-buffer refresh: the device-local replacement of DistriFusion's
  * per-layer AllGather (atlas.scime.ai summary, Approach: AllGather overlaps
  * computation; limitations: NCCL kernels take SMs).  Copies the rows of band
  * `band` (all bands if band == -1) from `fresh` to `stale`; a band is
