@@ -204,6 +204,8 @@ def block_desc(B, wl, H=None):
     if wl.kind == "unet_sdxl":
         B.dp_block_desc_set_unet(d, wl.base, *wl.depths)
         B.dp_block_desc_set_time_embedding(d, wl.temb_dim)
+    if wl.kind == "transformer":
+        B.dp_block_desc_set_depth(d, wl.depth)
     if wl_context(wl):
         B.dp_block_desc_set_context(d, *wl_context(wl))
         if CTX_FIXED:
@@ -423,7 +425,7 @@ class Run:
                         synth.randn((wl.temb_dim,), wl.seed + 600).to(dev)]
         else:
             wts = synth.make_weights(wl)
-            self.dw = block_weights(wl.kind, wts, self.tdt, dev)
+            self.dw = block_weights(wl.kind, wts, self.tdt, dev, depth=wl.depth)
             if wl.kind == "transformer":     # the step's text context is the last pointer
                 self.dw.append(synth.context(wl).to(self.tdt).to(dev))
         unet = (wl.base,) + tuple(wl.depths) if wl.kind == "unet_sdxl" else None
@@ -431,6 +433,7 @@ class Run:
                            B.BF16 if wl.dtype == "bf16" else B.FP32, wl.silu, wl.eps, 1.0,
                            device=dev, gn_stats=GN_STATS, context=wl_context(wl), gn_fuse=GN_FUSE,
                            temb_dim=wl.temb_dim if wl.kind == "unet_sdxl" else 0, unet=unet,
+                           depth=wl.depth if wl.kind == "transformer" else 1,
                            context_fixed=CTX_FIXED and wl_context(wl) is not None)
         xs = synth.InputStream(wl)
         self.pool = pool
@@ -625,7 +628,8 @@ def time_e2e(run, steps, dist, dev):
 
 
 EXTRA_WORKLOADS = ["tiny_fp32_gn_conv", "resblock_320x128x128", "attn_640x64x64",
-                   "unet_mini_4x128x128", "transformer_640x64x64", "unet_sdxl_4x128x128"]
+                   "unet_mini_4x128x128", "transformer_640x64x64", "transformer_1280x32x32",
+                   "unet_sdxl_4x128x128"]
 
 
 def run_ours(args, wl):

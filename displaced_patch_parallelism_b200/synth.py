@@ -269,6 +269,13 @@ WORKLOADS: Dict[str, Workload] = {
         name="transformer_640x64x64", kind="transformer", C=640, H=64, W=64, P=4, heads=10,
         head_dim=64, silu=False, steps=50, warmup=4, drift=0.05, ctx_len=77, ctx_dim=2048,
         ff_inner=2560),
+    # SDXL's innermost transformer level at 1024 px ("next" item; not a headline workload):
+    # 1280 channels at 32x32 (1024 tokens), 20 heads, ten basic layers, the 77-token text
+    # context of width 2048, feed-forward 4C (0.35 billion parameters)
+    "transformer_1280x32x32": Workload(
+        name="transformer_1280x32x32", kind="transformer", C=1280, H=32, W=32, P=8, heads=20,
+        head_dim=64, silu=False, steps=20, warmup=4, drift=0.05, ctx_len=77, ctx_dim=2048,
+        ff_inner=5120, depth=10),
     "gn_conv_320x480x480": Workload(
         name="gn_conv_320x480x480", kind="gn_conv", C=320, H=480, W=480, P=8,
         steps=50, warmup=4, drift=0.05),
